@@ -1,0 +1,418 @@
+"""Pins for the CPU oracle: what the pages and the mathematics fix, checked by
+means other than re-running the oracle's own formulas.
+
+  * exhaustive brute-force nearest-grid search (ties to the even code) for E2M1,
+  * torch's float8_e4m3fn cast (a library routine) and brute force for E4M3,
+  * closed-form tie points, grid membership, the per-element error bound,
+  * brute-force quantization of tiny tensors (searches, not format rounding),
+  * round trips of grid-valued blocks, zero tensors, storage-ratio closed forms,
+  * one-hot products and a float64 library matmul for the GEMMs.
+"""
+import json
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from nvfp4_w4a4_gemm_quantize_b200 import synth
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "pages_facts.json")))
+
+# E2M1 magnitudes in code order (1 sign, 2 exponent, 1 mantissa bit): the set a
+# 1-2-1 binary float can hold.  The test below checks it against the page.
+E2M1_GRID = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+# All E4M3FN values, decoded by torch (library routine).
+_E4M3_ALL = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+E4M3_POS = [(c, _E4M3_ALL[c]) for c in range(0x7F)]      # codes 0x00..0x7E, non-negative finite
+
+
+def brute_e2m1(q: float) -> int:
+    """Nearest E2M1 magnitude by exhaustive search, ties to the even code,
+    sign copied from q; |q| above 6 clips to 6."""
+    m = abs(Fraction(float(q)))
+    best, bestd = None, None
+    for c, v in enumerate(E2M1_GRID):
+        d = abs(m - Fraction(v))
+        if bestd is None or d < bestd or (d == bestd and c % 2 == 0):
+            best, bestd = c, d
+    sign = 8 if np.signbit(q) else 0
+    return sign | best
+
+
+def brute_e4m3(v: float) -> int:
+    """Nearest non-negative finite E4M3 value by search, ties to the even code,
+    saturating at 448."""
+    m = Fraction(float(v))
+    best, bestd = None, None
+    for c, val in E4M3_POS:
+        d = abs(m - Fraction(val))
+        if bestd is None or d < bestd or (d == bestd and c % 2 == 0):
+            best, bestd = c, d
+    return best
+
+
+# ------------------------------------------------------------------ E2M1
+def test_e2m1_bit_split_and_grid_against_page():
+    vals = [oracle.e2m1_decode(c) for c in range(16)]
+    bits = GOLD["e2m1_bits"]["value"]
+    assert bits["sign"] + bits["exponent"] + bits["mantissa"] == 4
+    assert len(vals) == 2 ** 4
+    listed = set(GOLD["e2m1_listed_magnitudes"]["value"])
+    mags = sorted({abs(v) for v in vals})
+    # every non-zero magnitude of the format is on the page's list
+    assert set(m for m in mags if m != 0) <= listed
+    # 8 distinct magnitudes, sign bit is bit 3, max is the clip value
+    assert len(mags) == 8
+    assert max(mags) == GOLD["clip_range"]["value"][1]
+    for c in range(8):
+        assert vals[c + 8] == -vals[c]
+    assert [abs(v) for v in vals[:8]] == E2M1_GRID
+
+
+def test_e2m1_encode_exhaustive_bf16_patterns():
+    """Every bf16 bit pattern read as a quotient q: oracle == brute force."""
+    pats = np.arange(65536, dtype=np.uint32)
+    qs = (pats << 16).view(np.float32)
+    L = oracle.lib()
+    for q in qs:
+        if np.isnan(q):
+            continue
+        got = L.oracle_e2m1_encode(float(q))
+        if np.isinf(q):
+            assert got == (15 if q < 0 else 7)
+            continue
+        assert got == brute_e2m1(q), (q, got)
+
+
+def test_e2m1_encode_fp32_near_thresholds():
+    """fp32 values within a few ulps of every rounding threshold and grid point."""
+    L = oracle.lib()
+    pts = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    for p in pts:
+        base = int(np.array([p], np.float32).view(np.uint32)[0])
+        for d in range(-6, 7):
+            q = np.array([base + d], np.uint32).view(np.float32)[0]
+            for sq in (q, -q):
+                assert L.oracle_e2m1_encode(float(sq)) == brute_e2m1(sq), sq
+
+
+def test_e2m1_tie_points_closed_form():
+    # midpoints go to the even code: 0.25->0, 0.75->1, 1.25->1, 1.75->2, 2.5->2, 3.5->4, 5->4
+    expect = {0.25: 0.0, 0.75: 1.0, 1.25: 1.0, 1.75: 2.0, 2.5: 2.0, 3.5: 4.0, 5.0: 4.0}
+    for t, v in expect.items():
+        assert oracle.e2m1_decode(oracle.e2m1_encode(t)) == v
+        assert oracle.e2m1_decode(oracle.e2m1_encode(-t)) == -v
+    # clipping to [-6, 6]
+    assert oracle.e2m1_decode(oracle.e2m1_encode(6.375)) == 6.0
+    assert oracle.e2m1_decode(oracle.e2m1_encode(-1e30)) == -6.0
+    # sign of zero results follows x
+    assert oracle.e2m1_encode(-0.1) == 0x8
+    assert oracle.e2m1_encode(0.1) == 0x0
+
+
+# ------------------------------------------------------------------ E4M3
+def test_e4m3_decode_matches_library_cast():
+    for c in range(256):
+        o = oracle.e4m3_decode(c)
+        t = _E4M3_ALL[c]
+        if np.isnan(t):
+            assert np.isnan(o)
+        else:
+            assert o == t, c
+
+
+def test_e4m3_roundtrip_all_finite_codes():
+    for c, v in E4M3_POS:
+        assert oracle.e4m3_encode(v) == c
+
+
+def test_e4m3_encode_vs_library_and_brute_force():
+    rng = np.random.default_rng(0)
+    vals = np.concatenate([
+        np.exp(rng.uniform(np.log(2.0 ** -12), np.log(440.0), 4000)),
+        # midpoints between neighbours (ties) and one ulp either side
+        [(E4M3_POS[i][1] + E4M3_POS[i + 1][1]) / 2 for i in range(len(E4M3_POS) - 1)],
+    ]).astype(np.float32)
+    more = []
+    for v in vals[-(len(E4M3_POS) - 1):]:
+        u = int(np.array([v], np.float32).view(np.uint32)[0])
+        more += [np.array([u - 1], np.uint32).view(np.float32)[0], np.array([u + 1], np.uint32).view(np.float32)[0]]
+    vals = np.concatenate([vals, np.array(more, np.float32)])
+    lib_codes = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    for v, lc in zip(vals, lib_codes):
+        oc = oracle.e4m3_encode(v)
+        assert oc == brute_e4m3(v), v
+        if v <= 448.0:
+            assert oc == lc, (v, oc, lc)
+
+
+def test_e4m3_saturates():
+    for v in (448.0, 460.0, 464.0, 480.0, 1e6, 3.0e38, float("inf")):
+        assert oracle.e4m3_encode(v) == 0x7E
+    assert oracle.e4m3_decode(0x7E) == 448.0
+    assert oracle.e4m3_encode(2.0 ** -10) == 0       # tie between 0 and 2^-9 -> even (0)
+    assert oracle.e4m3_encode(1.5 * 2.0 ** -10) == 1
+
+
+# ------------------------------------------------------------------ bf16
+def test_bf16_rounding_vs_search():
+    rng = np.random.default_rng(1)
+    # doubles with up to 30 significant bits, like the exact dequantized products
+    m = rng.integers(1 << 29, 1 << 30, 3000).astype(np.float64)
+    e = rng.integers(-150, 100, 3000)
+    vals = np.ldexp(m, e - 29) * rng.choice([-1.0, 1.0], 3000)
+    allbf = (np.arange(0x7F81, dtype=np.uint32) << 16).view(np.float32).astype(np.float64)
+    for v in vals:
+        got = oracle.bf16_from_double(v)
+        a = Fraction(abs(v))
+        # search the two positive bf16 neighbours of |v|
+        f = np.float32(abs(v))
+        u = int(np.array([f], np.float32).view(np.uint32)[0] >> 16)
+        cands = [c for c in (u - 1, u, u + 1, u + 2) if 0 <= c < 0x7F81]
+        best = min(cands, key=lambda c: (abs(a - Fraction(float(allbf[c]))), c % 2))
+        if np.signbit(v):
+            best |= 0x8000
+        assert got == best, v
+
+
+# ------------------------------------------------------------------ SF layout
+def test_sf_offset_bijection_and_hand_values():
+    rows, k = 256, 128
+    kb = k // 16
+    seen = set()
+    for r in range(rows):
+        for c in range(kb):
+            seen.add(oracle.sf_offset(r, c, kb))
+    assert seen == set(range(oracle.sf_bytes(rows, k)))
+    # hand-derived: atom = 128 rows x 4 blocks = 512 bytes, line r%32, word (r%128)/32, byte c%4
+    assert oracle.sf_offset(0, 0, kb) == 0
+    assert oracle.sf_offset(0, 1, kb) == 1
+    assert oracle.sf_offset(1, 0, kb) == 16
+    assert oracle.sf_offset(32, 0, kb) == 4
+    assert oracle.sf_offset(127, 3, kb) == 31 * 16 + 3 * 4 + 3
+    assert oracle.sf_offset(0, 4, kb) == 512
+    assert oracle.sf_offset(128, 0, kb) == 2 * 512
+    assert oracle.sf_bytes(600, 4096) == 640 * 256
+
+
+def test_sf_matrix_helper_agrees_with_offset():
+    rows, k = 300, 192
+    rng = np.random.default_rng(2)
+    sf = rng.integers(0, 256, oracle.sf_bytes(rows, k)).astype(np.uint8)
+    mat = oracle.sf_matrix(sf, rows, k)
+    for r in range(0, rows, 7):
+        for c in range(k // 16):
+            assert mat[r, c] == sf[oracle.sf_offset(r, c, k // 16)]
+
+
+# ------------------------------------------------------------------ quantize
+def brute_quantize(xf32: np.ndarray, scale=None):
+    """Quantize by searches: g from amax, sf by nearest-E4M3 search, codes by
+    nearest-E2M1 search, every product/quotient a single fp32 rounding."""
+    rows, k = xf32.shape
+    f = np.float32
+    if scale is None:
+        amax = f(np.max(np.abs(xf32))) if xf32.size else f(0)
+        g = f(amax / f(2688.0))
+    else:
+        g = f(scale)
+    d = f(f(6.0) * g)
+    codes = np.zeros((rows, k), np.uint8)
+    sfm = np.zeros((rows, k // 16), np.uint8)
+    for r in range(rows):
+        for c in range(k // 16):
+            blk = xf32[r, 16 * c:16 * c + 16]
+            ab = f(np.max(np.abs(blk)))
+            sfc = brute_e4m3(f(ab / d)) if d > 0 else 0
+            sfm[r, c] = sfc
+            s = f(f(_E4M3_ALL[sfc]) * g)
+            for i in range(16):
+                codes[r, 16 * c + i] = brute_e2m1(f(blk[i] / s)) if s != 0 else 0
+    return codes, sfm, g
+
+
+@pytest.mark.parametrize("case", range(10))
+def test_quantize_vs_brute_force_tiny(case):
+    rng = np.random.default_rng(100 + case)
+    rows, k = [(1, 64), (3, 64), (2, 128), (5, 64), (4, 192)][case % 5]
+    x = rng.standard_normal((rows, k)).astype(np.float32)
+    if case % 3 == 1:
+        x *= np.exp(rng.uniform(-8, 8, (rows, 1))).astype(np.float32)   # wide dynamic range
+    if case % 4 == 2:
+        x[:, rng.integers(0, k, 3)] = 0.0
+        x[0, :16] = 0.0                                                  # an all-zero block
+    if case % 5 == 3:
+        x[1, 5] = -0.0
+        x[2, 7] = -1e-6                                                  # negative -> code 0x8
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    xf = xb.float().numpy()
+    scale = None if case < 7 else float(np.float32(np.max(np.abs(xf)) / 2000.0))
+    codes, sf, g = oracle.quantize(xb, scale)
+    bc, bsf, bg = brute_quantize(xf, scale)
+    assert np.float32(g) == bg
+    assert np.array_equal(oracle.unpack_codes(codes), bc)
+    assert np.array_equal(oracle.sf_matrix(sf, rows, k), bsf)
+
+
+def _grid_checks(xb, codes, sf, g):
+    """grid membership and the half-spacing error bound, per element."""
+    xf = xb.float().numpy().astype(np.float64)
+    rows, k = xf.shape
+    deq = oracle.dequantize(codes, sf, g, "f64")
+    sfm = oracle.sf_matrix(sf, rows, k)
+    s = np.repeat(_E4M3_ALL[sfm], 16, axis=1) * np.float64(np.float32(g))
+    s32 = np.repeat(np.float32(_E4M3_ALL[sfm]) * np.float32(g), 16, axis=1).astype(np.float64)
+    nz = s32 > 0
+    ratio = np.where(nz, deq / np.where(nz, s, 1.0), 0.0)
+    grid = set(E2M1_GRID) | {-v for v in E2M1_GRID}
+    assert set(np.unique(ratio)) <= grid
+    # error bound: spacing of the grid interval that holds |q|
+    q = np.abs(xf) / np.where(nz, s32, 1.0)
+    spacing = np.where(q < 2, 0.5, np.where(q < 4, 1.0, 2.0))
+    err = np.abs(xf - deq)
+    # |x - code*s| <= s*spacing/2 inside the grid, |x| - 6s when clipped; the
+    # fp32 quotient and the fp32 scale each add at most 2^-23 relative to |x|.
+    bound = np.where(q <= 6, s * spacing / 2, np.abs(xf) - 6 * s)
+    assert np.all(~nz | (err <= bound + 2.0 ** -21 * np.abs(xf)))
+    return deq
+
+
+@pytest.mark.parametrize("dist", ["normal", "student_t3", "outlier", "token_scaled"])
+def test_quantize_grid_membership_and_error_bound(dist):
+    xb = synth.random_bf16((256, 1024), seed=7, dist=dist)
+    codes, sf, g = oracle.quantize(xb)
+    _grid_checks(xb, codes, sf, g)
+
+
+def test_block_scale_never_exceeds_e4m3_range_and_scale_relation():
+    xb = synth.random_bf16((128, 512), seed=8, dist="student_t3")
+    codes, sf, g = oracle.quantize(xb)
+    amax = np.float32(np.max(np.abs(xb.float().numpy())))
+    assert g == np.float32(amax / np.float32(2688.0))
+    sfm = oracle.sf_matrix(sf, 128, 512)
+    assert sfm.max() <= 0x7E
+    # the largest block scale is the one of the block holding amax: E4M3(amax / (6 g)) ~ 448
+    assert _E4M3_ALL[sfm.max()] == 448.0
+
+
+def test_grid_valued_blocks_round_trip_exactly():
+    """Blocks of grid values times 2^m, with a power-of-two tensor scale, come
+    back unchanged: s = 2^m exactly, so every quotient is on the grid."""
+    rng = np.random.default_rng(3)
+    rows, k = 8, 128
+    vals = np.array(E2M1_GRID + [-v for v in E2M1_GRID[1:]], np.float64)
+    x = rng.choice(vals, (rows, k))
+    m = rng.integers(-12, 1, (rows, k // 16))     # block scale 2^(m+8) stays in E4M3 range
+    for r in range(rows):
+        for c in range(k // 16):
+            x[r, 16 * c] = 6.0                       # block amax = 6 * 2^m
+            x[r, 16 * c:16 * c + 16] *= 2.0 ** m[r, c]
+    xb = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16)
+    assert np.array_equal(xb.float().numpy(), x.astype(np.float32))
+    codes, sf, g = oracle.quantize(xb, scale=2.0 ** -8)
+    deq = oracle.dequantize(codes, sf, g, "f64")
+    assert np.array_equal(deq, x)
+
+
+def test_zero_tensor():
+    xb = torch.zeros(130, 64, dtype=torch.bfloat16)
+    codes, sf, g = oracle.quantize(xb)
+    assert g == 0.0 and not codes.any() and not sf.any()
+    assert not oracle.dequantize(codes, sf, g, "f64").any()
+
+
+def test_storage_ratios_from_page():
+    rows, k = 4096, 4096
+    total = rows * k // 2 + oracle.sf_bytes(rows, k) + 4
+    bits = total * 8 / (rows * k)
+    assert abs(bits - 4.5) < 1e-5
+    assert round(16 / bits, 1) == GOLD["memory_reduction_vs_fp16"]["value"] + 0.1 or \
+        abs(16 / bits - GOLD["memory_reduction_vs_fp16"]["value"]) < 0.1
+    assert abs(8 / bits - GOLD["memory_reduction_vs_fp8"]["value"]) < 0.05
+    assert 16 / (8 / GOLD["packed_codes_per_byte"]["value"]) == GOLD["packed_memory_reduction_vs_fp16"]["value"]
+
+
+def test_relative_error_next_to_page_bound():
+    """Lemma III.2 states eps = 2^-3.  The tensor-level relative error on
+    Gaussian and heavy-tailed inputs stays below it (the per-element worst case
+    of the format does not, see the design notes)."""
+    eps = GOLD["eps_fp4"]["value"]
+    for dist in ("normal", "student_t3"):
+        xb = synth.random_bf16((512, 1024), seed=9, dist=dist)
+        codes, sf, g = oracle.quantize(xb)
+        deq = oracle.dequantize(codes, sf, g, "f64")
+        xf = xb.float().numpy().astype(np.float64)
+        rel = np.linalg.norm(xf - deq) / np.linalg.norm(xf)
+        assert rel < eps, (dist, rel)
+
+
+# ------------------------------------------------------------------ dequantize
+def test_dequantize_roundings():
+    xb = synth.random_bf16((64, 256), seed=10, dist="student_t3")
+    codes, sf, g = oracle.quantize(xb)
+    d64 = oracle.dequantize(codes, sf, g, "f64")
+    d32 = oracle.dequantize(codes, sf, g, "f32")
+    db = oracle.dequantize(codes, sf, g, "bf16")
+    assert np.array_equal(d32, d64.astype(np.float32))            # library double->float (RNE)
+    for v, b in zip(d64.ravel()[:4000], db.ravel()[:4000]):
+        assert b == oracle.bf16_from_double(v)
+
+
+# ------------------------------------------------------------------ GEMM
+def _zero_operand(rows, k):
+    return np.zeros((rows, k // 2), np.uint8), np.zeros(oracle.sf_bytes(rows, k), np.uint8)
+
+
+@pytest.mark.parametrize("m0,n0,k0", [(0, 0, 0), (5, 3, 17), (127, 130, 63), (64, 255, 100)])
+def test_gemm_one_hot(m0, n0, k0):
+    M, N, K = 128, 256, 128
+    ac, asf = _zero_operand(M, K)
+    bc, bsf = _zero_operand(N, K)
+    ca, cb = 0x3, 0xB           # 1.5 and -1.5
+    ac[m0, k0 // 2] = ca << (4 * (k0 & 1))
+    bc[n0, k0 // 2] = cb << (4 * (k0 & 1))
+    asf[oracle.sf_offset(m0, k0 // 16, K // 16)] = 0x40     # 2.0
+    bsf[oracle.sf_offset(n0, k0 // 16, K // 16)] = 0x30     # 0.5
+    ga, gb = 0.25, 3.0
+    y = oracle.gemm_w4a4(ac, asf, ga, bc, bsf, gb)
+    expect = np.zeros((M, N))
+    expect[m0, n0] = ga * gb * (1.5 * 2.0) * (-1.5 * 0.5)
+    assert np.array_equal(y, expect)
+    # mismatched k positions give zero everywhere
+    bc2, _ = _zero_operand(N, K)
+    k1 = (k0 + 1) % K
+    bc2[n0, k1 // 2] = cb << (4 * (k1 & 1))
+    bsf2 = bsf.copy()
+    bsf2[oracle.sf_offset(n0, k1 // 16, K // 16)] = 0x30
+    assert not oracle.gemm_w4a4(ac, asf, ga, bc2, bsf2, gb).any()
+
+
+def test_gemm_vs_library_matmul():
+    x = synth.random_bf16((96, 320), seed=11, dist="outlier")
+    w = synth.random_bf16((160, 320), seed=12, scale=0.02)
+    ac, asf, ga = oracle.quantize(x)
+    bc, bsf, gb = oracle.quantize(w)
+    y = oracle.gemm_w4a4(ac, asf, ga, bc, bsf, gb)
+    da = torch.from_numpy(oracle.dequantize(ac, asf, ga, "f64"))
+    db = torch.from_numpy(oracle.dequantize(bc, bsf, gb, "f64"))
+    ref = (da @ db.T).numpy()
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+    # single-element and row-slice entry points agree with the full product
+    assert oracle.gemm_w4a4_at(ac, asf, ga, bc, bsf, gb, 17, 33) == pytest.approx(y[17, 33], rel=1e-13, abs=1e-300)
+    assert np.allclose(oracle.gemm_w4a4(ac, asf, ga, bc, bsf, gb, rows=slice(10, 20)), y[10:20], rtol=1e-13)
+
+
+def test_gemm_w4a16_vs_library_matmul():
+    x = synth.random_bf16((64, 256), seed=13)
+    w = synth.random_bf16((96, 256), seed=14, scale=0.015)
+    wc, wsf, gw = oracle.quantize(w)
+    y = oracle.gemm_w4a16(x, wc, wsf, gw)
+    dw = torch.from_numpy(oracle.dequantize(wc, wsf, gw, "f64"))
+    ref = (x.double() @ dw.T).numpy()
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+    xb = oracle.bf16_bits(x)
+    assert oracle.gemm_w4a16_at(xb, wc, wsf, gw, 5, 7) == pytest.approx(y[5, 7], rel=1e-13)
