@@ -1,0 +1,329 @@
+"""Benchmark of the NVFP4 hot path on the video-DiT layers (M=32768 tokens,
+hidden 3072: QKV 3072->9216, MLP fc1 3072->12288, fc2 12288->3072).
+
+One step = for every layer: NVFP4-quantize the bf16 activation X (tensor amax
+pass + quantize pass) and run the W4A4 GEMM Y = X W^T with a bf16 epilogue.
+Weights are quantized once, before timing (static weights).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Rank 0 prints one JSON line.  value = GEMM FLOPs of all ranks' steps / max
+over ranks of the device time of the K steps (quantization included).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = "video_dit"
+METRIC = "NVFP4 W4A4 GEMM TFLOPS and % of dense FP4 peak; quantize GB/s vs HBM"
+FP4_OVER_BF16 = 4.0          # nominal dense FP4 / dense bf16 tensor throughput (9 / 2.25 PFLOP/s)
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# quantize, algorithmic bytes per element: 2 (amax read) + 2 (read) + 0.5 (codes) + 1/16 (scales)
+QUANT_BYTES_PER_ELEM = 4.5625
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (clocks and throttle reasons)."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if os.environ.get("NVFP4_BENCH_BACKEND", "nccl") == "nccl" else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- oracle leg
+def oracle_sample(rows_per_layer: int):
+    """The CPU oracle on a bounded sample of the same step: quantize
+    rows_per_layer rows of every layer input and weight rows and form those
+    rows of Y.  Returns (gemm_flops, seconds, description)."""
+    import numpy as np
+    import torch
+    import oracle
+    from nvfp4_w4a4_gemm_quantize_b200 import synth
+    wl = synth.WORKLOADS[WORKLOAD]
+    flops, secs = 0, 0.0
+    for i, L in enumerate(wl.layers):
+        gen = torch.Generator().manual_seed(wl.seed * 1000 + i)
+        x = (torch.randn(rows_per_layer, L.K, generator=gen) *
+             torch.exp(torch.empty(rows_per_layer, 1).uniform_(np.log(0.1), np.log(10.0), generator=gen))
+             ).to(torch.bfloat16)
+        w = (torch.randn(L.N, L.K, generator=gen) * wl.w_std).to(torch.bfloat16)
+        bc, bsf, gb = oracle.quantize(w)            # weights: quantized once, untimed
+        t0 = time.perf_counter()
+        ac, asf, ga = oracle.quantize(x)
+        oracle.gemm_w4a4(ac, asf, ga, bc, bsf, gb)
+        secs += time.perf_counter() - t0
+        flops += 2 * rows_per_layer * L.N * L.K
+    desc = (f"oracle quantize + FP64 GEMM of {rows_per_layer} activation rows per layer "
+            f"(of {wl.layers[0].M}) for all {len(wl.layers)} {WORKLOAD} layers, 1 thread")
+    return flops, secs, desc
+
+
+def run_reference(args):
+    rank, world, local = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), 0
+    if rank != 0:
+        return 0
+    rows = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample(max(1, rows // 4))
+    fl, secs = 0, 0.0
+    desc = ""
+    for _ in range(args.steps):
+        f, s, desc = oracle_sample(rows)
+        fl += f
+        secs += s
+    v = fl / secs / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": f"{WORKLOAD} (row sample)", "rows_per_layer": rows},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ----------------------------------------------------------------- our leg
+def run_ours(args):
+    import torch
+    import nvfp4_w4a4_gemm_quantize_b200 as nv
+    from nvfp4_w4a4_gemm_quantize_b200 import build, synth
+
+    rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if rank == 0:
+        build.build()
+    barrier(world)
+    wl = synth.WORKLOADS[WORKLOAD]
+    peaks, peak_src = load_peaks()
+
+    # ---- data (resident in HBM before timing); each rank its own batch
+    xs, Ws, Aq, Ys = [], [], [], []
+    for L in wl.layers:
+        x, w = synth.layer_tensors(WORKLOAD, L.name, device=dev)
+        if rank:
+            x = x.roll(rank * 977, dims=0)
+        xs.append(x)
+        Ws.append(nv.quantize(w))                        # static weights, quantized once
+        del w
+        Aq.append(nv.NVFP4Tensor.empty(L.M, L.K, dev))
+        Ys.append(torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev))
+    ws = torch.empty(nv.nvfp4_quantize_workspace_bytes(1, 64), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    gemm_flops = sum(2 * L.M * L.N * L.K for L in wl.layers)
+    q_elems = sum(L.M * L.K for L in wl.layers)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    gemm_ev = [[(ev(), ev()) for _ in wl.layers] for _ in range(args.steps)]
+    quant_ev = [[(ev(), ev()) for _ in wl.layers] for _ in range(args.steps)]
+
+    def step(i=None):
+        for li, L in enumerate(wl.layers):
+            if i is not None:
+                quant_ev[i][li][0].record(stream)
+            nv.quantize(xs[li], out=Aq[li], workspace=ws)
+            if i is not None:
+                quant_ev[i][li][1].record(stream)
+                gemm_ev[i][li][0].record(stream)
+            nv.gemm_w4a4(Aq[li], Ws[li], out=Ys[li])
+            if i is not None:
+                gemm_ev[i][li][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    launches0 = nv.nvfp4_launch_count()
+    t0, t1 = ev(), ev()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    launches = nv.nvfp4_launch_count() - launches0
+    barrier(world)
+    clocks = sampler.stop()
+    dev_ms = t0.elapsed_time(t1)
+    max_ms = max_over_ranks(dev_ms, world, dev)
+
+    gemm_ms = [sum(s.elapsed_time(e) for s, e in (gemm_ev[i][li] for i in range(args.steps))) / args.steps
+               for li in range(len(wl.layers))]
+    quant_ms = [sum(s.elapsed_time(e) for s, e in (quant_ev[i][li] for i in range(args.steps))) / args.steps
+                for li in range(len(wl.layers))]
+
+    # ---- end to end through the public API with host buffers
+    xh = [x.cpu().pin_memory() for x in xs]
+    yh = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for y in Ys]
+    h2d = sum(x.numel() * x.element_size() for x in xh)
+    d2h = sum(y.numel() * y.element_size() for y in yh)
+
+    def e2e_step():
+        for li in range(len(wl.layers)):
+            xs[li].copy_(xh[li], non_blocking=True)
+            nv.quantize(xs[li], out=Aq[li], workspace=ws)
+            nv.gemm_w4a4(Aq[li], Ws[li], out=Ys[li])
+            yh[li].copy_(Ys[li], non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
+
+    # ---- cpu baseline (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        fl, secs, desc = oracle_sample(args.ref_rows)
+        cpu = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        fp4_peak = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"]) * FP4_OVER_BF16
+        hbm_peak = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
+        # dominant kernel: the GEMM of the largest layer (fc1, the 32768x3072x12288 shape)
+        li = [L.name for L in wl.layers].index("fc1")
+        L = wl.layers[li]
+        g_flops = 2 * L.M * L.N * L.K
+        g_tflops = g_flops / (gemm_ms[li] * 1e-3) / 1e12
+        q_gbs = [QUANT_BYTES_PER_ELEM * l.M * l.K / (quant_ms[j] * 1e-3) / 1e9 for j, l in enumerate(wl.layers)]
+        per_layer = {l.name: {"gemm_ms": round(gemm_ms[j], 4),
+                              "gemm_tflops": round(2 * l.M * l.N * l.K / (gemm_ms[j] * 1e-3) / 1e12, 1),
+                              "quant_ms": round(quant_ms[j], 4), "quant_gbs": round(q_gbs[j], 1)}
+                     for j, l in enumerate(wl.layers)}
+        value = world * args.steps * gemm_flops / (max_ms * 1e-3) / 1e12
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
+            "data": "synthetic",
+            "config": {"workload": f"{WORKLOAD}: M=32768, qkv 3072->9216, fc1 3072->12288, fc2 12288->3072 "
+                                   "(dynamic-scale activation quantize + W4A4 GEMM, bf16 out)",
+                       "l2": "inputs larger than L2 (X 201-805 MB per layer, >2 GB streamed per step)",
+                       "parallelism": f"replica per GPU x{world}"},
+            "roofline": {"bound": "tensor", "kernel": "gemm_w4a4 fc1 32768x3072x12288",
+                         "achieved": round(g_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                         "frac": round(g_tflops / fp4_peak, 4),
+                         "peak_source": f"{peak_src} bf16 x {FP4_OVER_BF16:g} (nominal FP4/bf16 ratio)",
+                         "traffic": None},
+            "quantize": {"bound": "hbm", "achieved": round(max(q_gbs), 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(max(q_gbs) / hbm_peak, 4), "bytes_per_elem": QUANT_BYTES_PER_ELEM,
+                         "peak_source": peak_src},
+            "layers": per_layer,
+            "e2e": {"value": round(world * gemm_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": int(launches),
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=48)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,168 @@
+/*
+ * nvfp4.h -- C ABI of the B200 (sm_100a) NVFP4 library: two-level NVFP4
+ * quantization and block-scaled FP4 matrix products for the linear layers of a
+ * diffusion transformer (QKV / out projections, MLP fc1 / fc2).
+ *
+ * Sources the operations follow (web pages, by title and section):
+ *  [DiT] "NVFP4-DiT: Efficient 4-Bit Audio-Guided Video Diffusion Transformers
+ *        for Low-Cost Video Generation", Methodology 1 (Definition III.1:
+ *        Q_FP4(v; s) = s * clip(round(v/s)_FP4, -6, 6); E2M1 = 1 sign,
+ *        2 exponent, 1 mantissa bit) and 3 (two FP4 values per byte, FP32
+ *        accumulation).
+ *  [RFC] "[RFC]: NVFP4 Quantization Support for Diffusion Models", Motivation
+ *        (two-level scaling: an FP8 scale per 16 values plus an FP32 tensor
+ *        scale; Blackwell SM100), Open Questions 1 (W4A16 and W4A4).
+ *
+ * Conventions shared by every call
+ *  - Row-major.  Activations X are [M, K], weights W are [N, K] (nn.Linear
+ *    layout), Y = X W^T is [M, N].  The 16-value quantization block runs along
+ *    K, the reduction axis, for both operands.
+ *  - An NVFP4 tensor of shape [rows, k] is three buffers:
+ *      codes  rows * k/2 bytes, row stride k/2; element 2j of a row sits in the
+ *             low nibble of byte j, element 2j+1 in the high nibble; a nibble
+ *             is sign(1) exponent(2) mantissa(1).
+ *      sf     nvfp4_sf_bytes(rows, k) bytes of unsigned E4M3 block scales in
+ *             the tensor-core scale-factor layout: the scale of row r, block c
+ *             (kb = k/16 blocks per row) sits at byte
+ *               ((r/128)*(kb/4) + c/4)*512 + (r%32)*16 + ((r%128)/32)*4 + c%4,
+ *             rows padded to a multiple of 128 with zero bytes.
+ *      scale  one float (device memory), the tensor scale g.
+ *    Element value = e2m1(code) * e4m3(sf) * g.
+ *  - Every pointer is DEVICE memory unless stated; the caller allocates and
+ *    owns every buffer.  Calls are asynchronous on `stream` (a cudaStream_t;
+ *    NULL = legacy default stream) and never synchronize the host.
+ *  - Argument checks run on the host before any launch; a failed check
+ *    returns an error and launches nothing.  Launch failures return
+ *    NVFP4_ERR_CUDA.
+ *  - `dev_status` (nullable, device int): a kernel that gives up on a bounded
+ *    internal wait writes NVFP4_ERR_TIMEOUT there and returns without hanging.
+ *    The library never clears it; the caller zeroes it and reads it after the
+ *    stream has synchronized.
+ *  - Inputs must be finite; non-finite values give unspecified codes.
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *nvfp4_stream_t;   /* same type as cudaStream_t */
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad flag/dtype      */
+    NVFP4_ERR_UNSUPPORTED_SHAPE = 2,  /* K or N not a supported multiple (see each call) */
+    NVFP4_ERR_MISALIGNED = 3,         /* pointer or row stride not 16-byte aligned        */
+    NVFP4_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not compute capability 10.0    */
+    NVFP4_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed                */
+    NVFP4_ERR_TIMEOUT = 6,            /* device-side bounded wait expired (dev_status)    */
+    NVFP4_ERR_WORKSPACE = 7           /* workspace missing or too small                   */
+} nvfp4_status;
+
+enum { NVFP4_DTYPE_BF16 = 0, NVFP4_DTYPE_F32 = 1 };
+
+/* nvfp4_quantize flags */
+enum { NVFP4_SCALE_GIVEN = 1 };
+
+/* Bytes of the scale buffer of a [rows, k] NVFP4 tensor:
+ * ceil(rows/128)*128 * k/16.  Returns 0 for rows < 0 or k not a multiple of 64. */
+size_t nvfp4_sf_bytes(int64_t rows, int64_t k);
+
+/* Bytes of device workspace nvfp4_quantize needs when it derives the tensor
+ * scale from the data (no NVFP4_SCALE_GIVEN): one partial maximum per CTA of
+ * the amax pass.  The contents need no initialisation and are not preserved. */
+size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t k);
+
+/*
+ * nvfp4_quantize -- two-level NVFP4 quantization of a bf16 tensor
+ * ([DiT] Definition III.1 with the [RFC] two-level scaling):
+ *   g   = amax(|x|) / (6 * 448)               (IEEE single division)
+ *   per row and 16-value block along k:  a_b = max|x|,
+ *         sf = E4M3_rne_satfinite(a_b / (6 g)),  s = e4m3(sf) * g
+ *   per element: code = E2M1_rne(clip(x / s, -6, 6)), sign of x kept;
+ *         a block with s == 0 gives codes 0.
+ * x_bf16        [rows, k] bf16, row stride ld_x elements (ld_x >= k, ld_x % 8 == 0,
+ *               pointer 16-byte aligned).
+ * rows >= 0;    k > 0 and k % 64 == 0.
+ * codes         out, rows * k/2 bytes (16-byte aligned).
+ * sf            out, nvfp4_sf_bytes(rows, k) bytes (16-byte aligned); padding rows
+ *               are written as zero.
+ * tensor_scale  device float.  With flags & NVFP4_SCALE_GIVEN it is read as g
+ *               (for weights quantized once, or a calibrated activation scale);
+ *               otherwise g is computed from the data and written there.
+ * workspace     device scratch of >= nvfp4_quantize_workspace_bytes(rows, k)
+ *               bytes, 16-byte aligned; unused (may be NULL) with SCALE_GIVEN.
+ * Two kernels on `stream` (amax pass, then quantize) or one with SCALE_GIVEN.
+ * rows == 0 is a no-op (g = 0 is written when not given).
+ */
+nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t rows, int64_t k, int64_t ld_x,
+                            uint8_t *codes, uint8_t *sf, float *tensor_scale,
+                            unsigned flags, void *workspace, size_t workspace_bytes,
+                            int *dev_status, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_dequantize -- v = (e2m1(code) * e4m3(sf)) * g, rounded once (RNE) to
+ * out_dtype ([DiT] Definition III.1: the quantizer returns s * round(...)).
+ * codes/sf/tensor_scale as produced by nvfp4_quantize for [rows, k];
+ * out: [rows, k] contiguous, NVFP4_DTYPE_BF16 or NVFP4_DTYPE_F32, 16-byte aligned.
+ */
+nvfp4_status nvfp4_dequantize(const uint8_t *codes, const uint8_t *sf,
+                              const float *tensor_scale, int64_t rows, int64_t k,
+                              void *out, int out_dtype, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_gemm_w4a4 -- block-scaled FP4 x FP4 product with FP32 accumulation
+ * ([DiT] 3. Systems optimization; [RFC] Open Questions 1, W4A4):
+ *   acc[m,n] = sum_k (e2m1(a)*e4m3(sfa)) * (e2m1(b)*e4m3(sfb))   (FP32, tensor cores)
+ *   Y[m,n]   = alpha * acc[m,n],  alpha = g_a * g_b              (FP32)
+ * A: a_codes [M, K/2], a_sf (nvfp4_sf_bytes(M, K)), a_scale (device float g_a).
+ * B: b_codes [N, K/2], b_sf (nvfp4_sf_bytes(N, K)), b_scale (device float g_b).
+ * M >= 0, N > 0, K > 0 with K % 64 == 0.
+ * Output, one of two forms:
+ *  - y != NULL: Y [M, N] row-major in y_dtype (BF16 rounded RNE, or F32);
+ *    N % 8 == 0 for BF16, N % 4 == 0 for F32; y 16-byte aligned.
+ *  - y == NULL and y_codes != NULL: the next layer's NVFP4 activations, Y
+ *    quantized in the epilogue with the caller's tensor scale g_y (*y_scale),
+ *    exactly as nvfp4_quantize with NVFP4_SCALE_GIVEN would quantize the FP32
+ *    value alpha*acc: y_codes [M, N/2], y_sf nvfp4_sf_bytes(M, N); needs
+ *    N % 64 == 0.  y_amax (nullable device float, caller-initialised): receives
+ *    the running max of |alpha*acc| (atomic max), from which the caller can
+ *    derive the next call's g_y.
+ * All code/scale pointers 16-byte aligned.  One persistent kernel on `stream`.
+ */
+nvfp4_status nvfp4_gemm_w4a4(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_scale,
+                             const uint8_t *b_codes, const uint8_t *b_sf, const float *b_scale,
+                             int64_t M, int64_t N, int64_t K,
+                             void *y, int y_dtype,
+                             uint8_t *y_codes, uint8_t *y_sf, const float *y_scale, float *y_amax,
+                             int *dev_status, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_gemm_w4a16 -- weights-only NVFP4 ([RFC] Open Questions 1, W4A16):
+ *   Y[m,n] = g_w * sum_k x[m,k] * (e2m1(w[n,k]) * e4m3(sfw))
+ * The weight element e2m1 * e4m3 is exact in bf16; it is formed in shared
+ * memory inside the kernel and fed to bf16 tensor-core MMAs with FP32
+ * accumulation; g_w is applied in the FP32 epilogue.
+ * x_bf16 [M, K] contiguous bf16 (16-byte aligned); w_codes [N, K/2], w_sf,
+ * w_scale as from nvfp4_quantize; K % 64 == 0; y [M, N] in y_dtype
+ * (N % 8 == 0 for BF16, N % 4 == 0 for F32).
+ */
+nvfp4_status nvfp4_gemm_w4a16(const void *x_bf16, const uint8_t *w_codes, const uint8_t *w_sf,
+                              const float *w_scale, int64_t M, int64_t N, int64_t K,
+                              void *y, int y_dtype, int *dev_status, nvfp4_stream_t stream);
+
+/* Static text for a status code. */
+const char *nvfp4_status_string(nvfp4_status s);
+
+/* Number of this library's kernels launched since load (host-side counter,
+ * all threads).  For accounting in benchmarks. */
+uint64_t nvfp4_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_H_ */

@@ -1,1 +1,162 @@
-"""NVFP4 two-level quantization and block-scaled FP4 GEMMs for B200 (sm_100a)."""
+"""NVFP4 two-level quantization and block-scaled FP4 GEMMs for B200 (sm_100a).
+
+Python binding of the C ABI in include/nvfp4.h.  Every function below only
+marshals torch tensors into pointers and sizes and calls the library of the
+same name; all arithmetic runs in the CUDA kernels.  torch supplies device
+memory and streams.
+
+Low-level (same names and argument order as the C calls):
+    nvfp4_sf_bytes, nvfp4_quantize_workspace_bytes, nvfp4_quantize,
+    nvfp4_dequantize, nvfp4_gemm_w4a4, nvfp4_gemm_w4a16, nvfp4_launch_count
+Convenience (allocate outputs with torch, then call the above):
+    NVFP4Tensor, quantize, dequantize, gemm_w4a4, gemm_w4a16
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from ._lib import NVFP4Error, check, lib  # noqa: F401
+
+NVFP4_DTYPE_BF16 = 0
+NVFP4_DTYPE_F32 = 1
+NVFP4_SCALE_GIVEN = 1
+
+_DT = {torch.bfloat16: NVFP4_DTYPE_BF16, torch.float32: NVFP4_DTYPE_F32}
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+# ----------------------------------------------------------------- C ABI
+def nvfp4_sf_bytes(rows: int, k: int) -> int:
+    return int(lib().nvfp4_sf_bytes(rows, k))
+
+
+def nvfp4_quantize_workspace_bytes(rows: int, k: int) -> int:
+    return int(lib().nvfp4_quantize_workspace_bytes(rows, k))
+
+
+def nvfp4_launch_count() -> int:
+    return int(lib().nvfp4_launch_count())
+
+
+def nvfp4_quantize(x, rows, k, ld_x, codes, sf, tensor_scale, flags=0, workspace=None,
+                   workspace_bytes=0, dev_status=None, stream=None) -> None:
+    st = lib().nvfp4_quantize(_ptr(x), rows, k, ld_x, _ptr(codes), _ptr(sf), _ptr(tensor_scale),
+                              flags, _ptr(workspace), workspace_bytes, _ptr(dev_status), _stream(stream))
+    check(st, "nvfp4_quantize")
+
+
+def nvfp4_dequantize(codes, sf, tensor_scale, rows, k, out, out_dtype, stream=None) -> None:
+    st = lib().nvfp4_dequantize(_ptr(codes), _ptr(sf), _ptr(tensor_scale), rows, k, _ptr(out),
+                                out_dtype, _stream(stream))
+    check(st, "nvfp4_dequantize")
+
+
+def nvfp4_gemm_w4a4(a_codes, a_sf, a_scale, b_codes, b_sf, b_scale, M, N, K, y=None,
+                    y_dtype=NVFP4_DTYPE_BF16, y_codes=None, y_sf=None, y_scale=None, y_amax=None,
+                    dev_status=None, stream=None) -> None:
+    st = lib().nvfp4_gemm_w4a4(_ptr(a_codes), _ptr(a_sf), _ptr(a_scale), _ptr(b_codes), _ptr(b_sf),
+                               _ptr(b_scale), M, N, K, _ptr(y), y_dtype, _ptr(y_codes), _ptr(y_sf),
+                               _ptr(y_scale), _ptr(y_amax), _ptr(dev_status), _stream(stream))
+    check(st, "nvfp4_gemm_w4a4")
+
+
+def nvfp4_gemm_w4a16(x, w_codes, w_sf, w_scale, M, N, K, y, y_dtype=NVFP4_DTYPE_BF16,
+                     dev_status=None, stream=None) -> None:
+    st = lib().nvfp4_gemm_w4a16(_ptr(x), _ptr(w_codes), _ptr(w_sf), _ptr(w_scale), M, N, K, _ptr(y),
+                                y_dtype, _ptr(dev_status), _stream(stream))
+    check(st, "nvfp4_gemm_w4a16")
+
+
+# ----------------------------------------------------------------- convenience
+@dataclass
+class NVFP4Tensor:
+    """codes [rows, k/2] uint8, sf [sf_bytes] uint8 (tensor-core layout),
+    scale [1] float32 -- all on one CUDA device."""
+    codes: torch.Tensor
+    sf: torch.Tensor
+    scale: torch.Tensor
+    rows: int
+    k: int
+
+    @staticmethod
+    def empty(rows: int, k: int, device) -> "NVFP4Tensor":
+        return NVFP4Tensor(torch.empty(rows, k // 2, dtype=torch.uint8, device=device),
+                           torch.empty(max(nvfp4_sf_bytes(rows, k), 16), dtype=torch.uint8, device=device),
+                           torch.zeros(1, dtype=torch.float32, device=device), rows, k)
+
+
+def quantize(x: torch.Tensor, scale: torch.Tensor | float | None = None, out: NVFP4Tensor | None = None,
+             workspace: torch.Tensor | None = None, dev_status=None, stream=None) -> NVFP4Tensor:
+    """Quantize a bf16 [rows, k] CUDA tensor.  ``scale`` given -> used as the
+    tensor scale g; otherwise g = amax / 2688 is computed on the device."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, k = x.shape
+    q = out if out is not None else NVFP4Tensor.empty(rows, k, x.device)
+    flags = 0
+    if scale is not None:
+        if isinstance(scale, torch.Tensor):
+            q.scale.copy_(scale.reshape(1).to(torch.float32))
+        else:
+            q.scale.fill_(float(scale))
+        flags = NVFP4_SCALE_GIVEN
+    wsb = nvfp4_quantize_workspace_bytes(rows, k)
+    if flags == 0 and workspace is None:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=x.device)
+    nvfp4_quantize(x, rows, k, x.stride(0), q.codes, q.sf, q.scale, flags,
+                   workspace if flags == 0 else None, wsb if flags == 0 else 0, dev_status, stream)
+    return q
+
+
+def dequantize(q: NVFP4Tensor, dtype=torch.bfloat16, stream=None) -> torch.Tensor:
+    out = torch.empty(q.rows, q.k, dtype=dtype, device=q.codes.device)
+    nvfp4_dequantize(q.codes, q.sf, q.scale, q.rows, q.k, out, _DT[dtype], stream)
+    return out
+
+
+def gemm_w4a4(a: NVFP4Tensor, b: NVFP4Tensor, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
+              dev_status=None, stream=None) -> torch.Tensor:
+    """Y = A B^T, A [M,K] activations, B [N,K] weights, both NVFP4."""
+    assert a.k == b.k
+    y = out if out is not None else torch.empty(a.rows, b.rows, dtype=out_dtype, device=a.codes.device)
+    nvfp4_gemm_w4a4(a.codes, a.sf, a.scale, b.codes, b.sf, b.scale, a.rows, b.rows, a.k, y=y,
+                    y_dtype=_DT[y.dtype], dev_status=dev_status, stream=stream)
+    return y
+
+
+def gemm_w4a4_nvfp4_out(a: NVFP4Tensor, b: NVFP4Tensor, y_scale: torch.Tensor, y_amax: torch.Tensor | None = None,
+                        out: NVFP4Tensor | None = None, dev_status=None, stream=None) -> NVFP4Tensor:
+    """Y = A B^T emitted directly as NVFP4 with the caller's tensor scale."""
+    q = out if out is not None else NVFP4Tensor.empty(a.rows, b.rows, a.codes.device)
+    q.scale.copy_(y_scale.reshape(1))
+    nvfp4_gemm_w4a4(a.codes, a.sf, a.scale, b.codes, b.sf, b.scale, a.rows, b.rows, a.k,
+                    y_codes=q.codes, y_sf=q.sf, y_scale=q.scale, y_amax=y_amax, dev_status=dev_status,
+                    stream=stream)
+    return q
+
+
+def gemm_w4a16(x: torch.Tensor, w: NVFP4Tensor, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
+               dev_status=None, stream=None) -> torch.Tensor:
+    """Y = X W^T, X bf16 [M,K], W NVFP4 [N,K]."""
+    assert x.dtype == torch.bfloat16 and x.is_contiguous() and x.shape[1] == w.k
+    y = out if out is not None else torch.empty(x.shape[0], w.rows, dtype=out_dtype, device=x.device)
+    nvfp4_gemm_w4a16(x, w.codes, w.sf, w.scale, x.shape[0], w.rows, w.k, y, _DT[y.dtype], dev_status, stream)
+    return y

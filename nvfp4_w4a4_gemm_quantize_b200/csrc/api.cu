@@ -1,0 +1,208 @@
+// api.cu -- the C ABI (include/nvfp4.h): host-side argument checks, device
+// capability check, and the kernel launches.  No call allocates device memory
+// and none synchronizes the host.
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/nvfp4.h"
+#include "internal.h"
+#include "tmap.h"
+
+namespace nvfp4 {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+// ------------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+CUresult make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes,
+                      uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                      CUtensorMapSwizzle swizzle) {
+    (void)elem_bytes;
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return CUDA_ERROR_NOT_FOUND;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+// ------------------------------------------------------------------ device
+struct DevInfo {
+    int checked = 0;   // 0 unknown, 1 ok, -1 unsupported
+    int sms = 0;
+};
+static DevInfo g_dev[64];
+
+static nvfp4_status device_ok(int* sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return NVFP4_ERR_UNSUPPORTED_DEVICE;
+    DevInfo& d = g_dev[dev];
+    if (d.checked == 0) {
+        int major = 0, minor = 0, n = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        d.sms = n;
+        d.checked = (major == 10 && minor == 0) ? 1 : -1;
+    }
+    if (d.checked < 0) return NVFP4_ERR_UNSUPPORTED_DEVICE;
+    if (sms) *sms = d.sms;
+    return NVFP4_OK;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" {
+
+size_t nvfp4_sf_bytes(int64_t rows, int64_t k) {
+    if (rows < 0 || k <= 0 || (k % 64) != 0) return 0;
+    return (size_t)((rows + 127) / 128) * 128 * (size_t)(k / 16);
+}
+
+size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t k) {
+    (void)rows;
+    (void)k;
+    return kQuantWorkspaceBytes;
+}
+
+nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, uint8_t* codes, uint8_t* sf,
+                            float* tensor_scale, unsigned flags, void* workspace, size_t workspace_bytes,
+                            int* dev_status, nvfp4_stream_t stream) {
+    (void)dev_status;
+    if (rows < 0 || k <= 0 || ld_x < k) return NVFP4_ERR_INVALID_ARG;
+    if ((flags & ~(unsigned)NVFP4_SCALE_GIVEN) != 0u) return NVFP4_ERR_INVALID_ARG;
+    if (!tensor_scale) return NVFP4_ERR_INVALID_ARG;
+    if (rows > 0 && (!x_bf16 || !codes || !sf)) return NVFP4_ERR_INVALID_ARG;
+    if (k % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (rows > (int64_t)1 << 31 || k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    const bool given = (flags & NVFP4_SCALE_GIVEN) != 0u;
+    if (!given && (!workspace || workspace_bytes < kQuantWorkspaceBytes)) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(sf) || (ld_x % 8) != 0 ||
+        (!given && !aligned16(workspace)) || (reinterpret_cast<uintptr_t>(tensor_scale) & 3u))
+        return NVFP4_ERR_MISALIGNED;
+    nvfp4_status st = device_ok(nullptr);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (rows == 0) {
+        if (!given) return cuda_status(cudaMemsetAsync(tensor_scale, 0, sizeof(float), s));
+        return NVFP4_OK;
+    }
+    return cuda_status(launch_quantize(static_cast<const uint16_t*>(x_bf16), rows, k, ld_x, codes, sf, tensor_scale,
+                                       given, static_cast<float*>(workspace), s));
+}
+
+nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* sf, const float* tensor_scale, int64_t rows,
+                              int64_t k, void* out, int out_dtype, nvfp4_stream_t stream) {
+    if (rows < 0 || k <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (out_dtype != NVFP4_DTYPE_BF16 && out_dtype != NVFP4_DTYPE_F32) return NVFP4_ERR_INVALID_ARG;
+    if (rows > 0 && (!codes || !sf || !tensor_scale || !out)) return NVFP4_ERR_INVALID_ARG;
+    if (k % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(codes) || !aligned16(sf) || !aligned16(out)) return NVFP4_ERR_MISALIGNED;
+    nvfp4_status st = device_ok(nullptr);
+    if (st != NVFP4_OK) return st;
+    if (rows == 0) return NVFP4_OK;
+    return cuda_status(launch_dequantize(codes, sf, tensor_scale, rows, k, out, out_dtype == NVFP4_DTYPE_BF16,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_scale,
+                             const uint8_t* b_codes, const uint8_t* b_sf, const float* b_scale, int64_t M, int64_t N,
+                             int64_t K, void* y, int y_dtype, uint8_t* y_codes, uint8_t* y_sf, const float* y_scale,
+                             float* y_amax, int* dev_status, nvfp4_stream_t stream) {
+    if (M < 0 || N <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (K % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0) return NVFP4_OK;                 /* nothing to read or write */
+    if (!a_codes || !a_sf || !b_codes || !b_sf || !a_scale || !b_scale) return NVFP4_ERR_INVALID_ARG;
+    if (y) {
+        if (y_dtype != NVFP4_DTYPE_BF16 && y_dtype != NVFP4_DTYPE_F32) return NVFP4_ERR_INVALID_ARG;
+        if (y_codes || y_sf) return NVFP4_ERR_INVALID_ARG;
+    } else {
+        if (!y_codes || !y_sf || !y_scale) return NVFP4_ERR_INVALID_ARG;
+    }
+    if (K % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (y && y_dtype == NVFP4_DTYPE_BF16 && N % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (y && y_dtype == NVFP4_DTYPE_F32 && N % 4 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!y && N % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (M >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(b_codes) || !aligned16(b_sf) ||
+        (y && !aligned16(y)) || (y_codes && !aligned16(y_codes)) || (y_sf && !aligned16(y_sf)))
+        return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    nvfp4_status st = device_ok(&sms);
+    if (st != NVFP4_OK) return st;
+    GemmW4A4Args a{a_codes, a_sf, a_scale, b_codes, b_sf, b_scale, M, N, K, y, y_dtype,
+                   y_codes, y_sf, y_scale, y_amax, dev_status};
+    return cuda_status(launch_gemm_w4a4(a, sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_gemm_w4a16(const void* x_bf16, const uint8_t* w_codes, const uint8_t* w_sf, const float* w_scale,
+                              int64_t M, int64_t N, int64_t K, void* y, int y_dtype, int* dev_status,
+                              nvfp4_stream_t stream) {
+    if (M < 0 || N <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (K % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0) return NVFP4_OK;                 /* nothing to read or write */
+    if (!x_bf16 || !w_codes || !w_sf || !w_scale || !y) return NVFP4_ERR_INVALID_ARG;
+    if (y_dtype != NVFP4_DTYPE_BF16 && y_dtype != NVFP4_DTYPE_F32) return NVFP4_ERR_INVALID_ARG;
+    if (K % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (y_dtype == NVFP4_DTYPE_BF16 && N % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (y_dtype == NVFP4_DTYPE_F32 && N % 4 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (M >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x_bf16) || !aligned16(w_codes) || !aligned16(w_sf) || !aligned16(y)) return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    nvfp4_status st = device_ok(&sms);
+    if (st != NVFP4_OK) return st;
+    GemmW4A16Args a{static_cast<const uint16_t*>(x_bf16), w_codes, w_sf, w_scale, M, N, K, y, y_dtype, dev_status};
+    return cuda_status(launch_gemm_w4a16(a, sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+const char* nvfp4_status_string(nvfp4_status s) {
+    switch (s) {
+        case NVFP4_OK: return "ok";
+        case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+        case NVFP4_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case NVFP4_ERR_MISALIGNED: return "pointer or stride not 16-byte aligned";
+        case NVFP4_ERR_UNSUPPORTED_DEVICE: return "device is not compute capability 10.0 (B200)";
+        case NVFP4_ERR_CUDA: return "CUDA error";
+        case NVFP4_ERR_TIMEOUT: return "device-side wait timed out";
+        case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+uint64_t nvfp4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_sf_offset.restype = _i64
         L.oracle_tensor_scale_f32.argtypes = [_p, _i64, _i64, _i64]
         L.oracle_tensor_scale_f32.restype = _f32
+        L.oracle_tensor_scale_bf16.argtypes = [_p, _i64, _i64, _i64]
+        L.oracle_tensor_scale_bf16.restype = _f32
         for name in ("oracle_quantize_f32", "oracle_quantize_bf16"):
             fn = getattr(L, name)
             fn.argtypes = [_p, _i64, _i64, _i64, ctypes.c_int, _p, _p, _p]
@@ -239,3 +241,16 @@ def sf_matrix(sf: np.ndarray, rows: int, k: int) -> np.ndarray:
     c = np.arange(kb)[None, :]
     off = ((r // 128) * (kb // 4) + c // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + c % 4
     return sf[off]
+
+
+def tensor_scale(x) -> np.float32:
+    """g = amax(|x|) / 2688 in IEEE single (the tensor-level scale of the RFC's
+    two-level scaling)."""
+    L = lib()
+    if isinstance(x, np.ndarray) and x.dtype == np.float32:
+        xa = np.ascontiguousarray(x)
+        rows, k = xa.shape
+        return np.float32(L.oracle_tensor_scale_f32(_ptr(xa), rows, k, k))
+    xb = bf16_bits(x)
+    rows, k = xb.shape
+    return np.float32(L.oracle_tensor_scale_bf16(_ptr(xb), rows, k, k))

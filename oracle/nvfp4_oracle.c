@@ -178,6 +178,18 @@ float oracle_tensor_scale_f32(const float *x, int64_t rows, int64_t k, int64_t l
     return amax / 2688.0f;
 }
 
+/* The same tensor scale over a bf16 tensor (bf16 -> fp32 is exact). */
+float oracle_tensor_scale_bf16(const uint16_t *x, int64_t rows, int64_t k, int64_t ld)
+{
+    float amax = 0.0f;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < k; ++j) {
+            float a = fabsf(oracle_bf16_to_f32(x[r * ld + j]));
+            if (a > amax) amax = a;
+        }
+    return amax / 2688.0f;
+}
+
 /* Two-level NVFP4 quantization of an FP32 tensor x[rows, k] (row stride ld):
  *   g  = amax / 2688 unless scale_given (then g = *g_io)        [RFC, Motivation]
  *   per row, per 16 consecutive values along k:

@@ -25,3 +25,10 @@ def cuda_ok():
     if not _has_gpu():
         pytest.skip("no CUDA device")
     return True
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _built_library():
+    """Compile libnvfp4.so (nvcc, sm_100a) if a source changed; cheap otherwise."""
+    from nvfp4_w4a4_gemm_quantize_b200 import build
+    build.build()

@@ -1,0 +1,121 @@
+"""The C ABI library loads and exports every symbol include/nvfp4.h declares;
+host-side argument checks reject bad calls before any launch (no GPU needed:
+each call below fails its checks before touching the device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from nvfp4_w4a4_gemm_quantize_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4.h")
+
+OK, INVALID, SHAPE, MISALIGNED, DEVICE, CUDA, TIMEOUT, WORKSPACE = range(8)
+A = 0x10000          # fake, 16-byte aligned device addresses (never dereferenced)
+B = 0x20000
+C = 0x30000
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _lib.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) == 8, names
+    for n in names:
+        assert hasattr(L, n), n
+        assert n in _lib.SIGNATURES, n
+
+
+def test_sf_bytes_and_workspace(L):
+    assert L.nvfp4_sf_bytes(128, 256) == 128 * 16
+    assert L.nvfp4_sf_bytes(600, 4096) == 640 * 256
+    assert L.nvfp4_sf_bytes(0, 64) == 0
+    assert L.nvfp4_sf_bytes(5, 32) == 0          # k not a multiple of 64
+    assert L.nvfp4_sf_bytes(-1, 64) == 0
+    assert L.nvfp4_quantize_workspace_bytes(32768, 12288) >= 1024
+
+
+def test_status_strings(L):
+    for s in range(8):
+        assert L.nvfp4_status_string(s)
+    assert b"unknown" in L.nvfp4_status_string(99)
+
+
+def test_quantize_rejects_bad_arguments(L):
+    q = L.nvfp4_quantize
+    # k not a multiple of 64
+    assert q(A, 128, 96, 96, B, C, A, 1, None, 0, None, None) == SHAPE
+    # null input
+    assert q(None, 128, 256, 256, B, C, A, 1, None, 0, None, None) == INVALID
+    # null tensor scale
+    assert q(A, 128, 256, 256, B, C, None, 1, None, 0, None, None) == INVALID
+    # ld_x < k
+    assert q(A, 128, 256, 128, B, C, A, 1, None, 0, None, None) == INVALID
+    # unknown flag
+    assert q(A, 128, 256, 256, B, C, A, 4, None, 0, None, None) == INVALID
+    # dynamic scale without workspace
+    assert q(A, 128, 256, 256, B, C, A, 0, None, 0, None, None) == WORKSPACE
+    assert q(A, 128, 256, 256, B, C, A, 0, A, 16, None, None) == WORKSPACE
+    # misaligned pointers / row stride
+    assert q(A + 2, 128, 256, 256, B, C, A, 1, None, 0, None, None) == MISALIGNED
+    assert q(A, 128, 256, 260, B, C, A, 1, None, 0, None, None) == MISALIGNED
+    assert q(A, 128, 256, 256, B + 8, C, A, 1, None, 0, None, None) == MISALIGNED
+
+
+def test_dequantize_rejects_bad_arguments(L):
+    d = L.nvfp4_dequantize
+    assert d(A, B, C, 128, 256, A, 7, None) == INVALID
+    assert d(A, B, C, 128, 100, A, 0, None) == SHAPE
+    assert d(None, B, C, 128, 256, A, 0, None) == INVALID
+    assert d(A + 4, B, C, 128, 256, A, 0, None) == MISALIGNED
+
+
+def test_gemm_rejects_bad_arguments(L):
+    g = L.nvfp4_gemm_w4a4
+    args = [A, B, C, A, B, C]
+    # K not multiple of 64
+    assert g(*args, 128, 256, 96, A, 0, None, None, None, None, None, None) == SHAPE
+    # N not multiple of 8 for bf16 output
+    assert g(*args, 128, 260, 256, A, 0, None, None, None, None, None, None) == SHAPE
+    # fused NVFP4 output needs N % 64 == 0
+    assert g(*args, 128, 96, 256, None, 0, A, B, C, None, None, None) == SHAPE
+    # both outputs given
+    assert g(*args, 128, 256, 256, A, 0, A, B, C, None, None, None) == INVALID
+    # no output at all
+    assert g(*args, 128, 256, 256, None, 0, None, None, None, None, None, None) == INVALID
+    # bad dtype
+    assert g(*args, 128, 256, 256, A, 5, None, None, None, None, None, None) == INVALID
+    # null scale
+    assert g(A, B, None, A, B, C, 128, 256, 256, A, 0, None, None, None, None, None, None) == INVALID
+    # misaligned operand
+    assert g(A + 1, B, C, A, B, C, 128, 256, 256, A, 0, None, None, None, None, None, None) == MISALIGNED
+    # negative M
+    assert g(*args, -1, 256, 256, A, 0, None, None, None, None, None, None) == INVALID
+
+
+def test_w4a16_rejects_bad_arguments(L):
+    g = L.nvfp4_gemm_w4a16
+    assert g(A, B, C, A, 128, 256, 96, A, 0, None, None) == SHAPE
+    assert g(A, B, C, A, 128, 250, 256, A, 0, None, None) == SHAPE
+    assert g(None, B, C, A, 128, 256, 256, A, 0, None, None) == INVALID
+    assert g(A, B, C, A, 128, 256, 256, None, 0, None, None) == INVALID
+    assert g(A + 2, B, C, A, 128, 256, 256, A, 0, None, None) == MISALIGNED
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "absent.so"))
+    monkeypatch.setattr(_lib, "_LIB", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        _lib.lib()
