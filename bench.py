@@ -175,12 +175,19 @@ def run_ours(args):
         build.build()
     barrier(world)
     wl = synth.WORKLOADS[WORKLOAD]
+    if args.layers or args.m:
+        # a reduced case for profiling captures: selected layers and/or fewer tokens
+        import dataclasses
+        keep = [L for L in wl.layers if not args.layers or L.name in args.layers.split(",")]
+        keep = [dataclasses.replace(L, M=args.m or L.M) for L in keep]
+        wl = dataclasses.replace(wl, layers=tuple(keep))
     peaks, peak_src = load_peaks()
 
     # ---- data (resident in HBM before timing); each rank its own batch
     xs, Ws, Aq, Ys = [], [], [], []
     for L in wl.layers:
         x, w = synth.layer_tensors(WORKLOAD, L.name, device=dev)
+        x = x[: L.M].contiguous()
         if rank:
             x = x.roll(rank * 977, dims=0)
         xs.append(x)
@@ -270,7 +277,8 @@ def run_ours(args):
         fp4_peak = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"]) * FP4_OVER_BF16
         hbm_peak = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
         # dominant kernel: the GEMM of the largest layer (fc1, the 32768x3072x12288 shape)
-        li = [L.name for L in wl.layers].index("fc1")
+        names = [L.name for L in wl.layers]
+        li = names.index("fc1") if "fc1" in names else 0
         L = wl.layers[li]
         g_flops = 2 * L.M * L.N * L.K
         g_tflops = g_flops / (gemm_ms[li] * 1e-3) / 1e12
@@ -289,7 +297,7 @@ def run_ours(args):
                                    "(dynamic-scale activation quantize + W4A4 GEMM, bf16 out)",
                        "l2": "inputs larger than L2 (X 201-805 MB per layer, >2 GB streamed per step)",
                        "parallelism": f"replica per GPU x{world}"},
-            "roofline": {"bound": "tensor", "kernel": "gemm_w4a4 fc1 32768x3072x12288",
+            "roofline": {"bound": "tensor", "kernel": f"gemm_w4a4 {L.name} {L.M}x{L.K}x{L.N}",
                          "achieved": round(g_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                          "frac": round(g_tflops / fp4_peak, 4),
                          "peak_source": f"{peak_src} bf16 x {FP4_OVER_BF16:g} (nominal FP4/bf16 ratio)",
@@ -319,6 +327,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-rows", type=int, default=48)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", default="", help="profiling: comma-separated subset of layers")
+    ap.add_argument("--m", type=int, default=0, help="profiling: tokens (rows of X) per layer")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

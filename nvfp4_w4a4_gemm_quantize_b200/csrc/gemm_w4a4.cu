@@ -414,15 +414,11 @@ cudaError_t launch_cfg(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) 
 cudaError_t launch_gemm_w4a4(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) {
     using namespace w4a4;
     if (a.M == 0) return cudaSuccess;
+    // N a multiple of 256: CTA-pair kernel with 256 x 256 tiles.  Otherwise
+    // (N = 1152, 3456, ...): single-CTA 128 x 128 tiles with a double-buffered
+    // accumulator, so no tile column is wasted on padding.
+    if (a.N % 256 == 0) return launch_gemm_w4a4_2sm(a, num_sms, stream);
     const int out = a.y != nullptr ? (a.y_dtype == 1 ? OUT_F32 : OUT_BF16) : OUT_NVFP4;
-    // N tile: 256 when N is a multiple of 256 (single accumulator, fewer
-    // operand re-reads), else 128 (double-buffered accumulator).
-    const bool wide = (a.N % 256) == 0;
-    if (wide) {
-        if (out == OUT_BF16) return launch_cfg<256, 3, OUT_BF16>(a, num_sms, stream);
-        if (out == OUT_F32) return launch_cfg<256, 3, OUT_F32>(a, num_sms, stream);
-        return launch_cfg<256, 3, OUT_NVFP4>(a, num_sms, stream);
-    }
     if (out == OUT_BF16) return launch_cfg<128, 5, OUT_BF16>(a, num_sms, stream);
     if (out == OUT_F32) return launch_cfg<128, 5, OUT_F32>(a, num_sms, stream);
     return launch_cfg<128, 5, OUT_NVFP4>(a, num_sms, stream);

@@ -1,0 +1,494 @@
+// gemm_w4a4_2sm.cu -- the W4A4 GEMM on CTA pairs (tcgen05 cta_group::2):
+// one 256 x 256 output tile per pair, each CTA holding 128 rows of A, one
+// 128-row half of B and the full 256-row set of B scales; per K step the
+// leader CTA issues a single M=256, N=256, K=64 block-scaled MMA whose
+// accumulator rows land in both CTAs' TMEM.
+//
+// Same operation as gemm_w4a4.cu ("NVFP4-DiT ..." README, Methodology 3;
+// "[RFC]: NVFP4 Quantization Support for Diffusion Models", Open Questions 1):
+//   Y[m,n] = (g_a g_b) * sum_k (e2m1(a) e4m3(sfa)) (e2m1(b) e4m3(sfb))
+//
+// Why pairs: per SM, a 128 x 256 x 256 K-stage needs 38 KB of operands
+// instead of 54 KB for a single-CTA 128 x 256 tile, so five stages fit in
+// shared memory, and L2 -> SM operand traffic per output drops by a third.
+//
+// Roles (512 threads per CTA, four warpgroups):
+//   warps 0-3  scale writers, both CTAs: per stage, every lane loads one
+//              16-byte row of each 512-byte scale atom from shared memory and
+//              tcgen05.st's it into its own TMEM lane quarter (the layout the
+//              block-scaled MMA reads: four replicated quarters).  Then the
+//              warp arrives on the leader's per-stage "ready" barrier, which
+//              therefore also says "this CTA's operands have landed".
+//              (tcgen05.cp of the 12 atoms per stage costs ~12 x 100 cycles
+//              of tensor-pipe time per pair, more than the 4 MMAs it feeds;
+//              the register path costs ~70 cycles per stage off that pipe.)
+//   warp 4     producer, both CTAs: TMA loads of this CTA's A rows, B half,
+//              A scales and all B scales into a STAGES-deep ring.
+//   warp 5     leader CTA: MMA issuer (tcgen05.mma cta_group::2, commits
+//              multicast to both CTAs' barriers).
+//   warps 8-15 epilogue, both CTAs: the 128 x 256 FP32 accumulator slice is
+//              read into registers (two warps per TMEM lane quarter, 128
+//              columns each) and released to the MMA issuer at once, then
+//              converted and stored while the next tile's mainloop runs.
+// Registers: launched at 128 per thread; warpgroups 0-1 drop to 56 and the
+// epilogue warpgroups rise to 200 (256 x 56 + 256 x 200 = 512 x 128).
+// No load uses cluster multicast: every CTA fetches its own tiles.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "quant_math.cuh"
+#include "tmap.h"
+
+namespace nvfp4 {
+namespace w4a4_2sm {
+
+constexpr int BK_BYTES = 128;                    // 256 FP4 values per row per stage
+constexpr int A_BYTES = 128 * BK_BYTES;          // this CTA's 128 rows of A
+constexpr int B_BYTES = 128 * BK_BYTES;          // this CTA's 128-row half of B
+constexpr int SF_ATOM = 512;
+constexpr int SFA_BYTES = 4 * SF_ATOM;           // 128 rows x 4 K=64 steps
+constexpr int SFB_BYTES = 2 * 4 * SF_ATOM;       // 256 rows x 4 K=64 steps
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // 38912
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 512;
+constexpr int kSfWarps = 4;
+constexpr int kRegsLow = 56;                     // warpgroups 0-1
+constexpr int kRegsHigh = 200;                   // epilogue warpgroups 2-3
+static_assert(256 * kRegsLow + 256 * kRegsHigh <= kThreads * 128, "register split exceeds the launch budget");
+constexpr int SF_COLS_STEP = 4 + 8;              // SFA 4 columns, SFB 8 columns per K=64 step
+constexpr int SF_COLS_STAGE = 4 * SF_COLS_STEP;
+constexpr int kGroupM = 8;                       // rasterisation group, in 256-row pair tiles
+constexpr int kSmemLimit = 232448;
+
+enum OutKind { OUT_BF16 = 0, OUT_F32 = 1, OUT_NVFP4 = 2 };
+
+template <int OUT>
+struct Cfg {
+    static constexpr int EPI_BUF = OUT == OUT_F32 ? 4096 : (OUT == OUT_BF16 ? 2048 : 0);   // 32 rows x 32 cols
+    static constexpr int EPI_BYTES = kEpiWarps * 2 * EPI_BUF;
+    static constexpr int FIT = (kSmemLimit - 1024 - EPI_BYTES) / STAGE_BYTES;
+    static constexpr int STAGES = FIT < 5 ? FIT : 5;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024;
+    static_assert(STAGES >= 3, "pipeline depth");
+    static_assert(256 + STAGES * SF_COLS_STAGE <= 512, "TMEM columns");
+};
+
+struct Params {
+    const float* a_scale;
+    const float* b_scale;
+    int M, N, K;
+    int num_mb2, num_nb, num_tiles;
+    uint8_t* y_codes;
+    uint8_t* y_sf;
+    const float* y_scale;
+    float* y_amax;
+    int* dev_status;
+};
+
+__device__ __forceinline__ void tile_coords(int t, int num_mb2, int num_nb, int& mb2, int& nb) {
+    const int per_group = kGroupM * num_nb;
+    const int group = t / per_group;
+    const int first = group * kGroupM;
+    const int gm = min(kGroupM, num_mb2 - first);
+    const int idx = t - group * per_group;
+    mb2 = first + idx % gm;
+    nb = idx / gm;
+}
+
+// Store 32 FP32 accumulator columns (alpha applied) of one row per lane
+// through a swizzled staging buffer and a TMA store of a 32 x 32 box.
+template <int OUT>
+__device__ __forceinline__ void store_chunk(const uint32_t* r, float alpha, uint8_t* buf, int lane,
+                                            const CUtensorMap* map, int x, int y) {
+    if (OUT == OUT_BF16) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(alpha, __uint_as_float(r[2 * j])),
+                                                     __fmul_rn(alpha, __uint_as_float(r[2 * j + 1])));
+            pk[j] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        // 64-byte rows, 64-byte swizzle: chunk j of row i at j ^ ((i >> 1) & 3)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int pos = j ^ ((lane >> 1) & 3);
+            *reinterpret_cast<uint4*>(buf + lane * 64 + pos * 16) =
+                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        }
+    } else {
+        // 128-byte rows, 128-byte swizzle: chunk j of row i at j ^ (i & 7)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int pos = j ^ (lane & 7);
+            *reinterpret_cast<float4*>(buf + lane * 128 + pos * 16) =
+                make_float4(__fmul_rn(alpha, __uint_as_float(r[4 * j])), __fmul_rn(alpha, __uint_as_float(r[4 * j + 1])),
+                            __fmul_rn(alpha, __uint_as_float(r[4 * j + 2])), __fmul_rn(alpha, __uint_as_float(r[4 * j + 3])));
+        }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(map, buf, x, y);
+        bulk_commit_group();
+    }
+}
+
+template <int OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+             const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
+             const __grid_constant__ CUtensorMap tmap_y, const Params p) {
+    using C = Cfg<OUT>;
+    constexpr int STAGES = C::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[STAGES], ready_bar[STAGES], empty_bar[STAGES];
+    __shared__ __align__(8) uint64_t accf_bar, acce_bar, drain_bar;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int pair = (int)cluster_id_x();
+    const int npairs = (int)nclusters_x();
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    WaitCtx wc{&abort_sh, p.dev_status};
+
+    if (threadIdx.x == 0) {
+        abort_sh = 0;
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&ready_bar[s], 2 * kSfWarps);
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(&accf_bar, 1);
+        mbar_init(&acce_bar, 2 * kEpiWarps);
+        mbar_init(&drain_bar, 1);
+        fence_barrier_init();
+        tma_prefetch_desc(&tmap_a);
+        tma_prefetch_desc(&tmap_b);
+        tma_prefetch_desc(&tmap_sfa);
+        tma_prefetch_desc(&tmap_sfb);
+        tma_prefetch_desc(&tmap_y);
+    }
+    // scale regions start as zeros (finite) so rows that are never loaded
+    // (beyond M or N) multiply zero codes by a finite scale
+    for (int s = 0; s < STAGES; ++s) {
+        uint32_t* z = reinterpret_cast<uint32_t*>(smem + s * STAGE_BYTES + A_BYTES + B_BYTES);
+        for (int i = threadIdx.x; i < (SFA_BYTES + SFB_BYTES) / 4; i += kThreads) z[i] = 0u;
+    }
+    fence_proxy_async_smem();
+    cluster_sync_all();                       // barriers initialised in both CTAs
+    if (warp == 0) {
+        tmem_alloc2(&tmem_base_sh, 512);
+        tmem_relinquish2();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_sh;
+
+    const int num_kt = (p.K + 255) / 256;
+    const int k_atoms = p.K / 64;
+    const uint32_t sf_base = tmem_base + 256;
+    // one register-budget change per warpgroup, before the roles diverge
+    if (warp < 8)
+        regs_dec<kRegsLow>();
+    else
+        regs_inc<kRegsHigh>();
+
+    if (warp < 4) {
+        // ------------------------------------------------------------ scale writers (both CTAs)
+        const uint32_t q = (uint32_t)warp;            // TMEM lane quarter of this warp
+        const uint32_t lane_off = (q * 32u) << 16;
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int t = pair; t < p.num_tiles; t += npairs) {
+            bool ok = true;
+            for (int kt = 0; kt < num_kt; ++kt) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[stage], phase, wc) ? 1 : 0)) { ok = false; break; }
+                const uint8_t* sfa_s = smem + stage * STAGE_BYTES + A_BYTES + B_BYTES;
+                const uint8_t* sfb_s = sfa_s + SFA_BYTES;
+                const uint32_t col0 = sf_base + lane_off + stage * SF_COLS_STAGE;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint4 va = *reinterpret_cast<const uint4*>(sfa_s + ks * SF_ATOM + lane * 16);
+                    const uint4 vb0 = *reinterpret_cast<const uint4*>(sfb_s + ks * SF_ATOM + lane * 16);
+                    const uint4 vb1 = *reinterpret_cast<const uint4*>(sfb_s + 4 * SF_ATOM + ks * SF_ATOM + lane * 16);
+                    const uint32_t col = col0 + ks * SF_COLS_STEP;
+                    tmem_st_32x32b_x4(col, va.x, va.y, va.z, va.w);
+                    tmem_st_32x32b_x4(col + 4, vb0.x, vb0.y, vb0.z, vb0.w);
+                    tmem_st_32x32b_x4(col + 8, vb1.x, vb1.y, vb1.z, vb1.w);
+                }
+                tmem_st_wait();                       // the scale columns are in TMEM
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (rank == 0)
+                        mbar_arrive(&ready_bar[stage]);
+                    else
+                        mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&ready_bar[stage]), 0));
+                }
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+        }
+    } else if (warp == 4) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        if (lane == 0) {
+            const uint64_t pol_a = policy_evict_normal();
+            const uint64_t pol_b = policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0, issued = 0, issued_any = 0;
+            bool ok = true;
+            for (int t = pair; t < p.num_tiles && ok; t += npairs) {
+                int mb2, nb;
+                tile_coords(t, p.num_mb2, p.num_nb, mb2, nb);
+                const int arow = mb2 * 256 + (int)rank * 128;
+                const int brow = nb * 256 + (int)rank * 128;
+                const int sfa_row = (mb2 * 2 + (int)rank) * k_atoms;
+                const int sfb_row0 = (nb * 2) * k_atoms, sfb_row1 = (nb * 2 + 1) * k_atoms;
+                for (int kt = 0; kt < num_kt; ++kt) {
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, wc)) { ok = false; break; }
+                    uint8_t* sb = smem + stage * STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full_bar[stage], STAGE_BYTES);
+                    tma_load_2d(sb, &tmap_a, &full_bar[stage], kt * BK_BYTES, arow, pol_a);
+                    tma_load_2d(sb + A_BYTES, &tmap_b, &full_bar[stage], kt * BK_BYTES, brow, pol_b);
+                    tma_load_2d(sb + A_BYTES + B_BYTES, &tmap_sfa, &full_bar[stage], 0, sfa_row + kt * 4, pol_a);
+                    tma_load_2d(sb + A_BYTES + B_BYTES + SFA_BYTES, &tmap_sfb, &full_bar[stage], 0,
+                                sfb_row0 + kt * 4, pol_b);
+                    tma_load_2d(sb + A_BYTES + B_BYTES + SFA_BYTES + 4 * SF_ATOM, &tmap_sfb, &full_bar[stage], 0,
+                                sfb_row1 + kt * 4, pol_b);
+                    issued = (issued & ~(1u << stage)) | (phase << stage);
+                    issued_any |= 1u << stage;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            // this CTA's own loads have all landed before it may exit
+            int no_abort = 0;
+            WaitCtx w2{&no_abort, p.dev_status};
+            for (int s = 0; s < STAGES; ++s)
+                if (issued_any & (1u << s)) mbar_wait(&full_bar[s], (issued >> s) & 1u, w2);
+        }
+    } else if (warp < 8) {
+        if (warp == 5 && lane == 0 && rank == 0) {
+            // -------------------------------------------------------- MMA issuer (leader)
+            constexpr uint32_t idesc = idesc_nvf4(256, 256);
+            int stage = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int t = pair; t < p.num_tiles && ok; t += npairs) {
+                if (!mbar_wait_cluster(&acce_bar, acc_phase ^ 1u, wc)) { ok = false; break; }
+                tc_fence_after();
+                for (int kt = 0; kt < num_kt; ++kt) {
+                    // both CTAs' operands have landed and their scales sit in TMEM
+                    if (!mbar_wait_cluster(&ready_bar[stage], phase, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sb = smem_u32(smem + stage * STAGE_BYTES);
+                    const uint32_t sf_col = sf_base + stage * SF_COLS_STAGE;
+                    const int nks = min(4, k_atoms - kt * 4);
+                    for (int ks = 0; ks < nks; ++ks) {
+                        const uint32_t col = sf_col + ks * SF_COLS_STEP;
+                        tc_mma2_nvf4(tmem_base, sdesc_kmajor_sw128(sb + ks * 32),
+                                     sdesc_kmajor_sw128(sb + A_BYTES + ks * 32), idesc, col, col + 4,
+                                     (kt | ks) != 0 ? 1u : 0u);
+                    }
+                    tc_commit2_mc(&empty_bar[stage], 0x3);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit2_mc(&accf_bar, 0x3);
+                acc_phase ^= 1u;
+            }
+            tc_commit2_mc(&drain_bar, 0x1);
+            int no_abort = 0;
+            WaitCtx w2{&no_abort, p.dev_status};
+            mbar_wait(&drain_bar, 0, w2);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3;                       // TMEM lane quarter
+        const int h = (warp - 8) >> 2;                // column half: [0,128) or [128,256)
+        const int row_t = (int)rank * 128 + q * 32 + lane;    // row inside the pair tile
+        const float alpha = __fmul_rn(*p.a_scale, *p.b_scale);
+        float g_y = 0.0f, d_y = 0.0f;
+        if (OUT == OUT_NVFP4) {
+            g_y = *p.y_scale;
+            d_y = __fmul_rn(6.0f, g_y);
+        }
+        const uint32_t acce_addr = mapa_shared(smem_u32(&acce_bar), 0);
+        uint8_t* ebuf = smem + STAGES * STAGE_BYTES + (warp - 8) * 2 * C::EPI_BUF;
+        uint32_t acc_phase = 0;
+        int nstore = 0;
+        float amax_run = 0.0f;
+        for (int t = pair; t < p.num_tiles; t += npairs) {
+            int mb2, nb;
+            tile_coords(t, p.num_mb2, p.num_nb, mb2, nb);
+            if (!__all_sync(0xffffffffu, mbar_wait(&accf_bar, acc_phase, wc) ? 1 : 0)) break;
+            tc_fence_after();
+            uint32_t r[128];
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + h * 128;
+            tmem_ld_32x32b_x32(tbase, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+            tmem_ld_32x32b_x32(tbase + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+            tmem_ld_32x32b_x32(tbase + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
+            tmem_ld_32x32b_x32(tbase + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
+            tmem_ld_wait();
+            // the accumulator is in registers: hand TMEM back to the MMA issuer
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acce_addr);
+            acc_phase ^= 1u;
+
+            const int m0 = mb2 * 256 + (int)rank * 128 + q * 32;
+            const int n0 = nb * 256 + h * 128;
+            if (OUT == OUT_NVFP4) {
+                const int64_t grow = (int64_t)mb2 * 256 + row_t;
+                const int kb4 = p.N / 64;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int ncol = n0 + c * 64;
+                    if (ncol >= p.N) continue;
+                    uint32_t sfw = 0u, cw[8];
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        float v[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(alpha, __uint_as_float(r[c * 64 + b * 16 + j]));
+                        float ab = 0.0f;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) ab = fmaxf(ab, fabsf(v[j]));
+                        if (grow < p.M) amax_run = fmaxf(amax_run, ab);
+                        const uint32_t sfc = block_scale_code(ab, d_y);
+                        const float s = __fmul_rn(e4m3_to_f32(sfc), g_y);
+                        float lo[8], hi[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) { lo[j] = v[j]; hi[j] = v[8 + j]; }
+                        cw[2 * b] = quantize8(lo, s);
+                        cw[2 * b + 1] = quantize8(hi, s);
+                        sfw |= sfc << (8 * b);
+                    }
+                    if (grow < p.M) {
+                        uint4* dst = reinterpret_cast<uint4*>(p.y_codes + grow * (p.N / 2) + ncol / 2);
+                        dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+                        dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+                    }
+                    // rows past M inside the padded scale buffer get zero scales
+                    if (grow < (int64_t)((p.M + 127) / 128) * 128) {
+                        const int rb = (int)(grow >> 7), rr = (int)(grow & 127);
+                        const int64_t atom = (int64_t)rb * kb4 + ncol / 64;
+                        *reinterpret_cast<uint32_t*>(p.y_sf + atom * SF_ATOM + (rr & 31) * 16 + (rr >> 5) * 4) = sfw;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    if (n0 + c * 32 >= p.N) continue;
+                    uint8_t* buf = ebuf + (nstore & 1) * C::EPI_BUF;
+                    if (lane == 0) bulk_wait_group_read<1>();
+                    __syncwarp();
+                    store_chunk<OUT>(&r[c * 32], alpha, buf, lane, &tmap_y, n0 + c * 32, m0);
+                    ++nstore;
+                }
+            }
+        }
+        if (lane == 0) bulk_wait_group<0>();
+        if (OUT == OUT_NVFP4 && p.y_amax != nullptr) {
+            for (int o = 16; o > 0; o >>= 1) amax_run = fmaxf(amax_run, __shfl_xor_sync(0xffffffffu, amax_run, o));
+            if (lane == 0 && amax_run > 0.0f) atomicMax(reinterpret_cast<int*>(p.y_amax), __float_as_int(amax_run));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();                       // the leader's MMAs are done with both CTAs' memory
+    if (warp == 0) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc2(tmem_base, 512);
+    }
+}
+
+template <int OUT>
+cudaError_t launch_out(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) {
+    using C = Cfg<OUT>;
+    CUtensorMap ta, tb, tsa, tsb, ty;
+    const uint64_t kh = (uint64_t)(a.K / 2);
+    const uint64_t atoms_a = (uint64_t)((a.M + 127) / 128) * (uint64_t)(a.K / 64);
+    const uint64_t atoms_b = (uint64_t)((a.N + 127) / 128) * (uint64_t)(a.K / 64);
+    if (make_tmap_2d(&ta, a.a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kh, (uint64_t)a.M, kh, BK_BYTES, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
+        make_tmap_2d(&tb, a.b_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kh, (uint64_t)a.N, kh, BK_BYTES, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
+        make_tmap_2d(&tsa, a.a_sf, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, 128, atoms_a, SF_ATOM, 128, 4,
+                     CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
+        make_tmap_2d(&tsb, a.b_sf, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, 128, atoms_b, SF_ATOM, 128, 4,
+                     CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    CUresult r = CUDA_SUCCESS;
+    if (OUT == OUT_BF16)
+        r = make_tmap_2d(&ty, a.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.N, (uint64_t)a.M,
+                         (uint64_t)a.N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+    else if (OUT == OUT_F32)
+        r = make_tmap_2d(&ty, a.y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)a.N, (uint64_t)a.M,
+                         (uint64_t)a.N * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+    else
+        ty = ta;
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+
+    Params p;
+    p.a_scale = a.a_scale;
+    p.b_scale = a.b_scale;
+    p.M = (int)a.M;
+    p.N = (int)a.N;
+    p.K = (int)a.K;
+    p.num_mb2 = (int)((a.M + 255) / 256);
+    p.num_nb = (int)((a.N + 255) / 256);
+    p.num_tiles = p.num_mb2 * p.num_nb;
+    p.y_codes = a.y_codes;
+    p.y_sf = a.y_sf;
+    p.y_scale = a.y_scale;
+    p.y_amax = a.y_amax;
+    p.dev_status = a.dev_status;
+
+    auto kern = gemm2_kernel<OUT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // as many pairs as can be resident at once (persistent over tiles)
+    int max_clusters = 0;
+    cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
+    if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess || max_clusters < 1)
+        max_clusters = num_sms / 2;
+    int pairs = p.num_tiles < max_clusters ? p.num_tiles : max_clusters;
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, ty, p);
+    count_launch(1);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace w4a4_2sm
+
+cudaError_t launch_gemm_w4a4_2sm(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) {
+    using namespace w4a4_2sm;
+    if (a.y != nullptr) {
+        if (a.y_dtype == 1) return launch_out<OUT_F32>(a, num_sms, stream);
+        return launch_out<OUT_BF16>(a, num_sms, stream);
+    }
+    return launch_out<OUT_NVFP4>(a, num_sms, stream);
+}
+
+}  // namespace nvfp4

@@ -40,6 +40,7 @@ struct GemmW4A4Args {
 };
 
 cudaError_t launch_gemm_w4a4(const GemmW4A4Args& a, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemm_w4a4_2sm(const GemmW4A4Args& a, int num_sms, cudaStream_t stream);
 
 struct GemmW4A16Args {
     const uint16_t* x;
