@@ -105,6 +105,28 @@ nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t rows, int64_t k, int64_t
                             int *dev_status, nvfp4_stream_t stream);
 
 /*
+ * nvfp4_quantize_noalloc -- the source pages have no counterpart: this is a
+ * deployment variant of nvfp4_quantize.  Same arguments, same results, bit
+ * for bit, minus the workspace, for callers that cannot allocate device
+ * memory (a plugin whose host application owns all device memory, a server
+ * that allocates nothing after start-up, a caller without a CUDA allocator).
+ * The amax pass keeps its per-CTA partial maxima in a fixed device array of
+ * NVFP4_NOALLOC_SCRATCH_FLOATS floats (1 KB) that every GPU loading the
+ * library holds until the process exits.  That pass never needs more entries
+ * than that, whatever the tensor size; a problem that would is rejected with
+ * NVFP4_ERR_WORKSPACE.  Nothing in the array has to start at zero.  Every call
+ * shares the one array: calls that overlap on the GPU (for instance on two
+ * streams) race and may produce wrong scales -- serialize them.  The first call
+ * on each device looks up the array's device address (a runtime call, no
+ * allocation); make that first call before any stream capture.  The call
+ * itself allocates nothing.
+ */
+enum { NVFP4_NOALLOC_SCRATCH_FLOATS = 256 };
+nvfp4_status nvfp4_quantize_noalloc(const void *x_bf16, int64_t rows, int64_t k, int64_t ld_x,
+                                    uint8_t *codes, uint8_t *sf, float *tensor_scale,
+                                    unsigned flags, int *dev_status, nvfp4_stream_t stream);
+
+/*
  * nvfp4_dequantize -- v = (e2m1(code) * e4m3(sf)) * g, rounded once (RNE) to
  * out_dtype ([DiT] Definition III.1: the quantizer returns s * round(...)).
  * codes/sf/tensor_scale as produced by nvfp4_quantize for [rows, k];

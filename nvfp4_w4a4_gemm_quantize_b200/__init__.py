@@ -7,7 +7,7 @@ memory and streams.
 
 Low-level (same names and argument order as the C calls):
     nvfp4_sf_bytes, nvfp4_quantize_workspace_bytes, nvfp4_quantize,
-    nvfp4_dequantize, nvfp4_gemm_w4a4, nvfp4_gemm_w4a16, nvfp4_launch_count
+    nvfp4_quantize_noalloc, nvfp4_dequantize, nvfp4_gemm_w4a4, nvfp4_gemm_w4a16, nvfp4_launch_count
 Convenience (allocate outputs with torch, then call the above):
     NVFP4Tensor, quantize, dequantize, gemm_w4a4, gemm_w4a16
 """
@@ -62,6 +62,16 @@ def nvfp4_quantize(x, rows, k, ld_x, codes, sf, tensor_scale, flags=0, workspace
     st = lib().nvfp4_quantize(_ptr(x), rows, k, ld_x, _ptr(codes), _ptr(sf), _ptr(tensor_scale),
                               flags, _ptr(workspace), workspace_bytes, _ptr(dev_status), _stream(stream))
     check(st, "nvfp4_quantize")
+
+
+def nvfp4_quantize_noalloc(x, rows, k, ld_x, codes, sf, tensor_scale, flags=0, dev_status=None,
+                           stream=None) -> None:
+    """nvfp4_quantize without a workspace argument, for callers that cannot
+    allocate device memory (the amax scratch is a fixed device array inside the
+    library; overlapping calls race, see include/nvfp4.h)."""
+    st = lib().nvfp4_quantize_noalloc(_ptr(x), rows, k, ld_x, _ptr(codes), _ptr(sf), _ptr(tensor_scale), flags,
+                                      _ptr(dev_status), _stream(stream))
+    check(st, "nvfp4_quantize_noalloc")
 
 
 def nvfp4_dequantize(codes, sf, tensor_scale, rows, k, out, out_dtype, stream=None) -> None:

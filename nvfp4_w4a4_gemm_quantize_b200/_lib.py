@@ -31,6 +31,7 @@ SIGNATURES = {
     "nvfp4_sf_bytes": (ctypes.c_size_t, [_i64, _i64]),
     "nvfp4_quantize_workspace_bytes": (ctypes.c_size_t, [_i64, _i64]),
     "nvfp4_quantize": (_status, [_p, _i64, _i64, _i64, _p, _p, _p, ctypes.c_uint, _p, ctypes.c_size_t, _p, _p]),
+    "nvfp4_quantize_noalloc": (_status, [_p, _i64, _i64, _i64, _p, _p, _p, ctypes.c_uint, _p, _p]),
     "nvfp4_dequantize": (_status, [_p, _p, _p, _i64, _i64, _p, _int, _p]),
     "nvfp4_gemm_w4a4": (_status, [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _p, _int, _p, _p, _p, _p, _p, _p]),
     "nvfp4_gemm_w4a16": (_status, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _int, _p, _p]),
