@@ -313,11 +313,9 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
         const int h = (warp - 8) >> 2;                // column half: [0,128) or [128,256)
         const int row_t = (int)rank * 128 + q * 32 + lane;    // row inside the pair tile
         const float alpha = __fmul_rn(*p.a_scale, *p.b_scale);
-        float g_y = 0.0f, d_y = 0.0f;
-        if (OUT == OUT_NVFP4) {
-            g_y = *p.y_scale;
-            d_y = __fmul_rn(6.0f, g_y);
-        }
+        float g_y = 0.0f;
+        if (OUT == OUT_NVFP4) g_y = *p.y_scale;
+        const ScaleConsts sc_y = scale_consts(g_y);
         const uint32_t acce_addr = mapa_shared(smem_u32(&acce_bar), 0);
         uint8_t* ebuf = smem + STAGES * STAGE_BYTES + (warp - 8) * 2 * C::EPI_BUF;
         uint32_t acc_phase = 0;
@@ -360,7 +358,7 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
 #pragma unroll
                         for (int j = 0; j < 16; ++j) ab = fmaxf(ab, fabsf(v[j]));
                         if (grow < p.M) amax_run = fmaxf(amax_run, ab);
-                        const uint32_t sfc = block_scale_code(ab, d_y);
+                        const uint32_t sfc = block_scale_code(ab, sc_y);
                         const float s = __fmul_rn(e4m3_to_f32(sfc), g_y);
                         float lo[8], hi[8];
 #pragma unroll

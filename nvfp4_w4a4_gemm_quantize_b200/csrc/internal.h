@@ -8,7 +8,7 @@ namespace nvfp4 {
 
 constexpr int kAmaxThreads = 256;
 constexpr int kAmaxMaxCtas = 256;        // partial maxima, one float each
-constexpr int kQuantThreads = 256;
+constexpr int kQuantThreads = 512;
 constexpr size_t kQuantWorkspaceBytes = kAmaxMaxCtas * sizeof(float);
 
 void count_launch(int n);

@@ -79,8 +79,9 @@ amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
 
 // ------------------------------------------------------------------ quantize
 // One CTA quantizes a 128-row x 256-column tile (four 512-byte scale atoms).
-// Warp w owns rows 16w .. 16w+15; lane l owns columns 8l .. 8l+7 of a row, so
-// a 16-value block is a lane pair and a row is one coalesced 512-byte load.
+// Warp w owns rows 8w .. 8w+7; lane l owns columns 8l .. 8l+7 of a row, so a
+// 16-value block is a lane pair and a row is one coalesced 512-byte load.  All
+// eight loads of a warp are issued before any is used.
 template <bool kDynamic>
 __global__ void __launch_bounds__(kQuantThreads)
 quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
@@ -105,7 +106,7 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
     }
     __syncthreads();
     const float g = g_sh;
-    const float d = __fmul_rn(6.0f, g);
+    const ScaleConsts sc = scale_consts(g);
 
     const int64_t row0 = (int64_t)blockIdx.y * 128;
     const int64_t c0 = (int64_t)blockIdx.x * 256;
@@ -113,10 +114,11 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
     const bool col_ok = lane * 8 < ncols;
     const int64_t kh = k >> 1;
 
-    uint4 v[16];
+    constexpr int kRows = 128 / (kQuantThreads / 32);   // rows per warp
+    uint4 v[kRows];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int64_t r = row0 + warp * 16 + i;
+    for (int i = 0; i < kRows; ++i) {
+        const int64_t r = row0 + warp * kRows + i;
         if (r < rows && col_ok)
             v[i] = __ldcs(reinterpret_cast<const uint4*>(x + r * ld + c0) + lane);
         else
@@ -124,8 +126,8 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
     }
 
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int rt = warp * 16 + i;                // row inside the tile
+    for (int i = 0; i < kRows; ++i) {
+        const int rt = warp * kRows + i;             // row inside the tile
         const int64_t r = row0 + rt;
         const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
         // block amax over the lane pair (integer max of |bf16| patterns)
@@ -134,7 +136,7 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
         hb = max(hb, __shfl_xor_sync(0xffffffffu, hb, 1));
         const float ab = __uint_as_float(hb << 16);
 
-        const uint32_t sfc = block_scale_code(ab, d);
+        const uint32_t sfc = block_scale_code(ab, sc);
         const float s = __fmul_rn(e4m3_to_f32(sfc), g);
         float f[8];
 #pragma unroll
