@@ -61,12 +61,23 @@ __device__ __forceinline__ uint32_t block_scale_code(float ab, const ScaleConsts
     return cvt_e4m3(r);
 }
 
+// Pack four E2M1 pairs (each in the low byte of a word) into one word.
+__device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+    uint32_t lo, hi, r;
+    asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(lo) : "r"(b0), "r"(b1));
+    asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(hi) : "r"(b2), "r"(b3));
+    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+
 // Eight values with decoded block scale s -> four packed bytes (element 2j in
 // the low nibble of byte j).  The quotient is the IEEE single quotient: the
 // product with the approximate reciprocal lies within 3 ulps of it, and E2M1
-// rounding can only differ near a midpoint or grid point, where the exact
-// division is used (near_grid); blocks whose s is outside [2^-125, 2^125] use
-// the exact division throughout.
+// rounding can only differ near a midpoint or grid point (a value whose low 21
+// fraction bits are zero), where the exact division is used.  The test maps
+// (bits + 8) mod 2^21 to the top of a word with one multiply-add, so "within
+// 8 ulps" is one unsigned comparison of the minimum.  Blocks whose s is
+// outside [2^-125, 2^125] use the exact division throughout.
 __device__ __forceinline__ uint32_t quantize8(const float (&f)[8], float s) {
     if (s == 0.0f) return 0u;
     float q[8];
@@ -76,9 +87,9 @@ __device__ __forceinline__ uint32_t quantize8(const float (&f)[8], float s) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             q[j] = __fmul_rn(f[j], rcp);
-            mn = min(mn, (__float_as_uint(q[j]) + 8u) & 0x1FFFF0u);
+            mn = min(mn, __float_as_uint(q[j]) * 2048u + 16384u);
         }
-        if (mn == 0u) {
+        if (mn < 32768u) {
 #pragma unroll
             for (int j = 0; j < 8; ++j)
                 if (near_grid(q[j])) q[j] = __fdiv_rn(f[j], s);
@@ -87,10 +98,7 @@ __device__ __forceinline__ uint32_t quantize8(const float (&f)[8], float s) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) q[j] = __fdiv_rn(f[j], s);
     }
-    uint32_t packed = 0u;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) packed |= cvt_e2m1x2(q[2 * j], q[2 * j + 1]) << (8 * j);
-    return packed;
+    return pack4(cvt_e2m1x2(q[0], q[1]), cvt_e2m1x2(q[2], q[3]), cvt_e2m1x2(q[4], q[5]), cvt_e2m1x2(q[6], q[7]));
 }
 
 }  // namespace nvfp4

@@ -32,10 +32,18 @@
 namespace nvfp4 {
 
 // ------------------------------------------------------------------ amax
-// Per-half maxima of |x| over 8 bf16 values (sign bits cleared first).
+// Per-half maxima of |x| over 8 bf16 values: the sign bits are cleared and the
+// patterns compared as unsigned 16-bit integers (for non-negative IEEE values
+// the order of the patterns is the order of the values).
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t absmax_bf16x8(uint4 a) {
-    return __vmaxu2(__vmaxu2(a.x & 0x7FFF7FFFu, a.y & 0x7FFF7FFFu),
-                    __vmaxu2(a.z & 0x7FFF7FFFu, a.w & 0x7FFF7FFFu));
+    return max_u16x2(max_u16x2(a.x & 0x7FFF7FFFu, a.y & 0x7FFF7FFFu),
+                     max_u16x2(a.z & 0x7FFF7FFFu, a.w & 0x7FFF7FFFu));
 }
 
 // Partial max |x| per CTA over a [rows, k] bf16 tensor with row stride ld.
@@ -55,14 +63,14 @@ amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
         for (; v + 3 * stride < nvec; v += 4 * stride) {
             const uint4 a = __ldcs(p + v), b = __ldcs(p + v + stride);
             const uint4 c = __ldcs(p + v + 2 * stride), d = __ldcs(p + v + 3 * stride);
-            m = __vmaxu2(m, __vmaxu2(absmax_bf16x8(a), absmax_bf16x8(b)));
-            m = __vmaxu2(m, __vmaxu2(absmax_bf16x8(c), absmax_bf16x8(d)));
+            m = max_u16x2(m, max_u16x2(absmax_bf16x8(a), absmax_bf16x8(b)));
+            m = max_u16x2(m, max_u16x2(absmax_bf16x8(c), absmax_bf16x8(d)));
         }
-        for (; v < nvec; v += stride) m = __vmaxu2(m, absmax_bf16x8(__ldcs(p + v)));
+        for (; v < nvec; v += stride) m = max_u16x2(m, absmax_bf16x8(__ldcs(p + v)));
     } else {
         for (; v < nvec; v += stride) {
             const int64_t r = v / k8, c = v - r * k8;
-            m = __vmaxu2(m, absmax_bf16x8(__ldcs(reinterpret_cast<const uint4*>(x + r * ld) + c)));
+            m = max_u16x2(m, absmax_bf16x8(__ldcs(reinterpret_cast<const uint4*>(x + r * ld) + c)));
         }
     }
     uint32_t h = max(m & 0xFFFFu, m >> 16);
@@ -79,15 +87,21 @@ amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
 
 // ------------------------------------------------------------------ quantize
 // One CTA quantizes a 128-row x 256-column tile (four 512-byte scale atoms).
-// Warp w owns rows 8w .. 8w+7; lane l owns columns 8l .. 8l+7 of a row, so a
-// 16-value block is a lane pair and a row is one coalesced 512-byte load.  All
-// eight loads of a warp are issued before any is used.
+// Warp w owns rows 8w .. 8w+7, two rows per step: lanes 0-15 one row, lanes
+// 16-31 the next, lane l owning the 16-value block l % 16 of its row (two
+// 16-byte loads; a row is one coalesced 512-byte span).  A lane therefore
+// holds a whole block: its maximum, scale and reciprocal are computed once
+// per 16 values without any shuffle.  All loads of a warp are issued before
+// any is used.
 template <bool kDynamic>
 __global__ void __launch_bounds__(kQuantThreads)
 quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
                 uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
                 float* __restrict__ tensor_scale, const float* __restrict__ partials, int nparts) {
-    __shared__ uint32_t sf_stage[4 * 128];      // 4 atoms x 512 bytes
+    // four 512-byte atoms, each padded by 4 bytes so that the eight words two
+    // rows write (one per atom and row) fall in different banks
+    constexpr int kAtomPitch = 516;
+    __shared__ __align__(16) uint8_t sf_stage[4 * kAtomPitch];
     __shared__ float g_sh;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -111,58 +125,62 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
     const int64_t row0 = (int64_t)blockIdx.y * 128;
     const int64_t c0 = (int64_t)blockIdx.x * 256;
     const int ncols = (k - c0) < 256 ? (int)(k - c0) : 256;   // multiple of 64
-    const bool col_ok = lane * 8 < ncols;
+    const int half = lane >> 4;                   // which row of the pair
+    const int blk = lane & 15;                    // 16-value block inside the tile row
+    const bool col_ok = blk * 16 < ncols;
     const int64_t kh = k >> 1;
 
     constexpr int kRows = 128 / (kQuantThreads / 32);   // rows per warp
-    uint4 v[kRows];
+    constexpr int kSteps = kRows / 2;
+    uint4 v[2 * kSteps];
 #pragma unroll
-    for (int i = 0; i < kRows; ++i) {
-        const int64_t r = row0 + warp * kRows + i;
-        if (r < rows && col_ok)
-            v[i] = __ldcs(reinterpret_cast<const uint4*>(x + r * ld + c0) + lane);
-        else
-            v[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = 0; i < kSteps; ++i) {
+        const int64_t r = row0 + warp * kRows + 2 * i + half;
+        if (r < rows && col_ok) {
+            const uint4* src = reinterpret_cast<const uint4*>(x + r * ld + c0) + 2 * blk;
+            v[2 * i] = __ldcs(src);
+            v[2 * i + 1] = __ldcs(src + 1);
+        } else {
+            v[2 * i] = make_uint4(0u, 0u, 0u, 0u);
+            v[2 * i + 1] = make_uint4(0u, 0u, 0u, 0u);
+        }
     }
 
 #pragma unroll
-    for (int i = 0; i < kRows; ++i) {
-        const int rt = warp * kRows + i;             // row inside the tile
+    for (int i = 0; i < kSteps; ++i) {
+        const int rt = warp * kRows + 2 * i + half;   // row inside the tile
         const int64_t r = row0 + rt;
-        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-        // block amax over the lane pair (integer max of |bf16| patterns)
-        const uint32_t mm = absmax_bf16x8(v[i]);
-        uint32_t hb = max(mm & 0xFFFFu, mm >> 16);
-        hb = max(hb, __shfl_xor_sync(0xffffffffu, hb, 1));
+        const uint32_t w[8] = {v[2 * i].x, v[2 * i].y, v[2 * i].z, v[2 * i].w,
+                               v[2 * i + 1].x, v[2 * i + 1].y, v[2 * i + 1].z, v[2 * i + 1].w};
+        // block amax (integer max of |bf16| patterns)
+        const uint32_t mm = max_u16x2(absmax_bf16x8(v[2 * i]), absmax_bf16x8(v[2 * i + 1]));
+        const uint32_t hb = max(mm & 0xFFFFu, mm >> 16);
         const float ab = __uint_as_float(hb << 16);
 
         const uint32_t sfc = block_scale_code(ab, sc);
         const float s = __fmul_rn(e4m3_to_f32(sfc), g);
-        float f[8];
+        float f0[8], f1[8];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            f[2 * j] = __uint_as_float(w[j] << 16);
-            f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+            f0[2 * j] = __uint_as_float(w[j] << 16);
+            f0[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+            f1[2 * j] = __uint_as_float(w[4 + j] << 16);
+            f1[2 * j + 1] = __uint_as_float(w[4 + j] & 0xFFFF0000u);
         }
-        const uint32_t packed = quantize8(f, s);
+        const uint32_t lo = quantize8(f0, s);
+        const uint32_t hi = quantize8(f1, s);
         if (r < rows && col_ok)
-            *reinterpret_cast<uint32_t*>(codes + r * kh + (c0 >> 1) + lane * 4) = packed;
-
-        // scale bytes of blocks 4a..4a+3 live on lanes 8a, 8a+2, 8a+4, 8a+6
-        const uint32_t b1 = __shfl_down_sync(0xffffffffu, sfc, 2);
-        const uint32_t b2 = __shfl_down_sync(0xffffffffu, sfc, 4);
-        const uint32_t b3 = __shfl_down_sync(0xffffffffu, sfc, 6);
-        if ((lane & 7) == 0 && col_ok) {
-            const int a = lane >> 3;
-            sf_stage[a * 128 + (rt & 31) * 4 + (rt >> 5)] = sfc | (b1 << 8) | (b2 << 16) | (b3 << 24);
-        }
+            *reinterpret_cast<uint2*>(codes + r * kh + (c0 >> 1) + blk * 8) = make_uint2(lo, hi);
+        // block blk of this row: atom blk / 4, byte blk % 4 of the row's word
+        if (col_ok) sf_stage[(blk >> 2) * kAtomPitch + (rt & 31) * 16 + (rt >> 5) * 4 + (blk & 3)] = (uint8_t)sfc;
     }
     __syncthreads();
     // this tile's atoms are consecutive in the scale buffer
     const int natoms = ncols >> 6;
     const int64_t kb4 = k >> 6;                       // atoms per 128-row block
     uint32_t* dst = reinterpret_cast<uint32_t*>(sf + (((int64_t)blockIdx.y * kb4 + blockIdx.x * 4) << 9));
-    for (int i = threadIdx.x; i < natoms * 128; i += kQuantThreads) dst[i] = sf_stage[i];
+    for (int i = threadIdx.x; i < natoms * 128; i += kQuantThreads)
+        dst[i] = *reinterpret_cast<const uint32_t*>(sf_stage + (i >> 7) * kAtomPitch + (i & 127) * 4);
 }
 
 // ------------------------------------------------------------------ dequantize
