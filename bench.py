@@ -162,6 +162,46 @@ def run_reference(args):
     return 0
 
 
+# ----------------------------------------------------------------- extra measurements
+def time_device(fn, iters=10, warmup=3):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters
+
+
+def reference_points(dev, layers):
+    """cuBLAS bf16 on the same shapes (a reference point, never the product
+    path) and this library's W4A16 kernel on the weights-only workload."""
+    import torch
+    import nvfp4_w4a4_gemm_quantize_b200 as nv
+    from nvfp4_w4a4_gemm_quantize_b200 import synth
+    out = {"cublas_bf16_tflops": {}, "w4a16": {}}
+    for L in layers:
+        x, w = synth.layer_tensors(WORKLOAD, L.name, device=dev)
+        ms = time_device(lambda: torch.matmul(x, w.t()))
+        out["cublas_bf16_tflops"][L.name] = round(2 * L.M * L.N * L.K / (ms * 1e-3) / 1e12, 1)
+        del x, w
+    for L in synth.WORKLOADS["w4a16"].layers:
+        x, w = synth.layer_tensors("w4a16", L.name, device=dev)
+        W = nv.quantize(w)
+        del w
+        y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev)
+        ms = time_device(lambda: nv.gemm_w4a16(x, W, out=y))
+        out["w4a16"][L.name] = {"shape": f"{L.M}x{L.K}x{L.N}", "ms": round(ms, 4),
+                                "tflops": round(2 * L.M * L.N * L.K / (ms * 1e-3) / 1e12, 1)}
+        del x, W, y
+    torch.cuda.empty_cache()
+    return out
+
+
 # ----------------------------------------------------------------- our leg
 def run_ours(args):
     import torch
@@ -267,6 +307,11 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
 
+    extra = None
+    if rank == 0 and world == 1 and not args.no_reference_points:
+        del xh, yh
+        extra = reference_points(dev, wl.layers)
+
     # ---- cpu baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -311,6 +356,7 @@ def run_ours(args):
             "gpu_launches": int(launches),
             "clocks": clocks,
             "cpu_baseline": cpu,
+            "reference_points": extra,
         }
         print(json.dumps(line))
     if world > 1:
@@ -327,6 +373,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-rows", type=int, default=48)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-reference-points", action="store_true")
     ap.add_argument("--layers", default="", help="profiling: comma-separated subset of layers")
     ap.add_argument("--m", type=int, default=0, help="profiling: tokens (rows of X) per layer")
     args = ap.parse_args()
