@@ -177,7 +177,7 @@ def time_device(fn, iters=10, warmup=3):
     return e0.elapsed_time(e1) / iters
 
 
-def reference_points(dev, layers):
+def reference_points(dev, layers, w4a16_layers):
     """cuBLAS bf16 on the same shapes (a reference point, never the product
     path) and this library's W4A16 kernel on the weights-only workload."""
     import torch
@@ -186,11 +186,13 @@ def reference_points(dev, layers):
     out = {"cublas_bf16_tflops": {}, "w4a16": {}}
     for L in layers:
         x, w = synth.layer_tensors(WORKLOAD, L.name, device=dev)
+        x = x[: L.M]
         ms = time_device(lambda: torch.matmul(x, w.t()))
         out["cublas_bf16_tflops"][L.name] = round(2 * L.M * L.N * L.K / (ms * 1e-3) / 1e12, 1)
         del x, w
-    for L in synth.WORKLOADS["w4a16"].layers:
+    for L in w4a16_layers:
         x, w = synth.layer_tensors("w4a16", L.name, device=dev)
+        x = x[: L.M].contiguous()
         W = nv.quantize(w)
         del w
         y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev)
@@ -200,6 +202,50 @@ def reference_points(dev, layers):
         del x, W, y
     torch.cuda.empty_cache()
     return out
+
+
+def reduced(wl, args):
+    """A reduced case for profiling captures: selected layers and/or fewer
+    tokens (rows of X) per layer."""
+    if not (args.layers or args.m):
+        return wl
+    import dataclasses
+    keep = [L for L in wl.layers if not args.layers or L.name in args.layers.split(",")]
+    keep = [dataclasses.replace(L, M=min(args.m, L.M) if args.m else L.M) for L in keep]
+    return dataclasses.replace(wl, layers=tuple(keep))
+
+
+def kernel_source_hash() -> str:
+    """SHA-256 over the library's CUDA sources (names and contents).  A DRAM
+    traffic figure recorded under profiles/ is reported only while this
+    matches the hash recorded beside it: any source change voids it."""
+    import hashlib
+    d = os.path.join(ROOT, "nvfp4_w4a4_gemm_quantize_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            h.update(open(os.path.join(d, name), "rb").read())
+    return h.hexdigest()
+
+
+def profiled_traffic(summary: str):
+    """DRAM bytes per launch (read + write) from an ncu summary under
+    profiles/, or None when it is absent or was taken on other sources."""
+    p = os.path.join(ROOT, "profiles", summary)
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    for line in open(p):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    if kv.get("source_sha256") != kernel_source_hash():
+        return None
+    try:
+        return int(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 # ----------------------------------------------------------------- our leg
@@ -214,13 +260,8 @@ def run_ours(args):
     if rank == 0:
         build.build()
     barrier(world)
-    wl = synth.WORKLOADS[WORKLOAD]
-    if args.layers or args.m:
-        # a reduced case for profiling captures: selected layers and/or fewer tokens
-        import dataclasses
-        keep = [L for L in wl.layers if not args.layers or L.name in args.layers.split(",")]
-        keep = [dataclasses.replace(L, M=args.m or L.M) for L in keep]
-        wl = dataclasses.replace(wl, layers=tuple(keep))
+    wl = reduced(synth.WORKLOADS[WORKLOAD], args)
+    wl16 = reduced(synth.WORKLOADS["w4a16"], args)
     peaks, peak_src = load_peaks()
 
     # ---- data (resident in HBM before timing); each rank its own batch
@@ -310,7 +351,7 @@ def run_ours(args):
     extra = None
     if rank == 0 and world == 1 and not args.no_reference_points:
         del xh, yh
-        extra = reference_points(dev, wl.layers)
+        extra = reference_points(dev, wl.layers, wl16.layers)
 
     # ---- cpu baseline (rank 0, N = 1 only)
     cpu = None
@@ -328,6 +369,11 @@ def run_ours(args):
         g_flops = 2 * L.M * L.N * L.K
         g_tflops = g_flops / (gemm_ms[li] * 1e-3) / 1e12
         q_gbs = [QUANT_BYTES_PER_ELEM * l.M * l.K / (quant_ms[j] * 1e-3) / 1e9 for j, l in enumerate(wl.layers)]
+        # quantize: the largest activation (fc2's input, 32768 x 12288)
+        qi = names.index("fc2") if "fc2" in names else 0
+        full = not (args.layers or args.m)
+        g_traffic = profiled_traffic("gemm_w4a4_fc1_32768x3072x12288.txt") if full else None
+        q_traffic = profiled_traffic("quantize_fc2_32768x12288.txt") if full else None
         per_layer = {l.name: {"gemm_ms": round(gemm_ms[j], 4),
                               "gemm_tflops": round(2 * l.M * l.N * l.K / (gemm_ms[j] * 1e-3) / 1e12, 1),
                               "quant_ms": round(quant_ms[j], 4), "quant_gbs": round(q_gbs[j], 1)}
@@ -346,10 +392,12 @@ def run_ours(args):
                          "achieved": round(g_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                          "frac": round(g_tflops / fp4_peak, 4),
                          "peak_source": f"{peak_src} bf16 x {FP4_OVER_BF16:g} (nominal FP4/bf16 ratio)",
-                         "traffic": None},
-            "quantize": {"bound": "hbm", "achieved": round(max(q_gbs), 1), "peak": hbm_peak, "unit": "GB/s",
-                         "frac": round(max(q_gbs) / hbm_peak, 4), "bytes_per_elem": QUANT_BYTES_PER_ELEM,
-                         "peak_source": peak_src},
+                         "traffic": g_traffic},
+            "quantize": {"bound": "hbm", "kernel": f"amax + quantize {wl.layers[qi].name} input "
+                                                   f"{wl.layers[qi].M}x{wl.layers[qi].K}",
+                         "achieved": round(q_gbs[qi], 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(q_gbs[qi] / hbm_peak, 4), "bytes_per_elem": QUANT_BYTES_PER_ELEM,
+                         "peak_source": peak_src, "traffic": q_traffic},
             "layers": per_layer,
             "e2e": {"value": round(world * gemm_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
