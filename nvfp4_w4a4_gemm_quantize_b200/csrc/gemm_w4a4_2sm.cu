@@ -16,20 +16,28 @@
 //   warps 0-3  scale writers, both CTAs: per stage, every lane loads one
 //              16-byte row of each 512-byte scale atom from shared memory and
 //              tcgen05.st's it into its own TMEM lane quarter (the layout the
-//              block-scaled MMA reads: four replicated quarters).  Then the
-//              warp arrives on the leader's per-stage "ready" barrier, which
-//              therefore also says "this CTA's operands have landed".
+//              block-scaled MMA reads: four replicated quarters), then arrives
+//              on the leader's per-stage "ready" barrier.
 //              (tcgen05.cp of the 12 atoms per stage costs ~12 x 100 cycles
 //              of tensor-pipe time per pair, more than the 4 MMAs it feeds;
 //              the register path costs ~70 cycles per stage off that pipe.)
-//   warp 4     producer, both CTAs: TMA loads of this CTA's A rows, B half,
-//              A scales and all B scales into a STAGES-deep ring.
+//   warp 4     producer, both CTAs: TMA loads of this CTA's A scales and all
+//              B scales (completing on its own barrier), then of its A rows
+//              and B half, which complete on the LEADER's barrier
+//              (cta_group::2), so one wait tells the MMA issuer that both
+//              CTAs' operand tiles have landed.
 //   warp 5     leader CTA: MMA issuer (tcgen05.mma cta_group::2, commits
-//              multicast to both CTAs' barriers).
+//              multicast to both CTAs' barriers).  The whole warp runs the
+//              loop and one elected lane issues: with the loop in a single
+//              lane the descriptors are not warp-uniform and the issue of
+//              four MMAs took as long as their execution.
 //   warps 8-15 epilogue, both CTAs: the 128 x 256 FP32 accumulator slice is
 //              read into registers (two warps per TMEM lane quarter, 128
 //              columns each) and released to the MMA issuer at once, then
 //              converted and stored while the next tile's mainloop runs.
+// Every cross-CTA arrive is relaxed: what the waiter needs is ordered before
+// it by tcgen05.wait::{st,ld} and tcgen05.fence::before_thread_sync (a
+// cluster-scope release costs about a microsecond per arrive).
 // Registers: launched at 128 per thread; warpgroups 0-1 drop to 56 and the
 // epilogue warpgroups rise to 200 (256 x 56 + 256 x 200 = 512 x 128).
 // No load uses cluster multicast: every CTA fetches its own tiles.
@@ -144,7 +152,12 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     using C = Cfg<OUT>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full_bar[STAGES], ready_bar[STAGES], empty_bar[STAGES];
+    // fullab: the leader's, both CTAs' A/B tiles of a stage have landed (the
+    //         peer's loads signal it through cta_group::2);
+    // sff:    this CTA's scale atoms of a stage have landed;
+    // ready:  the leader's, both CTAs' scale columns are in TMEM;
+    // empty:  both CTAs', the MMAs of a stage have completed.
+    __shared__ __align__(8) uint64_t fullab_bar[STAGES], sff_bar[STAGES], ready_bar[STAGES], empty_bar[STAGES];
     __shared__ __align__(8) uint64_t accf_bar, acce_bar, drain_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
@@ -159,7 +172,8 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     if (threadIdx.x == 0) {
         abort_sh = 0;
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full_bar[s], 1);
+            mbar_init(&fullab_bar[s], 1);
+            mbar_init(&sff_bar[s], 1);
             mbar_init(&ready_bar[s], 2 * kSfWarps);
             mbar_init(&empty_bar[s], 1);
         }
@@ -208,7 +222,7 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
         for (int t = pair; t < p.num_tiles; t += npairs) {
             bool ok = true;
             for (int kt = 0; kt < num_kt; ++kt) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[stage], phase, wc) ? 1 : 0)) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, mbar_wait(&sff_bar[stage], phase, wc) ? 1 : 0)) { ok = false; break; }
                 const uint8_t* sfa_s = smem + stage * STAGE_BYTES + A_BYTES + B_BYTES;
                 const uint8_t* sfb_s = sfa_s + SFA_BYTES;
                 const uint32_t col0 = sf_base + lane_off + stage * SF_COLS_STAGE;
@@ -253,56 +267,90 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                 for (int kt = 0; kt < num_kt; ++kt) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1u, wc)) { ok = false; break; }
                     uint8_t* sb = smem + stage * STAGE_BYTES;
-                    mbar_arrive_expect_tx(&full_bar[stage], STAGE_BYTES);
-                    tma_load_2d(sb, &tmap_a, &full_bar[stage], kt * BK_BYTES, arow, pol_a);
-                    tma_load_2d(sb + A_BYTES, &tmap_b, &full_bar[stage], kt * BK_BYTES, brow, pol_b);
-                    tma_load_2d(sb + A_BYTES + B_BYTES, &tmap_sfa, &full_bar[stage], 0, sfa_row + kt * 4, pol_a);
-                    tma_load_2d(sb + A_BYTES + B_BYTES + SFA_BYTES, &tmap_sfb, &full_bar[stage], 0,
+                    // scale atoms first (the scale writers turn them into TMEM columns
+                    // while the operand tiles are still in flight)
+                    mbar_arrive_expect_tx(&sff_bar[stage], SFA_BYTES + SFB_BYTES);
+                    tma_load_2d(sb + A_BYTES + B_BYTES, &tmap_sfa, &sff_bar[stage], 0, sfa_row + kt * 4, pol_a);
+                    tma_load_2d(sb + A_BYTES + B_BYTES + SFA_BYTES, &tmap_sfb, &sff_bar[stage], 0,
                                 sfb_row0 + kt * 4, pol_b);
-                    tma_load_2d(sb + A_BYTES + B_BYTES + SFA_BYTES + 4 * SF_ATOM, &tmap_sfb, &full_bar[stage], 0,
+                    tma_load_2d(sb + A_BYTES + B_BYTES + SFA_BYTES + 4 * SF_ATOM, &tmap_sfb, &sff_bar[stage], 0,
                                 sfb_row1 + kt * 4, pol_b);
+                    // operand tiles of both CTAs complete on the leader's barrier,
+                    // which the leader arms with the bytes of the pair
+                    if (rank == 0) mbar_arrive_expect_tx(&fullab_bar[stage], 2 * (A_BYTES + B_BYTES));
+                    const uint32_t fab = mapa_shared(smem_u32(&fullab_bar[stage]), 0);
+                    tma_load_2d_pair(sb, &tmap_a, fab, kt * BK_BYTES, arow, pol_a);
+                    tma_load_2d_pair(sb + A_BYTES, &tmap_b, fab, kt * BK_BYTES, brow, pol_b);
                     issued = (issued & ~(1u << stage)) | (phase << stage);
                     issued_any |= 1u << stage;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
-            // this CTA's own loads have all landed before it may exit
+            // loads in flight land before the CTAs may exit: this CTA's scale
+            // atoms, and (seen by the leader) both CTAs' operand tiles; the peer
+            // is held at the final cluster barrier until the leader has seen them
             int no_abort = 0;
             WaitCtx w2{&no_abort, p.dev_status};
             for (int s = 0; s < STAGES; ++s)
-                if (issued_any & (1u << s)) mbar_wait(&full_bar[s], (issued >> s) & 1u, w2);
+                if (issued_any & (1u << s)) {
+                    mbar_wait(&sff_bar[s], (issued >> s) & 1u, w2);
+                    if (rank == 0) mbar_wait(&fullab_bar[s], (issued >> s) & 1u, w2);
+                }
         }
     } else if (warp < 8) {
-        if (warp == 5 && lane == 0 && rank == 0) {
+        if (warp == 5 && rank == 0) {
             // -------------------------------------------------------- MMA issuer (leader)
+            // The whole warp runs the loop so that the descriptors stay
+            // warp-uniform; one elected lane issues.
             constexpr uint32_t idesc = idesc_nvf4(256, 256);
+            const uint32_t smem0 = smem_u32(smem);
             int stage = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             for (int t = pair; t < p.num_tiles && ok; t += npairs) {
-                if (!mbar_wait_cluster(&acce_bar, acc_phase ^ 1u, wc)) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, mbar_wait_cluster(&acce_bar, acc_phase ^ 1u, wc) ? 1 : 0)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 for (int kt = 0; kt < num_kt; ++kt) {
-                    // both CTAs' operands have landed and their scales sit in TMEM
-                    if (!mbar_wait_cluster(&ready_bar[stage], phase, wc)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t sb = smem_u32(smem + stage * STAGE_BYTES);
-                    const uint32_t sf_col = sf_base + stage * SF_COLS_STAGE;
-                    const int nks = min(4, k_atoms - kt * 4);
-                    for (int ks = 0; ks < nks; ++ks) {
-                        const uint32_t col = sf_col + ks * SF_COLS_STEP;
-                        tc_mma2_nvf4(tmem_base, sdesc_kmajor_sw128(sb + ks * 32),
-                                     sdesc_kmajor_sw128(sb + A_BYTES + ks * 32), idesc, col, col + 4,
-                                     (kt | ks) != 0 ? 1u : 0u);
+                    // both CTAs' operand tiles have landed and their scales sit in TMEM
+                    if (!__all_sync(0xffffffffu, (mbar_wait(&fullab_bar[stage], phase, wc) &&
+                                                  mbar_wait_cluster(&ready_bar[stage], phase, wc)) ? 1 : 0)) {
+                        ok = false;
+                        break;
                     }
-                    tc_commit2_mc(&empty_bar[stage], 0x3);
+                    tc_fence_after();
+                    const uint32_t sb = smem0 + stage * STAGE_BYTES;
+                    const uint32_t sf_col = sf_base + stage * SF_COLS_STAGE;
+                    const int nks = k_atoms - kt * 4;
+                    if (elect_one()) {
+                        if (nks >= 4) {
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks)
+                                tc_mma2_nvf4(tmem_base, sdesc_kmajor_sw128(sb + ks * 32),
+                                             sdesc_kmajor_sw128(sb + A_BYTES + ks * 32), idesc,
+                                             sf_col + ks * SF_COLS_STEP, sf_col + ks * SF_COLS_STEP + 4,
+                                             (kt | ks) != 0 ? 1u : 0u);
+                        } else {
+                            for (int ks = 0; ks < nks; ++ks)
+                                tc_mma2_nvf4(tmem_base, sdesc_kmajor_sw128(sb + ks * 32),
+                                             sdesc_kmajor_sw128(sb + A_BYTES + ks * 32), idesc,
+                                             sf_col + ks * SF_COLS_STEP, sf_col + ks * SF_COLS_STEP + 4,
+                                             (kt | ks) != 0 ? 1u : 0u);
+                        }
+                        tc_commit2_mc(&empty_bar[stage], 0x3);
+                    }
+                    __syncwarp();
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
-                tc_commit2_mc(&accf_bar, 0x3);
+                if (elect_one()) tc_commit2_mc(&accf_bar, 0x3);
+                __syncwarp();
                 acc_phase ^= 1u;
             }
-            tc_commit2_mc(&drain_bar, 0x1);
+            if (elect_one()) tc_commit2_mc(&drain_bar, 0x1);
+            __syncwarp();
             int no_abort = 0;
             WaitCtx w2{&no_abort, p.dev_status};
             mbar_wait(&drain_bar, 0, w2);
@@ -336,7 +384,12 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
             // the accumulator is in registers: hand TMEM back to the MMA issuer
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acce_addr);
+            if (lane == 0) {
+                if (rank == 0)
+                    mbar_arrive(&acce_bar);
+                else
+                    mbar_arrive_cluster_relaxed(acce_addr);
+            }
             acc_phase ^= 1u;
 
             const int m0 = mb2 * 256 + (int)rank * 128 + q * 32;

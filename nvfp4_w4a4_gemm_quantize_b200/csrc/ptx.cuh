@@ -360,6 +360,20 @@ __device__ __forceinline__ void tc_cp2_32x128b_warpx4(uint32_t taddr, uint64_t s
     asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
+// TMA tile load into this CTA's shared memory whose completion is signalled
+// on an mbarrier of either CTA of the pair (`bar_cluster` is a shared::cluster
+// address, e.g. from mapa_shared).  No multicast: only this CTA's memory is
+// written.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int32_t x, int32_t y, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster),
+          "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+
 // Pair MMA: M = 256 (128 rows of A in each CTA), N split in halves across the
 // two CTAs' shared memory; each CTA's TMEM receives its 128 rows of D.
 __device__ __forceinline__ void tc_mma2_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
