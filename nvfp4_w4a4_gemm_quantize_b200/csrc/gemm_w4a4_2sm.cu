@@ -12,32 +12,29 @@
 // instead of 54 KB for a single-CTA 128 x 256 tile, so five stages fit in
 // shared memory, and L2 -> SM operand traffic per output drops by a third.
 //
-// Roles (512 threads per CTA, four warpgroups):
-//   warps 0-3  scale writers, both CTAs: per stage, every lane loads one
-//              16-byte row of each 512-byte scale atom from shared memory and
-//              tcgen05.st's it into its own TMEM lane quarter (the layout the
-//              block-scaled MMA reads: four replicated quarters), then arrives
-//              on the leader's per-stage "ready" barrier.
-//              (tcgen05.cp of the 12 atoms per stage costs ~12 x 100 cycles
-//              of tensor-pipe time per pair, more than the 4 MMAs it feeds;
-//              the register path costs ~70 cycles per stage off that pipe.)
-//   warp 4     producer, both CTAs: TMA loads of this CTA's A scales and all
-//              B scales (completing on its own barrier), then of its A rows
-//              and B half, which complete on the LEADER's barrier
-//              (cta_group::2), so one wait tells the MMA issuer that both
-//              CTAs' operand tiles have landed.
-//   warp 5     leader CTA: MMA issuer (tcgen05.mma cta_group::2, commits
-//              multicast to both CTAs' barriers).  The whole warp runs the
-//              loop and one elected lane issues: with the loop in a single
-//              lane the descriptors are not warp-uniform and the issue of
-//              four MMAs took as long as their execution.
+// Roles (512 threads per CTA):
+//   warp 0     producer, both CTAs: TMA loads of this CTA's scale atoms (its
+//              128 A rows, all 256 B rows), A rows and B half into a
+//              STAGES-deep ring.  Every load of the pair completes on the
+//              LEADER's full barrier (cta_group::2), which the leader arms
+//              with the bytes of both CTAs: one wait per stage tells the MMA
+//              issuer that both CTAs' operands have landed.
+//   warp 1     leader CTA: MMA issuer.  Per K=64 step three tcgen05.cp of
+//              the scale atoms into the stage's TMEM columns, then one
+//              tcgen05.mma cta_group::2; one commit per stage, multicast to
+//              both CTAs' "empty" barriers.
 //   warps 8-15 epilogue, both CTAs: the 128 x 256 FP32 accumulator slice is
 //              read into registers (two warps per TMEM lane quarter, 128
 //              columns each) and released to the MMA issuer at once, then
 //              converted and stored while the next tile's mainloop runs.
-// Every cross-CTA arrive is relaxed: what the waiter needs is ordered before
-// it by tcgen05.wait::{st,ld} and tcgen05.fence::before_thread_sync (a
-// cluster-scope release costs about a microsecond per arrive).
+// Producer and MMA issuer run on whole warps with one elected lane issuing:
+// the descriptors, coordinates and addresses then stay warp-uniform.  Issued
+// from a single lane, the same copies and MMAs took longer to issue than to
+// execute (the copies looked expensive; in a warp-uniform loop twelve copies
+// and four MMAs per stage issue in the MMAs' own 515 cycles).
+// The cross-CTA release of the accumulator is a relaxed arrive ordered by
+// tcgen05.wait::ld and tcgen05.fence::before_thread_sync (a cluster-scope
+// release costs about a microsecond per arrive).
 // Registers: launched at 128 per thread; warpgroups 0-1 drop to 56 and the
 // epilogue warpgroups rise to 200 (256 x 56 + 256 x 200 = 512 x 128).
 // No load uses cluster multicast: every CTA fetches its own tiles.
@@ -62,7 +59,6 @@ constexpr int SFB_BYTES = 2 * 4 * SF_ATOM;       // 256 rows x 4 K=64 steps
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // 38912
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 512;
-constexpr int kSfWarps = 4;
 constexpr int kRegsLow = 56;                     // warpgroups 0-1
 constexpr int kRegsHigh = 200;                   // epilogue warpgroups 2-3
 static_assert(256 * kRegsLow + 256 * kRegsHigh <= kThreads * 128, "register split exceeds the launch budget");
@@ -144,6 +140,18 @@ __device__ __forceinline__ void store_chunk(const uint32_t* r, float alpha, uint
     }
 }
 
+// One K=64 step of the pair: copy the step's scale atoms (A: 128 rows of this
+// CTA, B: all 256 rows, in both CTAs) into TMEM, then the block-scaled MMA.
+__device__ __forceinline__ void k_step(uint32_t tmem_acc, uint32_t sb, uint32_t sfs, uint32_t sf_col, int ks,
+                                       uint32_t idesc, bool accumulate) {
+    const uint32_t col = sf_col + ks * SF_COLS_STEP;
+    tc_cp2_32x128b_warpx4(col, sdesc_sf(sfs + ks * SF_ATOM));
+    tc_cp2_32x128b_warpx4(col + 4, sdesc_sf(sfs + SFA_BYTES + ks * SF_ATOM));
+    tc_cp2_32x128b_warpx4(col + 8, sdesc_sf(sfs + SFA_BYTES + 4 * SF_ATOM + ks * SF_ATOM));
+    tc_mma2_nvf4(tmem_acc, sdesc_kmajor_sw128(sb + ks * 32), sdesc_kmajor_sw128(sb + A_BYTES + ks * 32), idesc, col,
+                 col + 4, accumulate ? 1u : 0u);
+}
+
 template <int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
@@ -152,12 +160,10 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     using C = Cfg<OUT>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
-    // fullab: the leader's, both CTAs' A/B tiles of a stage have landed (the
-    //         peer's loads signal it through cta_group::2);
-    // sff:    this CTA's scale atoms of a stage have landed;
-    // ready:  the leader's, both CTAs' scale columns are in TMEM;
-    // empty:  both CTAs', the MMAs of a stage have completed.
-    __shared__ __align__(8) uint64_t fullab_bar[STAGES], sff_bar[STAGES], ready_bar[STAGES], empty_bar[STAGES];
+    // full:  the leader's; both CTAs' operand tiles and scale atoms of a stage
+    //        have landed (the peer's loads signal it through cta_group::2);
+    // empty: both CTAs'; the MMAs of a stage have completed.
+    __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES];
     __shared__ __align__(8) uint64_t accf_bar, acce_bar, drain_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
@@ -172,9 +178,7 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     if (threadIdx.x == 0) {
         abort_sh = 0;
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&fullab_bar[s], 1);
-            mbar_init(&sff_bar[s], 1);
-            mbar_init(&ready_bar[s], 2 * kSfWarps);
+            mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
         }
         mbar_init(&accf_bar, 1);
@@ -208,50 +212,12 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     const int k_atoms = p.K / 64;
     const uint32_t sf_base = tmem_base + 256;
     // one register-budget change per warpgroup, before the roles diverge
-    if (warp < 8)
+    // (the epilogue code sits under the same branch as its increase, so that
+    // ptxas allocates it against the raised budget)
+    if (warp < 8) {
         regs_dec<kRegsLow>();
-    else
-        regs_inc<kRegsHigh>();
-
-    if (warp < 4) {
-        // ------------------------------------------------------------ scale writers (both CTAs)
-        const uint32_t q = (uint32_t)warp;            // TMEM lane quarter of this warp
-        const uint32_t lane_off = (q * 32u) << 16;
-        int stage = 0;
-        uint32_t phase = 0;
-        for (int t = pair; t < p.num_tiles; t += npairs) {
-            bool ok = true;
-            for (int kt = 0; kt < num_kt; ++kt) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&sff_bar[stage], phase, wc) ? 1 : 0)) { ok = false; break; }
-                const uint8_t* sfa_s = smem + stage * STAGE_BYTES + A_BYTES + B_BYTES;
-                const uint8_t* sfb_s = sfa_s + SFA_BYTES;
-                const uint32_t col0 = sf_base + lane_off + stage * SF_COLS_STAGE;
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint4 va = *reinterpret_cast<const uint4*>(sfa_s + ks * SF_ATOM + lane * 16);
-                    const uint4 vb0 = *reinterpret_cast<const uint4*>(sfb_s + ks * SF_ATOM + lane * 16);
-                    const uint4 vb1 = *reinterpret_cast<const uint4*>(sfb_s + 4 * SF_ATOM + ks * SF_ATOM + lane * 16);
-                    const uint32_t col = col0 + ks * SF_COLS_STEP;
-                    tmem_st_32x32b_x4(col, va.x, va.y, va.z, va.w);
-                    tmem_st_32x32b_x4(col + 4, vb0.x, vb0.y, vb0.z, vb0.w);
-                    tmem_st_32x32b_x4(col + 8, vb1.x, vb1.y, vb1.z, vb1.w);
-                }
-                tmem_st_wait();                       // the scale columns are in TMEM
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    if (rank == 0)
-                        mbar_arrive(&ready_bar[stage]);
-                    else
-                        mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&ready_bar[stage]), 0));
-                }
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-            }
-            if (!ok) break;
-        }
-    } else if (warp == 4) {
-        // ------------------------------------------------------------ producer (both CTAs)
-        if (lane == 0) {
+        if (warp == 0) {
+            // ------------------------------------------------------------ producer (both CTAs)
             const uint64_t pol_a = policy_evict_normal();
             const uint64_t pol_b = policy_evict_last();
             int stage = 0;
@@ -265,97 +231,95 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                 const int sfa_row = (mb2 * 2 + (int)rank) * k_atoms;
                 const int sfb_row0 = (nb * 2) * k_atoms, sfb_row1 = (nb * 2 + 1) * k_atoms;
                 for (int kt = 0; kt < num_kt; ++kt) {
-                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, wc)) { ok = false; break; }
+                    if (!__all_sync(0xffffffffu, mbar_wait(&empty_bar[stage], phase ^ 1u, wc) ? 1 : 0)) {
+                        ok = false;
+                        break;
+                    }
                     uint8_t* sb = smem + stage * STAGE_BYTES;
-                    // scale atoms first (the scale writers turn them into TMEM columns
-                    // while the operand tiles are still in flight)
-                    mbar_arrive_expect_tx(&sff_bar[stage], SFA_BYTES + SFB_BYTES);
-                    tma_load_2d(sb + A_BYTES + B_BYTES, &tmap_sfa, &sff_bar[stage], 0, sfa_row + kt * 4, pol_a);
-                    tma_load_2d(sb + A_BYTES + B_BYTES + SFA_BYTES, &tmap_sfb, &sff_bar[stage], 0,
-                                sfb_row0 + kt * 4, pol_b);
-                    tma_load_2d(sb + A_BYTES + B_BYTES + SFA_BYTES + 4 * SF_ATOM, &tmap_sfb, &sff_bar[stage], 0,
-                                sfb_row1 + kt * 4, pol_b);
-                    // operand tiles of both CTAs complete on the leader's barrier,
-                    // which the leader arms with the bytes of the pair
-                    if (rank == 0) mbar_arrive_expect_tx(&fullab_bar[stage], 2 * (A_BYTES + B_BYTES));
-                    const uint32_t fab = mapa_shared(smem_u32(&fullab_bar[stage]), 0);
-                    tma_load_2d_pair(sb, &tmap_a, fab, kt * BK_BYTES, arow, pol_a);
-                    tma_load_2d_pair(sb + A_BYTES, &tmap_b, fab, kt * BK_BYTES, brow, pol_b);
+                    if (elect_one()) {
+                        // every load of the pair completes on the leader's barrier,
+                        // which the leader arms with the bytes of both CTAs
+                        if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * STAGE_BYTES);
+                        const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
+                        uint8_t* sfs = sb + A_BYTES + B_BYTES;
+                        tma_load_2d_pair(sfs, &tmap_sfa, fb, 0, sfa_row + kt * 4, pol_a);
+                        tma_load_2d_pair(sfs + SFA_BYTES, &tmap_sfb, fb, 0, sfb_row0 + kt * 4, pol_b);
+                        tma_load_2d_pair(sfs + SFA_BYTES + 4 * SF_ATOM, &tmap_sfb, fb, 0, sfb_row1 + kt * 4, pol_b);
+                        tma_load_2d_pair(sb, &tmap_a, fb, kt * BK_BYTES, arow, pol_a);
+                        tma_load_2d_pair(sb + A_BYTES, &tmap_b, fb, kt * BK_BYTES, brow, pol_b);
+                    }
+                    __syncwarp();
                     issued = (issued & ~(1u << stage)) | (phase << stage);
                     issued_any |= 1u << stage;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
-            // loads in flight land before the CTAs may exit: this CTA's scale
-            // atoms, and (seen by the leader) both CTAs' operand tiles; the peer
-            // is held at the final cluster barrier until the leader has seen them
-            int no_abort = 0;
-            WaitCtx w2{&no_abort, p.dev_status};
-            for (int s = 0; s < STAGES; ++s)
-                if (issued_any & (1u << s)) {
-                    mbar_wait(&sff_bar[s], (issued >> s) & 1u, w2);
-                    if (rank == 0) mbar_wait(&fullab_bar[s], (issued >> s) & 1u, w2);
-                }
-        }
-    } else if (warp < 8) {
-        if (warp == 5 && rank == 0) {
-            // -------------------------------------------------------- MMA issuer (leader)
-            // The whole warp runs the loop so that the descriptors stay
-            // warp-uniform; one elected lane issues.
-            constexpr uint32_t idesc = idesc_nvf4(256, 256);
-            const uint32_t smem0 = smem_u32(smem);
-            int stage = 0;
-            uint32_t phase = 0, acc_phase = 0;
-            bool ok = true;
-            for (int t = pair; t < p.num_tiles && ok; t += npairs) {
-                if (!__all_sync(0xffffffffu, mbar_wait_cluster(&acce_bar, acc_phase ^ 1u, wc) ? 1 : 0)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                for (int kt = 0; kt < num_kt; ++kt) {
-                    // both CTAs' operand tiles have landed and their scales sit in TMEM
-                    if (!__all_sync(0xffffffffu, (mbar_wait(&fullab_bar[stage], phase, wc) &&
-                                                  mbar_wait_cluster(&ready_bar[stage], phase, wc)) ? 1 : 0)) {
+            // loads in flight land before the CTAs may exit; the leader sees both
+            // CTAs' loads complete and the peer is held at the final cluster
+            // barrier until then
+            if (lane == 0 && rank == 0) {
+                int no_abort = 0;
+                WaitCtx w2{&no_abort, p.dev_status};
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued_any & (1u << s)) mbar_wait(&full_bar[s], (issued >> s) & 1u, w2);
+            }
+        } else if (warp == 1) {
+            if (rank == 0) {
+                // -------------------------------------------------------- MMA issuer (leader)
+                // The whole warp runs the loop so that descriptors and addresses
+                // stay warp-uniform; one elected lane issues.  Per K=64 step: three
+                // scale copies (this CTA's 128 A rows, the 256 B rows) from shared
+                // memory into the TMEM slot of the stage, then the MMA; copies and
+                // MMAs of one thread execute in issue order.
+                constexpr uint32_t idesc = idesc_nvf4(256, 256);
+                const uint32_t smem0 = smem_u32(smem);
+                int stage = 0;
+                uint32_t phase = 0, acc_phase = 0;
+                bool ok = true;
+                for (int t = pair; t < p.num_tiles && ok; t += npairs) {
+                    if (!__all_sync(0xffffffffu, mbar_wait_cluster(&acce_bar, acc_phase ^ 1u, wc) ? 1 : 0)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sb = smem0 + stage * STAGE_BYTES;
-                    const uint32_t sf_col = sf_base + stage * SF_COLS_STAGE;
-                    const int nks = k_atoms - kt * 4;
-                    if (elect_one()) {
-                        if (nks >= 4) {
-#pragma unroll
-                            for (int ks = 0; ks < 4; ++ks)
-                                tc_mma2_nvf4(tmem_base, sdesc_kmajor_sw128(sb + ks * 32),
-                                             sdesc_kmajor_sw128(sb + A_BYTES + ks * 32), idesc,
-                                             sf_col + ks * SF_COLS_STEP, sf_col + ks * SF_COLS_STEP + 4,
-                                             (kt | ks) != 0 ? 1u : 0u);
-                        } else {
-                            for (int ks = 0; ks < nks; ++ks)
-                                tc_mma2_nvf4(tmem_base, sdesc_kmajor_sw128(sb + ks * 32),
-                                             sdesc_kmajor_sw128(sb + A_BYTES + ks * 32), idesc,
-                                             sf_col + ks * SF_COLS_STEP, sf_col + ks * SF_COLS_STEP + 4,
-                                             (kt | ks) != 0 ? 1u : 0u);
+                    for (int kt = 0; kt < num_kt; ++kt) {
+                        if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[stage], phase, wc) ? 1 : 0)) {
+                            ok = false;
+                            break;
                         }
-                        tc_commit2_mc(&empty_bar[stage], 0x3);
+                        tc_fence_after();
+                        const uint32_t sb = smem0 + stage * STAGE_BYTES;
+                        const uint32_t sfs = sb + A_BYTES + B_BYTES;
+                        const uint32_t sf_col = sf_base + stage * SF_COLS_STAGE;
+                        const int nks = k_atoms - kt * 4;
+                        if (elect_one()) {
+                            if (nks >= 4) {
+    #pragma unroll
+                                for (int ks = 0; ks < 4; ++ks)
+                                    k_step(tmem_base, sb, sfs, sf_col, ks, idesc, (kt | ks) != 0);
+                            } else {
+                                for (int ks = 0; ks < nks; ++ks)
+                                    k_step(tmem_base, sb, sfs, sf_col, ks, idesc, (kt | ks) != 0);
+                            }
+                            tc_commit2_mc(&empty_bar[stage], 0x3);
+                        }
+                        __syncwarp();
+                        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                     }
+                    if (!ok) break;
+                    if (elect_one()) tc_commit2_mc(&accf_bar, 0x3);
                     __syncwarp();
-                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                    acc_phase ^= 1u;
                 }
-                if (!ok) break;
-                if (elect_one()) tc_commit2_mc(&accf_bar, 0x3);
+                if (elect_one()) tc_commit2_mc(&drain_bar, 0x1);
                 __syncwarp();
-                acc_phase ^= 1u;
+                int no_abort = 0;
+                WaitCtx w2{&no_abort, p.dev_status};
+                mbar_wait(&drain_bar, 0, w2);
             }
-            if (elect_one()) tc_commit2_mc(&drain_bar, 0x1);
-            __syncwarp();
-            int no_abort = 0;
-            WaitCtx w2{&no_abort, p.dev_status};
-            mbar_wait(&drain_bar, 0, w2);
         }
     } else {
+        regs_inc<kRegsHigh>();
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int q = warp & 3;                       // TMEM lane quarter
         const int h = (warp - 8) >> 2;                // column half: [0,128) or [128,256)
