@@ -10,12 +10,6 @@
 
 namespace nvfp4 {
 
-// True when q is within 8 ulps of a value whose low 21 fraction bits are
-// zero: every E2M1 rounding midpoint and grid point is such a value.
-__device__ __forceinline__ bool near_grid(float q) {
-    return ((__float_as_uint(q) + 8u) & 0x1FFFF0u) == 0u;
-}
-
 // True when r is within 8 ulps of a value whose low 19 fraction bits are zero:
 // every E4M3 rounding midpoint (4 significant bits, normal or subnormal) is
 // such a value.
@@ -70,35 +64,140 @@ __device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2,
     return r;
 }
 
-// Eight values with decoded block scale s -> four packed bytes (element 2j in
-// the low nibble of byte j).  The quotient is the IEEE single quotient: the
-// product with the approximate reciprocal lies within 3 ulps of it, and E2M1
-// rounding can only differ near a midpoint or grid point (a value whose low 21
-// fraction bits are zero), where the exact division is used.  The test maps
-// (bits + 8) mod 2^21 to the top of a word with one multiply-add, so "within
-// 8 ulps" is one unsigned comparison of the minimum.  Blocks whose s is
-// outside [2^-125, 2^125] use the exact division throughout.
+// Two FP32 values in one 64-bit register (low word first) for the packed
+// FP32 instructions of sm_100.
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// E2M1 pair (satfinite, round to nearest even) of a packed FP32 pair: the
+// low word's code in the low nibble.
+__device__ __forceinline__ uint32_t cvt_e2m1x2_packed(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return cvt_e2m1x2(lo, hi);
+}
+
+// Reciprocal bracket of s: rl <= 1/s <= rh, four ulps either side of the
+// hardware approximation (which is within one ulp of 1/s for normal s).
+struct RcpBracket {
+    uint64_t lo, hi;
+};
+
+__device__ __forceinline__ RcpBracket rcp_bracket(float s) {
+    const uint32_t rb = __float_as_uint(rcp_approx(s));
+    const float rl = __uint_as_float(rb - 4u), rh = __uint_as_float(rb + 4u);
+    return {f32x2(rl, rl), f32x2(rh, rh)};
+}
+
+// E2M1 codes of eight values given as four packed pairs, divided by the
+// decoded block scale s (IEEE single quotient, then RNE to E2M1, saturating).
+// The quotient is bracketed: |x * rl| <= |x / s| <= |x * rh| for the
+// reciprocal bracket of s, and both rounding to single precision and the
+// E2M1 rounding are monotone in magnitude, so where the codes of the two
+// bounds agree they are the code of the exact quotient.  Returns the codes
+// of the lower bound (element 2j in the low nibble of byte j) and, in `d`,
+// the nibbles where the bounds disagree (a rounding boundary lies inside the
+// bracket: about 1 value in 2000, because quotients a unit in the last place
+// from an E2M1 midpoint are common); those values must be divided exactly.
+__device__ __forceinline__ uint32_t bracket_codes8(const uint64_t (&x)[4], float s, uint32_t& d) {
+    const RcpBracket rb = rcp_bracket(s);
+    uint32_t cl[4], ch[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        cl[j] = cvt_e2m1x2_packed(mul_f32x2(x[j], rb.lo));
+        ch[j] = cvt_e2m1x2_packed(mul_f32x2(x[j], rb.hi));
+    }
+    const uint32_t w = pack4(cl[0], cl[1], cl[2], cl[3]);
+    d = w ^ pack4(ch[0], ch[1], ch[2], ch[3]);
+    return w;
+}
+
+// Replace nibble j of w by the E2M1 code of v / s (exact IEEE quotient).
+__device__ __forceinline__ uint32_t patch_exact(uint32_t w, int j, float v, float s) {
+    const uint32_t c = cvt_e2m1x2(__fdiv_rn(v, s), 0.0f) & 0xFu;
+    return (w & ~(0xFu << (4 * j))) | (c << (4 * j));
+}
+
+// s in the range where the reciprocal bracket is valid (normal reciprocal).
+__device__ __forceinline__ bool bracket_ok(float s) { return s >= 0x1p-125f && s <= 0x1p125f; }
+
+// Eight FP32 values (element 2j in the low nibble of byte j).  Blocks whose s
+// is outside the bracket range are divided exactly throughout.
 __device__ __forceinline__ uint32_t quantize8(const float (&f)[8], float s) {
     if (s == 0.0f) return 0u;
-    float q[8];
-    if (s >= 0x1p-125f && s <= 0x1p125f) {
-        const float rcp = rcp_approx(s);
-        uint32_t mn = 0xFFFFFFFFu;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            q[j] = __fmul_rn(f[j], rcp);
-            mn = min(mn, __float_as_uint(q[j]) * 2048u + 16384u);
-        }
-        if (mn < 32768u) {
+    uint32_t w = 0u;
+    if (bracket_ok(s)) {
+        const uint64_t x[4] = {f32x2(f[0], f[1]), f32x2(f[2], f[3]), f32x2(f[4], f[5]), f32x2(f[6], f[7])};
+        uint32_t d;
+        w = bracket_codes8(x, s, d);
+        // rare: the disagreeing values, by an unrolled scan (a register array
+        // indexed at run time would live in local memory)
+        if (d != 0u) {
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-                if (near_grid(q[j])) q[j] = __fdiv_rn(f[j], s);
+                if ((d >> (4 * j)) & 0xFu) w = patch_exact(w, j, f[j], s);
         }
     } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) q[j] = __fdiv_rn(f[j], s);
+        for (int j = 0; j < 8; ++j) w = patch_exact(w, j, f[j], s);
     }
-    return pack4(cvt_e2m1x2(q[0], q[1]), cvt_e2m1x2(q[2], q[3]), cvt_e2m1x2(q[4], q[5]), cvt_e2m1x2(q[6], q[7]));
+    return w;
+}
+
+// bf16 value j (0..7) of four words, the lower half of each word first, as FP32.
+__device__ __forceinline__ float bf16_at(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, int j) {
+    const uint32_t w = j < 2 ? w0 : j < 4 ? w1 : j < 6 ? w2 : w3;
+    return __uint_as_float((j & 1) ? (w & 0xFFFF0000u) : (w << 16));
+}
+
+// Eight bf16 values in four words (the lower half of each word first).
+__device__ __forceinline__ uint32_t quantize8_bf16(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float s) {
+    if (s == 0.0f) return 0u;
+    uint32_t w = 0u;
+    if (bracket_ok(s)) {
+        const uint64_t x[4] = {f32x2(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xFFFF0000u)),
+                               f32x2(__uint_as_float(w1 << 16), __uint_as_float(w1 & 0xFFFF0000u)),
+                               f32x2(__uint_as_float(w2 << 16), __uint_as_float(w2 & 0xFFFF0000u)),
+                               f32x2(__uint_as_float(w3 << 16), __uint_as_float(w3 & 0xFFFF0000u))};
+        uint32_t d;
+        w = bracket_codes8(x, s, d);
+        while (d != 0u) {                       // rare: one pass per disagreeing value
+            const int j = (31 - __clz(d)) >> 2;
+            w = patch_exact(w, j, bf16_at(w0, w1, w2, w3, j), s);
+            d &= ~(0xFu << (4 * j));
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w = patch_exact(w, j, bf16_at(w0, w1, w2, w3, j), s);
+    }
+    return w;
+}
+
+// Largest magnitude of two packed bf16 pairs, per half (sign bits are the
+// XOR of the inputs' and are cleared by the caller).  NaN operands are
+// ignored when the other operand is a number.
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// |x| pattern (sign cleared) of the largest-magnitude value among 16 bf16
+// values in eight words.
+__device__ __forceinline__ uint32_t block_absmax16(const uint32_t (&w)[8]) {
+    const uint32_t m = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(w[0], w[1]), absmax_bf16x2(w[2], w[3])),
+                                     absmax_bf16x2(absmax_bf16x2(w[4], w[5]), absmax_bf16x2(w[6], w[7])));
+    const uint32_t lo = m & 0x7FFFu, hi = (m >> 16) & 0x7FFFu;
+    return lo > hi ? lo : hi;
 }
 
 }  // namespace nvfp4

@@ -15,13 +15,10 @@
 //   sf = E4M3_rne_satfinite(a_b / (6 g)),  s = e4m3(sf) * g
 //   q  = x / s  (IEEE single quotient)   code = E2M1_rne_satfinite(q)
 //
-// Fast path for the quotient: q' = x * rn(1/s) lies within 3 ulps of the IEEE
-// quotient rn(x/s).  E2M1 rounding only depends on where q sits relative to
-// the seven midpoints {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5}; all of them (and
-// all grid points) have the low 21 fraction bits clear.  A lane whose q' is
-// within 4 ulps of such a value redoes that element with the exact quotient,
-// so the code always equals RNE(rn(x/s)).  Blocks whose s is outside
-// [2^-125, 2^125] (where 1/s loses bits) take the exact quotient throughout.
+// The quotient is bracketed by two products with a reciprocal bracket of s,
+// on packed FP32 pairs; where the two bounds give the same code it is the
+// code of the IEEE quotient, otherwise the values are divided exactly (see
+// quant_math.cuh).
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -32,24 +29,16 @@
 namespace nvfp4 {
 
 // ------------------------------------------------------------------ amax
-// Per-half maxima of |x| over 8 bf16 values: the sign bits are cleared and the
-// patterns compared as unsigned 16-bit integers (for non-negative IEEE values
-// the order of the patterns is the order of the values).
-__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
-    uint32_t r;
-    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-    return r;
-}
-
+// Per-half largest magnitude of 8 bf16 values (sign bits not meaningful).
 __device__ __forceinline__ uint32_t absmax_bf16x8(uint4 a) {
-    return max_u16x2(max_u16x2(a.x & 0x7FFF7FFFu, a.y & 0x7FFF7FFFu),
-                     max_u16x2(a.z & 0x7FFF7FFFu, a.w & 0x7FFF7FFFu));
+    return absmax_bf16x2(absmax_bf16x2(a.x, a.y), absmax_bf16x2(a.z, a.w));
 }
 
-// Partial max |x| per CTA over a [rows, k] bf16 tensor with row stride ld.
-// For non-negative IEEE values the bit patterns order like unsigned integers,
-// so |x| is the pattern with the sign cleared and the max is an integer max
-// on bf16 halves.
+// Partial max |x| per CTA over a [rows, k] bf16 tensor with row stride ld,
+// on bf16 pairs (max.xorsign.abs); NaNs are ignored when a number is beside
+// them, as in a max that skips unordered comparisons.  The final per-CTA
+// value compares non-negative bf16 patterns as integers (for non-negative
+// IEEE values the order of the patterns is the order of the values).
 __global__ void __launch_bounds__(kAmaxThreads)
 amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
             float* __restrict__ partials) {
@@ -63,16 +52,17 @@ amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
         for (; v + 3 * stride < nvec; v += 4 * stride) {
             const uint4 a = __ldcs(p + v), b = __ldcs(p + v + stride);
             const uint4 c = __ldcs(p + v + 2 * stride), d = __ldcs(p + v + 3 * stride);
-            m = max_u16x2(m, max_u16x2(absmax_bf16x8(a), absmax_bf16x8(b)));
-            m = max_u16x2(m, max_u16x2(absmax_bf16x8(c), absmax_bf16x8(d)));
+            m = absmax_bf16x2(m, absmax_bf16x2(absmax_bf16x8(a), absmax_bf16x8(b)));
+            m = absmax_bf16x2(m, absmax_bf16x2(absmax_bf16x8(c), absmax_bf16x8(d)));
         }
-        for (; v < nvec; v += stride) m = max_u16x2(m, absmax_bf16x8(__ldcs(p + v)));
+        for (; v < nvec; v += stride) m = absmax_bf16x2(m, absmax_bf16x8(__ldcs(p + v)));
     } else {
         for (; v < nvec; v += stride) {
             const int64_t r = v / k8, c = v - r * k8;
-            m = max_u16x2(m, absmax_bf16x8(__ldcs(reinterpret_cast<const uint4*>(x + r * ld) + c)));
+            m = absmax_bf16x2(m, absmax_bf16x8(__ldcs(reinterpret_cast<const uint4*>(x + r * ld) + c)));
         }
     }
+    m &= 0x7FFF7FFFu;
     uint32_t h = max(m & 0xFFFFu, m >> 16);
     for (int o = 16; o > 0; o >>= 1) h = max(h, __shfl_xor_sync(0xffffffffu, h, o));
     __shared__ uint32_t red[kAmaxThreads / 32];
@@ -102,9 +92,10 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
     // rows write (one per atom and row) fall in different banks
     constexpr int kAtomPitch = 516;
     __shared__ __align__(16) uint8_t sf_stage[4 * kAtomPitch];
-    __shared__ float g_sh;
+    __shared__ ScaleConsts sc_sh;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+    // the tensor scale and its block-scale constants, once per CTA
     if (warp == 0) {
         float g;
         if (kDynamic) {
@@ -116,11 +107,11 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
         } else {
             g = *tensor_scale;
         }
-        if (lane == 0) g_sh = g;
+        if (lane == 0) sc_sh = scale_consts(g);
     }
     __syncthreads();
-    const float g = g_sh;
-    const ScaleConsts sc = scale_consts(g);
+    const ScaleConsts sc = sc_sh;
+    const float g = sc.g;
 
     const int64_t row0 = (int64_t)blockIdx.y * 128;
     const int64_t c0 = (int64_t)blockIdx.x * 256;
@@ -152,23 +143,11 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
         const int64_t r = row0 + rt;
         const uint32_t w[8] = {v[2 * i].x, v[2 * i].y, v[2 * i].z, v[2 * i].w,
                                v[2 * i + 1].x, v[2 * i + 1].y, v[2 * i + 1].z, v[2 * i + 1].w};
-        // block amax (integer max of |bf16| patterns)
-        const uint32_t mm = max_u16x2(absmax_bf16x8(v[2 * i]), absmax_bf16x8(v[2 * i + 1]));
-        const uint32_t hb = max(mm & 0xFFFFu, mm >> 16);
-        const float ab = __uint_as_float(hb << 16);
-
+        const float ab = __uint_as_float(block_absmax16(w) << 16);      // block amax
         const uint32_t sfc = block_scale_code(ab, sc);
         const float s = __fmul_rn(e4m3_to_f32(sfc), g);
-        float f0[8], f1[8];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            f0[2 * j] = __uint_as_float(w[j] << 16);
-            f0[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-            f1[2 * j] = __uint_as_float(w[4 + j] << 16);
-            f1[2 * j + 1] = __uint_as_float(w[4 + j] & 0xFFFF0000u);
-        }
-        const uint32_t lo = quantize8(f0, s);
-        const uint32_t hi = quantize8(f1, s);
+        const uint32_t lo = quantize8_bf16(w[0], w[1], w[2], w[3], s);
+        const uint32_t hi = quantize8_bf16(w[4], w[5], w[6], w[7], s);
         if (r < rows && col_ok)
             *reinterpret_cast<uint2*>(codes + r * kh + (c0 >> 1) + blk * 8) = make_uint2(lo, hi);
         // block blk of this row: atom blk / 4, byte blk % 4 of the row's word
