@@ -242,23 +242,25 @@ def reduced(wl, args):
     return dataclasses.replace(wl, layers=tuple(keep))
 
 
-def kernel_source_hash() -> str:
-    """SHA-256 over the library's CUDA sources (names and contents).  A DRAM
-    traffic figure recorded under profiles/ is reported only while this
-    matches the hash recorded beside it: any source change voids it."""
+def kernel_source_hash(files=None) -> str:
+    """SHA-256 over CUDA sources of the library (names and contents): the
+    given file names under csrc/, or all of them.  A DRAM traffic figure
+    recorded under profiles/ is reported only while this matches the hash
+    recorded beside it: a change to any of those sources voids it."""
     import hashlib
     d = os.path.join(ROOT, "nvfp4_w4a4_gemm_quantize_b200", "csrc")
+    names = sorted(files) if files else sorted(n for n in os.listdir(d) if n.endswith((".cu", ".cuh", ".h")))
     h = hashlib.sha256()
-    for name in sorted(os.listdir(d)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            h.update(name.encode())
-            h.update(open(os.path.join(d, name), "rb").read())
+    for name in names:
+        h.update(name.encode())
+        h.update(open(os.path.join(d, name), "rb").read())
     return h.hexdigest()
 
 
 def profiled_traffic(summary: str):
     """DRAM bytes per launch (read + write) from an ncu summary under
-    profiles/, or None when it is absent or was taken on other sources."""
+    profiles/, or None when it is absent or was taken on other sources (the
+    summary lists its `source_files` and their `source_sha256`)."""
     p = os.path.join(ROOT, "profiles", summary)
     if not os.path.exists(p):
         return None
@@ -266,12 +268,13 @@ def profiled_traffic(summary: str):
     for line in open(p):
         if ":" in line:
             k, v = line.split(":", 1)
-            kv[k.strip()] = v.strip()
-    if kv.get("source_sha256") != kernel_source_hash():
-        return None
+            kv.setdefault(k.strip(), v.strip())
+    files = kv.get("source_files", "").split() or None
     try:
+        if kv.get("source_sha256") != kernel_source_hash(files):
+            return None
         return int(kv["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
+    except (KeyError, ValueError, OSError):
         return None
 
 

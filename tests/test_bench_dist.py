@@ -110,3 +110,12 @@ def test_recorded_traffic_is_void_when_sources_change(tmp_path, monkeypatch):
     (src / "k.cu").write_text("// kernel v2\n")
     assert bench.kernel_source_hash() != h
     assert bench.profiled_traffic("k.txt") is None
+    # a summary that names its sources is voided only by those
+    (src / "other.cu").write_text("// unrelated kernel\n")
+    h2 = bench.kernel_source_hash(["k.cu"])
+    (prof / "k2.txt").write_text(f"source_files: k.cu\nsource_sha256: {h2}\ndram_bytes_per_launch: 7\n")
+    assert bench.profiled_traffic("k2.txt") == 7
+    (src / "other.cu").write_text("// unrelated kernel, changed\n")
+    assert bench.profiled_traffic("k2.txt") == 7
+    (src / "k.cu").write_text("// kernel v3\n")
+    assert bench.profiled_traffic("k2.txt") is None
