@@ -78,12 +78,23 @@ __device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
     return r;
 }
 
-// E2M1 pair (satfinite, round to nearest even) of a packed FP32 pair: the
-// low word's code in the low nibble.
-__device__ __forceinline__ uint32_t cvt_e2m1x2_packed(uint64_t v) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-    return cvt_e2m1x2(lo, hi);
+// E2M1 codes of four packed FP32 pairs (satfinite, RNE) in one word: byte j
+// holds pair j, its low word's code in the low nibble.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(uint64_t p0, uint64_t p1, uint64_t p2, uint64_t p3) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t0, t1, t2, t3;\n\t.reg .f32 a0, a1, a2, a3, a4, a5, a6, a7;\n\t"
+        "mov.b64 {a0, a1}, %1;\n\t"
+        "mov.b64 {a2, a3}, %2;\n\t"
+        "mov.b64 {a4, a5}, %3;\n\t"
+        "mov.b64 {a6, a7}, %4;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t0, a1, a0;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t1, a3, a2;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t2, a5, a4;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t3, a7, a6;\n\t"
+        "mov.b32 %0, {t0, t1, t2, t3};\n\t}"
+        : "=r"(r)
+        : "l"(p0), "l"(p1), "l"(p2), "l"(p3));
+    return r;
 }
 
 // Reciprocal bracket of s: rl <= 1/s <= rh, four ulps either side of the
@@ -110,14 +121,10 @@ __device__ __forceinline__ RcpBracket rcp_bracket(float s) {
 // from an E2M1 midpoint are common); those values must be divided exactly.
 __device__ __forceinline__ uint32_t bracket_codes8(const uint64_t (&x)[4], float s, uint32_t& d) {
     const RcpBracket rb = rcp_bracket(s);
-    uint32_t cl[4], ch[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        cl[j] = cvt_e2m1x2_packed(mul_f32x2(x[j], rb.lo));
-        ch[j] = cvt_e2m1x2_packed(mul_f32x2(x[j], rb.hi));
-    }
-    const uint32_t w = pack4(cl[0], cl[1], cl[2], cl[3]);
-    d = w ^ pack4(ch[0], ch[1], ch[2], ch[3]);
+    const uint32_t w = cvt_e2m1x8(mul_f32x2(x[0], rb.lo), mul_f32x2(x[1], rb.lo), mul_f32x2(x[2], rb.lo),
+                                  mul_f32x2(x[3], rb.lo));
+    d = w ^ cvt_e2m1x8(mul_f32x2(x[0], rb.hi), mul_f32x2(x[1], rb.hi), mul_f32x2(x[2], rb.hi),
+                       mul_f32x2(x[3], rb.hi));
     return w;
 }
 

@@ -123,14 +123,24 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
 
     constexpr int kRows = 128 / (kQuantThreads / 32);   // rows per warp
     constexpr int kSteps = kRows / 2;
+    // step i handles row rt0 + 2i of the tile; pointers for step 0, advanced
+    // by two rows per step (ld and kh are multiples of 8 and 32)
+    const int rt0 = warp * kRows + half;
+    const int64_t r0 = row0 + rt0;
+    const int64_t rows_left = rows - r0;          // step i is in range iff 2i < rows_left
+    const uint4* xp = reinterpret_cast<const uint4*>(x + r0 * ld + c0) + 2 * blk;
+    const int64_t xstep = ld >> 2;                // two rows, in 16-byte units
+    uint2* cp = reinterpret_cast<uint2*>(codes + r0 * kh + (c0 >> 1)) + blk;
+    const int64_t cstep = kh >> 2;                // two rows, in 8-byte units
+    // block blk of row rt: atom blk / 4, byte blk % 4 of the row's word
+    const int sbase = (blk >> 2) * kAtomPitch + (rt0 & 31) * 16 + (rt0 >> 5) * 4 + (blk & 3);
+
     uint4 v[2 * kSteps];
 #pragma unroll
     for (int i = 0; i < kSteps; ++i) {
-        const int64_t r = row0 + warp * kRows + 2 * i + half;
-        if (r < rows && col_ok) {
-            const uint4* src = reinterpret_cast<const uint4*>(x + r * ld + c0) + 2 * blk;
-            v[2 * i] = __ldcs(src);
-            v[2 * i + 1] = __ldcs(src + 1);
+        if (2 * i < rows_left && col_ok) {
+            v[2 * i] = __ldcs(xp + i * xstep);
+            v[2 * i + 1] = __ldcs(xp + i * xstep + 1);
         } else {
             v[2 * i] = make_uint4(0u, 0u, 0u, 0u);
             v[2 * i + 1] = make_uint4(0u, 0u, 0u, 0u);
@@ -139,8 +149,6 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
 
 #pragma unroll
     for (int i = 0; i < kSteps; ++i) {
-        const int rt = warp * kRows + 2 * i + half;   // row inside the tile
-        const int64_t r = row0 + rt;
         const uint32_t w[8] = {v[2 * i].x, v[2 * i].y, v[2 * i].z, v[2 * i].w,
                                v[2 * i + 1].x, v[2 * i + 1].y, v[2 * i + 1].z, v[2 * i + 1].w};
         const float ab = __uint_as_float(block_absmax16(w) << 16);      // block amax
@@ -148,18 +156,17 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
         const float s = __fmul_rn(e4m3_to_f32(sfc), g);
         const uint32_t lo = quantize8_bf16(w[0], w[1], w[2], w[3], s);
         const uint32_t hi = quantize8_bf16(w[4], w[5], w[6], w[7], s);
-        if (r < rows && col_ok)
-            *reinterpret_cast<uint2*>(codes + r * kh + (c0 >> 1) + blk * 8) = make_uint2(lo, hi);
-        // block blk of this row: atom blk / 4, byte blk % 4 of the row's word
-        if (col_ok) sf_stage[(blk >> 2) * kAtomPitch + (rt & 31) * 16 + (rt >> 5) * 4 + (blk & 3)] = (uint8_t)sfc;
+        if (2 * i < rows_left && col_ok) cp[i * cstep] = make_uint2(lo, hi);
+        if (col_ok) sf_stage[sbase + 32 * i] = (uint8_t)sfc;
     }
     __syncthreads();
-    // this tile's atoms are consecutive in the scale buffer
+    // this tile's atoms are consecutive in the scale buffer: one word per thread
+    static_assert(4 * 128 <= kQuantThreads, "scale copy-out: one word per thread");
     const int natoms = ncols >> 6;
     const int64_t kb4 = k >> 6;                       // atoms per 128-row block
     uint32_t* dst = reinterpret_cast<uint32_t*>(sf + (((int64_t)blockIdx.y * kb4 + blockIdx.x * 4) << 9));
-    for (int i = threadIdx.x; i < natoms * 128; i += kQuantThreads)
-        dst[i] = *reinterpret_cast<const uint32_t*>(sf_stage + (i >> 7) * kAtomPitch + (i & 127) * 4);
+    const int i = threadIdx.x;
+    if (i < natoms * 128) dst[i] = *reinterpret_cast<const uint32_t*>(sf_stage + (i >> 7) * kAtomPitch + (i & 127) * 4);
 }
 
 // ------------------------------------------------------------------ dequantize
