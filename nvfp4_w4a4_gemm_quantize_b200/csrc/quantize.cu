@@ -42,6 +42,9 @@ __device__ __forceinline__ uint32_t absmax_bf16x8(uint4 a) {
 __global__ void __launch_bounds__(kAmaxThreads)
 amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
             float* __restrict__ partials) {
+    // the quantize kernel that follows may start (and load X) now; it waits
+    // for this grid's results before it reads the partial maxima
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t k8 = k >> 3;                        // 16-byte vectors per row
     const int64_t nvec = rows * k8;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -50,16 +53,16 @@ amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
     if (ld == k) {
         const uint4* p = reinterpret_cast<const uint4*>(x);
         for (; v + 3 * stride < nvec; v += 4 * stride) {
-            const uint4 a = __ldcs(p + v), b = __ldcs(p + v + stride);
-            const uint4 c = __ldcs(p + v + 2 * stride), d = __ldcs(p + v + 3 * stride);
+            const uint4 a = __ldg(p + v), b = __ldg(p + v + stride);
+            const uint4 c = __ldg(p + v + 2 * stride), d = __ldg(p + v + 3 * stride);
             m = absmax_bf16x2(m, absmax_bf16x2(absmax_bf16x8(a), absmax_bf16x8(b)));
             m = absmax_bf16x2(m, absmax_bf16x2(absmax_bf16x8(c), absmax_bf16x8(d)));
         }
-        for (; v < nvec; v += stride) m = absmax_bf16x2(m, absmax_bf16x8(__ldcs(p + v)));
+        for (; v < nvec; v += stride) m = absmax_bf16x2(m, absmax_bf16x8(__ldg(p + v)));
     } else {
         for (; v < nvec; v += stride) {
             const int64_t r = v / k8, c = v - r * k8;
-            m = absmax_bf16x2(m, absmax_bf16x8(__ldcs(reinterpret_cast<const uint4*>(x + r * ld) + c)));
+            m = absmax_bf16x2(m, absmax_bf16x8(__ldg(reinterpret_cast<const uint4*>(x + r * ld) + c)));
         }
     }
     m &= 0x7FFF7FFFu;
@@ -95,25 +98,10 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
     __shared__ ScaleConsts sc_sh;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // the tensor scale and its block-scale constants, once per CTA
-    if (warp == 0) {
-        float g;
-        if (kDynamic) {
-            float mx = 0.0f;
-            for (int i = lane; i < nparts; i += 32) mx = fmaxf(mx, partials[i]);
-            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            g = __fdiv_rn(mx, 2688.0f);
-            if (blockIdx.x == 0 && blockIdx.y == 0 && lane == 0) *tensor_scale = g;
-        } else {
-            g = *tensor_scale;
-        }
-        if (lane == 0) sc_sh = scale_consts(g);
-    }
-    __syncthreads();
-    const ScaleConsts sc = sc_sh;
-    const float g = sc.g;
-
-    const int64_t row0 = (int64_t)blockIdx.y * 128;
+    // row blocks in reverse launch order: the amax pass read the tensor front
+    // to back, so its tail is the part still in L2 when the first CTAs start
+    const int64_t rblk = (int64_t)(gridDim.y - 1 - blockIdx.y);
+    const int64_t row0 = rblk * 128;
     const int64_t c0 = (int64_t)blockIdx.x * 256;
     const int ncols = (k - c0) < 256 ? (int)(k - c0) : 256;   // multiple of 64
     const int half = lane >> 4;                   // which row of the pair
@@ -147,6 +135,26 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
         }
     }
 
+    // the tensor scale and its block-scale constants, once per CTA, after the
+    // amax grid (when launched as its programmatic dependent) has completed
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (warp == 0) {
+        float g;
+        if (kDynamic) {
+            float mx = 0.0f;
+            for (int i = lane; i < nparts; i += 32) mx = fmaxf(mx, partials[i]);
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            g = __fdiv_rn(mx, 2688.0f);
+            if (blockIdx.x == 0 && blockIdx.y == 0 && lane == 0) *tensor_scale = g;   // one writer
+        } else {
+            g = *tensor_scale;
+        }
+        if (lane == 0) sc_sh = scale_consts(g);
+    }
+    __syncthreads();
+    const ScaleConsts sc = sc_sh;
+    const float g = sc.g;
+
 #pragma unroll
     for (int i = 0; i < kSteps; ++i) {
         const uint32_t w[8] = {v[2 * i].x, v[2 * i].y, v[2 * i].z, v[2 * i].w,
@@ -164,7 +172,7 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
     static_assert(4 * 128 <= kQuantThreads, "scale copy-out: one word per thread");
     const int natoms = ncols >> 6;
     const int64_t kb4 = k >> 6;                       // atoms per 128-row block
-    uint32_t* dst = reinterpret_cast<uint32_t*>(sf + (((int64_t)blockIdx.y * kb4 + blockIdx.x * 4) << 9));
+    uint32_t* dst = reinterpret_cast<uint32_t*>(sf + ((rblk * kb4 + blockIdx.x * 4) << 9));
     const int i = threadIdx.x;
     if (i < natoms * 128) dst[i] = *reinterpret_cast<const uint32_t*>(sf_stage + (i >> 7) * kAtomPitch + (i & 127) * 4);
 }
@@ -246,9 +254,22 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t k, int64_t 
     }
     const int ag = amax_grid(rows, k);
     amax_kernel<<<ag, kAmaxThreads, 0, stream>>>(x, rows, k, ld, partials);
-    quantize_kernel<true><<<grid, kQuantThreads, 0, stream>>>(x, rows, k, ld, codes, sf, tensor_scale,
-                                                             partials, ag);
+    // programmatic dependent launch: the quantize CTAs start loading X while
+    // the amax grid finishes, and wait for it before reading its partials
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kQuantThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, quantize_kernel<true>, x, rows, k, ld, codes, sf, tensor_scale,
+                                       (const float*)partials, ag);
     count_launch(2);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
