@@ -38,7 +38,9 @@
  *    internal wait writes NVFP4_ERR_TIMEOUT there and returns without hanging.
  *    The library never clears it; the caller zeroes it and reads it after the
  *    stream has synchronized.
- *  - Inputs must be finite; non-finite values give unspecified codes.
+ *  - Inputs must be finite; non-finite values give unspecified codes.  The
+ *    amax pass of nvfp4_quantize (data-derived tensor scale) detects them and
+ *    writes NVFP4_ERR_NONFINITE to dev_status (if no error is there yet).
  */
 #ifndef NVFP4_H_
 #define NVFP4_H_
@@ -60,7 +62,8 @@ typedef enum {
     NVFP4_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not compute capability 10.0    */
     NVFP4_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed                */
     NVFP4_ERR_TIMEOUT = 6,            /* device-side bounded wait expired (dev_status)    */
-    NVFP4_ERR_WORKSPACE = 7           /* workspace missing or too small                   */
+    NVFP4_ERR_WORKSPACE = 7,          /* workspace missing or too small                   */
+    NVFP4_ERR_NONFINITE = 8           /* input held Inf or NaN (dev_status, amax pass)     */
 } nvfp4_status;
 
 enum { NVFP4_DTYPE_BF16 = 0, NVFP4_DTYPE_F32 = 1 };
@@ -183,6 +186,23 @@ const char *nvfp4_status_string(nvfp4_status s);
 /* Number of this library's kernels launched since load (host-side counter,
  * all threads).  For accounting in benchmarks. */
 uint64_t nvfp4_launch_count(void);
+
+/* Forget the library's host-side caches (per-device capability checks and the
+ * device address of nvfp4_quantize_noalloc's scratch array); the next call
+ * looks them up again.  Frees nothing on the device (the library holds no
+ * device allocation).  Not safe concurrently with other calls. */
+void nvfp4_shutdown(void);
+
+/*
+ * nvfp4_debug_wait_timeout -- the pages have no counterpart: a check of the
+ * library's failure detection.  Launches one warp that waits, through the
+ * same bounded mbarrier wait the GEMM and quantize kernels use, on a barrier
+ * that nothing ever arrives at.  After limit_us microseconds (1 .. 2000000)
+ * the wait gives up, the kernel writes NVFP4_ERR_TIMEOUT to *dev_status and
+ * returns: the stream and the context stay usable.  dev_status must be a
+ * device int the caller zeroed.
+ */
+nvfp4_status nvfp4_debug_wait_timeout(int *dev_status, int64_t limit_us, nvfp4_stream_t stream);
 
 #ifdef __cplusplus
 }

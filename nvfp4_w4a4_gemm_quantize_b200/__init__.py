@@ -57,6 +57,18 @@ def nvfp4_launch_count() -> int:
     return int(lib().nvfp4_launch_count())
 
 
+def nvfp4_shutdown() -> None:
+    lib().nvfp4_shutdown()
+
+
+def nvfp4_debug_wait_timeout(dev_status, limit_us: int, stream=None) -> None:
+    """Check of the failure detection: one warp waits, with the library's
+    bounded wait, on a barrier nothing arrives at, gives up after limit_us and
+    writes NVFP4_ERR_TIMEOUT to dev_status (a zeroed device int32)."""
+    st = lib().nvfp4_debug_wait_timeout(_ptr(dev_status), limit_us, _stream(stream))
+    check(st, "nvfp4_debug_wait_timeout")
+
+
 def nvfp4_quantize(x, rows, k, ld_x, codes, sf, tensor_scale, flags=0, workspace=None,
                    workspace_bytes=0, dev_status=None, stream=None) -> None:
     st = lib().nvfp4_quantize(_ptr(x), rows, k, ld_x, _ptr(codes), _ptr(sf), _ptr(tensor_scale),

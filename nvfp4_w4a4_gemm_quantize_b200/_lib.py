@@ -23,7 +23,7 @@ _status = ctypes.c_int
 STATUS = {
     0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_UNSUPPORTED_SHAPE",
     3: "NVFP4_ERR_MISALIGNED", 4: "NVFP4_ERR_UNSUPPORTED_DEVICE", 5: "NVFP4_ERR_CUDA",
-    6: "NVFP4_ERR_TIMEOUT", 7: "NVFP4_ERR_WORKSPACE",
+    6: "NVFP4_ERR_TIMEOUT", 7: "NVFP4_ERR_WORKSPACE", 8: "NVFP4_ERR_NONFINITE",
 }
 
 # every symbol include/nvfp4.h declares, with (restype, argtypes)
@@ -37,6 +37,8 @@ SIGNATURES = {
     "nvfp4_gemm_w4a16": (_status, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _int, _p, _p]),
     "nvfp4_status_string": (ctypes.c_char_p, [_int]),
     "nvfp4_launch_count": (ctypes.c_uint64, []),
+    "nvfp4_shutdown": (None, []),
+    "nvfp4_debug_wait_timeout": (_status, [_p, _i64, _p]),
 }
 
 

@@ -100,7 +100,6 @@ size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t k) {
 nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, uint8_t* codes, uint8_t* sf,
                             float* tensor_scale, unsigned flags, void* workspace, size_t workspace_bytes,
                             int* dev_status, nvfp4_stream_t stream) {
-    (void)dev_status;
     if (rows < 0 || k <= 0 || ld_x < k) return NVFP4_ERR_INVALID_ARG;
     if ((flags & ~(unsigned)NVFP4_SCALE_GIVEN) != 0u) return NVFP4_ERR_INVALID_ARG;
     if (!tensor_scale) return NVFP4_ERR_INVALID_ARG;
@@ -120,7 +119,7 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t
         return NVFP4_OK;
     }
     return cuda_status(launch_quantize(static_cast<const uint16_t*>(x_bf16), rows, k, ld_x, codes, sf, tensor_scale,
-                                       given, static_cast<float*>(workspace), s));
+                                       given, static_cast<float*>(workspace), dev_status, s));
 }
 
 nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* sf, const float* tensor_scale, int64_t rows,
@@ -199,10 +198,25 @@ const char* nvfp4_status_string(nvfp4_status s) {
         case NVFP4_ERR_CUDA: return "CUDA error";
         case NVFP4_ERR_TIMEOUT: return "device-side wait timed out";
         case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+        case NVFP4_ERR_NONFINITE: return "input holds Inf or NaN";
     }
     return "unknown status";
 }
 
 uint64_t nvfp4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void nvfp4_shutdown(void) {
+    for (auto& d : g_dev) d = DevInfo{};
+    reset_noalloc_cache();
+}
+
+nvfp4_status nvfp4_debug_wait_timeout(int* dev_status, int64_t limit_us, nvfp4_stream_t stream) {
+    if (!dev_status || limit_us < 1 || limit_us > 2000000) return NVFP4_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0u) return NVFP4_ERR_MISALIGNED;
+    nvfp4_status st = device_ok(nullptr);
+    if (st != NVFP4_OK) return st;
+    return cuda_status(launch_debug_wait_timeout(dev_status, (uint64_t)limit_us * 1000ull,
+                                                 reinterpret_cast<cudaStream_t>(stream)));
+}
 
 }  // extern "C"

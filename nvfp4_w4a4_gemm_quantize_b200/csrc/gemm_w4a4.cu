@@ -11,8 +11,9 @@
 // Kernel shape (one CTA per SM, persistent over output tiles):
 //   warp 0      TMA producer: code tiles (tensor maps, 128-byte swizzle) and
 //               scale atoms (bulk copies) into a STAGES-deep shared ring.
-//   warp 1      TMEM owner and MMA issuer: per stage, tcgen05.cp moves the
-//               scale atoms into TMEM, then one tcgen05.mma per K=64 step.
+//   warp 1      TMEM owner and MMA issuer: per K=64 step, tcgen05.cp moves
+//               the step's scale atoms into TMEM, then one tcgen05.mma.
+//   (both run the loop on the whole warp; one elected lane issues)
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator, alpha, conversion,
 //               TMA stores (bf16 / FP32) or direct stores (NVFP4).
 // Tile: 128 (M) x BN (N) x 256 (K per stage).  TMEM: 512 columns, the
@@ -133,27 +134,33 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
     const int num_kt = (p.K + 255) / 256;
     const int k_atoms = p.K / 64;                 // scale atoms per 128-row block
 
+    // Producer and MMA issuer run on whole warps with one elected lane issuing,
+    // so descriptors, coordinates and addresses stay warp-uniform (from a
+    // single lane each tcgen05 or TMA instruction costs tens of cycles to issue).
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            const uint64_t pol_a = policy_evict_normal();
-            const uint64_t pol_b = policy_evict_last();
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t issued = 0;                     // bit s: parity of the last load into stage s
-            uint32_t issued_any = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-                int mb, nb;
-                tile_coords(t, p.num_mb, p.num_nb, mb, nb);
-                const int nblk0 = nb * (BN / 128);
-                const int nblk_total = (p.N + 127) / 128;
-                for (int kt = 0; kt < num_kt; ++kt) {
-                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, wc)) { ok = false; break; }
-                    uint8_t* sbase = smem + stage * C::STAGE_BYTES;
-                    const int natoms = min(4, k_atoms - kt * 4);
-                    int nsfb = 0;
-                    for (int j = 0; j < BN / 128; ++j) nsfb += (nblk0 + j < nblk_total) ? 1 : 0;
+        const uint64_t pol_a = policy_evict_normal();
+        const uint64_t pol_b = policy_evict_last();
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t issued = 0;                     // bit s: parity of the last load into stage s
+        uint32_t issued_any = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+            int mb, nb;
+            tile_coords(t, p.num_mb, p.num_nb, mb, nb);
+            const int nblk0 = nb * (BN / 128);
+            const int nblk_total = (p.N + 127) / 128;
+            for (int kt = 0; kt < num_kt; ++kt) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&empty_bar[stage], phase ^ 1u, wc) ? 1 : 0)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* sbase = smem + stage * C::STAGE_BYTES;
+                const int natoms = min(4, k_atoms - kt * 4);
+                int nsfb = 0;
+                for (int j = 0; j < BN / 128; ++j) nsfb += (nblk0 + j < nblk_total) ? 1 : 0;
+                if (elect_one()) {
                     const uint32_t bytes = A_BYTES + C::B_BYTES + natoms * SF_ATOM * (1 + nsfb);
                     mbar_arrive_expect_tx(&full_bar[stage], bytes);
                     tma_load_2d(sbase, &tmap_a, &full_bar[stage], kt * BK_BYTES, mb * BM, pol_a);
@@ -165,12 +172,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
                         bulk_load(sbase + A_BYTES + C::B_BYTES + SFA_BYTES + j * SFA_BYTES,
                                   p.b_sf + ((int64_t)(nblk0 + j) * k_atoms + kt * 4) * SF_ATOM,
                                   natoms * SF_ATOM, &full_bar[stage], pol_b);
-                    issued = (issued & ~(1u << stage)) | (phase << stage);
-                    issued_any |= 1u << stage;
-                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
+                __syncwarp();
+                issued = (issued & ~(1u << stage)) | (phase << stage);
+                issued_any |= 1u << stage;
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
-            // every load this thread issued has landed before the CTA may exit
+        }
+        // every load this warp issued has landed before the CTA may exit
+        if (lane == 0) {
             for (int s = 0; s < STAGES; ++s)
                 if (issued_any & (1u << s)) {
                     WaitCtx w2{&abort_sh, p.dev_status};
@@ -181,53 +191,60 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_nvf4(BM, BN);
-            int stage = 0;
-            uint32_t phase = 0;
-            int acc = 0;
-            uint32_t acc_phase = 0;
-            bool ok = true;
-            const uint32_t sf_base = tmem_base + 256;
-            for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-                if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, wc)) { ok = false; break; }
+        constexpr uint32_t idesc = idesc_nvf4(BM, BN);
+        const uint32_t smem0 = smem_u32(smem);
+        int stage = 0;
+        uint32_t phase = 0;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        const uint32_t sf_base = tmem_base + 256;
+        for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&acce_bar[acc], acc_phase ^ 1u, wc) ? 1 : 0)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + acc * BN;
+            for (int kt = 0; kt < num_kt; ++kt) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[stage], phase, wc) ? 1 : 0)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + acc * BN;
-                for (int kt = 0; kt < num_kt; ++kt) {
-                    if (!mbar_wait(&full_bar[stage], phase, wc)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t sbase = smem_u32(smem + stage * C::STAGE_BYTES);
-                    const uint32_t sfa_s = sbase + A_BYTES + C::B_BYTES;
-                    const uint32_t sfb_s = sfa_s + SFA_BYTES;
-                    const uint32_t sf_col = sf_base + stage * C::SF_COLS_STAGE;
-                    const int nks = min(4, k_atoms - kt * 4);
+                const uint32_t sbase = smem0 + stage * C::STAGE_BYTES;
+                const uint32_t sfa_s = sbase + A_BYTES + C::B_BYTES;
+                const uint32_t sfb_s = sfa_s + SFA_BYTES;
+                const uint32_t sf_col = sf_base + stage * C::SF_COLS_STAGE;
+                const int nks = min(4, k_atoms - kt * 4);
+                if (elect_one()) {
                     for (int ks = 0; ks < nks; ++ks) {
                         const uint32_t col = sf_col + ks * C::SF_COLS_STEP;
                         tc_cp_32x128b_warpx4(col, sdesc_sf(sfa_s + ks * SF_ATOM));
 #pragma unroll
                         for (int j = 0; j < BN / 128; ++j)
                             tc_cp_32x128b_warpx4(col + 4 + 4 * j, sdesc_sf(sfb_s + j * SFA_BYTES + ks * SF_ATOM));
-                    }
-                    for (int ks = 0; ks < nks; ++ks) {
-                        const uint32_t col = sf_col + ks * C::SF_COLS_STEP;
                         tc_mma_nvf4(d_tmem, sdesc_kmajor_sw128(sbase + ks * 32),
                                     sdesc_kmajor_sw128(sbase + A_BYTES + ks * 32), idesc, col, col + 4,
                                     (kt | ks) != 0 ? 1u : 0u);
                     }
                     tc_commit(&empty_bar[stage]);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
-                if (!ok) break;
-                tc_commit(&accf_bar[acc]);
-                if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
+                __syncwarp();
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
-            // all MMAs issued by this thread complete before TMEM is released
-            tc_commit(&drain_bar);
-            WaitCtx w2{&abort_sh, p.dev_status};
-            int dummy_abort = 0;
-            w2.abort_flag = &dummy_abort;
-            mbar_wait(&drain_bar, 0, w2);
+            if (!ok) break;
+            if (elect_one()) tc_commit(&accf_bar[acc]);
+            __syncwarp();
+            if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
         }
+        // all MMAs issued by this warp complete before TMEM is released
+        if (elect_one()) tc_commit(&drain_bar);
+        __syncwarp();
+        WaitCtx w2{&abort_sh, p.dev_status};
+        int dummy_abort = 0;
+        w2.abort_flag = &dummy_abort;
+        mbar_wait(&drain_bar, 0, w2);
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;                       // TMEM lane quarter

@@ -17,7 +17,11 @@ int amax_grid(int64_t rows, int64_t k);
 
 cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes,
                             uint8_t* sf, float* tensor_scale, bool scale_given, float* partials,
-                            cudaStream_t stream);
+                            int* dev_status, cudaStream_t stream);
+
+cudaError_t launch_debug_wait_timeout(int* dev_status, uint64_t limit_ns, cudaStream_t stream);
+
+void reset_noalloc_cache();
 
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* sf, const float* tensor_scale,
                               int64_t rows, int64_t k, void* out, bool bf16, cudaStream_t stream);

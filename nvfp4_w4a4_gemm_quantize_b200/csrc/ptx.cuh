@@ -97,6 +97,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     }
 }
 
+// The same bounded wait with a caller-given limit in nanoseconds.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, const WaitCtx& w, uint64_t limit_ns) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    uint64_t t0 = globaltimer_ns();
+    uint32_t n = 0;
+    while (true) {
+        if (mbar_try_wait(a, parity)) return true;
+        if ((++n & 255u) == 0u) {
+            if (*w.abort_flag) return false;
+            if (globaltimer_ns() - t0 > limit_ns) {
+                report_timeout(w);
+                return false;
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------ fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -34,6 +34,23 @@ __device__ __forceinline__ uint32_t absmax_bf16x8(uint4 a) {
     return absmax_bf16x2(absmax_bf16x2(a.x, a.y), absmax_bf16x2(a.z, a.w));
 }
 
+// Per-half largest exponent field of 8 bf16 values (0xFF in a half: an Inf or
+// a NaN is among them).
+__device__ __forceinline__ uint32_t expmax_bf16x8(uint4 a) {
+    const uint32_t m = 0x7F807F80u;
+    uint32_t r, t;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a.x & m), "r"(a.y & m));
+    asm("max.u16x2 %0, %1, %2;" : "=r"(t) : "r"(a.z & m), "r"(a.w & m));
+    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(r), "r"(t));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 // Partial max |x| per CTA over a [rows, k] bf16 tensor with row stride ld,
 // on bf16 pairs (max.xorsign.abs); NaNs are ignored when a number is beside
 // them, as in a max that skips unordered comparisons.  The final per-CTA
@@ -41,7 +58,7 @@ __device__ __forceinline__ uint32_t absmax_bf16x8(uint4 a) {
 // IEEE values the order of the patterns is the order of the values).
 __global__ void __launch_bounds__(kAmaxThreads)
 amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
-            float* __restrict__ partials) {
+            float* __restrict__ partials, int* __restrict__ dev_status) {
     // the quantize kernel that follows may start (and load X) now; it waits
     // for this grid's results before it reads the partial maxima
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -49,6 +66,7 @@ amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
     const int64_t nvec = rows * k8;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     uint32_t m = 0;                                   // two bf16 |x| maxima
+    uint32_t e = 0;                                   // two exponent-field maxima
     int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (ld == k) {
         const uint4* p = reinterpret_cast<const uint4*>(x);
@@ -57,14 +75,26 @@ amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
             const uint4 c = __ldg(p + v + 2 * stride), d = __ldg(p + v + 3 * stride);
             m = absmax_bf16x2(m, absmax_bf16x2(absmax_bf16x8(a), absmax_bf16x8(b)));
             m = absmax_bf16x2(m, absmax_bf16x2(absmax_bf16x8(c), absmax_bf16x8(d)));
+            e = max_u16x2(e, max_u16x2(max_u16x2(expmax_bf16x8(a), expmax_bf16x8(b)),
+                                       max_u16x2(expmax_bf16x8(c), expmax_bf16x8(d))));
         }
-        for (; v < nvec; v += stride) m = absmax_bf16x2(m, absmax_bf16x8(__ldg(p + v)));
+        for (; v < nvec; v += stride) {
+            const uint4 a = __ldg(p + v);
+            m = absmax_bf16x2(m, absmax_bf16x8(a));
+            e = max_u16x2(e, expmax_bf16x8(a));
+        }
     } else {
         for (; v < nvec; v += stride) {
             const int64_t r = v / k8, c = v - r * k8;
-            m = absmax_bf16x2(m, absmax_bf16x8(__ldg(reinterpret_cast<const uint4*>(x + r * ld) + c)));
+            const uint4 a = __ldg(reinterpret_cast<const uint4*>(x + r * ld) + c);
+            m = absmax_bf16x2(m, absmax_bf16x8(a));
+            e = max_u16x2(e, expmax_bf16x8(a));
         }
     }
+    // any Inf or NaN: flag it (the first error written stays)
+    const bool nonfinite = (e & 0xFFFFu) == 0x7F80u || (e >> 16) == 0x7F80u;
+    if (__syncthreads_or(nonfinite ? 1 : 0) && threadIdx.x == 0 && dev_status)
+        atomicCAS(dev_status, 0, (int)NVFP4_ERR_NONFINITE);
     m &= 0x7FFF7FFFu;
     uint32_t h = max(m & 0xFFFFu, m >> 16);
     for (int o = 16; o > 0; o >>= 1) h = max(h, __shfl_xor_sync(0xffffffffu, h, o));
@@ -244,7 +274,7 @@ int amax_grid(int64_t rows, int64_t k) {
 
 cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes,
                             uint8_t* sf, float* tensor_scale, bool scale_given, float* partials,
-                            cudaStream_t stream) {
+                            int* dev_status, cudaStream_t stream) {
     const dim3 grid((unsigned)((k + 255) / 256), (unsigned)((rows + 127) / 128));
     if (scale_given) {
         quantize_kernel<false><<<grid, kQuantThreads, 0, stream>>>(x, rows, k, ld, codes, sf, tensor_scale,
@@ -253,7 +283,7 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t k, int64_t 
         return cudaGetLastError();
     }
     const int ag = amax_grid(rows, k);
-    amax_kernel<<<ag, kAmaxThreads, 0, stream>>>(x, rows, k, ld, partials);
+    amax_kernel<<<ag, kAmaxThreads, 0, stream>>>(x, rows, k, ld, partials, dev_status);
     // programmatic dependent launch: the quantize CTAs start loading X while
     // the amax grid finishes, and wait for it before reading its partials
     cudaLaunchConfig_t cfg = {};
@@ -270,6 +300,30 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t k, int64_t 
                                        (const float*)partials, ag);
     count_launch(2);
     if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ failure-detection check
+// One warp waits, through the bounded mbarrier wait of the GEMM and quantize
+// kernels, on a barrier nothing arrives at; the wait gives up after limit_ns
+// and reports NVFP4_ERR_TIMEOUT.
+__global__ void __launch_bounds__(32) debug_wait_kernel(int* dev_status, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_sh;
+    if (threadIdx.x == 0) {
+        abort_sh = 0;
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+    WaitCtx wc{&abort_sh, dev_status};
+    if (threadIdx.x == 0) mbar_wait_limit(&bar, 0, wc, limit_ns);
+    __syncwarp();
+}
+
+cudaError_t launch_debug_wait_timeout(int* dev_status, uint64_t limit_ns, cudaStream_t stream) {
+    debug_wait_kernel<<<1, 32, 0, stream>>>(dev_status, limit_ns);
+    count_launch(1);
     return cudaGetLastError();
 }
 

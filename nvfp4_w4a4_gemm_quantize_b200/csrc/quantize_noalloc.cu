@@ -53,6 +53,11 @@ static cudaError_t noalloc_scratch(float** out) {
 
 static bool noalloc_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+void reset_noalloc_cache() {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    for (auto& q : g_noalloc_ptr) q = nullptr;
+}
+
 }  // namespace nvfp4
 
 using namespace nvfp4;
@@ -60,7 +65,6 @@ using namespace nvfp4;
 extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x,
                                                uint8_t* codes, uint8_t* sf, float* tensor_scale, unsigned flags,
                                                int* dev_status, nvfp4_stream_t stream) {
-    (void)dev_status;
     if (rows < 0 || k <= 0 || ld_x < k) return NVFP4_ERR_INVALID_ARG;
     if ((flags & ~(unsigned)NVFP4_SCALE_GIVEN) != 0u) return NVFP4_ERR_INVALID_ARG;
     if (!tensor_scale) return NVFP4_ERR_INVALID_ARG;
@@ -89,6 +93,6 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows,
     float* partials = nullptr;
     if (!given && noalloc_scratch(&partials) != cudaSuccess) return NVFP4_ERR_CUDA;
     const cudaError_t e = launch_quantize(static_cast<const uint16_t*>(x_bf16), rows, k, ld_x, codes, sf,
-                                          tensor_scale, given, partials, s);
+                                          tensor_scale, given, partials, dev_status, s);
     return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }

@@ -12,7 +12,7 @@ from nvfp4_w4a4_gemm_quantize_b200 import _lib, build
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "nvfp4.h")
 
-OK, INVALID, SHAPE, MISALIGNED, DEVICE, CUDA, TIMEOUT, WORKSPACE = range(8)
+OK, INVALID, SHAPE, MISALIGNED, DEVICE, CUDA, TIMEOUT, WORKSPACE, NONFINITE = range(9)
 A = 0x10000          # fake, 16-byte aligned device addresses (never dereferenced)
 B = 0x20000
 C = 0x30000
@@ -32,7 +32,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 9, names
+    assert len(names) == 11, names
     for n in names:
         assert hasattr(L, n), n
         assert n in _lib.SIGNATURES, n
@@ -48,9 +48,23 @@ def test_sf_bytes_and_workspace(L):
 
 
 def test_status_strings(L):
-    for s in range(8):
+    for s in range(9):
         assert L.nvfp4_status_string(s)
+        assert b"unknown" not in L.nvfp4_status_string(s)
     assert b"unknown" in L.nvfp4_status_string(99)
+
+
+def test_debug_wait_rejects_bad_arguments(L):
+    w = L.nvfp4_debug_wait_timeout
+    assert w(None, 1000, None) == INVALID
+    assert w(A, 0, None) == INVALID
+    assert w(A, 2000001, None) == INVALID
+    assert w(A + 2, 1000, None) == MISALIGNED
+
+
+def test_shutdown_runs_without_a_device(L):
+    L.nvfp4_shutdown()
+    L.nvfp4_shutdown()
 
 
 def test_quantize_rejects_bad_arguments(L):
