@@ -76,8 +76,10 @@ enum { NVFP4_SCALE_GIVEN = 1 };
 size_t nvfp4_sf_bytes(int64_t rows, int64_t k);
 
 /* Bytes of device workspace nvfp4_quantize needs when it derives the tensor
- * scale from the data (no NVFP4_SCALE_GIVEN): one partial maximum per CTA of
- * the amax pass.  The contents need no initialisation and are not preserved. */
+ * scale from the data (no NVFP4_SCALE_GIVEN): per-CTA partial maxima, each
+ * tagged with a per-call number so that the contents need no initialisation
+ * (they are not preserved).  Calls that overlap on the GPU must not share a
+ * workspace. */
 size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t k);
 
 /*
@@ -99,8 +101,11 @@ size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t k);
  *               otherwise g is computed from the data and written there.
  * workspace     device scratch of >= nvfp4_quantize_workspace_bytes(rows, k)
  *               bytes, 16-byte aligned; unused (may be NULL) with SCALE_GIVEN.
- * Two kernels on `stream` (amax pass, then quantize) or one with SCALE_GIVEN.
- * rows == 0 is a no-op (g = 0 is written when not given).
+ * One kernel on `stream`: with a data-derived scale a persistent,
+ * co-resident grid reduces amax, hands it over grid-wide (a bounded wait) and
+ * quantizes; when the grid cannot be co-resident, two kernels (amax pass, then
+ * quantize) give the same result.  rows == 0 is a no-op (g = 0 is written when
+ * not given).
  */
 nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t rows, int64_t k, int64_t ld_x,
                             uint8_t *codes, uint8_t *sf, float *tensor_scale,

@@ -111,15 +111,25 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t
     if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(sf) || (ld_x % 8) != 0 ||
         (!given && !aligned16(workspace)) || (reinterpret_cast<uintptr_t>(tensor_scale) & 3u))
         return NVFP4_ERR_MISALIGNED;
-    nvfp4_status st = device_ok(nullptr);
+    int sms = 0;
+    nvfp4_status st = device_ok(&sms);
     if (st != NVFP4_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (rows == 0) {
         if (!given) return cuda_status(cudaMemsetAsync(tensor_scale, 0, sizeof(float), s));
         return NVFP4_OK;
     }
-    return cuda_status(launch_quantize(static_cast<const uint16_t*>(x_bf16), rows, k, ld_x, codes, sf, tensor_scale,
-                                       given, static_cast<float*>(workspace), dev_status, s));
+    const uint16_t* xb = static_cast<const uint16_t*>(x_bf16);
+    if (!given) {
+        // one kernel (amax and quantize with a grid-wide handoff); the
+        // two-kernel path when the grid cannot be co-resident
+        const cudaError_t e = launch_quantize_fused(xb, rows, k, ld_x, codes, sf, tensor_scale,
+                                                    static_cast<unsigned long long*>(workspace), kFusedSlots,
+                                                    dev_status, sms, s);
+        if (e != cudaErrorNotSupported) return cuda_status(e);
+    }
+    return cuda_status(launch_quantize(xb, rows, k, ld_x, codes, sf, tensor_scale, given, static_cast<float*>(workspace),
+                                       dev_status, s));
 }
 
 nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* sf, const float* tensor_scale, int64_t rows,

@@ -6,10 +6,12 @@
 
 namespace nvfp4 {
 
-constexpr int kAmaxThreads = 256;
+constexpr int kAmaxThreads = 512;
 constexpr int kAmaxMaxCtas = 256;        // partial maxima, one float each
 constexpr int kQuantThreads = 512;
-constexpr size_t kQuantWorkspaceBytes = kAmaxMaxCtas * sizeof(float);
+constexpr int kFusedSlots = 512;         // one-kernel quantize: (generation, max) per CTA
+constexpr size_t kQuantWorkspaceBytes = kFusedSlots * sizeof(unsigned long long);
+static_assert(kQuantWorkspaceBytes >= kAmaxMaxCtas * sizeof(float), "workspace holds the two-kernel partials too");
 
 void count_launch(int n);
 
@@ -18,6 +20,10 @@ int amax_grid(int64_t rows, int64_t k);
 cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes,
                             uint8_t* sf, float* tensor_scale, bool scale_given, float* partials,
                             int* dev_status, cudaStream_t stream);
+
+cudaError_t launch_quantize_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes,
+                                  uint8_t* sf, float* tensor_scale, unsigned long long* slots, int max_slots,
+                                  int* dev_status, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_debug_wait_timeout(int* dev_status, uint64_t limit_ns, cudaStream_t stream);
 

@@ -19,6 +19,8 @@
 // on packed FP32 pairs; where the two bounds give the same code it is the
 // code of the IEEE quotient, otherwise the values are divided exactly (see
 // quant_math.cuh).
+#include <atomic>
+
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -29,33 +31,27 @@
 namespace nvfp4 {
 
 // ------------------------------------------------------------------ amax
+// Largest magnitude of two packed bf16 pairs, per half, with NaN propagation
+// (a NaN operand gives NaN).  For the tensor amax: finite inputs give the
+// same maximum as any other order, and an Inf or NaN anywhere leaves a half
+// with the all-ones exponent, which flags the input as non-finite (the
+// contract's inputs are finite; the scale is then unspecified).
+__device__ __forceinline__ uint32_t absmax_nan_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 // Per-half largest magnitude of 8 bf16 values (sign bits not meaningful).
 __device__ __forceinline__ uint32_t absmax_bf16x8(uint4 a) {
-    return absmax_bf16x2(absmax_bf16x2(a.x, a.y), absmax_bf16x2(a.z, a.w));
-}
-
-// Per-half largest exponent field of 8 bf16 values (0xFF in a half: an Inf or
-// a NaN is among them).
-__device__ __forceinline__ uint32_t expmax_bf16x8(uint4 a) {
-    const uint32_t m = 0x7F807F80u;
-    uint32_t r, t;
-    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a.x & m), "r"(a.y & m));
-    asm("max.u16x2 %0, %1, %2;" : "=r"(t) : "r"(a.z & m), "r"(a.w & m));
-    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(r), "r"(t));
-    return r;
-}
-
-__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
-    uint32_t r;
-    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-    return r;
+    return absmax_nan_bf16x2(absmax_nan_bf16x2(a.x, a.y), absmax_nan_bf16x2(a.z, a.w));
 }
 
 // Partial max |x| per CTA over a [rows, k] bf16 tensor with row stride ld,
-// on bf16 pairs (max.xorsign.abs); NaNs are ignored when a number is beside
-// them, as in a max that skips unordered comparisons.  The final per-CTA
-// value compares non-negative bf16 patterns as integers (for non-negative
-// IEEE values the order of the patterns is the order of the values).
+// on bf16 pairs (max.NaN.xorsign.abs).  The final per-CTA value compares
+// non-negative bf16 patterns as integers (for non-negative IEEE values the
+// order of the patterns is the order of the values); a value with the
+// all-ones exponent means an Inf or NaN was read.
 __global__ void __launch_bounds__(kAmaxThreads)
 amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
             float* __restrict__ partials, int* __restrict__ dev_status) {
@@ -66,36 +62,27 @@ amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
     const int64_t nvec = rows * k8;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     uint32_t m = 0;                                   // two bf16 |x| maxima
-    uint32_t e = 0;                                   // two exponent-field maxima
     int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (ld == k) {
         const uint4* p = reinterpret_cast<const uint4*>(x);
         for (; v + 3 * stride < nvec; v += 4 * stride) {
             const uint4 a = __ldg(p + v), b = __ldg(p + v + stride);
             const uint4 c = __ldg(p + v + 2 * stride), d = __ldg(p + v + 3 * stride);
-            m = absmax_bf16x2(m, absmax_bf16x2(absmax_bf16x8(a), absmax_bf16x8(b)));
-            m = absmax_bf16x2(m, absmax_bf16x2(absmax_bf16x8(c), absmax_bf16x8(d)));
-            e = max_u16x2(e, max_u16x2(max_u16x2(expmax_bf16x8(a), expmax_bf16x8(b)),
-                                       max_u16x2(expmax_bf16x8(c), expmax_bf16x8(d))));
+            m = absmax_nan_bf16x2(m, absmax_nan_bf16x2(absmax_bf16x8(a), absmax_bf16x8(b)));
+            m = absmax_nan_bf16x2(m, absmax_nan_bf16x2(absmax_bf16x8(c), absmax_bf16x8(d)));
         }
-        for (; v < nvec; v += stride) {
-            const uint4 a = __ldg(p + v);
-            m = absmax_bf16x2(m, absmax_bf16x8(a));
-            e = max_u16x2(e, expmax_bf16x8(a));
-        }
+        for (; v < nvec; v += stride) m = absmax_nan_bf16x2(m, absmax_bf16x8(__ldg(p + v)));
     } else {
         for (; v < nvec; v += stride) {
             const int64_t r = v / k8, c = v - r * k8;
-            const uint4 a = __ldg(reinterpret_cast<const uint4*>(x + r * ld) + c);
-            m = absmax_bf16x2(m, absmax_bf16x8(a));
-            e = max_u16x2(e, expmax_bf16x8(a));
+            m = absmax_nan_bf16x2(m, absmax_bf16x8(__ldg(reinterpret_cast<const uint4*>(x + r * ld) + c)));
         }
     }
+    m &= 0x7FFF7FFFu;
     // any Inf or NaN: flag it (the first error written stays)
-    const bool nonfinite = (e & 0xFFFFu) == 0x7F80u || (e >> 16) == 0x7F80u;
+    const bool nonfinite = (m & 0xFFFFu) >= 0x7F80u || (m >> 16) >= 0x7F80u;
     if (__syncthreads_or(nonfinite ? 1 : 0) && threadIdx.x == 0 && dev_status)
         atomicCAS(dev_status, 0, (int)NVFP4_ERR_NONFINITE);
-    m &= 0x7FFF7FFFu;
     uint32_t h = max(m & 0xFFFFu, m >> 16);
     for (int o = 16; o > 0; o >>= 1) h = max(h, __shfl_xor_sync(0xffffffffu, h, o));
     __shared__ uint32_t red[kAmaxThreads / 32];
@@ -109,61 +96,115 @@ amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
 }
 
 // ------------------------------------------------------------------ quantize
-// One CTA quantizes a 128-row x 256-column tile (four 512-byte scale atoms).
-// Warp w owns rows 8w .. 8w+7, two rows per step: lanes 0-15 one row, lanes
-// 16-31 the next, lane l owning the 16-value block l % 16 of its row (two
-// 16-byte loads; a row is one coalesced 512-byte span).  A lane therefore
-// holds a whole block: its maximum, scale and reciprocal are computed once
-// per 16 values without any shuffle.  All loads of a warp are issued before
-// any is used.
-template <bool kDynamic>
-__global__ void __launch_bounds__(kQuantThreads)
-quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
-                uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
-                float* __restrict__ tensor_scale, const float* __restrict__ partials, int nparts) {
-    // four 512-byte atoms, each padded by 4 bytes so that the eight words two
-    // rows write (one per atom and row) fall in different banks
-    constexpr int kAtomPitch = 516;
-    __shared__ __align__(16) uint8_t sf_stage[4 * kAtomPitch];
-    __shared__ ScaleConsts sc_sh;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// A tile is 128 rows x 256 columns (four 512-byte scale atoms) handled by one
+// 512-thread CTA.  Warp w owns rows 8w .. 8w+7, two rows per step: lanes 0-15
+// one row, lanes 16-31 the next, lane l owning the 16-value block l % 16 of
+// its row (two 16-byte loads; a row is one coalesced 512-byte span).  A lane
+// therefore holds a whole block: its maximum, scale and reciprocal are
+// computed once per 16 values without any shuffle.
+constexpr int kTileRows = 128;
+constexpr int kTileCols = 256;
+constexpr int kRows = kTileRows / (kQuantThreads / 32);   // rows per warp
+constexpr int kSteps = kRows / 2;
+// four 512-byte atoms, each padded by 4 bytes so that the eight words two
+// rows write (one per atom and row) fall in different banks
+constexpr int kAtomPitch = 516;
 
-    // row blocks in reverse launch order: the amax pass read the tensor front
-    // to back, so its tail is the part still in L2 when the first CTAs start
-    const int64_t rblk = (int64_t)(gridDim.y - 1 - blockIdx.y);
-    const int64_t row0 = rblk * 128;
-    const int64_t c0 = (int64_t)blockIdx.x * 256;
-    const int ncols = (k - c0) < 256 ? (int)(k - c0) : 256;   // multiple of 64
-    const int half = lane >> 4;                   // which row of the pair
-    const int blk = lane & 15;                    // 16-value block inside the tile row
-    const bool col_ok = blk * 16 < ncols;
-    const int64_t kh = k >> 1;
+// Per-lane view of one tile: step i handles row rt0 + 2i of the tile; the
+// pointers are for step 0 and advance by two rows per step (ld and kh are
+// multiples of 8 and 32).
+struct TileLane {
+    const uint4* xp;
+    uint2* cp;
+    int64_t xstep, cstep, rows_left;
+    int sbase;
+    bool col_ok;
+};
 
-    constexpr int kRows = 128 / (kQuantThreads / 32);   // rows per warp
-    constexpr int kSteps = kRows / 2;
-    // step i handles row rt0 + 2i of the tile; pointers for step 0, advanced
-    // by two rows per step (ld and kh are multiples of 8 and 32)
+__device__ __forceinline__ TileLane tile_lane(const uint16_t* x, uint8_t* codes, int64_t rows, int64_t k, int64_t ld,
+                                              int64_t rblk, int64_t cblk, int warp, int lane) {
+    TileLane t;
+    const int64_t c0 = cblk * kTileCols;
+    const int ncols = (k - c0) < kTileCols ? (int)(k - c0) : kTileCols;   // multiple of 64
+    const int half = lane >> 4, blk = lane & 15;
     const int rt0 = warp * kRows + half;
-    const int64_t r0 = row0 + rt0;
-    const int64_t rows_left = rows - r0;          // step i is in range iff 2i < rows_left
-    const uint4* xp = reinterpret_cast<const uint4*>(x + r0 * ld + c0) + 2 * blk;
-    const int64_t xstep = ld >> 2;                // two rows, in 16-byte units
-    uint2* cp = reinterpret_cast<uint2*>(codes + r0 * kh + (c0 >> 1)) + blk;
-    const int64_t cstep = kh >> 2;                // two rows, in 8-byte units
+    const int64_t r0 = rblk * kTileRows + rt0;
+    const int64_t kh = k >> 1;
+    t.col_ok = blk * 16 < ncols;
+    t.rows_left = rows - r0;                      // step i is in range iff 2i < rows_left
+    t.xp = reinterpret_cast<const uint4*>(x + r0 * ld + c0) + 2 * blk;
+    t.xstep = ld >> 2;                            // two rows, in 16-byte units
+    t.cp = reinterpret_cast<uint2*>(codes + r0 * kh + (c0 >> 1)) + blk;
+    t.cstep = kh >> 2;                            // two rows, in 8-byte units
     // block blk of row rt: atom blk / 4, byte blk % 4 of the row's word
-    const int sbase = (blk >> 2) * kAtomPitch + (rt0 & 31) * 16 + (rt0 >> 5) * 4 + (blk & 3);
+    t.sbase = (blk >> 2) * kAtomPitch + (rt0 & 31) * 16 + (rt0 >> 5) * 4 + (blk & 3);
+    return t;
+}
 
-    uint4 v[2 * kSteps];
+// All loads of a lane for one tile (rows beyond the tensor and columns beyond
+// k read as zeros).
+__device__ __forceinline__ void load_tile(const TileLane& t, uint4 (&v)[2 * kSteps]) {
 #pragma unroll
     for (int i = 0; i < kSteps; ++i) {
-        if (2 * i < rows_left && col_ok) {
-            v[2 * i] = __ldcs(xp + i * xstep);
-            v[2 * i + 1] = __ldcs(xp + i * xstep + 1);
+        if (2 * i < t.rows_left && t.col_ok) {
+            v[2 * i] = __ldcs(t.xp + i * t.xstep);
+            v[2 * i + 1] = __ldcs(t.xp + i * t.xstep + 1);
         } else {
             v[2 * i] = make_uint4(0u, 0u, 0u, 0u);
             v[2 * i + 1] = make_uint4(0u, 0u, 0u, 0u);
         }
     }
+}
+
+// Quantize a lane's loaded blocks: codes straight to global memory, scale
+// bytes to the CTA's staging atoms.
+__device__ __forceinline__ void quantize_lane(const TileLane& t, const uint4 (&v)[2 * kSteps], const ScaleConsts& sc,
+                                              uint8_t* sf_stage) {
+#pragma unroll
+    for (int i = 0; i < kSteps; ++i) {
+        const uint32_t w[8] = {v[2 * i].x, v[2 * i].y, v[2 * i].z, v[2 * i].w,
+                               v[2 * i + 1].x, v[2 * i + 1].y, v[2 * i + 1].z, v[2 * i + 1].w};
+        const float ab = __uint_as_float(block_absmax16(w) << 16);      // block amax
+        const uint32_t sfc = block_scale_code(ab, sc);
+        const float s = __fmul_rn(e4m3_to_f32(sfc), sc.g);
+        const uint32_t lo = quantize8_bf16(w[0], w[1], w[2], w[3], s);
+        const uint32_t hi = quantize8_bf16(w[4], w[5], w[6], w[7], s);
+        if (2 * i < t.rows_left && t.col_ok) t.cp[i * t.cstep] = make_uint2(lo, hi);
+        if (t.col_ok) sf_stage[t.sbase + 32 * i] = (uint8_t)sfc;
+    }
+}
+
+// Copy a tile's staged scale atoms (consecutive in the scale buffer) out, one
+// word per thread.  The caller synchronizes the CTA before and after.
+__device__ __forceinline__ void store_tile_scales(const uint8_t* sf_stage, uint8_t* sf, int64_t k, int64_t rblk,
+                                                  int64_t cblk) {
+    static_assert(4 * 128 <= kQuantThreads, "scale copy-out: one word per thread");
+    const int64_t c0 = cblk * kTileCols;
+    const int ncols = (k - c0) < kTileCols ? (int)(k - c0) : kTileCols;
+    const int natoms = ncols >> 6;
+    const int64_t kb4 = k >> 6;                   // atoms per 128-row block
+    uint32_t* dst = reinterpret_cast<uint32_t*>(sf + ((rblk * kb4 + cblk * 4) << 9));
+    const int i = threadIdx.x;
+    if (i < natoms * 128) dst[i] = *reinterpret_cast<const uint32_t*>(sf_stage + (i >> 7) * kAtomPitch + (i & 127) * 4);
+}
+
+// Two-kernel form: one CTA per tile, after the amax pass (or with a given
+// tensor scale).
+template <bool kDynamic>
+__global__ void __launch_bounds__(kQuantThreads)
+quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
+                uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                float* __restrict__ tensor_scale, const float* __restrict__ partials, int nparts) {
+    __shared__ __align__(16) uint8_t sf_stage[4 * kAtomPitch];
+    __shared__ ScaleConsts sc_sh;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // row blocks in reverse launch order: the amax pass read the tensor front
+    // to back, so its tail is the part still in L2 when the first CTAs start
+    const int64_t rblk = (int64_t)(gridDim.y - 1 - blockIdx.y);
+    const int64_t cblk = blockIdx.x;
+    const TileLane t = tile_lane(x, codes, rows, k, ld, rblk, cblk, warp, lane);
+    uint4 v[2 * kSteps];
+    load_tile(t, v);
 
     // the tensor scale and its block-scale constants, once per CTA, after the
     // amax grid (when launched as its programmatic dependent) has completed
@@ -182,29 +223,103 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
         if (lane == 0) sc_sh = scale_consts(g);
     }
     __syncthreads();
-    const ScaleConsts sc = sc_sh;
-    const float g = sc.g;
+    quantize_lane(t, v, sc_sh, sf_stage);
+    __syncthreads();
+    store_tile_scales(sf_stage, sf, k, rblk, cblk);
+}
 
+// One-kernel form with a data-derived tensor scale: a persistent grid whose
+// CTAs all stay resident (cooperative launch) takes the tiles t = blockIdx.x,
+// blockIdx.x + gridDim.x, ...  Phase 1 reduces |x| over the CTA's tiles and
+// publishes (generation, partial max) in the CTA's slot; every CTA then waits
+// (bounded) until all slots carry this call's generation -- the generation is
+// a per-call number from the host, so the slots need no initialisation -- and
+// takes the maximum itself.  Phase 2 quantizes the same tiles in reverse
+// order, so the first ones re-read what phase 1 read last, still in L2.
+__global__ void __launch_bounds__(kQuantThreads)
+quantize_fused_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
+                      uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ tensor_scale,
+                      unsigned long long* __restrict__ slots, uint32_t gen, int ntiles_c, int ntiles,
+                      int* __restrict__ dev_status) {
+    __shared__ __align__(16) uint8_t sf_stage[4 * kAtomPitch];
+    __shared__ ScaleConsts sc_sh;
+    __shared__ uint32_t red[kQuantThreads / 32];
+    __shared__ int ok_sh;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // ---- phase 1: |x| maximum (and the largest exponent field) of this CTA's tiles
+    uint32_t m = 0u;
+    for (int tt = blockIdx.x; tt < ntiles; tt += gridDim.x) {
+        const TileLane t = tile_lane(x, codes, rows, k, ld, tt / ntiles_c, tt % ntiles_c, warp, lane);
+        uint4 v[2 * kSteps];
 #pragma unroll
-    for (int i = 0; i < kSteps; ++i) {
-        const uint32_t w[8] = {v[2 * i].x, v[2 * i].y, v[2 * i].z, v[2 * i].w,
-                               v[2 * i + 1].x, v[2 * i + 1].y, v[2 * i + 1].z, v[2 * i + 1].w};
-        const float ab = __uint_as_float(block_absmax16(w) << 16);      // block amax
-        const uint32_t sfc = block_scale_code(ab, sc);
-        const float s = __fmul_rn(e4m3_to_f32(sfc), g);
-        const uint32_t lo = quantize8_bf16(w[0], w[1], w[2], w[3], s);
-        const uint32_t hi = quantize8_bf16(w[4], w[5], w[6], w[7], s);
-        if (2 * i < rows_left && col_ok) cp[i * cstep] = make_uint2(lo, hi);
-        if (col_ok) sf_stage[sbase + 32 * i] = (uint8_t)sfc;
+        for (int i = 0; i < kSteps; ++i) {
+            if (2 * i < t.rows_left && t.col_ok) {
+                v[2 * i] = __ldg(t.xp + i * t.xstep);
+                v[2 * i + 1] = __ldg(t.xp + i * t.xstep + 1);
+            } else {
+                v[2 * i] = make_uint4(0u, 0u, 0u, 0u);
+                v[2 * i + 1] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 2 * kSteps; ++i) m = absmax_nan_bf16x2(m, absmax_bf16x8(v[i]));
+    }
+    m &= 0x7FFF7FFFu;
+    uint32_t h = max(m & 0xFFFFu, m >> 16);
+    for (int o = 16; o > 0; o >>= 1) h = max(h, __shfl_xor_sync(0xffffffffu, h, o));
+    if (lane == 0) red[warp] = h;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t tm = lane < kQuantThreads / 32 ? red[lane] : 0u;
+        for (int o = 16; o > 0; o >>= 1) tm = max(tm, __shfl_xor_sync(0xffffffffu, tm, o));
+        if (lane == 0) {
+            if (tm >= 0x7F80u && dev_status) atomicCAS(dev_status, 0, (int)NVFP4_ERR_NONFINITE);
+            const unsigned long long word = ((unsigned long long)gen << 32) | (unsigned long long)(tm << 16);
+            asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(slots + blockIdx.x), "l"(word) : "memory");
+        }
+        // ---- every CTA's slot carries this generation: the tensor maximum
+        float mx = 0.0f;
+        bool ok = true;
+        const uint64_t t0 = globaltimer_ns();
+        for (int i = lane; i < (int)gridDim.x; i += 32) {
+            unsigned long long w;
+            uint32_t n = 0;
+            while (true) {
+                asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(slots + i) : "memory");
+                if ((uint32_t)(w >> 32) == gen) break;
+                if ((++n & 63u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) { ok = false; break; }
+            }
+            if (!ok) break;
+            mx = fmaxf(mx, __uint_as_float((uint32_t)w));
+        }
+        ok = __all_sync(0xffffffffu, ok ? 1 : 0) != 0;
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) {
+            if (!ok && dev_status) atomicExch(dev_status, (int)NVFP4_ERR_TIMEOUT);
+            const float g = __fdiv_rn(mx, 2688.0f);
+            if (blockIdx.x == 0 && ok) *tensor_scale = g;
+            sc_sh = scale_consts(g);
+            ok_sh = ok ? 1 : 0;
+        }
     }
     __syncthreads();
-    // this tile's atoms are consecutive in the scale buffer: one word per thread
-    static_assert(4 * 128 <= kQuantThreads, "scale copy-out: one word per thread");
-    const int natoms = ncols >> 6;
-    const int64_t kb4 = k >> 6;                       // atoms per 128-row block
-    uint32_t* dst = reinterpret_cast<uint32_t*>(sf + ((rblk * kb4 + blockIdx.x * 4) << 9));
-    const int i = threadIdx.x;
-    if (i < natoms * 128) dst[i] = *reinterpret_cast<const uint32_t*>(sf_stage + (i >> 7) * kAtomPitch + (i & 127) * 4);
+    if (!ok_sh) return;                           // gave up waiting: outputs unspecified
+    const ScaleConsts sc = sc_sh;
+
+    // ---- phase 2: quantize the same tiles, last first
+    const int nmine = ntiles > (int)blockIdx.x ? (ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    for (int j = nmine - 1; j >= 0; --j) {
+        const int tt = (int)blockIdx.x + j * (int)gridDim.x;
+        const int64_t rblk = tt / ntiles_c, cblk = tt % ntiles_c;
+        const TileLane t = tile_lane(x, codes, rows, k, ld, rblk, cblk, warp, lane);
+        uint4 v[2 * kSteps];
+        load_tile(t, v);
+        quantize_lane(t, v, sc, sf_stage);
+        __syncthreads();
+        store_tile_scales(sf_stage, sf, k, rblk, cblk);
+        __syncthreads();
+    }
 }
 
 // ------------------------------------------------------------------ dequantize
@@ -300,6 +415,47 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t k, int64_t 
                                        (const float*)partials, ag);
     count_launch(2);
     if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+// One-kernel dynamic quantization (see quantize_fused_kernel).  Returns
+// cudaErrorNotSupported when the grid cannot be co-resident (the caller then
+// takes the two-kernel path, which computes the same codes).
+cudaError_t launch_quantize_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes,
+                                  uint8_t* sf, float* tensor_scale, unsigned long long* slots, int max_slots,
+                                  int* dev_status, int num_sms, cudaStream_t stream) {
+    static std::atomic<uint32_t> generation{0};
+    const int ntiles_c = (int)((k + kTileCols - 1) / kTileCols);
+    const int64_t ntiles64 = ((rows + kTileRows - 1) / kTileRows) * ntiles_c;
+    if (ntiles64 > (int64_t)1 << 30) return cudaErrorNotSupported;
+    const int ntiles = (int)ntiles64;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_fused_kernel, kQuantThreads, 0);
+    if (e != cudaSuccess) return e;
+    int grid = per_sm * num_sms;
+    if (grid > max_slots) grid = max_slots;
+    if (grid > ntiles) grid = ntiles;
+    if (grid < 1) return cudaErrorNotSupported;
+    uint32_t gen = generation.fetch_add(1u) + 1u;
+    if (gen == 0u) gen = generation.fetch_add(1u) + 1u;     // 0 never marks a slot
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;           // every CTA resident at once
+    attr[0].val.cooperative = 1;
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kQuantThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, quantize_fused_kernel, x, rows, k, ld, codes, sf, tensor_scale, slots, gen,
+                           ntiles_c, ntiles, dev_status);
+    if (e == cudaErrorCooperativeLaunchTooLarge) {
+        (void)cudaGetLastError();
+        return cudaErrorNotSupported;
+    }
+    if (e != cudaSuccess) return e;
+    count_launch(1);
     return cudaGetLastError();
 }
 
