@@ -350,10 +350,18 @@ def run_ours(args):
     dev_ms = t0.elapsed_time(t1)
     max_ms = max_over_ranks(dev_ms, world, dev)
 
-    gemm_ms = [sum(s.elapsed_time(e) for s, e in (gemm_ev[i][li] for i in range(args.steps))) / args.steps
-               for li in range(len(wl.layers))]
-    quant_ms = [sum(s.elapsed_time(e) for s, e in (quant_ev[i][li] for i in range(args.steps))) / args.steps
+    gemm_all = [[gemm_ev[i][li][0].elapsed_time(gemm_ev[i][li][1]) for i in range(args.steps)]
                 for li in range(len(wl.layers))]
+    quant_all = [[quant_ev[i][li][0].elapsed_time(quant_ev[i][li][1]) for i in range(args.steps)]
+                 for li in range(len(wl.layers))]
+    gemm_ms = [sum(v) / len(v) for v in gemm_all]
+    quant_ms = [sum(v) / len(v) for v in quant_all]
+
+    def pct(v):
+        """p10 / median / p90 of per-step times (ms)."""
+        q = sorted(v)
+        at = lambda f: q[min(len(q) - 1, int(round(f * (len(q) - 1))))]
+        return [round(at(0.1), 4), round(at(0.5), 4), round(at(0.9), 4)]
 
     # ---- end to end through the public API with host buffers
     xh = [x.cpu().pin_memory() for x in xs]
@@ -408,7 +416,9 @@ def run_ours(args):
         q_traffic = profiled_traffic("quantize_fc2_32768x12288.txt") if full else None
         per_layer = {l.name: {"gemm_ms": round(gemm_ms[j], 4),
                               "gemm_tflops": round(2 * l.M * l.N * l.K / (gemm_ms[j] * 1e-3) / 1e12, 1),
-                              "quant_ms": round(quant_ms[j], 4), "quant_gbs": round(q_gbs[j], 1)}
+                              "gemm_ms_p10_p50_p90": pct(gemm_all[j]),
+                              "quant_ms": round(quant_ms[j], 4), "quant_gbs": round(q_gbs[j], 1),
+                              "quant_ms_p10_p50_p90": pct(quant_all[j])}
                      for j, l in enumerate(wl.layers)}
         value = world * args.steps * gemm_flops / (max_ms * 1e-3) / 1e12
         line = {
