@@ -19,19 +19,21 @@
 //              LEADER's full barrier (cta_group::2), which the leader arms
 //              with the bytes of both CTAs: one wait per stage tells the MMA
 //              issuer that both CTAs' operands have landed.
-//   warp 1     leader CTA: MMA issuer.  Per K=64 step three tcgen05.cp of
-//              the scale atoms into the stage's TMEM columns, then one
-//              tcgen05.mma cta_group::2; one commit per stage, multicast to
-//              both CTAs' "empty" barriers.
+//   warp 2     leader CTA: scale copier.  Per K=64 step three tcgen05.cp of
+//              the scale atoms into the stage's TMEM columns; one commit per
+//              stage to the leader's "scaled" barrier.
+//   warp 1     leader CTA: MMA issuer.  Per K=64 step one tcgen05.mma
+//              cta_group::2; one commit per stage, multicast to both CTAs'
+//              "empty" barriers.
 //   warps 8-15 epilogue, both CTAs: the 128 x 256 FP32 accumulator slice is
 //              read into registers (two warps per TMEM lane quarter, 128
 //              columns each) and released to the MMA issuer at once, then
 //              converted and stored while the next tile's mainloop runs.
-// Producer and MMA issuer run on whole warps with one elected lane issuing:
-// the descriptors, coordinates and addresses then stay warp-uniform.  Issued
-// from a single lane, the same copies and MMAs took longer to issue than to
-// execute (the copies looked expensive; in a warp-uniform loop twelve copies
-// and four MMAs per stage issue in the MMAs' own 515 cycles).
+// Producer, copier and MMA issuer run on whole warps with one elected lane
+// issuing: the descriptors, coordinates and addresses then stay warp-uniform.
+// Issued from a single lane, the same copies and MMAs took longer to issue
+// than to execute; on one warp the twelve copies still cost the MMA loop ~90
+// cycles per stage (~626 against ~533), hence the separate copier.
 // The cross-CTA release of the accumulator is a relaxed arrive ordered by
 // tcgen05.wait::ld and tcgen05.fence::before_thread_sync (a cluster-scope
 // release costs about a microsecond per arrive).
@@ -140,14 +142,20 @@ __device__ __forceinline__ void store_chunk(const uint32_t* r, float alpha, uint
     }
 }
 
-// One K=64 step of the pair: copy the step's scale atoms (A: 128 rows of this
-// CTA, B: all 256 rows, in both CTAs) into TMEM, then the block-scaled MMA.
-__device__ __forceinline__ void k_step(uint32_t tmem_acc, uint32_t sb, uint32_t sfs, uint32_t sf_col, int ks,
-                                       uint32_t idesc, bool accumulate) {
+// Scale atoms of one K=64 step of the pair (A: 128 rows of this CTA, B: all
+// 256 rows, in both CTAs) into the step's TMEM columns.
+__device__ __forceinline__ void k_copy_scales(uint32_t sfs, uint32_t sf_col, int ks) {
     const uint32_t col = sf_col + ks * SF_COLS_STEP;
     tc_cp2_32x128b_warpx4(col, sdesc_sf(sfs + ks * SF_ATOM));
     tc_cp2_32x128b_warpx4(col + 4, sdesc_sf(sfs + SFA_BYTES + ks * SF_ATOM));
     tc_cp2_32x128b_warpx4(col + 8, sdesc_sf(sfs + SFA_BYTES + 4 * SF_ATOM + ks * SF_ATOM));
+}
+
+// One K=64 step of the pair: the block-scaled MMA reading the step's scale
+// columns.
+__device__ __forceinline__ void k_mma(uint32_t tmem_acc, uint32_t sb, uint32_t sf_col, int ks, uint32_t idesc,
+                                      bool accumulate) {
+    const uint32_t col = sf_col + ks * SF_COLS_STEP;
     tc_mma2_nvf4(tmem_acc, sdesc_kmajor_sw128(sb + ks * 32), sdesc_kmajor_sw128(sb + A_BYTES + ks * 32), idesc, col,
                  col + 4, accumulate ? 1u : 0u);
 }
@@ -160,10 +168,11 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     using C = Cfg<OUT>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
-    // full:  the leader's; both CTAs' operand tiles and scale atoms of a stage
-    //        have landed (the peer's loads signal it through cta_group::2);
-    // empty: both CTAs'; the MMAs of a stage have completed.
-    __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES];
+    // full:   the leader's; both CTAs' operand tiles and scale atoms of a stage
+    //         have landed (the peer's loads signal it through cta_group::2);
+    // scaled: the leader's; the stage's scale atoms are in both CTAs' TMEM;
+    // empty:  both CTAs'; the MMAs of a stage have completed.
+    __shared__ __align__(8) uint64_t full_bar[STAGES], scaled_bar[STAGES], empty_bar[STAGES];
     __shared__ __align__(8) uint64_t accf_bar, acce_bar, drain_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
@@ -179,6 +188,7 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
         abort_sh = 0;
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full_bar[s], 1);
+            mbar_init(&scaled_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
         }
         mbar_init(&accf_bar, 1);
@@ -263,14 +273,46 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                 for (int s = 0; s < STAGES; ++s)
                     if (issued_any & (1u << s)) mbar_wait(&full_bar[s], (issued >> s) & 1u, w2);
             }
+        } else if (warp == 2) {
+            if (rank == 0) {
+                // -------------------------------------------------------- scale copier (leader)
+                // Per stage: wait for the operands, copy the stage's scale atoms of
+                // both CTAs into TMEM, commit to the stage's "scaled" barrier.
+                // (From the MMA warp the twelve copies per stage cost issue slots
+                // that the four MMAs need: ~626 cycles per stage against ~533.)
+                const uint32_t smem0 = smem_u32(smem);
+                int stage = 0;
+                uint32_t phase = 0;
+                bool ok = true;
+                for (int t = pair; t < p.num_tiles && ok; t += npairs) {
+                    for (int kt = 0; kt < num_kt; ++kt) {
+                        if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[stage], phase, wc) ? 1 : 0)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t sfs = smem0 + stage * STAGE_BYTES + A_BYTES + B_BYTES;
+                        const uint32_t sf_col = sf_base + stage * SF_COLS_STAGE;
+                        const int nks = k_atoms - kt * 4;
+                        if (elect_one()) {
+                            if (nks >= 4) {
+#pragma unroll
+                                for (int ks = 0; ks < 4; ++ks) k_copy_scales(sfs, sf_col, ks);
+                            } else {
+                                for (int ks = 0; ks < nks; ++ks) k_copy_scales(sfs, sf_col, ks);
+                            }
+                            tc_commit2_mc(&scaled_bar[stage], 0x1);
+                        }
+                        __syncwarp();
+                        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                    }
+                }
+            }
         } else if (warp == 1) {
             if (rank == 0) {
                 // -------------------------------------------------------- MMA issuer (leader)
                 // The whole warp runs the loop so that descriptors and addresses
-                // stay warp-uniform; one elected lane issues.  Per K=64 step: three
-                // scale copies (this CTA's 128 A rows, the 256 B rows) from shared
-                // memory into the TMEM slot of the stage, then the MMA; copies and
-                // MMAs of one thread execute in issue order.
+                // stay warp-uniform; one elected lane issues four MMAs per stage.
                 constexpr uint32_t idesc = idesc_nvf4(256, 256);
                 const uint32_t smem0 = smem_u32(smem);
                 int stage = 0;
@@ -283,23 +325,21 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                     }
                     tc_fence_after();
                     for (int kt = 0; kt < num_kt; ++kt) {
-                        if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[stage], phase, wc) ? 1 : 0)) {
+                        // operands landed and the stage's scales are in TMEM
+                        if (!__all_sync(0xffffffffu, mbar_wait(&scaled_bar[stage], phase, wc) ? 1 : 0)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                         const uint32_t sb = smem0 + stage * STAGE_BYTES;
-                        const uint32_t sfs = sb + A_BYTES + B_BYTES;
                         const uint32_t sf_col = sf_base + stage * SF_COLS_STAGE;
                         const int nks = k_atoms - kt * 4;
                         if (elect_one()) {
                             if (nks >= 4) {
     #pragma unroll
-                                for (int ks = 0; ks < 4; ++ks)
-                                    k_step(tmem_base, sb, sfs, sf_col, ks, idesc, (kt | ks) != 0);
+                                for (int ks = 0; ks < 4; ++ks) k_mma(tmem_base, sb, sf_col, ks, idesc, (kt | ks) != 0);
                             } else {
-                                for (int ks = 0; ks < nks; ++ks)
-                                    k_step(tmem_base, sb, sfs, sf_col, ks, idesc, (kt | ks) != 0);
+                                for (int ks = 0; ks < nks; ++ks) k_mma(tmem_base, sb, sf_col, ks, idesc, (kt | ks) != 0);
                             }
                             tc_commit2_mc(&empty_bar[stage], 0x3);
                         }
