@@ -369,12 +369,32 @@ def run_ours(args):
     h2d = sum(x.numel() * x.element_size() for x in xh)
     d2h = sum(y.numel() * y.element_size() for y in yh)
 
+    # copies in and out run on their own streams (PCIe is full duplex), layer
+    # by layer, so the inputs of the next layer and the outputs of the last one
+    # move while a layer computes; events keep each buffer's reuse in order
+    nl = len(wl.layers)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(nl)]      # X landed on the device
+    ev_used = [torch.cuda.Event() for _ in range(nl)]    # X read by the quantize kernel
+    ev_done = [torch.cuda.Event() for _ in range(nl)]    # Y computed
+    ev_out = [torch.cuda.Event() for _ in range(nl)]     # Y copied to the host
+
     def e2e_step():
-        for li in range(len(wl.layers)):
-            xs[li].copy_(xh[li], non_blocking=True)
+        for li in range(nl):
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev_used[li])
+                xs[li].copy_(xh[li], non_blocking=True)
+                ev_in[li].record(s_in)
+            stream.wait_event(ev_in[li])
             nv.quantize(xs[li], out=Aq[li], workspace=ws)
+            ev_used[li].record(stream)
+            stream.wait_event(ev_out[li])
             nv.gemm_w4a4(Aq[li], Ws[li], out=Ys[li])
-            yh[li].copy_(Ys[li], non_blocking=True)
+            ev_done[li].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[li])
+                yh[li].copy_(Ys[li], non_blocking=True)
+                ev_out[li].record(s_out)
 
     e2e_steps = max(1, min(args.steps, 5))
     e2e_step()
@@ -382,8 +402,12 @@ def run_ours(args):
     barrier(world)
     e0, e1 = ev(), ev()
     e0.record(stream)
+    s_in.wait_stream(stream)
+    s_out.wait_stream(stream)
     for _ in range(e2e_steps):
         e2e_step()
+    stream.wait_stream(s_in)
+    stream.wait_stream(s_out)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
