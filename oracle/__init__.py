@@ -22,6 +22,11 @@ Parity status per function:
       products, round-trip of grid-valued blocks)
   gemm_w4a4 / gemm_w4a16                                -- pinned (one-hot
       products, float64 library matmul of the dequantized operands)
+  fake_quantize                                         -- pinned (brute force
+      on tiny inputs, idempotence under a fixed tensor scale, the closed form
+      of saturating elements)
+  ste_backward                                          -- pinned (closed form
+      through numpy's bit unpacking)
 """
 from __future__ import annotations
 
@@ -78,6 +83,10 @@ def lib() -> ctypes.CDLL:
         L.oracle_gemm_w4a16_rows.restype = None
         L.oracle_gemm_w4a16_at.argtypes = [_p, _p, _p, _f32, _i64, _i64, _i64]
         L.oracle_gemm_w4a16_at.restype = ctypes.c_double
+        L.oracle_fake_quantize_bf16.argtypes = [_p, _i64, _i64, _i64, ctypes.c_int, _p, ctypes.c_int, _p, _p]
+        L.oracle_fake_quantize_bf16.restype = None
+        L.oracle_ste_backward.argtypes = [_p, _p, _i64, _i64, ctypes.c_int, _p]
+        L.oracle_ste_backward.restype = None
         _LIB = L
     return _LIB
 
@@ -254,3 +263,40 @@ def tensor_scale(x) -> np.float32:
     xb = bf16_bits(x)
     rows, k = xb.shape
     return np.float32(L.oracle_tensor_scale_bf16(_ptr(xb), rows, k, k))
+
+
+# ---------------------------------------------------------------- QAT
+def fake_quantize(x, scale: float | None = None, out: str = "bf16", mask: bool = True):
+    """Fake quantization for QAT (NVFP4-DiT README, Definition III.1, and
+    Methodology 2's straight-through estimator): y = e2m1(code) * dec(sf) * g
+    rounded once to bf16 (uint16 bits) or f32, with the codes and scales of
+    ``quantize``; the clip mask marks s > 0 and |x| > 6 s, packed 8 elements
+    per byte (element j of a row: bit j % 8 of byte j / 8).  Returns
+    (y, mask or None, g)."""
+    L = lib()
+    xb = bf16_bits(x)
+    rows, k = xb.shape
+    assert k % 64 == 0
+    y = np.empty((rows, k), np.float32 if out == "f32" else np.uint16)
+    m = np.zeros((rows, k // 8), np.uint8) if mask else None
+    g = np.zeros(1, np.float32)
+    if scale is not None:
+        g[0] = np.float32(scale)
+    L.oracle_fake_quantize_bf16(_ptr(xb), rows, k, k, 1 if scale is not None else 0, _ptr(g),
+                                1 if out == "f32" else 0, _ptr(y), _ptr(m) if m is not None else None)
+    return y, m, np.float32(g[0])
+
+
+def ste_backward(grad_y: np.ndarray, mask: np.ndarray) -> np.ndarray:
+    """Straight-through estimator backward with the clip mask: grad_y where
+    the element was not clipped, +0 where it was.  ``grad_y`` is uint16 bf16
+    bits or float32, shape [rows, k]."""
+    L = lib()
+    gy = np.ascontiguousarray(grad_y)
+    assert gy.dtype in (np.uint16, np.float32)
+    m = np.ascontiguousarray(mask, np.uint8)
+    rows, k = gy.shape
+    assert m.shape == (rows, k // 8)
+    gx = np.empty_like(gy)
+    L.oracle_ste_backward(_ptr(gy), _ptr(m), rows, k, gy.dtype.itemsize, _ptr(gx))
+    return gx

@@ -36,6 +36,12 @@
  *  - The 16-value block runs along K (the reduction axis); scales are stored
  *    in the tensor-core scale-factor layout (128-row x 4-block atoms of 512
  *    bytes), rows padded to a multiple of 128 with zero bytes.
+ *  - Fake quantization (QAT) returns the same value the dequantizer gives
+ *    for the codes (e2m1 * dec(sf) * g, rounded once), so a trained model sees
+ *    in its forward pass exactly what the W4A4 product will multiply.  The
+ *    straight-through estimator passes the gradient unchanged; the optional
+ *    clip mask marks elements with |x| > 6 s (clip's derivative is zero
+ *    there), and a zero scale s clips nothing.
  *
  * Build: plain C99, no fast-math, no FMA contraction (see oracle/build.py).
  */
@@ -368,4 +374,66 @@ double oracle_gemm_w4a16_at(const uint16_t *x, const uint8_t *w_codes, const uin
     for (int64_t j = 0; j < K; ++j)
         acc += (double)oracle_bf16_to_f32(x[m * K + j]) * deq_elem(w_codes, w_sf, n, j, K);
     return (double)g_w * acc;
+}
+
+/* ----------------------- QAT fake quantization --------------------------- */
+/* Fake quantization for quantization-aware training [DiT, Definition III.1;
+ * Methodology 2: a straight-through estimator carries the gradient through
+ * the fake-quantize op].  The forward value is the quantizer's output
+ *   y = Q_FP4(x; s) = e2m1(code) * dec(sf) * g,  rounded once to bf16 or f32,
+ * with the codes and scales oracle_quantize_bf16 makes (same tensor-scale
+ * rule, g_io in/out), and the clip indicator that the estimator's backward
+ * rule uses:
+ *   clipped = s > 0 and |x| > 6 s      (exact comparison, s = fl32(dec(sf) * g))
+ * i.e. the elements whose scaled value x / s lies outside clip's range
+ * [-6, 6].  A block with s == 0 (all zero, or a zero tensor scale) has no
+ * clipped element: its values flush to zero by rounding, not by clip.
+ * y: rows * k values, row stride k; bf16 bits when out_f32 == 0, else float.
+ * mask (nullable): rows * k/8 bytes, row stride k/8; element j of a row is
+ * bit j % 8 of byte j / 8.                                                    */
+void oracle_fake_quantize_bf16(const uint16_t *x, int64_t rows, int64_t k, int64_t ld,
+                               int scale_given, float *g_io, int out_f32, void *y, uint8_t *mask)
+{
+    const int64_t kb = k / 16;
+    uint8_t *codes = (uint8_t *)malloc((size_t)(rows * (k / 2)) + 1);
+    uint8_t *sf = (uint8_t *)malloc((size_t)oracle_sf_bytes(rows, k) + 1);
+    if (!codes || !sf) { free(codes); free(sf); return; }
+    oracle_quantize_bf16(x, rows, k, ld, scale_given, g_io, codes, sf);
+    const float g = *g_io;
+    if (out_f32) oracle_dequantize_f32(codes, sf, g, rows, k, (float *)y);
+    else oracle_dequantize_bf16(codes, sf, g, rows, k, (uint16_t *)y);
+    if (mask) {
+        memset(mask, 0, (size_t)(rows * (k / 8)));
+        for (int64_t r = 0; r < rows; ++r)
+            for (int64_t j = 0; j < k; ++j) {
+                float sdec = (float)oracle_e4m3_decode(sf[oracle_sf_offset(r, j / 16, kb)]);
+                float s = sdec * g;                       /* the quantizer's s, as above */
+                double a = fabs((double)oracle_bf16_to_f32(x[r * ld + j]));
+                if (s > 0.0f && a > 6.0 * (double)s)      /* 6 s exact in double */
+                    mask[r * (k / 8) + j / 8] |= (uint8_t)(1u << (j % 8));
+            }
+    }
+    free(codes);
+    free(sf);
+}
+
+/* Backward rule of the straight-through estimator with the clip indicator
+ * [DiT, Methodology 2]: the gradient passes unchanged (the estimator treats
+ * round() as the identity) except where clip() cut the value off, whose
+ * derivative is zero there:
+ *   grad_x = 0 where clipped, grad_y elsewhere        (masked elements: +0)
+ * grad_y, grad_x: rows * k elements of elem_bytes bytes (2: bf16, 4: f32),
+ * row stride k; mask as oracle_fake_quantize_bf16 writes it.                  */
+void oracle_ste_backward(const void *grad_y, const uint8_t *mask, int64_t rows, int64_t k,
+                         int elem_bytes, void *grad_x)
+{
+    const uint8_t *src = (const uint8_t *)grad_y;
+    uint8_t *dst = (uint8_t *)grad_x;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < k; ++j) {
+            int64_t e = r * k + j;
+            int clipped = (mask[r * (k / 8) + j / 8] >> (j % 8)) & 1;
+            if (clipped) memset(dst + e * elem_bytes, 0, (size_t)elem_bytes);
+            else memcpy(dst + e * elem_bytes, src + e * elem_bytes, (size_t)elem_bytes);
+        }
 }

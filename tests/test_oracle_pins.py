@@ -416,3 +416,162 @@ def test_gemm_w4a16_vs_library_matmul():
     assert np.allclose(y, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
     xb = oracle.bf16_bits(x)
     assert oracle.gemm_w4a16_at(xb, wc, wsf, gw, 5, 7) == pytest.approx(y[5, 7], rel=1e-13)
+
+
+# ------------------------------------------------------------------ QAT fake quantization
+def bf16_by_search(v: Fraction) -> int:
+    """bf16 bits of the nearest bf16 value to an exact rational (ties to the
+    even pattern), by searching the neighbours of its float32 conversion."""
+    a = abs(v)
+    f = np.float32(float(a))
+    u = int(np.array([f], np.float32).view(np.uint32)[0] >> 16)
+    cands = [c for c in (u - 1, u, u + 1, u + 2) if 0 <= c < 0x7F80]
+    val = lambda c: Fraction(float((np.array([c << 16], np.uint32)).view(np.float32)[0]))
+    best = min(cands, key=lambda c: (abs(a - val(c)), c % 2))
+    return best
+
+
+def brute_fake_quantize(xf32: np.ndarray, scale=None):
+    """Fake quantization by searches: the brute-force codes and scales, each
+    value e2m1 * e4m3 * g formed as an exact rational and rounded to bf16 by
+    search, the clip mask by exact rational comparison |x| > 6 s."""
+    codes, sfm, g = brute_quantize(xf32, scale)
+    rows, k = xf32.shape
+    y = np.zeros((rows, k), np.uint16)
+    clip = np.zeros((rows, k), bool)
+    for r in range(rows):
+        for j in range(k):
+            c = int(codes[r, j])
+            dec = Fraction(float(_E4M3_ALL[sfm[r, j // 16]]))
+            mag = Fraction(E2M1_GRID[c & 7]) * dec * Fraction(float(g))
+            b = bf16_by_search(mag)
+            y[r, j] = b | (0x8000 if c & 8 else 0)
+            s = np.float32(np.float32(_E4M3_ALL[sfm[r, j // 16]]) * g)
+            clip[r, j] = s > 0 and abs(Fraction(float(xf32[r, j]))) > 6 * Fraction(float(s))
+    return y, clip, g
+
+
+def unpack_mask(m: np.ndarray, k: int) -> np.ndarray:
+    return np.unpackbits(m, axis=1, bitorder="little")[:, :k].astype(bool)
+
+
+@pytest.mark.parametrize("case", range(8))
+def test_fake_quantize_vs_brute_force_tiny(case):
+    rng = np.random.default_rng(200 + case)
+    rows, k = [(2, 64), (3, 128), (1, 192), (4, 64)][case % 4]
+    x = rng.standard_normal((rows, k)).astype(np.float32)
+    if case % 3 == 1:
+        x *= np.exp(rng.uniform(-9, 9, (rows, 1))).astype(np.float32)   # E4M3 subnormal scales
+    if case % 4 == 3:
+        x[0, :16] = 0.0
+        x[1, 3] = -1e-7
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    xf = xb.float().numpy()
+    amax = float(np.max(np.abs(xf)))
+    # a static scale: from the data (None), the data's own, or too small (clips)
+    scale = [None, None, float(np.float32(amax / 2688.0)), float(np.float32(amax / 20000.0))][case % 4]
+    y, m, g = oracle.fake_quantize(xb, scale)
+    by, bclip, bg = brute_fake_quantize(xf, scale)
+    assert np.float32(g) == bg
+    assert np.array_equal(y, by)
+    assert np.array_equal(unpack_mask(m, k), bclip)
+    y32, _, _ = oracle.fake_quantize(xb, scale, out="f32")
+    # f32 output: the same exact products, rounded by numpy's double -> float cast
+    codes, sf, _ = oracle.quantize(xb, scale)
+    assert np.array_equal(y32, oracle.dequantize(codes, sf, g, "f64").astype(np.float32))
+
+
+def test_fake_quantize_saturating_elements_closed_form():
+    """With a tensor scale g = 2^-e too small for the data, every element with
+    |x| > 2688 g lies in a block whose E4M3 scale saturates at 448, so it clips
+    to exactly +-2688 g (exact in bf16) and is marked; elements below stay
+    within half a grid spacing."""
+    xb = synth.random_bf16((128, 256), seed=21, dist="student_t3")
+    xf = xb.float().numpy().astype(np.float64)
+    amax = np.max(np.abs(xf))
+    e = int(np.ceil(np.log2(2688.0 / amax))) + 3          # 2688 g = amax / 8 .. amax / 4
+    g = 2.0 ** -e
+    y, m, gg = oracle.fake_quantize(xb, g)
+    assert gg == np.float32(g)
+    yf = oracle.bf16_to_f32(y).astype(np.float64)
+    big = np.abs(xf) > 2688.0 * g
+    assert big.sum() > 100
+    assert np.array_equal(yf[big], np.sign(xf[big]) * 2688.0 * g)
+    clip = unpack_mask(m, 256)
+    assert np.all(clip[big])
+    assert not np.any(clip[np.abs(xf) <= 2688.0 * g] & (np.abs(yf[np.abs(xf) <= 2688.0 * g]) == 0))
+
+
+@pytest.mark.parametrize("dist", ["normal", "student_t3", "token_scaled"])
+def test_fake_quantize_idempotent_under_fixed_scale(dist):
+    """Q(Q(x)) == Q(x) with the tensor scale held fixed: the output already
+    lies on the grid its own block scales define (a dropped factor, a swapped
+    sign or a wrong rounding would move it)."""
+    xb = synth.random_bf16((256, 512), seed=22, dist=dist)
+    _, _, g = oracle.fake_quantize(xb)
+    y1, _, _ = oracle.fake_quantize(xb, float(g))
+    y2, _, _ = oracle.fake_quantize(y1.view(np.uint16).reshape(256, 512), float(g))
+    assert np.array_equal(y1, y2)
+
+
+def test_fake_quantize_zero_cases():
+    z = torch.zeros(130, 64, dtype=torch.bfloat16)
+    y, m, g = oracle.fake_quantize(z)
+    assert g == 0.0 and not y.any() and not m.any()
+    # a zero tensor scale: every block scale is 0, every value flushes to +0, nothing clips
+    xb = synth.random_bf16((64, 128), seed=23, dist="normal")
+    y, m, _ = oracle.fake_quantize(xb, 0.0)
+    assert not y.any() and not m.any()
+
+
+def test_fake_quantize_unclipped_elements_within_half_spacing():
+    """Where the mask is clear, |x - y| is at most half the grid spacing at
+    |x / s| (plus the bf16 rounding of y); where it is set, |y| is the block's
+    largest grid value 6 s."""
+    xb = synth.random_bf16((256, 1024), seed=24, dist="outlier")
+    y, m, g = oracle.fake_quantize(xb)
+    xf = xb.float().numpy().astype(np.float64)
+    yf = oracle.bf16_to_f32(y).astype(np.float64)
+    codes, sf, _ = oracle.quantize(xb)
+    sfm = oracle.sf_matrix(sf, 256, 1024)
+    s32 = np.repeat(np.float32(_E4M3_ALL[sfm]) * np.float32(g), 16, axis=1).astype(np.float64)
+    clip = unpack_mask(m, 1024)
+    q = np.abs(xf) / np.where(s32 > 0, s32, 1.0)
+    spacing = np.where(q < 2, 0.5, np.where(q < 4, 1.0, 2.0))
+    ok = ~clip & (s32 > 0)
+    assert np.all(np.abs(xf - yf)[ok] <= (s32 * spacing / 2 + 2.0 ** -8 * np.abs(yf) + 2.0 ** -21 * np.abs(xf))[ok])
+    assert np.all(np.abs(np.abs(yf[clip]) - 6 * s32[clip]) <= 2.0 ** -8 * 6 * s32[clip])
+    assert np.all(q[clip] > 6)
+
+
+def test_ste_backward_closed_form():
+    rng = np.random.default_rng(25)
+    rows, k = 96, 256
+    m = rng.integers(0, 256, (rows, k // 8)).astype(np.uint8)
+    keep = ~unpack_mask(m, k)
+    g32 = rng.standard_normal((rows, k)).astype(np.float32)
+    out = oracle.ste_backward(g32, m)
+    assert np.array_equal(out, np.where(keep, g32, np.float32(0.0)))
+    assert not np.signbit(out[~keep]).any()
+    gb = rng.integers(0, 1 << 16, (rows, k)).astype(np.uint16)
+    out = oracle.ste_backward(gb, m)
+    assert np.array_equal(out, np.where(keep, gb, np.uint16(0)))
+
+
+def test_fake_quantize_grid_valued_input_is_a_fixed_point():
+    """Grid values times 2^m per block with g = 2^-8: s = 2^m exactly, every
+    value comes back unchanged, and the block maxima (|x| = 6 s exactly, on
+    clip's boundary) are not marked as clipped."""
+    rng = np.random.default_rng(26)
+    rows, k = 8, 128
+    vals = np.array(E2M1_GRID + [-v for v in E2M1_GRID[1:]], np.float64)
+    x = rng.choice(vals, (rows, k))
+    m = rng.integers(-12, 1, (rows, k // 16))
+    for r in range(rows):
+        for c in range(k // 16):
+            x[r, 16 * c] = -6.0 if (r + c) % 2 else 6.0
+            x[r, 16 * c:16 * c + 16] *= 2.0 ** m[r, c]
+    xb = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16)
+    y, mask, _ = oracle.fake_quantize(xb, 2.0 ** -8)
+    assert np.array_equal(oracle.bf16_to_f32(y).astype(np.float64), x)
+    assert not mask.any()
