@@ -30,6 +30,12 @@ FP4_OVER_BF16 = 4.0          # nominal dense FP4 / dense bf16 tensor throughput 
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # quantize, algorithmic bytes per element: 2 (amax read) + 2 (read) + 0.5 (codes) + 1/16 (scales)
 QUANT_BYTES_PER_ELEM = 4.5625
+# fake quantization (bf16 in, bf16 out, 1-bit clip mask): 2 (amax read) + 2 (read) + 2 (y) + 1/8 (mask);
+# with a given tensor scale no amax read; the masked STE backward reads the gradient and the mask and
+# writes the gradient
+QAT_FWD_DYNAMIC_BYTES = 6.125
+QAT_FWD_GIVEN_BYTES = 4.125
+QAT_BWD_BYTES = 4.125
 
 
 def load_peaks():
@@ -227,6 +233,37 @@ def reference_points(dev, layers, w4a16_layers):
         out["w4a16"][L.name] = {"shape": f"{L.M}x{L.K}x{L.N}", "ms": round(ms, 4),
                                 "tflops": round(2 * L.M * L.N * L.K / (ms * 1e-3) / 1e12, 1)}
         del x, W, y
+    # quantization-aware training: fake quantization (forward, clip mask
+    # included) and the masked straight-through backward on the fc1 / fc2
+    # inputs; HBM-bound, bytes per element as listed
+    hbm = load_peaks()[0].get("hbm_gbs", FALLBACK["hbm_gbs"])
+    out["qat"] = {}
+    for name in ("fc1", "fc2"):
+        if name not in [L.name for L in layers]:
+            continue
+        x, = synth.layer_tensors(WORKLOAD, name, device=dev, want=("x",))
+        x = x[: [L.M for L in layers if L.name == name][0]].contiguous()
+        rows, k = x.shape
+        y = torch.empty_like(x)
+        m = torch.empty(rows, k // 8, dtype=torch.uint8, device=dev)
+        g = torch.zeros(1, dtype=torch.float32, device=dev)
+        wsb = nv.nvfp4_quantize_workspace_bytes(rows, k)
+        ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+        gx = torch.empty_like(x)
+        runs = {
+            "fake_quantize_dynamic": (lambda: nv.nvfp4_fake_quantize(x, rows, k, k, y, 0, m, g, 0, ws, wsb),
+                                      QAT_FWD_DYNAMIC_BYTES),
+            "fake_quantize_given": (lambda: nv.nvfp4_fake_quantize(x, rows, k, k, y, 0, m, g, 1, None, 0),
+                                    QAT_FWD_GIVEN_BYTES),
+            "ste_backward": (lambda: nv.nvfp4_ste_backward(x, m, rows, k, 0, gx), QAT_BWD_BYTES),
+        }
+        res = {"shape": f"{rows}x{k}"}
+        for key, (fn, bpe) in runs.items():
+            ms = time_device(fn)
+            gbs = bpe * rows * k / (ms * 1e-3) / 1e9
+            res[key] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / hbm, 4), "bytes_per_elem": bpe}
+        out["qat"][name] = res
+        del x, y, m, gx, ws
     torch.cuda.empty_cache()
     return out
 

@@ -145,6 +145,48 @@ nvfp4_status nvfp4_dequantize(const uint8_t *codes, const uint8_t *sf,
                               void *out, int out_dtype, nvfp4_stream_t stream);
 
 /*
+ * nvfp4_fake_quantize -- fake quantization for quantization-aware training
+ * ([DiT] Definition III.1 and Methodology 2, where a straight-through
+ * estimator carries gradients through the fake-quantize op): quantization
+ * exactly as nvfp4_quantize (same tensor-scale rule, block scales and
+ * codes), followed in the same kernel by
+ *   y = e2m1(code) * e4m3(sf) * g,  rounded once (RNE) to y_dtype,
+ * the value nvfp4_dequantize would return, so that training sees in its
+ * forward pass what the W4A4 product multiplies.  No codes or scales are
+ * stored.
+ * x_bf16, rows, k, ld_x, tensor_scale, flags, workspace, workspace_bytes,
+ *               dev_status: as nvfp4_quantize (the workspace is needed unless
+ *               NVFP4_SCALE_GIVEN; nvfp4_quantize_workspace_bytes gives its size).
+ * y             out, [rows, k] contiguous (row stride k), NVFP4_DTYPE_BF16 or
+ *               NVFP4_DTYPE_F32, 16-byte aligned.
+ * clip_mask     out, nullable: rows * k/8 bytes, row stride k/8, 16-byte
+ *               aligned; bit j % 8 of byte j / 8 of a row is set where
+ *               element j was clipped, i.e. s > 0 and |x| > 6 s with the
+ *               block's s = e4m3(sf) * g (IEEE single product), compared
+ *               exactly.  A block with s == 0 clips nothing.
+ * One kernel with a given scale; with a data-derived scale, one kernel when
+ * the grid can be co-resident, else two (amax pass, then fake quantization).
+ */
+nvfp4_status nvfp4_fake_quantize(const void *x_bf16, int64_t rows, int64_t k, int64_t ld_x,
+                                 void *y, int y_dtype, uint8_t *clip_mask,
+                                 float *tensor_scale, unsigned flags,
+                                 void *workspace, size_t workspace_bytes,
+                                 int *dev_status, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_ste_backward -- backward rule of the straight-through estimator with
+ * the clip mask ([DiT] Methodology 2; clip's derivative is zero outside its
+ * range): grad_x = grad_y where the mask bit is clear, +0 where it is set.
+ * (The plain estimator, without the mask, is the identity and needs no call.)
+ * grad_y, grad_x [rows, k] contiguous in dtype (NVFP4_DTYPE_BF16 or
+ * NVFP4_DTYPE_F32), 16-byte aligned; grad_x may be grad_y (in place).
+ * clip_mask as written by nvfp4_fake_quantize for [rows, k].
+ * rows >= 0, k > 0 and k % 16 == 0.  One kernel on `stream`.
+ */
+nvfp4_status nvfp4_ste_backward(const void *grad_y, const uint8_t *clip_mask, int64_t rows, int64_t k,
+                                int dtype, void *grad_x, nvfp4_stream_t stream);
+
+/*
  * nvfp4_gemm_w4a4 -- block-scaled FP4 x FP4 product with FP32 accumulation
  * ([DiT] 3. Systems optimization; [RFC] Open Questions 1, W4A4):
  *   acc[m,n] = sum_k (e2m1(a)*e4m3(sfa)) * (e2m1(b)*e4m3(sfb))   (FP32, tensor cores)

@@ -7,9 +7,11 @@ memory and streams.
 
 Low-level (same names and argument order as the C calls):
     nvfp4_sf_bytes, nvfp4_quantize_workspace_bytes, nvfp4_quantize,
-    nvfp4_quantize_noalloc, nvfp4_dequantize, nvfp4_gemm_w4a4, nvfp4_gemm_w4a16, nvfp4_launch_count
+    nvfp4_quantize_noalloc, nvfp4_dequantize, nvfp4_fake_quantize, nvfp4_ste_backward,
+    nvfp4_gemm_w4a4, nvfp4_gemm_w4a16, nvfp4_launch_count
 Convenience (allocate outputs with torch, then call the above):
-    NVFP4Tensor, quantize, dequantize, gemm_w4a4, gemm_w4a16
+    NVFP4Tensor, quantize, dequantize, gemm_w4a4, gemm_w4a16,
+    fake_quantize, ste_backward, FakeQuantizeSTE (autograd: the two kernels)
 """
 from __future__ import annotations
 
@@ -90,6 +92,18 @@ def nvfp4_dequantize(codes, sf, tensor_scale, rows, k, out, out_dtype, stream=No
     st = lib().nvfp4_dequantize(_ptr(codes), _ptr(sf), _ptr(tensor_scale), rows, k, _ptr(out),
                                 out_dtype, _stream(stream))
     check(st, "nvfp4_dequantize")
+
+
+def nvfp4_fake_quantize(x, rows, k, ld_x, y, y_dtype, clip_mask, tensor_scale, flags=0, workspace=None,
+                        workspace_bytes=0, dev_status=None, stream=None) -> None:
+    st = lib().nvfp4_fake_quantize(_ptr(x), rows, k, ld_x, _ptr(y), y_dtype, _ptr(clip_mask), _ptr(tensor_scale),
+                                   flags, _ptr(workspace), workspace_bytes, _ptr(dev_status), _stream(stream))
+    check(st, "nvfp4_fake_quantize")
+
+
+def nvfp4_ste_backward(grad_y, clip_mask, rows, k, dtype, grad_x, stream=None) -> None:
+    st = lib().nvfp4_ste_backward(_ptr(grad_y), _ptr(clip_mask), rows, k, dtype, _ptr(grad_x), _stream(stream))
+    check(st, "nvfp4_ste_backward")
 
 
 def nvfp4_gemm_w4a4(a_codes, a_sf, a_scale, b_codes, b_sf, b_scale, M, N, K, y=None,
@@ -182,3 +196,60 @@ def gemm_w4a16(x: torch.Tensor, w: NVFP4Tensor, out_dtype=torch.bfloat16, out: t
     y = out if out is not None else torch.empty(x.shape[0], w.rows, dtype=out_dtype, device=x.device)
     nvfp4_gemm_w4a16(x, w.codes, w.sf, w.scale, x.shape[0], w.rows, w.k, y, _DT[y.dtype], dev_status, stream)
     return y
+
+
+# ----------------------------------------------------------------- QAT
+def fake_quantize(x: torch.Tensor, scale: torch.Tensor | float | None = None, out_dtype=torch.bfloat16,
+                  clip_mask: bool = True, workspace: torch.Tensor | None = None, dev_status=None, stream=None):
+    """Fake-quantize a bf16 [rows, k] CUDA tensor: returns (y, mask, scale) with
+    y = the NVFP4 value of each element (bf16 or f32), mask the packed clip
+    bits ([rows, k/8] uint8, None unless ``clip_mask``) and scale the tensor
+    scale used (computed on the device unless given)."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, k = x.shape
+    y = torch.empty(rows, k, dtype=out_dtype, device=x.device)
+    m = torch.empty(rows, k // 8, dtype=torch.uint8, device=x.device) if clip_mask else None
+    g = torch.zeros(1, dtype=torch.float32, device=x.device)
+    flags = 0
+    if scale is not None:
+        if isinstance(scale, torch.Tensor):
+            g.copy_(scale.reshape(1).to(torch.float32))
+        else:
+            g.fill_(float(scale))
+        flags = NVFP4_SCALE_GIVEN
+    wsb = nvfp4_quantize_workspace_bytes(rows, k)
+    if flags == 0 and workspace is None:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=x.device)
+    nvfp4_fake_quantize(x, rows, k, x.stride(0), y, _DT[out_dtype], m, g, flags,
+                        workspace if flags == 0 else None, wsb if flags == 0 else 0, dev_status, stream)
+    return y, m, g
+
+
+def ste_backward(grad_y: torch.Tensor, clip_mask: torch.Tensor, out: torch.Tensor | None = None,
+                 stream=None) -> torch.Tensor:
+    """grad_y where the clip mask is clear, +0 where set (``out`` may be grad_y)."""
+    assert grad_y.dim() == 2 and grad_y.is_contiguous() and grad_y.dtype in _DT
+    rows, k = grad_y.shape
+    gx = out if out is not None else torch.empty_like(grad_y)
+    nvfp4_ste_backward(grad_y, clip_mask, rows, k, _DT[grad_y.dtype], gx, stream)
+    return gx
+
+
+class FakeQuantizeSTE(torch.autograd.Function):
+    """Autograd wrapper of the two kernels: forward = nvfp4_fake_quantize,
+    backward = nvfp4_ste_backward with the forward's clip mask (masked=True)
+    or the identity (masked=False, the plain straight-through estimator)."""
+
+    @staticmethod
+    def forward(ctx, x, scale=None, masked=True):
+        y, m, _ = fake_quantize(x, scale, clip_mask=masked)
+        ctx.save_for_backward(*([m] if masked else []))
+        ctx.masked = masked
+        return y
+
+    @staticmethod
+    def backward(ctx, grad_y):
+        if not ctx.masked:
+            return grad_y, None, None
+        (m,) = ctx.saved_tensors
+        return ste_backward(grad_y.contiguous(), m), None, None

@@ -33,6 +33,9 @@ SIGNATURES = {
     "nvfp4_quantize": (_status, [_p, _i64, _i64, _i64, _p, _p, _p, ctypes.c_uint, _p, ctypes.c_size_t, _p, _p]),
     "nvfp4_quantize_noalloc": (_status, [_p, _i64, _i64, _i64, _p, _p, _p, ctypes.c_uint, _p, _p]),
     "nvfp4_dequantize": (_status, [_p, _p, _p, _i64, _i64, _p, _int, _p]),
+    "nvfp4_fake_quantize": (_status, [_p, _i64, _i64, _i64, _p, _int, _p, _p, ctypes.c_uint, _p, ctypes.c_size_t,
+                                      _p, _p]),
+    "nvfp4_ste_backward": (_status, [_p, _p, _i64, _i64, _int, _p, _p]),
     "nvfp4_gemm_w4a4": (_status, [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _p, _int, _p, _p, _p, _p, _p, _p]),
     "nvfp4_gemm_w4a16": (_status, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _int, _p, _p]),
     "nvfp4_status_string": (ctypes.c_char_p, [_int]),

@@ -146,6 +146,50 @@ nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* sf, const flo
                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 
+nvfp4_status nvfp4_fake_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, void* y, int y_dtype,
+                                 uint8_t* clip_mask, float* tensor_scale, unsigned flags, void* workspace,
+                                 size_t workspace_bytes, int* dev_status, nvfp4_stream_t stream) {
+    if (rows < 0 || k <= 0 || ld_x < k) return NVFP4_ERR_INVALID_ARG;
+    if ((flags & ~(unsigned)NVFP4_SCALE_GIVEN) != 0u) return NVFP4_ERR_INVALID_ARG;
+    if (y_dtype != NVFP4_DTYPE_BF16 && y_dtype != NVFP4_DTYPE_F32) return NVFP4_ERR_INVALID_ARG;
+    if (!tensor_scale) return NVFP4_ERR_INVALID_ARG;
+    if (rows > 0 && (!x_bf16 || !y)) return NVFP4_ERR_INVALID_ARG;
+    if (k % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (rows > (int64_t)1 << 31 || k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    const bool given = (flags & NVFP4_SCALE_GIVEN) != 0u;
+    if (!given && (!workspace || workspace_bytes < kQuantWorkspaceBytes)) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(x_bf16) || !aligned16(y) || (clip_mask && !aligned16(clip_mask)) || (ld_x % 8) != 0 ||
+        (!given && !aligned16(workspace)) || (reinterpret_cast<uintptr_t>(tensor_scale) & 3u))
+        return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    nvfp4_status st = device_ok(&sms);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (rows == 0) {
+        if (!given) return cuda_status(cudaMemsetAsync(tensor_scale, 0, sizeof(float), s));
+        return NVFP4_OK;
+    }
+    return cuda_status(launch_fake_quantize(static_cast<const uint16_t*>(x_bf16), rows, k, ld_x, y,
+                                            y_dtype == NVFP4_DTYPE_F32, clip_mask, tensor_scale, given, workspace,
+                                            dev_status, sms, s));
+}
+
+nvfp4_status nvfp4_ste_backward(const void* grad_y, const uint8_t* clip_mask, int64_t rows, int64_t k, int dtype,
+                                void* grad_x, nvfp4_stream_t stream) {
+    if (rows < 0 || k <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (dtype != NVFP4_DTYPE_BF16 && dtype != NVFP4_DTYPE_F32) return NVFP4_ERR_INVALID_ARG;
+    if (rows > 0 && (!grad_y || !clip_mask || !grad_x)) return NVFP4_ERR_INVALID_ARG;
+    if (k % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (rows > (int64_t)1 << 31 || k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(grad_y) || !aligned16(clip_mask) || !aligned16(grad_x)) return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    nvfp4_status st = device_ok(&sms);
+    if (st != NVFP4_OK) return st;
+    if (rows == 0) return NVFP4_OK;
+    return cuda_status(launch_ste_backward(grad_y, clip_mask, rows, k, dtype == NVFP4_DTYPE_F32, grad_x, sms,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
 nvfp4_status nvfp4_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_scale,
                              const uint8_t* b_codes, const uint8_t* b_sf, const float* b_scale, int64_t M, int64_t N,
                              int64_t K, void* y, int y_dtype, uint8_t* y_codes, uint8_t* y_sf, const float* y_scale,

@@ -25,6 +25,13 @@ cudaError_t launch_quantize_fused(const uint16_t* x, int64_t rows, int64_t k, in
                                   uint8_t* sf, float* tensor_scale, unsigned long long* slots, int max_slots,
                                   int* dev_status, int num_sms, cudaStream_t stream);
 
+cudaError_t launch_fake_quantize(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, void* y, bool y_f32,
+                                 uint8_t* mask, float* tensor_scale, bool scale_given, void* workspace,
+                                 int* dev_status, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_ste_backward(const void* grad_y, const uint8_t* mask, int64_t rows, int64_t k, bool f32,
+                                void* grad_x, int num_sms, cudaStream_t stream);
+
 cudaError_t launch_debug_wait_timeout(int* dev_status, uint64_t limit_ns, cudaStream_t stream);
 
 void reset_noalloc_cache();

@@ -111,17 +111,17 @@ constexpr int kSteps = kRows / 2;
 constexpr int kAtomPitch = 516;
 
 // Per-lane view of one tile: step i handles row rt0 + 2i of the tile; the
-// pointers are for step 0 and advance by two rows per step (ld and kh are
-// multiples of 8 and 32).
+// input pointer is for step 0 and advances by two rows per step (ld is a
+// multiple of 8).  e0 is the index of the lane's first value in a contiguous
+// [rows, k] layout, from which each output places its results.
 struct TileLane {
     const uint4* xp;
-    uint2* cp;
-    int64_t xstep, cstep, rows_left;
+    int64_t xstep, rows_left, e0;
     int sbase;
     bool col_ok;
 };
 
-__device__ __forceinline__ TileLane tile_lane(const uint16_t* x, uint8_t* codes, int64_t rows, int64_t k, int64_t ld,
+__device__ __forceinline__ TileLane tile_lane(const uint16_t* x, int64_t rows, int64_t k, int64_t ld,
                                               int64_t rblk, int64_t cblk, int warp, int lane) {
     TileLane t;
     const int64_t c0 = cblk * kTileCols;
@@ -129,13 +129,11 @@ __device__ __forceinline__ TileLane tile_lane(const uint16_t* x, uint8_t* codes,
     const int half = lane >> 4, blk = lane & 15;
     const int rt0 = warp * kRows + half;
     const int64_t r0 = rblk * kTileRows + rt0;
-    const int64_t kh = k >> 1;
     t.col_ok = blk * 16 < ncols;
     t.rows_left = rows - r0;                      // step i is in range iff 2i < rows_left
     t.xp = reinterpret_cast<const uint4*>(x + r0 * ld + c0) + 2 * blk;
     t.xstep = ld >> 2;                            // two rows, in 16-byte units
-    t.cp = reinterpret_cast<uint2*>(codes + r0 * kh + (c0 >> 1)) + blk;
-    t.cstep = kh >> 2;                            // two rows, in 8-byte units
+    t.e0 = r0 * k + c0 + 16 * blk;
     // block blk of row rt: atom blk / 4, byte blk % 4 of the row's word
     t.sbase = (blk >> 2) * kAtomPitch + (rt0 & 31) * 16 + (rt0 >> 5) * 4 + (blk & 3);
     return t;
@@ -156,24 +154,6 @@ __device__ __forceinline__ void load_tile(const TileLane& t, uint4 (&v)[2 * kSte
     }
 }
 
-// Quantize a lane's loaded blocks: codes straight to global memory, scale
-// bytes to the CTA's staging atoms.
-__device__ __forceinline__ void quantize_lane(const TileLane& t, const uint4 (&v)[2 * kSteps], const ScaleConsts& sc,
-                                              uint8_t* sf_stage) {
-#pragma unroll
-    for (int i = 0; i < kSteps; ++i) {
-        const uint32_t w[8] = {v[2 * i].x, v[2 * i].y, v[2 * i].z, v[2 * i].w,
-                               v[2 * i + 1].x, v[2 * i + 1].y, v[2 * i + 1].z, v[2 * i + 1].w};
-        const float ab = __uint_as_float(block_absmax16(w) << 16);      // block amax
-        const uint32_t sfc = block_scale_code(ab, sc);
-        const float s = __fmul_rn(e4m3_to_f32(sfc), sc.g);
-        const uint32_t lo = quantize8_bf16(w[0], w[1], w[2], w[3], s);
-        const uint32_t hi = quantize8_bf16(w[4], w[5], w[6], w[7], s);
-        if (2 * i < t.rows_left && t.col_ok) t.cp[i * t.cstep] = make_uint2(lo, hi);
-        if (t.col_ok) sf_stage[t.sbase + 32 * i] = (uint8_t)sfc;
-    }
-}
-
 // Copy a tile's staged scale atoms (consecutive in the scale buffer) out, one
 // word per thread.  The caller synchronizes the CTA before and after.
 __device__ __forceinline__ void store_tile_scales(const uint8_t* sf_stage, uint8_t* sf, int64_t k, int64_t rblk,
@@ -188,12 +168,212 @@ __device__ __forceinline__ void store_tile_scales(const uint8_t* sf_stage, uint8
     if (i < natoms * 128) dst[i] = *reinterpret_cast<const uint32_t*>(sf_stage + (i >> 7) * kAtomPitch + (i & 127) * 4);
 }
 
+// ---------------------------------------------------------------- outputs
+// What a lane does with a quantized block.  Each output type gives a per-lane
+// view (pointers for step 0 and their two-row advance) and emit(), called once
+// per step with the block's bf16 words, scale code, decoded scale s and codes.
+
+// nvfp4_quantize: packed codes straight to global memory (8 bytes per block);
+// scale bytes staged per tile in the tensor-core layout.
+struct CodesOut {
+    uint8_t* codes;
+    uint8_t* sf;
+    static constexpr bool kScales = true;
+    static constexpr int kMinBlocks = 0;          // unforced: the compiler fits 64 registers (2 CTAs per SM)
+    struct Lane {
+        uint2* cp;
+        int64_t step;
+    };
+    __device__ __forceinline__ Lane lane(const TileLane& t, int64_t k) const {
+        return {reinterpret_cast<uint2*>(codes) + (t.e0 >> 4), k >> 3};
+    }
+    __device__ __forceinline__ void emit(const Lane& l, int i, bool ok, const uint32_t (&)[8], uint32_t, float,
+                                         uint32_t lo, uint32_t hi, const ScaleConsts&) const {
+        if (ok) l.cp[i * l.step] = make_uint2(lo, hi);
+    }
+    __device__ __forceinline__ void store_scales(const uint8_t* sf_stage, int64_t k, int64_t rblk,
+                                                 int64_t cblk) const {
+        store_tile_scales(sf_stage, sf, k, rblk, cblk);
+    }
+};
+
+// f16x2 of two E2M1 codes (one byte, the low nibble in the low half) times
+// the block's decoded scale (f16 in both halves of sd2): exact, since the
+// product has at most 6 significant bits and lies within [2^-10, 2688].
+__device__ __forceinline__ uint32_t e2m1x2_times_scale(uint32_t byte, uint32_t sd2) {
+    uint32_t h2, e2;
+    asm("{\n\t.reg .b8 c;\n\t"
+        "cvt.u8.u32 c, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, c;\n\t}"
+        : "=r"(h2)
+        : "r"(byte));
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(e2) : "r"(h2), "r"(sd2));
+    return e2;
+}
+
+// The two halves of an f16x2 as a packed FP32 pair (low half first).
+__device__ __forceinline__ uint64_t f16x2_to_f32x2(uint32_t h2) {
+    uint64_t r;
+    asm("{\n\t.reg .f16 a, b;\n\t.reg .f32 fa, fb;\n\t"
+        "mov.b32 {a, b}, %1;\n\t"
+        "cvt.f32.f16 fa, a;\n\t"
+        "cvt.f32.f16 fb, b;\n\t"
+        "mov.b64 %0, {fa, fb};\n\t}"
+        : "=l"(r)
+        : "r"(h2));
+    return r;
+}
+
+// bf16x2 of e * g rounded once (RNE) for a packed pair e of exact FP32
+// values, ng2 = (-g, -g): the product truncated to FP32 is made odd when the
+// residual e*g - rz(e*g) (exact by the FMA) is not zero, and that
+// round-to-odd value, with 16 spare bits, rounds to bf16 as the exact product
+// would.  Valid while every nonzero |e * g| >= 2^-120 (the residual is then
+// representable); e == 0 gives a zero of e's sign.
+__device__ __forceinline__ uint32_t bf16x2_round_once(uint64_t e2, uint64_t g2, uint64_t ng2) {
+    uint64_t t, r;
+    asm("mul.rz.f32x2 %0, %1, %2;" : "=l"(t) : "l"(e2), "l"(g2));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(e2), "l"(ng2), "l"(t));
+    uint32_t tl, th, rl, rh, out;
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(tl), "=r"(th) : "l"(t));
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(rl), "=r"(rh) : "l"(r));
+    tl |= (rl << 1) != 0u ? 1u : 0u;
+    th |= (rh << 1) != 0u ? 1u : 0u;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(__uint_as_float(th)), "f"(__uint_as_float(tl)));
+    return out;
+}
+
+// The same for blocks with a tiny scale: the product formed exactly in
+// double, truncated to FP32 with the sticky bit, then rounded to bf16.
+__device__ __forceinline__ uint32_t bf16x2_round_once_slow(uint64_t e2, float g) {
+    uint32_t el, eh, out;
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(el), "=r"(eh) : "l"(e2));
+    float v[2];
+    const uint32_t e[2] = {el, eh};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const double p = (double)__uint_as_float(e[h]) * (double)g;    // exact
+        float t = __double2float_rz(p);
+        if ((double)t != p) t = __uint_as_float(__float_as_uint(t) | 1u);
+        v[h] = t;
+    }
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(v[1]), "f"(v[0]));
+    return out;
+}
+
+// Clip mask of 16 bf16 values (eight words, element 2j in the low half of
+// word j): bit e set where |x_e| > 6 s, s > 0.  For bf16 x, |x| > 6 s exactly
+// iff |x| > RD_bf16(6 s), and RD_bf16(RD_f32(6 s)) = RD_bf16(6 s); as
+// non-negative patterns compare like their values, each half then tests
+// |x| >= tb with tb = RD_bf16(6 s) + 1 by one subtraction from 0x8000 + |x|
+// (no borrow crosses the halves).  s == 0 gives tb = 0x8000: nothing clips.
+__device__ __forceinline__ uint32_t clip_mask16(const uint32_t (&w)[8], float s) {
+    const uint32_t tb = s > 0.0f ? (__float_as_uint(__fmul_rd(6.0f, s)) >> 16) + 1u : 0x8000u;
+    const uint32_t t2 = tb | (tb << 16);
+    uint32_t acc = 0u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc |= (((w[j] | 0x80008000u) - t2) >> 15 & 0x00010001u) << (2 * j);
+    return (acc & 0x5555u) | ((acc >> 15) & 0xAAAAu);
+}
+
+// nvfp4_fake_quantize: y = e2m1(code) * dec(sf) * g rounded once to bf16 (or
+// FP32), 16 values per lane and step, and the optional clip mask (2 bytes per
+// lane and step).  Scales are not stored.
+template <bool kF32>
+struct FakeOut {
+    void* y;
+    uint8_t* mask;                                // nullable
+    static constexpr bool kScales = false;
+    static constexpr int kMinBlocks = 2;          // 64 registers: 2 CTAs (32 warps) per SM
+    struct Lane {
+        uint4* yp;
+        uint16_t* mp;
+        int64_t ystep, mstep;
+    };
+    __device__ __forceinline__ Lane lane(const TileLane& t, int64_t k) const {
+        Lane l;
+        l.yp = reinterpret_cast<uint4*>(y) + (kF32 ? (t.e0 >> 2) : (t.e0 >> 3));
+        l.ystep = kF32 ? (k >> 1) : (k >> 2);      // two rows, in 16-byte units
+        l.mp = reinterpret_cast<uint16_t*>(mask) + (t.e0 >> 4);
+        l.mstep = k >> 3;
+        return l;
+    }
+    __device__ __forceinline__ void emit(const Lane& l, int i, bool ok, const uint32_t (&w)[8], uint32_t sfc,
+                                         float s, uint32_t lo, uint32_t hi, const ScaleConsts& sc) const {
+        uint32_t sd2;
+        {
+            const uint16_t in = (uint16_t)(sfc | (sfc << 8));
+            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(sd2) : "h"(in));
+        }
+        const uint64_t g2 = f32x2(sc.g, sc.g);
+        const uint32_t codes[2] = {lo, hi};
+        if (kF32) {
+            uint32_t o[16];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint64_t p = mul_f32x2(f16x2_to_f32x2(e2m1x2_times_scale(codes[h] >> (8 * j), sd2)), g2);
+                    asm("mov.b64 {%0, %1}, %2;" : "=r"(o[8 * h + 2 * j]), "=r"(o[8 * h + 2 * j + 1]) : "l"(p));
+                }
+            if (ok) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    l.yp[i * l.ystep + q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+            }
+        } else {
+            uint32_t o[8];
+            if (s >= 0x1p-118f || s == 0.0f) {
+                const uint64_t ng2 = f32x2(-sc.g, -sc.g);
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        o[4 * h + j] = bf16x2_round_once(f16x2_to_f32x2(e2m1x2_times_scale(codes[h] >> (8 * j), sd2)),
+                                                         g2, ng2);
+            } else {
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        o[4 * h + j] =
+                            bf16x2_round_once_slow(f16x2_to_f32x2(e2m1x2_times_scale(codes[h] >> (8 * j), sd2)), sc.g);
+            }
+            if (ok) {
+                l.yp[i * l.ystep] = make_uint4(o[0], o[1], o[2], o[3]);
+                l.yp[i * l.ystep + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+            }
+        }
+        if (mask != nullptr && ok) l.mp[i * l.mstep] = (uint16_t)clip_mask16(w, s);
+    }
+    __device__ __forceinline__ void store_scales(const uint8_t*, int64_t, int64_t, int64_t) const {}
+};
+
+// Quantize a lane's loaded blocks and hand each to the output; scale bytes go
+// to the CTA's staging atoms when the output stores scales.
+template <class Out>
+__device__ __forceinline__ void quantize_lane(const TileLane& t, const uint4 (&v)[2 * kSteps], const ScaleConsts& sc,
+                                              uint8_t* sf_stage, const Out& out, int64_t k) {
+    const typename Out::Lane ol = out.lane(t, k);
+#pragma unroll
+    for (int i = 0; i < kSteps; ++i) {
+        const uint32_t w[8] = {v[2 * i].x, v[2 * i].y, v[2 * i].z, v[2 * i].w,
+                               v[2 * i + 1].x, v[2 * i + 1].y, v[2 * i + 1].z, v[2 * i + 1].w};
+        const float ab = __uint_as_float(block_absmax16(w) << 16);      // block amax
+        const uint32_t sfc = block_scale_code(ab, sc);
+        const float s = __fmul_rn(e4m3_to_f32(sfc), sc.g);
+        const uint32_t lo = quantize8_bf16(w[0], w[1], w[2], w[3], s);
+        const uint32_t hi = quantize8_bf16(w[4], w[5], w[6], w[7], s);
+        out.emit(ol, i, 2 * i < t.rows_left && t.col_ok, w, sfc, s, lo, hi, sc);
+        if (Out::kScales && t.col_ok) sf_stage[t.sbase + 32 * i] = (uint8_t)sfc;
+    }
+}
+
 // Two-kernel form: one CTA per tile, after the amax pass (or with a given
 // tensor scale).
-template <bool kDynamic>
-__global__ void __launch_bounds__(kQuantThreads)
-quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
-                uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+template <bool kDynamic, class Out>
+__global__ void __launch_bounds__(kQuantThreads, Out::kMinBlocks)
+quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld, const Out out,
                 float* __restrict__ tensor_scale, const float* __restrict__ partials, int nparts) {
     __shared__ __align__(16) uint8_t sf_stage[4 * kAtomPitch];
     __shared__ ScaleConsts sc_sh;
@@ -202,7 +382,7 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
     // to back, so its tail is the part still in L2 when the first CTAs start
     const int64_t rblk = (int64_t)(gridDim.y - 1 - blockIdx.y);
     const int64_t cblk = blockIdx.x;
-    const TileLane t = tile_lane(x, codes, rows, k, ld, rblk, cblk, warp, lane);
+    const TileLane t = tile_lane(x, rows, k, ld, rblk, cblk, warp, lane);
     uint4 v[2 * kSteps];
     load_tile(t, v);
 
@@ -223,9 +403,11 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
         if (lane == 0) sc_sh = scale_consts(g);
     }
     __syncthreads();
-    quantize_lane(t, v, sc_sh, sf_stage);
-    __syncthreads();
-    store_tile_scales(sf_stage, sf, k, rblk, cblk);
+    quantize_lane(t, v, sc_sh, sf_stage, out, k);
+    if (Out::kScales) {
+        __syncthreads();
+        out.store_scales(sf_stage, k, rblk, cblk);
+    }
 }
 
 // One-kernel form with a data-derived tensor scale: a persistent grid whose
@@ -236,9 +418,10 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t
 // a per-call number from the host, so the slots need no initialisation -- and
 // takes the maximum itself.  Phase 2 quantizes the same tiles in reverse
 // order, so the first ones re-read what phase 1 read last, still in L2.
-__global__ void __launch_bounds__(kQuantThreads)
-quantize_fused_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
-                      uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ tensor_scale,
+template <class Out>
+__global__ void __launch_bounds__(kQuantThreads, Out::kMinBlocks)
+quantize_fused_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ld, const Out out,
+                      float* __restrict__ tensor_scale,
                       unsigned long long* __restrict__ slots, uint32_t gen, int ntiles_c, int ntiles,
                       int* __restrict__ dev_status) {
     __shared__ __align__(16) uint8_t sf_stage[4 * kAtomPitch];
@@ -250,7 +433,7 @@ quantize_fused_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, i
     // ---- phase 1: |x| maximum (and the largest exponent field) of this CTA's tiles
     uint32_t m = 0u;
     for (int tt = blockIdx.x; tt < ntiles; tt += gridDim.x) {
-        const TileLane t = tile_lane(x, codes, rows, k, ld, tt / ntiles_c, tt % ntiles_c, warp, lane);
+        const TileLane t = tile_lane(x, rows, k, ld, tt / ntiles_c, tt % ntiles_c, warp, lane);
         uint4 v[2 * kSteps];
 #pragma unroll
         for (int i = 0; i < kSteps; ++i) {
@@ -312,13 +495,15 @@ quantize_fused_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, i
     for (int j = nmine - 1; j >= 0; --j) {
         const int tt = (int)blockIdx.x + j * (int)gridDim.x;
         const int64_t rblk = tt / ntiles_c, cblk = tt % ntiles_c;
-        const TileLane t = tile_lane(x, codes, rows, k, ld, rblk, cblk, warp, lane);
+        const TileLane t = tile_lane(x, rows, k, ld, rblk, cblk, warp, lane);
         uint4 v[2 * kSteps];
         load_tile(t, v);
-        quantize_lane(t, v, sc, sf_stage);
-        __syncthreads();
-        store_tile_scales(sf_stage, sf, k, rblk, cblk);
-        __syncthreads();
+        quantize_lane(t, v, sc, sf_stage, out, k);
+        if (Out::kScales) {
+            __syncthreads();
+            out.store_scales(sf_stage, k, rblk, cblk);
+            __syncthreads();
+        }
     }
 }
 
@@ -378,6 +563,56 @@ dequantize_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__
     }
 }
 
+// ------------------------------------------------------------------ STE backward
+// grad_x = grad_y where the clip mask is clear, +0 where it is set.  One
+// thread per 16 elements (one 16-bit mask word), two groups in flight per
+// iteration; contiguous [rows, k] buffers seen as a flat array.  grad_x may
+// be grad_y (each element is read, then written, by the same thread), so the
+// pointers are not declared restrict.
+template <bool kF32>
+__global__ void __launch_bounds__(256)
+ste_backward_kernel(const uint4* gy, const uint16_t* mask, int64_t ngroups, uint4* gx) {
+    constexpr int kVec = kF32 ? 4 : 2;                // 16-byte vectors per group
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < ngroups; g += 2 * stride) {
+        const bool two = g + stride < ngroups;
+        uint4 a[kVec], b[kVec];
+        uint32_t ma = __ldcs(mask + g), mb = 0u;
+#pragma unroll
+        for (int q = 0; q < kVec; ++q) a[q] = __ldcs(gy + g * kVec + q);
+        if (two) {
+            mb = __ldcs(mask + g + stride);
+#pragma unroll
+            for (int q = 0; q < kVec; ++q) b[q] = __ldcs(gy + (g + stride) * kVec + q);
+        }
+        auto apply = [](uint4 (&v)[kVec], uint32_t m) {
+#pragma unroll
+            for (int q = 0; q < kVec; ++q) {
+                uint32_t* w = &v[q].x;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (kF32) {
+                        const int e = 4 * q + j;
+                        if ((m >> e) & 1u) w[j] = 0u;
+                    } else {
+                        const int e = 8 * q + 2 * j;      // elements e (low half), e + 1 (high half)
+                        const uint32_t clear = (((m >> e) & 1u) * 0x0000FFFFu) | (((m >> (e + 1)) & 1u) * 0xFFFF0000u);
+                        w[j] &= ~clear;
+                    }
+                }
+            }
+        };
+        apply(a, ma);
+#pragma unroll
+        for (int q = 0; q < kVec; ++q) __stcs(gx + g * kVec + q, a[q]);
+        if (two) {
+            apply(b, mb);
+#pragma unroll
+            for (int q = 0; q < kVec; ++q) __stcs(gx + (g + stride) * kVec + q, b[q]);
+        }
+    }
+}
+
 // ------------------------------------------------------------------ launchers
 int amax_grid(int64_t rows, int64_t k) {
     const int64_t nvec = rows * (k >> 3);
@@ -387,13 +622,15 @@ int amax_grid(int64_t rows, int64_t k) {
     return (int)g;
 }
 
-cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes,
-                            uint8_t* sf, float* tensor_scale, bool scale_given, float* partials,
-                            int* dev_status, cudaStream_t stream) {
+// Two-kernel form (or one kernel with a given scale) for any output.
+template <class Out>
+static cudaError_t launch_two_kernel(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, const Out& out,
+                                     float* tensor_scale, bool scale_given, float* partials, int* dev_status,
+                                     cudaStream_t stream) {
     const dim3 grid((unsigned)((k + 255) / 256), (unsigned)((rows + 127) / 128));
     if (scale_given) {
-        quantize_kernel<false><<<grid, kQuantThreads, 0, stream>>>(x, rows, k, ld, codes, sf, tensor_scale,
-                                                                  nullptr, 0);
+        quantize_kernel<false, Out><<<grid, kQuantThreads, 0, stream>>>(x, rows, k, ld, out, tensor_scale,
+                                                                       nullptr, 0);
         count_launch(1);
         return cudaGetLastError();
     }
@@ -411,26 +648,28 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t k, int64_t 
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, quantize_kernel<true>, x, rows, k, ld, codes, sf, tensor_scale,
+    cudaError_t e = cudaLaunchKernelEx(&cfg, quantize_kernel<true, Out>, x, rows, k, ld, out, tensor_scale,
                                        (const float*)partials, ag);
     count_launch(2);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
-// One-kernel dynamic quantization (see quantize_fused_kernel).  Returns
-// cudaErrorNotSupported when the grid cannot be co-resident (the caller then
-// takes the two-kernel path, which computes the same codes).
-cudaError_t launch_quantize_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes,
-                                  uint8_t* sf, float* tensor_scale, unsigned long long* slots, int max_slots,
-                                  int* dev_status, int num_sms, cudaStream_t stream) {
+// One-kernel form with a data-derived scale (see quantize_fused_kernel).
+// Returns cudaErrorNotSupported when the grid cannot be co-resident (the
+// caller then takes the two-kernel form, which computes the same result).
+template <class Out>
+static cudaError_t launch_one_kernel(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, const Out& out,
+                                     float* tensor_scale, unsigned long long* slots, int max_slots, int* dev_status,
+                                     int num_sms, cudaStream_t stream) {
     static std::atomic<uint32_t> generation{0};
     const int ntiles_c = (int)((k + kTileCols - 1) / kTileCols);
     const int64_t ntiles64 = ((rows + kTileRows - 1) / kTileRows) * ntiles_c;
     if (ntiles64 > (int64_t)1 << 30) return cudaErrorNotSupported;
     const int ntiles = (int)ntiles64;
     int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_fused_kernel, kQuantThreads, 0);
+    cudaError_t e =
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_fused_kernel<Out>, kQuantThreads, 0);
     if (e != cudaSuccess) return e;
     int grid = per_sm * num_sms;
     if (grid > max_slots) grid = max_slots;
@@ -448,7 +687,7 @@ cudaError_t launch_quantize_fused(const uint16_t* x, int64_t rows, int64_t k, in
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, quantize_fused_kernel, x, rows, k, ld, codes, sf, tensor_scale, slots, gen,
+    e = cudaLaunchKernelEx(&cfg, quantize_fused_kernel<Out>, x, rows, k, ld, out, tensor_scale, slots, gen,
                            ntiles_c, ntiles, dev_status);
     if (e == cudaErrorCooperativeLaunchTooLarge) {
         (void)cudaGetLastError();
@@ -457,6 +696,38 @@ cudaError_t launch_quantize_fused(const uint16_t* x, int64_t rows, int64_t k, in
     if (e != cudaSuccess) return e;
     count_launch(1);
     return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes,
+                            uint8_t* sf, float* tensor_scale, bool scale_given, float* partials,
+                            int* dev_status, cudaStream_t stream) {
+    return launch_two_kernel(x, rows, k, ld, CodesOut{codes, sf}, tensor_scale, scale_given, partials, dev_status,
+                             stream);
+}
+
+cudaError_t launch_quantize_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes,
+                                  uint8_t* sf, float* tensor_scale, unsigned long long* slots, int max_slots,
+                                  int* dev_status, int num_sms, cudaStream_t stream) {
+    return launch_one_kernel(x, rows, k, ld, CodesOut{codes, sf}, tensor_scale, slots, max_slots, dev_status,
+                             num_sms, stream);
+}
+
+// Fake quantization: one kernel with a data-derived scale when the grid can
+// be co-resident, else the two-kernel form; one kernel with a given scale.
+cudaError_t launch_fake_quantize(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, void* y, bool y_f32,
+                                 uint8_t* mask, float* tensor_scale, bool scale_given, void* workspace,
+                                 int* dev_status, int num_sms, cudaStream_t stream) {
+    auto run = [&](auto out) -> cudaError_t {
+        if (!scale_given) {
+            const cudaError_t e = launch_one_kernel(x, rows, k, ld, out, tensor_scale,
+                                                    static_cast<unsigned long long*>(workspace), kFusedSlots,
+                                                    dev_status, num_sms, stream);
+            if (e != cudaErrorNotSupported) return e;
+        }
+        return launch_two_kernel(x, rows, k, ld, out, tensor_scale, scale_given, static_cast<float*>(workspace),
+                                 dev_status, stream);
+    };
+    return y_f32 ? run(FakeOut<true>{y, mask}) : run(FakeOut<false>{y, mask});
 }
 
 // ------------------------------------------------------------------ failure-detection check
@@ -493,6 +764,23 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* sf, const flo
         dequantize_kernel<true><<<(unsigned)g, 256, 0, stream>>>(codes, sf, tensor_scale, rows, k, out);
     else
         dequantize_kernel<false><<<(unsigned)g, 256, 0, stream>>>(codes, sf, tensor_scale, rows, k, out);
+    count_launch(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ste_backward(const void* grad_y, const uint8_t* mask, int64_t rows, int64_t k, bool f32,
+                                void* grad_x, int num_sms, cudaStream_t stream) {
+    const int64_t ngroups = rows * (k >> 4);
+    int64_t g = (ngroups + 2 * 256 - 1) / (2 * 256);
+    if (g > (int64_t)num_sms * 16) g = (int64_t)num_sms * 16;
+    if (g < 1) g = 1;
+    const uint4* src = static_cast<const uint4*>(grad_y);
+    const uint16_t* m = reinterpret_cast<const uint16_t*>(mask);
+    uint4* dst = static_cast<uint4*>(grad_x);
+    if (f32)
+        ste_backward_kernel<true><<<(unsigned)g, 256, 0, stream>>>(src, m, ngroups, dst);
+    else
+        ste_backward_kernel<false><<<(unsigned)g, 256, 0, stream>>>(src, m, ngroups, dst);
     count_launch(1);
     return cudaGetLastError();
 }

@@ -32,7 +32,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 11, names
+    assert len(names) == 13, names
     for n in names:
         assert hasattr(L, n), n
         assert n in _lib.SIGNATURES, n
@@ -117,6 +117,32 @@ def test_gemm_rejects_bad_arguments(L):
     assert g(A + 1, B, C, A, B, C, 128, 256, 256, A, 0, None, None, None, None, None, None) == MISALIGNED
     # negative M
     assert g(*args, -1, 256, 256, A, 0, None, None, None, None, None, None) == INVALID
+
+
+def test_fake_quantize_rejects_bad_arguments(L):
+    f = L.nvfp4_fake_quantize
+    # (x, rows, k, ld, y, y_dtype, mask, scale, flags, ws, ws_bytes, dev_status, stream)
+    assert f(A, 128, 96, 96, B, 0, C, A, 1, None, 0, None, None) == SHAPE
+    assert f(None, 128, 256, 256, B, 0, C, A, 1, None, 0, None, None) == INVALID
+    assert f(A, 128, 256, 256, None, 0, C, A, 1, None, 0, None, None) == INVALID
+    assert f(A, 128, 256, 256, B, 3, C, A, 1, None, 0, None, None) == INVALID
+    assert f(A, 128, 256, 256, B, 0, C, None, 1, None, 0, None, None) == INVALID
+    assert f(A, 128, 256, 128, B, 0, C, A, 1, None, 0, None, None) == INVALID
+    assert f(A, 128, 256, 256, B, 0, C, A, 2, None, 0, None, None) == INVALID
+    assert f(A, 128, 256, 256, B, 0, C, A, 0, None, 0, None, None) == WORKSPACE
+    assert f(A, 128, 256, 256, B + 8, 0, C, A, 1, None, 0, None, None) == MISALIGNED
+    assert f(A, 128, 256, 256, B, 0, C + 2, A, 1, None, 0, None, None) == MISALIGNED
+    assert f(A, 128, 256, 260, B, 0, None, A, 1, None, 0, None, None) == MISALIGNED
+
+
+def test_ste_backward_rejects_bad_arguments(L):
+    s = L.nvfp4_ste_backward
+    assert s(A, B, 128, 24, 0, C, None) == SHAPE
+    assert s(A, B, 128, 256, 2, C, None) == INVALID
+    assert s(None, B, 128, 256, 0, C, None) == INVALID
+    assert s(A, None, 128, 256, 0, C, None) == INVALID
+    assert s(A, B, -1, 256, 0, C, None) == INVALID
+    assert s(A, B + 2, 128, 256, 0, C, None) == MISALIGNED
 
 
 def test_w4a16_rejects_bad_arguments(L):
