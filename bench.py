@@ -233,11 +233,21 @@ def reference_points(dev, layers, w4a16_layers):
         out["w4a16"][L.name] = {"shape": f"{L.M}x{L.K}x{L.N}", "ms": round(ms, 4),
                                 "tflops": round(2 * L.M * L.N * L.K / (ms * 1e-3) / 1e12, 1)}
         del x, W, y
-    # quantization-aware training: fake quantization (forward, clip mask
-    # included) and the masked straight-through backward on the fc1 / fc2
-    # inputs; HBM-bound, bytes per element as listed
+    out["qat"] = qat_points(dev, layers)
+    torch.cuda.empty_cache()
+    return out
+
+
+def qat_points(dev, layers):
+    """Quantization-aware training kernels on the fc1 / fc2 inputs (the
+    fake-quantized forward with its clip mask, dynamic and given tensor
+    scale, and the masked straight-through backward); HBM-bound, algorithmic
+    bytes per element as the QAT_* constants state."""
+    import torch
+    import nvfp4_w4a4_gemm_quantize_b200 as nv
+    from nvfp4_w4a4_gemm_quantize_b200 import synth
     hbm = load_peaks()[0].get("hbm_gbs", FALLBACK["hbm_gbs"])
-    out["qat"] = {}
+    res_all = {}
     for name in ("fc1", "fc2"):
         if name not in [L.name for L in layers]:
             continue
@@ -262,10 +272,10 @@ def reference_points(dev, layers, w4a16_layers):
             ms = time_device(fn)
             gbs = bpe * rows * k / (ms * 1e-3) / 1e9
             res[key] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / hbm, 4), "bytes_per_elem": bpe}
-        out["qat"][name] = res
+        res_all[name] = res
         del x, y, m, gx, ws
     torch.cuda.empty_cache()
-    return out
+    return res_all
 
 
 def reduced(wl, args):
@@ -330,6 +340,13 @@ def run_ours(args):
     wl = reduced(synth.WORKLOADS[WORKLOAD], args)
     wl16 = reduced(synth.WORKLOADS["w4a16"], args)
     peaks, peak_src = load_peaks()
+    if args.qat:
+        # profiling aid: only the quantization-aware-training kernels
+        res = qat_points(dev, wl.layers)
+        if rank == 0:
+            print(json.dumps({"qat": res, "peak_gbs": peaks.get("hbm_gbs", FALLBACK["hbm_gbs"]),
+                              "peak_source": peak_src}))
+        return 0
 
     # ---- data (resident in HBM before timing); each rank its own batch
     xs, Ws, Aq, Ys = [], [], [], []
@@ -527,6 +544,7 @@ def main():
     ap.add_argument("--no-reference-points", action="store_true")
     ap.add_argument("--layers", default="", help="profiling: comma-separated subset of layers")
     ap.add_argument("--m", type=int, default=0, help="profiling: tokens (rows of X) per layer")
+    ap.add_argument("--qat", action="store_true", help="profiling: time only the QAT kernels (fc1 / fc2 inputs)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

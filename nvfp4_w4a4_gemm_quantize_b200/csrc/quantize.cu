@@ -211,6 +211,14 @@ __device__ __forceinline__ uint32_t e2m1x2_times_scale(uint32_t byte, uint32_t s
     return e2;
 }
 
+// E4M3 scale byte -> f16 in both halves (exact).
+__device__ __forceinline__ uint32_t e4m3_to_f16x2(uint32_t sfc) {
+    uint32_t sd2;
+    const uint16_t in = (uint16_t)(sfc | (sfc << 8));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(sd2) : "h"(in));
+    return sd2;
+}
+
 // The two halves of an f16x2 as a packed FP32 pair (low half first).
 __device__ __forceinline__ uint64_t f16x2_to_f32x2(uint32_t h2) {
     uint64_t r;
@@ -261,6 +269,46 @@ __device__ __forceinline__ uint32_t bf16x2_round_once_slow(uint64_t e2, float g)
     return out;
 }
 
+// Per-block table of the bf16 results y = RN_bf16(v * e4m3(sf) * g) for the
+// eight E2M1 magnitudes v = 0, 0.5, 1, 1.5, 2, 3, 4, 6 (magnitude code m),
+// as byte planes for prmt lookups: lo0 / lo1 hold the low bytes of entries
+// 0-3 / 4-7, hi0 / hi1 the high bytes.  With b1 = RN_bf16(S) and
+// b3 = RN_bf16(1.5 S), S = e4m3(sf) * g exact, every entry is b1 or b3 times
+// a power of two (v = 2^j or 1.5 * 2^j), and scaling a normal bf16 by 2^j is
+// an exponent add that commutes with rounding -- valid while 0.5 b1 and 4 b3
+// stay normal and finite, i.e. for s in [2^-118, 2^124].
+struct ValueTable {
+    uint32_t lo0, lo1, hi0, hi1;
+};
+
+__device__ __forceinline__ ValueTable value_table(float dec, const ScaleConsts& sc) {
+    const uint64_t g2 = f32x2(sc.g, sc.g), ng2 = f32x2(-sc.g, -sc.g);
+    const uint32_t p = bf16x2_round_once(f32x2(dec, 1.5f * dec), g2, ng2);   // b1 | b3 << 16
+    const uint32_t q01 = (p << 16) - 0x00800000u;      // entries 0, 1: 0, b1 / 2
+    const uint32_t q45 = p + 0x00800080u;              // entries 4, 5: 2 b1, 2 b3
+    const uint32_t q67 = p + 0x01000100u;              // entries 6, 7: 4 b1, 4 b3
+    ValueTable t;
+    asm("prmt.b32 %0, %1, %2, 0x6420;" : "=r"(t.lo0) : "r"(q01), "r"(p));
+    asm("prmt.b32 %0, %1, %2, 0x7531;" : "=r"(t.hi0) : "r"(q01), "r"(p));
+    asm("prmt.b32 %0, %1, %2, 0x6420;" : "=r"(t.lo1) : "r"(q45), "r"(q67));
+    asm("prmt.b32 %0, %1, %2, 0x7531;" : "=r"(t.hi1) : "r"(q45), "r"(q67));
+    return t;
+}
+
+// bf16x2 results of four elements (magnitude codes in the low four nibbles of
+// cm, sign bits cleared), as two words: elements 0, 1 and elements 2, 3; the
+// signs come from the input words (for s > 0 the code keeps the sign of x).
+__device__ __forceinline__ void table_lookup4(const ValueTable& t, uint32_t cm, uint32_t w01, uint32_t w23,
+                                              uint32_t& y01, uint32_t& y23) {
+    uint32_t lo, hi;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(lo) : "r"(t.lo0), "r"(t.lo1), "r"(cm));
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(hi) : "r"(t.hi0), "r"(t.hi1), "r"(cm));
+    asm("prmt.b32 %0, %1, %2, 0x5140;" : "=r"(y01) : "r"(lo), "r"(hi));
+    asm("prmt.b32 %0, %1, %2, 0x7362;" : "=r"(y23) : "r"(lo), "r"(hi));
+    y01 |= w01 & 0x80008000u;
+    y23 |= w23 & 0x80008000u;
+}
+
 // Clip mask of 16 bf16 values (eight words, element 2j in the low half of
 // word j): bit e set where |x_e| > 6 s, s > 0.  For bf16 x, |x| > 6 s exactly
 // iff |x| > RD_bf16(6 s), and RD_bf16(RD_f32(6 s)) = RD_bf16(6 s); as
@@ -270,9 +318,10 @@ __device__ __forceinline__ uint32_t bf16x2_round_once_slow(uint64_t e2, float g)
 __device__ __forceinline__ uint32_t clip_mask16(const uint32_t (&w)[8], float s) {
     const uint32_t tb = s > 0.0f ? (__float_as_uint(__fmul_rd(6.0f, s)) >> 16) + 1u : 0x8000u;
     const uint32_t t2 = tb | (tb << 16);
+    // flags of pair j (bits 15 and 31) move to bits 2j and 16 + 2j
     uint32_t acc = 0u;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc |= (((w[j] | 0x80008000u) - t2) >> 15 & 0x00010001u) << (2 * j);
+    for (int j = 0; j < 8; ++j) acc |= (((w[j] | 0x80008000u) - t2) >> (15 - 2 * j)) & (0x00010001u << (2 * j));
     return (acc & 0x5555u) | ((acc >> 15) & 0xAAAAu);
 }
 
@@ -300,14 +349,10 @@ struct FakeOut {
     }
     __device__ __forceinline__ void emit(const Lane& l, int i, bool ok, const uint32_t (&w)[8], uint32_t sfc,
                                          float s, uint32_t lo, uint32_t hi, const ScaleConsts& sc) const {
-        uint32_t sd2;
-        {
-            const uint16_t in = (uint16_t)(sfc | (sfc << 8));
-            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(sd2) : "h"(in));
-        }
-        const uint64_t g2 = f32x2(sc.g, sc.g);
         const uint32_t codes[2] = {lo, hi};
         if (kF32) {
+            const uint32_t sd2 = e4m3_to_f16x2(sfc);
+            const uint64_t g2 = f32x2(sc.g, sc.g);
             uint32_t o[16];
 #pragma unroll
             for (int h = 0; h < 2; ++h)
@@ -323,15 +368,17 @@ struct FakeOut {
             }
         } else {
             uint32_t o[8];
-            if (s >= 0x1p-118f || s == 0.0f) {
-                const uint64_t ng2 = f32x2(-sc.g, -sc.g);
+            if (s >= 0x1p-118f && s <= 0x1p124f) {
+                const ValueTable tb = value_table(e4m3_to_f32(sfc), sc);
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        o[4 * h + j] = bf16x2_round_once(f16x2_to_f32x2(e2m1x2_times_scale(codes[h] >> (8 * j), sd2)),
-                                                         g2, ng2);
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t cm = codes[h] & 0x77777777u;
+                    table_lookup4(tb, cm, w[4 * h], w[4 * h + 1], o[4 * h], o[4 * h + 1]);
+                    table_lookup4(tb, cm >> 16, w[4 * h + 2], w[4 * h + 3], o[4 * h + 2], o[4 * h + 3]);
+                }
             } else {
+                // tiny, huge or zero block scales: every value rounded exactly
+                const uint32_t sd2 = e4m3_to_f16x2(sfc);
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
 #pragma unroll
