@@ -268,10 +268,16 @@ def qat_points(dev, layers):
             "ste_backward": (lambda: nv.nvfp4_ste_backward(x, m, rows, k, 0, gx), QAT_BWD_BYTES),
         }
         res = {"shape": f"{rows}x{k}"}
+        full = name == "fc2" and rows == 32768
+        traffic_keys = {"fake_quantize_dynamic": "dram_bytes_per_launch_dynamic",
+                        "fake_quantize_given": "dram_bytes_per_launch_given",
+                        "ste_backward": "dram_bytes_per_launch_ste"}
         for key, (fn, bpe) in runs.items():
             ms = time_device(fn)
             gbs = bpe * rows * k / (ms * 1e-3) / 1e9
-            res[key] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / hbm, 4), "bytes_per_elem": bpe}
+            res[key] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / hbm, 4), "bytes_per_elem": bpe,
+                        "traffic": profiled_traffic("fake_quantize_ste_fc2_32768x12288.txt", traffic_keys[key])
+                        if full else None}
         res_all[name] = res
         del x, y, m, gx, ws
     torch.cuda.empty_cache()
@@ -304,10 +310,11 @@ def kernel_source_hash(files=None) -> str:
     return h.hexdigest()
 
 
-def profiled_traffic(summary: str):
+def profiled_traffic(summary: str, key: str = "dram_bytes_per_launch"):
     """DRAM bytes per launch (read + write) from an ncu summary under
-    profiles/, or None when it is absent or was taken on other sources (the
-    summary lists its `source_files` and their `source_sha256`)."""
+    profiles/ (the line `key: <bytes>`), or None when it is absent or was
+    taken on other sources (the summary lists its `source_files` and their
+    `source_sha256`)."""
     p = os.path.join(ROOT, "profiles", summary)
     if not os.path.exists(p):
         return None
@@ -320,7 +327,7 @@ def profiled_traffic(summary: str):
     try:
         if kv.get("source_sha256") != kernel_source_hash(files):
             return None
-        return int(kv["dram_bytes_per_launch"])
+        return int(kv[key])
     except (KeyError, ValueError, OSError):
         return None
 

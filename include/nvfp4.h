@@ -147,7 +147,7 @@ nvfp4_status nvfp4_dequantize(const uint8_t *codes, const uint8_t *sf,
 /*
  * nvfp4_fake_quantize -- fake quantization for quantization-aware training
  * ([DiT] Definition III.1 and Methodology 2, where a straight-through
- * estimator carries gradients through the fake-quantize op): quantization
+ * estimator is used across the fake quantizer in training): quantization
  * exactly as nvfp4_quantize (same tensor-scale rule, block scales and
  * codes), followed in the same kernel by
  *   y = e2m1(code) * e4m3(sf) * g,  rounded once (RNE) to y_dtype,

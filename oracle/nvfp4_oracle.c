@@ -378,8 +378,8 @@ double oracle_gemm_w4a16_at(const uint16_t *x, const uint8_t *w_codes, const uin
 
 /* ----------------------- QAT fake quantization --------------------------- */
 /* Fake quantization for quantization-aware training [DiT, Definition III.1;
- * Methodology 2: a straight-through estimator carries the gradient through
- * the fake-quantize op].  The forward value is the quantizer's output
+ * Methodology 2: training uses a straight-through estimator across the
+ * fake quantizer].  The forward value is the quantizer's output
  *   y = Q_FP4(x; s) = e2m1(code) * dec(sf) * g,  rounded once to bf16 or f32,
  * with the codes and scales oracle_quantize_bf16 makes (same tensor-scale
  * rule, g_io in/out), and the clip indicator that the estimator's backward
