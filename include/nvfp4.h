@@ -214,6 +214,44 @@ nvfp4_status nvfp4_gemm_w4a4(const uint8_t *a_codes, const uint8_t *a_sf, const 
                              int *dev_status, nvfp4_stream_t stream);
 
 /*
+ * nvfp4_gemm_w4a4_grouped -- up to NVFP4_MAX_GROUP independent W4A4 products
+ * in one persistent launch (the product of each is nvfp4_gemm_w4a4's): the
+ * linear layers of a transformer block that do not depend on each other --
+ * e.g. the self-attention QKV projection of the image tokens and the
+ * cross-attention K and V projections of the text tokens, which have
+ * different M, N and K -- share one tile scheduler, so the small ones do not
+ * each pay a launch and a partly idle wave.  ([DiT] Methodology 3 runs every
+ * linear layer through the FP4-packed matmul.)
+ * problems   HOST array of `count` (1 .. NVFP4_MAX_GROUP) descriptions; each
+ *            field means what the argument of the same name of
+ *            nvfp4_gemm_w4a4 means and is checked the same way.  Every problem
+ *            has the same output kind: all y != NULL (then y_dtype applies to
+ *            all), or all y == NULL with NVFP4 outputs (y_codes, y_sf, y_scale,
+ *            optional y_amax).  Problems with M == 0 are skipped.
+ * One launch of the single-CTA kernel (128 x 128 tiles) for any N; the
+ * array is read during the call only.
+ */
+typedef struct {
+    const uint8_t *a_codes;
+    const uint8_t *a_sf;
+    const float *a_scale;
+    const uint8_t *b_codes;
+    const uint8_t *b_sf;
+    const float *b_scale;
+    int64_t M, N, K;
+    void *y;
+    uint8_t *y_codes;
+    uint8_t *y_sf;
+    const float *y_scale;
+    float *y_amax;
+} nvfp4_gemm_problem;
+
+enum { NVFP4_MAX_GROUP = 8 };
+
+nvfp4_status nvfp4_gemm_w4a4_grouped(const nvfp4_gemm_problem *problems, int count, int y_dtype,
+                                     int *dev_status, nvfp4_stream_t stream);
+
+/*
  * nvfp4_gemm_w4a16 -- weights-only NVFP4 ([RFC] Open Questions 1, W4A16):
  *   Y[m,n] = g_w * sum_k x[m,k] * (e2m1(w[n,k]) * e4m3(sfw))
  * The weight element e2m1 * e4m3 is exact in bf16; it is formed in shared

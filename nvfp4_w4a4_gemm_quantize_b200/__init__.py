@@ -8,18 +8,19 @@ memory and streams.
 Low-level (same names and argument order as the C calls):
     nvfp4_sf_bytes, nvfp4_quantize_workspace_bytes, nvfp4_quantize,
     nvfp4_quantize_noalloc, nvfp4_dequantize, nvfp4_fake_quantize, nvfp4_ste_backward,
-    nvfp4_gemm_w4a4, nvfp4_gemm_w4a16, nvfp4_launch_count
+    nvfp4_gemm_w4a4, nvfp4_gemm_w4a4_grouped, nvfp4_gemm_w4a16, nvfp4_launch_count
 Convenience (allocate outputs with torch, then call the above):
-    NVFP4Tensor, quantize, dequantize, gemm_w4a4, gemm_w4a16,
+    NVFP4Tensor, quantize, dequantize, gemm_w4a4, gemm_w4a4_grouped, gemm_w4a16,
     fake_quantize, ste_backward, FakeQuantizeSTE (autograd: the two kernels)
 """
 from __future__ import annotations
 
+import ctypes
 from dataclasses import dataclass
 
 import torch
 
-from ._lib import NVFP4Error, check, lib  # noqa: F401
+from ._lib import MAX_GROUP, NVFP4Error, NVFP4GemmProblem, check, lib  # noqa: F401
 
 NVFP4_DTYPE_BF16 = 0
 NVFP4_DTYPE_F32 = 1
@@ -115,6 +116,19 @@ def nvfp4_gemm_w4a4(a_codes, a_sf, a_scale, b_codes, b_sf, b_scale, M, N, K, y=N
     check(st, "nvfp4_gemm_w4a4")
 
 
+def nvfp4_gemm_w4a4_grouped(problems, y_dtype=NVFP4_DTYPE_BF16, dev_status=None, stream=None) -> None:
+    """``problems``: a list of dicts with the fields of nvfp4_gemm_problem
+    (tensors or None for the pointers, ints for M, N, K)."""
+    arr = (NVFP4GemmProblem * len(problems))()
+    for i, d in enumerate(problems):
+        for name, _ in NVFP4GemmProblem._fields_:
+            v = d.get(name)
+            setattr(arr[i], name, int(v) if name in ("M", "N", "K") else _ptr(v))
+    st = lib().nvfp4_gemm_w4a4_grouped(ctypes.addressof(arr), len(problems), y_dtype, _ptr(dev_status),
+                                       _stream(stream))
+    check(st, "nvfp4_gemm_w4a4_grouped")
+
+
 def nvfp4_gemm_w4a16(x, w_codes, w_sf, w_scale, M, N, K, y, y_dtype=NVFP4_DTYPE_BF16,
                      dev_status=None, stream=None) -> None:
     st = lib().nvfp4_gemm_w4a16(_ptr(x), _ptr(w_codes), _ptr(w_sf), _ptr(w_scale), M, N, K, _ptr(y),
@@ -187,6 +201,20 @@ def gemm_w4a4_nvfp4_out(a: NVFP4Tensor, b: NVFP4Tensor, y_scale: torch.Tensor, y
                     y_codes=q.codes, y_sf=q.sf, y_scale=q.scale, y_amax=y_amax, dev_status=dev_status,
                     stream=stream)
     return q
+
+
+def gemm_w4a4_grouped(pairs, out_dtype=torch.bfloat16, dev_status=None, stream=None) -> list:
+    """Y_i = A_i B_i^T for up to MAX_GROUP independent (A_i, B_i) NVFP4 pairs in
+    one launch; returns the outputs in order."""
+    ys, probs = [], []
+    for a, b in pairs:
+        assert a.k == b.k
+        y = torch.empty(a.rows, b.rows, dtype=out_dtype, device=a.codes.device)
+        ys.append(y)
+        probs.append(dict(a_codes=a.codes, a_sf=a.sf, a_scale=a.scale, b_codes=b.codes, b_sf=b.sf,
+                          b_scale=b.scale, M=a.rows, N=b.rows, K=a.k, y=y))
+    nvfp4_gemm_w4a4_grouped(probs, _DT[out_dtype], dev_status, stream)
+    return ys
 
 
 def gemm_w4a16(x: torch.Tensor, w: NVFP4Tensor, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,

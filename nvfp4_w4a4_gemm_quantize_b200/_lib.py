@@ -26,6 +26,16 @@ STATUS = {
     6: "NVFP4_ERR_TIMEOUT", 7: "NVFP4_ERR_WORKSPACE", 8: "NVFP4_ERR_NONFINITE",
 }
 
+class NVFP4GemmProblem(ctypes.Structure):
+    """nvfp4_gemm_problem (include/nvfp4.h): one product of a grouped call."""
+    _fields_ = [("a_codes", _p), ("a_sf", _p), ("a_scale", _p),
+                ("b_codes", _p), ("b_sf", _p), ("b_scale", _p),
+                ("M", _i64), ("N", _i64), ("K", _i64),
+                ("y", _p), ("y_codes", _p), ("y_sf", _p), ("y_scale", _p), ("y_amax", _p)]
+
+
+MAX_GROUP = 8
+
 # every symbol include/nvfp4.h declares, with (restype, argtypes)
 SIGNATURES = {
     "nvfp4_sf_bytes": (ctypes.c_size_t, [_i64, _i64]),
@@ -37,6 +47,7 @@ SIGNATURES = {
                                       _p, _p]),
     "nvfp4_ste_backward": (_status, [_p, _p, _i64, _i64, _int, _p, _p]),
     "nvfp4_gemm_w4a4": (_status, [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _p, _int, _p, _p, _p, _p, _p, _p]),
+    "nvfp4_gemm_w4a4_grouped": (_status, [_p, _int, _int, _p, _p]),
     "nvfp4_gemm_w4a16": (_status, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _int, _p, _p]),
     "nvfp4_status_string": (ctypes.c_char_p, [_int]),
     "nvfp4_launch_count": (ctypes.c_uint64, []),

@@ -190,13 +190,14 @@ nvfp4_status nvfp4_ste_backward(const void* grad_y, const uint8_t* clip_mask, in
                                            reinterpret_cast<cudaStream_t>(stream)));
 }
 
-nvfp4_status nvfp4_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_scale,
-                             const uint8_t* b_codes, const uint8_t* b_sf, const float* b_scale, int64_t M, int64_t N,
-                             int64_t K, void* y, int y_dtype, uint8_t* y_codes, uint8_t* y_sf, const float* y_scale,
-                             float* y_amax, int* dev_status, nvfp4_stream_t stream) {
+// Checks of one W4A4 problem (shared by the single and the grouped call).
+static nvfp4_status check_gemm_problem(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_scale,
+                                       const uint8_t* b_codes, const uint8_t* b_sf, const float* b_scale, int64_t M,
+                                       int64_t N, int64_t K, const void* y, int y_dtype, const uint8_t* y_codes,
+                                       const uint8_t* y_sf, const float* y_scale) {
     if (M < 0 || N <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
     if (K % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (M == 0) return NVFP4_OK;                 /* nothing to read or write */
+    if (M == 0) return NVFP4_OK;
     if (!a_codes || !a_sf || !b_codes || !b_sf || !a_scale || !b_scale) return NVFP4_ERR_INVALID_ARG;
     if (y) {
         if (y_dtype != NVFP4_DTYPE_BF16 && y_dtype != NVFP4_DTYPE_F32) return NVFP4_ERR_INVALID_ARG;
@@ -204,21 +205,55 @@ nvfp4_status nvfp4_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_sf, const 
     } else {
         if (!y_codes || !y_sf || !y_scale) return NVFP4_ERR_INVALID_ARG;
     }
-    if (K % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (y && y_dtype == NVFP4_DTYPE_BF16 && N % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (y && y_dtype == NVFP4_DTYPE_F32 && N % 4 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (!y && N % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (M >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31))
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(b_codes) || !aligned16(b_sf) ||
-        (y && !aligned16(y)) || (y_codes && !aligned16(y_codes)) || (y_sf && !aligned16(y_sf)))
+    if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(b_codes) || !aligned16(b_sf) || (y && !aligned16(y)) ||
+        (y_codes && !aligned16(y_codes)) || (y_sf && !aligned16(y_sf)))
         return NVFP4_ERR_MISALIGNED;
+    return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_scale,
+                             const uint8_t* b_codes, const uint8_t* b_sf, const float* b_scale, int64_t M, int64_t N,
+                             int64_t K, void* y, int y_dtype, uint8_t* y_codes, uint8_t* y_sf, const float* y_scale,
+                             float* y_amax, int* dev_status, nvfp4_stream_t stream) {
+    const nvfp4_status chk = check_gemm_problem(a_codes, a_sf, a_scale, b_codes, b_sf, b_scale, M, N, K, y, y_dtype,
+                                                y_codes, y_sf, y_scale);
+    if (chk != NVFP4_OK) return chk;
+    if (M == 0) return NVFP4_OK;                 /* nothing to read or write */
     int sms = 0;
     nvfp4_status st = device_ok(&sms);
     if (st != NVFP4_OK) return st;
     GemmW4A4Args a{a_codes, a_sf, a_scale, b_codes, b_sf, b_scale, M, N, K, y, y_dtype,
                    y_codes, y_sf, y_scale, y_amax, dev_status};
     return cuda_status(launch_gemm_w4a4(a, sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_gemm_w4a4_grouped(const nvfp4_gemm_problem* problems, int count, int y_dtype, int* dev_status,
+                                     nvfp4_stream_t stream) {
+    if (!problems || count < 1 || count > NVFP4_MAX_GROUP) return NVFP4_ERR_INVALID_ARG;
+    if (NVFP4_MAX_GROUP > gemm_w4a4_max_group()) return NVFP4_ERR_INVALID_ARG;
+    const bool nvfp4_out = problems[0].y == nullptr;
+    GemmW4A4Args args[NVFP4_MAX_GROUP];
+    int n = 0;
+    for (int i = 0; i < count; ++i) {
+        const nvfp4_gemm_problem& q = problems[i];
+        if ((q.y == nullptr) != nvfp4_out) return NVFP4_ERR_INVALID_ARG;   // one output kind per launch
+        const nvfp4_status st = check_gemm_problem(q.a_codes, q.a_sf, q.a_scale, q.b_codes, q.b_sf, q.b_scale, q.M,
+                                                   q.N, q.K, q.y, y_dtype, q.y_codes, q.y_sf, q.y_scale);
+        if (st != NVFP4_OK) return st;
+        if (q.M == 0) continue;                  // nothing to read or write
+        args[n++] = GemmW4A4Args{q.a_codes, q.a_sf, q.a_scale, q.b_codes, q.b_sf, q.b_scale, q.M, q.N, q.K,
+                                 q.y, y_dtype, q.y_codes, q.y_sf, q.y_scale, q.y_amax, dev_status};
+    }
+    int sms = 0;
+    nvfp4_status st = device_ok(&sms);
+    if (st != NVFP4_OK) return st;
+    if (n == 0) return NVFP4_OK;
+    return cuda_status(launch_gemm_w4a4_grouped(args, n, sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 nvfp4_status nvfp4_gemm_w4a16(const void* x_bf16, const uint8_t* w_codes, const uint8_t* w_sf, const float* w_scale,

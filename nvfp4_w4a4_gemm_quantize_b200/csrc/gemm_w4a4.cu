@@ -8,6 +8,12 @@
 // Diffusion Models", Open Questions 1: W4A4):
 //   Y[m,n] = (g_a g_b) * sum_k (e2m1(a) e4m3(sfa)) (e2m1(b) e4m3(sfb))
 //
+// One launch may carry up to kMaxGroup independent problems (a grouped GEMM:
+// e.g. a block's QKV projection and its cross-attention K and V projections,
+// each with its own operands, shape and output); their tiles form one tile
+// space that the persistent CTAs walk, each tile finding its problem from the
+// problems' first-tile indices.  A plain call is a group of one.
+//
 // Kernel shape (one CTA per SM, persistent over output tiles):
 //   warp 0      TMA producer: code tiles (tensor maps, 128-byte swizzle) and
 //               scale atoms (bulk copies) into a STAGES-deep shared ring.
@@ -19,6 +25,8 @@
 // Tile: 128 (M) x BN (N) x 256 (K per stage).  TMEM: 512 columns, the
 // accumulator(s) in [0, 256) (two buffers when BN = 128 so the epilogue of
 // one tile overlaps the mainloop of the next), the scale ring in [256, 512).
+#include <cstring>
+
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -59,19 +67,41 @@ struct Cfg {
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-struct Params {
+constexpr int kMaxGroup = 8;
+
+struct Problem {
     const uint8_t* a_sf;
     const uint8_t* b_sf;
     const float* a_scale;
     const float* b_scale;
-    int M, N, K;
-    int num_mb, num_nb, num_tiles;
     uint8_t* y_codes;
     uint8_t* y_sf;
     const float* y_scale;
     float* y_amax;
+    int M, N, K;
+    int num_mb, num_nb, tile0;                   // tiles [tile0, tile0 + num_mb * num_nb)
+};
+
+struct Params {
+    Problem pr[kMaxGroup];
+    int count, num_tiles;
     int* dev_status;
 };
+
+// Tensor maps of every problem: A codes, B codes, Y (bf16 / FP32 output).
+struct Maps {
+    CUtensorMap a[kMaxGroup], b[kMaxGroup], y[kMaxGroup];
+};
+static_assert(sizeof(Maps) + sizeof(Params) <= 4096, "kernel parameters");
+
+// Problem of global tile t (problems are in tile order).
+__device__ __forceinline__ int find_problem(const Params& p, int t) {
+    int g = 0;
+#pragma unroll 1
+    for (int i = 1; i < p.count; ++i)
+        if (t >= p.pr[i].tile0) g = i;
+    return g;
+}
 
 __device__ __forceinline__ void tile_coords(int t, int num_mb, int num_nb, int& mb, int& nb) {
     const int per_group = kGroupM * num_nb;
@@ -83,10 +113,17 @@ __device__ __forceinline__ void tile_coords(int t, int num_mb, int num_nb, int& 
     nb = idx / gm;
 }
 
+// Warp-wide maximum of a non-negative running |y| maximum, merged into the
+// caller's device float (atomic max on the bit pattern: order-preserving for
+// non-negative floats).  Whole warp; a null destination is skipped.
+__device__ __forceinline__ void flush_amax(float v, float* dst, int lane) {
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (dst != nullptr && lane == 0 && v > 0.0f) atomicMax(reinterpret_cast<int*>(dst), __float_as_int(v));
+}
+
 template <int BN, int STAGES, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
-gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-            const __grid_constant__ CUtensorMap tmap_y, const Params p) {
+gemm_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p) {
     using C = Cfg<BN, STAGES>;
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES];
@@ -111,9 +148,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
         }
         mbar_init(&drain_bar, 1);
         fence_barrier_init();
-        tma_prefetch_desc(&tmap_a);
-        tma_prefetch_desc(&tmap_b);
-        tma_prefetch_desc(&tmap_y);
+        for (int g = 0; g < p.count; ++g) {
+            tma_prefetch_desc(&maps.a[g]);
+            tma_prefetch_desc(&maps.b[g]);
+            if (OUT != OUT_NVFP4) tma_prefetch_desc(&maps.y[g]);
+        }
     }
     // Scale bytes of absent 128-row blocks are never loaded; zero every scale
     // region once so such rows read finite scales (their codes are zero).
@@ -131,8 +170,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_sh;
 
-    const int num_kt = (p.K + 255) / 256;
-    const int k_atoms = p.K / 64;                 // scale atoms per 128-row block
 
     // Producer and MMA issuer run on whole warps with one elected lane issuing,
     // so descriptors, coordinates and addresses stay warp-uniform (from a
@@ -147,10 +184,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
         uint32_t issued_any = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+            const int g = find_problem(p, t);
+            const Problem& pr = p.pr[g];
             int mb, nb;
-            tile_coords(t, p.num_mb, p.num_nb, mb, nb);
+            tile_coords(t - pr.tile0, pr.num_mb, pr.num_nb, mb, nb);
             const int nblk0 = nb * (BN / 128);
-            const int nblk_total = (p.N + 127) / 128;
+            const int nblk_total = (pr.N + 127) / 128;
+            const int num_kt = (pr.K + 255) / 256;
+            const int k_atoms = pr.K / 64;        // scale atoms per 128-row block
             for (int kt = 0; kt < num_kt; ++kt) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&empty_bar[stage], phase ^ 1u, wc) ? 1 : 0)) {
                     ok = false;
@@ -163,14 +204,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
                 if (elect_one()) {
                     const uint32_t bytes = A_BYTES + C::B_BYTES + natoms * SF_ATOM * (1 + nsfb);
                     mbar_arrive_expect_tx(&full_bar[stage], bytes);
-                    tma_load_2d(sbase, &tmap_a, &full_bar[stage], kt * BK_BYTES, mb * BM, pol_a);
-                    tma_load_2d(sbase + A_BYTES, &tmap_b, &full_bar[stage], kt * BK_BYTES, nb * BN, pol_b);
+                    tma_load_2d(sbase, &maps.a[g], &full_bar[stage], kt * BK_BYTES, mb * BM, pol_a);
+                    tma_load_2d(sbase + A_BYTES, &maps.b[g], &full_bar[stage], kt * BK_BYTES, nb * BN, pol_b);
                     bulk_load(sbase + A_BYTES + C::B_BYTES,
-                              p.a_sf + ((int64_t)mb * k_atoms + kt * 4) * SF_ATOM, natoms * SF_ATOM,
+                              pr.a_sf + ((int64_t)mb * k_atoms + kt * 4) * SF_ATOM, natoms * SF_ATOM,
                               &full_bar[stage], pol_a);
                     for (int j = 0; j < nsfb; ++j)
                         bulk_load(sbase + A_BYTES + C::B_BYTES + SFA_BYTES + j * SFA_BYTES,
-                                  p.b_sf + ((int64_t)(nblk0 + j) * k_atoms + kt * 4) * SF_ATOM,
+                                  pr.b_sf + ((int64_t)(nblk0 + j) * k_atoms + kt * 4) * SF_ATOM,
                                   natoms * SF_ATOM, &full_bar[stage], pol_b);
                 }
                 __syncwarp();
@@ -205,6 +246,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
                 break;
             }
             tc_fence_after();
+            const Problem& pr = p.pr[find_problem(p, t)];
+            const int num_kt = (pr.K + 255) / 256;
+            const int k_atoms = pr.K / 64;
             const uint32_t d_tmem = tmem_base + acc * BN;
             for (int kt = 0; kt < num_kt; ++kt) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[stage], phase, wc) ? 1 : 0)) {
@@ -249,18 +293,29 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;                       // TMEM lane quarter
         const int row_t = q * 32 + lane;              // row inside the tile
-        const float alpha = __fmul_rn(*p.a_scale, *p.b_scale);
-        float g_y = 0.0f;
-        if (OUT == OUT_NVFP4) g_y = *p.y_scale;
-        const ScaleConsts sc_y = scale_consts(g_y);
         uint8_t* ebuf = smem + STAGES * C::STAGE_BYTES + (warp - 2) * 2 * C::EPI_BUF_BYTES;
         int acc = 0;
         uint32_t acc_phase = 0;
         int nstore = 0;
-        float amax_run = 0.0f;
+        int g_prev = -1;
+        float alpha = 0.0f, g_y = 0.0f, amax_run = 0.0f;
+        ScaleConsts sc_y = scale_consts(0.0f);
         for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+            const int g = find_problem(p, t);
+            const Problem& pr = p.pr[g];
+            if (g != g_prev) {
+                // a new problem: flush the previous one's running amax, load this one's scales
+                if (OUT == OUT_NVFP4 && g_prev >= 0) flush_amax(amax_run, p.pr[g_prev].y_amax, lane);
+                amax_run = 0.0f;
+                alpha = __fmul_rn(*pr.a_scale, *pr.b_scale);
+                if (OUT == OUT_NVFP4) {
+                    g_y = *pr.y_scale;
+                    sc_y = scale_consts(g_y);
+                }
+                g_prev = g;
+            }
             int mb, nb;
-            tile_coords(t, p.num_mb, p.num_nb, mb, nb);
+            tile_coords(t - pr.tile0, pr.num_mb, pr.num_nb, mb, nb);
             // warp-uniform decision: the TMEM loads below are .sync.aligned
             if (!__all_sync(0xffffffffu, mbar_wait(&accf_bar[acc], acc_phase, wc) ? 1 : 0)) break;
             tc_fence_after();
@@ -268,14 +323,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
             const int m0 = mb * BM, n0 = nb * BN;
             if (OUT == OUT_NVFP4) {
                 const int64_t grow = (int64_t)m0 + row_t;
-                const int kb4 = p.N / 64;
+                const int kb4 = pr.N / 64;
                 for (int c = 0; c < BN / 64; ++c) {
                     const int ncol = n0 + c * 64;
                     uint32_t r0[32], r1[32];
                     tmem_ld_32x32b_x32(tbase + c * 64, r0);
                     tmem_ld_32x32b_x32(tbase + c * 64 + 32, r1);
                     tmem_ld_wait();
-                    if (ncol >= p.N) continue;
+                    if (ncol >= pr.N) continue;
                     uint32_t sfw = 0u;
                     uint32_t cw[8];
 #pragma unroll
@@ -289,7 +344,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
                         float ab = 0.0f;
 #pragma unroll
                         for (int j = 0; j < 16; ++j) ab = fmaxf(ab, fabsf(v[j]));
-                        if (grow < p.M) amax_run = fmaxf(amax_run, ab);
+                        if (grow < pr.M) amax_run = fmaxf(amax_run, ab);
                         const uint32_t sfc = block_scale_code(ab, sc_y);
                         const float s = __fmul_rn(e4m3_to_f32(sfc), g_y);
                         float lo[8], hi[8];
@@ -299,20 +354,20 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
                         cw[2 * b + 1] = quantize8(hi, s);
                         sfw |= sfc << (8 * b);
                     }
-                    if (grow < p.M) {
-                        uint4* dst = reinterpret_cast<uint4*>(p.y_codes + grow * (p.N / 2) + ncol / 2);
+                    if (grow < pr.M) {
+                        uint4* dst = reinterpret_cast<uint4*>(pr.y_codes + grow * (pr.N / 2) + ncol / 2);
                         dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
                         dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
                     }
                     const int64_t atom = (int64_t)mb * kb4 + ncol / 64;
-                    *reinterpret_cast<uint32_t*>(p.y_sf + atom * SF_ATOM + (row_t & 31) * 16 + (row_t >> 5) * 4) = sfw;
+                    *reinterpret_cast<uint32_t*>(pr.y_sf + atom * SF_ATOM + (row_t & 31) * 16 + (row_t >> 5) * 4) = sfw;
                 }
             } else {
                 for (int c = 0; c < BN / 32; ++c) {
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(tbase + c * 32, r);
                     tmem_ld_wait();
-                    if (n0 + c * 32 >= p.N) continue;
+                    if (n0 + c * 32 >= pr.N) continue;
                     uint8_t* buf = ebuf + (nstore & 1) * C::EPI_BUF_BYTES;
                     // the store that last used this buffer has finished reading it
                     if (lane == 0) bulk_wait_group_read<1>();
@@ -347,7 +402,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_2d(&tmap_y, buf, n0 + c * 32, m0 + q * 32);
+                        tma_store_2d(&maps.y[g], buf, n0 + c * 32, m0 + q * 32);
                         bulk_commit_group();
                     }
                     ++nstore;
@@ -360,11 +415,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
             if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
         }
         if (lane == 0) bulk_wait_group<0>();
-        if (OUT == OUT_NVFP4 && p.y_amax != nullptr) {
-            for (int o = 16; o > 0; o >>= 1) amax_run = fmaxf(amax_run, __shfl_xor_sync(0xffffffffu, amax_run, o));
-            if (lane == 0 && amax_run > 0.0f)
-                atomicMax(reinterpret_cast<int*>(p.y_amax), __float_as_int(amax_run));
-        }
+        if (OUT == OUT_NVFP4 && g_prev >= 0) flush_amax(amax_run, p.pr[g_prev].y_amax, lane);
     }
 
     tc_fence_before();
@@ -377,51 +428,65 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
 }
 
 template <int BN, int STAGES, int OUT>
-cudaError_t launch_cfg(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) {
+cudaError_t launch_cfg(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream) {
     using C = Cfg<BN, STAGES>;
-    CUtensorMap ta, tb, ty;
-    CUresult r;
-    r = make_tmap_2d(&ta, a.a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)(a.K / 2), (uint64_t)a.M,
-                     (uint64_t)(a.K / 2), BK_BYTES, BM, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    r = make_tmap_2d(&tb, a.b_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)(a.K / 2), (uint64_t)a.N,
-                     (uint64_t)(a.K / 2), BK_BYTES, BN, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    if (OUT == OUT_BF16) {
-        r = make_tmap_2d(&ty, a.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.N, (uint64_t)a.M,
-                         (uint64_t)a.N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
-    } else if (OUT == OUT_F32) {
-        r = make_tmap_2d(&ty, a.y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)a.N, (uint64_t)a.M,
-                         (uint64_t)a.N * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
-    } else {
-        ty = ta;   // unused by the NVFP4 epilogue
-    }
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-
+    if (count < 1 || count > kMaxGroup) return cudaErrorInvalidValue;
+    Maps maps;
     Params p;
-    p.a_sf = a.a_sf;
-    p.b_sf = a.b_sf;
-    p.a_scale = a.a_scale;
-    p.b_scale = a.b_scale;
-    p.M = (int)a.M;
-    p.N = (int)a.N;
-    p.K = (int)a.K;
-    p.num_mb = (int)((a.M + BM - 1) / BM);
-    p.num_nb = (int)((a.N + BN - 1) / BN);
-    p.num_tiles = p.num_mb * p.num_nb;
-    p.y_codes = a.y_codes;
-    p.y_sf = a.y_sf;
-    p.y_scale = a.y_scale;
-    p.y_amax = a.y_amax;
-    p.dev_status = a.dev_status;
+    memset(&maps, 0, sizeof(maps));
+    memset(&p, 0, sizeof(p));
+    int tiles = 0;
+    for (int g = 0; g < count; ++g) {
+        const GemmW4A4Args& a = probs[g];
+        CUresult r;
+        r = make_tmap_2d(&maps.a[g], a.a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)(a.K / 2),
+                         (uint64_t)(a.M > 0 ? a.M : 1), (uint64_t)(a.K / 2), BK_BYTES, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+        r = make_tmap_2d(&maps.b[g], a.b_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)(a.K / 2), (uint64_t)a.N,
+                         (uint64_t)(a.K / 2), BK_BYTES, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+        if (OUT == OUT_BF16) {
+            r = make_tmap_2d(&maps.y[g], a.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.N,
+                             (uint64_t)(a.M > 0 ? a.M : 1), (uint64_t)a.N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+        } else if (OUT == OUT_F32) {
+            r = make_tmap_2d(&maps.y[g], a.y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)a.N,
+                             (uint64_t)(a.M > 0 ? a.M : 1), (uint64_t)a.N * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+        }
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+        Problem& pr = p.pr[g];
+        pr.a_sf = a.a_sf;
+        pr.b_sf = a.b_sf;
+        pr.a_scale = a.a_scale;
+        pr.b_scale = a.b_scale;
+        pr.y_codes = a.y_codes;
+        pr.y_sf = a.y_sf;
+        pr.y_scale = a.y_scale;
+        pr.y_amax = a.y_amax;
+        pr.M = (int)a.M;
+        pr.N = (int)a.N;
+        pr.K = (int)a.K;
+        pr.num_mb = (int)((a.M + BM - 1) / BM);
+        pr.num_nb = (int)((a.N + BN - 1) / BN);
+        pr.tile0 = tiles;
+        tiles += pr.num_mb * pr.num_nb;          // M == 0: no tiles
+    }
+    p.count = count;
+    p.num_tiles = tiles;
+    p.dev_status = probs[0].dev_status;
+    if (tiles == 0) return cudaSuccess;
 
     auto kern = gemm_kernel<BN, STAGES, OUT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
-    kern<<<grid, kThreads, C::SMEM_BYTES, stream>>>(ta, tb, ty, p);
+    const int grid = tiles < num_sms ? tiles : num_sms;
+    kern<<<grid, kThreads, C::SMEM_BYTES, stream>>>(maps, p);
     count_launch(1);
     return cudaGetLastError();
+}
+
+template <int OUT>
+static cudaError_t launch_group(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream) {
+    return launch_cfg<128, 5, OUT>(probs, count, num_sms, stream);
 }
 
 }  // namespace w4a4
@@ -433,10 +498,19 @@ cudaError_t launch_gemm_w4a4(const GemmW4A4Args& a, int num_sms, cudaStream_t st
     // (N = 1152, 3456, ...): single-CTA 128 x 128 tiles with a double-buffered
     // accumulator, so no tile column is wasted on padding.
     if (a.N % 256 == 0) return launch_gemm_w4a4_2sm(a, num_sms, stream);
-    const int out = a.y != nullptr ? (a.y_dtype == 1 ? OUT_F32 : OUT_BF16) : OUT_NVFP4;
-    if (out == OUT_BF16) return launch_cfg<128, 5, OUT_BF16>(a, num_sms, stream);
-    if (out == OUT_F32) return launch_cfg<128, 5, OUT_F32>(a, num_sms, stream);
-    return launch_cfg<128, 5, OUT_NVFP4>(a, num_sms, stream);
+    return launch_gemm_w4a4_grouped(&a, 1, num_sms, stream);
 }
+
+// Up to kMaxGroup problems in one launch of the single-CTA kernel; every
+// problem has the same output kind (bf16, FP32 or NVFP4).
+cudaError_t launch_gemm_w4a4_grouped(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream) {
+    using namespace w4a4;
+    const int out = probs[0].y != nullptr ? (probs[0].y_dtype == 1 ? OUT_F32 : OUT_BF16) : OUT_NVFP4;
+    if (out == OUT_BF16) return launch_group<OUT_BF16>(probs, count, num_sms, stream);
+    if (out == OUT_F32) return launch_group<OUT_F32>(probs, count, num_sms, stream);
+    return launch_group<OUT_NVFP4>(probs, count, num_sms, stream);
+}
+
+int gemm_w4a4_max_group() { return w4a4::kMaxGroup; }
 
 }  // namespace nvfp4

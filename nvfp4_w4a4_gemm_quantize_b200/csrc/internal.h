@@ -57,6 +57,8 @@ struct GemmW4A4Args {
 };
 
 cudaError_t launch_gemm_w4a4(const GemmW4A4Args& a, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemm_w4a4_grouped(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream);
+int gemm_w4a4_max_group();
 cudaError_t launch_gemm_w4a4_2sm(const GemmW4A4Args& a, int num_sms, cudaStream_t stream);
 
 struct GemmW4A16Args {

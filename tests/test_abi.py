@@ -32,7 +32,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 13, names
+    assert len(names) == 14, names
     for n in names:
         assert hasattr(L, n), n
         assert n in _lib.SIGNATURES, n
@@ -143,6 +143,40 @@ def test_ste_backward_rejects_bad_arguments(L):
     assert s(A, None, 128, 256, 0, C, None) == INVALID
     assert s(A, B, -1, 256, 0, C, None) == INVALID
     assert s(A, B + 2, 128, 256, 0, C, None) == MISALIGNED
+
+
+def _problems(n, over=None):
+    arr = (_lib.NVFP4GemmProblem * n)()
+    for i in range(n):
+        pr = arr[i]
+        pr.a_codes, pr.a_sf, pr.a_scale, pr.b_codes, pr.b_sf, pr.b_scale = A, B, C, A, B, C
+        pr.M, pr.N, pr.K, pr.y = 128, 256, 256, A
+        for k, v in (over or {}).get(i, {}).items():
+            setattr(pr, k, v)
+    return arr
+
+
+def test_grouped_gemm_rejects_bad_arguments(L):
+    g = L.nvfp4_gemm_w4a4_grouped
+    addr = ctypes.addressof
+    assert g(None, 1, 0, None, None) == INVALID
+    arr = _problems(9)
+    assert g(addr(arr), 0, 0, None, None) == INVALID
+    assert g(addr(arr), 9, 0, None, None) == INVALID
+    assert g(addr(arr), 2, 7, None, None) == INVALID                                 # bad dtype
+    # mixed output kinds in one launch
+    arr = _problems(2, {1: dict(y=None, y_codes=A, y_sf=B, y_scale=C)})
+    assert g(addr(arr), 2, 0, None, None) == INVALID
+    arr = _problems(3, {2: dict(K=96)})
+    assert g(addr(arr), 3, 0, None, None) == SHAPE
+    arr = _problems(2, {1: dict(N=260)})
+    assert g(addr(arr), 2, 0, None, None) == SHAPE
+    arr = _problems(2, {0: dict(a_codes=A + 4)})
+    assert g(addr(arr), 2, 0, None, None) == MISALIGNED
+    arr = _problems(2, {1: dict(b_scale=None)})
+    assert g(addr(arr), 2, 0, None, None) == INVALID
+    arr = _problems(2, {0: dict(M=-1)})
+    assert g(addr(arr), 2, 0, None, None) == INVALID
 
 
 def test_w4a16_rejects_bad_arguments(L):
