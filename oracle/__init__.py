@@ -27,6 +27,9 @@ Parity status per function:
       of saturating elements)
   ste_backward                                          -- pinned (closed form
       through numpy's bit unpacking)
+  gelu_tanh                                             -- pinned (torch's
+      float64 tanh-form GELU, the odd-part identity g(v) - g(-v) = v, the erf
+      form within 1e-3, limits)
 """
 from __future__ import annotations
 
@@ -87,6 +90,10 @@ def lib() -> ctypes.CDLL:
         L.oracle_fake_quantize_bf16.restype = None
         L.oracle_ste_backward.argtypes = [_p, _p, _i64, _i64, ctypes.c_int, _p]
         L.oracle_ste_backward.restype = None
+        L.oracle_gelu_tanh.argtypes = [ctypes.c_double]
+        L.oracle_gelu_tanh.restype = ctypes.c_double
+        L.oracle_gelu_tanh_array.argtypes = [_p, _i64, _p]
+        L.oracle_gelu_tanh_array.restype = None
         _LIB = L
     return _LIB
 
@@ -300,3 +307,16 @@ def ste_backward(grad_y: np.ndarray, mask: np.ndarray) -> np.ndarray:
     gx = np.empty_like(gy)
     L.oracle_ste_backward(_ptr(gy), _ptr(m), rows, k, gy.dtype.itemsize, _ptr(gx))
     return gx
+
+
+# ---------------------------------------------------------------- epilogue activation
+def gelu_tanh(v):
+    """GELU, tanh form, in double (the fused GEMM epilogue's activation; the
+    pages name none, a reading).  Scalar or float64 array."""
+    L = lib()
+    if np.isscalar(v):
+        return float(L.oracle_gelu_tanh(float(v)))
+    a = np.ascontiguousarray(v, np.float64)
+    out = np.empty_like(a)
+    L.oracle_gelu_tanh_array(_ptr(a), a.size, _ptr(out))
+    return out

@@ -437,3 +437,19 @@ void oracle_ste_backward(const void *grad_y, const uint8_t *mask, int64_t rows, 
             else memcpy(dst + e * elem_bytes, src + e * elem_bytes, (size_t)elem_bytes);
         }
 }
+
+/* ------------------------- epilogue activation --------------------------- */
+/* GELU in its tanh form, 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))), in
+ * double.  The pages name no activation; this is the one the DiT family's
+ * MLPs use (a reading), applied by the fused GEMM epilogue to alpha * acc.   */
+double oracle_gelu_tanh(double v)
+{
+    const double c = sqrt(2.0 / 3.14159265358979323846);
+    return 0.5 * v * (1.0 + tanh(c * (v + 0.044715 * v * v * v)));
+}
+
+/* Elementwise over n doubles (in place allowed). */
+void oracle_gelu_tanh_array(const double *in, int64_t n, double *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_gelu_tanh(in[i]);
+}

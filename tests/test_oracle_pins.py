@@ -575,3 +575,21 @@ def test_fake_quantize_grid_valued_input_is_a_fixed_point():
     y, mask, _ = oracle.fake_quantize(xb, 2.0 ** -8)
     assert np.array_equal(oracle.bf16_to_f32(y).astype(np.float64), x)
     assert not mask.any()
+
+
+# ------------------------------------------------------------------ epilogue activation
+def test_gelu_tanh_against_library_and_identities():
+    """The tanh-form GELU: torch's float64 implementation (a library routine),
+    the identity g(v) - g(-v) = v (the tanh term is odd), the erf form within
+    1e-3, and the limits."""
+    import math
+    rng = np.random.default_rng(30)
+    v = np.concatenate([rng.standard_normal(4000) * 3, np.linspace(-12, 12, 2001), [0.0, 1e-30, -1e-30]])
+    g = oracle.gelu_tanh(v)
+    ref = torch.nn.functional.gelu(torch.from_numpy(v), approximate="tanh").numpy()
+    assert np.max(np.abs(g - ref)) <= 1e-14 * np.maximum(1.0, np.abs(v)).max()
+    assert np.max(np.abs(g - oracle.gelu_tanh(-v) - v)) <= 1e-13
+    erf = np.array([0.5 * x * (1 + math.erf(x / math.sqrt(2))) for x in v])
+    assert np.max(np.abs(g - erf)) < 1e-3
+    assert oracle.gelu_tanh(0.0) == 0.0
+    assert oracle.gelu_tanh(40.0) == 40.0 and oracle.gelu_tanh(-40.0) == 0.0
