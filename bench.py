@@ -234,6 +234,8 @@ def reference_points(dev, layers, w4a16_layers):
                                 "tflops": round(2 * L.M * L.N * L.K / (ms * 1e-3) / 1e12, 1)}
         del x, W, y
     out["qat"] = qat_points(dev, layers)
+    out["mlp_fc1_gelu"] = mlp_fusion_points(dev, layers)
+    out["grouped"] = grouped_points(dev)
     torch.cuda.empty_cache()
     return out
 
@@ -282,6 +284,69 @@ def qat_points(dev, layers):
         del x, y, m, gx, ws
     torch.cuda.empty_cache()
     return res_all
+
+
+def mlp_fusion_points(dev, layers):
+    """The MLP's first layer with GELU and the second layer's NVFP4 input
+    produced in the GEMM epilogue (one kernel), against the same result made
+    in three steps: the GEMM writing bf16, GELU (torch, a reference point
+    only), and the dynamic-scale quantize of the activation."""
+    import torch
+    import nvfp4_w4a4_gemm_quantize_b200 as nv
+    from nvfp4_w4a4_gemm_quantize_b200 import synth
+    L = [l for l in layers if l.name == "fc1"]
+    if not L:
+        return None
+    L = L[0]
+    x, w = synth.layer_tensors(WORKLOAD, "fc1", device=dev)
+    A, W = nv.quantize(x[: L.M].contiguous()), nv.quantize(w)
+    del x, w
+    y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev)
+    q = nv.NVFP4Tensor.empty(L.M, L.N, dev)
+    amax = torch.zeros(1, dtype=torch.float32, device=dev)
+    ws = torch.empty(nv.nvfp4_quantize_workspace_bytes(L.M, L.N), dtype=torch.uint8, device=dev)
+    nv.gemm_w4a4(A, W, out=y, act=nv.NVFP4_ACT_GELU_TANH)
+    q.scale.copy_(torch.max(torch.abs(y.float())).reshape(1) / 2688.0)
+    gy = q.scale.clone()
+    fused = time_device(lambda: nv.gemm_w4a4_nvfp4_out(A, W, gy, y_amax=amax, out=q, act=nv.NVFP4_ACT_GELU_TANH))
+    g_ms = time_device(lambda: nv.gemm_w4a4(A, W, out=y))
+    a_ms = time_device(lambda: torch.nn.functional.gelu(y, approximate="tanh"))
+    h = torch.nn.functional.gelu(y, approximate="tanh")
+    q_ms = time_device(lambda: nv.quantize(h, out=q, workspace=ws))
+    del y, h, q, A, W
+    torch.cuda.empty_cache()
+    fl = 2 * L.M * L.N * L.K
+    return {"shape": f"{L.M}x{L.K}x{L.N}", "fused_ms": round(fused, 4),
+            "fused_tflops": round(fl / (fused * 1e-3) / 1e12, 1),
+            "three_step_ms": round(g_ms + a_ms + q_ms, 4),
+            "three_step_parts_ms": {"gemm_bf16": round(g_ms, 4), "gelu_torch": round(a_ms, 4),
+                                    "quantize": round(q_ms, 4)}}
+
+
+def grouped_points(dev):
+    """One PixArt-1024 block's independent projections (image-token QKV,
+    text-token cross-attention K and V) as one grouped launch vs three."""
+    import torch
+    import nvfp4_w4a4_gemm_quantize_b200 as nv
+    from nvfp4_w4a4_gemm_quantize_b200 import synth
+    pairs, fl = [], 0
+    for name in ("qkv", "xattn_k", "xattn_v"):
+        x, w = synth.layer_tensors("pixart1024", name, device=dev)
+        pairs.append((nv.quantize(x), nv.quantize(w)))
+        fl += 2 * x.shape[0] * x.shape[1] * w.shape[0]
+    ys = [torch.empty(A.rows, B.rows, dtype=torch.bfloat16, device=dev) for A, B in pairs]
+    probs = [dict(a_codes=A.codes, a_sf=A.sf, a_scale=A.scale, b_codes=B.codes, b_sf=B.sf, b_scale=B.scale,
+                  M=A.rows, N=B.rows, K=A.k, y=y) for (A, B), y in zip(pairs, ys)]
+
+    def separate():
+        for (A, B), y in zip(pairs, ys):
+            nv.gemm_w4a4(A, B, out=y)
+
+    sep = time_device(separate, iters=50, warmup=5)
+    grp = time_device(lambda: nv.nvfp4_gemm_w4a4_grouped(probs), iters=50, warmup=5)
+    return {"problems": "pixart1024 qkv 8192x1152x3456 + xattn_k/v 600x4096x1152",
+            "separate_us": round(sep * 1e3, 1), "grouped_us": round(grp * 1e3, 1),
+            "grouped_tflops": round(fl / (grp * 1e-3) / 1e12, 1)}
 
 
 def reduced(wl, args):

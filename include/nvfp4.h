@@ -71,6 +71,13 @@ enum { NVFP4_DTYPE_BF16 = 0, NVFP4_DTYPE_F32 = 1 };
 /* nvfp4_quantize flags */
 enum { NVFP4_SCALE_GIVEN = 1 };
 
+/* GEMM epilogue activations, applied to alpha * acc before the output is
+ * formed (bf16 / FP32 values, or the NVFP4 codes of the next layer):
+ *   NVFP4_ACT_GELU_TANH  0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))), tanh
+ *                        from the hardware approximation (relative error about
+ *                        2^-11), the activation of the DiT family's MLPs. */
+enum { NVFP4_ACT_NONE = 0, NVFP4_ACT_GELU_TANH = 1 };
+
 /* Bytes of the scale buffer of a [rows, k] NVFP4 tensor:
  * ceil(rows/128)*128 * k/16.  Returns 0 for rows < 0 or k not a multiple of 64. */
 size_t nvfp4_sf_bytes(int64_t rows, int64_t k);
@@ -202,8 +209,11 @@ nvfp4_status nvfp4_ste_backward(const void *grad_y, const uint8_t *clip_mask, in
  *    exactly as nvfp4_quantize with NVFP4_SCALE_GIVEN would quantize the FP32
  *    value alpha*acc: y_codes [M, N/2], y_sf nvfp4_sf_bytes(M, N); needs
  *    N % 64 == 0.  y_amax (nullable device float, caller-initialised): receives
- *    the running max of |alpha*acc| (atomic max), from which the caller can
+ *    the running max of |output value| (atomic max), from which the caller can
  *    derive the next call's g_y.
+ * act: NVFP4_ACT_NONE, or NVFP4_ACT_GELU_TANH to output GELU(alpha*acc) -- for
+ *    an MLP's first layer with the NVFP4 output, the second layer's input is
+ *    produced without writing or re-reading the activation in 16-bit form.
  * All code/scale pointers 16-byte aligned.  One persistent kernel on `stream`.
  */
 nvfp4_status nvfp4_gemm_w4a4(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_scale,
@@ -211,7 +221,7 @@ nvfp4_status nvfp4_gemm_w4a4(const uint8_t *a_codes, const uint8_t *a_sf, const 
                              int64_t M, int64_t N, int64_t K,
                              void *y, int y_dtype,
                              uint8_t *y_codes, uint8_t *y_sf, const float *y_scale, float *y_amax,
-                             int *dev_status, nvfp4_stream_t stream);
+                             int act, int *dev_status, nvfp4_stream_t stream);
 
 /*
  * nvfp4_gemm_w4a4_grouped -- up to NVFP4_MAX_GROUP independent W4A4 products
@@ -227,7 +237,8 @@ nvfp4_status nvfp4_gemm_w4a4(const uint8_t *a_codes, const uint8_t *a_sf, const 
  *            nvfp4_gemm_w4a4 means and is checked the same way.  Every problem
  *            has the same output kind: all y != NULL (then y_dtype applies to
  *            all), or all y == NULL with NVFP4 outputs (y_codes, y_sf, y_scale,
- *            optional y_amax).  Problems with M == 0 are skipped.
+ *            optional y_amax), and the same act.  Problems with M == 0 are
+ *            skipped.
  * One launch of the single-CTA kernel (128 x 128 tiles) for any N; the
  * array is read during the call only.
  */
@@ -244,6 +255,7 @@ typedef struct {
     uint8_t *y_sf;
     const float *y_scale;
     float *y_amax;
+    int act;
 } nvfp4_gemm_problem;
 
 enum { NVFP4_MAX_GROUP = 8 };

@@ -25,6 +25,8 @@ from ._lib import MAX_GROUP, NVFP4Error, NVFP4GemmProblem, check, lib  # noqa: F
 NVFP4_DTYPE_BF16 = 0
 NVFP4_DTYPE_F32 = 1
 NVFP4_SCALE_GIVEN = 1
+NVFP4_ACT_NONE = 0
+NVFP4_ACT_GELU_TANH = 1
 
 _DT = {torch.bfloat16: NVFP4_DTYPE_BF16, torch.float32: NVFP4_DTYPE_F32}
 
@@ -109,10 +111,10 @@ def nvfp4_ste_backward(grad_y, clip_mask, rows, k, dtype, grad_x, stream=None) -
 
 def nvfp4_gemm_w4a4(a_codes, a_sf, a_scale, b_codes, b_sf, b_scale, M, N, K, y=None,
                     y_dtype=NVFP4_DTYPE_BF16, y_codes=None, y_sf=None, y_scale=None, y_amax=None,
-                    dev_status=None, stream=None) -> None:
+                    act=0, dev_status=None, stream=None) -> None:
     st = lib().nvfp4_gemm_w4a4(_ptr(a_codes), _ptr(a_sf), _ptr(a_scale), _ptr(b_codes), _ptr(b_sf),
                                _ptr(b_scale), M, N, K, _ptr(y), y_dtype, _ptr(y_codes), _ptr(y_sf),
-                               _ptr(y_scale), _ptr(y_amax), _ptr(dev_status), _stream(stream))
+                               _ptr(y_scale), _ptr(y_amax), act, _ptr(dev_status), _stream(stream))
     check(st, "nvfp4_gemm_w4a4")
 
 
@@ -123,7 +125,7 @@ def nvfp4_gemm_w4a4_grouped(problems, y_dtype=NVFP4_DTYPE_BF16, dev_status=None,
     for i, d in enumerate(problems):
         for name, _ in NVFP4GemmProblem._fields_:
             v = d.get(name)
-            setattr(arr[i], name, int(v) if name in ("M", "N", "K") else _ptr(v))
+            setattr(arr[i], name, int(v or 0) if name in ("M", "N", "K", "act") else _ptr(v))
     st = lib().nvfp4_gemm_w4a4_grouped(ctypes.addressof(arr), len(problems), y_dtype, _ptr(dev_status),
                                        _stream(stream))
     check(st, "nvfp4_gemm_w4a4_grouped")
@@ -183,27 +185,28 @@ def dequantize(q: NVFP4Tensor, dtype=torch.bfloat16, stream=None) -> torch.Tenso
 
 
 def gemm_w4a4(a: NVFP4Tensor, b: NVFP4Tensor, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
-              dev_status=None, stream=None) -> torch.Tensor:
-    """Y = A B^T, A [M,K] activations, B [N,K] weights, both NVFP4."""
+              act=NVFP4_ACT_NONE, dev_status=None, stream=None) -> torch.Tensor:
+    """Y = act(A B^T), A [M,K] activations, B [N,K] weights, both NVFP4."""
     assert a.k == b.k
     y = out if out is not None else torch.empty(a.rows, b.rows, dtype=out_dtype, device=a.codes.device)
     nvfp4_gemm_w4a4(a.codes, a.sf, a.scale, b.codes, b.sf, b.scale, a.rows, b.rows, a.k, y=y,
-                    y_dtype=_DT[y.dtype], dev_status=dev_status, stream=stream)
+                    y_dtype=_DT[y.dtype], act=act, dev_status=dev_status, stream=stream)
     return y
 
 
 def gemm_w4a4_nvfp4_out(a: NVFP4Tensor, b: NVFP4Tensor, y_scale: torch.Tensor, y_amax: torch.Tensor | None = None,
-                        out: NVFP4Tensor | None = None, dev_status=None, stream=None) -> NVFP4Tensor:
-    """Y = A B^T emitted directly as NVFP4 with the caller's tensor scale."""
+                        out: NVFP4Tensor | None = None, act=NVFP4_ACT_NONE, dev_status=None,
+                        stream=None) -> NVFP4Tensor:
+    """act(Y = A B^T) emitted directly as NVFP4 with the caller's tensor scale."""
     q = out if out is not None else NVFP4Tensor.empty(a.rows, b.rows, a.codes.device)
     q.scale.copy_(y_scale.reshape(1))
     nvfp4_gemm_w4a4(a.codes, a.sf, a.scale, b.codes, b.sf, b.scale, a.rows, b.rows, a.k,
-                    y_codes=q.codes, y_sf=q.sf, y_scale=q.scale, y_amax=y_amax, dev_status=dev_status,
+                    y_codes=q.codes, y_sf=q.sf, y_scale=q.scale, y_amax=y_amax, act=act, dev_status=dev_status,
                     stream=stream)
     return q
 
 
-def gemm_w4a4_grouped(pairs, out_dtype=torch.bfloat16, dev_status=None, stream=None) -> list:
+def gemm_w4a4_grouped(pairs, out_dtype=torch.bfloat16, act=NVFP4_ACT_NONE, dev_status=None, stream=None) -> list:
     """Y_i = A_i B_i^T for up to MAX_GROUP independent (A_i, B_i) NVFP4 pairs in
     one launch; returns the outputs in order."""
     ys, probs = [], []
@@ -212,7 +215,7 @@ def gemm_w4a4_grouped(pairs, out_dtype=torch.bfloat16, dev_status=None, stream=N
         y = torch.empty(a.rows, b.rows, dtype=out_dtype, device=a.codes.device)
         ys.append(y)
         probs.append(dict(a_codes=a.codes, a_sf=a.sf, a_scale=a.scale, b_codes=b.codes, b_sf=b.sf,
-                          b_scale=b.scale, M=a.rows, N=b.rows, K=a.k, y=y))
+                          b_scale=b.scale, M=a.rows, N=b.rows, K=a.k, y=y, act=act))
     nvfp4_gemm_w4a4_grouped(probs, _DT[out_dtype], dev_status, stream)
     return ys
 

@@ -31,7 +31,7 @@ class NVFP4GemmProblem(ctypes.Structure):
     _fields_ = [("a_codes", _p), ("a_sf", _p), ("a_scale", _p),
                 ("b_codes", _p), ("b_sf", _p), ("b_scale", _p),
                 ("M", _i64), ("N", _i64), ("K", _i64),
-                ("y", _p), ("y_codes", _p), ("y_sf", _p), ("y_scale", _p), ("y_amax", _p)]
+                ("y", _p), ("y_codes", _p), ("y_sf", _p), ("y_scale", _p), ("y_amax", _p), ("act", _int)]
 
 
 MAX_GROUP = 8
@@ -46,7 +46,8 @@ SIGNATURES = {
     "nvfp4_fake_quantize": (_status, [_p, _i64, _i64, _i64, _p, _int, _p, _p, ctypes.c_uint, _p, ctypes.c_size_t,
                                       _p, _p]),
     "nvfp4_ste_backward": (_status, [_p, _p, _i64, _i64, _int, _p, _p]),
-    "nvfp4_gemm_w4a4": (_status, [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _p, _int, _p, _p, _p, _p, _p, _p]),
+    "nvfp4_gemm_w4a4": (_status, [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _p, _int, _p, _p, _p, _p, _int, _p,
+                                  _p]),
     "nvfp4_gemm_w4a4_grouped": (_status, [_p, _int, _int, _p, _p]),
     "nvfp4_gemm_w4a16": (_status, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _int, _p, _p]),
     "nvfp4_status_string": (ctypes.c_char_p, [_int]),

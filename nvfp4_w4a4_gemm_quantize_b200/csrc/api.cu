@@ -219,16 +219,17 @@ static nvfp4_status check_gemm_problem(const uint8_t* a_codes, const uint8_t* a_
 nvfp4_status nvfp4_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_scale,
                              const uint8_t* b_codes, const uint8_t* b_sf, const float* b_scale, int64_t M, int64_t N,
                              int64_t K, void* y, int y_dtype, uint8_t* y_codes, uint8_t* y_sf, const float* y_scale,
-                             float* y_amax, int* dev_status, nvfp4_stream_t stream) {
+                             float* y_amax, int act, int* dev_status, nvfp4_stream_t stream) {
     const nvfp4_status chk = check_gemm_problem(a_codes, a_sf, a_scale, b_codes, b_sf, b_scale, M, N, K, y, y_dtype,
                                                 y_codes, y_sf, y_scale);
     if (chk != NVFP4_OK) return chk;
+    if (act != NVFP4_ACT_NONE && act != NVFP4_ACT_GELU_TANH) return NVFP4_ERR_INVALID_ARG;
     if (M == 0) return NVFP4_OK;                 /* nothing to read or write */
     int sms = 0;
     nvfp4_status st = device_ok(&sms);
     if (st != NVFP4_OK) return st;
     GemmW4A4Args a{a_codes, a_sf, a_scale, b_codes, b_sf, b_scale, M, N, K, y, y_dtype,
-                   y_codes, y_sf, y_scale, y_amax, dev_status};
+                   y_codes, y_sf, y_scale, y_amax, dev_status, act};
     return cuda_status(launch_gemm_w4a4(a, sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -237,17 +238,19 @@ nvfp4_status nvfp4_gemm_w4a4_grouped(const nvfp4_gemm_problem* problems, int cou
     if (!problems || count < 1 || count > NVFP4_MAX_GROUP) return NVFP4_ERR_INVALID_ARG;
     if (NVFP4_MAX_GROUP > gemm_w4a4_max_group()) return NVFP4_ERR_INVALID_ARG;
     const bool nvfp4_out = problems[0].y == nullptr;
+    const int act = problems[0].act;
+    if (act != NVFP4_ACT_NONE && act != NVFP4_ACT_GELU_TANH) return NVFP4_ERR_INVALID_ARG;
     GemmW4A4Args args[NVFP4_MAX_GROUP];
     int n = 0;
     for (int i = 0; i < count; ++i) {
         const nvfp4_gemm_problem& q = problems[i];
-        if ((q.y == nullptr) != nvfp4_out) return NVFP4_ERR_INVALID_ARG;   // one output kind per launch
+        if ((q.y == nullptr) != nvfp4_out || q.act != act) return NVFP4_ERR_INVALID_ARG;   // one kind per launch
         const nvfp4_status st = check_gemm_problem(q.a_codes, q.a_sf, q.a_scale, q.b_codes, q.b_sf, q.b_scale, q.M,
                                                    q.N, q.K, q.y, y_dtype, q.y_codes, q.y_sf, q.y_scale);
         if (st != NVFP4_OK) return st;
         if (q.M == 0) continue;                  // nothing to read or write
         args[n++] = GemmW4A4Args{q.a_codes, q.a_sf, q.a_scale, q.b_codes, q.b_sf, q.b_scale, q.M, q.N, q.K,
-                                 q.y, y_dtype, q.y_codes, q.y_sf, q.y_scale, q.y_amax, dev_status};
+                                 q.y, y_dtype, q.y_codes, q.y_sf, q.y_scale, q.y_amax, dev_status, act};
     }
     int sms = 0;
     nvfp4_status st = device_ok(&sms);

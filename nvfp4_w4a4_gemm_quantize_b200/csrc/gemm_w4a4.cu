@@ -121,7 +121,7 @@ __device__ __forceinline__ void flush_amax(float v, float* dst, int lane) {
     if (dst != nullptr && lane == 0 && v > 0.0f) atomicMax(reinterpret_cast<int*>(dst), __float_as_int(v));
 }
 
-template <int BN, int STAGES, int OUT>
+template <int BN, int STAGES, int OUT, int ACT>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p) {
     using C = Cfg<BN, STAGES>;
@@ -339,7 +339,7 @@ gemm_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p)
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const uint32_t bits = (b < 2) ? r0[b * 16 + j] : r1[(b - 2) * 16 + j];
-                            v[j] = __fmul_rn(alpha, __uint_as_float(bits));
+                            v[j] = epi_value<ACT>(alpha, bits);
                         }
                         float ab = 0.0f;
 #pragma unroll
@@ -376,8 +376,8 @@ gemm_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p)
                         uint32_t pk[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
-                            __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(alpha, __uint_as_float(r[2 * j])),
-                                                                     __fmul_rn(alpha, __uint_as_float(r[2 * j + 1])));
+                            __nv_bfloat162 h = __floats2bfloat162_rn(epi_value<ACT>(alpha, r[2 * j]),
+                                                                     epi_value<ACT>(alpha, r[2 * j + 1]));
                             pk[j] = *reinterpret_cast<uint32_t*>(&h);
                         }
                         // 64-byte rows, 64-byte swizzle: chunk j of row i at j ^ ((i >> 1) & 3)
@@ -392,10 +392,8 @@ gemm_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p)
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
                             const int pos = j ^ (lane & 7);
-                            float4 o = make_float4(__fmul_rn(alpha, __uint_as_float(r[4 * j])),
-                                                   __fmul_rn(alpha, __uint_as_float(r[4 * j + 1])),
-                                                   __fmul_rn(alpha, __uint_as_float(r[4 * j + 2])),
-                                                   __fmul_rn(alpha, __uint_as_float(r[4 * j + 3])));
+                            float4 o = make_float4(epi_value<ACT>(alpha, r[4 * j]), epi_value<ACT>(alpha, r[4 * j + 1]),
+                                                   epi_value<ACT>(alpha, r[4 * j + 2]), epi_value<ACT>(alpha, r[4 * j + 3]));
                             *reinterpret_cast<float4*>(buf + lane * 128 + pos * 16) = o;
                         }
                     }
@@ -427,7 +425,7 @@ gemm_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p)
     }
 }
 
-template <int BN, int STAGES, int OUT>
+template <int BN, int STAGES, int OUT, int ACT>
 cudaError_t launch_cfg(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream) {
     using C = Cfg<BN, STAGES>;
     if (count < 1 || count > kMaxGroup) return cudaErrorInvalidValue;
@@ -475,7 +473,7 @@ cudaError_t launch_cfg(const GemmW4A4Args* probs, int count, int num_sms, cudaSt
     p.dev_status = probs[0].dev_status;
     if (tiles == 0) return cudaSuccess;
 
-    auto kern = gemm_kernel<BN, STAGES, OUT>;
+    auto kern = gemm_kernel<BN, STAGES, OUT, ACT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const int grid = tiles < num_sms ? tiles : num_sms;
@@ -486,7 +484,8 @@ cudaError_t launch_cfg(const GemmW4A4Args* probs, int count, int num_sms, cudaSt
 
 template <int OUT>
 static cudaError_t launch_group(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream) {
-    return launch_cfg<128, 5, OUT>(probs, count, num_sms, stream);
+    if (probs[0].act == ACT_GELU_TANH) return launch_cfg<128, 5, OUT, ACT_GELU_TANH>(probs, count, num_sms, stream);
+    return launch_cfg<128, 5, OUT, ACT_NONE>(probs, count, num_sms, stream);
 }
 
 }  // namespace w4a4
@@ -502,7 +501,7 @@ cudaError_t launch_gemm_w4a4(const GemmW4A4Args& a, int num_sms, cudaStream_t st
 }
 
 // Up to kMaxGroup problems in one launch of the single-CTA kernel; every
-// problem has the same output kind (bf16, FP32 or NVFP4).
+// problem has the same output kind (bf16, FP32 or NVFP4) and activation.
 cudaError_t launch_gemm_w4a4_grouped(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream) {
     using namespace w4a4;
     const int out = probs[0].y != nullptr ? (probs[0].y_dtype == 1 ? OUT_F32 : OUT_BF16) : OUT_NVFP4;

@@ -106,15 +106,14 @@ __device__ __forceinline__ void tile_coords(int t, int num_mb2, int num_nb, int&
 
 // Store 32 FP32 accumulator columns (alpha applied) of one row per lane
 // through a swizzled staging buffer and a TMA store of a 32 x 32 box.
-template <int OUT>
+template <int OUT, int ACT>
 __device__ __forceinline__ void store_chunk(const uint32_t* r, float alpha, uint8_t* buf, int lane,
                                             const CUtensorMap* map, int x, int y) {
     if (OUT == OUT_BF16) {
         uint32_t pk[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(alpha, __uint_as_float(r[2 * j])),
-                                                     __fmul_rn(alpha, __uint_as_float(r[2 * j + 1])));
+            __nv_bfloat162 h = __floats2bfloat162_rn(epi_value<ACT>(alpha, r[2 * j]), epi_value<ACT>(alpha, r[2 * j + 1]));
             pk[j] = *reinterpret_cast<uint32_t*>(&h);
         }
         // 64-byte rows, 64-byte swizzle: chunk j of row i at j ^ ((i >> 1) & 3)
@@ -130,8 +129,8 @@ __device__ __forceinline__ void store_chunk(const uint32_t* r, float alpha, uint
         for (int j = 0; j < 8; ++j) {
             const int pos = j ^ (lane & 7);
             *reinterpret_cast<float4*>(buf + lane * 128 + pos * 16) =
-                make_float4(__fmul_rn(alpha, __uint_as_float(r[4 * j])), __fmul_rn(alpha, __uint_as_float(r[4 * j + 1])),
-                            __fmul_rn(alpha, __uint_as_float(r[4 * j + 2])), __fmul_rn(alpha, __uint_as_float(r[4 * j + 3])));
+                make_float4(epi_value<ACT>(alpha, r[4 * j]), epi_value<ACT>(alpha, r[4 * j + 1]),
+                            epi_value<ACT>(alpha, r[4 * j + 2]), epi_value<ACT>(alpha, r[4 * j + 3]));
         }
     }
     fence_proxy_async_smem();
@@ -160,7 +159,7 @@ __device__ __forceinline__ void k_mma(uint32_t tmem_acc, uint32_t sb, uint32_t s
                  col + 4, accumulate ? 1u : 0u);
 }
 
-template <int OUT>
+template <int OUT, int ACT>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
              const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
@@ -410,7 +409,7 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                     for (int b = 0; b < 4; ++b) {
                         float v[16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(alpha, __uint_as_float(r[c * 64 + b * 16 + j]));
+                        for (int j = 0; j < 16; ++j) v[j] = epi_value<ACT>(alpha, r[c * 64 + b * 16 + j]);
                         float ab = 0.0f;
 #pragma unroll
                         for (int j = 0; j < 16; ++j) ab = fmaxf(ab, fabsf(v[j]));
@@ -443,7 +442,7 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                     uint8_t* buf = ebuf + (nstore & 1) * C::EPI_BUF;
                     if (lane == 0) bulk_wait_group_read<1>();
                     __syncwarp();
-                    store_chunk<OUT>(&r[c * 32], alpha, buf, lane, &tmap_y, n0 + c * 32, m0);
+                    store_chunk<OUT, ACT>(&r[c * 32], alpha, buf, lane, &tmap_y, n0 + c * 32, m0);
                     ++nstore;
                 }
             }
@@ -465,7 +464,7 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     }
 }
 
-template <int OUT>
+template <int OUT, int ACT>
 cudaError_t launch_out(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) {
     using C = Cfg<OUT>;
     CUtensorMap ta, tb, tsa, tsb, ty;
@@ -507,7 +506,7 @@ cudaError_t launch_out(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) 
     p.y_amax = a.y_amax;
     p.dev_status = a.dev_status;
 
-    auto kern = gemm2_kernel<OUT>;
+    auto kern = gemm2_kernel<OUT, ACT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
 
@@ -539,11 +538,16 @@ cudaError_t launch_out(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) 
 
 cudaError_t launch_gemm_w4a4_2sm(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) {
     using namespace w4a4_2sm;
+    const bool gelu = a.act == ACT_GELU_TANH;
     if (a.y != nullptr) {
-        if (a.y_dtype == 1) return launch_out<OUT_F32>(a, num_sms, stream);
-        return launch_out<OUT_BF16>(a, num_sms, stream);
+        if (a.y_dtype == 1)
+            return gelu ? launch_out<OUT_F32, ACT_GELU_TANH>(a, num_sms, stream)
+                        : launch_out<OUT_F32, ACT_NONE>(a, num_sms, stream);
+        return gelu ? launch_out<OUT_BF16, ACT_GELU_TANH>(a, num_sms, stream)
+                    : launch_out<OUT_BF16, ACT_NONE>(a, num_sms, stream);
     }
-    return launch_out<OUT_NVFP4>(a, num_sms, stream);
+    return gelu ? launch_out<OUT_NVFP4, ACT_GELU_TANH>(a, num_sms, stream)
+                : launch_out<OUT_NVFP4, ACT_NONE>(a, num_sms, stream);
 }
 
 }  // namespace nvfp4

@@ -54,6 +54,7 @@ struct GemmW4A4Args {
     const float* y_scale;
     float* y_amax;
     int* dev_status;
+    int act;                  // epilogue activation: 0 none, 1 GELU (tanh form)
 };
 
 cudaError_t launch_gemm_w4a4(const GemmW4A4Args& a, int num_sms, cudaStream_t stream);

@@ -100,23 +100,25 @@ def test_gemm_rejects_bad_arguments(L):
     g = L.nvfp4_gemm_w4a4
     args = [A, B, C, A, B, C]
     # K not multiple of 64
-    assert g(*args, 128, 256, 96, A, 0, None, None, None, None, None, None) == SHAPE
+    assert g(*args, 128, 256, 96, A, 0, None, None, None, None, 0, None, None) == SHAPE
     # N not multiple of 8 for bf16 output
-    assert g(*args, 128, 260, 256, A, 0, None, None, None, None, None, None) == SHAPE
+    assert g(*args, 128, 260, 256, A, 0, None, None, None, None, 0, None, None) == SHAPE
     # fused NVFP4 output needs N % 64 == 0
-    assert g(*args, 128, 96, 256, None, 0, A, B, C, None, None, None) == SHAPE
+    assert g(*args, 128, 96, 256, None, 0, A, B, C, None, 0, None, None) == SHAPE
     # both outputs given
-    assert g(*args, 128, 256, 256, A, 0, A, B, C, None, None, None) == INVALID
+    assert g(*args, 128, 256, 256, A, 0, A, B, C, None, 0, None, None) == INVALID
     # no output at all
-    assert g(*args, 128, 256, 256, None, 0, None, None, None, None, None, None) == INVALID
+    assert g(*args, 128, 256, 256, None, 0, None, None, None, None, 0, None, None) == INVALID
     # bad dtype
-    assert g(*args, 128, 256, 256, A, 5, None, None, None, None, None, None) == INVALID
+    assert g(*args, 128, 256, 256, A, 5, None, None, None, None, 0, None, None) == INVALID
     # null scale
-    assert g(A, B, None, A, B, C, 128, 256, 256, A, 0, None, None, None, None, None, None) == INVALID
+    assert g(A, B, None, A, B, C, 128, 256, 256, A, 0, None, None, None, None, 0, None, None) == INVALID
     # misaligned operand
-    assert g(A + 1, B, C, A, B, C, 128, 256, 256, A, 0, None, None, None, None, None, None) == MISALIGNED
+    assert g(A + 1, B, C, A, B, C, 128, 256, 256, A, 0, None, None, None, None, 0, None, None) == MISALIGNED
+    # unknown activation
+    assert g(*args, 128, 256, 256, A, 0, None, None, None, None, 2, None, None) == INVALID
     # negative M
-    assert g(*args, -1, 256, 256, A, 0, None, None, None, None, None, None) == INVALID
+    assert g(*args, -1, 256, 256, A, 0, None, None, None, None, 0, None, None) == INVALID
 
 
 def test_fake_quantize_rejects_bad_arguments(L):
@@ -176,6 +178,8 @@ def test_grouped_gemm_rejects_bad_arguments(L):
     arr = _problems(2, {1: dict(b_scale=None)})
     assert g(addr(arr), 2, 0, None, None) == INVALID
     arr = _problems(2, {0: dict(M=-1)})
+    assert g(addr(arr), 2, 0, None, None) == INVALID
+    arr = _problems(2, {1: dict(act=1)})                                              # mixed activations
     assert g(addr(arr), 2, 0, None, None) == INVALID
 
 
