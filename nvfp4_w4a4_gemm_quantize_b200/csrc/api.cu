@@ -11,6 +11,7 @@
 
 #include "../../include/nvfp4.h"
 #include "internal.h"
+#include "gemm.h"
 #include "tmap.h"
 
 namespace nvfp4 {

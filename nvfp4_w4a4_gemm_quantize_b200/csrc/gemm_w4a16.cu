@@ -40,6 +40,7 @@
 #include <cuda_runtime.h>
 
 #include "internal.h"
+#include "gemm.h"
 #include "ptx.cuh"
 #include "tmap.h"
 

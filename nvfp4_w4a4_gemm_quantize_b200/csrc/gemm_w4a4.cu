@@ -32,8 +32,10 @@
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "gemm.h"
 #include "ptx.cuh"
 #include "quant_math.cuh"
+#include "epilogue.cuh"
 #include "tmap.h"
 
 namespace nvfp4 {

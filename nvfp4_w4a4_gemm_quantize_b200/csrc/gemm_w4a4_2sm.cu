@@ -45,8 +45,10 @@
 #include <cuda_runtime.h>
 
 #include "internal.h"
+#include "gemm.h"
 #include "ptx.cuh"
 #include "quant_math.cuh"
+#include "epilogue.cuh"
 #include "tmap.h"
 
 namespace nvfp4 {
