@@ -27,6 +27,9 @@ Parity status per function:
       of saturating elements)
   ste_backward                                          -- pinned (closed form
       through numpy's bit unpacking)
+  mx_quantize / mx_dequantize / mx_gemm                 -- pinned (brute-force
+      exponent and nearest-grid searches on tiny inputs, grid membership and
+      the error bound, power-of-two fixed points, a float64 library matmul)
   gelu_tanh                                             -- pinned (torch's
       float64 tanh-form GELU, the odd-part identity g(v) - g(-v) = v, the erf
       form within 1e-3, limits)
@@ -90,6 +93,14 @@ def lib() -> ctypes.CDLL:
         L.oracle_fake_quantize_bf16.restype = None
         L.oracle_ste_backward.argtypes = [_p, _p, _i64, _i64, ctypes.c_int, _p]
         L.oracle_ste_backward.restype = None
+        L.oracle_mx_sf_bytes.argtypes = [_i64, _i64]
+        L.oracle_mx_sf_bytes.restype = _i64
+        L.oracle_mx_quantize_bf16.argtypes = [_p, _i64, _i64, _i64, _p, _p]
+        L.oracle_mx_quantize_bf16.restype = None
+        L.oracle_mx_dequantize_f64.argtypes = [_p, _p, _i64, _i64, _p]
+        L.oracle_mx_dequantize_f64.restype = None
+        L.oracle_mx_gemm_rows.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p]
+        L.oracle_mx_gemm_rows.restype = None
         L.oracle_gelu_tanh.argtypes = [ctypes.c_double]
         L.oracle_gelu_tanh.restype = ctypes.c_double
         L.oracle_gelu_tanh_array.argtypes = [_p, _i64, _p]
@@ -320,3 +331,55 @@ def gelu_tanh(v):
     out = np.empty_like(a)
     L.oracle_gelu_tanh_array(_ptr(a), a.size, _ptr(out))
     return out
+
+
+# ---------------------------------------------------------------- MXFP4
+def mx_sf_bytes(rows: int, k: int) -> int:
+    return int(lib().oracle_mx_sf_bytes(rows, k))
+
+
+def mx_quantize(x):
+    """MXFP4 (OCP MX reading): E2M1 codes [rows, k/2] and E8M0 block-32 scales
+    in the tensor-core layout (k % 128 == 0)."""
+    L = lib()
+    xb = bf16_bits(x)
+    rows, k = xb.shape
+    assert k % 128 == 0
+    codes = np.zeros((rows, k // 2), np.uint8)
+    sf = np.zeros(mx_sf_bytes(rows, k), np.uint8)
+    L.oracle_mx_quantize_bf16(_ptr(xb), rows, k, k, _ptr(codes), _ptr(sf))
+    return codes, sf
+
+
+def mx_dequantize(codes: np.ndarray, sf: np.ndarray) -> np.ndarray:
+    L = lib()
+    codes = np.ascontiguousarray(codes, np.uint8)
+    sf = np.ascontiguousarray(sf, np.uint8)
+    rows, kh = codes.shape
+    out = np.empty((rows, kh * 2), np.float64)
+    L.oracle_mx_dequantize_f64(_ptr(codes), _ptr(sf), rows, kh * 2, _ptr(out))
+    return out
+
+
+def mx_gemm(a_codes, a_sf, b_codes, b_sf, rows: slice | None = None) -> np.ndarray:
+    """Y = A B^T of two MXFP4 operands, in double."""
+    L = lib()
+    a_codes = np.ascontiguousarray(a_codes, np.uint8)
+    b_codes = np.ascontiguousarray(b_codes, np.uint8)
+    a_sf = np.ascontiguousarray(a_sf, np.uint8)
+    b_sf = np.ascontiguousarray(b_sf, np.uint8)
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    N = b_codes.shape[0]
+    m0, m1 = (0, M) if rows is None else (rows.start or 0, rows.stop)
+    y = np.empty((m1 - m0, N), np.float64)
+    L.oracle_mx_gemm_rows(_ptr(a_codes), _ptr(a_sf), _ptr(b_codes), _ptr(b_sf), N, K, m0, m1 - m0, _ptr(y))
+    return y
+
+
+def mx_sf_matrix(sf: np.ndarray, rows: int, k: int) -> np.ndarray:
+    """The E8M0 bytes as a [rows, k/32] matrix."""
+    kb = k // 32
+    r = np.arange(rows)[:, None]
+    c = np.arange(kb)[None, :]
+    off = ((r // 128) * (kb // 4) + c // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + c % 4
+    return sf[off]

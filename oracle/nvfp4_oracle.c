@@ -453,3 +453,89 @@ void oracle_gelu_tanh_array(const double *in, int64_t n, double *out)
 {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_gelu_tanh(in[i]);
 }
+
+/* ------------------------------ MXFP4 ------------------------------------ */
+/* The MX variant ("[RFC]: NVFP4 Quantization Support for Diffusion Models",
+ * Related: the MXFP4 RFC, a related format): E2M1 elements in blocks of 32
+ * along k, one power-of-two scale per block stored as an unsigned E8M0 byte
+ * (value 2^(byte - 127)), no tensor scale.  The pages give no rule for the
+ * scale; the reading taken is the OCP Microscaling (MX) specification's:
+ *   shared exponent  e = floor(log2(max|x|)) - 2      (2 = E2M1's largest exponent)
+ *   clamped to [-127, 127]; an all-zero block takes e = -127 (byte 0);
+ *   element code     RNE_E2M1(clip(x / 2^e, -6, 6)), sign of x kept.
+ * x / 2^e is exact (a power-of-two scaling), so no quotient rounding arises.
+ * Scales use the tensor-core scale layout with kb32 = k/32 blocks per row
+ * (k a multiple of 128, so that a row's blocks fill whole 4-block words).   */
+int64_t oracle_mx_sf_bytes(int64_t rows, int64_t k)
+{
+    return ((rows + 127) / 128) * 128 * (k / 32);
+}
+
+void oracle_mx_quantize_bf16(const uint16_t *x, int64_t rows, int64_t k, int64_t ld,
+                             uint8_t *codes, uint8_t *sf)
+{
+    const int64_t kb = k / 32;
+    memset(sf, 0, (size_t)oracle_mx_sf_bytes(rows, k));
+    memset(codes, 0, (size_t)(rows * (k / 2)));
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < kb; ++c) {
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                double a = fabs((double)oracle_bf16_to_f32(x[r * ld + c * 32 + i]));
+                if (a > amax) amax = a;
+            }
+            int e = -127;
+            if (amax > 0.0) {
+                int ex;
+                (void)frexp(amax, &ex);          /* amax = f 2^ex, f in [0.5, 1) */
+                e = (ex - 1) - 2;
+                if (e < -127) e = -127;
+                if (e > 127) e = 127;
+            }
+            sf[oracle_sf_offset(r, c, kb)] = (uint8_t)(e + 127);
+            for (int i = 0; i < 32; ++i) {
+                int64_t j = c * 32 + i;
+                double q = ldexp((double)oracle_bf16_to_f32(x[r * ld + j]), -e);   /* exact */
+                unsigned code = oracle_e2m1_encode((float)q);                     /* |q| < 8: exact in float */
+                codes[r * (k / 2) + j / 2] |= (uint8_t)(code << (4 * (j & 1)));
+            }
+        }
+}
+
+/* v = e2m1(code) * 2^(sf - 127), exact in double. */
+static double mx_deq_elem(const uint8_t *codes, const uint8_t *sf, int64_t r, int64_t j, int64_t k)
+{
+    uint8_t byte = codes[r * (k / 2) + j / 2];
+    unsigned code = (j & 1) ? (byte >> 4) : (byte & 15u);
+    int s = (int)sf[oracle_sf_offset(r, j / 32, k / 32)] - 127;
+    return ldexp(oracle_e2m1_decode(code), s);
+}
+
+void oracle_mx_dequantize_f64(const uint8_t *codes, const uint8_t *sf, int64_t rows, int64_t k, double *out)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < k; ++j)
+            out[r * k + j] = mx_deq_elem(codes, sf, r, j, k);
+}
+
+/* MX x MX product in double: Y[m,n] = sum_k a^[m,k] b^[n,k], rows m0.. of Y. */
+void oracle_mx_gemm_rows(const uint8_t *a_codes, const uint8_t *a_sf, const uint8_t *b_codes,
+                         const uint8_t *b_sf, int64_t N, int64_t K, int64_t m0, int64_t mrows, double *y)
+{
+    double *bh = (double *)malloc((size_t)(N * K) * sizeof(double));
+    double *ah = (double *)malloc((size_t)K * sizeof(double));
+    if (!bh || !ah) { free(bh); free(ah); return; }
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t j = 0; j < K; ++j)
+            bh[n * K + j] = mx_deq_elem(b_codes, b_sf, n, j, K);
+    for (int64_t i = 0; i < mrows; ++i) {
+        for (int64_t j = 0; j < K; ++j) ah[j] = mx_deq_elem(a_codes, a_sf, m0 + i, j, K);
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < K; ++j) acc += ah[j] * bh[n * K + j];
+            y[i * N + n] = acc;
+        }
+    }
+    free(bh);
+    free(ah);
+}

@@ -593,3 +593,86 @@ def test_gelu_tanh_against_library_and_identities():
     assert np.max(np.abs(g - erf)) < 1e-3
     assert oracle.gelu_tanh(0.0) == 0.0
     assert oracle.gelu_tanh(40.0) == 40.0 and oracle.gelu_tanh(-40.0) == 0.0
+
+
+# ------------------------------------------------------------------ MXFP4
+def brute_mx(xf32: np.ndarray):
+    """MX quantization by searches: the block exponent s is the integer with
+    4 * 2^s <= max|x| < 8 * 2^s (searched, clamped to [-127, 127]; -127 for an
+    all-zero block), codes by the nearest-grid search of x / 2^s."""
+    rows, k = xf32.shape
+    codes = np.zeros((rows, k), np.uint8)
+    exps = np.zeros((rows, k // 32), np.int64)
+    for r in range(rows):
+        for c in range(k // 32):
+            blk = [Fraction(float(v)) for v in xf32[r, 32 * c:32 * c + 32]]
+            amax = max(abs(v) for v in blk)
+            s = -127
+            if amax > 0:
+                s = next(t for t in range(-160, 160) if 4 * Fraction(2) ** t <= amax < 8 * Fraction(2) ** t)
+                s = min(max(s, -127), 127)
+            exps[r, c] = s
+            for i, v in enumerate(blk):
+                q = v / Fraction(2) ** s
+                code = brute_e2m1(float(q))
+                if v == 0 and np.signbit(xf32[r, 32 * c + i]):
+                    code |= 8
+                codes[r, 32 * c + i] = code
+    return codes, exps
+
+
+@pytest.mark.parametrize("case", range(6))
+def test_mx_quantize_vs_brute_force_tiny(case):
+    rng = np.random.default_rng(300 + case)
+    rows, k = [(1, 128), (3, 128), (2, 256)][case % 3]
+    x = rng.standard_normal((rows, k)).astype(np.float32)
+    x *= np.exp2(rng.uniform(-30, 30, (rows, k // 32))).repeat(32, axis=1).astype(np.float32)
+    if case == 4:
+        x[0, :32] = 0.0
+        x[0, 3] = -0.0
+    if case == 5:
+        x[1, 32:64] = (rng.standard_normal(32) * 2.0 ** -128).astype(np.float32)   # bf16 subnormals:
+        x[0, 64:96] = np.float32(2.0 ** -133)                                      # exponent clamps at -127
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    xf = xb.float().numpy()
+    codes, sf = oracle.mx_quantize(xb)
+    bc, be = brute_mx(xf)
+    assert np.array_equal(oracle.unpack_codes(codes), bc)
+    assert np.array_equal(oracle.mx_sf_matrix(sf, rows, k).astype(np.int64) - 127, be)
+
+
+def test_mx_grid_membership_error_bound_and_fixed_points():
+    xb = synth.random_bf16((256, 1024), seed=31, dist="outlier")
+    codes, sf = oracle.mx_quantize(xb)
+    xf = xb.float().numpy().astype(np.float64)
+    deq = oracle.mx_dequantize(codes, sf)
+    X = np.exp2(oracle.mx_sf_matrix(sf, 256, 1024).astype(np.float64) - 127).repeat(32, axis=1)
+    grid = set(E2M1_GRID) | {-v for v in E2M1_GRID}
+    assert set(np.unique(deq / X)) <= grid
+    q = np.abs(xf) / X
+    spacing = np.where(q < 2, 0.5, np.where(q < 4, 1.0, 2.0))
+    bound = np.where(q <= 6, X * spacing / 2, np.abs(xf) - 6 * X)
+    assert np.all(np.abs(xf - deq) <= bound)
+    assert q.max() < 8 and (q > 6).any()                       # the block maximum can clip (8 > 6)
+    # grid values times 2^m whose block maximum is 4 or 6 come back unchanged
+    rng = np.random.default_rng(32)
+    vals = np.array(E2M1_GRID + [-v for v in E2M1_GRID[1:]])
+    g = rng.choice(vals, (8, 256))
+    g[:, ::32] = rng.choice([4.0, -6.0, 6.0], (8, 8))
+    g *= np.exp2(rng.integers(-20, 20, (8, 8))).repeat(32, axis=1)
+    gb = torch.from_numpy(g.astype(np.float32)).to(torch.bfloat16)
+    c2, s2 = oracle.mx_quantize(gb)
+    assert np.array_equal(oracle.mx_dequantize(c2, s2), g)
+
+
+def test_mx_zero_tensor_and_gemm_vs_library_matmul():
+    codes, sf = oracle.mx_quantize(torch.zeros(130, 128, dtype=torch.bfloat16))
+    assert not codes.any() and not oracle.mx_sf_matrix(sf, 130, 128).any()
+    x = synth.random_bf16((64, 384), seed=33, dist="student_t3")
+    w = synth.random_bf16((48, 384), seed=34, dist="normal", scale=0.02)
+    ac, asf = oracle.mx_quantize(x)
+    bc, bsf = oracle.mx_quantize(w)
+    y = oracle.mx_gemm(ac, asf, bc, bsf)
+    ref = torch.from_numpy(oracle.mx_dequantize(ac, asf)) @ torch.from_numpy(oracle.mx_dequantize(bc, bsf)).T
+    assert np.allclose(y, ref.numpy(), rtol=1e-12, atol=1e-12 * np.abs(y).max())
+    assert np.array_equal(oracle.mx_gemm(ac, asf, bc, bsf, rows=slice(5, 9)), y[5:9])
