@@ -277,6 +277,41 @@ nvfp4_status nvfp4_gemm_w4a16(const void *x_bf16, const uint8_t *w_codes, const 
                               const float *w_scale, int64_t M, int64_t N, int64_t K,
                               void *y, int y_dtype, int *dev_status, nvfp4_stream_t stream);
 
+/*
+ * MX variant ([RFC] Related: the MXFP4 format, "related but different"):
+ * E2M1 elements in blocks of 32 along k, one power-of-two scale per block as
+ * an unsigned E8M0 byte (value 2^(byte - 127)), no tensor scale.  The pages
+ * give no scale rule; the OCP Microscaling one is used:
+ *   e = floor(log2 max|x|) - 2, clamped to [-127, 127] (-127 for an all-zero
+ *   block); byte = e + 127; code = E2M1_rne(clip(x / 2^e, -6, 6)), sign kept.
+ * Codes [rows, k/2] as for NVFP4; scales in the same tensor-core layout with
+ * kb = k/32 blocks per row:
+ *   byte of (row r, block c) at ((r/128)*(kb/4) + c/4)*512 + (r%32)*16
+ *                               + ((r%128)/32)*4 + c%4,
+ * rows padded to 128 with zero bytes.  k must be a multiple of 128.
+ */
+size_t nvfp4_mx_sf_bytes(int64_t rows, int64_t k);      /* ceil(rows/128)*128 * k/32, 0 if invalid */
+
+/* MX quantization of a bf16 [rows, k] tensor (row stride ld_x, ld_x % 8 == 0),
+ * rows <= 4194240.  One kernel; pointers 16-byte aligned. */
+nvfp4_status nvfp4_mx_quantize(const void *x_bf16, int64_t rows, int64_t k, int64_t ld_x,
+                               uint8_t *codes, uint8_t *sf, nvfp4_stream_t stream);
+
+/* v = e2m1(code) * 2^(byte - 127), exact in bf16 and FP32; out [rows, k]. */
+nvfp4_status nvfp4_mx_dequantize(const uint8_t *codes, const uint8_t *sf, int64_t rows, int64_t k,
+                                 void *out, int out_dtype, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_mx_gemm -- Y = act(sum_k a^ b^), a^ = e2m1(a) * 2^(sfa - 127) (and b^),
+ * with the block-32 E8M0 tensor-core MMA (kind::mxf4), FP32 accumulation.
+ * A [M, K] and B [N, K] as nvfp4_mx_quantize writes them; K % 128 == 0;
+ * Y [M, N] bf16 (N % 8 == 0) or FP32 (N % 4 == 0); act as nvfp4_gemm_w4a4.
+ * One persistent kernel (128 x 128 tiles).
+ */
+nvfp4_status nvfp4_mx_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const uint8_t *b_codes,
+                           const uint8_t *b_sf, int64_t M, int64_t N, int64_t K, void *y, int y_dtype,
+                           int act, int *dev_status, nvfp4_stream_t stream);
+
 /* Static text for a status code. */
 const char *nvfp4_status_string(nvfp4_status s);
 

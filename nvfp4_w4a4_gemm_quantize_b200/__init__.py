@@ -8,10 +8,12 @@ memory and streams.
 Low-level (same names and argument order as the C calls):
     nvfp4_sf_bytes, nvfp4_quantize_workspace_bytes, nvfp4_quantize,
     nvfp4_quantize_noalloc, nvfp4_dequantize, nvfp4_fake_quantize, nvfp4_ste_backward,
-    nvfp4_gemm_w4a4, nvfp4_gemm_w4a4_grouped, nvfp4_gemm_w4a16, nvfp4_launch_count
+    nvfp4_gemm_w4a4, nvfp4_gemm_w4a4_grouped, nvfp4_gemm_w4a16, nvfp4_mx_sf_bytes, nvfp4_mx_quantize,
+    nvfp4_mx_dequantize, nvfp4_mx_gemm, nvfp4_launch_count
 Convenience (allocate outputs with torch, then call the above):
     NVFP4Tensor, quantize, dequantize, gemm_w4a4, gemm_w4a4_grouped, gemm_w4a16,
-    fake_quantize, ste_backward, FakeQuantizeSTE (autograd: the two kernels)
+    fake_quantize, ste_backward, FakeQuantizeSTE (autograd: the two kernels),
+    MXTensor, mx_quantize, mx_dequantize, mx_gemm
 """
 from __future__ import annotations
 
@@ -129,6 +131,26 @@ def nvfp4_gemm_w4a4_grouped(problems, y_dtype=NVFP4_DTYPE_BF16, dev_status=None,
     st = lib().nvfp4_gemm_w4a4_grouped(ctypes.addressof(arr), len(problems), y_dtype, _ptr(dev_status),
                                        _stream(stream))
     check(st, "nvfp4_gemm_w4a4_grouped")
+
+
+def nvfp4_mx_sf_bytes(rows: int, k: int) -> int:
+    return int(lib().nvfp4_mx_sf_bytes(rows, k))
+
+
+def nvfp4_mx_quantize(x, rows, k, ld_x, codes, sf, stream=None) -> None:
+    check(lib().nvfp4_mx_quantize(_ptr(x), rows, k, ld_x, _ptr(codes), _ptr(sf), _stream(stream)),
+          "nvfp4_mx_quantize")
+
+
+def nvfp4_mx_dequantize(codes, sf, rows, k, out, out_dtype, stream=None) -> None:
+    check(lib().nvfp4_mx_dequantize(_ptr(codes), _ptr(sf), rows, k, _ptr(out), out_dtype, _stream(stream)),
+          "nvfp4_mx_dequantize")
+
+
+def nvfp4_mx_gemm(a_codes, a_sf, b_codes, b_sf, M, N, K, y, y_dtype=NVFP4_DTYPE_BF16, act=0, dev_status=None,
+                  stream=None) -> None:
+    check(lib().nvfp4_mx_gemm(_ptr(a_codes), _ptr(a_sf), _ptr(b_codes), _ptr(b_sf), M, N, K, _ptr(y), y_dtype, act,
+                              _ptr(dev_status), _stream(stream)), "nvfp4_mx_gemm")
 
 
 def nvfp4_gemm_w4a16(x, w_codes, w_sf, w_scale, M, N, K, y, y_dtype=NVFP4_DTYPE_BF16,
@@ -284,3 +306,40 @@ class FakeQuantizeSTE(torch.autograd.Function):
             return grad_y, None, None
         (m,) = ctx.saved_tensors
         return ste_backward(grad_y.contiguous(), m), None, None
+
+
+# ----------------------------------------------------------------- MX variant
+@dataclass
+class MXTensor:
+    """codes [rows, k/2] uint8, sf [mx_sf_bytes] uint8 (E8M0, block 32)."""
+    codes: torch.Tensor
+    sf: torch.Tensor
+    rows: int
+    k: int
+
+    @staticmethod
+    def empty(rows: int, k: int, device) -> "MXTensor":
+        return MXTensor(torch.empty(rows, k // 2, dtype=torch.uint8, device=device),
+                        torch.empty(max(nvfp4_mx_sf_bytes(rows, k), 16), dtype=torch.uint8, device=device), rows, k)
+
+
+def mx_quantize(x: torch.Tensor, out: MXTensor | None = None, stream=None) -> MXTensor:
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, k = x.shape
+    q = out if out is not None else MXTensor.empty(rows, k, x.device)
+    nvfp4_mx_quantize(x, rows, k, x.stride(0), q.codes, q.sf, stream)
+    return q
+
+
+def mx_dequantize(q: MXTensor, dtype=torch.bfloat16, stream=None) -> torch.Tensor:
+    out = torch.empty(q.rows, q.k, dtype=dtype, device=q.codes.device)
+    nvfp4_mx_dequantize(q.codes, q.sf, q.rows, q.k, out, _DT[dtype], stream)
+    return out
+
+
+def mx_gemm(a: MXTensor, b: MXTensor, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
+            act=NVFP4_ACT_NONE, dev_status=None, stream=None) -> torch.Tensor:
+    assert a.k == b.k
+    y = out if out is not None else torch.empty(a.rows, b.rows, dtype=out_dtype, device=a.codes.device)
+    nvfp4_mx_gemm(a.codes, a.sf, b.codes, b.sf, a.rows, b.rows, a.k, y, _DT[y.dtype], act, dev_status, stream)
+    return y

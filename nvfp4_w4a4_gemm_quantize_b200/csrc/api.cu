@@ -260,6 +260,63 @@ nvfp4_status nvfp4_gemm_w4a4_grouped(const nvfp4_gemm_problem* problems, int cou
     return cuda_status(launch_gemm_w4a4_grouped(args, n, sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t nvfp4_mx_sf_bytes(int64_t rows, int64_t k) {
+    if (rows < 0 || k <= 0 || (k % 128) != 0) return 0;
+    return (size_t)((rows + 127) / 128) * 128 * (size_t)(k / 32);
+}
+
+nvfp4_status nvfp4_mx_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, uint8_t* codes, uint8_t* sf,
+                               nvfp4_stream_t stream) {
+    if (rows < 0 || k <= 0 || ld_x < k) return NVFP4_ERR_INVALID_ARG;
+    if (rows > 0 && (!x_bf16 || !codes || !sf)) return NVFP4_ERR_INVALID_ARG;
+    if (k % 128 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (rows > (int64_t)65535 * 64 || k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(sf) || (ld_x % 8) != 0) return NVFP4_ERR_MISALIGNED;
+    nvfp4_status st = device_ok(nullptr);
+    if (st != NVFP4_OK) return st;
+    if (rows == 0) return NVFP4_OK;
+    return cuda_status(launch_mx_quantize(static_cast<const uint16_t*>(x_bf16), rows, k, ld_x, codes, sf,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_mx_dequantize(const uint8_t* codes, const uint8_t* sf, int64_t rows, int64_t k, void* out,
+                                 int out_dtype, nvfp4_stream_t stream) {
+    if (rows < 0 || k <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (out_dtype != NVFP4_DTYPE_BF16 && out_dtype != NVFP4_DTYPE_F32) return NVFP4_ERR_INVALID_ARG;
+    if (rows > 0 && (!codes || !sf || !out)) return NVFP4_ERR_INVALID_ARG;
+    if (k % 128 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(codes) || !aligned16(sf) || !aligned16(out)) return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    nvfp4_status st = device_ok(&sms);
+    if (st != NVFP4_OK) return st;
+    if (rows == 0) return NVFP4_OK;
+    return cuda_status(launch_mx_dequantize(codes, sf, rows, k, out, out_dtype == NVFP4_DTYPE_BF16, sms,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_mx_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const uint8_t* b_codes, const uint8_t* b_sf,
+                           int64_t M, int64_t N, int64_t K, void* y, int y_dtype, int act, int* dev_status,
+                           nvfp4_stream_t stream) {
+    if (M < 0 || N <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (K % 128 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0) return NVFP4_OK;
+    if (!a_codes || !a_sf || !b_codes || !b_sf || !y) return NVFP4_ERR_INVALID_ARG;
+    if (y_dtype != NVFP4_DTYPE_BF16 && y_dtype != NVFP4_DTYPE_F32) return NVFP4_ERR_INVALID_ARG;
+    if (act != NVFP4_ACT_NONE && act != NVFP4_ACT_GELU_TANH) return NVFP4_ERR_INVALID_ARG;
+    if (y_dtype == NVFP4_DTYPE_BF16 && N % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (y_dtype == NVFP4_DTYPE_F32 && N % 4 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (M >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(b_codes) || !aligned16(b_sf) || !aligned16(y))
+        return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    nvfp4_status st = device_ok(&sms);
+    if (st != NVFP4_OK) return st;
+    GemmW4A4Args a{a_codes, a_sf, nullptr, b_codes, b_sf, nullptr, M, N, K, y, y_dtype,
+                   nullptr, nullptr, nullptr, nullptr, dev_status, act, true};
+    return cuda_status(launch_gemm_w4a4(a, sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 nvfp4_status nvfp4_gemm_w4a16(const void* x_bf16, const uint8_t* w_codes, const uint8_t* w_sf, const float* w_scale,
                               int64_t M, int64_t N, int64_t K, void* y, int y_dtype, int* dev_status,
                               nvfp4_stream_t stream) {

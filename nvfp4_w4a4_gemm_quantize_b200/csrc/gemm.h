@@ -22,6 +22,7 @@ struct GemmW4A4Args {
     float* y_amax;
     int* dev_status;
     int act;                  // epilogue activation: 0 none, 1 GELU (tanh form)
+    bool mx;                  // MX operands: blocks of 32, E8M0 scales, no tensor scale
 };
 
 cudaError_t launch_gemm_w4a4(const GemmW4A4Args& a, int num_sms, cudaStream_t stream);

@@ -46,21 +46,25 @@ constexpr int BM = 128;
 constexpr int BK_BYTES = 128;                    // 256 FP4 values per row per stage
 constexpr int A_BYTES = BM * BK_BYTES;           // 16 KB
 constexpr int SF_ATOM = 512;                     // 128 rows x 4 blocks
-constexpr int SFA_BYTES = 4 * SF_ATOM;           // 4 K=64 steps
 constexpr int kThreads = 192;
 constexpr int kEpiWarps = 4;
 constexpr int kGroupM = 16;                      // rasterisation group (M blocks)
 
 enum OutKind { OUT_BF16 = 0, OUT_F32 = 1, OUT_NVFP4 = 2 };
 
-template <int BN, int STAGES>
+// MXS: the MX operand format (blocks of 32 with E8M0 scales, kind::mxf4,
+// two scale atoms per 256-K stage, one per two K = 64 steps); otherwise
+// NVFP4 (blocks of 16 with E4M3 scales, four atoms per stage).
+template <int BN, int STAGES, bool MXS = false>
 struct Cfg {
+    static constexpr int SF_ATOMS = MXS ? 2 : 4;              // scale atoms per 128 rows per stage
+    static constexpr int SFA_BYTES = SF_ATOMS * SF_ATOM;
     static constexpr int B_BYTES = BN * BK_BYTES;
     static constexpr int SFB_BYTES = (BN / 128) * SFA_BYTES;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
     static constexpr int ACC_BUFS = (BN == 128) ? 2 : 1;
-    static constexpr int SF_COLS_STEP = 4 + BN / 32;          // SFA 4 columns + SFB BN/32
-    static constexpr int SF_COLS_STAGE = 4 * SF_COLS_STEP;
+    static constexpr int SF_COLS_STEP = 4 + BN / 32;          // per atom group: SFA 4 columns + SFB BN/32
+    static constexpr int SF_COLS_STAGE = SF_ATOMS * SF_COLS_STEP;
     static constexpr int EPI_BUF_BYTES = 32 * 128;            // 32 rows x 128 B (f32 worst case)
     static constexpr int EPI_BYTES = kEpiWarps * 2 * EPI_BUF_BYTES;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024;
@@ -123,10 +127,11 @@ __device__ __forceinline__ void flush_amax(float v, float* dst, int lane) {
     if (dst != nullptr && lane == 0 && v > 0.0f) atomicMax(reinterpret_cast<int*>(dst), __float_as_int(v));
 }
 
-template <int BN, int STAGES, int OUT, int ACT>
+template <int BN, int STAGES, int OUT, int ACT, bool MXS>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p) {
-    using C = Cfg<BN, STAGES>;
+    using C = Cfg<BN, STAGES, MXS>;
+    constexpr int kAtomK = MXS ? 128 : 64;        // K covered by one 128-row scale atom
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES];
     __shared__ __align__(8) uint64_t accf_bar[C::ACC_BUFS], acce_bar[C::ACC_BUFS];
@@ -160,7 +165,7 @@ gemm_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p)
     // region once so such rows read finite scales (their codes are zero).
     for (int s = 0; s < STAGES; ++s) {
         uint32_t* z = reinterpret_cast<uint32_t*>(smem + s * C::STAGE_BYTES + A_BYTES + C::B_BYTES);
-        for (int i = threadIdx.x; i < (SFA_BYTES + C::SFB_BYTES) / 4; i += kThreads) z[i] = 0u;
+        for (int i = threadIdx.x; i < (C::SFA_BYTES + C::SFB_BYTES) / 4; i += kThreads) z[i] = 0u;
     }
     fence_proxy_async_smem();
     if (warp == 1) {
@@ -193,14 +198,14 @@ gemm_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p)
             const int nblk0 = nb * (BN / 128);
             const int nblk_total = (pr.N + 127) / 128;
             const int num_kt = (pr.K + 255) / 256;
-            const int k_atoms = pr.K / 64;        // scale atoms per 128-row block
+            const int k_atoms = pr.K / kAtomK;    // scale atoms per 128-row block
             for (int kt = 0; kt < num_kt; ++kt) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&empty_bar[stage], phase ^ 1u, wc) ? 1 : 0)) {
                     ok = false;
                     break;
                 }
                 uint8_t* sbase = smem + stage * C::STAGE_BYTES;
-                const int natoms = min(4, k_atoms - kt * 4);
+                const int natoms = min(C::SF_ATOMS, k_atoms - kt * C::SF_ATOMS);
                 int nsfb = 0;
                 for (int j = 0; j < BN / 128; ++j) nsfb += (nblk0 + j < nblk_total) ? 1 : 0;
                 if (elect_one()) {
@@ -209,11 +214,11 @@ gemm_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p)
                     tma_load_2d(sbase, &maps.a[g], &full_bar[stage], kt * BK_BYTES, mb * BM, pol_a);
                     tma_load_2d(sbase + A_BYTES, &maps.b[g], &full_bar[stage], kt * BK_BYTES, nb * BN, pol_b);
                     bulk_load(sbase + A_BYTES + C::B_BYTES,
-                              pr.a_sf + ((int64_t)mb * k_atoms + kt * 4) * SF_ATOM, natoms * SF_ATOM,
+                              pr.a_sf + ((int64_t)mb * k_atoms + kt * C::SF_ATOMS) * SF_ATOM, natoms * SF_ATOM,
                               &full_bar[stage], pol_a);
                     for (int j = 0; j < nsfb; ++j)
-                        bulk_load(sbase + A_BYTES + C::B_BYTES + SFA_BYTES + j * SFA_BYTES,
-                                  pr.b_sf + ((int64_t)(nblk0 + j) * k_atoms + kt * 4) * SF_ATOM,
+                        bulk_load(sbase + A_BYTES + C::B_BYTES + C::SFA_BYTES + j * C::SFA_BYTES,
+                                  pr.b_sf + ((int64_t)(nblk0 + j) * k_atoms + kt * C::SF_ATOMS) * SF_ATOM,
                                   natoms * SF_ATOM, &full_bar[stage], pol_b);
                 }
                 __syncwarp();
@@ -234,7 +239,7 @@ gemm_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        constexpr uint32_t idesc = idesc_nvf4(BM, BN);
+        constexpr uint32_t idesc = MXS ? idesc_mxf4(BM, BN) : idesc_nvf4(BM, BN);
         const uint32_t smem0 = smem_u32(smem);
         int stage = 0;
         uint32_t phase = 0;
@@ -250,7 +255,7 @@ gemm_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p)
             tc_fence_after();
             const Problem& pr = p.pr[find_problem(p, t)];
             const int num_kt = (pr.K + 255) / 256;
-            const int k_atoms = pr.K / 64;
+            const int k_steps = pr.K / 64;       // K = 64 MMA steps
             const uint32_t d_tmem = tmem_base + acc * BN;
             for (int kt = 0; kt < num_kt; ++kt) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[stage], phase, wc) ? 1 : 0)) {
@@ -260,19 +265,33 @@ gemm_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p)
                 tc_fence_after();
                 const uint32_t sbase = smem0 + stage * C::STAGE_BYTES;
                 const uint32_t sfa_s = sbase + A_BYTES + C::B_BYTES;
-                const uint32_t sfb_s = sfa_s + SFA_BYTES;
+                const uint32_t sfb_s = sfa_s + C::SFA_BYTES;
                 const uint32_t sf_col = sf_base + stage * C::SF_COLS_STAGE;
-                const int nks = min(4, k_atoms - kt * 4);
+                const int nks = min(4, k_steps - kt * 4);
                 if (elect_one()) {
                     for (int ks = 0; ks < nks; ++ks) {
-                        const uint32_t col = sf_col + ks * C::SF_COLS_STEP;
-                        tc_cp_32x128b_warpx4(col, sdesc_sf(sfa_s + ks * SF_ATOM));
+                        // NVFP4: one atom per K = 64 step; MX: one per two steps,
+                        // the step's two scale bytes selected by a byte id (0 or 2)
+                        const int at = MXS ? (ks >> 1) : ks;
+                        const uint32_t col = sf_col + at * C::SF_COLS_STEP;
+                        if (!MXS || (ks & 1) == 0) {
+                            tc_cp_32x128b_warpx4(col, sdesc_sf(sfa_s + at * SF_ATOM));
 #pragma unroll
-                        for (int j = 0; j < BN / 128; ++j)
-                            tc_cp_32x128b_warpx4(col + 4 + 4 * j, sdesc_sf(sfb_s + j * SFA_BYTES + ks * SF_ATOM));
-                        tc_mma_nvf4(d_tmem, sdesc_kmajor_sw128(sbase + ks * 32),
-                                    sdesc_kmajor_sw128(sbase + A_BYTES + ks * 32), idesc, col, col + 4,
-                                    (kt | ks) != 0 ? 1u : 0u);
+                            for (int j = 0; j < BN / 128; ++j)
+                                tc_cp_32x128b_warpx4(col + 4 + 4 * j,
+                                                     sdesc_sf(sfb_s + j * C::SFA_BYTES + at * SF_ATOM));
+                        }
+                        if (MXS) {
+                            const uint32_t byte = (uint32_t)(ks & 1) * 2u;
+                            tc_mma_mxf4(d_tmem, sdesc_kmajor_sw128(sbase + ks * 32),
+                                        sdesc_kmajor_sw128(sbase + A_BYTES + ks * 32),
+                                        idesc | (byte << 29) | (byte << 4), col | (byte << 30),
+                                        (col + 4) | (byte << 30), (kt | ks) != 0 ? 1u : 0u);
+                        } else {
+                            tc_mma_nvf4(d_tmem, sdesc_kmajor_sw128(sbase + ks * 32),
+                                        sdesc_kmajor_sw128(sbase + A_BYTES + ks * 32), idesc, col, col + 4,
+                                        (kt | ks) != 0 ? 1u : 0u);
+                        }
                     }
                     tc_commit(&empty_bar[stage]);
                 }
@@ -309,7 +328,8 @@ gemm_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p)
                 // a new problem: flush the previous one's running amax, load this one's scales
                 if (OUT == OUT_NVFP4 && g_prev >= 0) flush_amax(amax_run, p.pr[g_prev].y_amax, lane);
                 amax_run = 0.0f;
-                alpha = __fmul_rn(*pr.a_scale, *pr.b_scale);
+                // MX operands have no tensor scale: a null scale reads as 1
+                alpha = __fmul_rn(pr.a_scale ? *pr.a_scale : 1.0f, pr.b_scale ? *pr.b_scale : 1.0f);
                 if (OUT == OUT_NVFP4) {
                     g_y = *pr.y_scale;
                     sc_y = scale_consts(g_y);
@@ -427,9 +447,9 @@ gemm_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p)
     }
 }
 
-template <int BN, int STAGES, int OUT, int ACT>
+template <int BN, int STAGES, int OUT, int ACT, bool MXS>
 cudaError_t launch_cfg(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream) {
-    using C = Cfg<BN, STAGES>;
+    using C = Cfg<BN, STAGES, MXS>;
     if (count < 1 || count > kMaxGroup) return cudaErrorInvalidValue;
     Maps maps;
     Params p;
@@ -475,7 +495,7 @@ cudaError_t launch_cfg(const GemmW4A4Args* probs, int count, int num_sms, cudaSt
     p.dev_status = probs[0].dev_status;
     if (tiles == 0) return cudaSuccess;
 
-    auto kern = gemm_kernel<BN, STAGES, OUT, ACT>;
+    auto kern = gemm_kernel<BN, STAGES, OUT, ACT, MXS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const int grid = tiles < num_sms ? tiles : num_sms;
@@ -486,8 +506,12 @@ cudaError_t launch_cfg(const GemmW4A4Args* probs, int count, int num_sms, cudaSt
 
 template <int OUT>
 static cudaError_t launch_group(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream) {
-    if (probs[0].act == ACT_GELU_TANH) return launch_cfg<128, 5, OUT, ACT_GELU_TANH>(probs, count, num_sms, stream);
-    return launch_cfg<128, 5, OUT, ACT_NONE>(probs, count, num_sms, stream);
+    const bool gelu = probs[0].act == ACT_GELU_TANH;
+    if (probs[0].mx)
+        return gelu ? launch_cfg<128, 5, OUT, ACT_GELU_TANH, true>(probs, count, num_sms, stream)
+                    : launch_cfg<128, 5, OUT, ACT_NONE, true>(probs, count, num_sms, stream);
+    return gelu ? launch_cfg<128, 5, OUT, ACT_GELU_TANH, false>(probs, count, num_sms, stream)
+                : launch_cfg<128, 5, OUT, ACT_NONE, false>(probs, count, num_sms, stream);
 }
 
 }  // namespace w4a4
@@ -498,7 +522,7 @@ cudaError_t launch_gemm_w4a4(const GemmW4A4Args& a, int num_sms, cudaStream_t st
     // N a multiple of 256: CTA-pair kernel with 256 x 256 tiles.  Otherwise
     // (N = 1152, 3456, ...): single-CTA 128 x 128 tiles with a double-buffered
     // accumulator, so no tile column is wasted on padding.
-    if (a.N % 256 == 0) return launch_gemm_w4a4_2sm(a, num_sms, stream);
+    if (a.N % 256 == 0 && !a.mx) return launch_gemm_w4a4_2sm(a, num_sms, stream);
     return launch_gemm_w4a4_grouped(&a, 1, num_sms, stream);
 }
 

@@ -32,6 +32,12 @@ cudaError_t launch_fake_quantize(const uint16_t* x, int64_t rows, int64_t k, int
 cudaError_t launch_ste_backward(const void* grad_y, const uint8_t* mask, int64_t rows, int64_t k, bool f32,
                                 void* grad_x, int num_sms, cudaStream_t stream);
 
+cudaError_t launch_mx_quantize(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes, uint8_t* sf,
+                               cudaStream_t stream);
+
+cudaError_t launch_mx_dequantize(const uint8_t* codes, const uint8_t* sf, int64_t rows, int64_t k, void* out,
+                                 bool bf16, int num_sms, cudaStream_t stream);
+
 cudaError_t launch_debug_wait_timeout(int* dev_status, uint64_t limit_ns, cudaStream_t stream);
 
 void reset_noalloc_cache();

@@ -235,6 +235,19 @@ __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uin
         : "memory");
 }
 
+// D[tmem] (+)= A * B^T with MX operands: E2M1 in blocks of 32 with E8M0
+// scales (two per row per K = 64 step; the scale addresses carry the byte id
+// in bits 30-31, as the instruction descriptor does).
+__device__ __forceinline__ void tc_mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, FP32 accumulation.
 __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                             uint32_t accumulate) {
@@ -443,6 +456,13 @@ __device__ __forceinline__ uint64_t sdesc_sf(uint32_t saddr) {
 // UE4M3 (bit 23 = 0), M >> 4 in [24,29), scale-factor ids 0, dense K = 64.
 __host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
     return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Instruction descriptor, block-scaled kind::mxf4: as idesc_nvf4 with scale
+// type UE8M0 (bit 23 = 1); the scale-factor byte ids (bits [29,31) for A,
+// [4,6) for B) are added per MMA.
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N) {
+    return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24);
 }
 
 // Instruction descriptor, kind::f16 with bf16 A/B (format 1), FP32 D (bits

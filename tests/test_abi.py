@@ -32,7 +32,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 14, names
+    assert len(names) == 18, names
     for n in names:
         assert hasattr(L, n), n
         assert n in _lib.SIGNATURES, n
@@ -181,6 +181,29 @@ def test_grouped_gemm_rejects_bad_arguments(L):
     assert g(addr(arr), 2, 0, None, None) == INVALID
     arr = _problems(2, {1: dict(act=1)})                                              # mixed activations
     assert g(addr(arr), 2, 0, None, None) == INVALID
+
+
+def test_mx_calls_reject_bad_arguments(L):
+    assert L.nvfp4_mx_sf_bytes(128, 256) == 128 * 8
+    assert L.nvfp4_mx_sf_bytes(130, 384) == 256 * 12
+    assert L.nvfp4_mx_sf_bytes(128, 64) == 0                    # k not a multiple of 128
+    q = L.nvfp4_mx_quantize
+    assert q(A, 128, 192, 192, B, C, None) == SHAPE
+    assert q(None, 128, 256, 256, B, C, None) == INVALID
+    assert q(A, 128, 256, 128, B, C, None) == INVALID
+    assert q(A + 2, 128, 256, 256, B, C, None) == MISALIGNED
+    assert q(A, 128, 256, 260, B, C, None) == MISALIGNED
+    assert q(A, 65535 * 64 + 1, 256, 256, B, C, None) == SHAPE
+    d = L.nvfp4_mx_dequantize
+    assert d(A, B, 128, 256, C, 4, None) == INVALID
+    assert d(A, B, 128, 64, C, 0, None) == SHAPE
+    g = L.nvfp4_mx_gemm
+    assert g(A, B, A, B, 128, 256, 192, C, 0, 0, None, None) == SHAPE
+    assert g(A, B, A, B, 128, 260, 256, C, 0, 0, None, None) == SHAPE
+    assert g(A, B, A, B, 128, 256, 256, None, 0, 0, None, None) == INVALID
+    assert g(A, B, A, B, 128, 256, 256, C, 0, 3, None, None) == INVALID
+    assert g(A, B + 4, A, B, 128, 256, 256, C, 0, 0, None, None) == MISALIGNED
+    assert g(A, B, A, B, -2, 256, 256, C, 0, 0, None, None) == INVALID
 
 
 def test_w4a16_rejects_bad_arguments(L):
