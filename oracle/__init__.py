@@ -30,6 +30,9 @@ Parity status per function:
   mx_quantize / mx_dequantize / mx_gemm                 -- pinned (brute-force
       exponent and nearest-grid searches on tiny inputs, grid membership and
       the error bound, power-of-two fixed points, a float64 library matmul)
+  quantize_block / block_size_errors / select_block_size -- pinned (block 16
+      equals quantize, brute force for blocks 32 and 64, errors against the
+      dequantized oracle quantization and brute force, Eq. 9 limits)
   gelu_tanh                                             -- pinned (torch's
       float64 tanh-form GELU, the odd-part identity g(v) - g(-v) = v, the erf
       form within 1e-3, limits)
@@ -101,6 +104,12 @@ def lib() -> ctypes.CDLL:
         L.oracle_mx_dequantize_f64.restype = None
         L.oracle_mx_gemm_rows.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p]
         L.oracle_mx_gemm_rows.restype = None
+        L.oracle_quantize_block_bf16.argtypes = [_p, _i64, _i64, _i64, ctypes.c_int, ctypes.c_int, _p, _p, _p]
+        L.oracle_quantize_block_bf16.restype = None
+        L.oracle_block_size_errors.argtypes = [_p, _i64, _i64, _i64, _f32, _p, _p]
+        L.oracle_block_size_errors.restype = None
+        L.oracle_select_block_size.argtypes = [_p, ctypes.c_double, ctypes.c_double]
+        L.oracle_select_block_size.restype = ctypes.c_int
         L.oracle_gelu_tanh.argtypes = [ctypes.c_double]
         L.oracle_gelu_tanh.restype = ctypes.c_double
         L.oracle_gelu_tanh_array.argtypes = [_p, _i64, _p]
@@ -383,3 +392,42 @@ def mx_sf_matrix(sf: np.ndarray, rows: int, k: int) -> np.ndarray:
     c = np.arange(kb)[None, :]
     off = ((r // 128) * (kb // 4) + c // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + c % 4
     return sf[off]
+
+
+# ---------------------------------------------------------------- adaptive block size
+BLOCK_SIZES = (1, 2, 4, 8, 16, 32, 64)
+
+
+def quantize_block(x, block: int, scale: float | None = None):
+    """NVFP4 with `block` values per E4M3 scale (16, 32 or 64), scales repeated
+    into the block-16 layout.  Returns (codes, sf, g)."""
+    L = lib()
+    xb = bf16_bits(x)
+    rows, k = xb.shape
+    assert block in (16, 32, 64) and k % 64 == 0
+    codes = np.zeros((rows, k // 2), np.uint8)
+    sf = np.zeros(sf_bytes(rows, k), np.uint8)
+    g = np.zeros(1, np.float32)
+    if scale is not None:
+        g[0] = np.float32(scale)
+    L.oracle_quantize_block_bf16(_ptr(xb), rows, k, k, block, 1 if scale is not None else 0, _ptr(g),
+                                 _ptr(codes), _ptr(sf))
+    return codes, sf, np.float32(g[0])
+
+
+def block_size_errors(x, g: float):
+    """Squared quantization errors for b = 1, 2, ..., 64 (Eq. 9's Error before
+    normalisation) and the sum of squares of x."""
+    L = lib()
+    xb = bf16_bits(x)
+    rows, k = xb.shape
+    err = np.zeros(7, np.float64)
+    ss = np.zeros(1, np.float64)
+    L.oracle_block_size_errors(_ptr(xb), rows, k, k, float(g), _ptr(err), _ptr(ss))
+    return err, float(ss[0])
+
+
+def select_block_size(err, sumsq: float, lam: float) -> int:
+    """Eq. 9: argmin_b Error(b) / sum x^2 + lambda (4 + 8/b) / 12."""
+    e = np.ascontiguousarray(err, np.float64)
+    return int(lib().oracle_select_block_size(_ptr(e), float(sumsq), float(lam)))

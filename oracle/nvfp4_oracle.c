@@ -539,3 +539,100 @@ void oracle_mx_gemm_rows(const uint8_t *a_codes, const uint8_t *a_sf, const uint
     free(bh);
     free(ah);
 }
+
+/* ---------------------- adaptive block size (Alg. 1) ---------------------- */
+/* Two-level NVFP4 quantization with a block of `block` values along k
+ * [DiT, Algorithmic framework: Algorithm 1 / Eq. 9 choose the block size per
+ * layer from {1, 2, 4, 8, 16, 32, 64}]: the same rule as oracle_quantize_f32
+ * with the block maximum taken over `block` values,
+ *   sf = E4M3(a_b / (6 g)),  s = dec(sf) * g,  code = E2M1(x / s).
+ * For block >= 16 (a multiple of 16 dividing 64) the codes and scales are
+ * written in the block-16 tensor-core layout, each block scale repeated in its
+ * block/16 slots, so the block-16 GEMM multiplies them unchanged.           */
+void oracle_quantize_block_bf16(const uint16_t *x, int64_t rows, int64_t k, int64_t ld, int block,
+                                int scale_given, float *g_io, uint8_t *codes, uint8_t *sf)
+{
+    float g = scale_given ? *g_io : oracle_tensor_scale_bf16(x, rows, k, ld);
+    if (!scale_given) *g_io = g;
+    const int64_t kb = k / 16;
+    memset(sf, 0, (size_t)oracle_sf_bytes(rows, k));
+    memset(codes, 0, (size_t)(rows * (k / 2)));
+    const float d = 6.0f * g;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < k / block; ++c) {
+            float ab = 0.0f;
+            for (int i = 0; i < block; ++i) {
+                float a = fabsf(oracle_bf16_to_f32(x[r * ld + c * block + i]));
+                if (a > ab) ab = a;
+            }
+            unsigned sfc = (d > 0.0f) ? oracle_e4m3_encode(ab / d) : 0u;
+            for (int t = 0; t < block / 16; ++t)
+                sf[oracle_sf_offset(r, c * (block / 16) + t, kb)] = (uint8_t)sfc;
+            float s = (float)oracle_e4m3_decode(sfc) * g;
+            for (int i = 0; i < block; ++i) {
+                int64_t j = c * block + i;
+                unsigned code = 0u;
+                if (s != 0.0f) code = oracle_e2m1_encode(oracle_bf16_to_f32(x[r * ld + j]) / s);
+                codes[r * (k / 2) + j / 2] |= (uint8_t)(code << (4 * (j & 1)));
+            }
+        }
+}
+
+/* Error(l, b) of Eq. 9 for every candidate block size b = 2^i, i = 0..6: the
+ * squared quantization error sum_j (x_j - Q_b(x)_j)^2, Q_b(x)_j =
+ * e2m1(code_j) * dec(sf) * g with the rule above (any b dividing k), in
+ * double; err[7] receives them and *sumsq = sum_j x_j^2.  The tensor scale
+ * is g (the caller's, e.g. amax / 2688).                                     */
+void oracle_block_size_errors(const uint16_t *x, int64_t rows, int64_t k, int64_t ld, float g,
+                              double *err, double *sumsq)
+{
+    const float d = 6.0f * g;
+    double ss = 0.0;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < k; ++j) {
+            double v = (double)oracle_bf16_to_f32(x[r * ld + j]);
+            ss += v * v;
+        }
+    *sumsq = ss;
+    for (int i = 0; i < 7; ++i) {
+        const int b = 1 << i;
+        double e = 0.0;
+        for (int64_t r = 0; r < rows; ++r)
+            for (int64_t c = 0; c < k / b; ++c) {
+                float ab = 0.0f;
+                for (int t = 0; t < b; ++t) {
+                    float a = fabsf(oracle_bf16_to_f32(x[r * ld + c * b + t]));
+                    if (a > ab) ab = a;
+                }
+                unsigned sfc = (d > 0.0f) ? oracle_e4m3_encode(ab / d) : 0u;
+                double sdec = oracle_e4m3_decode(sfc);
+                float s = (float)sdec * g;
+                for (int t = 0; t < b; ++t) {
+                    float xv = oracle_bf16_to_f32(x[r * ld + c * b + t]);
+                    double q = 0.0;
+                    if (s != 0.0f) q = oracle_e2m1_decode(oracle_e2m1_encode(xv / s)) * sdec * (double)g;
+                    double diff = (double)xv - q;
+                    e += diff * diff;
+                }
+            }
+        err[i] = e;
+    }
+}
+
+/* Eq. 9: argmin over b of Error(b) + lambda * Memory(b) / Memory_max, with
+ * Error(b) = err[b] / sumsq (relative squared error) and Memory(b) = 4 + 8/b
+ * bits per value (E2M1 element + one E8-bit E4M3 scale per block; the tensor
+ * scale's 32 bits are shared by the whole tensor and left out), so
+ * Memory_max = Memory(1) = 12.  Returns the chosen b (the first minimum).    */
+int oracle_select_block_size(const double *err, double sumsq, double lambda)
+{
+    int best = 1;
+    double bestv = 0.0;
+    for (int i = 0; i < 7; ++i) {
+        const int b = 1 << i;
+        double e = sumsq > 0.0 ? err[i] / sumsq : 0.0;
+        double v = e + lambda * (4.0 + 8.0 / b) / 12.0;
+        if (i == 0 || v < bestv) { bestv = v; best = b; }
+    }
+    return best;
+}

@@ -676,3 +676,84 @@ def test_mx_zero_tensor_and_gemm_vs_library_matmul():
     ref = torch.from_numpy(oracle.mx_dequantize(ac, asf)) @ torch.from_numpy(oracle.mx_dequantize(bc, bsf)).T
     assert np.allclose(y, ref.numpy(), rtol=1e-12, atol=1e-12 * np.abs(y).max())
     assert np.array_equal(oracle.mx_gemm(ac, asf, bc, bsf, rows=slice(5, 9)), y[5:9])
+
+
+# ------------------------------------------------------------------ adaptive block size (Alg. 1, Eq. 9)
+def brute_block_quantize(xf32: np.ndarray, block: int, g: np.float32):
+    """Per `block` values: the E4M3 scale by search, codes by nearest-grid
+    search, the dequantized value e2m1 * e4m3 * g as an exact rational."""
+    rows, k = xf32.shape
+    f = np.float32
+    d = f(f(6.0) * g)
+    codes = np.zeros((rows, k), np.uint8)
+    scales = np.zeros((rows, k // block), np.uint8)
+    deq = np.zeros((rows, k), object)
+    for r in range(rows):
+        for c in range(k // block):
+            blk = xf32[r, block * c:block * c + block]
+            ab = f(np.max(np.abs(blk)))
+            sfc = brute_e4m3(f(ab / d)) if d > 0 else 0
+            scales[r, c] = sfc
+            s = f(f(_E4M3_ALL[sfc]) * g)
+            for i in range(block):
+                code = brute_e2m1(f(blk[i] / s)) if s != 0 else 0
+                codes[r, block * c + i] = code
+                mag = Fraction(E2M1_GRID[code & 7]) * Fraction(float(_E4M3_ALL[sfc])) * Fraction(float(g))
+                deq[r, block * c + i] = -mag if code & 8 else mag
+    return codes, scales, deq
+
+
+def test_quantize_block_16_is_quantize_and_larger_blocks_vs_brute_force():
+    xb = synth.random_bf16((130, 256), seed=40, dist="outlier")
+    c16, s16, g16 = oracle.quantize_block(xb, 16)
+    c, s, g = oracle.quantize(xb)
+    assert g16 == g and np.array_equal(c16, c) and np.array_equal(s16, s)
+    rng = np.random.default_rng(41)
+    x = (rng.standard_normal((3, 128)) * np.exp2(rng.uniform(-6, 6, (3, 1)))).astype(np.float32)
+    xt = torch.from_numpy(x).to(torch.bfloat16)
+    xf = xt.float().numpy()
+    for block in (32, 64):
+        codes, sf, g = oracle.quantize_block(xt, block)
+        bc, bs, _ = brute_block_quantize(xf, block, np.float32(g))
+        assert np.array_equal(oracle.unpack_codes(codes), bc)
+        # each block scale repeated in its block/16 slots of the block-16 layout
+        assert np.array_equal(oracle.sf_matrix(sf, 3, 128), np.repeat(bs, block // 16, axis=1))
+
+
+def test_block_size_errors_vs_brute_force_and_dequantized_quantization():
+    rng = np.random.default_rng(42)
+    x = (rng.standard_normal((2, 64)) * np.exp2(rng.uniform(-4, 4, (2, 64)))).astype(np.float32)
+    xt = torch.from_numpy(x).to(torch.bfloat16)
+    xf = xt.float().numpy()
+    g = oracle.tensor_scale(xt)
+    err, ss = oracle.block_size_errors(xt, g)
+    assert ss == pytest.approx(float(np.sum(xf.astype(np.float64) ** 2)), rel=1e-15)
+    for i, b in enumerate(oracle.BLOCK_SIZES):
+        _, _, deq = brute_block_quantize(xf, b, np.float32(g))
+        exact = sum((Fraction(float(v)) - q) ** 2 for v, q in zip(xf.ravel(), deq.ravel()))
+        assert err[i] == pytest.approx(float(exact), rel=1e-12), b
+    # on a larger tensor: blocks 16 / 32 / 64 match the dequantized block quantization
+    xb = synth.random_bf16((64, 512), seed=43, dist="student_t3")
+    g = oracle.tensor_scale(xb)
+    err, _ = oracle.block_size_errors(xb, g)
+    xd = xb.float().numpy().astype(np.float64)
+    for i, b in ((4, 16), (5, 32), (6, 64)):
+        c, s, gg = oracle.quantize_block(xb, b, float(g))
+        assert err[i] == pytest.approx(float(np.sum((xd - oracle.dequantize(c, s, gg)) ** 2)), rel=1e-12)
+
+
+def test_select_block_size_limits():
+    xb = synth.random_bf16((64, 256), seed=44, dist="student_t3")
+    err, ss = oracle.block_size_errors(xb, oracle.tensor_scale(xb))
+    rel = err / ss
+    assert oracle.select_block_size(err, ss, 0.0) == oracle.BLOCK_SIZES[int(np.argmin(rel))]
+    assert oracle.select_block_size(err, ss, 1e6) == 64
+    # hand case: only 8 and 16 differ and memory decides at lambda = 1
+    e = np.array([1.0, 1.0, 1.0, 0.10, 0.10, 1.0, 1.0]) * 100.0
+    assert oracle.select_block_size(e, 100.0, 0.0) == 8                 # first minimum
+    assert oracle.select_block_size(e, 100.0, 1.0) == 16                # 4 + 8/16 < 4 + 8/8
+    # Memory is normalised by Memory(1) = 12 bits: errors 0.10 (b = 8) and 0.15
+    # (b = 16) against memory terms lambda * 5/12 and lambda * 4.5/12
+    e = np.array([1.0, 1.0, 1.0, 0.10, 0.15, 1.0, 1.0]) * 100.0
+    assert oracle.select_block_size(e, 100.0, 1.0) == 8                 # 0.5167 < 0.525
+    assert oracle.select_block_size(e, 100.0, 2.0) == 16                # 0.9333 > 0.9
