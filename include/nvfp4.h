@@ -142,6 +142,39 @@ nvfp4_status nvfp4_quantize_noalloc(const void *x_bf16, int64_t rows, int64_t k,
                                     unsigned flags, int *dev_status, nvfp4_stream_t stream);
 
 /*
+ * Block size per layer ([DiT] Algorithmic framework, Algorithm 1 / Eq. 9:
+ *   BlockSize(l) = argmin_{b in {1,2,4,8,16,32,64}} Error(l,b) + lambda Memory(b)/Memory_max).
+ *
+ * nvfp4_quantize_block -- nvfp4_quantize with `block` (16, 32 or 64) values per
+ * E4M3 scale: the block maximum is taken over `block` values along k and the
+ * scale byte is repeated in each of its block/16 slots of the block-16
+ * scale layout, so nvfp4_gemm_w4a4 multiplies the result unchanged.  Other
+ * arguments as nvfp4_quantize (block 16 is nvfp4_quantize itself).
+ *
+ * nvfp4_block_size_errors -- one pass over x computing Error(l, b) before
+ * normalisation for every candidate: errors[i] = sum_j (x_j - Q_b(x)_j)^2 for
+ * b = 2^i (i = 0..6), Q_b the two-level quantization with the block maximum
+ * over b values and tensor scale *tensor_scale (device float, e.g. from
+ * nvfp4_quantize), in double (element differences rounded once in FP32);
+ * errors[7] = sum_j x_j^2.  errors: 8 device doubles, overwritten.
+ * x as nvfp4_quantize (k % 64 == 0).  One kernel (after a memset of errors).
+ *
+ * nvfp4_select_block_size -- host function, Eq. 9 on HOST errors[8] (as
+ * above, copied back): Error(b) = errors[i] / errors[7], Memory(b) = 4 + 8/b
+ * bits per value (E2M1 plus one 8-bit scale per block; the tensor scale is
+ * shared by the whole tensor and left out), Memory_max = Memory(1) = 12.
+ * Returns the b of the first minimum, or 0 for a null pointer or a negative
+ * or NaN lambda.  The pages give no value for lambda.
+ */
+nvfp4_status nvfp4_quantize_block(const void *x_bf16, int64_t rows, int64_t k, int64_t ld_x, int block,
+                                  uint8_t *codes, uint8_t *sf, float *tensor_scale, unsigned flags,
+                                  void *workspace, size_t workspace_bytes, int *dev_status,
+                                  nvfp4_stream_t stream);
+nvfp4_status nvfp4_block_size_errors(const void *x_bf16, int64_t rows, int64_t k, int64_t ld_x,
+                                     const float *tensor_scale, double *errors, nvfp4_stream_t stream);
+int nvfp4_select_block_size(const double *errors, double lambda);
+
+/*
  * nvfp4_dequantize -- v = (e2m1(code) * e4m3(sf)) * g, rounded once (RNE) to
  * out_dtype ([DiT] Definition III.1: the quantizer returns s * round(...)).
  * codes/sf/tensor_scale as produced by nvfp4_quantize for [rows, k];

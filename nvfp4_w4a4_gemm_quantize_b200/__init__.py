@@ -7,13 +7,14 @@ memory and streams.
 
 Low-level (same names and argument order as the C calls):
     nvfp4_sf_bytes, nvfp4_quantize_workspace_bytes, nvfp4_quantize,
-    nvfp4_quantize_noalloc, nvfp4_dequantize, nvfp4_fake_quantize, nvfp4_ste_backward,
+    nvfp4_quantize_noalloc, nvfp4_quantize_block, nvfp4_block_size_errors, nvfp4_select_block_size,
+    nvfp4_dequantize, nvfp4_fake_quantize, nvfp4_ste_backward,
     nvfp4_gemm_w4a4, nvfp4_gemm_w4a4_grouped, nvfp4_gemm_w4a16, nvfp4_mx_sf_bytes, nvfp4_mx_quantize,
     nvfp4_mx_dequantize, nvfp4_mx_gemm, nvfp4_launch_count
 Convenience (allocate outputs with torch, then call the above):
     NVFP4Tensor, quantize, dequantize, gemm_w4a4, gemm_w4a4_grouped, gemm_w4a16,
     fake_quantize, ste_backward, FakeQuantizeSTE (autograd: the two kernels),
-    MXTensor, mx_quantize, mx_dequantize, mx_gemm
+    MXTensor, mx_quantize, mx_dequantize, mx_gemm, quantize_block, block_size_errors, select_block_size
 """
 from __future__ import annotations
 
@@ -91,6 +92,24 @@ def nvfp4_quantize_noalloc(x, rows, k, ld_x, codes, sf, tensor_scale, flags=0, d
     st = lib().nvfp4_quantize_noalloc(_ptr(x), rows, k, ld_x, _ptr(codes), _ptr(sf), _ptr(tensor_scale), flags,
                                       _ptr(dev_status), _stream(stream))
     check(st, "nvfp4_quantize_noalloc")
+
+
+def nvfp4_quantize_block(x, rows, k, ld_x, block, codes, sf, tensor_scale, flags=0, workspace=None,
+                         workspace_bytes=0, dev_status=None, stream=None) -> None:
+    st = lib().nvfp4_quantize_block(_ptr(x), rows, k, ld_x, block, _ptr(codes), _ptr(sf), _ptr(tensor_scale), flags,
+                                    _ptr(workspace), workspace_bytes, _ptr(dev_status), _stream(stream))
+    check(st, "nvfp4_quantize_block")
+
+
+def nvfp4_block_size_errors(x, rows, k, ld_x, tensor_scale, errors, stream=None) -> None:
+    check(lib().nvfp4_block_size_errors(_ptr(x), rows, k, ld_x, _ptr(tensor_scale), _ptr(errors), _stream(stream)),
+          "nvfp4_block_size_errors")
+
+
+def nvfp4_select_block_size(errors_host, lam: float) -> int:
+    """Eq. 9 on a host sequence of 8 doubles (the device errors copied back)."""
+    arr = (ctypes.c_double * 8)(*[float(v) for v in errors_host])
+    return int(lib().nvfp4_select_block_size(ctypes.addressof(arr), float(lam)))
 
 
 def nvfp4_dequantize(codes, sf, tensor_scale, rows, k, out, out_dtype, stream=None) -> None:
@@ -343,3 +362,43 @@ def mx_gemm(a: MXTensor, b: MXTensor, out_dtype=torch.bfloat16, out: torch.Tenso
     y = out if out is not None else torch.empty(a.rows, b.rows, dtype=out_dtype, device=a.codes.device)
     nvfp4_mx_gemm(a.codes, a.sf, b.codes, b.sf, a.rows, b.rows, a.k, y, _DT[y.dtype], act, dev_status, stream)
     return y
+
+
+# ----------------------------------------------------------------- block size (Algorithm 1 / Eq. 9)
+def quantize_block(x: torch.Tensor, block: int, scale: torch.Tensor | float | None = None,
+                   out: NVFP4Tensor | None = None, workspace: torch.Tensor | None = None, dev_status=None,
+                   stream=None) -> NVFP4Tensor:
+    """quantize() with `block` (16, 32, 64) values per scale; scales repeated in
+    the block-16 layout, so gemm_w4a4 takes the result as it is."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, k = x.shape
+    q = out if out is not None else NVFP4Tensor.empty(rows, k, x.device)
+    flags = 0
+    if scale is not None:
+        if isinstance(scale, torch.Tensor):
+            q.scale.copy_(scale.reshape(1).to(torch.float32))
+        else:
+            q.scale.fill_(float(scale))
+        flags = NVFP4_SCALE_GIVEN
+    wsb = nvfp4_quantize_workspace_bytes(rows, k)
+    if flags == 0 and workspace is None:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=x.device)
+    nvfp4_quantize_block(x, rows, k, x.stride(0), block, q.codes, q.sf, q.scale, flags,
+                         workspace if flags == 0 else None, wsb if flags == 0 else 0, dev_status, stream)
+    return q
+
+
+def block_size_errors(x: torch.Tensor, tensor_scale: torch.Tensor, stream=None) -> torch.Tensor:
+    """Device float64 [8]: squared errors for b = 1, 2, ..., 64 and sum x^2."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    errors = torch.empty(8, dtype=torch.float64, device=x.device)
+    nvfp4_block_size_errors(x, x.shape[0], x.shape[1], x.stride(0), tensor_scale, errors, stream)
+    return errors
+
+
+def select_block_size(x: torch.Tensor, lam: float, tensor_scale: torch.Tensor | None = None) -> int:
+    """Algorithm 1 / Eq. 9 for one tensor: errors on the device, the argmin on
+    the host (one 64-byte copy)."""
+    if tensor_scale is None:
+        tensor_scale = quantize(x).scale
+    return nvfp4_select_block_size(block_size_errors(x, tensor_scale).cpu().tolist(), lam)

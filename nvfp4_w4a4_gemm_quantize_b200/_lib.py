@@ -43,6 +43,10 @@ SIGNATURES = {
     "nvfp4_quantize": (_status, [_p, _i64, _i64, _i64, _p, _p, _p, ctypes.c_uint, _p, ctypes.c_size_t, _p, _p]),
     "nvfp4_quantize_noalloc": (_status, [_p, _i64, _i64, _i64, _p, _p, _p, ctypes.c_uint, _p, _p]),
     "nvfp4_dequantize": (_status, [_p, _p, _p, _i64, _i64, _p, _int, _p]),
+    "nvfp4_quantize_block": (_status, [_p, _i64, _i64, _i64, _int, _p, _p, _p, ctypes.c_uint, _p, ctypes.c_size_t,
+                                       _p, _p]),
+    "nvfp4_block_size_errors": (_status, [_p, _i64, _i64, _i64, _p, _p, _p]),
+    "nvfp4_select_block_size": (_int, [_p, ctypes.c_double]),
     "nvfp4_fake_quantize": (_status, [_p, _i64, _i64, _i64, _p, _int, _p, _p, ctypes.c_uint, _p, ctypes.c_size_t,
                                       _p, _p]),
     "nvfp4_ste_backward": (_status, [_p, _p, _i64, _i64, _int, _p, _p]),

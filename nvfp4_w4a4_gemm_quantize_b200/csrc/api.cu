@@ -133,6 +133,70 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t
                                        dev_status, s));
 }
 
+nvfp4_status nvfp4_quantize_block(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, int block,
+                                  uint8_t* codes, uint8_t* sf, float* tensor_scale, unsigned flags, void* workspace,
+                                  size_t workspace_bytes, int* dev_status, nvfp4_stream_t stream) {
+    if (block != 16 && block != 32 && block != 64) return NVFP4_ERR_INVALID_ARG;
+    if (block == 16)
+        return nvfp4_quantize(x_bf16, rows, k, ld_x, codes, sf, tensor_scale, flags, workspace, workspace_bytes,
+                              dev_status, stream);
+    if (rows < 0 || k <= 0 || ld_x < k) return NVFP4_ERR_INVALID_ARG;
+    if ((flags & ~(unsigned)NVFP4_SCALE_GIVEN) != 0u) return NVFP4_ERR_INVALID_ARG;
+    if (!tensor_scale) return NVFP4_ERR_INVALID_ARG;
+    if (rows > 0 && (!x_bf16 || !codes || !sf)) return NVFP4_ERR_INVALID_ARG;
+    if (k % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (rows > (int64_t)1 << 31 || k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    const bool given = (flags & NVFP4_SCALE_GIVEN) != 0u;
+    if (!given && (!workspace || workspace_bytes < kQuantWorkspaceBytes)) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(sf) || (ld_x % 8) != 0 ||
+        (!given && !aligned16(workspace)) || (reinterpret_cast<uintptr_t>(tensor_scale) & 3u))
+        return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    nvfp4_status st = device_ok(&sms);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (rows == 0) {
+        if (!given) return cuda_status(cudaMemsetAsync(tensor_scale, 0, sizeof(float), s));
+        return NVFP4_OK;
+    }
+    return cuda_status(launch_quantize_block(static_cast<const uint16_t*>(x_bf16), rows, k, ld_x, block, codes, sf,
+                                             tensor_scale, given, workspace, dev_status, sms, s));
+}
+
+nvfp4_status nvfp4_block_size_errors(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x,
+                                     const float* tensor_scale, double* errors, nvfp4_stream_t stream) {
+    if (rows < 0 || k <= 0 || ld_x < k) return NVFP4_ERR_INVALID_ARG;
+    if (!tensor_scale || !errors || (rows > 0 && !x_bf16)) return NVFP4_ERR_INVALID_ARG;
+    if (k % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (rows > (int64_t)1 << 31 || k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x_bf16) || (ld_x % 8) != 0 || (reinterpret_cast<uintptr_t>(errors) & 7u) ||
+        (reinterpret_cast<uintptr_t>(tensor_scale) & 3u))
+        return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    nvfp4_status st = device_ok(&sms);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (rows == 0) return cuda_status(cudaMemsetAsync(errors, 0, 8 * sizeof(double), s));
+    return cuda_status(launch_block_size_errors(static_cast<const uint16_t*>(x_bf16), rows, k, ld_x, tensor_scale,
+                                                errors, sms, s));
+}
+
+int nvfp4_select_block_size(const double* errors, double lambda) {
+    if (!errors || !(lambda >= 0.0)) return 0;
+    int best = 1;
+    double bestv = 0.0;
+    for (int i = 0; i < 7; ++i) {
+        const int b = 1 << i;
+        const double e = errors[7] > 0.0 ? errors[i] / errors[7] : 0.0;
+        const double v = e + lambda * (4.0 + 8.0 / b) / 12.0;
+        if (i == 0 || v < bestv) {
+            bestv = v;
+            best = b;
+        }
+    }
+    return best;
+}
+
 nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* sf, const float* tensor_scale, int64_t rows,
                               int64_t k, void* out, int out_dtype, nvfp4_stream_t stream) {
     if (rows < 0 || k <= 0) return NVFP4_ERR_INVALID_ARG;

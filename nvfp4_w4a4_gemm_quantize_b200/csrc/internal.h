@@ -25,6 +25,13 @@ cudaError_t launch_quantize_fused(const uint16_t* x, int64_t rows, int64_t k, in
                                   uint8_t* sf, float* tensor_scale, unsigned long long* slots, int max_slots,
                                   int* dev_status, int num_sms, cudaStream_t stream);
 
+cudaError_t launch_quantize_block(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, int block, uint8_t* codes,
+                                  uint8_t* sf, float* tensor_scale, bool scale_given, void* workspace,
+                                  int* dev_status, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_block_size_errors(const uint16_t* x, int64_t rows, int64_t k, int64_t ld,
+                                     const float* tensor_scale, double* errors, int num_sms, cudaStream_t stream);
+
 cudaError_t launch_fake_quantize(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, void* y, bool y_f32,
                                  uint8_t* mask, float* tensor_scale, bool scale_given, void* workspace,
                                  int* dev_status, int num_sms, cudaStream_t stream);

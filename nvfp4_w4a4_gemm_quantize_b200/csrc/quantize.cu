@@ -180,6 +180,7 @@ struct CodesOut {
     uint8_t* sf;
     static constexpr bool kScales = true;
     static constexpr int kMinBlocks = 0;          // unforced: the compiler fits 64 registers (2 CTAs per SM)
+    static constexpr int kGroup = 1;              // lanes (16-value blocks) per scale block
     struct Lane {
         uint2* cp;
         int64_t step;
@@ -195,6 +196,15 @@ struct CodesOut {
                                                  int64_t cblk) const {
         store_tile_scales(sf_stage, sf, k, rblk, cblk);
     }
+};
+
+// Codes and scales with one scale per G consecutive 16-value blocks (blocks
+// of 32 or 64 values along k): the G lanes of a scale block share its
+// maximum, and each writes the shared scale byte into its own 16-block slot,
+// so the block-16 GEMM reads the result unchanged.
+template <int G>
+struct CodesOutG : CodesOut {
+    static constexpr int kGroup = G;
 };
 
 // f16x2 of two E2M1 codes (one byte, the low nibble in the low half) times
@@ -334,6 +344,7 @@ struct FakeOut {
     uint8_t* mask;                                // nullable
     static constexpr bool kScales = false;
     static constexpr int kMinBlocks = 2;          // 64 registers: 2 CTAs (32 warps) per SM
+    static constexpr int kGroup = 1;
     struct Lane {
         uint4* yp;
         uint16_t* mp;
@@ -406,7 +417,9 @@ __device__ __forceinline__ void quantize_lane(const TileLane& t, const uint4 (&v
     for (int i = 0; i < kSteps; ++i) {
         const uint32_t w[8] = {v[2 * i].x, v[2 * i].y, v[2 * i].z, v[2 * i].w,
                                v[2 * i + 1].x, v[2 * i + 1].y, v[2 * i + 1].z, v[2 * i + 1].w};
-        const float ab = __uint_as_float(block_absmax16(w) << 16);      // block amax
+        float ab = __uint_as_float(block_absmax16(w) << 16);            // block amax
+        if (Out::kGroup >= 2) ab = fmaxf(ab, __shfl_xor_sync(0xffffffffu, ab, 1));   // lanes of one row:
+        if (Out::kGroup >= 4) ab = fmaxf(ab, __shfl_xor_sync(0xffffffffu, ab, 2));   // consecutive blocks
         const uint32_t sfc = block_scale_code(ab, sc);
         const float s = __fmul_rn(e4m3_to_f32(sfc), sc.g);
         const uint32_t lo = quantize8_bf16(w[0], w[1], w[2], w[3], s);
@@ -702,6 +715,12 @@ static cudaError_t launch_two_kernel(const uint16_t* x, int64_t rows, int64_t k,
     return cudaGetLastError();
 }
 
+// Per-call numbers tagging the one-kernel form's workspace slots: one counter
+// for every output type, so that no two calls in the process share a number
+// (a workspace used by one output type and then another must not hold a
+// slot that carries the new call's number).
+static std::atomic<uint32_t> g_generation{0};
+
 // One-kernel form with a data-derived scale (see quantize_fused_kernel).
 // Returns cudaErrorNotSupported when the grid cannot be co-resident (the
 // caller then takes the two-kernel form, which computes the same result).
@@ -709,7 +728,7 @@ template <class Out>
 static cudaError_t launch_one_kernel(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, const Out& out,
                                      float* tensor_scale, unsigned long long* slots, int max_slots, int* dev_status,
                                      int num_sms, cudaStream_t stream) {
-    static std::atomic<uint32_t> generation{0};
+    std::atomic<uint32_t>& generation = g_generation;
     const int ntiles_c = (int)((k + kTileCols - 1) / kTileCols);
     const int64_t ntiles64 = ((rows + kTileRows - 1) / kTileRows) * ntiles_c;
     if (ntiles64 > (int64_t)1 << 30) return cudaErrorNotSupported;
@@ -757,6 +776,27 @@ cudaError_t launch_quantize_fused(const uint16_t* x, int64_t rows, int64_t k, in
                                   int* dev_status, int num_sms, cudaStream_t stream) {
     return launch_one_kernel(x, rows, k, ld, CodesOut{codes, sf}, tensor_scale, slots, max_slots, dev_status,
                              num_sms, stream);
+}
+
+// Quantization with 32 or 64 values per scale (scales repeated in the block-16
+// layout): one kernel with a data-derived scale when the grid can be
+// co-resident, else two; one kernel with a given scale.
+cudaError_t launch_quantize_block(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, int block, uint8_t* codes,
+                                  uint8_t* sf, float* tensor_scale, bool scale_given, void* workspace,
+                                  int* dev_status, int num_sms, cudaStream_t stream) {
+    auto run = [&](auto out) -> cudaError_t {
+        if (!scale_given) {
+            const cudaError_t e = launch_one_kernel(x, rows, k, ld, out, tensor_scale,
+                                                    static_cast<unsigned long long*>(workspace), kFusedSlots,
+                                                    dev_status, num_sms, stream);
+            if (e != cudaErrorNotSupported) return e;
+        }
+        return launch_two_kernel(x, rows, k, ld, out, tensor_scale, scale_given, static_cast<float*>(workspace),
+                                 dev_status, stream);
+    };
+    if (block == 32) return run(CodesOutG<2>{{codes, sf}});
+    if (block == 64) return run(CodesOutG<4>{{codes, sf}});
+    return run(CodesOut{codes, sf});
 }
 
 // Fake quantization: one kernel with a data-derived scale when the grid can

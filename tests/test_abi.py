@@ -32,7 +32,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 18, names
+    assert len(names) == 21, names
     for n in names:
         assert hasattr(L, n), n
         assert n in _lib.SIGNATURES, n
@@ -204,6 +204,24 @@ def test_mx_calls_reject_bad_arguments(L):
     assert g(A, B, A, B, 128, 256, 256, C, 0, 3, None, None) == INVALID
     assert g(A, B + 4, A, B, 128, 256, 256, C, 0, 0, None, None) == MISALIGNED
     assert g(A, B, A, B, -2, 256, 256, C, 0, 0, None, None) == INVALID
+
+
+def test_block_size_calls(L):
+    qb = L.nvfp4_quantize_block
+    assert qb(A, 128, 256, 256, 48, B, C, A, 1, None, 0, None, None) == INVALID     # block not 16/32/64
+    assert qb(A, 128, 96, 96, 32, B, C, A, 1, None, 0, None, None) == SHAPE
+    assert qb(A, 128, 256, 256, 64, B, C, A, 0, None, 0, None, None) == WORKSPACE
+    assert qb(A + 2, 128, 256, 256, 32, B, C, A, 1, None, 0, None, None) == MISALIGNED
+    e = L.nvfp4_block_size_errors
+    assert e(A, 128, 96, 96, B, C, None) == SHAPE
+    assert e(A, 128, 256, 256, None, C, None) == INVALID
+    assert e(A, 128, 256, 256, B, C + 4, None) == MISALIGNED
+    sel = L.nvfp4_select_block_size
+    err = (ctypes.c_double * 8)(1.0, 1.0, 1.0, 0.10, 0.15, 1.0, 1.0, 1.0)
+    assert sel(ctypes.addressof(err), 0.0) == 8
+    assert sel(ctypes.addressof(err), 2.0) == 16
+    assert sel(ctypes.addressof(err), 1e6) == 64
+    assert sel(None, 1.0) == 0 and sel(ctypes.addressof(err), -1.0) == 0
 
 
 def test_w4a16_rejects_bad_arguments(L):
