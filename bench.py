@@ -36,6 +36,8 @@ QUANT_BYTES_PER_ELEM = 4.5625
 QAT_FWD_DYNAMIC_BYTES = 6.125
 QAT_FWD_GIVEN_BYTES = 4.125
 QAT_BWD_BYTES = 4.125
+# MX quantize: 2 (read) + 0.5 (codes) + 1/32 (E8M0 scales), no amax pass
+MX_QUANT_BYTES_PER_ELEM = 2.53125
 
 
 def load_peaks():
@@ -236,6 +238,7 @@ def reference_points(dev, layers, w4a16_layers):
     out["qat"] = qat_points(dev, layers)
     out["mlp_fc1_gelu"] = mlp_fusion_points(dev, layers)
     out["grouped"] = grouped_points(dev)
+    out["mx_and_block_size"] = mx_points(dev, layers)
     torch.cuda.empty_cache()
     return out
 
@@ -347,6 +350,52 @@ def grouped_points(dev):
     return {"problems": "pixart1024 qkv 8192x1152x3456 + xattn_k/v 600x4096x1152",
             "separate_us": round(sep * 1e3, 1), "grouped_us": round(grp * 1e3, 1),
             "grouped_tflops": round(fl / (grp * 1e-3) / 1e12, 1)}
+
+
+def mx_points(dev, layers):
+    """The MX variant (block 32, E8M0 scales) on the fc2 input and the fc1 /
+    fc2 products, next to NVFP4; and the Eq. 9 block-size measurement on the
+    fc2 input (the relative squared error of every candidate block size)."""
+    import torch
+    import nvfp4_w4a4_gemm_quantize_b200 as nv
+    from nvfp4_w4a4_gemm_quantize_b200 import synth
+    hbm = load_peaks()[0].get("hbm_gbs", FALLBACK["hbm_gbs"])
+    res = {}
+    names = [L.name for L in layers]
+    if "fc2" in names:
+        L = layers[names.index("fc2")]
+        x, = synth.layer_tensors(WORKLOAD, "fc2", device=dev, want=("x",))
+        x = x[: L.M].contiguous()
+        n = x.numel()
+        mq = nv.MXTensor.empty(*x.shape, dev)
+        ms = time_device(lambda: nv.mx_quantize(x, out=mq))
+        gbs = MX_QUANT_BYTES_PER_ELEM * n / (ms * 1e-3) / 1e9
+        res["mx_quantize_fc2"] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / hbm, 4),
+                                  "bytes_per_elem": MX_QUANT_BYTES_PER_ELEM}
+        g = nv.quantize(x).scale
+        e = torch.empty(8, dtype=torch.float64, device=dev)
+        ms = time_device(lambda: nv.nvfp4_block_size_errors(x, x.shape[0], x.shape[1], x.shape[1], g, e), iters=3,
+                         warmup=1)
+        rel = (e[:7] / e[7]).cpu().tolist()
+        res["block_size_errors_fc2"] = {"ms": round(ms, 3),
+                                        "relative_sq_error": {str(b): round(v, 6) for b, v in zip((1, 2, 4, 8, 16, 32, 64), rel)},
+                                        "selected": {str(lam): nv.nvfp4_select_block_size(e.cpu().tolist(), lam)
+                                                     for lam in (0.001, 0.01, 0.1)}}
+        del x, mq, e
+    for name in ("fc1", "fc2"):
+        if name not in names:
+            continue
+        L = layers[names.index(name)]
+        x, w = synth.layer_tensors(WORKLOAD, name, device=dev)
+        x = x[: L.M].contiguous()
+        A, W = nv.mx_quantize(x), nv.mx_quantize(w)
+        y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev)
+        ms = time_device(lambda: nv.mx_gemm(A, W, out=y))
+        res[f"mx_gemm_{name}"] = {"shape": f"{L.M}x{L.K}x{L.N}", "ms": round(ms, 4),
+                                  "tflops": round(2 * L.M * L.N * L.K / (ms * 1e-3) / 1e12, 1)}
+        del x, w, A, W, y
+    torch.cuda.empty_cache()
+    return res
 
 
 def reduced(wl, args):
