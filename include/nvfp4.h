@@ -311,7 +311,7 @@ nvfp4_status nvfp4_gemm_w4a16(const void *x_bf16, const uint8_t *w_codes, const 
                               void *y, int y_dtype, int *dev_status, nvfp4_stream_t stream);
 
 /*
- * MX variant ([RFC] Related: the MXFP4 format, "related but different"):
+ * MX variant (the [RFC] lists MXFP4 among related issues, as another format):
  * E2M1 elements in blocks of 32 along k, one power-of-two scale per block as
  * an unsigned E8M0 byte (value 2^(byte - 127)), no tensor scale.  The pages
  * give no scale rule; the OCP Microscaling one is used:
