@@ -33,6 +33,9 @@ Parity status per function:
   quantize_block / block_size_errors / select_block_size -- pinned (block 16
       equals quantize, brute force for blocks 32 and 64, errors against the
       dequantized oracle quantization and brute force, Eq. 9 limits)
+  attention                                             -- pinned (float64
+      library attention of the dequantized operands, rows of p summing to
+      one, invariance under the per-head term, a one-hot case)
   gelu_tanh                                             -- pinned (torch's
       float64 tanh-form GELU, the odd-part identity g(v) - g(-v) = v, the erf
       form within 1e-3, limits)
@@ -110,6 +113,9 @@ def lib() -> ctypes.CDLL:
         L.oracle_block_size_errors.restype = None
         L.oracle_select_block_size.argtypes = [_p, ctypes.c_double, ctypes.c_double]
         L.oracle_select_block_size.restype = ctypes.c_int
+        L.oracle_attention_rows.argtypes = [_p, _p, _f32, _p, _p, _f32, _p, _p, _f32, _i64, _i64, _i64, _p, _i64,
+                                            _i64, _i64, _p]
+        L.oracle_attention_rows.restype = None
         L.oracle_gelu_tanh.argtypes = [ctypes.c_double]
         L.oracle_gelu_tanh.restype = ctypes.c_double
         L.oracle_gelu_tanh_array.argtypes = [_p, _i64, _p]
@@ -431,3 +437,19 @@ def select_block_size(err, sumsq: float, lam: float) -> int:
     """Eq. 9: argmin_b Error(b) / sum x^2 + lambda (4 + 8/b) / 12."""
     e = np.ascontiguousarray(err, np.float64)
     return int(lib().oracle_select_block_size(_ptr(e), float(sumsq), float(lam)))
+
+
+# ---------------------------------------------------------------- attention
+def attention(q, k, v, s_head, H: int, Lq: int, Lk: int, d: int, h: int, rows: slice | None = None) -> np.ndarray:
+    """O of head h (Eq. 10 over NVFP4 Q, K, V; q/k/v = (codes, sf, g) of
+    [H*Lq, d] / [H*Lk, d] tensors), query rows `rows` (all by default), in
+    double."""
+    L = lib()
+    (qc, qs, gq), (kc, ks, gk), (vc, vs, gv) = q, k, v
+    qc, qs, kc, ks, vc, vs = (np.ascontiguousarray(a, np.uint8) for a in (qc, qs, kc, ks, vc, vs))
+    sh = np.ascontiguousarray(s_head, np.float64)
+    q0, q1 = (0, Lq) if rows is None else (rows.start or 0, rows.stop)
+    out = np.empty((q1 - q0, d), np.float64)
+    L.oracle_attention_rows(_ptr(qc), _ptr(qs), float(gq), _ptr(kc), _ptr(ks), float(gk), _ptr(vc), _ptr(vs),
+                            float(gv), Lq, Lk, d, _ptr(sh), h, q0, q1 - q0, _ptr(out))
+    return out

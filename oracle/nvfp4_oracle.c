@@ -636,3 +636,53 @@ int oracle_select_block_size(const double *err, double sumsq, double lambda)
     }
     return best;
 }
+
+/* ------------------------ attention over NVFP4 K / V ---------------------- */
+/* Attention of one head over NVFP4 operands [DiT, Algorithmic framework,
+ * Eq. 10: Attention(Q, K, V) = softmax(Q K^T / sqrt(d_k) + log(s_head)) V, with
+ * a learnable per-head scale s_head; Systems optimization: FP4-packed
+ * attention].  Q [H*Lq, d], K and V [H*Lk, d] are NVFP4 tensors quantized
+ * along d (blocks of 16, tensor scales g_q, g_k, g_v); head h owns rows
+ * h*Lq .. and h*Lk .. .  In double, from the exact element values:
+ *   z[i][j] = (q^_i . k^_j) / sqrt(d) + log(s_head[h])
+ *   p[i][j] = exp(z[i][j] - max_j z[i][j]) / sum_j exp(...)
+ *   O[i]    = sum_j p[i][j] v^_j
+ * for query rows q0 .. q0+nq-1 of head h; out holds nq * d doubles.          */
+void oracle_attention_rows(const uint8_t *q_codes, const uint8_t *q_sf, float g_q,
+                           const uint8_t *k_codes, const uint8_t *k_sf, float g_k,
+                           const uint8_t *v_codes, const uint8_t *v_sf, float g_v,
+                           int64_t Lq, int64_t Lk, int64_t d, const double *s_head, int64_t h,
+                           int64_t q0, int64_t nq, double *out)
+{
+    double *kh = (double *)malloc((size_t)(Lk * d) * sizeof(double));
+    double *vh = (double *)malloc((size_t)(Lk * d) * sizeof(double));
+    double *z = (double *)malloc((size_t)Lk * sizeof(double));
+    double *qi = (double *)malloc((size_t)d * sizeof(double));
+    if (!kh || !vh || !z || !qi) { free(kh); free(vh); free(z); free(qi); return; }
+    for (int64_t j = 0; j < Lk; ++j)
+        for (int64_t c = 0; c < d; ++c) {
+            kh[j * d + c] = deq_elem(k_codes, k_sf, h * Lk + j, c, d) * (double)g_k;
+            vh[j * d + c] = deq_elem(v_codes, v_sf, h * Lk + j, c, d) * (double)g_v;
+        }
+    const double bias = log(s_head[h]);
+    const double inv_sqrt_d = 1.0 / sqrt((double)d);
+    for (int64_t t = 0; t < nq; ++t) {
+        const int64_t i = q0 + t;
+        for (int64_t c = 0; c < d; ++c) qi[c] = deq_elem(q_codes, q_sf, h * Lq + i, c, d) * (double)g_q;
+        double zmax = -INFINITY;
+        for (int64_t j = 0; j < Lk; ++j) {
+            double acc = 0.0;
+            for (int64_t c = 0; c < d; ++c) acc += qi[c] * kh[j * d + c];
+            z[j] = acc * inv_sqrt_d + bias;
+            if (z[j] > zmax) zmax = z[j];
+        }
+        double l = 0.0;
+        for (int64_t j = 0; j < Lk; ++j) { z[j] = exp(z[j] - zmax); l += z[j]; }
+        for (int64_t c = 0; c < d; ++c) {
+            double o = 0.0;
+            for (int64_t j = 0; j < Lk; ++j) o += z[j] * vh[j * d + c];
+            out[t * d + c] = o / l;
+        }
+    }
+    free(kh); free(vh); free(z); free(qi);
+}

@@ -757,3 +757,53 @@ def test_select_block_size_limits():
     e = np.array([1.0, 1.0, 1.0, 0.10, 0.15, 1.0, 1.0]) * 100.0
     assert oracle.select_block_size(e, 100.0, 1.0) == 8                 # 0.5167 < 0.525
     assert oracle.select_block_size(e, 100.0, 2.0) == 16                # 0.9333 > 0.9
+
+
+# ------------------------------------------------------------------ attention (Eq. 10)
+def _attn_operands(H, Lq, Lk, d, seed):
+    q = oracle.quantize(synth.random_bf16((H * Lq, d), seed=seed, dist="normal"))
+    k = oracle.quantize(synth.random_bf16((H * Lk, d), seed=seed + 1, dist="normal"))
+    v = oracle.quantize(synth.random_bf16((H * Lk, d), seed=seed + 2, dist="student_t3"))
+    return q, k, v
+
+
+def test_attention_vs_library_and_identities():
+    H, Lq, Lk, d = 2, 40, 96, 64
+    q, k, v = _attn_operands(H, Lq, Lk, d, 60)
+    s_head = np.array([1.0, 3.5])
+    qd = oracle.dequantize(*q).reshape(H, Lq, d)
+    kd = oracle.dequantize(*k).reshape(H, Lk, d)
+    vd = oracle.dequantize(*v).reshape(H, Lk, d)
+    ref = torch.nn.functional.scaled_dot_product_attention(torch.from_numpy(qd), torch.from_numpy(kd),
+                                                           torch.from_numpy(vd)).numpy()
+    for h in range(H):
+        o = oracle.attention(q, k, v, s_head, H, Lq, Lk, d, h)
+        assert np.allclose(o, ref[h], rtol=1e-12, atol=1e-12 * np.abs(vd).max())
+        # the per-head term is a constant shift of every logit of the head
+        o1 = oracle.attention(q, k, v, np.ones(H), H, Lq, Lk, d, h)
+        assert np.allclose(o, o1, rtol=1e-12, atol=1e-12 * np.abs(vd).max())
+        assert np.array_equal(oracle.attention(q, k, v, s_head, H, Lq, Lk, d, h, rows=slice(7, 11)), o[7:11])
+    # rows of p sum to one: with a constant V the output is that constant
+    ones = oracle.quantize(torch.ones(H * Lk, d, dtype=torch.bfloat16))
+    c = oracle.dequantize(*ones)[0, 0]
+    o = oracle.attention(q, k, ones, s_head, H, Lq, Lk, d, 1)
+    assert np.allclose(o, c, rtol=1e-14)
+
+
+def test_attention_one_hot_selects_the_matching_key():
+    """Q row i a large multiple of K row (3 i mod Lk) (logit 512 against 0):
+    the output is V of that key."""
+    H, Lq, Lk, d = 1, 16, 64, 64
+    eye = torch.zeros(Lk, d)
+    for j in range(Lk):
+        eye[j, j] = 1.0
+    kq = oracle.quantize(eye.bfloat16())
+    qx = torch.zeros(Lq, d)
+    for i in range(Lq):
+        qx[i, (3 * i) % Lk] = 4096.0
+    q = oracle.quantize(qx.bfloat16())
+    v = oracle.quantize(synth.random_bf16((Lk, d), seed=61, dist="normal"))
+    o = oracle.attention(q, kq, v, np.ones(1), H, Lq, Lk, d, 0)
+    vd = oracle.dequantize(*v)
+    for i in range(Lq):
+        assert np.allclose(o[i], vd[(3 * i) % Lk], rtol=1e-12, atol=1e-12)
