@@ -1,0 +1,446 @@
+// attn.cu -- attention over an NVFP4 key / value cache, one head per CTA row
+// of the grid ("NVFP4-DiT ..." README, Algorithmic framework, Eq. 10:
+// Attention(Q, K, V) = softmax(Q K^T / sqrt(d_k) + log(s_head)) V with a
+// per-head scale s_head; Systems optimization: FP4-packed attention).
+//
+// Q, K, V are NVFP4 tensors quantized along the head dimension d = 128
+// (blocks of 16, tensor scales g_q, g_k, g_v): Q [H*Lq, d], K and V [H*Lk, d].
+// Per CTA: 128 queries of one head, keys in tiles of 128.
+//   S = Q K^T     block-scaled FP4 MMA (kind::mxf4nvf4, K = d), FP32 in TMEM,
+//                 two S buffers so the next tile's product overlaps softmax;
+//   softmax       one query row per thread (online: running max m, sum l),
+//                 exp2 of (S * g_q g_k log2(e) / sqrt(d) + log2(s_head) - m),
+//                 P rounded to bf16 into a 128-byte-swizzled K-major tile, and
+//                 the running output rescaled in TMEM when m grows;
+//   V             dequantized exactly to bf16 (e2m1 * e4m3 has at most 6
+//                 significant bits) into a K-major V^T tile by four warps;
+//   O += P V      bf16 MMA (kind::f16), FP32 in TMEM;
+//   output        O * g_v / l, rounded to bf16.
+// Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 4-7
+// softmax and output, warps 8-11 V dequantization; every wait is bounded.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "quant_math.cuh"
+#include "tmap.h"
+
+namespace nvfp4 {
+
+namespace attn {
+
+constexpr int kD = 128;                      // head dimension
+constexpr int kBQ = 128;                     // queries per CTA
+constexpr int kBK = 128;                     // keys per tile
+constexpr int kThreads = 384;
+constexpr int kStages = 2;                   // K / V code stages
+constexpr int kCodeBytes = kBK * kD / 2;     // 8 KB: 128 rows x 64 bytes
+constexpr int kSfBytes = 1024;               // two 512-byte scale atoms (128 rows x 8 blocks)
+constexpr int kStageBytes = 2 * kCodeBytes + 2 * kSfBytes;
+constexpr int kTileBf16 = kBQ * kBK * 2;     // 32 KB: two 64-key chunks of 128 rows x 128 bytes
+constexpr int kChunk = 128 * 128;            // 16 KB
+
+// shared memory (offsets from a 1024-aligned base)
+constexpr int kOffQ = 0;
+constexpr int kOffQsf = kOffQ + kCodeBytes;
+constexpr int kOffStages = kOffQsf + kSfBytes;
+constexpr int kOffP = kOffStages + kStages * kStageBytes;          // 2 P tiles
+constexpr int kOffVt = kOffP + 2 * kTileBf16;                      // kStages V^T tiles
+constexpr int kSmemBytes = kOffVt + kStages * kTileBf16 + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+// TMEM columns
+constexpr uint32_t kColS = 0;                // two S buffers: [0,128), [128,256)
+constexpr uint32_t kColO = 256;              // O: [256, 384)
+constexpr uint32_t kColSfQ = 384;            // Q scales: 2 K-steps x 4 columns
+constexpr uint32_t kColSfK = 392;            // K scales per S buffer: 2 x (2 x 4)
+
+struct Params {
+    const uint8_t* q_sf;
+    const uint8_t* k_sf;
+    const uint8_t* v_sf;
+    const float* g_q;
+    const float* g_k;
+    const float* g_v;
+    const float* s_head;                     // nullable: 1 for every head
+    uint16_t* out;                           // bf16 [H*Lq, d]
+    int Lq, Lk, H;
+    int* dev_status;
+};
+
+// K-major operand rows of 64 bytes with the 64-byte swizzle (8-row groups
+// 512 bytes apart).
+__device__ __forceinline__ uint64_t sdesc_kmajor_sw64(uint32_t saddr) { return make_sdesc(saddr, 16, 512, 4); }
+
+__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+          "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+          "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// E2M1 code -> value (exact).
+__device__ __forceinline__ float e2m1_val(uint32_t c) {
+    const uint32_t e = (c >> 1) & 3u, m = c & 1u;
+    const float mag = e == 0u ? 0.5f * (float)m : __uint_as_float(((e + 126u) << 23) | (m << 22));
+    return (c & 8u) ? -mag : mag;
+}
+
+// Byte of (row r, 16-value block c) inside a 128-row group's two scale atoms.
+__device__ __forceinline__ int sf_byte(int r, int c) { return (c >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (c & 3); }
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+            const __grid_constant__ CUtensorMap tmap_v, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t q_full, kv_full[kStages], kv_empty[kStages], vt_full[kStages], vt_empty[kStages];
+    __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_done, drain;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    WaitCtx wc{&abort_sh, p.dev_status};
+    const int h = blockIdx.y;
+    const int qrow0 = h * p.Lq + blockIdx.x * kBQ;          // first query row of this CTA
+    const int krow0 = h * p.Lk;
+    const int ntiles = p.Lk / kBK;
+
+    if (threadIdx.x == 0) {
+        abort_sh = 0;
+        mbar_init(&q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1 + 4);          // the S product's commit + four dequantizer warps
+            mbar_init(&vt_full[s], 4);
+            mbar_init(&vt_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&s_full[b], 1);
+            mbar_init(&s_empty[b], 4);
+            mbar_init(&p_full[b], 4);
+            mbar_init(&p_empty[b], 1);
+        }
+        mbar_init(&o_done, 1);
+        mbar_init(&drain, 1);
+        fence_barrier_init();
+        tma_prefetch_desc(&tmap_q);
+        tma_prefetch_desc(&tmap_k);
+        tma_prefetch_desc(&tmap_v);
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_sh, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        const uint64_t pol = policy_evict_normal();
+        bool ok = true;
+        if (elect_one()) {
+            mbar_arrive_expect_tx(&q_full, kCodeBytes + kSfBytes);
+            tma_load_2d(smem + kOffQ, &tmap_q, &q_full, 0, qrow0, pol);
+            bulk_load(smem + kOffQsf, p.q_sf + (int64_t)(qrow0 >> 7) * kSfBytes, kSfBytes, &q_full, pol);
+        }
+        __syncwarp();
+        for (int j = 0; j < ntiles && ok; ++j) {
+            const int s = j % kStages;
+            const uint32_t ph = (uint32_t)(j / kStages) & 1u;
+            if (!__all_sync(0xffffffffu, mbar_wait(&kv_empty[s], ph ^ 1u, wc) ? 1 : 0)) { ok = false; break; }
+            uint8_t* st = smem + kOffStages + s * kStageBytes;
+            const int kr = krow0 + j * kBK;
+            if (elect_one()) {
+                mbar_arrive_expect_tx(&kv_full[s], kStageBytes);
+                tma_load_2d(st, &tmap_k, &kv_full[s], 0, kr, pol);
+                tma_load_2d(st + kCodeBytes, &tmap_v, &kv_full[s], 0, kr, pol);
+                bulk_load(st + 2 * kCodeBytes, p.k_sf + (int64_t)(kr >> 7) * kSfBytes, kSfBytes, &kv_full[s], pol);
+                bulk_load(st + 2 * kCodeBytes + kSfBytes, p.v_sf + (int64_t)(kr >> 7) * kSfBytes, kSfBytes,
+                          &kv_full[s], pol);
+            }
+            __syncwarp();
+        }
+        // every load this warp issued has landed before the CTA may exit
+        if (lane == 0) {
+            int dummy = 0;
+            WaitCtx w2{&dummy, p.dev_status};
+            mbar_wait(&q_full, 0, w2);
+            for (int j = (ntiles > kStages ? ntiles - kStages : 0); j < ntiles; ++j)
+                mbar_wait(&kv_full[j % kStages], (uint32_t)(j / kStages) & 1u, w2);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc_s = idesc_nvf4(kBQ, kBK);
+        constexpr uint32_t idesc_o = idesc_bf16(kBQ, kD);
+        const uint32_t sm0 = smem_u32(smem);
+        bool ok = __all_sync(0xffffffffu, mbar_wait(&q_full, 0, wc) ? 1 : 0);
+        if (ok) {
+            tc_fence_after();
+            if (elect_one()) {
+                tc_cp_32x128b_warpx4(tmem + kColSfQ, sdesc_sf(sm0 + kOffQsf));
+                tc_cp_32x128b_warpx4(tmem + kColSfQ + 4, sdesc_sf(sm0 + kOffQsf + 512));
+            }
+            __syncwarp();
+        }
+        // S_j is issued one tile ahead of O += P_{j-1} V_{j-1}
+        for (int j = 0; j <= ntiles && ok; ++j) {
+            if (j < ntiles) {
+                const int s = j % kStages, b = j & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&kv_full[s], (uint32_t)(j / kStages) & 1u, wc) ? 1 : 0) ||
+                    !__all_sync(0xffffffffu, mbar_wait(&s_empty[b], ((uint32_t)(j >> 1) & 1u) ^ 1u, wc) ? 1 : 0)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t st = sm0 + kOffStages + s * kStageBytes;
+                const uint32_t sfk = tmem + kColSfK + b * 8;
+                if (elect_one()) {
+                    tc_cp_32x128b_warpx4(sfk, sdesc_sf(st + 2 * kCodeBytes));
+                    tc_cp_32x128b_warpx4(sfk + 4, sdesc_sf(st + 2 * kCodeBytes + 512));
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)
+                        tc_mma_nvf4(tmem + kColS + b * kBK, sdesc_kmajor_sw64(sm0 + kOffQ + ks * 32),
+                                    sdesc_kmajor_sw64(st + ks * 32), idesc_s, tmem + kColSfQ + ks * 4,
+                                    sfk + ks * 4, ks != 0 ? 1u : 0u);
+                    tc_commit(&s_full[b]);
+                    tc_commit(&kv_empty[s]);
+                }
+                __syncwarp();
+            }
+            if (j >= 1) {
+                const int jp = j - 1, s = jp % kStages, b = jp & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&p_full[b], (uint32_t)(jp >> 1) & 1u, wc) ? 1 : 0) ||
+                    !__all_sync(0xffffffffu, mbar_wait(&vt_full[s], (uint32_t)(jp / kStages) & 1u, wc) ? 1 : 0)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t pt = sm0 + kOffP + b * kTileBf16;
+                const uint32_t vt = sm0 + kOffVt + s * kTileBf16;
+                if (elect_one()) {
+#pragma unroll
+                    for (int kc = 0; kc < 2; ++kc)
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            tc_mma_bf16(tmem + kColO, sdesc_kmajor_sw128(pt + kc * kChunk + ks * 32),
+                                        sdesc_kmajor_sw128(vt + kc * kChunk + ks * 32), idesc_o,
+                                        (jp | kc | ks) != 0 ? 1u : 0u);
+                    tc_commit(&p_empty[b]);
+                    tc_commit(&vt_empty[s]);
+                    tc_commit(&o_done);
+                }
+                __syncwarp();
+            }
+        }
+        if (elect_one()) tc_commit(&drain);
+        __syncwarp();
+        int dummy = 0;
+        WaitCtx w2{&dummy, p.dev_status};
+        mbar_wait(&drain, 0, w2);
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ softmax and output
+        const int q = warp & 3;                     // TMEM lane quarter
+        const int r = q * 32 + lane;                // query row in the tile
+        const float c = __fmul_rn(__fmul_rn(*p.g_q, *p.g_k), 1.4426950408889634f / 11.313708498984761f);
+        const float bias = p.s_head ? log2f(p.s_head[h]) : 0.0f;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        float m = -INFINITY, l = 0.0f;
+        bool ok = true;
+        for (int j = 0; j < ntiles && ok; ++j) {
+            const int b = j & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[b], (uint32_t)(j >> 1) & 1u, wc) ? 1 : 0)) { ok = false; break; }
+            tc_fence_after();
+            // pass 1: the tile's largest logit (32 columns at a time: S stays in TMEM)
+            float mt = m;
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem + lane_base + kColS + b * kBK + c4 * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) mt = fmaxf(mt, fmaf(__uint_as_float(v[i]), c, bias));
+            }
+            const float alpha = ex2(m - mt);           // 0 on the first tile (m = -inf)
+            float sum = 0.0f;
+            // P tile reuse: the product that read this buffer two tiles ago is done
+            if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&p_empty[b], ((uint32_t)(j >> 1) & 1u) ^ 1u, wc) ? 1 : 0)) {
+                ok = false;
+                break;
+            }
+            // pass 2: p = exp2(z - m), rounded to bf16 into the swizzled K-major P tile
+            uint8_t* prow = smem + kOffP + b * kTileBf16 + r * 128;
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem + lane_base + kColS + b * kBK + c4 * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int g8 = 0; g8 < 4; ++g8) {           // 8 keys per 16-byte unit
+                    uint32_t w[4];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const float e0 = ex2(fmaf(__uint_as_float(v[g8 * 8 + 2 * t]), c, bias) - mt);
+                        const float e1 = ex2(fmaf(__uint_as_float(v[g8 * 8 + 2 * t + 1]), c, bias) - mt);
+                        sum += e0 + e1;
+                        __nv_bfloat162 hb = __floats2bfloat162_rn(e0, e1);
+                        w[t] = *reinterpret_cast<uint32_t*>(&hb);
+                    }
+                    const int c8 = c4 * 4 + g8, kc = c8 >> 3, pos = (c8 & 7) ^ (r & 7);
+                    *reinterpret_cast<uint4*>(prow + kc * kChunk + pos * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[b]);
+            l = fmaf(l, alpha, sum);
+            m = mt;
+            // rescale the running output by alpha once the previous product is done
+            if (j >= 1) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&o_done, (uint32_t)(j - 1) & 1u, wc) ? 1 : 0)) { ok = false; break; }
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(tmem + lane_base + kColO + c4 * 32, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+                        tmem_st_x32(tmem + lane_base + kColO + c4 * 32, v);
+                    }
+                    tmem_st_wait();
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[b]);
+        }
+        // output: O * g_v / l
+        if (ok && __all_sync(0xffffffffu, mbar_wait(&o_done, (uint32_t)(ntiles - 1) & 1u, wc) ? 1 : 0)) {
+            tc_fence_after();
+            const float sc = __fdiv_rn(*p.g_v, l);
+            uint16_t* orow = p.out + (int64_t)(qrow0 + r) * kD;
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem + lane_base + kColO + c4 * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(v[t * 8 + 2 * u]) * sc,
+                                                                  __uint_as_float(v[t * 8 + 2 * u + 1]) * sc);
+                        w[u] = *reinterpret_cast<uint32_t*>(&hb);
+                    }
+                    *reinterpret_cast<uint4*>(orow + c4 * 32 + t * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+        }
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------ V dequantization
+        const int jd = (warp - 8) * 32 + lane;      // row of V^T (a column of V)
+        bool ok = true;
+        for (int j = 0; j < ntiles && ok; ++j) {
+            const int s = j % kStages;
+            const uint32_t ph = (uint32_t)(j / kStages) & 1u;
+            if (!__all_sync(0xffffffffu, mbar_wait(&kv_full[s], ph, wc) ? 1 : 0) ||
+                !__all_sync(0xffffffffu, mbar_wait(&vt_empty[s], ph ^ 1u, wc) ? 1 : 0)) {
+                ok = false;
+                break;
+            }
+            const uint8_t* st = smem + kOffStages + s * kStageBytes;
+            const uint8_t* vc = st + kCodeBytes;
+            const uint8_t* vsf = st + 2 * kCodeBytes + kSfBytes;
+            uint8_t* vrow = smem + kOffVt + s * kTileBf16 + jd * 128;
+            const int shift = (jd & 1) * 4, blk = jd >> 4;
+#pragma unroll 2
+            for (int c8 = 0; c8 < 16; ++c8) {
+                uint32_t w[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    float f[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int key = c8 * 8 + 2 * t + u;
+                        const uint32_t code = (vc[key * 64 + (jd >> 1)] >> shift) & 15u;
+                        f[u] = e2m1_val(code) * e4m3_to_f32(vsf[sf_byte(key, blk)]);   // exact
+                    }
+                    w[t] = (__float_as_uint(f[0]) >> 16) | (__float_as_uint(f[1]) & 0xFFFF0000u);
+                }
+                const int kc = c8 >> 3, pos = (c8 & 7) ^ (jd & 7);
+                *reinterpret_cast<uint4*>(vrow + kc * kChunk + pos * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&vt_full[s]);
+                mbar_arrive(&kv_empty[s]);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace attn
+
+cudaError_t launch_attention(const uint8_t* q_codes, const uint8_t* q_sf, const float* g_q, const uint8_t* k_codes,
+                             const uint8_t* k_sf, const float* g_k, const uint8_t* v_codes, const uint8_t* v_sf,
+                             const float* g_v, const float* s_head, int64_t H, int64_t Lq, int64_t Lk, void* out,
+                             int* dev_status, cudaStream_t stream) {
+    using namespace attn;
+    CUtensorMap tq, tk, tv;
+    if (make_tmap_2d(&tq, q_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kD / 2, (uint64_t)(H * Lq), kD / 2, kD / 2, kBQ,
+                     CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
+        make_tmap_2d(&tk, k_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kD / 2, (uint64_t)(H * Lk), kD / 2, kD / 2, kBK,
+                     CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
+        make_tmap_2d(&tv, v_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kD / 2, (uint64_t)(H * Lk), kD / 2, kD / 2, kBK,
+                     CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    Params p;
+    p.q_sf = q_sf;
+    p.k_sf = k_sf;
+    p.v_sf = v_sf;
+    p.g_q = g_q;
+    p.g_k = g_k;
+    p.g_v = g_v;
+    p.s_head = s_head;
+    p.out = static_cast<uint16_t*>(out);
+    p.Lq = (int)Lq;
+    p.Lk = (int)Lk;
+    p.H = (int)H;
+    p.dev_status = dev_status;
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)(Lq / kBQ), (unsigned)H);
+    attn_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
+    count_launch(1);
+    return cudaGetLastError();
+}
+
+}  // namespace nvfp4
