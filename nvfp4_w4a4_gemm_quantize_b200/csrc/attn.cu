@@ -35,6 +35,10 @@ constexpr int kD = 128;                      // head dimension
 constexpr int kBQ = 128;                     // queries per CTA
 constexpr int kBK = 128;                     // keys per tile
 constexpr int kThreads = 384;
+constexpr int kRegsCtl = 48;                 // warps 0-3: producer, MMA issuer, two idle
+constexpr int kRegsSoftmax = 232;            // warps 4-7
+constexpr int kRegsDequant = 80;             // warps 8-11
+static_assert(128 * (kRegsCtl + kRegsSoftmax + kRegsDequant) <= kThreads * 120, "register split");
 constexpr int kStages = 2;                   // K / V code stages
 constexpr int kCodeBytes = kBK * kD / 2;     // 8 KB: 128 rows x 64 bytes
 constexpr int kSfBytes = 1024;               // two 512-byte scale atoms (128 rows x 8 blocks)
@@ -99,6 +103,29 @@ __device__ __forceinline__ float e2m1_val(uint32_t c) {
     return (c & 8u) ? -mag : mag;
 }
 
+// Two E2M1 codes (one byte, low nibble first) times their shared scale,
+// exactly, as a bf16 pair: the f16 decode shifted down three bits is the bf16
+// pattern of the value times 2^-112 (sign kept), and one bf16 multiply by the
+// scale times 2^112 gives the product (at most 6 significant bits).
+__device__ __forceinline__ uint32_t dequant_pair_attn(uint32_t byte, uint32_t scale_b2) {
+    uint32_t h2, out;
+    asm("{\n\t.reg .b8 c;\n\t"
+        "cvt.u8.u32 c, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, c;\n\t}"
+        : "=r"(h2)
+        : "r"(byte));
+    const uint32_t b2 = ((h2 >> 3) & 0x0FFF0FFFu) | (h2 & 0x80008000u);
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(out) : "r"(b2), "r"(scale_b2));
+    return out;
+}
+
+// E4M3 byte -> bf16 of (scale * 2^112) in both halves (exact).
+__device__ __forceinline__ uint32_t e4m3_to_b2_scaled_attn(uint32_t code) {
+    const float f = e4m3_to_f32(code) * 0x1p112f;
+    const uint32_t b = __float_as_uint(f) >> 16;
+    return b | (b << 16);
+}
+
 // Byte of (row r, 16-value block c) inside a 128-row group's two scale atoms.
 __device__ __forceinline__ int sf_byte(int r, int c) { return (c >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (c & 3); }
 
@@ -110,6 +137,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
     __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_done, drain;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
+    __shared__ uint32_t vlut[256];                // E4M3 byte -> bf16 pair of (scale * 2^112)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -150,6 +178,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
 
+    // registers: the softmax warpgroup holds a row of logits (128 values); the
+    // producer / MMA warpgroup and the dequantizers need few.  The shares add
+    // up to 128 * (48 + 232 + 80) = 46080 <= 384 * (registers at launch).
+    if (warp < 4) {
+    regs_dec<kRegsCtl>();
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         const uint64_t pol = policy_evict_normal();
@@ -253,7 +286,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
         int dummy = 0;
         WaitCtx w2{&dummy, p.dev_status};
         mbar_wait(&drain, 0, w2);
-    } else if (warp >= 4 && warp < 8) {
+    }
+    } else if (warp < 8) {
+        regs_inc<kRegsSoftmax>();
         // ------------------------------------------------------------ softmax and output
         const int q = warp & 3;                     // TMEM lane quarter
         const int r = q * 32 + lane;                // query row in the tile
@@ -266,50 +301,54 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
             const int b = j & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&s_full[b], (uint32_t)(j >> 1) & 1u, wc) ? 1 : 0)) { ok = false; break; }
             tc_fence_after();
-            // pass 1: the tile's largest logit (32 columns at a time: S stays in TMEM)
-            float mt = m;
+            // the tile's 128 logits of this row, in registers (one TMEM wait)
+            uint32_t v[kBK];
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem + lane_base + kColS + b * kBK + c4 * 32, v);
-                tmem_ld_wait();
+            for (int c4 = 0; c4 < 4; ++c4)
+                tmem_ld_32x32b_x32(tmem + lane_base + kColS + b * kBK + c4 * 32,
+                                   *reinterpret_cast<uint32_t(*)[32]>(&v[c4 * 32]));
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[b]);
+            float mt = -INFINITY;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) mt = fmaxf(mt, fmaf(__uint_as_float(v[i]), c, bias));
+            for (int i = 0; i < kBK; ++i) {
+                const float z = fmaf(__uint_as_float(v[i]), c, bias);
+                v[i] = __float_as_uint(z);
+                mt = fmaxf(mt, z);
             }
-            const float alpha = ex2(m - mt);           // 0 on the first tile (m = -inf)
+            // lazy rescaling: the reference maximum moves only when the tile's
+            // maximum exceeds it by more than 8 (p stays below 2^8); O and l are
+            // rescaled then, and share the reference
+            const bool move = mt > m + 8.0f;
+            const float mref = move ? mt : m;
+            const float alpha = move ? ex2(m - mt) : 1.0f;          // 0 on the first tile (m = -inf)
             float sum = 0.0f;
             // P tile reuse: the product that read this buffer two tiles ago is done
             if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&p_empty[b], ((uint32_t)(j >> 1) & 1u) ^ 1u, wc) ? 1 : 0)) {
                 ok = false;
                 break;
             }
-            // pass 2: p = exp2(z - m), rounded to bf16 into the swizzled K-major P tile
+            // p = exp2(z - mref), rounded to bf16 into the swizzled K-major P tile
             uint8_t* prow = smem + kOffP + b * kTileBf16 + r * 128;
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem + lane_base + kColS + b * kBK + c4 * 32, v);
-                tmem_ld_wait();
+            for (int c8 = 0; c8 < 16; ++c8) {              // 8 keys per 16-byte unit
+                uint32_t w[4];
 #pragma unroll
-                for (int g8 = 0; g8 < 4; ++g8) {           // 8 keys per 16-byte unit
-                    uint32_t w[4];
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const float e0 = ex2(fmaf(__uint_as_float(v[g8 * 8 + 2 * t]), c, bias) - mt);
-                        const float e1 = ex2(fmaf(__uint_as_float(v[g8 * 8 + 2 * t + 1]), c, bias) - mt);
-                        sum += e0 + e1;
-                        __nv_bfloat162 hb = __floats2bfloat162_rn(e0, e1);
-                        w[t] = *reinterpret_cast<uint32_t*>(&hb);
-                    }
-                    const int c8 = c4 * 4 + g8, kc = c8 >> 3, pos = (c8 & 7) ^ (r & 7);
-                    *reinterpret_cast<uint4*>(prow + kc * kChunk + pos * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+                for (int t = 0; t < 4; ++t) {
+                    const float e0 = ex2(__uint_as_float(v[c8 * 8 + 2 * t]) - mref);
+                    const float e1 = ex2(__uint_as_float(v[c8 * 8 + 2 * t + 1]) - mref);
+                    sum += e0 + e1;
+                    __nv_bfloat162 hb = __floats2bfloat162_rn(e0, e1);
+                    w[t] = *reinterpret_cast<uint32_t*>(&hb);
                 }
+                const int kc = c8 >> 3, pos = (c8 & 7) ^ (r & 7);
+                *reinterpret_cast<uint4*>(prow + kc * kChunk + pos * 16) = make_uint4(w[0], w[1], w[2], w[3]);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_empty[b]);
+            const float mt_used = mref;
             l = fmaf(l, alpha, sum);
-            m = mt;
+            m = mt_used;
             // rescale the running output by alpha once the previous product is done
             if (j >= 1) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&o_done, (uint32_t)(j - 1) & 1u, wc) ? 1 : 0)) { ok = false; break; }
@@ -355,9 +394,18 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
                 }
             }
         }
-    } else if (warp >= 8) {
+    } else {
+        regs_dec<kRegsDequant>();
         // ------------------------------------------------------------ V dequantization
-        const int jd = (warp - 8) * 32 + lane;      // row of V^T (a column of V)
+        // thread: a pair of V columns (d = 2 dp, 2 dp + 1: one code byte per key,
+        // one scale) and half of the tile's keys (one 64-key chunk of V^T); per
+        // key the pair is decoded at once (cvt e2m1x2 -> f16x2 -> bf16 2^-112,
+        // times the bf16 scale 2^112 from a 256-entry table: exact), and eight
+        // keys' pairs are regrouped by byte permutes into the two V^T rows.
+        const int t = threadIdx.x - 256;
+        const int dp = t & 63, kh = t >> 6;
+        for (int i = t; i < 256; i += 128) vlut[i] = e4m3_to_b2_scaled_attn((uint32_t)i);
+        asm volatile("bar.sync 1, 128;" ::: "memory");           // the four dequantizer warps only
         bool ok = true;
         for (int j = 0; j < ntiles && ok; ++j) {
             const int s = j % kStages;
@@ -370,24 +418,25 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
             const uint8_t* st = smem + kOffStages + s * kStageBytes;
             const uint8_t* vc = st + kCodeBytes;
             const uint8_t* vsf = st + 2 * kCodeBytes + kSfBytes;
-            uint8_t* vrow = smem + kOffVt + s * kTileBf16 + jd * 128;
-            const int shift = (jd & 1) * 4, blk = jd >> 4;
+            uint8_t* row0 = smem + kOffVt + s * kTileBf16 + kh * kChunk + (2 * dp) * 128;
+            uint8_t* row1 = row0 + 128;
+            const int blk = dp >> 3;
 #pragma unroll 2
-            for (int c8 = 0; c8 < 16; ++c8) {
-                uint32_t w[4];
+            for (int g = 0; g < 8; ++g) {
+                uint32_t pr[8];
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    float f[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int key = c8 * 8 + 2 * t + u;
-                        const uint32_t code = (vc[key * 64 + (jd >> 1)] >> shift) & 15u;
-                        f[u] = e2m1_val(code) * e4m3_to_f32(vsf[sf_byte(key, blk)]);   // exact
-                    }
-                    w[t] = (__float_as_uint(f[0]) >> 16) | (__float_as_uint(f[1]) & 0xFFFF0000u);
+                for (int u = 0; u < 8; ++u) {
+                    const int key = kh * 64 + g * 8 + u;
+                    pr[u] = dequant_pair_attn(vc[key * 64 + dp], vlut[vsf[sf_byte(key, blk)]]);
                 }
-                const int kc = c8 >> 3, pos = (c8 & 7) ^ (jd & 7);
-                *reinterpret_cast<uint4*>(vrow + kc * kChunk + pos * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+                uint32_t e[4], o[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(e[u]) : "r"(pr[2 * u]), "r"(pr[2 * u + 1]));
+                    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(o[u]) : "r"(pr[2 * u]), "r"(pr[2 * u + 1]));
+                }
+                *reinterpret_cast<uint4*>(row0 + ((g ^ ((2 * dp) & 7)) * 16)) = make_uint4(e[0], e[1], e[2], e[3]);
+                *reinterpret_cast<uint4*>(row1 + ((g ^ ((2 * dp + 1) & 7)) * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
             }
             fence_proxy_async_smem();
             __syncwarp();
