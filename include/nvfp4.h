@@ -353,20 +353,24 @@ nvfp4_status nvfp4_mx_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const ui
  *   (quantized along d), head h owning rows h*Lq .. and h*Lk .. ; tensor scales
  *   q_scale, k_scale, v_scale (device floats).
  *   S = Q K^T on the block-scaled FP4 tensor cores (FP32); online softmax in
- *   FP32 with the hardware exp2; P rounded to bf16; V dequantized exactly to
- *   bf16; O = P V on the bf16 tensor cores (FP32), divided by the row sum and
- *   multiplied by g_v, rounded to bf16.
- * s_head   nullable device float [H] (1 for every head).  Within one head's
- *          softmax the log(s_head) term is a constant shift of every logit.
- * out      bf16 [H*Lq, d], 16-byte aligned.
- * d == 128, Lq and Lk multiples of 128 (no masking), H <= 65535.  One kernel:
- * a CTA per (128 queries, head).
+ *   FP32 with the hardware exp2; P rounded to bf16; V decoded exactly to bf16
+ *   (e2m1 * e4m3); O = P V on the bf16 tensor cores (FP32), divided by the row
+ *   sum and multiplied by g_v, rounded to bf16.
+ * s_head    nullable device float [H] (1 for every head).  Within one head's
+ *           softmax the log(s_head) term is a constant shift of every logit.
+ * out       bf16 [H*Lq, d], 16-byte aligned.
+ * workspace device scratch of >= nvfp4_attention_workspace_bytes(H, Lk, d)
+ *           bytes, 16-byte aligned: V decoded to bf16 and transposed (once
+ *           per call, then read by every query tile); not preserved.
+ * d == 128, Lq and Lk multiples of 128 (no masking), H <= 65535.  Two kernels:
+ * the V transpose, then a CTA per (128 queries, head).
  */
+size_t nvfp4_attention_workspace_bytes(int64_t H, int64_t Lk, int64_t d);   /* H * d * Lk * 2 */
 nvfp4_status nvfp4_attention(const uint8_t *q_codes, const uint8_t *q_sf, const float *q_scale,
                              const uint8_t *k_codes, const uint8_t *k_sf, const float *k_scale,
                              const uint8_t *v_codes, const uint8_t *v_sf, const float *v_scale,
                              const float *s_head, int64_t H, int64_t Lq, int64_t Lk, int64_t d, void *out,
-                             int *dev_status, nvfp4_stream_t stream);
+                             void *workspace, size_t workspace_bytes, int *dev_status, nvfp4_stream_t stream);
 
 /* Static text for a status code. */
 const char *nvfp4_status_string(nvfp4_status s);

@@ -10,7 +10,7 @@ Low-level (same names and argument order as the C calls):
     nvfp4_quantize_noalloc, nvfp4_quantize_block, nvfp4_block_size_errors, nvfp4_select_block_size,
     nvfp4_dequantize, nvfp4_fake_quantize, nvfp4_ste_backward,
     nvfp4_gemm_w4a4, nvfp4_gemm_w4a4_grouped, nvfp4_gemm_w4a16, nvfp4_mx_sf_bytes, nvfp4_mx_quantize,
-    nvfp4_mx_dequantize, nvfp4_mx_gemm, nvfp4_attention, nvfp4_launch_count
+    nvfp4_mx_dequantize, nvfp4_mx_gemm, nvfp4_attention, nvfp4_attention_workspace_bytes, nvfp4_launch_count
 Convenience (allocate outputs with torch, then call the above):
     NVFP4Tensor, quantize, dequantize, gemm_w4a4, gemm_w4a4_grouped, gemm_w4a16,
     fake_quantize, ste_backward, FakeQuantizeSTE (autograd: the two kernels),
@@ -173,11 +173,16 @@ def nvfp4_mx_gemm(a_codes, a_sf, b_codes, b_sf, M, N, K, y, y_dtype=NVFP4_DTYPE_
                               _ptr(dev_status), _stream(stream)), "nvfp4_mx_gemm")
 
 
+def nvfp4_attention_workspace_bytes(H: int, Lk: int, d: int) -> int:
+    return int(lib().nvfp4_attention_workspace_bytes(H, Lk, d))
+
+
 def nvfp4_attention(q_codes, q_sf, q_scale, k_codes, k_sf, k_scale, v_codes, v_sf, v_scale, s_head, H, Lq, Lk, d,
-                    out, dev_status=None, stream=None) -> None:
+                    out, workspace, workspace_bytes, dev_status=None, stream=None) -> None:
     check(lib().nvfp4_attention(_ptr(q_codes), _ptr(q_sf), _ptr(q_scale), _ptr(k_codes), _ptr(k_sf), _ptr(k_scale),
                                 _ptr(v_codes), _ptr(v_sf), _ptr(v_scale), _ptr(s_head), H, Lq, Lk, d, _ptr(out),
-                                _ptr(dev_status), _stream(stream)), "nvfp4_attention")
+                                _ptr(workspace), workspace_bytes, _ptr(dev_status), _stream(stream)),
+          "nvfp4_attention")
 
 
 def nvfp4_gemm_w4a16(x, w_codes, w_sf, w_scale, M, N, K, y, y_dtype=NVFP4_DTYPE_BF16,
@@ -414,12 +419,16 @@ def select_block_size(x: torch.Tensor, lam: float, tensor_scale: torch.Tensor | 
 
 # ----------------------------------------------------------------- attention (Eq. 10)
 def attention(q: NVFP4Tensor, k: NVFP4Tensor, v: NVFP4Tensor, H: int, s_head: torch.Tensor | None = None,
-              out: torch.Tensor | None = None, dev_status=None, stream=None) -> torch.Tensor:
+              out: torch.Tensor | None = None, workspace: torch.Tensor | None = None, dev_status=None,
+              stream=None) -> torch.Tensor:
     """softmax(Q K^T / sqrt(d) + log s_head) V per head over NVFP4 Q [H*Lq, d],
     K and V [H*Lk, d] (d = 128); returns bf16 [H*Lq, d]."""
     d = q.k
     Lq, Lk = q.rows // H, k.rows // H
     o = out if out is not None else torch.empty(q.rows, d, dtype=torch.bfloat16, device=q.codes.device)
+    wsb = nvfp4_attention_workspace_bytes(H, Lk, d)
+    if workspace is None:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=q.codes.device)
     nvfp4_attention(q.codes, q.sf, q.scale, k.codes, k.sf, k.scale, v.codes, v.sf, v.scale, s_head, H, Lq, Lk, d, o,
-                    dev_status, stream)
+                    workspace, wsb, dev_status, stream)
     return o

@@ -54,7 +54,9 @@ SIGNATURES = {
                                   _p]),
     "nvfp4_gemm_w4a4_grouped": (_status, [_p, _int, _int, _p, _p]),
     "nvfp4_gemm_w4a16": (_status, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _int, _p, _p]),
-    "nvfp4_attention": (_status, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _p]),
+    "nvfp4_attention": (_status, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p,
+                                  ctypes.c_size_t, _p, _p]),
+    "nvfp4_attention_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64]),
     "nvfp4_mx_sf_bytes": (ctypes.c_size_t, [_i64, _i64]),
     "nvfp4_mx_quantize": (_status, [_p, _i64, _i64, _i64, _p, _p, _p]),
     "nvfp4_mx_dequantize": (_status, [_p, _p, _i64, _i64, _p, _int, _p]),

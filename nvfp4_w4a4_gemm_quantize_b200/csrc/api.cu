@@ -385,20 +385,28 @@ nvfp4_status nvfp4_attention(const uint8_t* q_codes, const uint8_t* q_sf, const 
                              const uint8_t* k_codes, const uint8_t* k_sf, const float* k_scale,
                              const uint8_t* v_codes, const uint8_t* v_sf, const float* v_scale,
                              const float* s_head, int64_t H, int64_t Lq, int64_t Lk, int64_t d, void* out,
-                             int* dev_status, nvfp4_stream_t stream) {
+                             void* workspace, size_t workspace_bytes, int* dev_status, nvfp4_stream_t stream) {
     if (H <= 0 || Lq <= 0 || Lk <= 0 || d <= 0) return NVFP4_ERR_INVALID_ARG;
     if (!q_codes || !q_sf || !q_scale || !k_codes || !k_sf || !k_scale || !v_codes || !v_sf || !v_scale || !out)
         return NVFP4_ERR_INVALID_ARG;
     if (d != 128 || Lq % 128 != 0 || Lk % 128 != 0 || H > 65535 || H * Lq >= ((int64_t)1 << 31) ||
         H * Lk >= ((int64_t)1 << 31))
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!workspace || workspace_bytes < attention_workspace_bytes(H, Lk, d)) return NVFP4_ERR_WORKSPACE;
     if (!aligned16(q_codes) || !aligned16(q_sf) || !aligned16(k_codes) || !aligned16(k_sf) || !aligned16(v_codes) ||
-        !aligned16(v_sf) || !aligned16(out) || (s_head && (reinterpret_cast<uintptr_t>(s_head) & 3u)))
+        !aligned16(v_sf) || !aligned16(out) || !aligned16(workspace) ||
+        (s_head && (reinterpret_cast<uintptr_t>(s_head) & 3u)))
         return NVFP4_ERR_MISALIGNED;
     nvfp4_status st = device_ok(nullptr);
     if (st != NVFP4_OK) return st;
     return cuda_status(launch_attention(q_codes, q_sf, q_scale, k_codes, k_sf, k_scale, v_codes, v_sf, v_scale,
-                                        s_head, H, Lq, Lk, out, dev_status, reinterpret_cast<cudaStream_t>(stream)));
+                                        s_head, H, Lq, Lk, out, workspace, dev_status,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t nvfp4_attention_workspace_bytes(int64_t H, int64_t Lk, int64_t d) {
+    if (H <= 0 || Lk <= 0 || d <= 0) return 0;
+    return attention_workspace_bytes(H, Lk, d);
 }
 
 nvfp4_status nvfp4_gemm_w4a16(const void* x_bf16, const uint8_t* w_codes, const uint8_t* w_sf, const float* w_scale,

@@ -1,23 +1,26 @@
-// attn.cu -- attention over an NVFP4 key / value cache, one head per CTA row
-// of the grid ("NVFP4-DiT ..." README, Algorithmic framework, Eq. 10:
-// Attention(Q, K, V) = softmax(Q K^T / sqrt(d_k) + log(s_head)) V with a
-// per-head scale s_head; Systems optimization: FP4-packed attention).
+// attn.cu -- attention over an NVFP4 key / value cache ("NVFP4-DiT ..."
+// README, Algorithmic framework, Eq. 10: Attention(Q, K, V) =
+// softmax(Q K^T / sqrt(d_k) + log(s_head)) V with a per-head scale s_head;
+// Systems optimization: FP4-packed attention).
 //
 // Q, K, V are NVFP4 tensors quantized along the head dimension d = 128
 // (blocks of 16, tensor scales g_q, g_k, g_v): Q [H*Lq, d], K and V [H*Lk, d].
-// Per CTA: 128 queries of one head, keys in tiles of 128.
-//   S = Q K^T     block-scaled FP4 MMA (kind::mxf4nvf4, K = d), FP32 in TMEM,
+// Two kernels:
+//   v_transpose   V decoded exactly to bf16 (e2m1 * e4m3: at most 6
+//                 significant bits) and transposed to V^T [H*d, Lk] in the
+//                 caller's workspace -- once per call, instead of once per
+//                 query tile;
+//   attention     per CTA 128 queries of one head, keys in tiles of 128:
+//     S = Q K^T   block-scaled FP4 MMA (kind::mxf4nvf4, K = d), FP32 in TMEM,
 //                 two S buffers so the next tile's product overlaps softmax;
-//   softmax       one query row per thread (online: running max m, sum l),
-//                 exp2 of (S * g_q g_k log2(e) / sqrt(d) + log2(s_head) - m),
-//                 P rounded to bf16 into a 128-byte-swizzled K-major tile, and
-//                 the running output rescaled in TMEM when m grows;
-//   V             dequantized exactly to bf16 (e2m1 * e4m3 has at most 6
-//                 significant bits) into a K-major V^T tile by four warps;
-//   O += P V      bf16 MMA (kind::f16), FP32 in TMEM;
-//   output        O * g_v / l, rounded to bf16.
+//     softmax     one query row per thread (online: reference maximum m, sum
+//                 l), exp2 of (S * g_q g_k log2(e) / sqrt(d) + log2(s_head) - m),
+//                 P rounded to bf16 into a 128-byte-swizzled K-major tile; the
+//                 running output is rescaled in TMEM when m moves;
+//     O += P V    bf16 MMA (kind::f16) on TMA-loaded V^T tiles, FP32 in TMEM;
+//     output      O * g_v / l, rounded to bf16.
 // Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 4-7
-// softmax and output, warps 8-11 V dequantization; every wait is bounded.
+// softmax and output; every wait is bounded.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -34,25 +37,24 @@ namespace attn {
 constexpr int kD = 128;                      // head dimension
 constexpr int kBQ = 128;                     // queries per CTA
 constexpr int kBK = 128;                     // keys per tile
-constexpr int kThreads = 384;
-constexpr int kRegsCtl = 48;                 // warps 0-3: producer, MMA issuer, two idle
-constexpr int kRegsSoftmax = 232;            // warps 4-7
-constexpr int kRegsDequant = 80;             // warps 8-11
-static_assert(128 * (kRegsCtl + kRegsSoftmax + kRegsDequant) <= kThreads * 120, "register split");
+constexpr int kThreads = 256;
 constexpr int kStages = 2;                   // K / V code stages
 constexpr int kCodeBytes = kBK * kD / 2;     // 8 KB: 128 rows x 64 bytes
 constexpr int kSfBytes = 1024;               // two 512-byte scale atoms (128 rows x 8 blocks)
-constexpr int kStageBytes = 2 * kCodeBytes + 2 * kSfBytes;
 constexpr int kTileBf16 = kBQ * kBK * 2;     // 32 KB: two 64-key chunks of 128 rows x 128 bytes
 constexpr int kChunk = 128 * 128;            // 16 KB
+// stage: K codes (64-byte swizzle), K scales, V^T bf16 tile (128-byte swizzle, 1024-aligned)
+constexpr int kOffStVt = kCodeBytes + kSfBytes;
+constexpr int kStageBytes = kOffStVt + kTileBf16;
 
 // shared memory (offsets from a 1024-aligned base)
 constexpr int kOffQ = 0;
 constexpr int kOffQsf = kOffQ + kCodeBytes;
 constexpr int kOffStages = kOffQsf + kSfBytes;
 constexpr int kOffP = kOffStages + kStages * kStageBytes;          // 2 P tiles
-constexpr int kOffVt = kOffP + 2 * kTileBf16;                      // kStages V^T tiles
-constexpr int kSmemBytes = kOffVt + kStages * kTileBf16 + 1024;
+constexpr int kSmemBytes = kOffP + 2 * kTileBf16 + 1024;
+static_assert(kOffStVt % 1024 == 0 && kStageBytes % 1024 == 0 && kOffStages % 1024 == 0 && kOffP % 1024 == 0,
+              "swizzled tiles are 1024-byte aligned");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 // TMEM columns
@@ -131,13 +133,12 @@ __device__ __forceinline__ int sf_byte(int r, int c) { return (c >> 2) * 512 + (
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-            const __grid_constant__ CUtensorMap tmap_v, const Params p) {
+            const __grid_constant__ CUtensorMap tmap_vt, const Params p) {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t q_full, kv_full[kStages], kv_empty[kStages], vt_full[kStages], vt_empty[kStages];
+    __shared__ __align__(8) uint64_t q_full, kv_full[kStages], kv_empty[kStages];
     __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_done, drain;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
-    __shared__ uint32_t vlut[256];                // E4M3 byte -> bf16 pair of (scale * 2^112)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -152,9 +153,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
         mbar_init(&q_full, 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1 + 4);          // the S product's commit + four dequantizer warps
-            mbar_init(&vt_full[s], 4);
-            mbar_init(&vt_empty[s], 1);
+            mbar_init(&kv_empty[s], 2);              // the S product's and the PV product's commits
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
@@ -167,7 +166,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
         fence_barrier_init();
         tma_prefetch_desc(&tmap_q);
         tma_prefetch_desc(&tmap_k);
-        tma_prefetch_desc(&tmap_v);
+        tma_prefetch_desc(&tmap_vt);
     }
     if (warp == 1) {
         tmem_alloc(&tmem_base_sh, 512);
@@ -178,11 +177,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
 
-    // registers: the softmax warpgroup holds a row of logits (128 values); the
-    // producer / MMA warpgroup and the dequantizers need few.  The shares add
-    // up to 128 * (48 + 232 + 80) = 46080 <= 384 * (registers at launch).
     if (warp < 4) {
-    regs_dec<kRegsCtl>();
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         const uint64_t pol = policy_evict_normal();
@@ -202,10 +197,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
             if (elect_one()) {
                 mbar_arrive_expect_tx(&kv_full[s], kStageBytes);
                 tma_load_2d(st, &tmap_k, &kv_full[s], 0, kr, pol);
-                tma_load_2d(st + kCodeBytes, &tmap_v, &kv_full[s], 0, kr, pol);
-                bulk_load(st + 2 * kCodeBytes, p.k_sf + (int64_t)(kr >> 7) * kSfBytes, kSfBytes, &kv_full[s], pol);
-                bulk_load(st + 2 * kCodeBytes + kSfBytes, p.v_sf + (int64_t)(kr >> 7) * kSfBytes, kSfBytes,
-                          &kv_full[s], pol);
+                bulk_load(st + kCodeBytes, p.k_sf + (int64_t)(kr >> 7) * kSfBytes, kSfBytes, &kv_full[s], pol);
+                // V^T rows h*d .. h*d + 127, keys j*128 .. j*128 + 127, as two 64-key chunks
+                tma_load_2d(st + kOffStVt, &tmap_vt, &kv_full[s], j * kBK, h * kD, pol);
+                tma_load_2d(st + kOffStVt + kChunk, &tmap_vt, &kv_full[s], j * kBK + 64, h * kD, pol);
             }
             __syncwarp();
         }
@@ -244,8 +239,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
                 const uint32_t st = sm0 + kOffStages + s * kStageBytes;
                 const uint32_t sfk = tmem + kColSfK + b * 8;
                 if (elect_one()) {
-                    tc_cp_32x128b_warpx4(sfk, sdesc_sf(st + 2 * kCodeBytes));
-                    tc_cp_32x128b_warpx4(sfk + 4, sdesc_sf(st + 2 * kCodeBytes + 512));
+                    tc_cp_32x128b_warpx4(sfk, sdesc_sf(st + kCodeBytes));
+                    tc_cp_32x128b_warpx4(sfk + 4, sdesc_sf(st + kCodeBytes + 512));
 #pragma unroll
                     for (int ks = 0; ks < 2; ++ks)
                         tc_mma_nvf4(tmem + kColS + b * kBK, sdesc_kmajor_sw64(sm0 + kOffQ + ks * 32),
@@ -258,14 +253,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
             }
             if (j >= 1) {
                 const int jp = j - 1, s = jp % kStages, b = jp & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&p_full[b], (uint32_t)(jp >> 1) & 1u, wc) ? 1 : 0) ||
-                    !__all_sync(0xffffffffu, mbar_wait(&vt_full[s], (uint32_t)(jp / kStages) & 1u, wc) ? 1 : 0)) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&p_full[b], (uint32_t)(jp >> 1) & 1u, wc) ? 1 : 0)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t pt = sm0 + kOffP + b * kTileBf16;
-                const uint32_t vt = sm0 + kOffVt + s * kTileBf16;
+                const uint32_t vt = sm0 + kOffStages + s * kStageBytes + kOffStVt;
                 if (elect_one()) {
 #pragma unroll
                     for (int kc = 0; kc < 2; ++kc)
@@ -275,7 +269,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
                                         sdesc_kmajor_sw128(vt + kc * kChunk + ks * 32), idesc_o,
                                         (jp | kc | ks) != 0 ? 1u : 0u);
                     tc_commit(&p_empty[b]);
-                    tc_commit(&vt_empty[s]);
+                    tc_commit(&kv_empty[s]);
                     tc_commit(&o_done);
                 }
                 __syncwarp();
@@ -287,8 +281,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
         WaitCtx w2{&dummy, p.dev_status};
         mbar_wait(&drain, 0, w2);
     }
-    } else if (warp < 8) {
-        regs_inc<kRegsSoftmax>();
+    } else {
         // ------------------------------------------------------------ softmax and output
         const int q = warp & 3;                     // TMEM lane quarter
         const int r = q * 32 + lane;                // query row in the tile
@@ -394,57 +387,6 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
                 }
             }
         }
-    } else {
-        regs_dec<kRegsDequant>();
-        // ------------------------------------------------------------ V dequantization
-        // thread: a pair of V columns (d = 2 dp, 2 dp + 1: one code byte per key,
-        // one scale) and half of the tile's keys (one 64-key chunk of V^T); per
-        // key the pair is decoded at once (cvt e2m1x2 -> f16x2 -> bf16 2^-112,
-        // times the bf16 scale 2^112 from a 256-entry table: exact), and eight
-        // keys' pairs are regrouped by byte permutes into the two V^T rows.
-        const int t = threadIdx.x - 256;
-        const int dp = t & 63, kh = t >> 6;
-        for (int i = t; i < 256; i += 128) vlut[i] = e4m3_to_b2_scaled_attn((uint32_t)i);
-        asm volatile("bar.sync 1, 128;" ::: "memory");           // the four dequantizer warps only
-        bool ok = true;
-        for (int j = 0; j < ntiles && ok; ++j) {
-            const int s = j % kStages;
-            const uint32_t ph = (uint32_t)(j / kStages) & 1u;
-            if (!__all_sync(0xffffffffu, mbar_wait(&kv_full[s], ph, wc) ? 1 : 0) ||
-                !__all_sync(0xffffffffu, mbar_wait(&vt_empty[s], ph ^ 1u, wc) ? 1 : 0)) {
-                ok = false;
-                break;
-            }
-            const uint8_t* st = smem + kOffStages + s * kStageBytes;
-            const uint8_t* vc = st + kCodeBytes;
-            const uint8_t* vsf = st + 2 * kCodeBytes + kSfBytes;
-            uint8_t* row0 = smem + kOffVt + s * kTileBf16 + kh * kChunk + (2 * dp) * 128;
-            uint8_t* row1 = row0 + 128;
-            const int blk = dp >> 3;
-#pragma unroll 2
-            for (int g = 0; g < 8; ++g) {
-                uint32_t pr[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int key = kh * 64 + g * 8 + u;
-                    pr[u] = dequant_pair_attn(vc[key * 64 + dp], vlut[vsf[sf_byte(key, blk)]]);
-                }
-                uint32_t e[4], o[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(e[u]) : "r"(pr[2 * u]), "r"(pr[2 * u + 1]));
-                    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(o[u]) : "r"(pr[2 * u]), "r"(pr[2 * u + 1]));
-                }
-                *reinterpret_cast<uint4*>(row0 + ((g ^ ((2 * dp) & 7)) * 16)) = make_uint4(e[0], e[1], e[2], e[3]);
-                *reinterpret_cast<uint4*>(row1 + ((g ^ ((2 * dp + 1) & 7)) * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&vt_full[s]);
-                mbar_arrive(&kv_empty[s]);
-            }
-        }
     }
 
     tc_fence_before();
@@ -456,21 +398,79 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
     }
 }
 
+// V [H*Lk, d] NVFP4 -> V^T [H*d, Lk] bf16, exact (the tensor scale g_v is
+// applied with the output).  A CTA per (64 keys, head): 256 threads decode 16
+// code bytes each (one key, 32 values of d) into a padded shared tile
+// [d][64 keys], then write its 128 rows of 128 bytes out.
+constexpr int kVtKeys = 64;
+constexpr int kVtPitch = kVtKeys + 2;            // bf16 elements per shared row (padding spreads banks)
+
+__global__ void __launch_bounds__(256)
+v_transpose_kernel(const uint8_t* __restrict__ v_codes, const uint8_t* __restrict__ v_sf, int Lk,
+                   uint16_t* __restrict__ vt) {
+    __shared__ uint16_t tile[kD * kVtPitch];
+    const int t = threadIdx.x;
+    const int h = blockIdx.y, key0 = blockIdx.x * kVtKeys;
+    const int key = t >> 2, part = t & 3;                  // 16 bytes: d = 32 part .. 32 part + 31
+    const int64_t row = (int64_t)h * Lk + key0 + key;      // row of V
+    const uint4 cb = *reinterpret_cast<const uint4*>(v_codes + row * (kD / 2) + part * 16);
+    const uint32_t w[4] = {cb.x, cb.y, cb.z, cb.w};
+    // scales of blocks 2 part and 2 part + 1 (16 values of d each); layout of a
+    // [rows, 128] tensor: two 512-byte atoms per 128-row group
+    const int rr = (int)(row & 127);
+    const uint8_t* sfr = v_sf + (row >> 7) * 1024 + (rr & 31) * 16 + (rr >> 5) * 4;
+#pragma unroll
+    for (int hb = 0; hb < 2; ++hb) {
+        const int blk = 2 * part + hb;
+        const uint32_t sc = e4m3_to_b2_scaled_attn(sfr[(blk >> 2) * 512 + (blk & 3)]);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const uint32_t word = w[2 * hb + q];
+#pragma unroll
+            for (int by = 0; by < 4; ++by) {
+                const uint32_t pr = dequant_pair_attn((word >> (8 * by)) & 0xFFu, sc);
+                const int d0 = 32 * part + 16 * hb + 8 * q + 2 * by;
+                tile[d0 * kVtPitch + key] = (uint16_t)(pr & 0xFFFFu);
+                tile[(d0 + 1) * kVtPitch + key] = (uint16_t)(pr >> 16);
+            }
+        }
+    }
+    __syncthreads();
+    // 128 rows x 64 keys out: thread -> half a row (32 keys, 64 bytes)
+    const int orow = t >> 1, half = t & 1;
+    uint16_t* dst = vt + ((int64_t)h * kD + orow) * Lk + key0 + half * 32;
+    const uint16_t* src = tile + orow * kVtPitch + half * 32;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t q[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) q[u] = (uint32_t)src[8 * i + 2 * u] | ((uint32_t)src[8 * i + 2 * u + 1] << 16);
+        *reinterpret_cast<uint4*>(dst + 8 * i) = make_uint4(q[0], q[1], q[2], q[3]);
+    }
+}
+
 }  // namespace attn
+
+size_t attention_workspace_bytes(int64_t H, int64_t Lk, int64_t d) { return (size_t)(H * d * Lk) * 2; }
 
 cudaError_t launch_attention(const uint8_t* q_codes, const uint8_t* q_sf, const float* g_q, const uint8_t* k_codes,
                              const uint8_t* k_sf, const float* g_k, const uint8_t* v_codes, const uint8_t* v_sf,
                              const float* g_v, const float* s_head, int64_t H, int64_t Lq, int64_t Lk, void* out,
-                             int* dev_status, cudaStream_t stream) {
+                             void* workspace, int* dev_status, cudaStream_t stream) {
     using namespace attn;
-    CUtensorMap tq, tk, tv;
+    uint16_t* vt = static_cast<uint16_t*>(workspace);
+    CUtensorMap tq, tk, tvt;
     if (make_tmap_2d(&tq, q_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kD / 2, (uint64_t)(H * Lq), kD / 2, kD / 2, kBQ,
                      CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
         make_tmap_2d(&tk, k_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kD / 2, (uint64_t)(H * Lk), kD / 2, kD / 2, kBK,
                      CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
-        make_tmap_2d(&tv, v_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kD / 2, (uint64_t)(H * Lk), kD / 2, kD / 2, kBK,
-                     CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+        make_tmap_2d(&tvt, vt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)Lk, (uint64_t)(H * kD),
+                     (uint64_t)Lk * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
+    v_transpose_kernel<<<dim3((unsigned)(Lk / kVtKeys), (unsigned)H), 256, 0, stream>>>(v_codes, v_sf, (int)Lk, vt);
+    count_launch(1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     Params p;
     p.q_sf = q_sf;
     p.k_sf = k_sf;
@@ -484,10 +484,10 @@ cudaError_t launch_attention(const uint8_t* q_codes, const uint8_t* q_sf, const 
     p.Lk = (int)Lk;
     p.H = (int)H;
     p.dev_status = dev_status;
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)(Lq / kBQ), (unsigned)H);
-    attn_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
+    attn_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tvt, p);
     count_launch(1);
     return cudaGetLastError();
 }

@@ -48,7 +48,9 @@ cudaError_t launch_mx_dequantize(const uint8_t* codes, const uint8_t* sf, int64_
 cudaError_t launch_attention(const uint8_t* q_codes, const uint8_t* q_sf, const float* g_q, const uint8_t* k_codes,
                              const uint8_t* k_sf, const float* g_k, const uint8_t* v_codes, const uint8_t* v_sf,
                              const float* g_v, const float* s_head, int64_t H, int64_t Lq, int64_t Lk, void* out,
-                             int* dev_status, cudaStream_t stream);
+                             void* workspace, int* dev_status, cudaStream_t stream);
+
+size_t attention_workspace_bytes(int64_t H, int64_t Lk, int64_t d);
 
 cudaError_t launch_debug_wait_timeout(int* dev_status, uint64_t limit_ns, cudaStream_t stream);
 

@@ -32,7 +32,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 22, names
+    assert len(names) == 23, names
     for n in names:
         assert hasattr(L, n), n
         assert n in _lib.SIGNATURES, n
@@ -227,14 +227,17 @@ def test_block_size_calls(L):
 def test_attention_rejects_bad_arguments(L):
     a = L.nvfp4_attention
     ops = [A, B, C] * 3
-    assert a(*ops, None, 2, 128, 256, 64, A, None, None) == SHAPE          # d != 128
-    assert a(*ops, None, 2, 100, 256, 128, A, None, None) == SHAPE         # Lq % 128
-    assert a(*ops, None, 2, 128, 200, 128, A, None, None) == SHAPE         # Lk % 128
-    assert a(*ops, None, 0, 128, 256, 128, A, None, None) == INVALID
-    assert a(None, B, C, A, B, C, A, B, C, None, 2, 128, 256, 128, A, None, None) == INVALID
-    assert a(*ops, None, 2, 128, 256, 128, None, None, None) == INVALID
-    assert a(A + 8, B, C, A, B, C, A, B, C, None, 2, 128, 256, 128, A, None, None) == MISALIGNED
-    assert a(*ops, C + 2, 2, 128, 256, 128, A, None, None) == MISALIGNED
+    assert a(*ops, None, 2, 128, 256, 64, A, C, 1 << 30, None, None) == SHAPE          # d != 128
+    assert a(*ops, None, 2, 100, 256, 128, A, C, 1 << 30, None, None) == SHAPE         # Lq % 128
+    assert a(*ops, None, 2, 128, 200, 128, A, C, 1 << 30, None, None) == SHAPE         # Lk % 128
+    assert a(*ops, None, 0, 128, 256, 128, A, C, 1 << 30, None, None) == INVALID
+    assert a(None, B, C, A, B, C, A, B, C, None, 2, 128, 256, 128, A, C, 1 << 30, None, None) == INVALID
+    assert a(*ops, None, 2, 128, 256, 128, None, C, 1 << 30, None, None) == INVALID
+    assert a(A + 8, B, C, A, B, C, A, B, C, None, 2, 128, 256, 128, A, C, 1 << 30, None, None) == MISALIGNED
+    assert a(*ops, C + 2, 2, 128, 256, 128, A, C, 1 << 30, None, None) == MISALIGNED
+    assert a(*ops, None, 2, 128, 256, 128, A, C, 100, None, None) == WORKSPACE
+    assert a(*ops, None, 2, 128, 256, 128, A, None, 1 << 30, None, None) == WORKSPACE
+    assert L.nvfp4_attention_workspace_bytes(2, 256, 128) == 2 * 128 * 256 * 2
 
 
 def test_w4a16_rejects_bad_arguments(L):
