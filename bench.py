@@ -239,6 +239,7 @@ def reference_points(dev, layers, w4a16_layers):
     out["mlp_fc1_gelu"] = mlp_fusion_points(dev, layers)
     out["grouped"] = grouped_points(dev)
     out["mx_and_block_size"] = mx_points(dev, layers)
+    out["attention"] = attention_points(dev)
     torch.cuda.empty_cache()
     return out
 
@@ -396,6 +397,30 @@ def mx_points(dev, layers):
         del x, w, A, W, y
     torch.cuda.empty_cache()
     return res
+
+
+def attention_points(dev):
+    """Attention over NVFP4 Q, K, V (Eq. 10) at the video DiT's spatial
+    attention: 16 frames x 24 heads (d = 128) of 2048 tokens each, i.e. 384
+    independent heads; torch's bf16 scaled-dot-product attention on bf16
+    tensors of the same shape as a library reference point."""
+    import torch
+    import nvfp4_w4a4_gemm_quantize_b200 as nv
+    from nvfp4_w4a4_gemm_quantize_b200 import synth
+    H, L, D = 384, 2048, 128
+    xs = [synth.random_bf16((H * L, D), seed=90 + i, dist="normal", device=dev) for i in range(3)]
+    Q, K, V = (nv.quantize(x) for x in xs)
+    o = torch.empty(H * L, D, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(nv.nvfp4_attention_workspace_bytes(H, L, D), dtype=torch.uint8, device=dev)
+    ms = time_device(lambda: nv.attention(Q, K, V, H, out=o, workspace=ws))
+    q4, k4, v4 = (x.view(1, H, L, D) for x in xs)
+    ms_ref = time_device(lambda: torch.nn.functional.scaled_dot_product_attention(q4, k4, v4))
+    fl = 4 * H * L * L * D
+    del xs, Q, K, V, o, ws, q4, k4, v4
+    torch.cuda.empty_cache()
+    return {"shape": f"{H} heads x {L} tokens x d {D}", "ms": round(ms, 4), "tflops": round(fl / (ms * 1e-3) / 1e12, 1),
+            "torch_sdpa_bf16_ms": round(ms_ref, 4),
+            "torch_sdpa_bf16_tflops": round(fl / (ms_ref * 1e-3) / 1e12, 1)}
 
 
 def reduced(wl, args):
