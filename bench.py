@@ -146,31 +146,48 @@ def max_over_ranks(v: float, world: int, device) -> float:
 
 
 # ----------------------------------------------------------------- oracle leg
-def oracle_sample(rows_per_layer: int):
-    """The CPU oracle on a bounded sample of the same step: quantize
-    rows_per_layer rows of every layer input and weight rows and form those
-    rows of Y.  Returns (gemm_flops, seconds, description)."""
+_ORACLE_WEIGHTS = {}
+
+
+def oracle_sample(rows_per_layer: int, col_frac: float = 1.0):
+    """The CPU oracle on a bounded sample of the same step: for every layer,
+    quantize rows_per_layer rows of the input X and form a rows_per_layer x n
+    tile of Y = X W^T, n = col_frac of the layer's output features (a multiple
+    of 128, at least 128), against those weight rows quantized with the whole
+    weight's tensor scale (once per process, untimed).  Returns (gemm_flops,
+    seconds, description)."""
     import numpy as np
     import torch
     import oracle
     from nvfp4_w4a4_gemm_quantize_b200 import synth
     wl = synth.WORKLOADS[WORKLOAD]
-    flops, secs = 0, 0.0
+    flops, secs, cols = 0, 0.0, []
     for i, L in enumerate(wl.layers):
         gen = torch.Generator().manual_seed(wl.seed * 1000 + i)
         x = (torch.randn(rows_per_layer, L.K, generator=gen) *
              torch.exp(torch.empty(rows_per_layer, 1).uniform_(np.log(0.1), np.log(10.0), generator=gen))
              ).to(torch.bfloat16)
-        w = (torch.randn(L.N, L.K, generator=gen) * wl.w_std).to(torch.bfloat16)
-        bc, bsf, gb = oracle.quantize(w)            # weights: quantized once, untimed
+        n = min(L.N, max(128, int(round(col_frac * L.N / 128)) * 128))
+        if (L.name, n) not in _ORACLE_WEIGHTS:
+            if L.name not in _ORACLE_WEIGHTS:
+                wgen = torch.Generator().manual_seed(wl.seed * 1000 + 100 + i)
+                w = (torch.randn(L.N, L.K, generator=wgen) * wl.w_std).to(torch.bfloat16)
+                _ORACLE_WEIGHTS[L.name] = (w, float(oracle.tensor_scale(w)))
+            w, gw = _ORACLE_WEIGHTS[L.name]
+            _ORACLE_WEIGHTS[(L.name, n)] = oracle.quantize(w[:n], gw)
+        bc, bsf, gb = _ORACLE_WEIGHTS[(L.name, n)]
         t0 = time.perf_counter()
         ac, asf, ga = oracle.quantize(x)
         oracle.gemm_w4a4(ac, asf, ga, bc, bsf, gb)
         secs += time.perf_counter() - t0
-        flops += 2 * rows_per_layer * L.N * L.K
-    desc = (f"oracle quantize + FP64 GEMM of {rows_per_layer} activation rows per layer "
-            f"(of {wl.layers[0].M}) for all {len(wl.layers)} {WORKLOAD} layers, 1 thread")
+        flops += 2 * rows_per_layer * n * L.K
+        cols.append(f"{L.name} {n}/{L.N}")
+    desc = (f"oracle quantize + FP64 GEMM of {rows_per_layer} activation rows (of {wl.layers[0].M}) x "
+            f"output features ({', '.join(cols)}) per {WORKLOAD} layer, 1 thread")
     return flops, secs, desc
+
+
+REF_BUDGET_S = 60.0     # CPU seconds the reference arm's timed steps may take in all
 
 
 def run_reference(args):
@@ -178,12 +195,22 @@ def run_reference(args):
     if rank != 0:
         return 0
     rows = args.ref_rows
-    for _ in range(args.warmup):
-        oracle_sample(max(1, rows // 4))
+    # warm-up on a tenth of the output features; the step's cost is close to
+    # proportional to the features sampled, so that sets the fraction that
+    # keeps all K timed steps within the budget
+    probe = 0.1
+    s = 0.0
+    for _ in range(max(1, args.warmup)):
+        _, s, _ = oracle_sample(rows, probe)
+    frac = min(1.0, probe * REF_BUDGET_S / max(1, args.steps) / max(s, 1e-9))
+    min_frac = 128 / 3072                       # one 128-feature tile of the narrowest layer
+    if frac < min_frac:                         # fewer rows once the features cannot shrink
+        rows = max(1, int(rows * frac / min_frac))
+        frac = min_frac
     fl, secs = 0, 0.0
     desc = ""
     for _ in range(args.steps):
-        f, s, desc = oracle_sample(rows)
+        f, s, desc = oracle_sample(rows, frac)
         fl += f
         secs += s
     v = fl / secs / 1e12
@@ -486,11 +513,17 @@ def run_ours(args):
     wl = reduced(synth.WORKLOADS[WORKLOAD], args)
     wl16 = reduced(synth.WORKLOADS["w4a16"], args)
     peaks, peak_src = load_peaks()
-    if args.qat:
-        # profiling aid: only the quantization-aware-training kernels
-        res = qat_points(dev, wl.layers)
+    if args.qat or args.only:
+        # profiling aid: one group of reference points alone
+        groups = {"qat": lambda: qat_points(dev, wl.layers), "mlp": lambda: mlp_fusion_points(dev, wl.layers),
+                  "grouped": lambda: grouped_points(dev), "mx": lambda: mx_points(dev, wl.layers),
+                  "attention": lambda: attention_points(dev)}
+        name = "qat" if args.qat else args.only
+        if name not in groups:
+            raise SystemExit(f"--only: one of {sorted(groups)}")
+        res = groups[name]()
         if rank == 0:
-            print(json.dumps({"qat": res, "peak_gbs": peaks.get("hbm_gbs", FALLBACK["hbm_gbs"]),
+            print(json.dumps({name: res, "peak_gbs": peaks.get("hbm_gbs", FALLBACK["hbm_gbs"]),
                               "peak_source": peak_src}))
         return 0
 
@@ -682,7 +715,7 @@ def run_ours(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-rows", type=int, default=48)
@@ -691,6 +724,8 @@ def main():
     ap.add_argument("--layers", default="", help="profiling: comma-separated subset of layers")
     ap.add_argument("--m", type=int, default=0, help="profiling: tokens (rows of X) per layer")
     ap.add_argument("--qat", action="store_true", help="profiling: time only the QAT kernels (fc1 / fc2 inputs)")
+    ap.add_argument("--only", default="", help="profiling: time one group of reference points "
+                                               "(qat, mlp, grouped, mx, attention)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
