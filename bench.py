@@ -426,7 +426,7 @@ def mx_points(dev, layers):
     return res
 
 
-def attention_points(dev):
+def attention_points(dev, heads=384):
     """Attention over NVFP4 Q, K, V (Eq. 10) at the video DiT's spatial
     attention: 16 frames x 24 heads (d = 128) of 2048 tokens each, i.e. 384
     independent heads; torch's bf16 scaled-dot-product attention on bf16
@@ -434,7 +434,7 @@ def attention_points(dev):
     import torch
     import nvfp4_w4a4_gemm_quantize_b200 as nv
     from nvfp4_w4a4_gemm_quantize_b200 import synth
-    H, L, D = 384, 2048, 128
+    H, L, D = heads, 2048, 128
     xs = [synth.random_bf16((H * L, D), seed=90 + i, dist="normal", device=dev) for i in range(3)]
     Q, K, V = (nv.quantize(x) for x in xs)
     o = torch.empty(H * L, D, dtype=torch.bfloat16, device=dev)
@@ -517,7 +517,7 @@ def run_ours(args):
         # profiling aid: one group of reference points alone
         groups = {"qat": lambda: qat_points(dev, wl.layers), "mlp": lambda: mlp_fusion_points(dev, wl.layers),
                   "grouped": lambda: grouped_points(dev), "mx": lambda: mx_points(dev, wl.layers),
-                  "attention": lambda: attention_points(dev)}
+                  "attention": lambda: attention_points(dev, args.heads or 384)}
         name = "qat" if args.qat else args.only
         if name not in groups:
             raise SystemExit(f"--only: one of {sorted(groups)}")
@@ -724,6 +724,7 @@ def main():
     ap.add_argument("--layers", default="", help="profiling: comma-separated subset of layers")
     ap.add_argument("--m", type=int, default=0, help="profiling: tokens (rows of X) per layer")
     ap.add_argument("--qat", action="store_true", help="profiling: time only the QAT kernels (fc1 / fc2 inputs)")
+    ap.add_argument("--heads", type=int, default=0, help="profiling: attention heads (default 384)")
     ap.add_argument("--only", default="", help="profiling: time one group of reference points "
                                                "(qat, mlp, grouped, mx, attention)")
     args = ap.parse_args()

@@ -19,8 +19,10 @@
 //                 running output is rescaled in TMEM when m moves;
 //     O += P V    bf16 MMA (kind::f16) on TMA-loaded V^T tiles, FP32 in TMEM;
 //     output      O * g_v / l, rounded to bf16.
-// Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 4-7
-// softmax and output; every wait is bounded.
+// Roles: warp 0 loads Q and the K ring, warp 3 the V^T ring; warp 1 owns TMEM
+// and issues S = Q K^T, warp 2 issues O += P V (two issuers, so that neither
+// product waits behind the other's operands); warps 4-7 softmax and output;
+// every wait is bounded.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -38,22 +40,24 @@ constexpr int kD = 128;                      // head dimension
 constexpr int kBQ = 128;                     // queries per CTA
 constexpr int kBK = 128;                     // keys per tile
 constexpr int kThreads = 256;
-constexpr int kStages = 2;                   // K / V code stages
+constexpr int kKStages = 4;                  // K code + scale stages
+constexpr int kVStages = 3;                  // V^T stages
 constexpr int kCodeBytes = kBK * kD / 2;     // 8 KB: 128 rows x 64 bytes
 constexpr int kSfBytes = 1024;               // two 512-byte scale atoms (128 rows x 8 blocks)
+constexpr int kKStageBytes = kCodeBytes + kSfBytes;
 constexpr int kTileBf16 = kBQ * kBK * 2;     // 32 KB: two 64-key chunks of 128 rows x 128 bytes
 constexpr int kChunk = 128 * 128;            // 16 KB
-// stage: K codes (64-byte swizzle), K scales, V^T bf16 tile (128-byte swizzle, 1024-aligned)
-constexpr int kOffStVt = kCodeBytes + kSfBytes;
-constexpr int kStageBytes = kOffStVt + kTileBf16;
 
-// shared memory (offsets from a 1024-aligned base)
+// shared memory (offsets from a 1024-aligned base): Q codes (64-byte swizzle)
+// and scales; the K ring (codes with the 64-byte swizzle, scales); the V^T
+// ring (bf16, 128-byte swizzle); two P tiles (bf16, 128-byte swizzle)
 constexpr int kOffQ = 0;
 constexpr int kOffQsf = kOffQ + kCodeBytes;
-constexpr int kOffStages = kOffQsf + kSfBytes;
-constexpr int kOffP = kOffStages + kStages * kStageBytes;          // 2 P tiles
+constexpr int kOffK = kOffQsf + kSfBytes;
+constexpr int kOffV = kOffK + kKStages * kKStageBytes;
+constexpr int kOffP = kOffV + kVStages * kTileBf16;
 constexpr int kSmemBytes = kOffP + 2 * kTileBf16 + 1024;
-static_assert(kOffStVt % 1024 == 0 && kStageBytes % 1024 == 0 && kOffStages % 1024 == 0 && kOffP % 1024 == 0,
+static_assert(kOffK % 1024 == 0 && kKStageBytes % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0,
               "swizzled tiles are 1024-byte aligned");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
@@ -98,6 +102,7 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+
 // E2M1 code -> value (exact).
 __device__ __forceinline__ float e2m1_val(uint32_t c) {
     const uint32_t e = (c >> 1) & 3u, m = c & 1u;
@@ -135,8 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
             const __grid_constant__ CUtensorMap tmap_vt, const Params p) {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t q_full, kv_full[kStages], kv_empty[kStages];
-    __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_done, drain;
+    __shared__ __align__(8) uint64_t q_full, k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+    __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_done, drain_s, drain_o;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
 
@@ -151,9 +156,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
     if (threadIdx.x == 0) {
         abort_sh = 0;
         mbar_init(&q_full, 1);
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 2);              // the S product's and the PV product's commits
+        for (int s = 0; s < kKStages; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);               // the S product's commit
+        }
+        for (int s = 0; s < kVStages; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);               // the PV product's commit
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
@@ -162,7 +171,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
             mbar_init(&p_empty[b], 1);
         }
         mbar_init(&o_done, 1);
-        mbar_init(&drain, 1);
+        mbar_init(&drain_s, 1);
+        mbar_init(&drain_o, 1);
         fence_barrier_init();
         tma_prefetch_desc(&tmap_q);
         tma_prefetch_desc(&tmap_k);
@@ -179,7 +189,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
 
     if (warp < 4) {
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
+        // ------------------------------------------------------------ Q and K producer
         const uint64_t pol = policy_evict_normal();
         bool ok = true;
         if (elect_one()) {
@@ -189,18 +199,15 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
         }
         __syncwarp();
         for (int j = 0; j < ntiles && ok; ++j) {
-            const int s = j % kStages;
-            const uint32_t ph = (uint32_t)(j / kStages) & 1u;
-            if (!__all_sync(0xffffffffu, mbar_wait(&kv_empty[s], ph ^ 1u, wc) ? 1 : 0)) { ok = false; break; }
-            uint8_t* st = smem + kOffStages + s * kStageBytes;
+            const int s = j % kKStages;
+            const uint32_t ph = (uint32_t)(j / kKStages) & 1u;
+            if (!__all_sync(0xffffffffu, mbar_wait(&k_empty[s], ph ^ 1u, wc) ? 1 : 0)) { ok = false; break; }
+            uint8_t* st = smem + kOffK + s * kKStageBytes;
             const int kr = krow0 + j * kBK;
             if (elect_one()) {
-                mbar_arrive_expect_tx(&kv_full[s], kStageBytes);
-                tma_load_2d(st, &tmap_k, &kv_full[s], 0, kr, pol);
-                bulk_load(st + kCodeBytes, p.k_sf + (int64_t)(kr >> 7) * kSfBytes, kSfBytes, &kv_full[s], pol);
-                // V^T rows h*d .. h*d + 127, keys j*128 .. j*128 + 127, as two 64-key chunks
-                tma_load_2d(st + kOffStVt, &tmap_vt, &kv_full[s], j * kBK, h * kD, pol);
-                tma_load_2d(st + kOffStVt + kChunk, &tmap_vt, &kv_full[s], j * kBK + 64, h * kD, pol);
+                mbar_arrive_expect_tx(&k_full[s], kKStageBytes);
+                tma_load_2d(st, &tmap_k, &k_full[s], 0, kr, pol);
+                bulk_load(st + kCodeBytes, p.k_sf + (int64_t)(kr >> 7) * kSfBytes, kSfBytes, &k_full[s], pol);
             }
             __syncwarp();
         }
@@ -209,13 +216,35 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
             int dummy = 0;
             WaitCtx w2{&dummy, p.dev_status};
             mbar_wait(&q_full, 0, w2);
-            for (int j = (ntiles > kStages ? ntiles - kStages : 0); j < ntiles; ++j)
-                mbar_wait(&kv_full[j % kStages], (uint32_t)(j / kStages) & 1u, w2);
+            for (int j = (ntiles > kKStages ? ntiles - kKStages : 0); j < ntiles; ++j)
+                mbar_wait(&k_full[j % kKStages], (uint32_t)(j / kKStages) & 1u, w2);
+        }
+    } else if (warp == 3) {
+        // ------------------------------------------------------------ V^T producer
+        const uint64_t pol = policy_evict_normal();
+        bool ok = true;
+        for (int j = 0; j < ntiles && ok; ++j) {
+            const int s = j % kVStages;
+            const uint32_t ph = (uint32_t)(j / kVStages) & 1u;
+            if (!__all_sync(0xffffffffu, mbar_wait(&v_empty[s], ph ^ 1u, wc) ? 1 : 0)) { ok = false; break; }
+            uint8_t* st = smem + kOffV + s * kTileBf16;
+            if (elect_one()) {
+                // V^T rows h*d .. h*d + 127, keys j*128 .. j*128 + 127, as two 64-key chunks
+                mbar_arrive_expect_tx(&v_full[s], kTileBf16);
+                tma_load_2d(st, &tmap_vt, &v_full[s], j * kBK, h * kD, pol);
+                tma_load_2d(st + kChunk, &tmap_vt, &v_full[s], j * kBK + 64, h * kD, pol);
+            }
+            __syncwarp();
+        }
+        if (lane == 0) {
+            int dummy = 0;
+            WaitCtx w2{&dummy, p.dev_status};
+            for (int j = (ntiles > kVStages ? ntiles - kVStages : 0); j < ntiles; ++j)
+                mbar_wait(&v_full[j % kVStages], (uint32_t)(j / kVStages) & 1u, w2);
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+        // ------------------------------------------------------------ S = Q K^T issuer (and TMEM owner)
         constexpr uint32_t idesc_s = idesc_nvf4(kBQ, kBK);
-        constexpr uint32_t idesc_o = idesc_bf16(kBQ, kD);
         const uint32_t sm0 = smem_u32(smem);
         bool ok = __all_sync(0xffffffffu, mbar_wait(&q_full, 0, wc) ? 1 : 0);
         if (ok) {
@@ -226,60 +255,68 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
             }
             __syncwarp();
         }
-        // S_j is issued one tile ahead of O += P_{j-1} V_{j-1}
-        for (int j = 0; j <= ntiles && ok; ++j) {
-            if (j < ntiles) {
-                const int s = j % kStages, b = j & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&kv_full[s], (uint32_t)(j / kStages) & 1u, wc) ? 1 : 0) ||
-                    !__all_sync(0xffffffffu, mbar_wait(&s_empty[b], ((uint32_t)(j >> 1) & 1u) ^ 1u, wc) ? 1 : 0)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t st = sm0 + kOffStages + s * kStageBytes;
-                const uint32_t sfk = tmem + kColSfK + b * 8;
-                if (elect_one()) {
-                    tc_cp_32x128b_warpx4(sfk, sdesc_sf(st + kCodeBytes));
-                    tc_cp_32x128b_warpx4(sfk + 4, sdesc_sf(st + kCodeBytes + 512));
-#pragma unroll
-                    for (int ks = 0; ks < 2; ++ks)
-                        tc_mma_nvf4(tmem + kColS + b * kBK, sdesc_kmajor_sw64(sm0 + kOffQ + ks * 32),
-                                    sdesc_kmajor_sw64(st + ks * 32), idesc_s, tmem + kColSfQ + ks * 4,
-                                    sfk + ks * 4, ks != 0 ? 1u : 0u);
-                    tc_commit(&s_full[b]);
-                    tc_commit(&kv_empty[s]);
-                }
-                __syncwarp();
+        for (int j = 0; j < ntiles && ok; ++j) {
+            const int s = j % kKStages, b = j & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&k_full[s], (uint32_t)(j / kKStages) & 1u, wc) ? 1 : 0) ||
+                !__all_sync(0xffffffffu, mbar_wait(&s_empty[b], ((uint32_t)(j >> 1) & 1u) ^ 1u, wc) ? 1 : 0)) {
+                ok = false;
+                break;
             }
-            if (j >= 1) {
-                const int jp = j - 1, s = jp % kStages, b = jp & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&p_full[b], (uint32_t)(jp >> 1) & 1u, wc) ? 1 : 0)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t pt = sm0 + kOffP + b * kTileBf16;
-                const uint32_t vt = sm0 + kOffStages + s * kStageBytes + kOffStVt;
-                if (elect_one()) {
+            tc_fence_after();
+            const uint32_t st = sm0 + kOffK + s * kKStageBytes;
+            const uint32_t sfk = tmem + kColSfK + b * 8;
+            if (elect_one()) {
+                tc_cp_32x128b_warpx4(sfk, sdesc_sf(st + kCodeBytes));
+                tc_cp_32x128b_warpx4(sfk + 4, sdesc_sf(st + kCodeBytes + 512));
 #pragma unroll
-                    for (int kc = 0; kc < 2; ++kc)
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            tc_mma_bf16(tmem + kColO, sdesc_kmajor_sw128(pt + kc * kChunk + ks * 32),
-                                        sdesc_kmajor_sw128(vt + kc * kChunk + ks * 32), idesc_o,
-                                        (jp | kc | ks) != 0 ? 1u : 0u);
-                    tc_commit(&p_empty[b]);
-                    tc_commit(&kv_empty[s]);
-                    tc_commit(&o_done);
-                }
-                __syncwarp();
+                for (int ks = 0; ks < 2; ++ks)
+                    tc_mma_nvf4(tmem + kColS + b * kBK, sdesc_kmajor_sw64(sm0 + kOffQ + ks * 32),
+                                sdesc_kmajor_sw64(st + ks * 32), idesc_s, tmem + kColSfQ + ks * 4, sfk + ks * 4,
+                                ks != 0 ? 1u : 0u);
+                tc_commit(&s_full[b]);
+                tc_commit(&k_empty[s]);
             }
+            __syncwarp();
         }
-        if (elect_one()) tc_commit(&drain);
+        if (elect_one()) tc_commit(&drain_s);
         __syncwarp();
         int dummy = 0;
         WaitCtx w2{&dummy, p.dev_status};
-        mbar_wait(&drain, 0, w2);
+        mbar_wait(&drain_s, 0, w2);
+    } else {
+        // ------------------------------------------------------------ O += P V issuer
+        constexpr uint32_t idesc_o = idesc_bf16(kBQ, kD);
+        const uint32_t sm0 = smem_u32(smem);
+        bool ok = true;
+        for (int j = 0; j < ntiles && ok; ++j) {
+            const int s = j % kVStages, b = j & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&p_full[b], (uint32_t)(j >> 1) & 1u, wc) ? 1 : 0) ||
+                !__all_sync(0xffffffffu, mbar_wait(&v_full[s], (uint32_t)(j / kVStages) & 1u, wc) ? 1 : 0)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t pt = sm0 + kOffP + b * kTileBf16;
+            const uint32_t vt = sm0 + kOffV + s * kTileBf16;
+            if (elect_one()) {
+#pragma unroll
+                for (int kc = 0; kc < 2; ++kc)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        tc_mma_bf16(tmem + kColO, sdesc_kmajor_sw128(pt + kc * kChunk + ks * 32),
+                                    sdesc_kmajor_sw128(vt + kc * kChunk + ks * 32), idesc_o,
+                                    (j | kc | ks) != 0 ? 1u : 0u);
+                tc_commit(&p_empty[b]);
+                tc_commit(&v_empty[s]);
+                tc_commit(&o_done);
+            }
+            __syncwarp();
+        }
+        if (elect_one()) tc_commit(&drain_o);
+        __syncwarp();
+        int dummy = 0;
+        WaitCtx w2{&dummy, p.dev_status};
+        mbar_wait(&drain_o, 0, w2);
     }
     } else {
         // ------------------------------------------------------------ softmax and output
@@ -304,20 +341,25 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_empty[b]);
-            float mt = -INFINITY;
+            // eight independent running maxima: short dependency chains
+            float mx8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
 #pragma unroll
             for (int i = 0; i < kBK; ++i) {
                 const float z = fmaf(__uint_as_float(v[i]), c, bias);
                 v[i] = __float_as_uint(z);
-                mt = fmaxf(mt, z);
+                mx8[i & 7] = fmaxf(mx8[i & 7], z);
             }
+            const float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             // lazy rescaling: the reference maximum moves only when the tile's
             // maximum exceeds it by more than 8 (p stays below 2^8); O and l are
             // rescaled then, and share the reference
             const bool move = mt > m + 8.0f;
             const float mref = move ? mt : m;
             const float alpha = move ? ex2(m - mt) : 1.0f;          // 0 on the first tile (m = -inf)
-            float sum = 0.0f;
+            float sum4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             // P tile reuse: the product that read this buffer two tiles ago is done
             if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&p_empty[b], ((uint32_t)(j >> 1) & 1u) ^ 1u, wc) ? 1 : 0)) {
                 ok = false;
@@ -330,9 +372,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
                 uint32_t w[4];
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
-                    const float e0 = ex2(__uint_as_float(v[c8 * 8 + 2 * t]) - mref);
-                    const float e1 = ex2(__uint_as_float(v[c8 * 8 + 2 * t + 1]) - mref);
-                    sum += e0 + e1;
+                    const float x0 = __uint_as_float(v[c8 * 8 + 2 * t]) - mref;
+                    const float x1 = __uint_as_float(v[c8 * 8 + 2 * t + 1]) - mref;
+                    const float e0 = ex2(x0);
+                    const float e1 = ex2(x1);
+                    sum4[t] += e0 + e1;
                     __nv_bfloat162 hb = __floats2bfloat162_rn(e0, e1);
                     w[t] = *reinterpret_cast<uint32_t*>(&hb);
                 }
@@ -340,7 +384,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
                 *reinterpret_cast<uint4*>(prow + kc * kChunk + pos * 16) = make_uint4(w[0], w[1], w[2], w[3]);
             }
             const float mt_used = mref;
-            l = fmaf(l, alpha, sum);
+            l = fmaf(l, alpha, (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
             m = mt_used;
             // rescale the running output by alpha once the previous product is done
             if (j >= 1) {
