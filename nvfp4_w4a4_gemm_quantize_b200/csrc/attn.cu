@@ -10,7 +10,8 @@
 //                 significant bits) and transposed to V^T [H*d, Lk] in the
 //                 caller's workspace -- once per call, instead of once per
 //                 query tile;
-//   attention     per CTA 128 queries of one head, keys in tiles of 128:
+//   attention     persistent, one CTA per SM; a work item is 128 queries of
+//                 one head, keys in tiles of 128:
 //     S = Q K^T   block-scaled FP4 MMA (kind::mxf4nvf4, K = d), FP32 in TMEM,
 //                 two S buffers so the next tile's product overlaps softmax;
 //     softmax     one query row per thread (online: reference maximum m, sum
@@ -48,12 +49,12 @@ constexpr int kKStageBytes = kCodeBytes + kSfBytes;
 constexpr int kTileBf16 = kBQ * kBK * 2;     // 32 KB: two 64-key chunks of 128 rows x 128 bytes
 constexpr int kChunk = 128 * 128;            // 16 KB
 
-// shared memory (offsets from a 1024-aligned base): Q codes (64-byte swizzle)
-// and scales; the K ring (codes with the 64-byte swizzle, scales); the V^T
+// shared memory (offsets from a 1024-aligned base): two Q buffers (codes with
+// the 64-byte swizzle, scales), so that the next work item's Q lands while
+// this one runs; the K ring (codes with the 64-byte swizzle, scales); the V^T
 // ring (bf16, 128-byte swizzle); two P tiles (bf16, 128-byte swizzle)
-constexpr int kOffQ = 0;
-constexpr int kOffQsf = kOffQ + kCodeBytes;
-constexpr int kOffK = kOffQsf + kSfBytes;
+constexpr int kOffQ = 0;                     // + qb * kKStageBytes
+constexpr int kOffK = 2 * kKStageBytes;
 constexpr int kOffV = kOffK + kKStages * kKStageBytes;
 constexpr int kOffP = kOffV + kVStages * kTileBf16;
 constexpr int kSmemBytes = kOffP + 2 * kTileBf16 + 1024;
@@ -64,8 +65,8 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 // TMEM columns
 constexpr uint32_t kColS = 0;                // two S buffers: [0,128), [128,256)
 constexpr uint32_t kColO = 256;              // O: [256, 384)
-constexpr uint32_t kColSfQ = 384;            // Q scales: 2 K-steps x 4 columns
-constexpr uint32_t kColSfK = 392;            // K scales per S buffer: 2 x (2 x 4)
+constexpr uint32_t kColSfQ = 384;            // Q scales per Q buffer: 2 x (2 K-steps x 4 columns)
+constexpr uint32_t kColSfK = 400;            // K scales per S buffer: 2 x (2 x 4)
 
 struct Params {
     const uint8_t* q_sf;
@@ -102,7 +103,6 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-
 // E2M1 code -> value (exact).
 __device__ __forceinline__ float e2m1_val(uint32_t c) {
     const uint32_t e = (c >> 1) & 3u, m = c & 1u;
@@ -136,26 +136,37 @@ __device__ __forceinline__ uint32_t e4m3_to_b2_scaled_attn(uint32_t code) {
 // Byte of (row r, 16-value block c) inside a 128-row group's two scale atoms.
 __device__ __forceinline__ int sf_byte(int r, int c) { return (c >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (c & 3); }
 
+// Persistent: CTA c takes work items (head, 128-query tile) c, c + grid, ...
+// Key tiles carry one running number n over all of a CTA's items, which
+// selects ring slots, S / P buffers and barrier phases, so every pipeline
+// stays full across item boundaries: the next item's Q, K and S go ahead
+// while this item's last products and output finish.
 __global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
             const __grid_constant__ CUtensorMap tmap_vt, const Params p) {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t q_full, k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
-    __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_done, drain_s, drain_o;
+    __shared__ __align__(8) uint64_t q_full[2], q_empty[2], k_full[kKStages], k_empty[kKStages];
+    __shared__ __align__(8) uint64_t v_full[kVStages], v_empty[kVStages];
+    __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_done, o_free, drain_s, drain_o;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     WaitCtx wc{&abort_sh, p.dev_status};
-    const int h = blockIdx.y;
-    const int qrow0 = h * p.Lq + blockIdx.x * kBQ;          // first query row of this CTA
-    const int krow0 = h * p.Lk;
     const int ntiles = p.Lk / kBK;
+    const int qtiles = p.Lq / kBQ;
+    const int nitems = p.H * qtiles;
+    // item -> head and first query row
+    auto item_head = [&](int it) { return it / qtiles; };
+    auto item_qrow = [&](int it) { return (it / qtiles) * p.Lq + (it % qtiles) * kBQ; };
 
     if (threadIdx.x == 0) {
         abort_sh = 0;
-        mbar_init(&q_full, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&q_full[b], 1);
+            mbar_init(&q_empty[b], 1);               // the item's last S product's commit
+        }
         for (int s = 0; s < kKStages; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);               // the S product's commit
@@ -171,6 +182,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
             mbar_init(&p_empty[b], 1);
         }
         mbar_init(&o_done, 1);
+        mbar_init(&o_free, 4);                       // the softmax warps have read O out
         mbar_init(&drain_s, 1);
         mbar_init(&drain_o, 1);
         fence_barrier_init();
@@ -192,91 +204,112 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
         // ------------------------------------------------------------ Q and K producer
         const uint64_t pol = policy_evict_normal();
         bool ok = true;
-        if (elect_one()) {
-            mbar_arrive_expect_tx(&q_full, kCodeBytes + kSfBytes);
-            tma_load_2d(smem + kOffQ, &tmap_q, &q_full, 0, qrow0, pol);
-            bulk_load(smem + kOffQsf, p.q_sf + (int64_t)(qrow0 >> 7) * kSfBytes, kSfBytes, &q_full, pol);
-        }
-        __syncwarp();
-        for (int j = 0; j < ntiles && ok; ++j) {
-            const int s = j % kKStages;
-            const uint32_t ph = (uint32_t)(j / kKStages) & 1u;
-            if (!__all_sync(0xffffffffu, mbar_wait(&k_empty[s], ph ^ 1u, wc) ? 1 : 0)) { ok = false; break; }
-            uint8_t* st = smem + kOffK + s * kKStageBytes;
-            const int kr = krow0 + j * kBK;
+        int n = 0, i = 0;
+        for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++i) {
+            const int qb = i & 1, qrow0 = item_qrow(it), krow0 = item_head(it) * p.Lk;
+            if (!__all_sync(0xffffffffu, mbar_wait(&q_empty[qb], ((uint32_t)(i >> 1) & 1u) ^ 1u, wc) ? 1 : 0)) {
+                ok = false;
+                break;
+            }
             if (elect_one()) {
-                mbar_arrive_expect_tx(&k_full[s], kKStageBytes);
-                tma_load_2d(st, &tmap_k, &k_full[s], 0, kr, pol);
-                bulk_load(st + kCodeBytes, p.k_sf + (int64_t)(kr >> 7) * kSfBytes, kSfBytes, &k_full[s], pol);
+                uint8_t* qs = smem + kOffQ + qb * kKStageBytes;
+                mbar_arrive_expect_tx(&q_full[qb], kKStageBytes);
+                tma_load_2d(qs, &tmap_q, &q_full[qb], 0, qrow0, pol);
+                bulk_load(qs + kCodeBytes, p.q_sf + (int64_t)(qrow0 >> 7) * kSfBytes, kSfBytes, &q_full[qb], pol);
             }
             __syncwarp();
+            for (int j = 0; j < ntiles; ++j, ++n) {
+                const int s = n % kKStages;
+                const uint32_t ph = (uint32_t)(n / kKStages) & 1u;
+                if (!__all_sync(0xffffffffu, mbar_wait(&k_empty[s], ph ^ 1u, wc) ? 1 : 0)) { ok = false; break; }
+                uint8_t* st = smem + kOffK + s * kKStageBytes;
+                const int kr = krow0 + j * kBK;
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(&k_full[s], kKStageBytes);
+                    tma_load_2d(st, &tmap_k, &k_full[s], 0, kr, pol);
+                    bulk_load(st + kCodeBytes, p.k_sf + (int64_t)(kr >> 7) * kSfBytes, kSfBytes, &k_full[s], pol);
+                }
+                __syncwarp();
+            }
         }
         // every load this warp issued has landed before the CTA may exit
         if (lane == 0) {
             int dummy = 0;
             WaitCtx w2{&dummy, p.dev_status};
-            mbar_wait(&q_full, 0, w2);
-            for (int j = (ntiles > kKStages ? ntiles - kKStages : 0); j < ntiles; ++j)
-                mbar_wait(&k_full[j % kKStages], (uint32_t)(j / kKStages) & 1u, w2);
+            for (int q = (i > 2 ? i - 2 : 0); q < i; ++q) mbar_wait(&q_full[q & 1], (uint32_t)(q >> 1) & 1u, w2);
+            for (int m = (n > kKStages ? n - kKStages : 0); m < n; ++m)
+                mbar_wait(&k_full[m % kKStages], (uint32_t)(m / kKStages) & 1u, w2);
         }
     } else if (warp == 3) {
         // ------------------------------------------------------------ V^T producer
         const uint64_t pol = policy_evict_normal();
         bool ok = true;
-        for (int j = 0; j < ntiles && ok; ++j) {
-            const int s = j % kVStages;
-            const uint32_t ph = (uint32_t)(j / kVStages) & 1u;
-            if (!__all_sync(0xffffffffu, mbar_wait(&v_empty[s], ph ^ 1u, wc) ? 1 : 0)) { ok = false; break; }
-            uint8_t* st = smem + kOffV + s * kTileBf16;
-            if (elect_one()) {
-                // V^T rows h*d .. h*d + 127, keys j*128 .. j*128 + 127, as two 64-key chunks
-                mbar_arrive_expect_tx(&v_full[s], kTileBf16);
-                tma_load_2d(st, &tmap_vt, &v_full[s], j * kBK, h * kD, pol);
-                tma_load_2d(st + kChunk, &tmap_vt, &v_full[s], j * kBK + 64, h * kD, pol);
+        int n = 0;
+        for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+            const int h = item_head(it);
+            for (int j = 0; j < ntiles; ++j, ++n) {
+                const int s = n % kVStages;
+                const uint32_t ph = (uint32_t)(n / kVStages) & 1u;
+                if (!__all_sync(0xffffffffu, mbar_wait(&v_empty[s], ph ^ 1u, wc) ? 1 : 0)) { ok = false; break; }
+                uint8_t* st = smem + kOffV + s * kTileBf16;
+                if (elect_one()) {
+                    // V^T rows h*d .. h*d + 127, keys j*128 .. j*128 + 127, as two 64-key chunks
+                    mbar_arrive_expect_tx(&v_full[s], kTileBf16);
+                    tma_load_2d(st, &tmap_vt, &v_full[s], j * kBK, h * kD, pol);
+                    tma_load_2d(st + kChunk, &tmap_vt, &v_full[s], j * kBK + 64, h * kD, pol);
+                }
+                __syncwarp();
             }
-            __syncwarp();
         }
         if (lane == 0) {
             int dummy = 0;
             WaitCtx w2{&dummy, p.dev_status};
-            for (int j = (ntiles > kVStages ? ntiles - kVStages : 0); j < ntiles; ++j)
-                mbar_wait(&v_full[j % kVStages], (uint32_t)(j / kVStages) & 1u, w2);
+            for (int m = (n > kVStages ? n - kVStages : 0); m < n; ++m)
+                mbar_wait(&v_full[m % kVStages], (uint32_t)(m / kVStages) & 1u, w2);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ S = Q K^T issuer (and TMEM owner)
         constexpr uint32_t idesc_s = idesc_nvf4(kBQ, kBK);
         const uint32_t sm0 = smem_u32(smem);
-        bool ok = __all_sync(0xffffffffu, mbar_wait(&q_full, 0, wc) ? 1 : 0);
-        if (ok) {
-            tc_fence_after();
-            if (elect_one()) {
-                tc_cp_32x128b_warpx4(tmem + kColSfQ, sdesc_sf(sm0 + kOffQsf));
-                tc_cp_32x128b_warpx4(tmem + kColSfQ + 4, sdesc_sf(sm0 + kOffQsf + 512));
-            }
-            __syncwarp();
-        }
-        for (int j = 0; j < ntiles && ok; ++j) {
-            const int s = j % kKStages, b = j & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&k_full[s], (uint32_t)(j / kKStages) & 1u, wc) ? 1 : 0) ||
-                !__all_sync(0xffffffffu, mbar_wait(&s_empty[b], ((uint32_t)(j >> 1) & 1u) ^ 1u, wc) ? 1 : 0)) {
+        bool ok = true;
+        int n = 0, i = 0;
+        for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++i) {
+            const int qb = i & 1;
+            const uint32_t qs = sm0 + kOffQ + qb * kKStageBytes, sfq = tmem + kColSfQ + qb * 8;
+            if (!__all_sync(0xffffffffu, mbar_wait(&q_full[qb], (uint32_t)(i >> 1) & 1u, wc) ? 1 : 0)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t st = sm0 + kOffK + s * kKStageBytes;
-            const uint32_t sfk = tmem + kColSfK + b * 8;
             if (elect_one()) {
-                tc_cp_32x128b_warpx4(sfk, sdesc_sf(st + kCodeBytes));
-                tc_cp_32x128b_warpx4(sfk + 4, sdesc_sf(st + kCodeBytes + 512));
-#pragma unroll
-                for (int ks = 0; ks < 2; ++ks)
-                    tc_mma_nvf4(tmem + kColS + b * kBK, sdesc_kmajor_sw64(sm0 + kOffQ + ks * 32),
-                                sdesc_kmajor_sw64(st + ks * 32), idesc_s, tmem + kColSfQ + ks * 4, sfk + ks * 4,
-                                ks != 0 ? 1u : 0u);
-                tc_commit(&s_full[b]);
-                tc_commit(&k_empty[s]);
+                tc_cp_32x128b_warpx4(sfq, sdesc_sf(qs + kCodeBytes));
+                tc_cp_32x128b_warpx4(sfq + 4, sdesc_sf(qs + kCodeBytes + 512));
             }
             __syncwarp();
+            for (int j = 0; j < ntiles; ++j, ++n) {
+                const int s = n % kKStages, b = n & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&k_full[s], (uint32_t)(n / kKStages) & 1u, wc) ? 1 : 0) ||
+                    !__all_sync(0xffffffffu, mbar_wait(&s_empty[b], ((uint32_t)(n >> 1) & 1u) ^ 1u, wc) ? 1 : 0)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t st = sm0 + kOffK + s * kKStageBytes;
+                const uint32_t sfk = tmem + kColSfK + b * 8;
+                if (elect_one()) {
+                    tc_cp_32x128b_warpx4(sfk, sdesc_sf(st + kCodeBytes));
+                    tc_cp_32x128b_warpx4(sfk + 4, sdesc_sf(st + kCodeBytes + 512));
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)
+                        tc_mma_nvf4(tmem + kColS + b * kBK, sdesc_kmajor_sw64(qs + ks * 32),
+                                    sdesc_kmajor_sw64(st + ks * 32), idesc_s, sfq + ks * 4, sfk + ks * 4,
+                                    ks != 0 ? 1u : 0u);
+                    tc_commit(&s_full[b]);
+                    tc_commit(&k_empty[s]);
+                    if (j == ntiles - 1) tc_commit(&q_empty[qb]);
+                }
+                __syncwarp();
+            }
         }
         if (elect_one()) tc_commit(&drain_s);
         __syncwarp();
@@ -288,29 +321,35 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
         constexpr uint32_t idesc_o = idesc_bf16(kBQ, kD);
         const uint32_t sm0 = smem_u32(smem);
         bool ok = true;
-        for (int j = 0; j < ntiles && ok; ++j) {
-            const int s = j % kVStages, b = j & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&p_full[b], (uint32_t)(j >> 1) & 1u, wc) ? 1 : 0) ||
-                !__all_sync(0xffffffffu, mbar_wait(&v_full[s], (uint32_t)(j / kVStages) & 1u, wc) ? 1 : 0)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t pt = sm0 + kOffP + b * kTileBf16;
-            const uint32_t vt = sm0 + kOffV + s * kTileBf16;
-            if (elect_one()) {
+        int n = 0, i = 0;
+        for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++i) {
+            for (int j = 0; j < ntiles; ++j, ++n) {
+                const int s = n % kVStages, b = n & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&p_full[b], (uint32_t)(n >> 1) & 1u, wc) ? 1 : 0) ||
+                    !__all_sync(0xffffffffu, mbar_wait(&v_full[s], (uint32_t)(n / kVStages) & 1u, wc) ? 1 : 0) ||
+                    // the first product of an item overwrites O: the previous item's O has been read out
+                    (j == 0 && i >= 1 &&
+                     !__all_sync(0xffffffffu, mbar_wait(&o_free, (uint32_t)(i - 1) & 1u, wc) ? 1 : 0))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t pt = sm0 + kOffP + b * kTileBf16;
+                const uint32_t vt = sm0 + kOffV + s * kTileBf16;
+                if (elect_one()) {
 #pragma unroll
-                for (int kc = 0; kc < 2; ++kc)
+                    for (int kc = 0; kc < 2; ++kc)
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        tc_mma_bf16(tmem + kColO, sdesc_kmajor_sw128(pt + kc * kChunk + ks * 32),
-                                    sdesc_kmajor_sw128(vt + kc * kChunk + ks * 32), idesc_o,
-                                    (j | kc | ks) != 0 ? 1u : 0u);
-                tc_commit(&p_empty[b]);
-                tc_commit(&v_empty[s]);
-                tc_commit(&o_done);
+                        for (int ks = 0; ks < 4; ++ks)
+                            tc_mma_bf16(tmem + kColO, sdesc_kmajor_sw128(pt + kc * kChunk + ks * 32),
+                                        sdesc_kmajor_sw128(vt + kc * kChunk + ks * 32), idesc_o,
+                                        (j | kc | ks) != 0 ? 1u : 0u);
+                    tc_commit(&p_empty[b]);
+                    tc_commit(&v_empty[s]);
+                    tc_commit(&o_done);
+                }
+                __syncwarp();
             }
-            __syncwarp();
         }
         if (elect_one()) tc_commit(&drain_o);
         __syncwarp();
@@ -322,113 +361,126 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
         // ------------------------------------------------------------ softmax and output
         const int q = warp & 3;                     // TMEM lane quarter
         const int r = q * 32 + lane;                // query row in the tile
+        // z = s c + bias: the logit in base 2 (c > 0, so the tile maximum of z
+        // is c times that of s, plus bias)
         const float c = __fmul_rn(__fmul_rn(*p.g_q, *p.g_k), 1.4426950408889634f / 11.313708498984761f);
-        const float bias = p.s_head ? log2f(p.s_head[h]) : 0.0f;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        float m = -INFINITY, l = 0.0f;
         bool ok = true;
-        for (int j = 0; j < ntiles && ok; ++j) {
-            const int b = j & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[b], (uint32_t)(j >> 1) & 1u, wc) ? 1 : 0)) { ok = false; break; }
-            tc_fence_after();
-            // the tile's 128 logits of this row, in registers (one TMEM wait)
-            uint32_t v[kBK];
+        int n = 0;
+        for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+            const float bias = p.s_head ? log2f(p.s_head[item_head(it)]) : 0.0f;
+            float m = -INFINITY, l = 0.0f;
+            for (int j = 0; j < ntiles; ++j, ++n) {
+                const int b = n & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&s_full[b], (uint32_t)(n >> 1) & 1u, wc) ? 1 : 0)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                // the tile's 128 logits of this row, in registers (one TMEM wait)
+                uint32_t v[kBK];
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4)
-                tmem_ld_32x32b_x32(tmem + lane_base + kColS + b * kBK + c4 * 32,
-                                   *reinterpret_cast<uint32_t(*)[32]>(&v[c4 * 32]));
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_empty[b]);
-            // eight independent running maxima: short dependency chains
-            float mx8[8];
+                for (int c4 = 0; c4 < 4; ++c4)
+                    tmem_ld_32x32b_x32(tmem + lane_base + kColS + b * kBK + c4 * 32,
+                                       *reinterpret_cast<uint32_t(*)[32]>(&v[c4 * 32]));
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_empty[b]);
+                // eight independent running maxima of s: short dependency chains
+                float mx8[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+                for (int i8 = 0; i8 < 8; ++i8) mx8[i8] = -INFINITY;
 #pragma unroll
-            for (int i = 0; i < kBK; ++i) {
-                const float z = fmaf(__uint_as_float(v[i]), c, bias);
-                v[i] = __float_as_uint(z);
-                mx8[i & 7] = fmaxf(mx8[i & 7], z);
+                for (int i8 = 0; i8 < kBK; ++i8) mx8[i8 & 7] = fmaxf(mx8[i8 & 7], __uint_as_float(v[i8]));
+                const float smax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                const float mt = fmaf(smax, c, bias);
+                // lazy rescaling: the reference maximum moves only when the tile's
+                // maximum exceeds it by more than 8 (p stays below 2^8); O and l are
+                // rescaled then, and share the reference
+                const bool move = mt > m + 8.0f;
+                const float mref = move ? mt : m;
+                const float alpha = move ? ex2(m - mt) : 1.0f;          // 0 on the first tile (m = -inf)
+                const float off = bias - mref;                          // exponent: s c + (bias - mref)
+                float sum4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                // P tile reuse: the product that read this buffer two tiles ago is done
+                if (n >= 2 &&
+                    !__all_sync(0xffffffffu, mbar_wait(&p_empty[b], ((uint32_t)(n >> 1) & 1u) ^ 1u, wc) ? 1 : 0)) {
+                    ok = false;
+                    break;
+                }
+                // p = exp2(s c + bias - mref), rounded to bf16 into the swizzled K-major P tile
+                uint8_t* prow = smem + kOffP + b * kTileBf16 + r * 128;
+#pragma unroll
+                for (int c8 = 0; c8 < 16; ++c8) {              // 8 keys per 16-byte unit
+                    uint32_t w[4];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const float e0 = ex2(fmaf(__uint_as_float(v[c8 * 8 + 2 * t]), c, off));
+                        const float e1 = ex2(fmaf(__uint_as_float(v[c8 * 8 + 2 * t + 1]), c, off));
+                        sum4[t] += e0 + e1;
+                        __nv_bfloat162 hb = __floats2bfloat162_rn(e0, e1);
+                        w[t] = *reinterpret_cast<uint32_t*>(&hb);
+                    }
+                    const int kc = c8 >> 3, pos = (c8 & 7) ^ (r & 7);
+                    *reinterpret_cast<uint4*>(prow + kc * kChunk + pos * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+                l = fmaf(l, alpha, (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+                m = mref;
+                // rescale the running output by alpha once the previous product is done
+                if (j >= 1) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&o_done, (uint32_t)(n - 1) & 1u, wc) ? 1 : 0)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4) {
+                            uint32_t o[32];
+                            tmem_ld_32x32b_x32(tmem + lane_base + kColO + c4 * 32, o);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int i8 = 0; i8 < 32; ++i8) o[i8] = __float_as_uint(__uint_as_float(o[i8]) * alpha);
+                            tmem_st_x32(tmem + lane_base + kColO + c4 * 32, o);
+                        }
+                        tmem_st_wait();
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[b]);
             }
-            const float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-            // lazy rescaling: the reference maximum moves only when the tile's
-            // maximum exceeds it by more than 8 (p stays below 2^8); O and l are
-            // rescaled then, and share the reference
-            const bool move = mt > m + 8.0f;
-            const float mref = move ? mt : m;
-            const float alpha = move ? ex2(m - mt) : 1.0f;          // 0 on the first tile (m = -inf)
-            float sum4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            // P tile reuse: the product that read this buffer two tiles ago is done
-            if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&p_empty[b], ((uint32_t)(j >> 1) & 1u) ^ 1u, wc) ? 1 : 0)) {
+            if (!ok) break;
+            // output: O * g_v / l, once the item's last product is done; O is
+            // read into registers and released before the global stores
+            if (!__all_sync(0xffffffffu, mbar_wait(&o_done, (uint32_t)(n - 1) & 1u, wc) ? 1 : 0)) {
                 ok = false;
                 break;
             }
-            // p = exp2(z - mref), rounded to bf16 into the swizzled K-major P tile
-            uint8_t* prow = smem + kOffP + b * kTileBf16 + r * 128;
+            tc_fence_after();
+            uint32_t o[kD];
 #pragma unroll
-            for (int c8 = 0; c8 < 16; ++c8) {              // 8 keys per 16-byte unit
-                uint32_t w[4];
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const float x0 = __uint_as_float(v[c8 * 8 + 2 * t]) - mref;
-                    const float x1 = __uint_as_float(v[c8 * 8 + 2 * t + 1]) - mref;
-                    const float e0 = ex2(x0);
-                    const float e1 = ex2(x1);
-                    sum4[t] += e0 + e1;
-                    __nv_bfloat162 hb = __floats2bfloat162_rn(e0, e1);
-                    w[t] = *reinterpret_cast<uint32_t*>(&hb);
-                }
-                const int kc = c8 >> 3, pos = (c8 & 7) ^ (r & 7);
-                *reinterpret_cast<uint4*>(prow + kc * kChunk + pos * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            const float mt_used = mref;
-            l = fmaf(l, alpha, (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
-            m = mt_used;
-            // rescale the running output by alpha once the previous product is done
-            if (j >= 1) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&o_done, (uint32_t)(j - 1) & 1u, wc) ? 1 : 0)) { ok = false; break; }
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-#pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        uint32_t v[32];
-                        tmem_ld_32x32b_x32(tmem + lane_base + kColO + c4 * 32, v);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-                        tmem_st_x32(tmem + lane_base + kColO + c4 * 32, v);
-                    }
-                    tmem_st_wait();
-                }
-            }
-            fence_proxy_async_smem();
+            for (int c4 = 0; c4 < 4; ++c4)
+                tmem_ld_32x32b_x32(tmem + lane_base + kColO + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[c4 * 32]));
+            tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[b]);
-        }
-        // output: O * g_v / l
-        if (ok && __all_sync(0xffffffffu, mbar_wait(&o_done, (uint32_t)(ntiles - 1) & 1u, wc) ? 1 : 0)) {
-            tc_fence_after();
+            if (lane == 0) mbar_arrive(&o_free);
             const float sc = __fdiv_rn(*p.g_v, l);
-            uint16_t* orow = p.out + (int64_t)(qrow0 + r) * kD;
+            uint16_t* orow = p.out + (int64_t)(item_qrow(it) + r) * kD;
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem + lane_base + kColO + c4 * 32, v);
-                tmem_ld_wait();
+            for (int t = 0; t < 16; ++t) {
+                uint32_t w[4];
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(v[t * 8 + 2 * u]) * sc,
-                                                                  __uint_as_float(v[t * 8 + 2 * u + 1]) * sc);
-                        w[u] = *reinterpret_cast<uint32_t*>(&hb);
-                    }
-                    *reinterpret_cast<uint4*>(orow + c4 * 32 + t * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+                for (int u = 0; u < 4; ++u) {
+                    __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(o[t * 8 + 2 * u]) * sc,
+                                                              __uint_as_float(o[t * 8 + 2 * u + 1]) * sc);
+                    w[u] = *reinterpret_cast<uint32_t*>(&hb);
                 }
+                *reinterpret_cast<uint4*>(orow + t * 8) = make_uint4(w[0], w[1], w[2], w[3]);
             }
         }
     }
@@ -530,7 +582,12 @@ cudaError_t launch_attention(const uint8_t* q_codes, const uint8_t* q_sf, const 
     p.dev_status = dev_status;
     e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)(Lq / kBQ), (unsigned)H);
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    const int64_t items = (Lq / kBQ) * H;
+    const unsigned grid = (unsigned)(items < sms ? items : sms);     // one persistent CTA per SM
     attn_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tvt, p);
     count_launch(1);
     return cudaGetLastError();

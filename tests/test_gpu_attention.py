@@ -85,3 +85,44 @@ def test_attention_larger_sampled_rows_gpu_quantized(cuda_ok):
             ref = oracle.attention(q, k, v, np.ones(H), H, Lq, Lk, D, h, rows=slice(int(r), int(r) + 1))[0]
             err = np.abs(o[h * Lq + r].astype(np.float64) - ref)
             assert np.all(err <= 3e-3 * vmax[h] + 5e-3 * np.abs(ref))
+
+
+def _sampled_heads(xq, xk, xv, H, Lq, Lk, heads, rows, s_head=None):
+    """The kernel on the whole tensors (GPU-quantized) against the oracle on
+    the sampled heads' slices, quantized with the whole tensors' scales."""
+    Q, K, V = nv.quantize(xq.cuda()), nv.quantize(xk.cuda()), nv.quantize(xv.cuda())
+    sh_dev = torch.tensor(s_head, dtype=torch.float32, device="cuda") if s_head is not None else None
+    o = nv.attention(Q, K, V, H, s_head=sh_dev)
+    torch.cuda.synchronize()
+    gq, gk, gv = (oracle.tensor_scale(x) for x in (xq, xk, xv))
+    for h in heads:
+        q = oracle.quantize(xq[h * Lq:(h + 1) * Lq], gq)
+        k = oracle.quantize(xk[h * Lk:(h + 1) * Lk], gk)
+        v = oracle.quantize(xv[h * Lk:(h + 1) * Lk], gv)
+        vmax = np.abs(oracle.dequantize(*v)).max()
+        sh = np.array([1.0 if s_head is None else s_head[h]])
+        got = o[h * Lq:(h + 1) * Lq].float().cpu().numpy()
+        for r in rows:
+            ref = oracle.attention(q, k, v, sh, 1, Lq, Lk, D, 0, rows=slice(int(r), int(r) + 1))[0]
+            err = np.abs(got[r].astype(np.float64) - ref)
+            assert np.all(err <= 3e-3 * vmax + 5e-3 * np.abs(ref)), (h, r, float(err.max()))
+
+
+def test_attention_several_items_per_cta(cuda_ok):
+    """More work items (head, 128-query tile) than SMs: each persistent CTA
+    takes several, over different heads with different s_head; ring slots and
+    barrier phases run on across the item boundaries."""
+    H, Lq, Lk = 24, 2048, 512
+    xq = synth.random_bf16((H * Lq, D), seed=78, dist="token_scaled")
+    xk = synth.random_bf16((H * Lk, D), seed=79, dist="normal")
+    xv = synth.random_bf16((H * Lk, D), seed=80, dist="student_t3")
+    s_head = [0.5 + 0.25 * h for h in range(H)]
+    _sampled_heads(xq, xk, xv, H, Lq, Lk, heads=(0, 9, 10, 18, 23), rows=(0, 129, 1151, 2047), s_head=s_head)
+
+
+def test_attention_full_size_sampled(cuda_ok):
+    """The video DiT's spatial attention as timed: 384 heads x 2048 tokens,
+    d = 128 (6144 work items on the persistent grid), sampled heads and rows."""
+    H, L = 384, 2048
+    xs = [synth.random_bf16((H * L, D), seed=90 + i, dist="normal") for i in range(3)]
+    _sampled_heads(*xs, H, L, L, heads=(0, 147, 148, 295, 383), rows=(0, 777, 2047))
