@@ -522,7 +522,7 @@ cudaError_t launch_gemm_w4a4(const GemmW4A4Args& a, int num_sms, cudaStream_t st
     // N a multiple of 256: CTA-pair kernel with 256 x 256 tiles.  Otherwise
     // (N = 1152, 3456, ...): single-CTA 128 x 128 tiles with a double-buffered
     // accumulator, so no tile column is wasted on padding.
-    if (a.N % 256 == 0 && !a.mx) return launch_gemm_w4a4_2sm(a, num_sms, stream);
+    if (a.N % 256 == 0) return launch_gemm_w4a4_2sm(a, num_sms, stream);
     return launch_gemm_w4a4_grouped(&a, 1, num_sms, stream);
 }
 

@@ -58,30 +58,41 @@ constexpr int BK_BYTES = 128;                    // 256 FP4 values per row per s
 constexpr int A_BYTES = 128 * BK_BYTES;          // this CTA's 128 rows of A
 constexpr int B_BYTES = 128 * BK_BYTES;          // this CTA's 128-row half of B
 constexpr int SF_ATOM = 512;
-constexpr int SFA_BYTES = 4 * SF_ATOM;           // 128 rows x 4 K=64 steps
-constexpr int SFB_BYTES = 2 * 4 * SF_ATOM;       // 256 rows x 4 K=64 steps
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // 38912
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 512;
 constexpr int kRegsLow = 56;                     // warpgroups 0-1
 constexpr int kRegsHigh = 200;                   // epilogue warpgroups 2-3
 static_assert(256 * kRegsLow + 256 * kRegsHigh <= kThreads * 128, "register split exceeds the launch budget");
-constexpr int SF_COLS_STEP = 4 + 8;              // SFA 4 columns, SFB 8 columns per K=64 step
-constexpr int SF_COLS_STAGE = 4 * SF_COLS_STEP;
+constexpr int SF_COLS_ATOM = 4 + 8;              // SFA 4 columns, SFB 8 columns per scale atom
 constexpr int kGroupM = 8;                       // rasterisation group, in 256-row pair tiles
 constexpr int kSmemLimit = 232448;
 
 enum OutKind { OUT_BF16 = 0, OUT_F32 = 1, OUT_NVFP4 = 2 };
 
-template <int OUT>
+// Per-stage layout.  NVFP4 (kind::mxf4nvf4, block16): a 128-row scale atom
+// covers K = 64, four per stage.  MX (kind::mxf4, block32): an atom covers
+// K = 128, two per stage; each K = 64 MMA step reads two of a row's four
+// scale bytes, selected by a byte id.
+template <bool MXS>
+struct Lay {
+    static constexpr int SF_PER = MXS ? 2 : 4;   // scale atoms per 128 rows per stage
+    static constexpr int K_ATOM = MXS ? 128 : 64;
+    static constexpr int SFA_BYTES = SF_PER * SF_ATOM;            // this CTA's 128 A rows
+    static constexpr int SFB_BYTES = 2 * SFA_BYTES;               // all 256 B rows
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // 38912 (NVFP4)
+    static constexpr int SF_COLS_STAGE = SF_PER * SF_COLS_ATOM;
+};
+
+template <int OUT, bool MXS>
 struct Cfg {
+    static constexpr int STAGE_BYTES = Lay<MXS>::STAGE_BYTES;
     static constexpr int EPI_BUF = OUT == OUT_F32 ? 4096 : (OUT == OUT_BF16 ? 2048 : 0);   // 32 rows x 32 cols
     static constexpr int EPI_BYTES = kEpiWarps * 2 * EPI_BUF;
     static constexpr int FIT = (kSmemLimit - 1024 - EPI_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = FIT < 5 ? FIT : 5;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024;
     static_assert(STAGES >= 3, "pipeline depth");
-    static_assert(256 + STAGES * SF_COLS_STAGE <= 512, "TMEM columns");
+    static_assert(256 + STAGES * Lay<MXS>::SF_COLS_STAGE <= 512, "TMEM columns");
 };
 
 struct Params {
@@ -143,31 +154,43 @@ __device__ __forceinline__ void store_chunk(const uint32_t* r, float alpha, uint
     }
 }
 
-// Scale atoms of one K=64 step of the pair (A: 128 rows of this CTA, B: all
-// 256 rows, in both CTAs) into the step's TMEM columns.
-__device__ __forceinline__ void k_copy_scales(uint32_t sfs, uint32_t sf_col, int ks) {
-    const uint32_t col = sf_col + ks * SF_COLS_STEP;
-    tc_cp2_32x128b_warpx4(col, sdesc_sf(sfs + ks * SF_ATOM));
-    tc_cp2_32x128b_warpx4(col + 4, sdesc_sf(sfs + SFA_BYTES + ks * SF_ATOM));
-    tc_cp2_32x128b_warpx4(col + 8, sdesc_sf(sfs + SFA_BYTES + 4 * SF_ATOM + ks * SF_ATOM));
+// Scale atom `at` of a stage of the pair (A: 128 rows of this CTA, B: all
+// 256 rows, in both CTAs) into the atom's TMEM columns.
+template <bool MXS>
+__device__ __forceinline__ void k_copy_scales(uint32_t sfs, uint32_t sf_col, int at) {
+    using L = Lay<MXS>;
+    const uint32_t col = sf_col + at * SF_COLS_ATOM;
+    tc_cp2_32x128b_warpx4(col, sdesc_sf(sfs + at * SF_ATOM));
+    tc_cp2_32x128b_warpx4(col + 4, sdesc_sf(sfs + L::SFA_BYTES + at * SF_ATOM));
+    tc_cp2_32x128b_warpx4(col + 8, sdesc_sf(sfs + L::SFA_BYTES + L::SF_PER * SF_ATOM + at * SF_ATOM));
 }
 
 // One K=64 step of the pair: the block-scaled MMA reading the step's scale
-// columns.
+// columns (MX: the atom of steps 2i and 2i + 1, bytes 0-1 or 2-3 of each row's
+// scale word).
+template <bool MXS>
 __device__ __forceinline__ void k_mma(uint32_t tmem_acc, uint32_t sb, uint32_t sf_col, int ks, uint32_t idesc,
                                       bool accumulate) {
-    const uint32_t col = sf_col + ks * SF_COLS_STEP;
-    tc_mma2_nvf4(tmem_acc, sdesc_kmajor_sw128(sb + ks * 32), sdesc_kmajor_sw128(sb + A_BYTES + ks * 32), idesc, col,
-                 col + 4, accumulate ? 1u : 0u);
+    const uint64_t ad = sdesc_kmajor_sw128(sb + ks * 32), bd = sdesc_kmajor_sw128(sb + A_BYTES + ks * 32);
+    if (MXS) {
+        const uint32_t col = sf_col + (ks >> 1) * SF_COLS_ATOM, byte = (uint32_t)(ks & 1) * 2u;
+        tc_mma2_mxf4(tmem_acc, ad, bd, idesc | (byte << 29) | (byte << 4), col | (byte << 30), (col + 4) | (byte << 30),
+                     accumulate ? 1u : 0u);
+    } else {
+        const uint32_t col = sf_col + ks * SF_COLS_ATOM;
+        tc_mma2_nvf4(tmem_acc, ad, bd, idesc, col, col + 4, accumulate ? 1u : 0u);
+    }
 }
 
-template <int OUT, int ACT>
+template <int OUT, int ACT, bool MXS>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
              const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
              const __grid_constant__ CUtensorMap tmap_y, const Params p) {
-    using C = Cfg<OUT>;
+    using C = Cfg<OUT, MXS>;
+    using L = Lay<MXS>;
     constexpr int STAGES = C::STAGES;
+    constexpr int STAGE_BYTES = L::STAGE_BYTES;
     extern __shared__ uint8_t smem_raw[];
     // full:   the leader's; both CTAs' operand tiles and scale atoms of a stage
     //         have landed (the peer's loads signal it through cta_group::2);
@@ -206,7 +229,7 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     // (beyond M or N) multiply zero codes by a finite scale
     for (int s = 0; s < STAGES; ++s) {
         uint32_t* z = reinterpret_cast<uint32_t*>(smem + s * STAGE_BYTES + A_BYTES + B_BYTES);
-        for (int i = threadIdx.x; i < (SFA_BYTES + SFB_BYTES) / 4; i += kThreads) z[i] = 0u;
+        for (int i = threadIdx.x; i < (L::SFA_BYTES + L::SFB_BYTES) / 4; i += kThreads) z[i] = 0u;
     }
     fence_proxy_async_smem();
     cluster_sync_all();                       // barriers initialised in both CTAs
@@ -220,7 +243,8 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     const uint32_t tmem_base = tmem_base_sh;
 
     const int num_kt = (p.K + 255) / 256;
-    const int k_atoms = p.K / 64;
+    const int k_atoms = p.K / L::K_ATOM;             // scale atoms per 128 rows
+    const int k_steps = p.K / 64;                    // K = 64 MMA steps
     const uint32_t sf_base = tmem_base + 256;
     // one register-budget change per warpgroup, before the roles diverge
     // (the epilogue code sits under the same branch as its increase, so that
@@ -253,9 +277,10 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                         if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * STAGE_BYTES);
                         const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
                         uint8_t* sfs = sb + A_BYTES + B_BYTES;
-                        tma_load_2d_pair(sfs, &tmap_sfa, fb, 0, sfa_row + kt * 4, pol_a);
-                        tma_load_2d_pair(sfs + SFA_BYTES, &tmap_sfb, fb, 0, sfb_row0 + kt * 4, pol_b);
-                        tma_load_2d_pair(sfs + SFA_BYTES + 4 * SF_ATOM, &tmap_sfb, fb, 0, sfb_row1 + kt * 4, pol_b);
+                        tma_load_2d_pair(sfs, &tmap_sfa, fb, 0, sfa_row + kt * L::SF_PER, pol_a);
+                        tma_load_2d_pair(sfs + L::SFA_BYTES, &tmap_sfb, fb, 0, sfb_row0 + kt * L::SF_PER, pol_b);
+                        tma_load_2d_pair(sfs + L::SFA_BYTES + L::SF_PER * SF_ATOM, &tmap_sfb, fb, 0,
+                                         sfb_row1 + kt * L::SF_PER, pol_b);
                         tma_load_2d_pair(sb, &tmap_a, fb, kt * BK_BYTES, arow, pol_a);
                         tma_load_2d_pair(sb + A_BYTES, &tmap_b, fb, kt * BK_BYTES, brow, pol_b);
                     }
@@ -293,14 +318,14 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                         }
                         tc_fence_after();
                         const uint32_t sfs = smem0 + stage * STAGE_BYTES + A_BYTES + B_BYTES;
-                        const uint32_t sf_col = sf_base + stage * SF_COLS_STAGE;
-                        const int nks = k_atoms - kt * 4;
+                        const uint32_t sf_col = sf_base + stage * L::SF_COLS_STAGE;
+                        const int nat = k_atoms - kt * L::SF_PER;
                         if (elect_one()) {
-                            if (nks >= 4) {
+                            if (nat >= L::SF_PER) {
 #pragma unroll
-                                for (int ks = 0; ks < 4; ++ks) k_copy_scales(sfs, sf_col, ks);
+                                for (int at = 0; at < L::SF_PER; ++at) k_copy_scales<MXS>(sfs, sf_col, at);
                             } else {
-                                for (int ks = 0; ks < nks; ++ks) k_copy_scales(sfs, sf_col, ks);
+                                for (int at = 0; at < nat; ++at) k_copy_scales<MXS>(sfs, sf_col, at);
                             }
                             tc_commit2_mc(&scaled_bar[stage], 0x1);
                         }
@@ -314,7 +339,7 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                 // -------------------------------------------------------- MMA issuer (leader)
                 // The whole warp runs the loop so that descriptors and addresses
                 // stay warp-uniform; one elected lane issues four MMAs per stage.
-                constexpr uint32_t idesc = idesc_nvf4(256, 256);
+                constexpr uint32_t idesc = MXS ? idesc_mxf4(256, 256) : idesc_nvf4(256, 256);
                 const uint32_t smem0 = smem_u32(smem);
                 int stage = 0;
                 uint32_t phase = 0, acc_phase = 0;
@@ -333,14 +358,16 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                         }
                         tc_fence_after();
                         const uint32_t sb = smem0 + stage * STAGE_BYTES;
-                        const uint32_t sf_col = sf_base + stage * SF_COLS_STAGE;
-                        const int nks = k_atoms - kt * 4;
+                        const uint32_t sf_col = sf_base + stage * L::SF_COLS_STAGE;
+                        const int nks = k_steps - kt * 4;
                         if (elect_one()) {
                             if (nks >= 4) {
-    #pragma unroll
-                                for (int ks = 0; ks < 4; ++ks) k_mma(tmem_base, sb, sf_col, ks, idesc, (kt | ks) != 0);
+#pragma unroll
+                                for (int ks = 0; ks < 4; ++ks)
+                                    k_mma<MXS>(tmem_base, sb, sf_col, ks, idesc, (kt | ks) != 0);
                             } else {
-                                for (int ks = 0; ks < nks; ++ks) k_mma(tmem_base, sb, sf_col, ks, idesc, (kt | ks) != 0);
+                                for (int ks = 0; ks < nks; ++ks)
+                                    k_mma<MXS>(tmem_base, sb, sf_col, ks, idesc, (kt | ks) != 0);
                             }
                             tc_commit2_mc(&empty_bar[stage], 0x3);
                         }
@@ -365,7 +392,8 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
         const int q = warp & 3;                       // TMEM lane quarter
         const int h = (warp - 8) >> 2;                // column half: [0,128) or [128,256)
         const int row_t = (int)rank * 128 + q * 32 + lane;    // row inside the pair tile
-        const float alpha = __fmul_rn(*p.a_scale, *p.b_scale);
+        // MX operands have no tensor scale: a null scale reads as 1
+        const float alpha = __fmul_rn(p.a_scale ? *p.a_scale : 1.0f, p.b_scale ? *p.b_scale : 1.0f);
         float g_y = 0.0f;
         if (OUT == OUT_NVFP4) g_y = *p.y_scale;
         const ScaleConsts sc_y = scale_consts(g_y);
@@ -466,20 +494,21 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     }
 }
 
-template <int OUT, int ACT>
+template <int OUT, int ACT, bool MXS>
 cudaError_t launch_out(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) {
-    using C = Cfg<OUT>;
+    using C = Cfg<OUT, MXS>;
+    using L = Lay<MXS>;
     CUtensorMap ta, tb, tsa, tsb, ty;
     const uint64_t kh = (uint64_t)(a.K / 2);
-    const uint64_t atoms_a = (uint64_t)((a.M + 127) / 128) * (uint64_t)(a.K / 64);
-    const uint64_t atoms_b = (uint64_t)((a.N + 127) / 128) * (uint64_t)(a.K / 64);
+    const uint64_t atoms_a = (uint64_t)((a.M + 127) / 128) * (uint64_t)(a.K / L::K_ATOM);
+    const uint64_t atoms_b = (uint64_t)((a.N + 127) / 128) * (uint64_t)(a.K / L::K_ATOM);
     if (make_tmap_2d(&ta, a.a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kh, (uint64_t)a.M, kh, BK_BYTES, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
         make_tmap_2d(&tb, a.b_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kh, (uint64_t)a.N, kh, BK_BYTES, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
-        make_tmap_2d(&tsa, a.a_sf, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, 128, atoms_a, SF_ATOM, 128, 4,
+        make_tmap_2d(&tsa, a.a_sf, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, 128, atoms_a, SF_ATOM, 128, L::SF_PER,
                      CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
-        make_tmap_2d(&tsb, a.b_sf, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, 128, atoms_b, SF_ATOM, 128, 4,
+        make_tmap_2d(&tsb, a.b_sf, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, 128, atoms_b, SF_ATOM, 128, L::SF_PER,
                      CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     CUresult r = CUDA_SUCCESS;
@@ -508,7 +537,7 @@ cudaError_t launch_out(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) 
     p.y_amax = a.y_amax;
     p.dev_status = a.dev_status;
 
-    auto kern = gemm2_kernel<OUT, ACT>;
+    auto kern = gemm2_kernel<OUT, ACT, MXS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
 
@@ -541,15 +570,24 @@ cudaError_t launch_out(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) 
 cudaError_t launch_gemm_w4a4_2sm(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) {
     using namespace w4a4_2sm;
     const bool gelu = a.act == ACT_GELU_TANH;
+    if (a.mx) {
+        // MX operands: bf16 or FP32 output (no NVFP4 output of an MX product)
+        if (a.y == nullptr) return cudaErrorInvalidValue;
+        if (a.y_dtype == 1)
+            return gelu ? launch_out<OUT_F32, ACT_GELU_TANH, true>(a, num_sms, stream)
+                        : launch_out<OUT_F32, ACT_NONE, true>(a, num_sms, stream);
+        return gelu ? launch_out<OUT_BF16, ACT_GELU_TANH, true>(a, num_sms, stream)
+                    : launch_out<OUT_BF16, ACT_NONE, true>(a, num_sms, stream);
+    }
     if (a.y != nullptr) {
         if (a.y_dtype == 1)
-            return gelu ? launch_out<OUT_F32, ACT_GELU_TANH>(a, num_sms, stream)
-                        : launch_out<OUT_F32, ACT_NONE>(a, num_sms, stream);
-        return gelu ? launch_out<OUT_BF16, ACT_GELU_TANH>(a, num_sms, stream)
-                    : launch_out<OUT_BF16, ACT_NONE>(a, num_sms, stream);
+            return gelu ? launch_out<OUT_F32, ACT_GELU_TANH, false>(a, num_sms, stream)
+                        : launch_out<OUT_F32, ACT_NONE, false>(a, num_sms, stream);
+        return gelu ? launch_out<OUT_BF16, ACT_GELU_TANH, false>(a, num_sms, stream)
+                    : launch_out<OUT_BF16, ACT_NONE, false>(a, num_sms, stream);
     }
-    return gelu ? launch_out<OUT_NVFP4, ACT_GELU_TANH>(a, num_sms, stream)
-                : launch_out<OUT_NVFP4, ACT_NONE>(a, num_sms, stream);
+    return gelu ? launch_out<OUT_NVFP4, ACT_GELU_TANH, false>(a, num_sms, stream)
+                : launch_out<OUT_NVFP4, ACT_NONE, false>(a, num_sms, stream);
 }
 
 }  // namespace nvfp4

@@ -417,6 +417,17 @@ __device__ __forceinline__ void tc_mma2_nvf4(uint32_t d_tmem, uint64_t adesc, ui
         : "memory");
 }
 
+// The same on MX operands (E8M0 scales per 32 values, kind::mxf4).
+__device__ __forceinline__ void tc_mma2_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
 // Arrive on the barrier at this shared-memory offset in every CTA of `mask`
 // once all prior tcgen05 operations of the pair have completed.
 __device__ __forceinline__ void tc_commit2_mc(uint64_t* bar, uint16_t mask) {

@@ -100,7 +100,33 @@ def test_mx_gemm_one_hot(cuda_ok, m0, n0, k0):
     assert np.array_equal(oracle.mx_gemm(ac, asf, bc, bsf), expect)
 
 
-@pytest.mark.parametrize("M,N,K", [(300, 384, 1152), (128, 256, 256), (77, 1152, 640), (513, 136, 384)])
+@pytest.mark.parametrize("m0,n0,k0", [(0, 0, 0), (200, 300, 600), (383, 511, 639), (129, 129, 129),
+                                       (255, 256, 383), (130, 7, 300)])
+def test_mx_gemm_one_hot_pair_kernel(cuda_ok, m0, n0, k0):
+    """N = 512 (CTA-pair kernel): one nonzero product lands in the right
+    output, also in the second CTA's rows, the second B half and the last,
+    half-filled K stage."""
+    M, N, K = 384, 512, 640
+    kb = K // 32
+    ac = np.zeros((M, K // 2), np.uint8)
+    bc = np.zeros((N, K // 2), np.uint8)
+    ac[m0, k0 // 2] = 0x5 << (4 * (k0 & 1))             # 3.0
+    bc[n0, k0 // 2] = 0xB << (4 * (k0 & 1))             # -1.5
+    asf = np.full(oracle.mx_sf_bytes(M, K), 127, np.uint8)
+    bsf = np.full(oracle.mx_sf_bytes(N, K), 127, np.uint8)
+    asf[oracle.sf_offset(m0, k0 // 32, kb)] = 127 + 5
+    bsf[oracle.sf_offset(n0, k0 // 32, kb)] = 127 - 7
+    y = nv.mx_gemm(_upload(ac, asf, M, K), _upload(bc, bsf, N, K), out_dtype=torch.float32).cpu().numpy()
+    expect = np.zeros((M, N))
+    expect[m0, n0] = 3.0 * -1.5 * 2.0 ** 5 * 2.0 ** -7
+    assert np.array_equal(y, expect)
+    assert np.array_equal(oracle.mx_gemm(ac, asf, bc, bsf), expect)
+
+
+# N a multiple of 256 runs on the CTA-pair kernel (256 x 256 tiles), the rest on
+# the single-CTA kernel; K = 640 and 1152 end in a half stage (one MX scale atom)
+@pytest.mark.parametrize("M,N,K", [(300, 384, 1152), (128, 256, 256), (77, 1152, 640), (513, 136, 384),
+                                   (300, 512, 1152), (513, 768, 640), (64, 256, 384)])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 def test_mx_gemm_vs_oracle(cuda_ok, M, N, K, out_dtype):
     x = synth.random_bf16((M, K), seed=M + K, dist="student_t3")
