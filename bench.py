@@ -188,25 +188,31 @@ def oracle_sample(rows_per_layer: int, col_frac: float = 1.0):
 
 
 REF_BUDGET_S = 60.0     # CPU seconds the reference arm's timed steps may take in all
+REF_PROBE_FRAC = 0.1    # output-feature fraction of the reference arm's warm-up steps
+
+
+def ref_sample_size(rows: int, steps: int, probe_secs: float, budget_s: float = REF_BUDGET_S):
+    """Rows and output-feature fraction of one reference-arm step, from the
+    time of a warm-up step on `rows` rows and REF_PROBE_FRAC of the features:
+    the cost is close to proportional to the features sampled, so the
+    fraction is scaled to keep all `steps` timed steps within the budget;
+    below one 128-feature tile of the narrowest layer the rows shrink."""
+    frac = min(1.0, REF_PROBE_FRAC * budget_s / max(1, steps) / max(probe_secs, 1e-9))
+    min_frac = 128 / 3072
+    if frac < min_frac:
+        rows = max(1, int(rows * frac / min_frac))
+        frac = min_frac
+    return rows, frac
 
 
 def run_reference(args):
     rank, world, local = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), 0
     if rank != 0:
         return 0
-    rows = args.ref_rows
-    # warm-up on a tenth of the output features; the step's cost is close to
-    # proportional to the features sampled, so that sets the fraction that
-    # keeps all K timed steps within the budget
-    probe = 0.1
     s = 0.0
     for _ in range(max(1, args.warmup)):
-        _, s, _ = oracle_sample(rows, probe)
-    frac = min(1.0, probe * REF_BUDGET_S / max(1, args.steps) / max(s, 1e-9))
-    min_frac = 128 / 3072                       # one 128-feature tile of the narrowest layer
-    if frac < min_frac:                         # fewer rows once the features cannot shrink
-        rows = max(1, int(rows * frac / min_frac))
-        frac = min_frac
+        _, s, _ = oracle_sample(args.ref_rows, REF_PROBE_FRAC)
+    rows, frac = ref_sample_size(args.ref_rows, args.steps, s)
     fl, secs = 0, 0.0
     desc = ""
     for _ in range(args.steps):

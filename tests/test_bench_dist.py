@@ -84,6 +84,18 @@ def test_reference_arm_line_on_rank_zero(monkeypatch, capsys):
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
 
 
+def test_reference_sample_is_bounded():
+    """The reference arm's per-step sample shrinks with K so that the timed
+    steps stay within the budget: features first, then rows."""
+    rows, frac = bench.ref_sample_size(48, 10, probe_secs=0.5, budget_s=60.0)
+    assert rows == 48 and frac == 1.0                     # 10 x 5 s fits in 60 s
+    rows, frac = bench.ref_sample_size(48, 100, probe_secs=0.5, budget_s=60.0)
+    assert rows == 48 and abs(frac - 0.12) < 1e-12        # 100 steps x 0.6 s
+    rows, frac = bench.ref_sample_size(48, 5000, probe_secs=0.5, budget_s=60.0)
+    assert frac == 128 / 3072 and 1 <= rows < 48          # features at one tile, fewer rows
+    assert bench.ref_sample_size(48, 10 ** 9, probe_secs=0.5)[0] == 1
+
+
 def test_reduced_case_selects_layers_and_rows():
     class A:
         layers, m = "fc1,fc2", 4096
