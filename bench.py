@@ -663,7 +663,12 @@ def run_ours(args):
         cpu = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": desc}
 
     if rank == 0:
-        fp4_peak = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"]) * FP4_OVER_BF16
+        # the GEMM is timed inside a long step (back-to-back steps under the
+        # power cap) once the timed region lasts half a second or more: then
+        # the sustained bf16 figure is its denominator, else the burst one
+        sustained = max_ms >= 500.0
+        bf16_key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+        fp4_peak = peaks.get(bf16_key, FALLBACK[bf16_key]) * FP4_OVER_BF16
         hbm_peak = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
         # dominant kernel: the GEMM of the largest layer (fc1, the 32768x3072x12288 shape)
         names = [L.name for L in wl.layers]
@@ -696,7 +701,9 @@ def run_ours(args):
             "roofline": {"bound": "tensor", "kernel": f"gemm_w4a4 {L.name} {L.M}x{L.K}x{L.N}",
                          "achieved": round(g_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                          "frac": round(g_tflops / fp4_peak, 4),
-                         "peak_source": f"{peak_src} bf16 x {FP4_OVER_BF16:g} (nominal FP4/bf16 ratio)",
+                         "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'} x "
+                                        f"{FP4_OVER_BF16:g} (nominal FP4/bf16 ratio; timed region "
+                                        f"{max_ms / 1e3:.2f} s)",
                          "traffic": g_traffic},
             "quantize": {"bound": "hbm", "kernel": f"amax + quantize {wl.layers[qi].name} input "
                                                    f"{wl.layers[qi].M}x{wl.layers[qi].K}",
