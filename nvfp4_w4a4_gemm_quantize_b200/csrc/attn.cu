@@ -495,19 +495,26 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
 }
 
 // V [H*Lk, d] NVFP4 -> V^T [H*d, Lk] bf16, exact (the tensor scale g_v is
-// applied with the output).  A CTA per (64 keys, head): 256 threads decode 16
-// code bytes each (one key, 32 values of d) into a padded shared tile
-// [d][64 keys], then write its 128 rows of 128 bytes out.
+// applied with the output).  A CTA per (64 keys, head); thread t decodes the
+// 16 code bytes of key t / 4, d = 32 (t % 4) .. + 31.  Two threads of
+// neighbouring keys (lanes t and t ^ 4) trade halves of their bf16 pairs so
+// that each holds 32-bit words of two keys at one d -- the even-key thread
+// the even d, the odd-key thread the odd d -- and stores them into a shared
+// tile [d][32 key pairs]; its 128 rows of 128 bytes then go out in 16-byte
+// stores.  Tile row pitch 36 words and the key-pair column XORed with
+// 8 (d / 32): both the word stores and the 16-byte loads are free of bank
+// conflicts.
 constexpr int kVtKeys = 64;
-constexpr int kVtPitch = kVtKeys + 2;            // bf16 elements per shared row (padding spreads banks)
+constexpr int kVtPitch = 36;                     // 32-bit words per shared row (32 key pairs + 4)
 
 __global__ void __launch_bounds__(256)
 v_transpose_kernel(const uint8_t* __restrict__ v_codes, const uint8_t* __restrict__ v_sf, int Lk,
                    uint16_t* __restrict__ vt) {
-    __shared__ uint16_t tile[kD * kVtPitch];
+    __shared__ __align__(16) uint32_t tile[kD * kVtPitch];
     const int t = threadIdx.x;
     const int h = blockIdx.y, key0 = blockIdx.x * kVtKeys;
     const int key = t >> 2, part = t & 3;                  // 16 bytes: d = 32 part .. 32 part + 31
+    const int odd = key & 1, kp = key >> 1;
     const int64_t row = (int64_t)h * Lk + key0 + key;      // row of V
     const uint4 cb = *reinterpret_cast<const uint4*>(v_codes + row * (kD / 2) + part * 16);
     const uint32_t w[4] = {cb.x, cb.y, cb.z, cb.w};
@@ -515,6 +522,7 @@ v_transpose_kernel(const uint8_t* __restrict__ v_codes, const uint8_t* __restric
     // [rows, 128] tensor: two 512-byte atoms per 128-row group
     const int rr = (int)(row & 127);
     const uint8_t* sfr = v_sf + (row >> 7) * 1024 + (rr & 31) * 16 + (rr >> 5) * 4;
+    const int col = kp ^ (8 * part);
 #pragma unroll
     for (int hb = 0; hb < 2; ++hb) {
         const int blk = 2 * part + hb;
@@ -524,24 +532,26 @@ v_transpose_kernel(const uint8_t* __restrict__ v_codes, const uint8_t* __restric
             const uint32_t word = w[2 * hb + q];
 #pragma unroll
             for (int by = 0; by < 4; ++by) {
+                // own pair (d, d + 1) of this key; the neighbour key's pair at the same d
                 const uint32_t pr = dequant_pair_attn((word >> (8 * by)) & 0xFFu, sc);
-                const int d0 = 32 * part + 16 * hb + 8 * q + 2 * by;
-                tile[d0 * kVtPitch + key] = (uint16_t)(pr & 0xFFFFu);
-                tile[(d0 + 1) * kVtPitch + key] = (uint16_t)(pr >> 16);
+                const uint32_t nb = __shfl_xor_sync(0xffffffffu, pr, 4);
+                const int d = 32 * part + 16 * hb + 8 * q + 2 * by + odd;
+                // word at d: (even key, odd key) values, the even key in the low half
+                const uint32_t wd = odd ? (nb >> 16) | (pr & 0xFFFF0000u) : (pr & 0xFFFFu) | (nb << 16);
+                tile[d * kVtPitch + col] = wd;
             }
         }
     }
     __syncthreads();
-    // 128 rows x 64 keys out: thread -> half a row (32 keys, 64 bytes)
+    // 128 rows x 64 keys out: thread -> half a row (16 key pairs, 64 bytes)
     const int orow = t >> 1, half = t & 1;
     uint16_t* dst = vt + ((int64_t)h * kD + orow) * Lk + key0 + half * 32;
-    const uint16_t* src = tile + orow * kVtPitch + half * 32;
+    const uint32_t* src = tile + orow * kVtPitch;
+    const int sw = 8 * (orow >> 5);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        uint32_t q[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) q[u] = (uint32_t)src[8 * i + 2 * u] | ((uint32_t)src[8 * i + 2 * u + 1] << 16);
-        *reinterpret_cast<uint4*>(dst + 8 * i) = make_uint4(q[0], q[1], q[2], q[3]);
+    for (int j = 0; j < 4; ++j) {
+        const uint4 v = *reinterpret_cast<const uint4*>(src + ((16 * half + 4 * j) ^ sw));
+        *reinterpret_cast<uint4*>(dst + 8 * j) = v;
     }
 }
 
