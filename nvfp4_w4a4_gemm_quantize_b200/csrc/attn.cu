@@ -71,7 +71,6 @@ constexpr uint32_t kColSfK = 400;            // K scales per S buffer: 2 x (2 x 
 struct Params {
     const uint8_t* q_sf;
     const uint8_t* k_sf;
-    const uint8_t* v_sf;
     const float* g_q;
     const float* g_k;
     const float* g_v;
@@ -103,13 +102,6 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// E2M1 code -> value (exact).
-__device__ __forceinline__ float e2m1_val(uint32_t c) {
-    const uint32_t e = (c >> 1) & 3u, m = c & 1u;
-    const float mag = e == 0u ? 0.5f * (float)m : __uint_as_float(((e + 126u) << 23) | (m << 22));
-    return (c & 8u) ? -mag : mag;
-}
-
 // Two E2M1 codes (one byte, low nibble first) times their shared scale,
 // exactly, as a bf16 pair: the f16 decode shifted down three bits is the bf16
 // pattern of the value times 2^-112 (sign kept), and one bf16 multiply by the
@@ -132,9 +124,6 @@ __device__ __forceinline__ uint32_t e4m3_to_b2_scaled_attn(uint32_t code) {
     const uint32_t b = __float_as_uint(f) >> 16;
     return b | (b << 16);
 }
-
-// Byte of (row r, 16-value block c) inside a 128-row group's two scale atoms.
-__device__ __forceinline__ int sf_byte(int r, int c) { return (c >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (c & 3); }
 
 // Persistent: CTA c takes work items (head, 128-query tile) c, c + grid, ...
 // Key tiles carry one running number n over all of a CTA's items, which
@@ -580,7 +569,6 @@ cudaError_t launch_attention(const uint8_t* q_codes, const uint8_t* q_sf, const 
     Params p;
     p.q_sf = q_sf;
     p.k_sf = k_sf;
-    p.v_sf = v_sf;
     p.g_q = g_q;
     p.g_k = g_k;
     p.g_v = g_v;
