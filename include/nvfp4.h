@@ -339,7 +339,8 @@ nvfp4_status nvfp4_mx_dequantize(const uint8_t *codes, const uint8_t *sf, int64_
  * with the block-32 E8M0 tensor-core MMA (kind::mxf4), FP32 accumulation.
  * A [M, K] and B [N, K] as nvfp4_mx_quantize writes them; K % 128 == 0;
  * Y [M, N] bf16 (N % 8 == 0) or FP32 (N % 4 == 0); act as nvfp4_gemm_w4a4.
- * One persistent kernel (128 x 128 tiles).
+ * One persistent kernel: 256 x 256 tiles on CTA pairs (cta_group::2) when
+ * N % 256 == 0, else 128 x 128 tiles on single CTAs.
  */
 nvfp4_status nvfp4_mx_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const uint8_t *b_codes,
                            const uint8_t *b_sf, int64_t M, int64_t N, int64_t K, void *y, int y_dtype,
@@ -363,7 +364,8 @@ nvfp4_status nvfp4_mx_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const ui
  *           bytes, 16-byte aligned: V decoded to bf16 and transposed (once
  *           per call, then read by every query tile); not preserved.
  * d == 128, Lq and Lk multiples of 128 (no masking), H <= 65535.  Two kernels:
- * the V transpose, then a CTA per (128 queries, head).
+ * the V transpose, then a persistent kernel (one CTA per SM) over the work
+ * items (128 queries, head).
  */
 size_t nvfp4_attention_workspace_bytes(int64_t H, int64_t Lk, int64_t d);   /* H * d * Lk * 2 */
 nvfp4_status nvfp4_attention(const uint8_t *q_codes, const uint8_t *q_sf, const float *q_scale,
