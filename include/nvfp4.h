@@ -99,7 +99,8 @@ size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t k);
  *         a block with s == 0 gives codes 0.
  * x_bf16        [rows, k] bf16, row stride ld_x elements (ld_x >= k, ld_x % 8 == 0,
  *               pointer 16-byte aligned).
- * rows >= 0;    k > 0 and k % 64 == 0.
+ * rows >= 0;    k > 0 and k % 64 == 0.  rows <= 65535 * 128 = 8,388,480 (one
+ *               128-row block per grid row); larger is NVFP4_ERR_UNSUPPORTED_SHAPE.
  * codes         out, rows * k/2 bytes (16-byte aligned).
  * sf            out, nvfp4_sf_bytes(rows, k) bytes (16-byte aligned); padding rows
  *               are written as zero.
@@ -134,7 +135,10 @@ nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t rows, int64_t k, int64_t
  * streams) race and may produce wrong scales -- serialize them.  The first call
  * on each device looks up the array's device address (a runtime call, no
  * allocation); make that first call before any stream capture.  The call
- * itself allocates nothing.
+ * itself allocates nothing.  The looked-up address is kept until
+ * nvfp4_shutdown(): after cudaDeviceReset() (or anything else that destroys
+ * and recreates the device's primary context, which may move the array) call
+ * nvfp4_shutdown() before the next call.  Row limit as nvfp4_quantize.
  */
 enum { NVFP4_NOALLOC_SCRATCH_FLOATS = 256 };
 nvfp4_status nvfp4_quantize_noalloc(const void *x_bf16, int64_t rows, int64_t k, int64_t ld_x,

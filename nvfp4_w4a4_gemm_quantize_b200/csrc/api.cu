@@ -106,7 +106,7 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t
     if (!tensor_scale) return NVFP4_ERR_INVALID_ARG;
     if (rows > 0 && (!x_bf16 || !codes || !sf)) return NVFP4_ERR_INVALID_ARG;
     if (k % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (rows > (int64_t)1 << 31 || k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (rows > kQuantMaxRows || k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     const bool given = (flags & NVFP4_SCALE_GIVEN) != 0u;
     if (!given && (!workspace || workspace_bytes < kQuantWorkspaceBytes)) return NVFP4_ERR_WORKSPACE;
     if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(sf) || (ld_x % 8) != 0 ||
@@ -145,7 +145,7 @@ nvfp4_status nvfp4_quantize_block(const void* x_bf16, int64_t rows, int64_t k, i
     if (!tensor_scale) return NVFP4_ERR_INVALID_ARG;
     if (rows > 0 && (!x_bf16 || !codes || !sf)) return NVFP4_ERR_INVALID_ARG;
     if (k % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (rows > (int64_t)1 << 31 || k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (rows > kQuantMaxRows || k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     const bool given = (flags & NVFP4_SCALE_GIVEN) != 0u;
     if (!given && (!workspace || workspace_bytes < kQuantWorkspaceBytes)) return NVFP4_ERR_WORKSPACE;
     if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(sf) || (ld_x % 8) != 0 ||
@@ -220,7 +220,7 @@ nvfp4_status nvfp4_fake_quantize(const void* x_bf16, int64_t rows, int64_t k, in
     if (!tensor_scale) return NVFP4_ERR_INVALID_ARG;
     if (rows > 0 && (!x_bf16 || !y)) return NVFP4_ERR_INVALID_ARG;
     if (k % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (rows > (int64_t)1 << 31 || k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (rows > kQuantMaxRows || k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     const bool given = (flags & NVFP4_SCALE_GIVEN) != 0u;
     if (!given && (!workspace || workspace_bytes < kQuantWorkspaceBytes)) return NVFP4_ERR_WORKSPACE;
     if (!aligned16(x_bf16) || !aligned16(y) || (clip_mask && !aligned16(clip_mask)) || (ld_x % 8) != 0 ||

@@ -12,6 +12,10 @@ constexpr int kQuantThreads = 512;
 constexpr int kFusedSlots = 512;         // one-kernel quantize: (generation, max) per CTA
 constexpr size_t kQuantWorkspaceBytes = kFusedSlots * sizeof(unsigned long long);
 static_assert(kQuantWorkspaceBytes >= kAmaxMaxCtas * sizeof(float), "workspace holds the two-kernel partials too");
+// The tile quantizer's two-kernel form puts one 128-row block per grid row
+// (gridDim.y <= 65535), so the quantize entry points accept at most this many
+// rows (checked before any launch).
+constexpr int64_t kQuantMaxRows = (int64_t)65535 * 128;
 
 void count_launch(int n);
 

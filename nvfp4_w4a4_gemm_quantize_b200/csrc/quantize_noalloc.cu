@@ -26,8 +26,10 @@
 namespace nvfp4 {
 
 // One partial maximum per CTA of the amax pass; that pass never launches more
-// than kAmaxMaxCtas CTAs, whatever the tensor size.
-constexpr int kNoAllocPartials = kAmaxMaxCtas;
+// than kAmaxMaxCtas CTAs, whatever the tensor size.  The array's size is the
+// one the public header states.
+constexpr int kNoAllocPartials = NVFP4_NOALLOC_SCRATCH_FLOATS;
+static_assert(kNoAllocPartials == kAmaxMaxCtas, "the public scratch size must cover the amax pass's partials");
 static __device__ __align__(256) float g_noalloc_partials[kNoAllocPartials];
 
 static float* g_noalloc_ptr[64];
@@ -70,7 +72,7 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows,
     if (!tensor_scale) return NVFP4_ERR_INVALID_ARG;
     if (rows > 0 && (!x_bf16 || !codes || !sf)) return NVFP4_ERR_INVALID_ARG;
     if (k % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (rows > (int64_t)1 << 31 || k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (rows > kQuantMaxRows || k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (!noalloc_aligned16(x_bf16) || !noalloc_aligned16(codes) || !noalloc_aligned16(sf) || (ld_x % 8) != 0 ||
         (reinterpret_cast<uintptr_t>(tensor_scale) & 3u))
         return NVFP4_ERR_MISALIGNED;

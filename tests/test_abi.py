@@ -86,6 +86,13 @@ def test_quantize_rejects_bad_arguments(L):
     assert q(A + 2, 128, 256, 256, B, C, A, 1, None, 0, None, None) == MISALIGNED
     assert q(A, 128, 256, 260, B, C, A, 1, None, 0, None, None) == MISALIGNED
     assert q(A, 128, 256, 256, B + 8, C, A, 1, None, 0, None, None) == MISALIGNED
+    # more rows than the tile grid can hold (65535 row blocks of 128): rejected
+    # before any launch, by every quantize entry point that takes that grid
+    big = 65535 * 128 + 1
+    assert q(A, big, 64, 64, B, C, A, 1, None, 0, None, None) == SHAPE
+    assert L.nvfp4_quantize_block(A, big, 64, 64, 32, B, C, A, 1, None, 0, None, None) == SHAPE
+    assert L.nvfp4_fake_quantize(A, big, 64, 64, B, 0, None, A, 1, None, 0, None, None) == SHAPE
+    assert L.nvfp4_quantize_noalloc(A, big, 64, 64, B, C, A, 0, None, None) == SHAPE
 
 
 def test_dequantize_rejects_bad_arguments(L):

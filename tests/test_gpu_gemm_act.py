@@ -8,8 +8,9 @@ GELU of its FP64 product within a bound built from three parts:
   * the GEMM's own tolerance (1e-5 of |row(A^)| |row(B^)| for FP32
     accumulation), times 1.13, the largest slope of GELU;
   * the activation: |0.5 v| * 2^-11 * |tanh|, bounded here by 2^-10 |v|;
-  * the output rounding (bf16: 2^-9 relative; NVFP4: one block-scale step,
-    (1 + 2^-4) max|block| / 6, as in the plain NVFP4 epilogue test).
+  * the output rounding (bf16: 2^-9 relative).  The NVFP4 output must be the
+    exact rounding of some value within that bound of the oracle's GELU
+    (tests/nvfp4_validity.py: per block scale byte and per element code).
 With exactly representable products the accumulation term vanishes and the
 comparison isolates the activation."""
 import numpy as np
@@ -19,6 +20,7 @@ import torch
 import oracle
 import nvfp4_w4a4_gemm_quantize_b200 as nv
 from nvfp4_w4a4_gemm_quantize_b200 import synth
+from nvfp4_validity import assert_valid_nvfp4_rounding
 
 pytestmark = pytest.mark.gpu
 
@@ -106,9 +108,9 @@ def test_gelu_nvfp4_epilogue_is_a_valid_rounding(cuda_ok, M, N, K):
     deq = nv.dequantize(q, torch.float32).cpu().numpy().astype(np.float64)
     torch.cuda.synchronize()
     val = GELU_SLOPE * TOL_F32 * _den(a, b) + ACT_ERR * np.abs(v)
-    blk = (np.abs(g) + val).reshape(M, N // 16, 16).max(axis=2)
-    bound = np.repeat(blk * (1 + 2.0 ** -4) / 6.0, 16, axis=1) + val
-    assert np.all(np.abs(deq - g) <= bound)
+    assert_valid_nvfp4_rounding(q.codes.cpu().numpy(), oracle.sf_matrix(q.sf.cpu().numpy(), M, N), gy, g, val)
+    assert np.all(np.abs(deq - g) <= np.repeat((np.abs(g) + val).reshape(M, N // 16, 16).max(axis=2)
+                                               * (1 + 2.0 ** -4) / 6.0, 16, axis=1) + val)
     assert abs(amax.item() - np.abs(g).max()) <= val.max() + 1e-6 * np.abs(g).max()
 
 

@@ -807,3 +807,55 @@ def test_attention_one_hot_selects_the_matching_key():
     vd = oracle.dequantize(*v)
     for i in range(Lq):
         assert np.allclose(o[i], vd[(3 * i) % Lk], rtol=1e-12, atol=1e-12)
+
+
+def _tensor_scale_bf16_strided(bits: np.ndarray, k: int) -> np.float32:
+    """Call the oracle's bf16 tensor scale on the first k columns of a wider
+    row-major buffer (row stride = the buffer's width)."""
+    bits = np.ascontiguousarray(bits, np.uint16)
+    rows, ld = bits.shape
+    return np.float32(oracle.lib().oracle_tensor_scale_bf16(bits.ctypes.data, rows, k, ld))
+
+
+def _numpy_scale(bits: np.ndarray) -> np.float32:
+    """Independent value: numpy's float32 max |x| over the bf16 values, then
+    one IEEE float32 division by 6 * 448 (RFC, Motivation: one FP32 scale per
+    tensor; the tensor maximum maps onto 2688)."""
+    f = (bits.astype(np.uint32) << 16).view(np.float32)
+    return np.float32(np.max(np.abs(f))) / np.float32(2688.0) if f.size else np.float32(0.0)
+
+
+def test_tensor_scale_bf16_pinned_by_numpy():
+    rng = np.random.default_rng(11)
+    # bf16 bits by truncation of float32 (the test only needs some bf16 values)
+    f32 = lambda a: (np.asarray(a, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    # strided views: padding columns beyond k hold a value larger than any inside
+    for rows, k, ld in [(7, 64, 80), (130, 256, 264), (1, 1024, 1024)]:
+        x = f32(rng.standard_normal((rows, ld)) * 3.0)
+        x[:, k:] = f32(1e30)
+        inner = x[:, :k]
+        got = _tensor_scale_bf16_strided(x, k)
+        assert got.view(np.uint32) == _numpy_scale(inner).view(np.uint32)
+        # the maximum is in the last row and column
+        y = x.copy()
+        y[-1, k - 1] = f32(-1e4)
+        top = (np.uint32(y[-1, k - 1] & 0x7FFF) << 16).view(np.float32)
+        assert _tensor_scale_bf16_strided(y, k) == _numpy_scale(y[:, :k]) == top / np.float32(2688.0)
+    # a negative maximum magnitude
+    x = f32([[-5.0] + [1.0] * 63])
+    assert _tensor_scale_bf16_strided(x, 64) == np.float32(5.0) / np.float32(2688.0)
+    # -0 everywhere, +0 everywhere: g = +0
+    for z in (0x8000, 0x0000):
+        g = _tensor_scale_bf16_strided(np.full((3, 64), z, np.uint16), 64)
+        assert g == 0 and not np.signbit(g)
+    # bf16 subnormals: amax itself subnormal, quotient rounded (or flushed) by IEEE float32 rules
+    for top in (0x0001, 0x0007, 0x007F, 0x0080):
+        x = np.zeros((2, 64), np.uint16)
+        x[1, 5] = top
+        x[0, 3] = 0x8000 | max(top - 1, 0)
+        assert _tensor_scale_bf16_strided(x, 64).view(np.uint32) == _numpy_scale(x).view(np.uint32)
+    # every finite bf16 magnitude as the maximum of a small tensor (sampled)
+    for b in range(0, 0x7F80, 97):
+        x = np.zeros((1, 64), np.uint16)
+        x[0, 63] = b | 0x8000
+        assert _tensor_scale_bf16_strided(x, 64).view(np.uint32) == _numpy_scale(x).view(np.uint32)

@@ -54,6 +54,11 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls(cuda_ok):
         assert np.float32(g0) == np.float32(g1)
         assert np.array_equal(c0, c1)
         assert np.array_equal(s0, s1)
+    # after nvfp4_shutdown() the scratch address is looked up again: still the same results
+    L.nvfp4_shutdown()
+    x = synth.random_bf16((1024, 2048), seed=35, dist="student_t3", device="cuda")
+    (c0, s0, g0), (c1, s1, g1) = _quantize_both(L, x)
+    assert np.float32(g0) == np.float32(g1) and np.array_equal(c0, c1) and np.array_equal(s0, s1)
     # with a caller-given tensor scale (no scratch involved) the two agree too
     x = synth.random_bf16((256, 512), seed=34, device="cuda")
     (c0, s0, g0), (c1, s1, g1) = _quantize_both(L, x, given_scale=1e-3)
