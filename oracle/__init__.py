@@ -36,6 +36,10 @@ Parity status per function:
   attention                                             -- pinned (float64
       library attention of the dequantized operands, rows of p summing to
       one, invariance under the per-head term, a one-hot case)
+  layernorm / layernorm_quantize                        -- pinned (torch's
+      float64 layer_norm within the FP32 rounding of the normalisation,
+      zero-mean / unit-variance rows, constant rows, the per-group affine
+      against explicit rows, planted mistakes; the quantization is quantize)
   gelu_tanh                                             -- pinned (torch's
       float64 tanh-form GELU, the odd-part identity g(v) - g(-v) = v, the erf
       form within 1e-3, limits)
@@ -116,6 +120,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_attention_rows.argtypes = [_p, _p, _f32, _p, _p, _f32, _p, _p, _f32, _i64, _i64, _i64, _p, _i64,
                                             _i64, _i64, _p]
         L.oracle_attention_rows.restype = None
+        L.oracle_layernorm_f32.argtypes = [_p, _i64, _i64, _i64, _p, _p, _i64, ctypes.c_double, _p]
+        L.oracle_layernorm_f32.restype = None
         L.oracle_gelu_tanh.argtypes = [ctypes.c_double]
         L.oracle_gelu_tanh.restype = ctypes.c_double
         L.oracle_gelu_tanh_array.argtypes = [_p, _i64, _p]
@@ -296,6 +302,31 @@ def tensor_scale(x) -> np.float32:
     xb = bf16_bits(x)
     rows, k = xb.shape
     return np.float32(L.oracle_tensor_scale_bf16(_ptr(xb), rows, k, k))
+
+
+# ---------------------------------------------------------------- LayerNorm
+def layernorm(x, gamma=None, beta=None, rows_per_group: int = 0, eps: float = 1e-6) -> np.ndarray:
+    """LayerNorm over the last axis of a bf16 tensor with an optional affine per
+    group of rows (the DiT pre-norm and its adaLN modulation; a reading, the
+    pages do not define it): double statistics in index order, FP32
+    normalisation, one rounding per operation.  gamma / beta: float32
+    [groups, k] or [k].  Returns float32 [rows, k]."""
+    L = lib()
+    xb = bf16_bits(x)
+    rows, k = xb.shape
+    g = None if gamma is None else np.ascontiguousarray(np.asarray(gamma, np.float32).reshape(-1, k))
+    b = None if beta is None else np.ascontiguousarray(np.asarray(beta, np.float32).reshape(-1, k))
+    y = np.empty((rows, k), np.float32)
+    L.oracle_layernorm_f32(_ptr(xb), rows, k, k, None if g is None else _ptr(g), None if b is None else _ptr(b),
+                           int(rows_per_group), float(eps), _ptr(y))
+    return y
+
+
+def layernorm_quantize(x, gamma=None, beta=None, rows_per_group: int = 0, eps: float = 1e-6,
+                       scale: float | None = None):
+    """NVFP4 quantization (``quantize``) of the FP32 LayerNorm output: the
+    fused producer's result.  Returns (codes, sf, g)."""
+    return quantize(layernorm(x, gamma, beta, rows_per_group, eps), scale)
 
 
 # ---------------------------------------------------------------- QAT

@@ -686,3 +686,47 @@ void oracle_attention_rows(const uint8_t *q_codes, const uint8_t *q_sf, float g_
     }
     free(kh); free(vh); free(z); free(qi);
 }
+
+/* ------------------------------ LayerNorm -------------------------------- */
+/* The producer of a block's first projections.  The pages name LayerNorm
+ * only as part of the DiT blocks whose linear layers run in FP4 and do not
+ * define it; the reading taken is the DiT pre-norm: LayerNorm over the hidden
+ * dimension without its own affine, followed by the adaLN modulation
+ * x (1 + scale) + shift of each sample, which is a per-channel affine shared
+ * by a group of rows.  Written out:
+ *   S1 = sum_j x_j,  S2 = sum_j x_j^2          double, in index order
+ *   mu = S1 / k,  var = max(S2 / k - mu^2, 0),  rstd = 1 / sqrt(var + eps)
+ *                                              double, one rounding per op
+ *   y_j = ((x_j - (float)mu) * (float)rstd) * gamma_j + beta_j
+ *                                              FP32, one rounding per op
+ * gamma, beta: FP32 [groups, k] (row r uses group r / rows_per_group), or
+ * NULL for 1 and 0.  Every square of a bf16 value is exact in double, and so
+ * are the sums wherever the row's values span fewer than about 45 binary
+ * orders of magnitude; then any summation order gives these S1 and S2.
+ * y: FP32 [rows, k] contiguous.                                              */
+void oracle_layernorm_f32(const uint16_t *x, int64_t rows, int64_t k, int64_t ld, const float *gamma,
+                          const float *beta, int64_t rows_per_group, double eps, float *y)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        double s1 = 0.0, s2 = 0.0;
+        for (int64_t j = 0; j < k; ++j) {
+            const double v = (double)oracle_bf16_to_f32(x[r * ld + j]);
+            s1 += v;
+            s2 += v * v;
+        }
+        const double mu = s1 / (double)k;
+        double var = s2 / (double)k - mu * mu;
+        if (var < 0.0) var = 0.0;
+        const double rstd = 1.0 / sqrt(var + eps);
+        const float mu32 = (float)mu, rstd32 = (float)rstd;
+        const int64_t grp = rows_per_group > 0 ? r / rows_per_group : 0;
+        for (int64_t j = 0; j < k; ++j) {
+            const float xv = oracle_bf16_to_f32(x[r * ld + j]);
+            float v = xv - mu32;
+            v = v * rstd32;
+            if (gamma) v = v * gamma[grp * k + j];
+            if (beta) v = v + beta[grp * k + j];
+            y[r * k + j] = v;
+        }
+    }
+}

@@ -859,3 +859,74 @@ def test_tensor_scale_bf16_pinned_by_numpy():
         x = np.zeros((1, 64), np.uint16)
         x[0, 63] = b | 0x8000
         assert _tensor_scale_bf16_strided(x, 64).view(np.uint32) == _numpy_scale(x).view(np.uint32)
+
+
+# ---------------------------------------------------------------- LayerNorm (fused producer)
+def _ln_inputs(rows, k, seed, dist, groups):
+    x = synth.random_bf16((rows, k), seed=seed, dist=dist)
+    rng = np.random.default_rng(seed)
+    gamma = (1.0 + 0.5 * rng.standard_normal((groups, k))).astype(np.float32)
+    beta = (0.3 * rng.standard_normal((groups, k))).astype(np.float32)
+    return x, gamma, beta
+
+
+def _ln_library(x, gamma, beta, rows_per_group, eps):
+    """torch's float64 layer_norm (library routine), one group of rows at a time."""
+    xf = torch.from_numpy(oracle.bf16_to_f32(oracle.bf16_bits(x)).astype(np.float64))
+    rows, k = xf.shape
+    out = torch.empty_like(xf)
+    for r0 in range(0, rows, rows_per_group or rows):
+        r1 = min(rows, r0 + (rows_per_group or rows))
+        gi = r0 // rows_per_group if rows_per_group else 0
+        w = None if gamma is None else torch.from_numpy(gamma[gi].astype(np.float64))
+        b = None if beta is None else torch.from_numpy(beta[gi].astype(np.float64))
+        out[r0:r1] = torch.nn.functional.layer_norm(xf[r0:r1], (k,), w, b, eps)
+    return out.numpy(), xf.numpy()
+
+
+@pytest.mark.parametrize("rows,k,dist,groups,affine", [(37, 1152, "outlier", 5, True), (8, 3072, "token_scaled", 2, True),
+                                                        (16, 256, "student_t3", 1, False), (3, 5120, "normal", 3, True)])
+def test_layernorm_vs_library(rows, k, dist, groups, affine):
+    x, gamma, beta = _ln_inputs(rows, k, rows + k, dist, groups)
+    rpg = -(-rows // groups)
+    g, b = (gamma, beta) if affine else (None, None)
+    y = oracle.layernorm(x, g, b, rpg if affine else 0, 1e-6)
+    ref, xf = _ln_library(x, g, b, rpg if affine else 0, 1e-6)
+    mu = xf.mean(axis=1, keepdims=True)
+    rstd = 1.0 / np.sqrt(xf.var(axis=1, keepdims=True) + 1e-6)
+    gam = np.repeat(g, rpg, axis=0)[:rows].astype(np.float64) if affine else 1.0
+    bet = np.repeat(b, rpg, axis=0)[:rows].astype(np.float64) if affine else 0.0
+    # FP32 normalisation: a few roundings of |x - mu| rstd |gamma|, of the
+    # rounded mean and of the shift
+    tol = 2.0 ** -20 * ((np.abs(xf - mu) + np.abs(mu)) * rstd * np.abs(gam) + np.abs(bet)) + 1e-30
+    assert np.all(np.abs(y.astype(np.float64) - ref) <= tol)
+
+
+def test_layernorm_rows_are_standardized_and_constant_rows_give_beta():
+    x = synth.random_bf16((64, 1152), seed=9, dist="token_scaled")
+    y = oracle.layernorm(x).astype(np.float64)
+    xf = oracle.bf16_to_f32(oracle.bf16_bits(x)).astype(np.float64)
+    v = xf.var(axis=1)
+    assert np.all(np.abs(y.mean(axis=1)) <= 1e-6)
+    assert np.all(np.abs(y.var(axis=1) - v / (v + 1e-6)) <= 1e-5)
+    # a constant row normalises to exact zeros, so the output is beta itself
+    c = np.full((2, 256), 0x4049, np.uint16)                      # bf16 3.140625
+    beta = np.linspace(-1, 1, 256, dtype=np.float32)[None, :]
+    gamma = np.full((1, 256), 2.5, np.float32)
+    yc = oracle.layernorm(c, gamma, beta, 2, 1e-6)
+    assert np.array_equal(yc, np.repeat(beta, 2, axis=0))
+
+
+def test_layernorm_groups_match_rows_taken_one_group_at_a_time():
+    x, gamma, beta = _ln_inputs(12, 512, 4, "outlier", 3)
+    y = oracle.layernorm(x, gamma, beta, 4, 1e-6)
+    for gi in range(3):
+        yi = oracle.layernorm(x[4 * gi:4 * gi + 4], gamma[gi], beta[gi], 0, 1e-6)
+        assert np.array_equal(y[4 * gi:4 * gi + 4], yi)
+
+
+def test_layernorm_quantize_is_quantize_of_the_layernorm():
+    x, gamma, beta = _ln_inputs(130, 1152, 5, "student_t3", 1)
+    c, s, g = oracle.layernorm_quantize(x, gamma, beta, 0, 1e-6)
+    c2, s2, g2 = oracle.quantize(oracle.layernorm(x, gamma, beta, 0, 1e-6))
+    assert g == g2 and np.array_equal(c, c2) and np.array_equal(s, s2)
