@@ -29,6 +29,7 @@ cudaError_t launch_gemm_w4a4(const GemmW4A4Args& a, int num_sms, cudaStream_t st
 cudaError_t launch_gemm_w4a4_grouped(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream);
 int gemm_w4a4_max_group();
 cudaError_t launch_gemm_w4a4_2sm(const GemmW4A4Args& a, int num_sms, cudaStream_t stream);
+bool gemm_w4a4_2sm_supports(int64_t N);
 
 struct GemmW4A16Args {
     const uint16_t* x;

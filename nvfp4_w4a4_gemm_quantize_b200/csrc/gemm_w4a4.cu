@@ -27,6 +27,7 @@
 // one tile overlaps the mainloop of the next), the scale ring in [256, 512).
 #include <cstring>
 
+#include <cstdlib>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -519,10 +520,18 @@ static cudaError_t launch_group(const GemmW4A4Args* probs, int count, int num_sm
 cudaError_t launch_gemm_w4a4(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) {
     using namespace w4a4;
     if (a.M == 0) return cudaSuccess;
-    // N a multiple of 256: CTA-pair kernel with 256 x 256 tiles.  Otherwise
-    // (N = 1152, 3456, ...): single-CTA 128 x 128 tiles with a double-buffered
-    // accumulator, so no tile column is wasted on padding.
-    if (a.N % 256 == 0) return launch_gemm_w4a4_2sm(a, num_sms, stream);
+    // N a multiple of 192 or 256: CTA-pair kernel (256 x 192 or 256 x 256
+    // tiles) when there are enough pair tiles to fill the GPU; otherwise
+    // single-CTA 128 x 128 tiles with a double-buffered accumulator, whose
+    // finer tiles waste less of a small problem.  NVFP4_GEMM_KERNEL=pair or
+    // =single overrides the choice (where the shape allows) for measurements.
+    const char* env = getenv("NVFP4_GEMM_KERNEL");
+    const int forced = env ? (env[0] == 'p' ? 1 : env[0] == 's' ? 2 : 0) : 0;
+    if (gemm_w4a4_2sm_supports(a.N) && forced != 2) {
+        const int64_t bn = a.N % 256 == 0 ? 256 : 192;
+        const int64_t pair_tiles = ((a.M + 255) / 256) * (a.N / bn);
+        if (forced == 1 || pair_tiles >= num_sms / 2) return launch_gemm_w4a4_2sm(a, num_sms, stream);
+    }
     return launch_gemm_w4a4_grouped(&a, 1, num_sms, stream);
 }
 

@@ -1,34 +1,46 @@
 // gemm_w4a4_2sm.cu -- the W4A4 GEMM on CTA pairs (tcgen05 cta_group::2):
-// one 256 x 256 output tile per pair, each CTA holding 128 rows of A, one
-// 128-row half of B and the full 256-row set of B scales; per K step the
-// leader CTA issues a single M=256, N=256, K=64 block-scaled MMA whose
-// accumulator rows land in both CTAs' TMEM.
+// one 256 x BN output tile per pair (BN = 192 or 256), each CTA holding 128
+// rows of A, one BN/2-row half of B and the scales of every B row of the
+// tile; per K step the leader CTA issues a single M=256, N=BN, K=64
+// block-scaled MMA whose accumulator rows land in both CTAs' TMEM.
 //
 // Same operation as gemm_w4a4.cu ("NVFP4-DiT ..." README, Methodology 3;
 // "[RFC]: NVFP4 Quantization Support for Diffusion Models", Open Questions 1):
 //   Y[m,n] = (g_a g_b) * sum_k (e2m1(a) e4m3(sfa)) (e2m1(b) e4m3(sfb))
 //
 // Why pairs: per SM, a 128 x 256 x 256 K-stage needs 38 KB of operands
-// instead of 54 KB for a single-CTA 128 x 256 tile, so five stages fit in
-// shared memory, and L2 -> SM operand traffic per output drops by a third.
+// instead of 54 KB for a single-CTA 128 x 256 tile, and L2 -> SM operand
+// traffic per output drops by a third.
+//
+// Why BN = 192: TMEM has 512 columns.  A 256-wide tile's FP32 accumulator
+// takes 256 of them and the scale atoms of a stage 48 more, so a second
+// accumulator cannot fit and every tile boundary waits for the epilogue to
+// drain TMEM (about 1.5-2 k cycles per tile).  With BN = 192 two
+// accumulators (384 columns) and a two-slot scale ring (96 columns) fit: the
+// next tile's MMAs run while the epilogue drains the previous one.  A 192-row
+// B tile starts half-way into a 128-row scale atom on odd tiles; the atoms
+// are copied whole and the MMA's B-scale address is moved two columns on
+// (one TMEM column holds the scales of 32 B rows).
 //
 // Roles (512 threads per CTA):
 //   warp 0     producer, both CTAs: TMA loads of this CTA's scale atoms (its
-//              128 A rows, all 256 B rows), A rows and B half into a
-//              STAGES-deep ring.  Every load of the pair completes on the
-//              LEADER's full barrier (cta_group::2), which the leader arms
-//              with the bytes of both CTAs: one wait per stage tells the MMA
-//              issuer that both CTAs' operands have landed.
-//   warp 2     leader CTA: scale copier.  Per K=64 step three tcgen05.cp of
-//              the scale atoms into the stage's TMEM columns; one commit per
-//              stage to the leader's "scaled" barrier.
+//              128 A rows, both 128-row atom blocks the tile's B rows touch),
+//              A rows and B half into a STAGES-deep ring.  Every load of the
+//              pair completes on the LEADER's full barrier (cta_group::2),
+//              which the leader arms with the bytes of both CTAs: one wait
+//              per stage tells the MMA issuer that both CTAs' operands landed.
+//   warp 2     leader CTA, 256-wide tiles: scale copier.  Per K=64 step three
+//              tcgen05.cp of the scale atoms into the stage's TMEM scale slot;
+//              one commit per stage to the leader's "scaled" barrier.  With
+//              192-wide tiles (two slots) the MMA warp issues the same copies
+//              itself, just before the stage's MMAs.
 //   warp 1     leader CTA: MMA issuer.  Per K=64 step one tcgen05.mma
 //              cta_group::2; one commit per stage, multicast to both CTAs'
-//              "empty" barriers.
-//   warps 8-15 epilogue, both CTAs: the 128 x 256 FP32 accumulator slice is
-//              read into registers (two warps per TMEM lane quarter, 128
+//              "empty" barriers; one per tile to the accumulator's "full".
+//   warps 8-15 epilogue, both CTAs: the 128 x BN FP32 accumulator slice is
+//              read into registers (two warps per TMEM lane quarter, BN/2
 //              columns each) and released to the MMA issuer at once, then
-//              converted and stored while the next tile's mainloop runs.
+//              converted and stored while the mainloop runs.
 // Producer, copier and MMA issuer run on whole warps with one elected lane
 // issuing: the descriptors, coordinates and addresses then stay warp-uniform.
 // Issued from a single lane, the same copies and MMAs took longer to issue
@@ -38,8 +50,10 @@
 // tcgen05.wait::ld and tcgen05.fence::before_thread_sync (a cluster-scope
 // release costs about a microsecond per arrive).
 // Registers: launched at 128 per thread; warpgroups 0-1 drop to 56 and the
-// epilogue warpgroups rise to 200 (256 x 56 + 256 x 200 = 512 x 128).
+// epilogue warpgroups rise to 200 (256 x 56 + 256 x 200 = 512 x 128); 80 and
+// 176 with 192-wide tiles.
 // No load uses cluster multicast: every CTA fetches its own tiles.
+#include <cstdlib>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -56,14 +70,19 @@ namespace w4a4_2sm {
 
 constexpr int BK_BYTES = 128;                    // 256 FP4 values per row per stage
 constexpr int A_BYTES = 128 * BK_BYTES;          // this CTA's 128 rows of A
-constexpr int B_BYTES = 128 * BK_BYTES;          // this CTA's 128-row half of B
 constexpr int SF_ATOM = 512;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 512;
-constexpr int kRegsLow = 56;                     // warpgroups 0-1
-constexpr int kRegsHigh = 200;                   // epilogue warpgroups 2-3
-static_assert(256 * kRegsLow + 256 * kRegsHigh <= kThreads * 128, "register split exceeds the launch budget");
-constexpr int SF_COLS_ATOM = 4 + 8;              // SFA 4 columns, SFB 8 columns per scale atom
+// register split (setmaxnreg): warpgroups 0-1 (producer, MMA, copier) drop
+// to REGS_LOW, the epilogue warpgroups 2-3 rise to REGS_HIGH; a 256-wide
+// tile's epilogue holds 128 accumulator columns per thread, a 192-wide one 96
+template <int BN>
+struct Regs {
+    static constexpr int LOW = BN == 192 ? 80 : 56;
+    static constexpr int HIGH = BN == 192 ? 176 : 200;
+    static_assert(256 * LOW + 256 * HIGH <= kThreads * 128, "register split exceeds the launch budget");
+};
+constexpr int SF_COLS_ATOM = 4 + 8;              // SFA 4 columns, SFB 8 columns (two 128-row atoms) per scale atom
 constexpr int kGroupM = 8;                       // rasterisation group, in 256-row pair tiles
 constexpr int kSmemLimit = 232448;
 
@@ -72,27 +91,46 @@ enum OutKind { OUT_BF16 = 0, OUT_F32 = 1, OUT_NVFP4 = 2 };
 // Per-stage layout.  NVFP4 (kind::mxf4nvf4, block16): a 128-row scale atom
 // covers K = 64, four per stage.  MX (kind::mxf4, block32): an atom covers
 // K = 128, two per stage; each K = 64 MMA step reads two of a row's four
-// scale bytes, selected by a byte id.
-template <bool MXS>
+// scale bytes, selected by a byte id.  B scales: the two 128-row atom blocks
+// that the tile's BN rows touch.
+template <int BN, bool MXS>
 struct Lay {
+    static_assert(BN == 192 || BN == 256, "pair tile width");
+    static constexpr int B_ROWS = BN / 2;                         // this CTA's half of the tile's B rows
+    static constexpr int B_BYTES = B_ROWS * BK_BYTES;
     static constexpr int SF_PER = MXS ? 2 : 4;   // scale atoms per 128 rows per stage
     static constexpr int K_ATOM = MXS ? 128 : 64;
     static constexpr int SFA_BYTES = SF_PER * SF_ATOM;            // this CTA's 128 A rows
-    static constexpr int SFB_BYTES = 2 * SFA_BYTES;               // all 256 B rows
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // 38912 (NVFP4)
+    static constexpr int SFB_BYTES = 2 * SFA_BYTES;               // two 128-row blocks of B
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // NVFP4: 38912 / 34816
     static constexpr int SF_COLS_STAGE = SF_PER * SF_COLS_ATOM;
+    static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 128-byte-swizzled tiles 1024-byte aligned");
 };
 
-template <int OUT, bool MXS>
+template <int BN, int OUT, bool MXS>
 struct Cfg {
-    static constexpr int STAGE_BYTES = Lay<MXS>::STAGE_BYTES;
+    using L = Lay<BN, MXS>;
+    static constexpr int STAGE_BYTES = L::STAGE_BYTES;
     static constexpr int EPI_BUF = OUT == OUT_F32 ? 4096 : (OUT == OUT_BF16 ? 2048 : 0);   // 32 rows x 32 cols
     static constexpr int EPI_BYTES = kEpiWarps * 2 * EPI_BUF;
     static constexpr int FIT = (kSmemLimit - 1024 - EPI_BYTES) / STAGE_BYTES;
-    static constexpr int STAGES = FIT < 5 ? FIT : 5;
+    static constexpr int MAX_STAGES = BN == 192 ? 6 : 5;
+    static constexpr int STAGES = FIT < MAX_STAGES ? FIT : MAX_STAGES;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024;
+    // BN = 192: two accumulators and two scale slots; BN = 256: one
+    // accumulator and a scale slot per stage
+    static constexpr int ACC_BUFS = BN == 192 ? 2 : 1;
+    static constexpr int SF_SLOTS = BN == 192 ? 2 : STAGES;
+    // who copies the scale atoms into TMEM: with a slot per stage, a separate
+    // copier warp; with two slots, the MMA warp itself, right before the
+    // stage's MMAs (tcgen05 copies and MMAs issued by one thread execute in
+    // issue order, so a copy into a slot cannot overtake the MMAs that read it
+    // two stages earlier, and no barrier round trip sits between stages)
+    static constexpr bool COPY_IN_MMA = SF_SLOTS < STAGES;
+    static constexpr int EPI_COLS = BN / 2;                       // accumulator columns per epilogue warp
     static_assert(STAGES >= 3, "pipeline depth");
-    static_assert(256 + STAGES * Lay<MXS>::SF_COLS_STAGE <= 512, "TMEM columns");
+    static_assert(ACC_BUFS * BN + SF_SLOTS * L::SF_COLS_STAGE <= 512, "TMEM columns");
+    static_assert(EPI_COLS % 32 == 0, "epilogue chunks of 32 columns");
 };
 
 struct Params {
@@ -154,11 +192,11 @@ __device__ __forceinline__ void store_chunk(const uint32_t* r, float alpha, uint
     }
 }
 
-// Scale atom `at` of a stage of the pair (A: 128 rows of this CTA, B: all
-// 256 rows, in both CTAs) into the atom's TMEM columns.
-template <bool MXS>
+// Scale atom `at` of a stage of the pair (A: 128 rows of this CTA, B: the
+// tile's two 128-row atom blocks, in both CTAs) into the atom's TMEM columns.
+template <int BN, bool MXS>
 __device__ __forceinline__ void k_copy_scales(uint32_t sfs, uint32_t sf_col, int at) {
-    using L = Lay<MXS>;
+    using L = Lay<BN, MXS>;
     const uint32_t col = sf_col + at * SF_COLS_ATOM;
     tc_cp2_32x128b_warpx4(col, sdesc_sf(sfs + at * SF_ATOM));
     tc_cp2_32x128b_warpx4(col + 4, sdesc_sf(sfs + L::SFA_BYTES + at * SF_ATOM));
@@ -167,37 +205,44 @@ __device__ __forceinline__ void k_copy_scales(uint32_t sfs, uint32_t sf_col, int
 
 // One K=64 step of the pair: the block-scaled MMA reading the step's scale
 // columns (MX: the atom of steps 2i and 2i + 1, bytes 0-1 or 2-3 of each row's
-// scale word).
-template <bool MXS>
-__device__ __forceinline__ void k_mma(uint32_t tmem_acc, uint32_t sb, uint32_t sf_col, int ks, uint32_t idesc,
-                                      bool accumulate) {
+// scale word).  One TMEM column holds the scales of 32 B rows, so a tile
+// whose first B row lies `sfb_off` * 32 rows into its first atom block reads
+// B scales from `sfb_off` columns further on.
+template <int BN, bool MXS>
+__device__ __forceinline__ void k_mma(uint32_t tmem_acc, uint32_t sb, uint32_t sf_col, uint32_t sfb_off, int ks,
+                                      uint32_t idesc, bool accumulate) {
     const uint64_t ad = sdesc_kmajor_sw128(sb + ks * 32), bd = sdesc_kmajor_sw128(sb + A_BYTES + ks * 32);
     if (MXS) {
         const uint32_t col = sf_col + (ks >> 1) * SF_COLS_ATOM, byte = (uint32_t)(ks & 1) * 2u;
-        tc_mma2_mxf4(tmem_acc, ad, bd, idesc | (byte << 29) | (byte << 4), col | (byte << 30), (col + 4) | (byte << 30),
-                     accumulate ? 1u : 0u);
+        tc_mma2_mxf4(tmem_acc, ad, bd, idesc | (byte << 29) | (byte << 4), col | (byte << 30),
+                     (col + 4 + sfb_off) | (byte << 30), accumulate ? 1u : 0u);
     } else {
         const uint32_t col = sf_col + ks * SF_COLS_ATOM;
-        tc_mma2_nvf4(tmem_acc, ad, bd, idesc, col, col + 4, accumulate ? 1u : 0u);
+        tc_mma2_nvf4(tmem_acc, ad, bd, idesc, col, col + 4 + sfb_off, accumulate ? 1u : 0u);
     }
 }
 
-template <int OUT, int ACT, bool MXS>
+template <int BN, int OUT, int ACT, bool MXS>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
              const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
              const __grid_constant__ CUtensorMap tmap_y, const Params p) {
-    using C = Cfg<OUT, MXS>;
-    using L = Lay<MXS>;
+    using C = Cfg<BN, OUT, MXS>;
+    using L = Lay<BN, MXS>;
     constexpr int STAGES = C::STAGES;
     constexpr int STAGE_BYTES = L::STAGE_BYTES;
+    constexpr int ACC_BUFS = C::ACC_BUFS;
+    constexpr int SF_SLOTS = C::SF_SLOTS;
+    constexpr int EPI_COLS = C::EPI_COLS;
     extern __shared__ uint8_t smem_raw[];
     // full:   the leader's; both CTAs' operand tiles and scale atoms of a stage
     //         have landed (the peer's loads signal it through cta_group::2);
     // scaled: the leader's; the stage's scale atoms are in both CTAs' TMEM;
-    // empty:  both CTAs'; the MMAs of a stage have completed.
+    // empty:  both CTAs'; the MMAs of a stage have completed;
+    // accf:   both CTAs'; an accumulator holds a finished tile;
+    // acce:   the leader's; both CTAs' epilogues have read an accumulator.
     __shared__ __align__(8) uint64_t full_bar[STAGES], scaled_bar[STAGES], empty_bar[STAGES];
-    __shared__ __align__(8) uint64_t accf_bar, acce_bar, drain_bar;
+    __shared__ __align__(8) uint64_t accf_bar[ACC_BUFS], acce_bar[ACC_BUFS], drain_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
 
@@ -215,8 +260,10 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
             mbar_init(&scaled_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
         }
-        mbar_init(&accf_bar, 1);
-        mbar_init(&acce_bar, 2 * kEpiWarps);
+        for (int b = 0; b < ACC_BUFS; ++b) {
+            mbar_init(&accf_bar[b], 1);
+            mbar_init(&acce_bar[b], 2 * kEpiWarps);
+        }
         mbar_init(&drain_bar, 1);
         fence_barrier_init();
         tma_prefetch_desc(&tmap_a);
@@ -228,7 +275,7 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     // scale regions start as zeros (finite) so rows that are never loaded
     // (beyond M or N) multiply zero codes by a finite scale
     for (int s = 0; s < STAGES; ++s) {
-        uint32_t* z = reinterpret_cast<uint32_t*>(smem + s * STAGE_BYTES + A_BYTES + B_BYTES);
+        uint32_t* z = reinterpret_cast<uint32_t*>(smem + s * STAGE_BYTES + A_BYTES + L::B_BYTES);
         for (int i = threadIdx.x; i < (L::SFA_BYTES + L::SFB_BYTES) / 4; i += kThreads) z[i] = 0u;
     }
     fence_proxy_async_smem();
@@ -245,12 +292,12 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     const int num_kt = (p.K + 255) / 256;
     const int k_atoms = p.K / L::K_ATOM;             // scale atoms per 128 rows
     const int k_steps = p.K / 64;                    // K = 64 MMA steps
-    const uint32_t sf_base = tmem_base + 256;
+    const uint32_t sf_base = tmem_base + ACC_BUFS * BN;
     // one register-budget change per warpgroup, before the roles diverge
     // (the epilogue code sits under the same branch as its increase, so that
     // ptxas allocates it against the raised budget)
     if (warp < 8) {
-        regs_dec<kRegsLow>();
+        regs_dec<Regs<BN>::LOW>();
         if (warp == 0) {
             // ------------------------------------------------------------ producer (both CTAs)
             const uint64_t pol_a = policy_evict_normal();
@@ -262,9 +309,10 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                 int mb2, nb;
                 tile_coords(t, p.num_mb2, p.num_nb, mb2, nb);
                 const int arow = mb2 * 256 + (int)rank * 128;
-                const int brow = nb * 256 + (int)rank * 128;
+                const int brow = nb * BN + (int)rank * L::B_ROWS;
                 const int sfa_row = (mb2 * 2 + (int)rank) * k_atoms;
-                const int sfb_row0 = (nb * 2) * k_atoms, sfb_row1 = (nb * 2 + 1) * k_atoms;
+                const int sfb_blk = (nb * BN) >> 7;          // first 128-row atom block of the tile's B rows
+                const int sfb_row0 = sfb_blk * k_atoms, sfb_row1 = (sfb_blk + 1) * k_atoms;
                 for (int kt = 0; kt < num_kt; ++kt) {
                     if (!__all_sync(0xffffffffu, mbar_wait(&empty_bar[stage], phase ^ 1u, wc) ? 1 : 0)) {
                         ok = false;
@@ -276,7 +324,7 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                         // which the leader arms with the bytes of both CTAs
                         if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * STAGE_BYTES);
                         const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
-                        uint8_t* sfs = sb + A_BYTES + B_BYTES;
+                        uint8_t* sfs = sb + A_BYTES + L::B_BYTES;
                         tma_load_2d_pair(sfs, &tmap_sfa, fb, 0, sfa_row + kt * L::SF_PER, pol_a);
                         tma_load_2d_pair(sfs + L::SFA_BYTES, &tmap_sfb, fb, 0, sfb_row0 + kt * L::SF_PER, pol_b);
                         tma_load_2d_pair(sfs + L::SFA_BYTES + L::SF_PER * SF_ATOM, &tmap_sfb, fb, 0,
@@ -300,37 +348,51 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                     if (issued_any & (1u << s)) mbar_wait(&full_bar[s], (issued >> s) & 1u, w2);
             }
         } else if (warp == 2) {
-            if (rank == 0) {
+            if (rank == 0 && !C::COPY_IN_MMA) {
                 // -------------------------------------------------------- scale copier (leader)
-                // Per stage: wait for the operands, copy the stage's scale atoms of
-                // both CTAs into TMEM, commit to the stage's "scaled" barrier.
-                // (From the MMA warp the twelve copies per stage cost issue slots
-                // that the four MMAs need: ~626 cycles per stage against ~533.)
+                // Per stage: wait for the operands (and, with fewer scale slots
+                // than stages, for the MMAs that last read the slot), copy the
+                // stage's scale atoms of both CTAs into the slot, commit to the
+                // stage's "scaled" barrier.  (From the MMA warp the twelve copies
+                // per stage cost issue slots that the four MMAs need: ~626 cycles
+                // per stage against ~533.)
                 const uint32_t smem0 = smem_u32(smem);
-                int stage = 0;
-                uint32_t phase = 0;
+                // ring positions: this stage (stage, phase), its scale slot, and
+                // the stage SF_SLOTS back, whose MMAs last read that slot
+                int stage = 0, slot = 0, wstage = 0;
+                uint32_t phase = 0, wphase = 0, done = 0;
                 bool ok = true;
                 for (int t = pair; t < p.num_tiles && ok; t += npairs) {
                     for (int kt = 0; kt < num_kt; ++kt) {
-                        if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[stage], phase, wc) ? 1 : 0)) {
+                        bool got = mbar_wait(&full_bar[stage], phase, wc);
+                        if (SF_SLOTS < STAGES && done >= (uint32_t)SF_SLOTS && got) {
+                            // that stage's barrier cannot have moved on since: its
+                            // next completion needs this stage's MMAs
+                            got = mbar_wait(&empty_bar[wstage], wphase, wc);
+                        }
+                        if (!__all_sync(0xffffffffu, got ? 1 : 0)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
-                        const uint32_t sfs = smem0 + stage * STAGE_BYTES + A_BYTES + B_BYTES;
-                        const uint32_t sf_col = sf_base + stage * L::SF_COLS_STAGE;
+                        const uint32_t sfs = smem0 + stage * STAGE_BYTES + A_BYTES + L::B_BYTES;
+                        const uint32_t sf_col = sf_base + slot * L::SF_COLS_STAGE;
                         const int nat = k_atoms - kt * L::SF_PER;
                         if (elect_one()) {
                             if (nat >= L::SF_PER) {
 #pragma unroll
-                                for (int at = 0; at < L::SF_PER; ++at) k_copy_scales<MXS>(sfs, sf_col, at);
+                                for (int at = 0; at < L::SF_PER; ++at) k_copy_scales<BN, MXS>(sfs, sf_col, at);
                             } else {
-                                for (int at = 0; at < nat; ++at) k_copy_scales<MXS>(sfs, sf_col, at);
+                                for (int at = 0; at < nat; ++at) k_copy_scales<BN, MXS>(sfs, sf_col, at);
                             }
                             tc_commit2_mc(&scaled_bar[stage], 0x1);
                         }
                         __syncwarp();
                         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                        if (++slot == SF_SLOTS) slot = 0;
+                        if (++done > (uint32_t)SF_SLOTS) {
+                            if (++wstage == STAGES) { wstage = 0; wphase ^= 1u; }
+                        }
                     }
                 }
             }
@@ -339,45 +401,62 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                 // -------------------------------------------------------- MMA issuer (leader)
                 // The whole warp runs the loop so that descriptors and addresses
                 // stay warp-uniform; one elected lane issues four MMAs per stage.
-                constexpr uint32_t idesc = MXS ? idesc_mxf4(256, 256) : idesc_nvf4(256, 256);
+                constexpr uint32_t idesc = MXS ? idesc_mxf4(256, BN) : idesc_nvf4(256, BN);
                 const uint32_t smem0 = smem_u32(smem);
-                int stage = 0;
+                int stage = 0, slot = 0, buf = 0;
                 uint32_t phase = 0, acc_phase = 0;
                 bool ok = true;
                 for (int t = pair; t < p.num_tiles && ok; t += npairs) {
-                    if (!__all_sync(0xffffffffu, mbar_wait_cluster(&acce_bar, acc_phase ^ 1u, wc) ? 1 : 0)) {
+                    int mb2, nb;
+                    tile_coords(t, p.num_mb2, p.num_nb, mb2, nb);
+                    const uint32_t sfb_off = (uint32_t)(((nb * BN) & 127) >> 5);
+                    // the accumulator's previous tile has been read out by both epilogues
+                    if (!__all_sync(0xffffffffu, mbar_wait_cluster(&acce_bar[buf], acc_phase ^ 1u, wc) ? 1 : 0)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
+                    const uint32_t tmem_acc = tmem_base + buf * BN;
                     for (int kt = 0; kt < num_kt; ++kt) {
-                        // operands landed and the stage's scales are in TMEM
-                        if (!__all_sync(0xffffffffu, mbar_wait(&scaled_bar[stage], phase, wc) ? 1 : 0)) {
+                        // operands landed (and, from the copier, the stage's scales are in TMEM)
+                        uint64_t* ready = C::COPY_IN_MMA ? &full_bar[stage] : &scaled_bar[stage];
+                        if (!__all_sync(0xffffffffu, mbar_wait(ready, phase, wc) ? 1 : 0)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                         const uint32_t sb = smem0 + stage * STAGE_BYTES;
-                        const uint32_t sf_col = sf_base + stage * L::SF_COLS_STAGE;
+                        const uint32_t sf_col = sf_base + slot * L::SF_COLS_STAGE;
                         const int nks = k_steps - kt * 4;
+                        if (C::COPY_IN_MMA && elect_one()) {
+                            const uint32_t sfs = sb + A_BYTES + L::B_BYTES;
+                            const int nat = k_atoms - kt * L::SF_PER;
+                            if (nat >= L::SF_PER) {
+#pragma unroll
+                                for (int at = 0; at < L::SF_PER; ++at) k_copy_scales<BN, MXS>(sfs, sf_col, at);
+                            } else {
+                                for (int at = 0; at < nat; ++at) k_copy_scales<BN, MXS>(sfs, sf_col, at);
+                            }
+                        }
                         if (elect_one()) {
                             if (nks >= 4) {
 #pragma unroll
                                 for (int ks = 0; ks < 4; ++ks)
-                                    k_mma<MXS>(tmem_base, sb, sf_col, ks, idesc, (kt | ks) != 0);
+                                    k_mma<BN, MXS>(tmem_acc, sb, sf_col, sfb_off, ks, idesc, (kt | ks) != 0);
                             } else {
                                 for (int ks = 0; ks < nks; ++ks)
-                                    k_mma<MXS>(tmem_base, sb, sf_col, ks, idesc, (kt | ks) != 0);
+                                    k_mma<BN, MXS>(tmem_acc, sb, sf_col, sfb_off, ks, idesc, (kt | ks) != 0);
                             }
                             tc_commit2_mc(&empty_bar[stage], 0x3);
                         }
                         __syncwarp();
                         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                        if (++slot == SF_SLOTS) slot = 0;
                     }
                     if (!ok) break;
-                    if (elect_one()) tc_commit2_mc(&accf_bar, 0x3);
+                    if (elect_one()) tc_commit2_mc(&accf_bar[buf], 0x3);
                     __syncwarp();
-                    acc_phase ^= 1u;
+                    if (++buf == ACC_BUFS) { buf = 0; acc_phase ^= 1u; }
                 }
                 if (elect_one()) tc_commit2_mc(&drain_bar, 0x1);
                 __syncwarp();
@@ -387,59 +466,59 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
             }
         }
     } else {
-        regs_inc<kRegsHigh>();
+        regs_inc<Regs<BN>::HIGH>();
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int q = warp & 3;                       // TMEM lane quarter
-        const int h = (warp - 8) >> 2;                // column half: [0,128) or [128,256)
+        const int h = (warp - 8) >> 2;                // column half: [0, BN/2) or [BN/2, BN)
         const int row_t = (int)rank * 128 + q * 32 + lane;    // row inside the pair tile
         // MX operands have no tensor scale: a null scale reads as 1
         const float alpha = __fmul_rn(p.a_scale ? *p.a_scale : 1.0f, p.b_scale ? *p.b_scale : 1.0f);
         float g_y = 0.0f;
         if (OUT == OUT_NVFP4) g_y = *p.y_scale;
         const ScaleConsts sc_y = scale_consts(g_y);
-        const uint32_t acce_addr = mapa_shared(smem_u32(&acce_bar), 0);
         uint8_t* ebuf = smem + STAGES * STAGE_BYTES + (warp - 8) * 2 * C::EPI_BUF;
+        int nstore = 0, buf = 0;
         uint32_t acc_phase = 0;
-        int nstore = 0;
         float amax_run = 0.0f;
         for (int t = pair; t < p.num_tiles; t += npairs) {
             int mb2, nb;
             tile_coords(t, p.num_mb2, p.num_nb, mb2, nb);
-            if (!__all_sync(0xffffffffu, mbar_wait(&accf_bar, acc_phase, wc) ? 1 : 0)) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(&accf_bar[buf], acc_phase, wc) ? 1 : 0)) break;
             tc_fence_after();
-            uint32_t r[128];
-            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + h * 128;
-            tmem_ld_32x32b_x32(tbase, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-            tmem_ld_32x32b_x32(tbase + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-            tmem_ld_32x32b_x32(tbase + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
-            tmem_ld_32x32b_x32(tbase + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
+            uint32_t r[EPI_COLS];
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN + h * EPI_COLS;
+#pragma unroll
+            for (int c = 0; c < EPI_COLS / 32; ++c)
+                tmem_ld_32x32b_x32(tbase + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
             tmem_ld_wait();
             // the accumulator is in registers: hand TMEM back to the MMA issuer
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
                 if (rank == 0)
-                    mbar_arrive(&acce_bar);
+                    mbar_arrive(&acce_bar[buf]);
                 else
-                    mbar_arrive_cluster_relaxed(acce_addr);
+                    mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&acce_bar[buf]), 0));
             }
-            acc_phase ^= 1u;
+            if (++buf == ACC_BUFS) { buf = 0; acc_phase ^= 1u; }
 
             const int m0 = mb2 * 256 + (int)rank * 128 + q * 32;
-            const int n0 = nb * 256 + h * 128;
+            const int n0 = nb * BN + h * EPI_COLS;
             if (OUT == OUT_NVFP4) {
+                // 32 columns (two 16-value blocks) at a time: 16 bytes of codes
+                // and two scale bytes (half a scale word) per row
                 const int64_t grow = (int64_t)mb2 * 256 + row_t;
                 const int kb4 = p.N / 64;
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const int ncol = n0 + c * 64;
+                for (int c = 0; c < EPI_COLS / 32; ++c) {
+                    const int ncol = n0 + c * 32;
                     if (ncol >= p.N) continue;
-                    uint32_t sfw = 0u, cw[8];
+                    uint32_t sfh = 0u, cw[4];
 #pragma unroll
-                    for (int b = 0; b < 4; ++b) {
+                    for (int b = 0; b < 2; ++b) {
                         float v[16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) v[j] = epi_value<ACT>(alpha, r[c * 64 + b * 16 + j]);
+                        for (int j = 0; j < 16; ++j) v[j] = epi_value<ACT>(alpha, r[c * 32 + b * 16 + j]);
                         float ab = 0.0f;
 #pragma unroll
                         for (int j = 0; j < 16; ++j) ab = fmaxf(ab, fabsf(v[j]));
@@ -451,28 +530,27 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                         for (int j = 0; j < 8; ++j) { lo[j] = v[j]; hi[j] = v[8 + j]; }
                         cw[2 * b] = quantize8(lo, s);
                         cw[2 * b + 1] = quantize8(hi, s);
-                        sfw |= sfc << (8 * b);
+                        sfh |= sfc << (8 * b);
                     }
-                    if (grow < p.M) {
-                        uint4* dst = reinterpret_cast<uint4*>(p.y_codes + grow * (p.N / 2) + ncol / 2);
-                        dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-                        dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-                    }
+                    if (grow < p.M)
+                        *reinterpret_cast<uint4*>(p.y_codes + grow * (p.N / 2) + ncol / 2) =
+                            make_uint4(cw[0], cw[1], cw[2], cw[3]);
                     // rows past M inside the padded scale buffer get zero scales
                     if (grow < (int64_t)((p.M + 127) / 128) * 128) {
                         const int rb = (int)(grow >> 7), rr = (int)(grow & 127);
                         const int64_t atom = (int64_t)rb * kb4 + ncol / 64;
-                        *reinterpret_cast<uint32_t*>(p.y_sf + atom * SF_ATOM + (rr & 31) * 16 + (rr >> 5) * 4) = sfw;
+                        *reinterpret_cast<uint16_t*>(p.y_sf + atom * SF_ATOM + (rr & 31) * 16 + (rr >> 5) * 4 +
+                                                     ((ncol >> 4) & 3)) = (uint16_t)sfh;
                     }
                 }
             } else {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < EPI_COLS / 32; ++c) {
                     if (n0 + c * 32 >= p.N) continue;
-                    uint8_t* buf = ebuf + (nstore & 1) * C::EPI_BUF;
+                    uint8_t* buf_s = ebuf + (nstore & 1) * C::EPI_BUF;
                     if (lane == 0) bulk_wait_group_read<1>();
                     __syncwarp();
-                    store_chunk<OUT, ACT>(&r[c * 32], alpha, buf, lane, &tmap_y, n0 + c * 32, m0);
+                    store_chunk<OUT, ACT>(&r[c * 32], alpha, buf_s, lane, &tmap_y, n0 + c * 32, m0);
                     ++nstore;
                 }
             }
@@ -494,17 +572,17 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     }
 }
 
-template <int OUT, int ACT, bool MXS>
+template <int BN, int OUT, int ACT, bool MXS>
 cudaError_t launch_out(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) {
-    using C = Cfg<OUT, MXS>;
-    using L = Lay<MXS>;
+    using C = Cfg<BN, OUT, MXS>;
+    using L = Lay<BN, MXS>;
     CUtensorMap ta, tb, tsa, tsb, ty;
     const uint64_t kh = (uint64_t)(a.K / 2);
     const uint64_t atoms_a = (uint64_t)((a.M + 127) / 128) * (uint64_t)(a.K / L::K_ATOM);
     const uint64_t atoms_b = (uint64_t)((a.N + 127) / 128) * (uint64_t)(a.K / L::K_ATOM);
     if (make_tmap_2d(&ta, a.a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kh, (uint64_t)a.M, kh, BK_BYTES, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
-        make_tmap_2d(&tb, a.b_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kh, (uint64_t)a.N, kh, BK_BYTES, 128,
+        make_tmap_2d(&tb, a.b_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kh, (uint64_t)a.N, kh, BK_BYTES, L::B_ROWS,
                      CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
         make_tmap_2d(&tsa, a.a_sf, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, 128, atoms_a, SF_ATOM, 128, L::SF_PER,
                      CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
@@ -529,7 +607,7 @@ cudaError_t launch_out(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) 
     p.N = (int)a.N;
     p.K = (int)a.K;
     p.num_mb2 = (int)((a.M + 255) / 256);
-    p.num_nb = (int)((a.N + 255) / 256);
+    p.num_nb = (int)(a.N / BN);
     p.num_tiles = p.num_mb2 * p.num_nb;
     p.y_codes = a.y_codes;
     p.y_sf = a.y_sf;
@@ -537,7 +615,7 @@ cudaError_t launch_out(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) 
     p.y_amax = a.y_amax;
     p.dev_status = a.dev_status;
 
-    auto kern = gemm2_kernel<OUT, ACT, MXS>;
+    auto kern = gemm2_kernel<BN, OUT, ACT, MXS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
 
@@ -565,29 +643,46 @@ cudaError_t launch_out(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) 
     return cudaGetLastError();
 }
 
-}  // namespace w4a4_2sm
-
-cudaError_t launch_gemm_w4a4_2sm(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) {
-    using namespace w4a4_2sm;
+template <int BN>
+cudaError_t launch_bn(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) {
     const bool gelu = a.act == ACT_GELU_TANH;
     if (a.mx) {
         // MX operands: bf16 or FP32 output (no NVFP4 output of an MX product)
         if (a.y == nullptr) return cudaErrorInvalidValue;
         if (a.y_dtype == 1)
-            return gelu ? launch_out<OUT_F32, ACT_GELU_TANH, true>(a, num_sms, stream)
-                        : launch_out<OUT_F32, ACT_NONE, true>(a, num_sms, stream);
-        return gelu ? launch_out<OUT_BF16, ACT_GELU_TANH, true>(a, num_sms, stream)
-                    : launch_out<OUT_BF16, ACT_NONE, true>(a, num_sms, stream);
+            return gelu ? launch_out<BN, OUT_F32, ACT_GELU_TANH, true>(a, num_sms, stream)
+                        : launch_out<BN, OUT_F32, ACT_NONE, true>(a, num_sms, stream);
+        return gelu ? launch_out<BN, OUT_BF16, ACT_GELU_TANH, true>(a, num_sms, stream)
+                    : launch_out<BN, OUT_BF16, ACT_NONE, true>(a, num_sms, stream);
     }
     if (a.y != nullptr) {
         if (a.y_dtype == 1)
-            return gelu ? launch_out<OUT_F32, ACT_GELU_TANH, false>(a, num_sms, stream)
-                        : launch_out<OUT_F32, ACT_NONE, false>(a, num_sms, stream);
-        return gelu ? launch_out<OUT_BF16, ACT_GELU_TANH, false>(a, num_sms, stream)
-                    : launch_out<OUT_BF16, ACT_NONE, false>(a, num_sms, stream);
+            return gelu ? launch_out<BN, OUT_F32, ACT_GELU_TANH, false>(a, num_sms, stream)
+                        : launch_out<BN, OUT_F32, ACT_NONE, false>(a, num_sms, stream);
+        return gelu ? launch_out<BN, OUT_BF16, ACT_GELU_TANH, false>(a, num_sms, stream)
+                    : launch_out<BN, OUT_BF16, ACT_NONE, false>(a, num_sms, stream);
     }
-    return gelu ? launch_out<OUT_NVFP4, ACT_GELU_TANH, false>(a, num_sms, stream)
-                : launch_out<OUT_NVFP4, ACT_NONE, false>(a, num_sms, stream);
+    return gelu ? launch_out<BN, OUT_NVFP4, ACT_GELU_TANH, false>(a, num_sms, stream)
+                : launch_out<BN, OUT_NVFP4, ACT_NONE, false>(a, num_sms, stream);
 }
+
+}  // namespace w4a4_2sm
+
+// N % 256 == 0: 256 x 256 tiles; otherwise (N % 192 == 0) 256 x 192 tiles
+// with a double-buffered accumulator.  A pair MMA (M = 256, K = 64) takes
+// about 120 cycles whatever its N up to 192 and 128 at N = 256, so only the
+// 256-wide tile runs the tensor cores at full rate.  NVFP4_PAIR_TILE_N (192
+// or 256) picks the tile width for measurements, where N allows it.
+cudaError_t launch_gemm_w4a4_2sm(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) {
+    using namespace w4a4_2sm;
+    const char* env = getenv("NVFP4_PAIR_TILE_N");
+    const int forced = env ? atoi(env) : 0;
+    const bool can192 = a.N % 192 == 0, can256 = a.N % 256 == 0;
+    if (can256 && (forced != 192 || !can192)) return launch_bn<256>(a, num_sms, stream);
+    if (can192) return launch_bn<192>(a, num_sms, stream);
+    return cudaErrorInvalidValue;
+}
+
+bool gemm_w4a4_2sm_supports(int64_t N) { return N % 192 == 0 || N % 256 == 0; }
 
 }  // namespace nvfp4

@@ -18,6 +18,7 @@ import oracle
 import nvfp4_w4a4_gemm_quantize_b200 as nv
 from nvfp4_w4a4_gemm_quantize_b200 import synth
 from nvfp4_validity import assert_valid_nvfp4_rounding
+from gemm_kernels import KERNELS, select_kernel
 
 pytestmark = pytest.mark.gpu
 
@@ -64,10 +65,15 @@ def _one_hot_operands(rows, K, positions, code, sfbyte):
     return c, sf
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (300, 384, 1152), (256, 512, 320)])
-def test_one_hot_pins_nibble_order_and_scale_layout(cuda_ok, M, N, K):
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (300, 384, 1152), (256, 512, 320), (300, 576, 256),
+                                   (520, 768, 512)])
+def test_one_hot_pins_nibble_order_and_scale_layout(cuda_ok, monkeypatch, kernel, M, N, K):
     """Row m of A has one non-zero at k_a(m), row n of B one at k_b(n); Y[m,n]
-    is the single product when k_a(m) == k_b(n) and exactly 0 otherwise."""
+    is the single product when k_a(m) == k_b(n) and exactly 0 otherwise.
+    N = 576 and 768 give 192-wide tiles that start half-way into a 128-row
+    scale atom (odd tiles)."""
+    select_kernel(monkeypatch, kernel, N)
     rng = np.random.default_rng(M + N + K)
     ka = rng.integers(0, K, M)
     kb = rng.integers(0, K, N)
@@ -83,9 +89,12 @@ def test_one_hot_pins_nibble_order_and_scale_layout(cuda_ok, M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 256), (1, 256, 64), (200, 384, 320), (300, 1152, 1152),
-                                   (257, 512, 4608), (600, 1152, 4096), (129, 128, 192), (64, 640, 1024)])
+                                   (257, 512, 4608), (600, 1152, 4096), (129, 128, 192), (64, 640, 1024),
+                                   (700, 960, 704)])
 @pytest.mark.parametrize("out", [torch.bfloat16, torch.float32])
-def test_random_shapes_vs_oracle(cuda_ok, M, N, K, out):
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_random_shapes_vs_oracle(cuda_ok, monkeypatch, kernel, M, N, K, out):
+    select_kernel(monkeypatch, kernel, N)
     x = synth.random_bf16((M, K), seed=M * 7 + K, dist="outlier")
     w = synth.random_bf16((N, K), seed=N * 13 + K, scale=0.02)
     e = run_and_compare(x, w, out)
@@ -151,8 +160,10 @@ def _exact_operands(rows, K, seed):
     return codes, sf
 
 
-@pytest.mark.parametrize("M,N,K", [(256, 256, 1024), (300, 384, 4096), (128, 1152, 256)])
-def test_nvfp4_epilogue_bit_exact(cuda_ok, M, N, K):
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("M,N,K", [(256, 256, 1024), (300, 384, 4096), (128, 1152, 256), (260, 768, 512)])
+def test_nvfp4_epilogue_bit_exact(cuda_ok, monkeypatch, kernel, M, N, K):
+    select_kernel(monkeypatch, kernel, N)
     ac, asf = _exact_operands(M, K, 1)
     bc, bsf = _exact_operands(N, K, 2)
     ga, gb = 0.5, 0.25
@@ -171,7 +182,8 @@ def test_nvfp4_epilogue_bit_exact(cuda_ok, M, N, K):
     assert amax.item() == np.abs(yref32).max()
 
 
-def test_nvfp4_epilogue_random_data_is_a_valid_rounding(cuda_ok):
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_nvfp4_epilogue_random_data_is_a_valid_rounding(cuda_ok, monkeypatch, kernel):
     """Random operands: the accumulation order is not fixed, so the codes are
     not unique; every scale byte and code must be the exact rounding of SOME
     FP32 value within the FP32 tolerance of the oracle's FP64 product
@@ -180,6 +192,7 @@ def test_nvfp4_epilogue_random_data_is_a_valid_rounding(cuda_ok):
     x, w = synth.layer_tensors("dit_xl2", "fc1", device="cpu")
     M, K = x.shape
     N = w.shape[0]
+    select_kernel(monkeypatch, kernel, N)
     ac, asf, ga = oracle.quantize(x)
     bc, bsf, gb = oracle.quantize(w)
     rows = np.array([0, 1, 127, 128, 1000, 2047])

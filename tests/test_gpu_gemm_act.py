@@ -21,6 +21,7 @@ import oracle
 import nvfp4_w4a4_gemm_quantize_b200 as nv
 from nvfp4_w4a4_gemm_quantize_b200 import synth
 from nvfp4_validity import assert_valid_nvfp4_rounding
+from gemm_kernels import KERNELS, select_kernel
 
 pytestmark = pytest.mark.gpu
 
@@ -49,12 +50,14 @@ def _den(a, b):
     return na * nb
 
 
-SHAPES = [(300, 512, 1152), (256, 256, 256), (300, 384, 512), (130, 1152, 4096)]   # pair and single-CTA kernels
+SHAPES = [(300, 512, 1152), (256, 256, 256), (300, 384, 512), (130, 1152, 4096), (300, 576, 512)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
-def test_gelu_epilogue_values(cuda_ok, M, N, K, out_dtype):
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_gelu_epilogue_values(cuda_ok, monkeypatch, kernel, M, N, K, out_dtype):
+    select_kernel(monkeypatch, kernel, N)
     a, b = _operands(M, N, K, 70 + M + N)
     A, B = upload(*a, M, K), upload(*b, N, K)
     y = nv.gemm_w4a4(A, B, out_dtype=out_dtype, act=nv.NVFP4_ACT_GELU_TANH)
@@ -94,8 +97,10 @@ def test_gelu_epilogue_exact_products_isolate_the_activation(cuda_ok, M, N, K):
     assert np.abs(v).max() > 4 and (np.abs(v) < 1).mean() > 0.1
 
 
-@pytest.mark.parametrize("M,N,K", [(300, 512, 1152), (300, 384, 512)])
-def test_gelu_nvfp4_epilogue_is_a_valid_rounding(cuda_ok, M, N, K):
+@pytest.mark.parametrize("M,N,K", [(300, 512, 1152), (300, 384, 512), (300, 576, 512)])
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_gelu_nvfp4_epilogue_is_a_valid_rounding(cuda_ok, monkeypatch, kernel, M, N, K):
+    select_kernel(monkeypatch, kernel, N)
     """MLP fc1 with the next layer's input emitted directly: decoded codes are a
     valid NVFP4 rounding of GELU(y), and y_amax is the largest |GELU(y)|."""
     a, b = _operands(M, N, K, 90 + N)

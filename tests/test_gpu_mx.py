@@ -10,6 +10,7 @@ import torch
 import oracle
 import nvfp4_w4a4_gemm_quantize_b200 as nv
 from nvfp4_w4a4_gemm_quantize_b200 import synth
+from gemm_kernels import KERNELS, select_kernel
 
 pytestmark = pytest.mark.gpu
 
@@ -101,12 +102,15 @@ def test_mx_gemm_one_hot(cuda_ok, m0, n0, k0):
 
 
 @pytest.mark.parametrize("m0,n0,k0", [(0, 0, 0), (200, 300, 600), (383, 511, 639), (129, 129, 129),
-                                       (255, 256, 383), (130, 7, 300)])
-def test_mx_gemm_one_hot_pair_kernel(cuda_ok, m0, n0, k0):
-    """N = 512 (CTA-pair kernel): one nonzero product lands in the right
-    output, also in the second CTA's rows, the second B half and the last,
-    half-filled K stage."""
-    M, N, K = 384, 512, 640
+                                       (255, 256, 383), (130, 7, 300), (10, 200, 64)])
+@pytest.mark.parametrize("N,kernel", [(512, "pair256"), (576, "pair192")])
+def test_mx_gemm_one_hot_pair_kernel(cuda_ok, monkeypatch, N, kernel, m0, n0, k0):
+    """CTA-pair kernels (N = 512: 256-wide tiles; N = 576: 192-wide tiles,
+    the second one starting half-way into a scale atom): one nonzero product
+    lands in the right output, also in the second CTA's rows, the second B
+    half and the last, half-filled K stage."""
+    select_kernel(monkeypatch, kernel, N)
+    M, K = 384, 640
     kb = K // 32
     ac = np.zeros((M, K // 2), np.uint8)
     bc = np.zeros((N, K // 2), np.uint8)
@@ -123,12 +127,14 @@ def test_mx_gemm_one_hot_pair_kernel(cuda_ok, m0, n0, k0):
     assert np.array_equal(oracle.mx_gemm(ac, asf, bc, bsf), expect)
 
 
-# N a multiple of 256 runs on the CTA-pair kernel (256 x 256 tiles), the rest on
-# the single-CTA kernel; K = 640 and 1152 end in a half stage (one MX scale atom)
+# every kernel the shape allows (tests/gemm_kernels.py); K = 640 and 1152 end
+# in a half stage (one MX scale atom)
 @pytest.mark.parametrize("M,N,K", [(300, 384, 1152), (128, 256, 256), (77, 1152, 640), (513, 136, 384),
                                    (300, 512, 1152), (513, 768, 640), (64, 256, 384)])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
-def test_mx_gemm_vs_oracle(cuda_ok, M, N, K, out_dtype):
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_mx_gemm_vs_oracle(cuda_ok, monkeypatch, kernel, M, N, K, out_dtype):
+    select_kernel(monkeypatch, kernel, N)
     x = synth.random_bf16((M, K), seed=M + K, dist="student_t3")
     w = synth.random_bf16((N, K), seed=N + K, dist="normal", scale=0.02)
     ac, asf = oracle.mx_quantize(x)
