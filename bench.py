@@ -146,88 +146,272 @@ def max_over_ranks(v: float, world: int, device) -> float:
 
 
 # ----------------------------------------------------------------- oracle leg
-_ORACLE_WEIGHTS = {}
+# ----------------------------------------------------------------- CPU oracle legs
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
-def oracle_sample(rows_per_layer: int, col_frac: float = 1.0):
-    """The CPU oracle on a bounded sample of the same step: for every layer,
-    quantize rows_per_layer rows of the input X and form a rows_per_layer x n
-    tile of Y = X W^T, n = col_frac of the layer's output features (a multiple
-    of 128, at least 128), against those weight rows quantized with the whole
-    weight's tensor scale (once per process, untimed).  Returns (gemm_flops,
-    seconds, description)."""
-    import numpy as np
+class OracleRunner:
+    """The CPU oracle as it stands, spread over host threads by rows.
+
+    Rows are independent once the tensor scale is known, so a tensor's rows
+    are cut into slices (for the quantizer multiples of 128 rows, so that the
+    slices' scale buffers concatenate into the whole tensor's layout) and each
+    thread calls the unchanged oracle on one slice; the oracle's C library
+    releases the GIL while it runs.  The tensor scale of a whole tensor is the largest of
+    its slices' scales (the division by 2688 is monotone and rounds once)."""
+
+    def __init__(self, threads: int):
+        from concurrent.futures import ThreadPoolExecutor
+        self.threads = max(1, threads)
+        self.pool = ThreadPoolExecutor(self.threads) if self.threads > 1 else None
+
+    def _slices(self, rows: int, align: int = 128):
+        per = -(-rows // self.threads)
+        per = max(align, -(-per // align) * align)
+        return [slice(r, min(rows, r + per)) for r in range(0, rows, per)]
+
+    def _map(self, fn, items):
+        items = list(items)
+        if self.pool is None or len(items) == 1:
+            return [fn(i) for i in items]
+        return list(self.pool.map(fn, items))
+
+    def tensor_scale(self, x):
+        import numpy as np
+        import oracle
+        return max(self._map(lambda sl: np.float32(oracle.tensor_scale(x[sl])), self._slices(x.shape[0])))
+
+    def quantize(self, x, scale=None):
+        """(codes, sf, g) of oracle.quantize(x) with a data-derived (or given) scale."""
+        import numpy as np
+        import oracle
+        g = self.tensor_scale(x) if scale is None else np.float32(scale)
+        parts = self._map(lambda sl: oracle.quantize(x[sl], scale=float(g)), self._slices(x.shape[0]))
+        return np.concatenate([p[0] for p in parts]), np.concatenate([p[1] for p in parts]), np.float32(g)
+
+    def gemm(self, a, b):
+        """Y = A B^T of two oracle-quantized operands, FP64, rows spread over threads."""
+        import numpy as np
+        import oracle
+        ac, asf, ga = a
+        bc, bsf, gb = b
+        return np.concatenate(self._map(lambda sl: oracle.gemm_w4a4(ac, asf, ga, bc, bsf, gb, rows=sl),
+                                        self._slices(ac.shape[0], align=1)))
+
+
+def _timed(fn):
+    t0 = time.perf_counter()
+    out = fn()
+    return out, time.perf_counter() - t0
+
+
+_VIDEO = {}
+
+
+def host_tensors(workload: str, layer: str):
+    """(X, W) of one layer in host memory, drawn by synth on the GPU when
+    there is one (the very tensors the GPU arm multiplies, and far faster
+    than the host generator), else on the host."""
     import torch
+    from nvfp4_w4a4_gemm_quantize_b200 import synth
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x, w = synth.layer_tensors(workload, layer, device=dev)
+    return x.cpu(), w.cpu()
+
+
+def video_tensors(runner: OracleRunner):
+    """The video workload in host memory: X per layer, and W per layer
+    quantized once by the oracle with its own tensor scale (untimed)."""
+    from nvfp4_w4a4_gemm_quantize_b200 import synth
+    if not _VIDEO:
+        for L in synth.WORKLOADS[WORKLOAD].layers:
+            x, w = host_tensors(WORKLOAD, L.name)
+            _VIDEO[L.name] = (x, runner.quantize(w))
+    return _VIDEO
+
+
+def oracle_step(runner: OracleRunner, rows: int, offset: int = 0):
+    """One step of the hot path on the host: for every video layer, quantize
+    `rows` rows of its input (data-derived tensor scale over those rows) and
+    form those rows of Y = X W^T against all output features.  Returns (GEMM
+    FLOPs, seconds)."""
+    from nvfp4_w4a4_gemm_quantize_b200 import synth
+    data = video_tensors(runner)
+    flops, secs = 0, 0.0
+    for L in synth.WORKLOADS[WORKLOAD].layers:
+        x, wq = data[L.name]
+        r0 = (offset * rows) % max(1, L.M - rows + 1)
+        xs = x[r0:r0 + rows]
+        _, dt = _timed(lambda: runner.gemm(runner.quantize(xs), wq))
+        secs += dt
+        flops += 2 * xs.shape[0] * L.N * L.K
+    return flops, secs
+
+
+def oracle_quantize_rates(runner: OracleRunner, single: OracleRunner):
+    """The oracle's quantize (data-derived scale, 4.5625 algorithmic bytes per
+    element as on the GPU) on the full fc1 and fc2 inputs with every host
+    core, and on one core on their first 8192 and 2048 rows (25 M values)."""
+    data = video_tensors(runner)
+    out = {}
+    for name in ("fc1", "fc2"):
+        x = data[name][0]
+        _, t_all = _timed(lambda: runner.quantize(x))
+        xs = x[: (1 << 25) // x.shape[1]]
+        _, t_one = _timed(lambda: single.quantize(xs))
+        out[f"{name}_input_{x.shape[0]}x{x.shape[1]}"] = {
+            "all_cores_gbs": round(QUANT_BYTES_PER_ELEM * x.numel() / t_all / 1e9, 4),
+            "one_core_gbs": round(QUANT_BYTES_PER_ELEM * xs.numel() / t_one / 1e9, 4),
+            "one_core_rows": int(xs.shape[0])}
+    return out
+
+
+def oracle_gemm_rates(runner: OracleRunner, single: OracleRunner, step_rows: int, step_secs_per_row: dict):
+    """The FP64 GEMM oracle: PR1 in full on one core, the four DiT-XL/2
+    layers in full on every core, and the video layers extrapolated to M rows
+    from the step sample."""
+    from nvfp4_w4a4_gemm_quantize_b200 import synth
+    out = {}
+    x, w = host_tensors("pr1", "linear")
+    a, b = single.quantize(x), single.quantize(w)
+    _, dt = _timed(lambda: single.gemm(a, b))
+    out["pr1_128x256x256_one_core_gflops"] = round(2 * 128 * 256 * 256 / dt / 1e9, 3)
+    fl, secs = 0, 0.0
+    for L in synth.WORKLOADS["dit_xl2"].layers:
+        x, w = host_tensors("dit_xl2", L.name)
+        a, b = runner.quantize(x), runner.quantize(w)
+        _, dt = _timed(lambda: runner.gemm(a, b))
+        fl += 2 * L.M * L.N * L.K
+        secs += dt
+    out["dit_xl2_4_layers_all_cores_gflops"] = round(fl / secs / 1e9, 3)
+    out["video_step_extrapolated_s"] = round(sum(step_secs_per_row.values()) * 32768, 1)
+    out["video_step_extrapolated_from_rows"] = step_rows
+    return out
+
+
+def epsilon_report(runner: OracleRunner):
+    """Lemma III.2's relative error bound (NVFP4-DiT README: 2^-3) next to
+    what the quantizer does on each workload's tensors (oracle quantize and
+    exact dequantize): the largest per-element |x - Q(x)| / |x| (x != 0), the
+    distribution of ||x - Q(x)|| / ||x|| over 16-value blocks, and the
+    tensor-level ||x - Q(x)||_F / ||x||_F.  Activations and weights of every
+    layer; tensors beyond 1024 rows on their first 1024 rows, quantized with
+    the whole tensor's scale."""
+    import numpy as np
     import oracle
     from nvfp4_w4a4_gemm_quantize_b200 import synth
-    wl = synth.WORKLOADS[WORKLOAD]
-    flops, secs, cols = 0, 0.0, []
-    for i, L in enumerate(wl.layers):
-        gen = torch.Generator().manual_seed(wl.seed * 1000 + i)
-        x = (torch.randn(rows_per_layer, L.K, generator=gen) *
-             torch.exp(torch.empty(rows_per_layer, 1).uniform_(np.log(0.1), np.log(10.0), generator=gen))
-             ).to(torch.bfloat16)
-        n = min(L.N, max(128, int(round(col_frac * L.N / 128)) * 128))
-        if (L.name, n) not in _ORACLE_WEIGHTS:
-            if L.name not in _ORACLE_WEIGHTS:
-                wgen = torch.Generator().manual_seed(wl.seed * 1000 + 100 + i)
-                w = (torch.randn(L.N, L.K, generator=wgen) * wl.w_std).to(torch.bfloat16)
-                _ORACLE_WEIGHTS[L.name] = (w, float(oracle.tensor_scale(w)))
-            w, gw = _ORACLE_WEIGHTS[L.name]
-            _ORACLE_WEIGHTS[(L.name, n)] = oracle.quantize(w[:n], gw)
-        bc, bsf, gb = _ORACLE_WEIGHTS[(L.name, n)]
-        t0 = time.perf_counter()
-        ac, asf, ga = oracle.quantize(x)
-        oracle.gemm_w4a4(ac, asf, ga, bc, bsf, gb)
-        secs += time.perf_counter() - t0
-        flops += 2 * rows_per_layer * n * L.K
-        cols.append(f"{L.name} {n}/{L.N}")
-    desc = (f"oracle quantize + FP64 GEMM of {rows_per_layer} activation rows (of {wl.layers[0].M}) x "
-            f"output features ({', '.join(cols)}) per {WORKLOAD} layer, 1 thread")
-    return flops, secs, desc
+
+    def stats(t, rows=1024):
+        g = runner.tensor_scale(t)
+        ts = t[:rows]
+        codes, sf, _ = runner.quantize(ts, scale=g)
+        xv = oracle.bf16_to_f32(oracle.bf16_bits(ts)).astype(np.float64)
+        e = oracle.dequantize(codes, sf, g) - xv
+        nz = xv != 0
+        blk_e = np.sqrt((e.reshape(-1, 16) ** 2).sum(1))
+        blk_x = np.sqrt((xv.reshape(-1, 16) ** 2).sum(1))
+        rb = blk_e[blk_x > 0] / blk_x[blk_x > 0]
+        return {"elem_max": float(np.max(np.abs(e[nz]) / np.abs(xv[nz]))),
+                "block_p50": float(np.percentile(rb, 50)), "block_p90": float(np.percentile(rb, 90)),
+                "block_p99": float(np.percentile(rb, 99)), "block_max": float(rb.max()),
+                "block_frac_above_eps": float((rb > 0.125).mean()),
+                "tensor": float(np.sqrt((e ** 2).sum() / (xv ** 2).sum())),
+                "rows": int(ts.shape[0]), "of_rows": int(t.shape[0])}
+
+    rep = {"eps_page": 0.125}
+    for wl in ("pr1", "dit_xl2", "pixart1024", "video_dit", "w4a16"):
+        r = {}
+        for L in synth.WORKLOADS[wl].layers:
+            if wl == WORKLOAD:
+                x, w = _VIDEO[L.name][0], None
+            else:
+                x, w = host_tensors(wl, L.name)
+            if wl != "w4a16":                        # W4A16 keeps its activations in bf16
+                r[f"{L.name}.x"] = stats(x)
+            if w is not None:
+                r[f"{L.name}.w"] = stats(w)
+        rep[wl] = r
+    return rep
+
+
+def cpu_baseline_leg(args):
+    """The cpu_baseline object of the JSON line (rank 0, N = 1): the oracle on
+    the host cores -- the headline value on a row sample of the bench step,
+    plus the quantize and GEMM rates and the error report."""
+    cores = host_cores()
+    runner, single = OracleRunner(cores), OracleRunner(1)
+    video_tensors(runner)
+    rows = max(16, min(args.ref_rows * cores, 2048))
+    per_row = {}
+    fl, secs = 0, 0.0
+    from nvfp4_w4a4_gemm_quantize_b200 import synth
+    for L in synth.WORKLOADS[WORKLOAD].layers:
+        x, wq = _VIDEO[L.name]
+        _, dt = _timed(lambda: runner.gemm(runner.quantize(x[:rows]), wq))
+        per_row[L.name] = dt / rows
+        fl += 2 * rows * L.N * L.K
+        secs += dt
+    return {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": (f"oracle quantize (data-derived scale over the sampled rows) + FP64 GEMM of the first "
+                       f"{rows} of 32768 activation rows of each {WORKLOAD} layer against all output features, "
+                       f"rows spread over {cores} host threads"),
+            "quantize": oracle_quantize_rates(runner, single),
+            "gemm": oracle_gemm_rates(runner, single, rows, per_row),
+            "epsilon": epsilon_report(runner)}
 
 
 REF_BUDGET_S = 60.0     # CPU seconds the reference arm's timed steps may take in all
-REF_PROBE_FRAC = 0.1    # output-feature fraction of the reference arm's warm-up steps
 
 
-def ref_sample_size(rows: int, steps: int, probe_secs: float, budget_s: float = REF_BUDGET_S):
-    """Rows and output-feature fraction of one reference-arm step, from the
-    time of a warm-up step on `rows` rows and REF_PROBE_FRAC of the features:
-    the cost is close to proportional to the features sampled, so the
-    fraction is scaled to keep all `steps` timed steps within the budget;
-    below one 128-feature tile of the narrowest layer the rows shrink."""
-    frac = min(1.0, REF_PROBE_FRAC * budget_s / max(1, steps) / max(probe_secs, 1e-9))
-    min_frac = 128 / 3072
-    if frac < min_frac:
-        rows = max(1, int(rows * frac / min_frac))
-        frac = min_frac
-    return rows, frac
+def ref_rows_for_budget(probe_rows: int, probe_secs: float, steps: int, budget_s: float = REF_BUDGET_S) -> int:
+    """Rows per layer of one reference-arm step, from the time of a warm-up
+    step on probe_rows rows: the cost is close to proportional to the rows,
+    so they are scaled to keep all `steps` timed steps within the budget (at
+    least one row, at most the layer)."""
+    rows = int(probe_rows * budget_s / max(1, steps) / max(probe_secs, 1e-9))
+    return max(1, min(rows, 32768))
 
 
 def run_reference(args):
-    rank, world, local = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), 0
+    rank, world = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return 0
+    cores = host_cores()
+    runner = OracleRunner(cores)
+    video_tensors(runner)
+    probe = max(16, min(args.ref_rows * cores, 2048))
     s = 0.0
     for _ in range(max(1, args.warmup)):
-        _, s, _ = oracle_sample(args.ref_rows, REF_PROBE_FRAC)
-    rows, frac = ref_sample_size(args.ref_rows, args.steps, s)
+        _, s = oracle_step(runner, probe)
+    rows = ref_rows_for_budget(probe, s, args.steps)
     fl, secs = 0, 0.0
-    desc = ""
-    for _ in range(args.steps):
-        f, s, desc = oracle_sample(rows, frac)
+    for i in range(args.steps):
+        f, dt = oracle_step(runner, rows, offset=i)
         fl += f
-        secs += s
+        secs += dt
     v = fl / secs / 1e12
+    desc = (f"oracle quantize + FP64 GEMM of {rows} of 32768 activation rows of each {WORKLOAD} layer per step "
+            f"(a different row window each step) against all output features, rows spread over {cores} host "
+            f"threads")
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": f"{WORKLOAD} (row sample)", "rows_per_layer": rows},
-            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": desc},
+            "data": "synthetic", "config": step_config(world),
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
     return 0
+
+
+def step_config(world: int) -> dict:
+    return {"workload": f"{WORKLOAD}: M=32768, qkv 3072->9216, fc1 3072->12288, fc2 12288->3072 "
+                        "(dynamic-scale activation quantize + W4A4 GEMM, bf16 out)",
+            "l2": "inputs larger than L2 (X 201-805 MB per layer, >2 GB streamed per step)",
+            "parallelism": f"replica per GPU x{world}"}
 
 
 # ----------------------------------------------------------------- extra measurements
@@ -270,6 +454,8 @@ def reference_points(dev, layers, w4a16_layers):
         del x, W, y
     out["qat"] = qat_points(dev, layers)
     out["mlp_fc1_gelu"] = mlp_fusion_points(dev, layers)
+    out["layernorm_nvfp4"] = layernorm_points(dev)
+    out["small_layers"] = small_layer_points(dev)
     out["grouped"] = grouped_points(dev)
     out["mx_and_block_size"] = mx_points(dev, layers)
     out["attention"] = attention_points(dev)
@@ -358,6 +544,123 @@ def mlp_fusion_points(dev, layers):
             "three_step_ms": round(g_ms + a_ms + q_ms, 4),
             "three_step_parts_ms": {"gemm_bf16": round(g_ms, 4), "gelu_torch": round(a_ms, 4),
                                     "quantize": round(q_ms, 4)}}
+
+
+def layernorm_points(dev):
+    """The block input's LayerNorm (adaLN: a per-sample affine) emitted as the
+    QKV projection's NVFP4 input in one kernel, data-derived tensor scale,
+    against LayerNorm + modulation in torch (bf16, a reference point only)
+    followed by the dynamic-scale quantize.  Video block input (32768 x 3072,
+    16 samples of 2048 tokens) and PixArt-1024's (8192 x 1152, 2 samples)."""
+    import torch
+    import nvfp4_w4a4_gemm_quantize_b200 as nv
+    from nvfp4_w4a4_gemm_quantize_b200 import synth
+    out = {}
+    hbm = load_peaks()[0].get("hbm_gbs", FALLBACK["hbm_gbs"])
+    for name, (M, K, groups, dist, seed) in {"video_dit": (32768, 3072, 16, "token_scaled", 31),
+                                             "pixart1024": (8192, 1152, 2, "student_t3", 32)}.items():
+        x = synth.random_bf16((M, K), seed=seed, dist=dist, device=dev)
+        gen = torch.Generator(device=dev).manual_seed(seed)
+        scale = 0.1 * torch.randn(groups, K, generator=gen, device=dev)
+        shift = 0.1 * torch.randn(groups, K, generator=gen, device=dev)
+        gamma, beta = (1.0 + scale).contiguous(), shift.contiguous()
+        q = nv.NVFP4Tensor.empty(M, K, dev)
+        ws = torch.empty(nv.nvfp4_quantize_workspace_bytes(M, K), dtype=torch.uint8, device=dev)
+        rpg = M // groups
+        fused = time_device(lambda: nv.layernorm_quantize(x, gamma, beta, rpg, 1e-6, out=q, workspace=ws))
+        g16 = gamma.to(torch.bfloat16).repeat_interleave(rpg, dim=0)
+        b16 = beta.to(torch.bfloat16).repeat_interleave(rpg, dim=0)
+
+        def ln_torch():
+            return torch.nn.functional.layer_norm(x, (K,), eps=1e-6) * g16 + b16
+        h = ln_torch()
+        ln_ms = time_device(ln_torch)
+        q_ms = time_device(lambda: nv.quantize(h, out=q, workspace=ws))
+        gbs = QUANT_BYTES_PER_ELEM * M * K / (fused * 1e-3) / 1e9
+        out[name] = {"shape": f"{M}x{K}", "samples": groups, "fused_ms": round(fused, 4),
+                     "fused_gbs": round(gbs, 1), "fused_frac_hbm": round(gbs / hbm, 4),
+                     "bytes_per_elem": QUANT_BYTES_PER_ELEM,
+                     "two_step_ms": round(ln_ms + q_ms, 4),
+                     "two_step_parts_ms": {"layernorm_modulate_torch_bf16": round(ln_ms, 4), "quantize": round(q_ms, 4)}}
+        del x, h, q, g16, b16
+        torch.cuda.empty_cache()
+    return out
+
+
+def time_flushed(fn, flush, iters=20, warmup=3):
+    """Median device time of fn with L2 flushed before every run (a write of a
+    buffer larger than L2), for operands that would otherwise stay in L2."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    ts = []
+    for _ in range(iters):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return statistics.median(ts)
+
+
+def small_layer_points(dev):
+    """Every DiT-XL/2 (M = 2048) and PixArt-1024 (M = 8192, cross-attention
+    M = 600) layer: the W4A4 GEMM (bf16 out) on each kernel the shape allows
+    (the library's choice, the single-CTA kernel, CTA pairs with 192- and
+    256-wide tiles), the dynamic-scale quantize of its input, and cuBLAS bf16
+    (a reference point), L2 flushed before every run.  Roofline per layer:
+    t = max(FLOPs / FP4 peak, (codes + scales of A and B + bf16 Y) / HBM peak)
+    with the measured peaks; frac = t / measured."""
+    import torch
+    import nvfp4_w4a4_gemm_quantize_b200 as nv
+    from nvfp4_w4a4_gemm_quantize_b200 import synth
+    peaks, _ = load_peaks()
+    fp4 = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"]) * FP4_OVER_BF16 * 1e12
+    hbm = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"]) * 1e9
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    kernels = {"auto": {}, "single": {"NVFP4_GEMM_KERNEL": "single"},
+               "pair192": {"NVFP4_GEMM_KERNEL": "pair", "NVFP4_PAIR_TILE_N": "192"},
+               "pair256": {"NVFP4_GEMM_KERNEL": "pair", "NVFP4_PAIR_TILE_N": "256"}}
+    out = {}
+    for wl in ("dit_xl2", "pixart1024"):
+        for L in synth.WORKLOADS[wl].layers:
+            x, w = synth.layer_tensors(wl, L.name, device=dev)
+            A, B = nv.quantize(x), nv.quantize(w)
+            y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev)
+            fl = 2 * L.M * L.N * L.K
+            byts = (L.M + L.N) * L.K * (0.5 + 1 / 16) + 2 * L.M * L.N
+            t_roof = max(fl / fp4, byts / hbm) * 1e3
+            r = {"shape": f"{L.M}x{L.K}x{L.N}", "roofline_ms": round(t_roof, 5),
+                 "bound": "tensor" if fl / fp4 > byts / hbm else "hbm"}
+            for name, env in kernels.items():
+                if name == "pair192" and L.N % 192 or name == "pair256" and L.N % 256:
+                    continue
+                saved = {k: os.environ.get(k) for k in env}
+                os.environ.update(env)
+                try:
+                    ms = time_flushed(lambda: nv.gemm_w4a4(A, B, out=y), flush)
+                finally:
+                    for k, v in saved.items():
+                        if v is None:
+                            os.environ.pop(k, None)
+                        else:
+                            os.environ[k] = v
+                r[name] = {"ms": round(ms, 5), "tflops": round(fl / (ms * 1e-3) / 1e12, 1),
+                           "frac": round(t_roof / ms, 3)}
+            q = nv.NVFP4Tensor.empty(L.M, L.K, dev)
+            ws = torch.empty(nv.nvfp4_quantize_workspace_bytes(L.M, L.K), dtype=torch.uint8, device=dev)
+            qms = time_flushed(lambda: nv.quantize(x, out=q, workspace=ws), flush)
+            r["quantize_ms"] = round(qms, 5)
+            r["quantize_frac_hbm"] = round(QUANT_BYTES_PER_ELEM * L.M * L.K / hbm * 1e3 / qms, 3)
+            bms = time_flushed(lambda: torch.matmul(x, w.t()), flush)
+            r["cublas_bf16_ms"] = round(bms, 5)
+            out[f"{wl}.{L.name}"] = r
+            del x, w, A, B, y, q
+    del flush
+    torch.cuda.empty_cache()
+    return out
 
 
 def grouped_points(dev):
@@ -522,6 +825,7 @@ def run_ours(args):
     if args.qat or args.only:
         # profiling aid: one group of reference points alone
         groups = {"qat": lambda: qat_points(dev, wl.layers), "mlp": lambda: mlp_fusion_points(dev, wl.layers),
+                  "layernorm": lambda: layernorm_points(dev), "small": lambda: small_layer_points(dev),
                   "grouped": lambda: grouped_points(dev), "mx": lambda: mx_points(dev, wl.layers),
                   "attention": lambda: attention_points(dev, args.heads or 384)}
         name = "qat" if args.qat else args.only
@@ -659,8 +963,7 @@ def run_ours(args):
     # ---- cpu baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        fl, secs, desc = oracle_sample(args.ref_rows)
-        cpu = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": desc}
+        cpu = cpu_baseline_leg(args)
 
     if rank == 0:
         # the GEMM is timed inside a long step (back-to-back steps under the
@@ -694,10 +997,7 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
             "data": "synthetic",
-            "config": {"workload": f"{WORKLOAD}: M=32768, qkv 3072->9216, fc1 3072->12288, fc2 12288->3072 "
-                                   "(dynamic-scale activation quantize + W4A4 GEMM, bf16 out)",
-                       "l2": "inputs larger than L2 (X 201-805 MB per layer, >2 GB streamed per step)",
-                       "parallelism": f"replica per GPU x{world}"},
+            "config": step_config(world),
             "roofline": {"bound": "tensor", "kernel": f"gemm_w4a4 {L.name} {L.M}x{L.K}x{L.N}",
                          "achieved": round(g_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                          "frac": round(g_tflops / fp4_peak, 4),
@@ -731,7 +1031,7 @@ def main():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--ref-rows", type=int, default=48)
+    ap.add_argument("--ref-rows", type=int, default=16, help="oracle rows per host core and layer")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-reference-points", action="store_true")
     ap.add_argument("--layers", default="", help="profiling: comma-separated subset of layers")
@@ -739,7 +1039,7 @@ def main():
     ap.add_argument("--qat", action="store_true", help="profiling: time only the QAT kernels (fc1 / fc2 inputs)")
     ap.add_argument("--heads", type=int, default=0, help="profiling: attention heads (default 384)")
     ap.add_argument("--only", default="", help="profiling: time one group of reference points "
-                                               "(qat, mlp, grouped, mx, attention)")
+                                               "(qat, mlp, layernorm, small, grouped, mx, attention)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

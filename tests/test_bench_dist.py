@@ -85,15 +85,31 @@ def test_reference_arm_line_on_rank_zero(monkeypatch, capsys):
 
 
 def test_reference_sample_is_bounded():
-    """The reference arm's per-step sample shrinks with K so that the timed
-    steps stay within the budget: features first, then rows."""
-    rows, frac = bench.ref_sample_size(48, 10, probe_secs=0.5, budget_s=60.0)
-    assert rows == 48 and frac == 1.0                     # 10 x 5 s fits in 60 s
-    rows, frac = bench.ref_sample_size(48, 100, probe_secs=0.5, budget_s=60.0)
-    assert rows == 48 and abs(frac - 0.12) < 1e-12        # 100 steps x 0.6 s
-    rows, frac = bench.ref_sample_size(48, 5000, probe_secs=0.5, budget_s=60.0)
-    assert frac == 128 / 3072 and 1 <= rows < 48          # features at one tile, fewer rows
-    assert bench.ref_sample_size(48, 10 ** 9, probe_secs=0.5)[0] == 1
+    """The reference arm's rows per step shrink with K so that the timed
+    steps stay within the budget (at least one row, at most the layer)."""
+    assert bench.ref_rows_for_budget(256, 0.5, 10, budget_s=60.0) == 3072      # 10 steps x 6 s
+    assert bench.ref_rows_for_budget(256, 0.5, 500, budget_s=60.0) == 61       # 500 steps x 0.12 s
+    assert bench.ref_rows_for_budget(256, 0.5, 10 ** 9) == 1
+    assert bench.ref_rows_for_budget(256, 1e-6, 1) == 32768
+
+
+def test_threaded_oracle_runner_equals_the_oracle():
+    """Spreading the oracle over threads by 128-row slices changes nothing:
+    the tensor scale, codes, scale layout and FP64 product are the whole-
+    tensor oracle's, bit for bit (300 rows: a ragged last slice)."""
+    import numpy as np
+    import oracle
+    x = synth.random_bf16((300, 512), seed=5, dist="token_scaled")
+    w = synth.random_bf16((200, 512), seed=6, scale=0.02)
+    r = bench.OracleRunner(4)
+    assert r.tensor_scale(x) == oracle.tensor_scale(x)
+    a, b = r.quantize(x), r.quantize(w)
+    a0, b0 = oracle.quantize(x), oracle.quantize(w)
+    for u, v in zip(a, a0):
+        assert np.array_equal(u, v)
+    for u, v in zip(b, b0):
+        assert np.array_equal(u, v)
+    assert np.array_equal(r.gemm(a, b), oracle.gemm_w4a4(*a0, *b0))
 
 
 def test_reduced_case_selects_layers_and_rows():
