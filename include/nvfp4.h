@@ -146,6 +146,42 @@ nvfp4_status nvfp4_quantize_noalloc(const void *x_bf16, int64_t rows, int64_t k,
                                     unsigned flags, int *dev_status, nvfp4_stream_t stream);
 
 /*
+ * nvfp4_layernorm_quantize -- the LayerNorm in front of a block's first
+ * projections, emitting their NVFP4 input directly ([DiT] Abstract and
+ * Methodology 3: every linear layer runs through the FP4 matmul; [RFC]
+ * Motivation: two-level scaling).  The pages do not define LayerNorm; the
+ * reading is the DiT pre-norm over the hidden dimension with the adaLN
+ * modulation x (1 + scale) + shift of each sample written as a per-channel
+ * affine shared by a group of rows:
+ *   mu, var of each row from S1 = sum x_j, S2 = sum x_j^2 in double,
+ *   var = max(S2 / k - mu^2, 0), rstd = 1 / sqrt(var + eps) (double, IEEE),
+ *   y_j = ((x_j - (float)mu) * (float)rstd) * gamma_j + beta_j  (FP32 ops),
+ * then y is quantized exactly as nvfp4_quantize quantizes an FP32 tensor (same
+ * tensor-scale rule, block scales, codes and layouts).  The bf16 LayerNorm
+ * output is never stored.  (Any summation order gives the same S1 and S2
+ * when a row's values span fewer than about 45 binary orders of magnitude,
+ * the case for activations; beyond that the statistics can differ from an
+ * index-order sum in their last bit.)
+ * x_bf16         [rows, k] bf16, row stride ld_x (as nvfp4_quantize).
+ * gamma, beta    nullable device FP32 [groups, k], 16-byte aligned; row r uses
+ *                group r / rows_per_group (rows_per_group == 0: one group);
+ *                NULL reads as 1 (gamma) and 0 (beta).
+ * eps            > 0 (DiT: 1e-6).
+ * codes, sf, tensor_scale, flags, workspace, workspace_bytes, dev_status:
+ *                as nvfp4_quantize (with NVFP4_SCALE_GIVEN the tensor scale is
+ *                read; otherwise it is the largest |y| / 2688, found in the
+ *                same kernel by a grid-wide handoff through the workspace).
+ * rows <= 2^31, k % 64 == 0, k <= 8192 (a row is held in a warp's registers).
+ * One kernel on `stream`.  Non-finite input is
+ * flagged in dev_status (NVFP4_ERR_NONFINITE) when the scale is data-derived.
+ */
+nvfp4_status nvfp4_layernorm_quantize(const void *x_bf16, int64_t rows, int64_t k, int64_t ld_x,
+                                      const float *gamma, const float *beta, int64_t rows_per_group,
+                                      double eps, uint8_t *codes, uint8_t *sf, float *tensor_scale,
+                                      unsigned flags, void *workspace, size_t workspace_bytes,
+                                      int *dev_status, nvfp4_stream_t stream);
+
+/*
  * Block size per layer ([DiT] Algorithmic framework, Algorithm 1 / Eq. 9:
  *   BlockSize(l) = argmin_{b in {1,2,4,8,16,32,64}} Error(l,b) + lambda Memory(b)/Memory_max).
  *

@@ -7,12 +7,12 @@ memory and streams.
 
 Low-level (same names and argument order as the C calls):
     nvfp4_sf_bytes, nvfp4_quantize_workspace_bytes, nvfp4_quantize,
-    nvfp4_quantize_noalloc, nvfp4_quantize_block, nvfp4_block_size_errors, nvfp4_select_block_size,
+    nvfp4_quantize_noalloc, nvfp4_layernorm_quantize, nvfp4_quantize_block, nvfp4_block_size_errors, nvfp4_select_block_size,
     nvfp4_dequantize, nvfp4_fake_quantize, nvfp4_ste_backward,
     nvfp4_gemm_w4a4, nvfp4_gemm_w4a4_grouped, nvfp4_gemm_w4a16, nvfp4_mx_sf_bytes, nvfp4_mx_quantize,
     nvfp4_mx_dequantize, nvfp4_mx_gemm, nvfp4_attention, nvfp4_attention_workspace_bytes, nvfp4_launch_count
 Convenience (allocate outputs with torch, then call the above):
-    NVFP4Tensor, quantize, dequantize, gemm_w4a4, gemm_w4a4_grouped, gemm_w4a16,
+    NVFP4Tensor, quantize, layernorm_quantize, dequantize, gemm_w4a4, gemm_w4a4_grouped, gemm_w4a16,
     fake_quantize, ste_backward, FakeQuantizeSTE (autograd: the two kernels),
     MXTensor, mx_quantize, mx_dequantize, mx_gemm, quantize_block, block_size_errors, select_block_size,
     attention
@@ -83,6 +83,14 @@ def nvfp4_quantize(x, rows, k, ld_x, codes, sf, tensor_scale, flags=0, workspace
     st = lib().nvfp4_quantize(_ptr(x), rows, k, ld_x, _ptr(codes), _ptr(sf), _ptr(tensor_scale),
                               flags, _ptr(workspace), workspace_bytes, _ptr(dev_status), _stream(stream))
     check(st, "nvfp4_quantize")
+
+
+def nvfp4_layernorm_quantize(x, rows, k, ld_x, gamma, beta, rows_per_group, eps, codes, sf, tensor_scale, flags=0,
+                             workspace=None, workspace_bytes=0, dev_status=None, stream=None) -> None:
+    st = lib().nvfp4_layernorm_quantize(_ptr(x), rows, k, ld_x, _ptr(gamma), _ptr(beta), rows_per_group, float(eps),
+                                        _ptr(codes), _ptr(sf), _ptr(tensor_scale), flags, _ptr(workspace),
+                                        workspace_bytes, _ptr(dev_status), _stream(stream))
+    check(st, "nvfp4_layernorm_quantize")
 
 
 def nvfp4_quantize_noalloc(x, rows, k, ld_x, codes, sf, tensor_scale, flags=0, dev_status=None,
@@ -229,6 +237,33 @@ def quantize(x: torch.Tensor, scale: torch.Tensor | float | None = None, out: NV
         workspace = torch.empty(wsb, dtype=torch.uint8, device=x.device)
     nvfp4_quantize(x, rows, k, x.stride(0), q.codes, q.sf, q.scale, flags,
                    workspace if flags == 0 else None, wsb if flags == 0 else 0, dev_status, stream)
+    return q
+
+
+def layernorm_quantize(x: torch.Tensor, gamma: torch.Tensor | None = None, beta: torch.Tensor | None = None,
+                       rows_per_group: int = 0, eps: float = 1e-6, scale: torch.Tensor | float | None = None,
+                       out: NVFP4Tensor | None = None, workspace: torch.Tensor | None = None, dev_status=None,
+                       stream=None) -> NVFP4Tensor:
+    """LayerNorm of a bf16 [rows, k] CUDA tensor (optional FP32 affine per
+    group of rows_per_group rows: gamma / beta [groups, k]) emitted directly as
+    NVFP4.  ``scale`` given -> the tensor scale; otherwise the largest |y| / 2688."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, k = x.shape
+    for t in (gamma, beta):
+        assert t is None or (t.dtype == torch.float32 and t.is_contiguous() and t.shape[-1] == k)
+    q = out if out is not None else NVFP4Tensor.empty(rows, k, x.device)
+    flags = 0
+    if scale is not None:
+        if isinstance(scale, torch.Tensor):
+            q.scale.copy_(scale.reshape(1).to(torch.float32))
+        else:
+            q.scale.fill_(float(scale))
+        flags = NVFP4_SCALE_GIVEN
+    wsb = nvfp4_quantize_workspace_bytes(rows, k)
+    if flags == 0 and workspace is None:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=x.device)
+    nvfp4_layernorm_quantize(x, rows, k, x.stride(0), gamma, beta, rows_per_group, eps, q.codes, q.sf, q.scale, flags,
+                             workspace if flags == 0 else None, wsb if flags == 0 else 0, dev_status, stream)
     return q
 
 

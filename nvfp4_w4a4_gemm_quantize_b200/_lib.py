@@ -42,6 +42,8 @@ SIGNATURES = {
     "nvfp4_quantize_workspace_bytes": (ctypes.c_size_t, [_i64, _i64]),
     "nvfp4_quantize": (_status, [_p, _i64, _i64, _i64, _p, _p, _p, ctypes.c_uint, _p, ctypes.c_size_t, _p, _p]),
     "nvfp4_quantize_noalloc": (_status, [_p, _i64, _i64, _i64, _p, _p, _p, ctypes.c_uint, _p, _p]),
+    "nvfp4_layernorm_quantize": (_status, [_p, _i64, _i64, _i64, _p, _p, _i64, ctypes.c_double, _p, _p, _p,
+                                           ctypes.c_uint, _p, ctypes.c_size_t, _p, _p]),
     "nvfp4_dequantize": (_status, [_p, _p, _p, _i64, _i64, _p, _int, _p]),
     "nvfp4_quantize_block": (_status, [_p, _i64, _i64, _i64, _int, _p, _p, _p, ctypes.c_uint, _p, ctypes.c_size_t,
                                        _p, _p]),

@@ -6,7 +6,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libnvfp4.so")
-SOURCES = ["api.cu", "quantize.cu", "quantize_noalloc.cu", "mx.cu", "blocksize.cu", "attn.cu", "gemm_w4a4.cu",
+SOURCES = ["api.cu", "quantize.cu", "quantize_noalloc.cu", "layernorm.cu", "mx.cu", "blocksize.cu", "attn.cu", "gemm_w4a4.cu",
            "gemm_w4a4_2sm.cu", "gemm_w4a16.cu"]
 HEADERS = ["ptx.cuh", "quant_math.cuh", "epilogue.cuh", "internal.h", "gemm.h", "tmap.h"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include", "nvfp4.h")

@@ -133,6 +133,36 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t
                                        dev_status, s));
 }
 
+nvfp4_status nvfp4_layernorm_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, const float* gamma,
+                                      const float* beta, int64_t rows_per_group, double eps, uint8_t* codes,
+                                      uint8_t* sf, float* tensor_scale, unsigned flags, void* workspace,
+                                      size_t workspace_bytes, int* dev_status, nvfp4_stream_t stream) {
+    if (rows < 0 || k <= 0 || ld_x < k || rows_per_group < 0) return NVFP4_ERR_INVALID_ARG;
+    if (!(eps > 0.0) || !(eps < 1.0e300)) return NVFP4_ERR_INVALID_ARG;
+    if ((flags & ~(unsigned)NVFP4_SCALE_GIVEN) != 0u) return NVFP4_ERR_INVALID_ARG;
+    if (!tensor_scale) return NVFP4_ERR_INVALID_ARG;
+    if (rows > 0 && (!x_bf16 || !codes || !sf)) return NVFP4_ERR_INVALID_ARG;
+    if (k % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (rows > ((int64_t)1 << 31) || k > layernorm_max_k()) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    const bool given = (flags & NVFP4_SCALE_GIVEN) != 0u;
+    if (!given && (!workspace || workspace_bytes < kQuantWorkspaceBytes)) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(sf) || (ld_x % 8) != 0 || !aligned16(gamma) ||
+        !aligned16(beta) || (!given && !aligned16(workspace)) || (reinterpret_cast<uintptr_t>(tensor_scale) & 3u))
+        return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    nvfp4_status st = device_ok(&sms);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (rows == 0) {
+        if (!given) return cuda_status(cudaMemsetAsync(tensor_scale, 0, sizeof(float), s));
+        return NVFP4_OK;
+    }
+    return cuda_status(launch_layernorm_quantize(static_cast<const uint16_t*>(x_bf16), rows, k, ld_x, gamma, beta,
+                                                 rows_per_group, eps, codes, sf, tensor_scale, given,
+                                                 static_cast<unsigned long long*>(workspace),
+                                                 given ? 0u : next_generation(), dev_status, sms, s));
+}
+
 nvfp4_status nvfp4_quantize_block(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, int block,
                                   uint8_t* codes, uint8_t* sf, float* tensor_scale, unsigned flags, void* workspace,
                                   size_t workspace_bytes, int* dev_status, nvfp4_stream_t stream) {

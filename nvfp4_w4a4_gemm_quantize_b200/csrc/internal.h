@@ -19,6 +19,17 @@ constexpr int64_t kQuantMaxRows = (int64_t)65535 * 128;
 
 void count_launch(int n);
 
+// Per-call number tagging the slots of a grid-wide handoff in a caller's
+// workspace (never 0; one counter for every kernel that hands over through
+// slots, so no two calls in the process share a number).
+uint32_t next_generation();
+
+cudaError_t launch_layernorm_quantize(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, const float* gamma,
+                                      const float* beta, int64_t rows_per_group, double eps, uint8_t* codes,
+                                      uint8_t* sf, float* tensor_scale, bool scale_given, unsigned long long* slots,
+                                      uint32_t gen, int* dev_status, int num_sms, cudaStream_t stream);
+int64_t layernorm_max_k();
+
 int amax_grid(int64_t rows, int64_t k);
 
 cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes,

@@ -20,6 +20,7 @@
 // code of the IEEE quotient, otherwise the values are divided exactly (see
 // quant_math.cuh).
 #include <atomic>
+#include <cstdlib>
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -27,6 +28,7 @@
 #include "ptx.cuh"
 #include "quant_math.cuh"
 #include "internal.h"
+#include "tmap.h"
 
 namespace nvfp4 {
 
@@ -407,11 +409,16 @@ struct FakeOut {
     __device__ __forceinline__ void store_scales(const uint8_t*, int64_t, int64_t, int64_t) const {}
 };
 
-// Quantize a lane's loaded blocks and hand each to the output; scale bytes go
-// to the CTA's staging atoms when the output stores scales.
-template <class Out>
+// Quantize a lane's loaded blocks and hand each to the output.  When the
+// output stores scales they go to the CTA's staging atoms (kStage) or, word by
+// word, straight to the scale buffer: the four lanes holding blocks 4a .. 4a+3
+// of a row share one 32-bit word of the layout, gathered by shuffles and
+// stored by the first of them (rows past the tensor quantize zeros, so the
+// padding rows of the layout get zero scales).
+template <class Out, bool kStage = true>
 __device__ __forceinline__ void quantize_lane(const TileLane& t, const uint4 (&v)[2 * kSteps], const ScaleConsts& sc,
-                                              uint8_t* sf_stage, const Out& out, int64_t k) {
+                                              uint8_t* sf_stage, const Out& out, int64_t k, int64_t rblk = 0,
+                                              int64_t cblk = 0) {
     const typename Out::Lane ol = out.lane(t, k);
 #pragma unroll
     for (int i = 0; i < kSteps; ++i) {
@@ -425,7 +432,22 @@ __device__ __forceinline__ void quantize_lane(const TileLane& t, const uint4 (&v
         const uint32_t lo = quantize8_bf16(w[0], w[1], w[2], w[3], s);
         const uint32_t hi = quantize8_bf16(w[4], w[5], w[6], w[7], s);
         out.emit(ol, i, 2 * i < t.rows_left && t.col_ok, w, sfc, s, lo, hi, sc);
-        if (Out::kScales && t.col_ok) sf_stage[t.sbase + 32 * i] = (uint8_t)sfc;
+        if constexpr (Out::kScales) {
+            if (kStage) {
+                if (t.col_ok) sf_stage[t.sbase + 32 * i] = (uint8_t)sfc;
+            } else {
+                uint32_t word = sfc;
+                word |= __shfl_down_sync(0xffffffffu, sfc, 1) << 8;
+                word |= __shfl_down_sync(0xffffffffu, sfc, 2) << 16;
+                word |= __shfl_down_sync(0xffffffffu, sfc, 3) << 24;
+                const int lane = threadIdx.x & 31, blk = lane & 15;
+                const int rt = ((threadIdx.x >> 5) & 15) * kRows + (lane >> 4) + 2 * i;     // row inside the tile
+                if ((blk & 3) == 0 && t.col_ok) {
+                    const int64_t atom = rblk * (k >> 6) + cblk * 4 + (blk >> 2);
+                    *reinterpret_cast<uint32_t*>(out.sf + (atom << 9) + (rt & 31) * 16 + (rt >> 5) * 4) = word;
+                }
+            }
+        }
     }
 }
 
@@ -563,6 +585,156 @@ quantize_fused_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, i
             __syncthreads();
             out.store_scales(sf_stage, k, rblk, cblk);
             __syncthreads();
+        }
+    }
+}
+
+// One-kernel form, streamed: the same two phases, with the tiles brought into
+// shared memory by TMA.  One CTA per SM (cooperative launch, so every CTA is
+// resident for the handoff): a producer warp keeps a ring of kStreamBufs tile
+// buffers filled -- the CTA's tiles in order for phase 1, then in reverse for
+// phase 2 -- while sixteen consumer warps work on the tile in front.  Loads
+// therefore overlap the arithmetic instead of alternating with it, and the
+// first phase-2 tiles are already on their way while the CTAs wait for each
+// other's maxima.  A consumer warp releases a buffer as soon as it holds its
+// part of the tile in registers.
+constexpr int kStreamBufs = 3;
+constexpr int kStreamTileBytes = kTileRows * kTileCols * 2;      // 64 KB of bf16
+constexpr int kStreamConsumers = kQuantThreads;                  // 16 warps
+constexpr int kStreamThreads = kStreamConsumers + 32;            // + the producer warp
+constexpr int kStreamSmem = kStreamBufs * kStreamTileBytes + 1024;
+
+__device__ __forceinline__ void consumers_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kStreamConsumers) : "memory");
+}
+
+template <class Out>
+__global__ void __launch_bounds__(kStreamThreads, 1)
+quantize_stream_kernel(const __grid_constant__ CUtensorMap tmap_x, int64_t rows, int64_t k, const Out out,
+                       float* __restrict__ tensor_scale, unsigned long long* __restrict__ slots, uint32_t gen,
+                       int ntiles_c, int ntiles, int* __restrict__ dev_status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ __align__(8) uint64_t full_bar[kStreamBufs], empty_bar[kStreamBufs];
+    __shared__ ScaleConsts sc_sh;
+    __shared__ uint32_t red[kStreamConsumers / 32];
+    __shared__ int abort_sh, ok_sh;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        abort_sh = 0;
+        for (int b = 0; b < kStreamBufs; ++b) {
+            mbar_init(&full_bar[b], 1);
+            mbar_init(&empty_bar[b], kStreamConsumers / 32);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+    WaitCtx wc{&abort_sh, dev_status};
+    const int nmine = ntiles > (int)blockIdx.x ? (ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+    if (warp == kStreamConsumers / 32) {
+        // ---- producer: phase-1 tiles in order, then the same tiles in reverse
+        if (lane == 0) {
+            tma_prefetch_desc(&tmap_x);
+            const uint64_t pol1 = policy_evict_normal(), pol2 = policy_evict_first();
+            int b = 0;
+            uint32_t ph = 0;
+            for (int q = 0; q < 2 * nmine; ++q) {
+                const int j = q < nmine ? q : 2 * nmine - 1 - q;
+                const int tt = (int)blockIdx.x + j * (int)gridDim.x;
+                if (!mbar_wait(&empty_bar[b], ph ^ 1u, wc)) break;
+                mbar_arrive_expect_tx(&full_bar[b], kStreamTileBytes);
+                tma_load_2d(tiles + b * kStreamTileBytes, &tmap_x, &full_bar[b], (tt % ntiles_c) * kTileCols,
+                            (tt / ntiles_c) * kTileRows, q < nmine ? pol1 : pol2);
+                if (++b == kStreamBufs) { b = 0; ph ^= 1u; }
+            }
+        }
+        return;
+    }
+
+    // ---- consumers, phase 1: |x| maximum of the CTA's tiles
+    int b = 0;
+    uint32_t ph = 0;
+    uint32_t m = 0u;
+    bool alive = true;
+    for (int q = 0; q < nmine; ++q) {
+        alive = alive && mbar_wait(&full_bar[b], ph, wc);
+        if (alive) {
+            const uint4* t = reinterpret_cast<const uint4*>(tiles + b * kStreamTileBytes);
+#pragma unroll
+            for (int i = 0; i < kStreamTileBytes / 16 / kStreamConsumers; ++i)
+                m = absmax_nan_bf16x2(m, absmax_bf16x8(t[threadIdx.x + i * kStreamConsumers]));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[b]);
+        if (++b == kStreamBufs) { b = 0; ph ^= 1u; }
+    }
+    m &= 0x7FFF7FFFu;
+    uint32_t h = max(m & 0xFFFFu, m >> 16);
+    for (int o = 16; o > 0; o >>= 1) h = max(h, __shfl_xor_sync(0xffffffffu, h, o));
+    if (lane == 0) red[warp] = h;
+    consumers_sync();
+    if (warp == 0) {
+        uint32_t tm = lane < kStreamConsumers / 32 ? red[lane] : 0u;
+        for (int o = 16; o > 0; o >>= 1) tm = max(tm, __shfl_xor_sync(0xffffffffu, tm, o));
+        if (lane == 0) {
+            if (tm >= 0x7F80u && dev_status) atomicCAS(dev_status, 0, (int)NVFP4_ERR_NONFINITE);
+            const unsigned long long word = ((unsigned long long)gen << 32) | (unsigned long long)(tm << 16);
+            asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(slots + blockIdx.x), "l"(word) : "memory");
+        }
+        // ---- every CTA's slot carries this generation: the tensor maximum
+        float mx = 0.0f;
+        bool ok = true;
+        const uint64_t t0 = globaltimer_ns();
+        for (int i = lane; i < (int)gridDim.x; i += 32) {
+            unsigned long long w;
+            uint32_t n = 0;
+            while (true) {
+                asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(slots + i) : "memory");
+                if ((uint32_t)(w >> 32) == gen) break;
+                if ((++n & 63u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) { ok = false; break; }
+            }
+            if (!ok) break;
+            mx = fmaxf(mx, __uint_as_float((uint32_t)w));
+        }
+        ok = __all_sync(0xffffffffu, ok ? 1 : 0) != 0;
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) {
+            if (!ok && dev_status) atomicExch(dev_status, (int)NVFP4_ERR_TIMEOUT);
+            const float g = __fdiv_rn(mx, 2688.0f);
+            if (blockIdx.x == 0 && ok) *tensor_scale = g;
+            sc_sh = scale_consts(g);
+            ok_sh = ok ? 1 : 0;
+        }
+    }
+    consumers_sync();
+    // gave up waiting: the tiles are still consumed (so that no load is left
+    // in flight when the CTA exits), but nothing is written
+    alive = alive && ok_sh != 0;
+    const ScaleConsts sc = sc_sh;
+
+    // ---- consumers, phase 2: quantize the same tiles, last first
+    for (int q = nmine - 1; q >= 0; --q) {
+        const int tt = (int)blockIdx.x + q * (int)gridDim.x;
+        const int64_t rblk = tt / ntiles_c, cblk = tt % ntiles_c;
+        alive = alive && mbar_wait(&full_bar[b], ph, wc);
+        uint4 v[2 * kSteps];
+        const int half = lane >> 4, blk = lane & 15;
+        if (alive) {
+            const uint8_t* base = tiles + b * kStreamTileBytes + (warp * kRows + half) * (kTileCols * 2) + blk * 32;
+#pragma unroll
+            for (int i = 0; i < kSteps; ++i) {
+                const uint4* r = reinterpret_cast<const uint4*>(base + 2 * i * (kTileCols * 2));
+                v[2 * i] = r[0];
+                v[2 * i + 1] = r[1];
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[b]);
+        if (++b == kStreamBufs) { b = 0; ph ^= 1u; }
+        if (alive) {
+            const TileLane t = tile_lane(nullptr, rows, k, k, rblk, cblk, warp, lane);
+            quantize_lane<Out, false>(t, v, sc, nullptr, out, k, rblk, cblk);
         }
     }
 }
@@ -721,14 +893,19 @@ static cudaError_t launch_two_kernel(const uint16_t* x, int64_t rows, int64_t k,
 // slot that carries the new call's number).
 static std::atomic<uint32_t> g_generation{0};
 
+uint32_t next_generation() {
+    uint32_t gen = g_generation.fetch_add(1u) + 1u;
+    if (gen == 0u) gen = g_generation.fetch_add(1u) + 1u;     // 0 never marks a slot
+    return gen;
+}
+
 // One-kernel form with a data-derived scale (see quantize_fused_kernel).
 // Returns cudaErrorNotSupported when the grid cannot be co-resident (the
 // caller then takes the two-kernel form, which computes the same result).
 template <class Out>
-static cudaError_t launch_one_kernel(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, const Out& out,
-                                     float* tensor_scale, unsigned long long* slots, int max_slots, int* dev_status,
-                                     int num_sms, cudaStream_t stream) {
-    std::atomic<uint32_t>& generation = g_generation;
+static cudaError_t launch_one_kernel_regs(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, const Out& out,
+                                          float* tensor_scale, unsigned long long* slots, int max_slots,
+                                          int* dev_status, int num_sms, cudaStream_t stream) {
     const int ntiles_c = (int)((k + kTileCols - 1) / kTileCols);
     const int64_t ntiles64 = ((rows + kTileRows - 1) / kTileRows) * ntiles_c;
     if (ntiles64 > (int64_t)1 << 30) return cudaErrorNotSupported;
@@ -741,8 +918,7 @@ static cudaError_t launch_one_kernel(const uint16_t* x, int64_t rows, int64_t k,
     if (grid > max_slots) grid = max_slots;
     if (grid > ntiles) grid = ntiles;
     if (grid < 1) return cudaErrorNotSupported;
-    uint32_t gen = generation.fetch_add(1u) + 1u;
-    if (gen == 0u) gen = generation.fetch_add(1u) + 1u;     // 0 never marks a slot
+    const uint32_t gen = next_generation();
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;           // every CTA resident at once
@@ -755,6 +931,63 @@ static cudaError_t launch_one_kernel(const uint16_t* x, int64_t rows, int64_t k,
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, quantize_fused_kernel<Out>, x, rows, k, ld, out, tensor_scale, slots, gen,
                            ntiles_c, ntiles, dev_status);
+    if (e == cudaErrorCooperativeLaunchTooLarge) {
+        (void)cudaGetLastError();
+        return cudaErrorNotSupported;
+    }
+    if (e != cudaSuccess) return e;
+    count_launch(1);
+    return cudaGetLastError();
+}
+
+// One-kernel form with a data-derived scale: for fake quantization the tiles
+// are streamed through shared memory by TMA (quantize_stream_kernel); codes
+// and scales are faster from registers (quantize_fused_kernel, two CTAs per
+// SM: the streamed form's shared-memory reads and scale-word shuffles cost it
+// a few per cent there).  NVFP4_QUANT_ONE_KERNEL=regs or =stream forces one
+// form, for measurements.  Returns
+// cudaErrorNotSupported when the grid cannot be co-resident or the tensor
+// cannot be described to TMA (the caller then takes the two-kernel form,
+// which computes the same result).
+template <class Out>
+static cudaError_t launch_one_kernel(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, const Out& out,
+                                     float* tensor_scale, unsigned long long* slots, int max_slots, int* dev_status,
+                                     int num_sms, cudaStream_t stream) {
+    const char* env = getenv("NVFP4_QUANT_ONE_KERNEL");
+    const bool stream_form = env ? env[0] == 's' : !Out::kScales;
+    if (!stream_form)
+        return launch_one_kernel_regs(x, rows, k, ld, out, tensor_scale, slots, max_slots, dev_status, num_sms,
+                                      stream);
+    const int ntiles_c = (int)((k + kTileCols - 1) / kTileCols);
+    const int64_t ntiles64 = ((rows + kTileRows - 1) / kTileRows) * ntiles_c;
+    if (ntiles64 > (int64_t)1 << 30) return cudaErrorNotSupported;
+    const int ntiles = (int)ntiles64;
+    CUtensorMap tm;
+    if (make_tmap_2d(&tm, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)k, (uint64_t)rows, (uint64_t)ld * 2,
+                     kTileCols, kTileRows, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+        return cudaErrorNotSupported;
+    auto kern = quantize_stream_kernel<Out>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kStreamThreads, kStreamSmem);
+    if (e != cudaSuccess) return e;
+    int grid = per_sm * num_sms;
+    if (grid > max_slots) grid = max_slots;
+    if (grid > ntiles) grid = ntiles;
+    if (grid < 1) return cudaErrorNotSupported;
+    const uint32_t gen = next_generation();
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;           // every CTA resident at once
+    attr[0].val.cooperative = 1;
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kStreamThreads);
+    cfg.dynamicSmemBytes = kStreamSmem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, tm, rows, k, out, tensor_scale, slots, gen, ntiles_c, ntiles, dev_status);
     if (e == cudaErrorCooperativeLaunchTooLarge) {
         (void)cudaGetLastError();
         return cudaErrorNotSupported;

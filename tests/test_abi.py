@@ -32,7 +32,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 23, names
+    assert len(names) == 24, names
     for n in names:
         assert hasattr(L, n), n
         assert n in _lib.SIGNATURES, n
@@ -93,6 +93,19 @@ def test_quantize_rejects_bad_arguments(L):
     assert L.nvfp4_quantize_block(A, big, 64, 64, 32, B, C, A, 1, None, 0, None, None) == SHAPE
     assert L.nvfp4_fake_quantize(A, big, 64, 64, B, 0, None, A, 1, None, 0, None, None) == SHAPE
     assert L.nvfp4_quantize_noalloc(A, big, 64, 64, B, C, A, 0, None, None) == SHAPE
+
+
+def test_layernorm_quantize_rejects_bad_arguments(L):
+    f = L.nvfp4_layernorm_quantize
+    # (x, rows, k, ld, gamma, beta, rows_per_group, eps, codes, sf, scale, flags, ws, ws_bytes, dev_status, stream)
+    assert f(A, 128, 96, 96, None, None, 0, 1e-6, B, C, A, 1, None, 0, None, None) == SHAPE
+    assert f(A, 128, 256, 256, None, None, 0, 0.0, B, C, A, 1, None, 0, None, None) == INVALID     # eps <= 0
+    assert f(A, 128, 256, 256, None, None, -1, 1e-6, B, C, A, 1, None, 0, None, None) == INVALID   # group size
+    assert f(None, 128, 256, 256, None, None, 0, 1e-6, B, C, A, 1, None, 0, None, None) == INVALID
+    assert f(A, 128, 256, 256, None, None, 0, 1e-6, B, C, None, 1, None, 0, None, None) == INVALID
+    assert f(A, 128, 256, 256, None, None, 0, 1e-6, B, C, A, 0, None, 0, None, None) == WORKSPACE
+    assert f(A, 128, 256, 256, A + 4, None, 0, 1e-6, B, C, A, 1, None, 0, None, None) == MISALIGNED
+    assert f(A, 128, 256, 260, None, None, 0, 1e-6, B, C, A, 1, None, 0, None, None) == MISALIGNED
 
 
 def test_dequantize_rejects_bad_arguments(L):
