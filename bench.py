@@ -664,29 +664,42 @@ def small_layer_points(dev):
 
 
 def grouped_points(dev):
-    """One PixArt-1024 block's independent projections (image-token QKV,
-    text-token cross-attention K and V) as one grouped launch vs three."""
+    """One PixArt-1024 block's independent projections as one grouped launch
+    vs separate launches: the image-token QKV with the text-token
+    cross-attention K and V, and the same with the MLP's fc1 added (every N a
+    multiple of 192, so the group runs on the CTA-pair kernel), L2 flushed
+    before every run."""
     import torch
     import nvfp4_w4a4_gemm_quantize_b200 as nv
     from nvfp4_w4a4_gemm_quantize_b200 import synth
-    pairs, fl = [], 0
-    for name in ("qkv", "xattn_k", "xattn_v"):
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ops = {}
+    for name in ("qkv", "xattn_k", "xattn_v", "fc1"):
         x, w = synth.layer_tensors("pixart1024", name, device=dev)
-        pairs.append((nv.quantize(x), nv.quantize(w)))
-        fl += 2 * x.shape[0] * x.shape[1] * w.shape[0]
-    ys = [torch.empty(A.rows, B.rows, dtype=torch.bfloat16, device=dev) for A, B in pairs]
-    probs = [dict(a_codes=A.codes, a_sf=A.sf, a_scale=A.scale, b_codes=B.codes, b_sf=B.sf, b_scale=B.scale,
-                  M=A.rows, N=B.rows, K=A.k, y=y) for (A, B), y in zip(pairs, ys)]
+        A, B = nv.quantize(x), nv.quantize(w)
+        ops[name] = (A, B, torch.empty(A.rows, B.rows, dtype=torch.bfloat16, device=dev),
+                     2 * x.shape[0] * x.shape[1] * w.shape[0])
+        del x, w
+    out = {}
+    for label, names in (("qkv_xattn", ("qkv", "xattn_k", "xattn_v")),
+                         ("qkv_xattn_fc1", ("qkv", "xattn_k", "xattn_v", "fc1"))):
+        sel = [ops[n] for n in names]
+        probs = [dict(a_codes=A.codes, a_sf=A.sf, a_scale=A.scale, b_codes=B.codes, b_sf=B.sf, b_scale=B.scale,
+                      M=A.rows, N=B.rows, K=A.k, y=y) for A, B, y, _ in sel]
+        fl = sum(f for *_, f in sel)
 
-    def separate():
-        for (A, B), y in zip(pairs, ys):
-            nv.gemm_w4a4(A, B, out=y)
+        def separate():
+            for A, B, y, _ in sel:
+                nv.gemm_w4a4(A, B, out=y)
 
-    sep = time_device(separate, iters=50, warmup=5)
-    grp = time_device(lambda: nv.nvfp4_gemm_w4a4_grouped(probs), iters=50, warmup=5)
-    return {"problems": "pixart1024 qkv 8192x1152x3456 + xattn_k/v 600x4096x1152",
-            "separate_us": round(sep * 1e3, 1), "grouped_us": round(grp * 1e3, 1),
-            "grouped_tflops": round(fl / (grp * 1e-3) / 1e12, 1)}
+        sep = time_flushed(separate, flush)
+        grp = time_flushed(lambda: nv.nvfp4_gemm_w4a4_grouped(probs), flush)
+        out[label] = {"problems": ", ".join(f"{n} {ops[n][0].rows}x{ops[n][0].k}x{ops[n][1].rows}" for n in names),
+                      "separate_us": round(sep * 1e3, 1), "grouped_us": round(grp * 1e3, 1),
+                      "grouped_tflops": round(fl / (grp * 1e-3) / 1e12, 1)}
+    del flush, ops
+    torch.cuda.empty_cache()
+    return out
 
 
 def mx_points(dev, layers):

@@ -27,8 +27,11 @@ struct GemmW4A4Args {
 
 cudaError_t launch_gemm_w4a4(const GemmW4A4Args& a, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemm_w4a4_grouped(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream);
+cudaError_t launch_group_single(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream);
 int gemm_w4a4_max_group();
 cudaError_t launch_gemm_w4a4_2sm(const GemmW4A4Args& a, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemm_w4a4_2sm_grouped(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream);
+int gemm_w4a4_2sm_tile_n(const GemmW4A4Args* probs, int count);
 bool gemm_w4a4_2sm_supports(int64_t N);
 
 struct GemmW4A16Args {

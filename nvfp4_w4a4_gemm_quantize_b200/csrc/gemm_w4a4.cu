@@ -532,12 +532,30 @@ cudaError_t launch_gemm_w4a4(const GemmW4A4Args& a, int num_sms, cudaStream_t st
         const int64_t pair_tiles = ((a.M + 255) / 256) * (a.N / bn);
         if (forced == 1 || pair_tiles >= num_sms / 2) return launch_gemm_w4a4_2sm(a, num_sms, stream);
     }
-    return launch_gemm_w4a4_grouped(&a, 1, num_sms, stream);
+    return launch_group_single(&a, 1, num_sms, stream);
 }
 
-// Up to kMaxGroup problems in one launch of the single-CTA kernel; every
-// problem has the same output kind (bf16, FP32 or NVFP4) and activation.
+// Up to kMaxGroup problems in one launch; every problem has the same output
+// kind (bf16, FP32 or NVFP4) and activation.  When every N allows one pair
+// tile width and the problems' pair tiles fill the GPU, the CTA-pair kernel
+// takes the whole group (one tile space); otherwise the single-CTA kernel.
+// NVFP4_GEMM_KERNEL=pair or =single overrides the choice (where the shapes
+// allow) for measurements.
 cudaError_t launch_gemm_w4a4_grouped(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream) {
+    using namespace w4a4;
+    const char* env = getenv("NVFP4_GEMM_KERNEL");
+    const int forced = env ? (env[0] == 'p' ? 1 : env[0] == 's' ? 2 : 0) : 0;
+    const int bn = count > 1 && forced != 2 && !probs[0].mx ? gemm_w4a4_2sm_tile_n(probs, count) : 0;
+    if (bn != 0) {
+        int64_t tiles = 0;
+        for (int i = 0; i < count; ++i) tiles += ((probs[i].M + 255) / 256) * (probs[i].N / bn);
+        if (forced == 1 || tiles >= num_sms / 2) return launch_gemm_w4a4_2sm_grouped(probs, count, num_sms, stream);
+    }
+    return launch_group_single(probs, count, num_sms, stream);
+}
+
+// The single-CTA kernel on a group (a plain call is a group of one).
+cudaError_t launch_group_single(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream) {
     using namespace w4a4;
     const int out = probs[0].y != nullptr ? (probs[0].y_dtype == 1 ? OUT_F32 : OUT_BF16) : OUT_NVFP4;
     if (out == OUT_BF16) return launch_group<OUT_BF16>(probs, count, num_sms, stream);

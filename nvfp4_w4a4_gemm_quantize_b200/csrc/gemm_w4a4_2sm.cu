@@ -84,6 +84,7 @@ struct Regs {
 };
 constexpr int SF_COLS_ATOM = 4 + 8;              // SFA 4 columns, SFB 8 columns (two 128-row atoms) per scale atom
 constexpr int kGroupM = 8;                       // rasterisation group, in 256-row pair tiles
+constexpr int kPairGroup = 8;                    // problems of a grouped launch
 constexpr int kSmemLimit = 232448;
 
 enum OutKind { OUT_BF16 = 0, OUT_F32 = 1, OUT_NVFP4 = 2 };
@@ -133,17 +134,37 @@ struct Cfg {
     static_assert(EPI_COLS % 32 == 0, "epilogue chunks of 32 columns");
 };
 
-struct Params {
+struct PairProblem {
     const float* a_scale;
     const float* b_scale;
     int M, N, K;
-    int num_mb2, num_nb, num_tiles;
+    int num_mb2, num_nb, first_tile;
     uint8_t* y_codes;
     uint8_t* y_sf;
     const float* y_scale;
     float* y_amax;
+};
+
+// Up to G independent problems sharing one tile space (G = 1: a plain call):
+// per problem its tensor maps (A, B, A scales, B scales, Y) and sizes; its
+// tiles are numbered from first_tile on.  Every role walks the same tile
+// sequence and finds a tile's problem by comparing with the first tiles.
+template <int G>
+struct alignas(64) PairGroup {
+    CUtensorMap map[G][5];
+    PairProblem prob[G];
+    int count, num_tiles;
     int* dev_status;
 };
+
+template <int G>
+__device__ __forceinline__ int problem_of(const PairGroup<G>& g, int t) {
+    int pi = 0;
+#pragma unroll
+    for (int i = 1; i < G; ++i)
+        if (i < g.count && t >= g.prob[i].first_tile) pi = i;
+    return pi;
+}
 
 __device__ __forceinline__ void tile_coords(int t, int num_mb2, int num_nb, int& mb2, int& nb) {
     const int per_group = kGroupM * num_nb;
@@ -159,7 +180,7 @@ __device__ __forceinline__ void tile_coords(int t, int num_mb2, int num_nb, int&
 // through a swizzled staging buffer and a TMA store of a 32 x 32 box.
 template <int OUT, int ACT>
 __device__ __forceinline__ void store_chunk(const uint32_t* r, float alpha, uint8_t* buf, int lane,
-                                            const CUtensorMap* map, int x, int y) {
+                                            const CUtensorMap* map, int x, int y, uint64_t policy) {
     if (OUT == OUT_BF16) {
         uint32_t pk[16];
 #pragma unroll
@@ -187,9 +208,18 @@ __device__ __forceinline__ void store_chunk(const uint32_t* r, float alpha, uint
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-        tma_store_2d(map, buf, x, y);
+        tma_store_2d_hint(map, buf, x, y, policy);
         bulk_commit_group();
     }
+}
+
+// Fold a warp's running maximum of |y| into a problem's y_amax (nullable) and
+// start a new one.  Non-negative floats order like their bit patterns.
+__device__ __forceinline__ void flush_amax(float& amax_run, float* y_amax, int lane) {
+    for (int o = 16; o > 0; o >>= 1) amax_run = fmaxf(amax_run, __shfl_xor_sync(0xffffffffu, amax_run, o));
+    if (y_amax != nullptr && lane == 0 && amax_run > 0.0f)
+        atomicMax(reinterpret_cast<int*>(y_amax), __float_as_int(amax_run));
+    amax_run = 0.0f;
 }
 
 // Scale atom `at` of a stage of the pair (A: 128 rows of this CTA, B: the
@@ -222,11 +252,9 @@ __device__ __forceinline__ void k_mma(uint32_t tmem_acc, uint32_t sb, uint32_t s
     }
 }
 
-template <int BN, int OUT, int ACT, bool MXS>
+template <int G, int BN, int OUT, int ACT, bool MXS>
 __global__ void __launch_bounds__(kThreads, 1)
-gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-             const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
-             const __grid_constant__ CUtensorMap tmap_y, const Params p) {
+gemm2_kernel(const __grid_constant__ PairGroup<G> g) {
     using C = Cfg<BN, OUT, MXS>;
     using L = Lay<BN, MXS>;
     constexpr int STAGES = C::STAGES;
@@ -251,7 +279,7 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     const int pair = (int)cluster_id_x();
     const int npairs = (int)nclusters_x();
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    WaitCtx wc{&abort_sh, p.dev_status};
+    WaitCtx wc{&abort_sh, g.dev_status};
 
     if (threadIdx.x == 0) {
         abort_sh = 0;
@@ -266,11 +294,8 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
         }
         mbar_init(&drain_bar, 1);
         fence_barrier_init();
-        tma_prefetch_desc(&tmap_a);
-        tma_prefetch_desc(&tmap_b);
-        tma_prefetch_desc(&tmap_sfa);
-        tma_prefetch_desc(&tmap_sfb);
-        tma_prefetch_desc(&tmap_y);
+        for (int i = 0; i < g.count; ++i)
+            for (int m = 0; m < 5; ++m) tma_prefetch_desc(&g.map[i][m]);
     }
     // scale regions start as zeros (finite) so rows that are never loaded
     // (beyond M or N) multiply zero codes by a finite scale
@@ -289,9 +314,6 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_sh;
 
-    const int num_kt = (p.K + 255) / 256;
-    const int k_atoms = p.K / L::K_ATOM;             // scale atoms per 128 rows
-    const int k_steps = p.K / 64;                    // K = 64 MMA steps
     const uint32_t sf_base = tmem_base + ACC_BUFS * BN;
     // one register-budget change per warpgroup, before the roles diverge
     // (the epilogue code sits under the same branch as its increase, so that
@@ -305,9 +327,13 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
             int stage = 0;
             uint32_t phase = 0, issued = 0, issued_any = 0;
             bool ok = true;
-            for (int t = pair; t < p.num_tiles && ok; t += npairs) {
+            for (int t = pair; t < g.num_tiles && ok; t += npairs) {
+                const int pi = problem_of(g, t);
+                const PairProblem& P = g.prob[pi];
+                const CUtensorMap* maps = g.map[pi];
+                const int num_kt = (P.K + 255) / 256, k_atoms = P.K / L::K_ATOM;
                 int mb2, nb;
-                tile_coords(t, p.num_mb2, p.num_nb, mb2, nb);
+                tile_coords(t - P.first_tile, P.num_mb2, P.num_nb, mb2, nb);
                 const int arow = mb2 * 256 + (int)rank * 128;
                 const int brow = nb * BN + (int)rank * L::B_ROWS;
                 const int sfa_row = (mb2 * 2 + (int)rank) * k_atoms;
@@ -325,12 +351,12 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                         if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * STAGE_BYTES);
                         const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
                         uint8_t* sfs = sb + A_BYTES + L::B_BYTES;
-                        tma_load_2d_pair(sfs, &tmap_sfa, fb, 0, sfa_row + kt * L::SF_PER, pol_a);
-                        tma_load_2d_pair(sfs + L::SFA_BYTES, &tmap_sfb, fb, 0, sfb_row0 + kt * L::SF_PER, pol_b);
-                        tma_load_2d_pair(sfs + L::SFA_BYTES + L::SF_PER * SF_ATOM, &tmap_sfb, fb, 0,
+                        tma_load_2d_pair(sfs, &maps[2], fb, 0, sfa_row + kt * L::SF_PER, pol_a);
+                        tma_load_2d_pair(sfs + L::SFA_BYTES, &maps[3], fb, 0, sfb_row0 + kt * L::SF_PER, pol_b);
+                        tma_load_2d_pair(sfs + L::SFA_BYTES + L::SF_PER * SF_ATOM, &maps[3], fb, 0,
                                          sfb_row1 + kt * L::SF_PER, pol_b);
-                        tma_load_2d_pair(sb, &tmap_a, fb, kt * BK_BYTES, arow, pol_a);
-                        tma_load_2d_pair(sb + A_BYTES, &tmap_b, fb, kt * BK_BYTES, brow, pol_b);
+                        tma_load_2d_pair(sb, &maps[0], fb, kt * BK_BYTES, arow, pol_a);
+                        tma_load_2d_pair(sb + A_BYTES, &maps[1], fb, kt * BK_BYTES, brow, pol_b);
                     }
                     __syncwarp();
                     issued = (issued & ~(1u << stage)) | (phase << stage);
@@ -343,7 +369,7 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
             // barrier until then
             if (lane == 0 && rank == 0) {
                 int no_abort = 0;
-                WaitCtx w2{&no_abort, p.dev_status};
+                WaitCtx w2{&no_abort, g.dev_status};
                 for (int s = 0; s < STAGES; ++s)
                     if (issued_any & (1u << s)) mbar_wait(&full_bar[s], (issued >> s) & 1u, w2);
             }
@@ -362,7 +388,9 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                 int stage = 0, slot = 0, wstage = 0;
                 uint32_t phase = 0, wphase = 0, done = 0;
                 bool ok = true;
-                for (int t = pair; t < p.num_tiles && ok; t += npairs) {
+                for (int t = pair; t < g.num_tiles && ok; t += npairs) {
+                    const PairProblem& P = g.prob[problem_of(g, t)];
+                    const int num_kt = (P.K + 255) / 256, k_atoms = P.K / L::K_ATOM;
                     for (int kt = 0; kt < num_kt; ++kt) {
                         bool got = mbar_wait(&full_bar[stage], phase, wc);
                         if (SF_SLOTS < STAGES && done >= (uint32_t)SF_SLOTS && got) {
@@ -406,9 +434,12 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                 int stage = 0, slot = 0, buf = 0;
                 uint32_t phase = 0, acc_phase = 0;
                 bool ok = true;
-                for (int t = pair; t < p.num_tiles && ok; t += npairs) {
+                for (int t = pair; t < g.num_tiles && ok; t += npairs) {
+                    const PairProblem& P = g.prob[problem_of(g, t)];
+                    const int num_kt = (P.K + 255) / 256, k_atoms = P.K / L::K_ATOM, k_steps = P.K / 64;
+                    (void)k_atoms;
                     int mb2, nb;
-                    tile_coords(t, p.num_mb2, p.num_nb, mb2, nb);
+                    tile_coords(t - P.first_tile, P.num_mb2, P.num_nb, mb2, nb);
                     const uint32_t sfb_off = (uint32_t)(((nb * BN) & 127) >> 5);
                     // the accumulator's previous tile has been read out by both epilogues
                     if (!__all_sync(0xffffffffu, mbar_wait_cluster(&acce_bar[buf], acc_phase ^ 1u, wc) ? 1 : 0)) {
@@ -461,7 +492,7 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                 if (elect_one()) tc_commit2_mc(&drain_bar, 0x1);
                 __syncwarp();
                 int no_abort = 0;
-                WaitCtx w2{&no_abort, p.dev_status};
+                WaitCtx w2{&no_abort, g.dev_status};
                 mbar_wait(&drain_bar, 0, w2);
             }
         }
@@ -471,18 +502,34 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
         const int q = warp & 3;                       // TMEM lane quarter
         const int h = (warp - 8) >> 2;                // column half: [0, BN/2) or [BN/2, BN)
         const int row_t = (int)rank * 128 + q * 32 + lane;    // row inside the pair tile
-        // MX operands have no tensor scale: a null scale reads as 1
-        const float alpha = __fmul_rn(p.a_scale ? *p.a_scale : 1.0f, p.b_scale ? *p.b_scale : 1.0f);
-        float g_y = 0.0f;
-        if (OUT == OUT_NVFP4) g_y = *p.y_scale;
-        const ScaleConsts sc_y = scale_consts(g_y);
+        // per-problem constants, refreshed when the tile sequence enters
+        // another problem (MX operands have no tensor scale: a null scale
+        // reads as 1)
+        int cur = -1;
+        float alpha = 0.0f, g_y = 0.0f;
+        ScaleConsts sc_y = scale_consts(0.0f);
         uint8_t* ebuf = smem + STAGES * STAGE_BYTES + (warp - 8) * 2 * C::EPI_BUF;
+        // the output is written once and not read again by this kernel: evict
+        // it from L2 first, so that its write-back to DRAM happens while the
+        // tensor cores run rather than in whatever kernel comes next
+        const uint64_t pol_y = policy_evict_first();
         int nstore = 0, buf = 0;
         uint32_t acc_phase = 0;
         float amax_run = 0.0f;
-        for (int t = pair; t < p.num_tiles; t += npairs) {
+        for (int t = pair; t < g.num_tiles; t += npairs) {
+            const int pi = problem_of(g, t);
+            const PairProblem& P = g.prob[pi];
+            if (pi != cur) {
+                if (OUT == OUT_NVFP4 && cur >= 0) flush_amax(amax_run, g.prob[cur].y_amax, lane);
+                cur = pi;
+                alpha = __fmul_rn(P.a_scale ? *P.a_scale : 1.0f, P.b_scale ? *P.b_scale : 1.0f);
+                if (OUT == OUT_NVFP4) {
+                    g_y = *P.y_scale;
+                    sc_y = scale_consts(g_y);
+                }
+            }
             int mb2, nb;
-            tile_coords(t, p.num_mb2, p.num_nb, mb2, nb);
+            tile_coords(t - P.first_tile, P.num_mb2, P.num_nb, mb2, nb);
             if (!__all_sync(0xffffffffu, mbar_wait(&accf_bar[buf], acc_phase, wc) ? 1 : 0)) break;
             tc_fence_after();
             uint32_t r[EPI_COLS];
@@ -508,11 +555,11 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                 // 32 columns (two 16-value blocks) at a time: 16 bytes of codes
                 // and two scale bytes (half a scale word) per row
                 const int64_t grow = (int64_t)mb2 * 256 + row_t;
-                const int kb4 = p.N / 64;
+                const int kb4 = P.N / 64;
 #pragma unroll
                 for (int c = 0; c < EPI_COLS / 32; ++c) {
                     const int ncol = n0 + c * 32;
-                    if (ncol >= p.N) continue;
+                    if (ncol >= P.N) continue;
                     uint32_t sfh = 0u, cw[4];
 #pragma unroll
                     for (int b = 0; b < 2; ++b) {
@@ -522,7 +569,7 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                         float ab = 0.0f;
 #pragma unroll
                         for (int j = 0; j < 16; ++j) ab = fmaxf(ab, fabsf(v[j]));
-                        if (grow < p.M) amax_run = fmaxf(amax_run, ab);
+                        if (grow < P.M) amax_run = fmaxf(amax_run, ab);
                         const uint32_t sfc = block_scale_code(ab, sc_y);
                         const float s = __fmul_rn(e4m3_to_f32(sfc), g_y);
                         float lo[8], hi[8];
@@ -532,34 +579,31 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                         cw[2 * b + 1] = quantize8(hi, s);
                         sfh |= sfc << (8 * b);
                     }
-                    if (grow < p.M)
-                        *reinterpret_cast<uint4*>(p.y_codes + grow * (p.N / 2) + ncol / 2) =
+                    if (grow < P.M)
+                        *reinterpret_cast<uint4*>(P.y_codes + grow * (P.N / 2) + ncol / 2) =
                             make_uint4(cw[0], cw[1], cw[2], cw[3]);
                     // rows past M inside the padded scale buffer get zero scales
-                    if (grow < (int64_t)((p.M + 127) / 128) * 128) {
+                    if (grow < (int64_t)((P.M + 127) / 128) * 128) {
                         const int rb = (int)(grow >> 7), rr = (int)(grow & 127);
                         const int64_t atom = (int64_t)rb * kb4 + ncol / 64;
-                        *reinterpret_cast<uint16_t*>(p.y_sf + atom * SF_ATOM + (rr & 31) * 16 + (rr >> 5) * 4 +
+                        *reinterpret_cast<uint16_t*>(P.y_sf + atom * SF_ATOM + (rr & 31) * 16 + (rr >> 5) * 4 +
                                                      ((ncol >> 4) & 3)) = (uint16_t)sfh;
                     }
                 }
             } else {
 #pragma unroll
                 for (int c = 0; c < EPI_COLS / 32; ++c) {
-                    if (n0 + c * 32 >= p.N) continue;
+                    if (n0 + c * 32 >= P.N) continue;
                     uint8_t* buf_s = ebuf + (nstore & 1) * C::EPI_BUF;
                     if (lane == 0) bulk_wait_group_read<1>();
                     __syncwarp();
-                    store_chunk<OUT, ACT>(&r[c * 32], alpha, buf_s, lane, &tmap_y, n0 + c * 32, m0);
+                    store_chunk<OUT, ACT>(&r[c * 32], alpha, buf_s, lane, &g.map[pi][4], n0 + c * 32, m0, pol_y);
                     ++nstore;
                 }
             }
         }
         if (lane == 0) bulk_wait_group<0>();
-        if (OUT == OUT_NVFP4 && p.y_amax != nullptr) {
-            for (int o = 16; o > 0; o >>= 1) amax_run = fmaxf(amax_run, __shfl_xor_sync(0xffffffffu, amax_run, o));
-            if (lane == 0 && amax_run > 0.0f) atomicMax(reinterpret_cast<int*>(p.y_amax), __float_as_int(amax_run));
-        }
+        if (OUT == OUT_NVFP4 && cur >= 0) flush_amax(amax_run, g.prob[cur].y_amax, lane);
     }
 
     tc_fence_before();
@@ -572,50 +616,70 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     }
 }
 
-template <int BN, int OUT, int ACT, bool MXS>
-cudaError_t launch_out(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) {
-    using C = Cfg<BN, OUT, MXS>;
+// Tensor maps of one problem: A and B codes, their scale atoms, and Y (bf16 or
+// FP32; with the NVFP4 output the map is unused and a copy of A's is kept).
+template <int BN, int OUT, bool MXS>
+static bool encode_maps(const GemmW4A4Args& a, CUtensorMap (&m)[5]) {
     using L = Lay<BN, MXS>;
-    CUtensorMap ta, tb, tsa, tsb, ty;
     const uint64_t kh = (uint64_t)(a.K / 2);
     const uint64_t atoms_a = (uint64_t)((a.M + 127) / 128) * (uint64_t)(a.K / L::K_ATOM);
     const uint64_t atoms_b = (uint64_t)((a.N + 127) / 128) * (uint64_t)(a.K / L::K_ATOM);
-    if (make_tmap_2d(&ta, a.a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kh, (uint64_t)a.M, kh, BK_BYTES, 128,
+    if (make_tmap_2d(&m[0], a.a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kh, (uint64_t)a.M, kh, BK_BYTES, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
-        make_tmap_2d(&tb, a.b_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kh, (uint64_t)a.N, kh, BK_BYTES, L::B_ROWS,
+        make_tmap_2d(&m[1], a.b_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kh, (uint64_t)a.N, kh, BK_BYTES, L::B_ROWS,
                      CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
-        make_tmap_2d(&tsa, a.a_sf, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, 128, atoms_a, SF_ATOM, 128, L::SF_PER,
+        make_tmap_2d(&m[2], a.a_sf, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, 128, atoms_a, SF_ATOM, 128, L::SF_PER,
                      CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
-        make_tmap_2d(&tsb, a.b_sf, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, 128, atoms_b, SF_ATOM, 128, L::SF_PER,
+        make_tmap_2d(&m[3], a.b_sf, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, 128, atoms_b, SF_ATOM, 128, L::SF_PER,
                      CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
-        return cudaErrorInvalidValue;
+        return false;
     CUresult r = CUDA_SUCCESS;
     if (OUT == OUT_BF16)
-        r = make_tmap_2d(&ty, a.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.N, (uint64_t)a.M,
+        r = make_tmap_2d(&m[4], a.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.N, (uint64_t)a.M,
                          (uint64_t)a.N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
     else if (OUT == OUT_F32)
-        r = make_tmap_2d(&ty, a.y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)a.N, (uint64_t)a.M,
+        r = make_tmap_2d(&m[4], a.y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)a.N, (uint64_t)a.M,
                          (uint64_t)a.N * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
     else
-        ty = ta;
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+        m[4] = m[0];
+    return r == CUDA_SUCCESS;
+}
 
-    Params p;
-    p.a_scale = a.a_scale;
-    p.b_scale = a.b_scale;
-    p.M = (int)a.M;
-    p.N = (int)a.N;
-    p.K = (int)a.K;
-    p.num_mb2 = (int)((a.M + 255) / 256);
-    p.num_nb = (int)(a.N / BN);
-    p.num_tiles = p.num_mb2 * p.num_nb;
-    p.y_codes = a.y_codes;
-    p.y_sf = a.y_sf;
-    p.y_scale = a.y_scale;
-    p.y_amax = a.y_amax;
-    p.dev_status = a.dev_status;
+template <int G, int BN, int OUT, int ACT, bool MXS>
+cudaError_t launch_out(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream) {
+    using C = Cfg<BN, OUT, MXS>;
+    if (count < 1 || count > G) return cudaErrorInvalidValue;
+    PairGroup<G> g;
+    int tiles = 0;
+    for (int i = 0; i < count; ++i) {
+        const GemmW4A4Args& a = probs[i];
+        if (!encode_maps<BN, OUT, MXS>(a, g.map[i])) return cudaErrorInvalidValue;
+        PairProblem& P = g.prob[i];
+        P.a_scale = a.a_scale;
+        P.b_scale = a.b_scale;
+        P.M = (int)a.M;
+        P.N = (int)a.N;
+        P.K = (int)a.K;
+        P.num_mb2 = (int)((a.M + 255) / 256);
+        P.num_nb = (int)(a.N / BN);
+        P.first_tile = tiles;
+        P.y_codes = a.y_codes;
+        P.y_sf = a.y_sf;
+        P.y_scale = a.y_scale;
+        P.y_amax = a.y_amax;
+        tiles += P.num_mb2 * P.num_nb;
+    }
+    for (int i = count; i < G; ++i) {
+        g.prob[i] = g.prob[0];
+        g.prob[i].first_tile = tiles;            // never reached
+        for (int m = 0; m < 5; ++m) g.map[i][m] = g.map[0][m];
+    }
+    g.count = count;
+    g.num_tiles = tiles;
+    g.dev_status = probs[0].dev_status;
+    if (tiles == 0) return cudaSuccess;
 
-    auto kern = gemm2_kernel<BN, OUT, ACT, MXS>;
+    auto kern = gemm2_kernel<G, BN, OUT, ACT, MXS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
 
@@ -635,51 +699,75 @@ cudaError_t launch_out(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) 
     cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
     if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess || max_clusters < 1)
         max_clusters = num_sms / 2;
-    int pairs = p.num_tiles < max_clusters ? p.num_tiles : max_clusters;
+    const int pairs = tiles < max_clusters ? tiles : max_clusters;
     cfg.gridDim = dim3(2 * pairs, 1, 1);
-    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, ty, p);
+    e = cudaLaunchKernelEx(&cfg, kern, g);
     count_launch(1);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
-template <int BN>
-cudaError_t launch_bn(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) {
+template <int G, int BN>
+cudaError_t launch_bn(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream) {
+    const GemmW4A4Args& a = probs[0];
     const bool gelu = a.act == ACT_GELU_TANH;
     if (a.mx) {
-        // MX operands: bf16 or FP32 output (no NVFP4 output of an MX product)
-        if (a.y == nullptr) return cudaErrorInvalidValue;
+        // MX operands: bf16 or FP32 output (no NVFP4 output of an MX product),
+        // plain calls only
+        if (G != 1 || a.y == nullptr) return cudaErrorInvalidValue;
         if (a.y_dtype == 1)
-            return gelu ? launch_out<BN, OUT_F32, ACT_GELU_TANH, true>(a, num_sms, stream)
-                        : launch_out<BN, OUT_F32, ACT_NONE, true>(a, num_sms, stream);
-        return gelu ? launch_out<BN, OUT_BF16, ACT_GELU_TANH, true>(a, num_sms, stream)
-                    : launch_out<BN, OUT_BF16, ACT_NONE, true>(a, num_sms, stream);
+            return gelu ? launch_out<1, BN, OUT_F32, ACT_GELU_TANH, true>(probs, count, num_sms, stream)
+                        : launch_out<1, BN, OUT_F32, ACT_NONE, true>(probs, count, num_sms, stream);
+        return gelu ? launch_out<1, BN, OUT_BF16, ACT_GELU_TANH, true>(probs, count, num_sms, stream)
+                    : launch_out<1, BN, OUT_BF16, ACT_NONE, true>(probs, count, num_sms, stream);
     }
     if (a.y != nullptr) {
         if (a.y_dtype == 1)
-            return gelu ? launch_out<BN, OUT_F32, ACT_GELU_TANH, false>(a, num_sms, stream)
-                        : launch_out<BN, OUT_F32, ACT_NONE, false>(a, num_sms, stream);
-        return gelu ? launch_out<BN, OUT_BF16, ACT_GELU_TANH, false>(a, num_sms, stream)
-                    : launch_out<BN, OUT_BF16, ACT_NONE, false>(a, num_sms, stream);
+            return gelu ? launch_out<G, BN, OUT_F32, ACT_GELU_TANH, false>(probs, count, num_sms, stream)
+                        : launch_out<G, BN, OUT_F32, ACT_NONE, false>(probs, count, num_sms, stream);
+        return gelu ? launch_out<G, BN, OUT_BF16, ACT_GELU_TANH, false>(probs, count, num_sms, stream)
+                    : launch_out<G, BN, OUT_BF16, ACT_NONE, false>(probs, count, num_sms, stream);
     }
-    return gelu ? launch_out<BN, OUT_NVFP4, ACT_GELU_TANH, false>(a, num_sms, stream)
-                : launch_out<BN, OUT_NVFP4, ACT_NONE, false>(a, num_sms, stream);
+    return gelu ? launch_out<G, BN, OUT_NVFP4, ACT_GELU_TANH, false>(probs, count, num_sms, stream)
+                : launch_out<G, BN, OUT_NVFP4, ACT_NONE, false>(probs, count, num_sms, stream);
 }
 
 }  // namespace w4a4_2sm
 
-// N % 256 == 0: 256 x 256 tiles; otherwise (N % 192 == 0) 256 x 192 tiles
-// with a double-buffered accumulator.  A pair MMA (M = 256, K = 64) takes
-// about 120 cycles whatever its N up to 192 and 128 at N = 256, so only the
-// 256-wide tile runs the tensor cores at full rate.  NVFP4_PAIR_TILE_N (192
-// or 256) picks the tile width for measurements, where N allows it.
-cudaError_t launch_gemm_w4a4_2sm(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) {
-    using namespace w4a4_2sm;
+// The pair kernel's tile width for a set of problems: 256 when every N is a
+// multiple of 256, else 192 when every N is a multiple of 192, else 0 (not
+// supported).  A pair MMA (M = 256, K = 64) takes about 120 cycles whatever
+// its N up to 192 and 128 at N = 256, so only the 256-wide tile runs the
+// tensor cores at full rate.  NVFP4_PAIR_TILE_N (192 or 256) picks the width
+// for measurements, where the shapes allow it.
+int gemm_w4a4_2sm_tile_n(const GemmW4A4Args* probs, int count) {
+    bool all256 = true, all192 = true;
+    for (int i = 0; i < count; ++i) {
+        all256 = all256 && probs[i].N % 256 == 0;
+        all192 = all192 && probs[i].N % 192 == 0;
+    }
     const char* env = getenv("NVFP4_PAIR_TILE_N");
     const int forced = env ? atoi(env) : 0;
-    const bool can192 = a.N % 192 == 0, can256 = a.N % 256 == 0;
-    if (can256 && (forced != 192 || !can192)) return launch_bn<256>(a, num_sms, stream);
-    if (can192) return launch_bn<192>(a, num_sms, stream);
+    if (all256 && (forced != 192 || !all192)) return 256;
+    if (all192) return 192;
+    return 0;
+}
+
+cudaError_t launch_gemm_w4a4_2sm(const GemmW4A4Args& a, int num_sms, cudaStream_t stream) {
+    using namespace w4a4_2sm;
+    const int bn = gemm_w4a4_2sm_tile_n(&a, 1);
+    if (bn == 256) return launch_bn<1, 256>(&a, 1, num_sms, stream);
+    if (bn == 192) return launch_bn<1, 192>(&a, 1, num_sms, stream);
+    return cudaErrorInvalidValue;
+}
+
+// Up to kPairGroup problems with one output kind and activation in one launch
+// of the pair kernel (one tile space).
+cudaError_t launch_gemm_w4a4_2sm_grouped(const GemmW4A4Args* probs, int count, int num_sms, cudaStream_t stream) {
+    using namespace w4a4_2sm;
+    const int bn = gemm_w4a4_2sm_tile_n(probs, count);
+    if (bn == 256) return launch_bn<kPairGroup, 256>(probs, count, num_sms, stream);
+    if (bn == 192) return launch_bn<kPairGroup, 192>(probs, count, num_sms, stream);
     return cudaErrorInvalidValue;
 }
 

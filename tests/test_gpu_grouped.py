@@ -138,3 +138,57 @@ def test_grouped_skips_empty_problems_and_group_of_one(cuda_ok):
     n0 = nv.nvfp4_launch_count()
     nv.nvfp4_gemm_w4a4_grouped(probs[:1])           # only an empty problem: nothing launched
     assert nv.nvfp4_launch_count() == n0
+
+
+PAIR_GROUPS = {256: [(300, 512, 1152), (128, 256, 256), (77, 768, 4096), (513, 256, 320)],
+               192: [(300, 384, 1152), (128, 192, 256), (77, 1152, 4096), (513, 576, 320)]}
+
+
+@pytest.mark.parametrize("bn", [256, 192])
+@pytest.mark.parametrize("out_dtype,tol", [(torch.bfloat16, TOL_BF16), (torch.float32, TOL_F32)])
+def test_grouped_on_the_pair_kernel(cuda_ok, monkeypatch, bn, out_dtype, tol):
+    """A group whose every N allows one pair tile width runs on the CTA-pair
+    kernel (forced here: the shapes are small); each output meets the oracle's
+    tolerance and equals the single pair-kernel call bit for bit (same tiles,
+    same accumulation order)."""
+    monkeypatch.setenv("NVFP4_GEMM_KERNEL", "pair")
+    monkeypatch.setenv("NVFP4_PAIR_TILE_N", str(bn))
+    shapes = PAIR_GROUPS[bn]
+    ops = [_operands(M, N, K, 140 + i) for i, (M, N, K) in enumerate(shapes)]
+    pairs = [(upload(*a, M, K), upload(*b, N, K)) for (a, b), (M, N, K) in zip(ops, shapes)]
+    ys = nv.gemm_w4a4_grouped(pairs, out_dtype=out_dtype)
+    singles = [nv.gemm_w4a4(A, B, out_dtype=out_dtype) for A, B in pairs]
+    torch.cuda.synchronize()
+    view = torch.int16 if out_dtype == torch.bfloat16 else torch.int32
+    for (a, b), (M, N, K), y, y1 in zip(ops, shapes, ys, singles):
+        yref = oracle.gemm_w4a4(*a, *b)
+        e = norm_err(y.float().cpu().numpy(), yref, oracle.dequantize(*a), oracle.dequantize(*b))
+        assert e <= tol, ((M, N, K), e)
+        assert torch.equal(y.view(view), y1.view(view))
+
+
+def test_grouped_pair_kernel_nvfp4_epilogue_bit_exact_and_amax_per_problem(cuda_ok, monkeypatch):
+    monkeypatch.setenv("NVFP4_GEMM_KERNEL", "pair")
+    shapes = [(256, 384, 1024), (300, 192, 256), (130, 576, 512)]
+    probs, expect = [], []
+    for i, (M, N, K) in enumerate(shapes):
+        ac, asf = _exact_operands(M, K, 30 + i)
+        bc, bsf = _exact_operands(N, K, 40 + i)
+        ga, gb = 0.5, 0.25 * (i + 1)
+        yref = oracle.gemm_w4a4(ac, asf, ga, bc, bsf, gb).astype(np.float32)
+        gy = float(np.float32(np.abs(yref).max() / 2688.0 * 0.8))
+        oc, osf, _ = oracle.quantize(yref, scale=gy)
+        A, B = upload(ac, asf, ga, M, K), upload(bc, bsf, gb, N, K)
+        q = nv.NVFP4Tensor.empty(M, N, "cuda")
+        q.scale.fill_(gy)
+        amax = torch.zeros(1, dtype=torch.float32, device="cuda")
+        probs.append(dict(a_codes=A.codes, a_sf=A.sf, a_scale=A.scale, b_codes=B.codes, b_sf=B.sf,
+                          b_scale=B.scale, M=M, N=N, K=K, y_codes=q.codes, y_sf=q.sf, y_scale=q.scale,
+                          y_amax=amax))
+        expect.append((oc, osf, np.abs(yref).max(), q, amax))
+    nv.nvfp4_gemm_w4a4_grouped(probs)
+    torch.cuda.synchronize()
+    for oc, osf, am, q, amax in expect:
+        assert np.array_equal(q.codes.cpu().numpy(), oc)
+        assert np.array_equal(q.sf.cpu().numpy()[: osf.size], osf)
+        assert amax.item() == am
