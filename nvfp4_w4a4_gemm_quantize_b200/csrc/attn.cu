@@ -24,6 +24,7 @@
 // and issues S = Q K^T, warp 2 issues O += P V (two issuers, so that neither
 // product waits behind the other's operands); warps 4-7 softmax and output;
 // every wait is bounded.
+#include <cstdlib>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -483,6 +484,422 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
     }
 }
 
+// ---------------------------------------------------------------------------
+// Two query tiles per CTA.  A work item is 256 queries of one head (query
+// tiles A and B); the K and V^T tiles are loaded once for both.  Two softmax
+// warpgroups, one per tile, take turns on the tensor core: while one computes
+// its exponentials the other's S = Q K^T runs, so the special-function units
+// (the exponentials) rather than one warp's latency set the pace.
+// TMEM: one S buffer, used in turn by A and B (a group releases it as soon as
+// its logits are in registers), O_A, O_B, and the scale slots.  Shared
+// memory: three bf16 P tiles taken in turn by the uses A0, B0, A1, B1, ... (a
+// group writes use u once the product of use u - 3 has read that tile, so it
+// never waits for its own previous product), a 3-stage K ring, a 2-stage V^T
+// ring and two Q buffers per tile.
+// Roles (384 threads): warp 0 Q and K producer, warp 3 V^T producer, warp 1 S
+// issuer (and TMEM owner), warp 2 P V issuer; warps 4-7 softmax of tile A,
+// warps 8-11 of tile B.  The register budget moves to the softmax warpgroups
+// (setmaxnreg: 48 for warpgroup 0, 224 for 1 and 2; 128 x 48 + 256 x 224 <=
+// 384 x 168).
+constexpr int kThreads2 = 384;
+constexpr int kKStages2 = 3;
+constexpr int kVStages2 = 2;
+constexpr int kPBufs2 = 3;                                   // P tiles, rotated over the two groups' uses
+constexpr int kOffQ2 = 0;                                    // + (qb * 2 + g) * kKStageBytes
+constexpr int kOffK2 = 4 * kKStageBytes;
+constexpr int kOffV2 = kOffK2 + kKStages2 * kKStageBytes;
+constexpr int kOffP2 = kOffV2 + kVStages2 * kTileBf16;        // + b * kTileBf16
+constexpr int kSmemBytes2 = kOffP2 + kPBufs2 * kTileBf16 + 1024;
+static_assert(kOffK2 % 1024 == 0 && kOffV2 % 1024 == 0 && kOffP2 % 1024 == 0, "swizzled tiles are 1024-byte aligned");
+static_assert(kSmemBytes2 <= 232448 - 512, "shared memory budget");
+constexpr uint32_t kColS2 = 0;                               // S: [0, 128)
+constexpr uint32_t kColO2 = 128;                             // O_g: [128 + 128 g, 256 + 128 g)
+constexpr uint32_t kColSfQ2 = 384;                           // Q scales: (qb * 2 + g) * 8
+constexpr uint32_t kColSfK2 = 416;                           // K scales: (n & 1) * 8
+constexpr int kRegsLow2 = 48;
+constexpr int kRegsHigh2 = 224;
+static_assert(128 * kRegsLow2 + 256 * kRegsHigh2 <= kThreads2 * 168, "register split exceeds the launch budget");
+
+__global__ void __launch_bounds__(kThreads2, 1)
+attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+             const __grid_constant__ CUtensorMap tmap_vt, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t q_full[2], q_empty[2], k_full[kKStages2], k_empty[kKStages2];
+    __shared__ __align__(8) uint64_t v_full[kVStages2], v_empty[kVStages2];
+    __shared__ __align__(8) uint64_t s_full[2], s_empty, p_full[kPBufs2], p_empty[kPBufs2];
+    __shared__ __align__(8) uint64_t o_done[2], o_free[2];
+    __shared__ __align__(8) uint64_t drain_s, drain_o;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    WaitCtx wc{&abort_sh, p.dev_status};
+    const int ntiles = p.Lk / kBK;
+    const int qpairs = p.Lq / (2 * kBQ);
+    const int nitems = p.H * qpairs;
+    auto item_head = [&](int it) { return it / qpairs; };
+    auto item_qrow = [&](int it, int g) { return (it / qpairs) * p.Lq + ((it % qpairs) * 2 + g) * kBQ; };
+
+    if (threadIdx.x == 0) {
+        abort_sh = 0;
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&q_full[b], 1);
+            mbar_init(&q_empty[b], 1);               // the item's last S product's commit
+            mbar_init(&s_full[b], 1);
+            mbar_init(&o_done[b], 1);
+            mbar_init(&o_free[b], 4);                // the group's softmax warps have read O out
+        }
+        for (int s = 0; s < kKStages2; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);               // both S products' commit
+        }
+        for (int s = 0; s < kVStages2; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);               // both P V products' commit
+        }
+        for (int b = 0; b < kPBufs2; ++b) {
+            mbar_init(&p_full[b], 4);                // written by one group's softmax warps
+            mbar_init(&p_empty[b], 1);               // the P V product that read it
+        }
+        mbar_init(&s_empty, 4);                      // the S buffer read out by one group
+        mbar_init(&drain_s, 1);
+        mbar_init(&drain_o, 1);
+        fence_barrier_init();
+        tma_prefetch_desc(&tmap_q);
+        tma_prefetch_desc(&tmap_k);
+        tma_prefetch_desc(&tmap_vt);
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_sh, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+
+    if (warp < 4) {
+        regs_dec<kRegsLow2>();
+        if (warp == 0) {
+            // -------------------------------------------------------- Q (both tiles) and K producer
+            const uint64_t pol = policy_evict_normal();
+            bool ok = true;
+            int n = 0, i = 0;
+            for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++i) {
+                const int qb = i & 1, krow0 = item_head(it) * p.Lk;
+                if (!__all_sync(0xffffffffu, mbar_wait(&q_empty[qb], ((uint32_t)(i >> 1) & 1u) ^ 1u, wc) ? 1 : 0)) {
+                    ok = false;
+                    break;
+                }
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(&q_full[qb], 2 * kKStageBytes);
+                    for (int g = 0; g < 2; ++g) {
+                        uint8_t* qs = smem + kOffQ2 + (qb * 2 + g) * kKStageBytes;
+                        const int qrow0 = item_qrow(it, g);
+                        tma_load_2d(qs, &tmap_q, &q_full[qb], 0, qrow0, pol);
+                        bulk_load(qs + kCodeBytes, p.q_sf + (int64_t)(qrow0 >> 7) * kSfBytes, kSfBytes, &q_full[qb],
+                                  pol);
+                    }
+                }
+                __syncwarp();
+                for (int j = 0; j < ntiles; ++j, ++n) {
+                    const int s = n % kKStages2;
+                    const uint32_t ph = (uint32_t)(n / kKStages2) & 1u;
+                    if (!__all_sync(0xffffffffu, mbar_wait(&k_empty[s], ph ^ 1u, wc) ? 1 : 0)) { ok = false; break; }
+                    uint8_t* st = smem + kOffK2 + s * kKStageBytes;
+                    const int kr = krow0 + j * kBK;
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(&k_full[s], kKStageBytes);
+                        tma_load_2d(st, &tmap_k, &k_full[s], 0, kr, pol);
+                        bulk_load(st + kCodeBytes, p.k_sf + (int64_t)(kr >> 7) * kSfBytes, kSfBytes, &k_full[s], pol);
+                    }
+                    __syncwarp();
+                }
+            }
+            // every load this warp issued has landed before the CTA may exit
+            if (lane == 0) {
+                int dummy = 0;
+                WaitCtx w2{&dummy, p.dev_status};
+                for (int q = (i > 2 ? i - 2 : 0); q < i; ++q) mbar_wait(&q_full[q & 1], (uint32_t)(q >> 1) & 1u, w2);
+                for (int m = (n > kKStages2 ? n - kKStages2 : 0); m < n; ++m)
+                    mbar_wait(&k_full[m % kKStages2], (uint32_t)(m / kKStages2) & 1u, w2);
+            }
+        } else if (warp == 3) {
+            // -------------------------------------------------------- V^T producer
+            const uint64_t pol = policy_evict_normal();
+            bool ok = true;
+            int n = 0;
+            for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+                const int h = item_head(it);
+                for (int j = 0; j < ntiles; ++j, ++n) {
+                    const int s = n % kVStages2;
+                    const uint32_t ph = (uint32_t)(n / kVStages2) & 1u;
+                    if (!__all_sync(0xffffffffu, mbar_wait(&v_empty[s], ph ^ 1u, wc) ? 1 : 0)) { ok = false; break; }
+                    uint8_t* st = smem + kOffV2 + s * kTileBf16;
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(&v_full[s], kTileBf16);
+                        tma_load_2d(st, &tmap_vt, &v_full[s], j * kBK, h * kD, pol);
+                        tma_load_2d(st + kChunk, &tmap_vt, &v_full[s], j * kBK + 64, h * kD, pol);
+                    }
+                    __syncwarp();
+                }
+            }
+            if (lane == 0) {
+                int dummy = 0;
+                WaitCtx w2{&dummy, p.dev_status};
+                for (int m = (n > kVStages2 ? n - kVStages2 : 0); m < n; ++m)
+                    mbar_wait(&v_full[m % kVStages2], (uint32_t)(m / kVStages2) & 1u, w2);
+            }
+        } else if (warp == 1) {
+            // -------------------------------------------------------- S = Q K^T issuer (and TMEM owner)
+            // The S buffer's uses alternate A, B, A, B, ...; use u waits until
+            // the group of use u - 1 has read it out.
+            constexpr uint32_t idesc_s = idesc_nvf4(kBQ, kBK);
+            const uint32_t sm0 = smem_u32(smem);
+            bool ok = true;
+            int n = 0, i = 0;
+            uint32_t u = 0;
+            for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++i) {
+                const int qb = i & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&q_full[qb], (uint32_t)(i >> 1) & 1u, wc) ? 1 : 0)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (elect_one()) {
+                    for (int g = 0; g < 2; ++g) {
+                        const uint32_t qs = sm0 + kOffQ2 + (qb * 2 + g) * kKStageBytes;
+                        const uint32_t sfq = tmem + kColSfQ2 + (qb * 2 + g) * 8;
+                        tc_cp_32x128b_warpx4(sfq, sdesc_sf(qs + kCodeBytes));
+                        tc_cp_32x128b_warpx4(sfq + 4, sdesc_sf(qs + kCodeBytes + 512));
+                    }
+                }
+                __syncwarp();
+                for (int j = 0; j < ntiles && ok; ++j, ++n) {
+                    const int s = n % kKStages2;
+                    if (!__all_sync(0xffffffffu, mbar_wait(&k_full[s], (uint32_t)(n / kKStages2) & 1u, wc) ? 1 : 0)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = sm0 + kOffK2 + s * kKStageBytes;
+                    const uint32_t sfk = tmem + kColSfK2 + (n & 1) * 8;
+                    if (elect_one()) {
+                        tc_cp_32x128b_warpx4(sfk, sdesc_sf(st + kCodeBytes));
+                        tc_cp_32x128b_warpx4(sfk + 4, sdesc_sf(st + kCodeBytes + 512));
+                    }
+                    __syncwarp();
+                    for (int g = 0; g < 2; ++g, ++u) {
+                        if (!__all_sync(0xffffffffu, mbar_wait(&s_empty, (u & 1u) ^ 1u, wc) ? 1 : 0)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t qs = sm0 + kOffQ2 + (qb * 2 + g) * kKStageBytes;
+                        const uint32_t sfq = tmem + kColSfQ2 + (qb * 2 + g) * 8;
+                        if (elect_one()) {
+#pragma unroll
+                            for (int ks = 0; ks < 2; ++ks)
+                                tc_mma_nvf4(tmem + kColS2, sdesc_kmajor_sw64(qs + ks * 32),
+                                            sdesc_kmajor_sw64(st + ks * 32), idesc_s, sfq + ks * 4, sfk + ks * 4,
+                                            ks != 0 ? 1u : 0u);
+                            tc_commit(&s_full[g]);
+                            if (g == 1) {
+                                tc_commit(&k_empty[s]);
+                                if (j == ntiles - 1) tc_commit(&q_empty[qb]);
+                            }
+                        }
+                        __syncwarp();
+                    }
+                }
+            }
+            if (elect_one()) tc_commit(&drain_s);
+            __syncwarp();
+            int dummy = 0;
+            WaitCtx w2{&dummy, p.dev_status};
+            mbar_wait(&drain_s, 0, w2);
+        } else {
+            // -------------------------------------------------------- O_g += P_g V issuer
+            constexpr uint32_t idesc_o = idesc_bf16(kBQ, kD);
+            const uint32_t sm0 = smem_u32(smem);
+            bool ok = true;
+            int n = 0, i = 0;
+            for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++i) {
+                for (int j = 0; j < ntiles && ok; ++j, ++n) {
+                    const int s = n % kVStages2;
+                    if (!__all_sync(0xffffffffu, mbar_wait(&v_full[s], (uint32_t)(n / kVStages2) & 1u, wc) ? 1 : 0)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t vt = sm0 + kOffV2 + s * kTileBf16;
+                    for (int g = 0; g < 2; ++g) {
+                        const uint32_t u = 2u * (uint32_t)n + (uint32_t)g;
+                        const int pb = (int)(u % kPBufs2);
+                        if (!__all_sync(0xffffffffu, mbar_wait(&p_full[pb], (u / kPBufs2) & 1u, wc) ? 1 : 0) ||
+                            // the first product of an item overwrites O_g: the previous item's O_g has been read out
+                            (j == 0 && i >= 1 &&
+                             !__all_sync(0xffffffffu, mbar_wait(&o_free[g], (uint32_t)(i - 1) & 1u, wc) ? 1 : 0))) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t pt = sm0 + kOffP2 + pb * kTileBf16;
+                        if (elect_one()) {
+#pragma unroll
+                            for (int kc = 0; kc < 2; ++kc)
+#pragma unroll
+                                for (int ks = 0; ks < 4; ++ks)
+                                    tc_mma_bf16(tmem + kColO2 + g * kD, sdesc_kmajor_sw128(pt + kc * kChunk + ks * 32),
+                                                sdesc_kmajor_sw128(vt + kc * kChunk + ks * 32), idesc_o,
+                                                (j | kc | ks) != 0 ? 1u : 0u);
+                            tc_commit(&p_empty[pb]);
+                            tc_commit(&o_done[g]);
+                            if (g == 1) tc_commit(&v_empty[s]);
+                        }
+                        __syncwarp();
+                    }
+                }
+            }
+            if (elect_one()) tc_commit(&drain_o);
+            __syncwarp();
+            int dummy = 0;
+            WaitCtx w2{&dummy, p.dev_status};
+            mbar_wait(&drain_o, 0, w2);
+        }
+    } else {
+        regs_inc<kRegsHigh2>();
+        // ------------------------------------------------------------ softmax and output of tile g
+        const int g = (warp - 4) >> 2;              // 0: tile A (warps 4-7), 1: tile B (warps 8-11)
+        const int q = warp & 3;                     // TMEM lane quarter
+        const int r = q * 32 + lane;                // query row in the tile
+        const float c = __fmul_rn(__fmul_rn(*p.g_q, *p.g_k), 1.4426950408889634f / 11.313708498984761f);
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        const uint32_t col_o = kColO2 + g * kD;
+        bool ok = true;
+        int n = 0;
+        for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+            const float bias = p.s_head ? log2f(p.s_head[item_head(it)]) : 0.0f;
+            float m = -INFINITY, l = 0.0f;
+            for (int j = 0; j < ntiles; ++j, ++n) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&s_full[g], (uint32_t)n & 1u, wc) ? 1 : 0)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t v[kBK];
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4)
+                    tmem_ld_32x32b_x32(tmem + lane_base + kColS2 + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c4 * 32]));
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_empty);
+                float mx8[8];
+#pragma unroll
+                for (int i8 = 0; i8 < 8; ++i8) mx8[i8] = -INFINITY;
+#pragma unroll
+                for (int i8 = 0; i8 < kBK; ++i8) mx8[i8 & 7] = fmaxf(mx8[i8 & 7], __uint_as_float(v[i8]));
+                const float smax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                const float mt = fmaf(smax, c, bias);
+                // lazy rescaling, as in the one-tile kernel
+                const bool move = mt > m + 8.0f;
+                const float mref = move ? mt : m;
+                const float alpha = move ? ex2(m - mt) : 1.0f;
+                const float off = bias - mref;
+                float sum4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                // P tile of use u = 2 n + g: the product that read it at use u - 3 is done
+                const uint32_t u = 2u * (uint32_t)n + (uint32_t)g;
+                const int pb = (int)(u % kPBufs2);
+                if (!__all_sync(0xffffffffu, mbar_wait(&p_empty[pb], ((u / kPBufs2) & 1u) ^ 1u, wc) ? 1 : 0)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* pbase = smem + kOffP2 + pb * kTileBf16 + r * 128;
+#pragma unroll
+                for (int c8 = 0; c8 < 16; ++c8) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const float e0 = ex2(fmaf(__uint_as_float(v[c8 * 8 + 2 * t]), c, off));
+                        const float e1 = ex2(fmaf(__uint_as_float(v[c8 * 8 + 2 * t + 1]), c, off));
+                        sum4[t] += e0 + e1;
+                        __nv_bfloat162 hb = __floats2bfloat162_rn(e0, e1);
+                        w[t] = *reinterpret_cast<uint32_t*>(&hb);
+                    }
+                    const int kc = c8 >> 3, pos = (c8 & 7) ^ (r & 7);
+                    *reinterpret_cast<uint4*>(pbase + kc * kChunk + pos * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+                l = fmaf(l, alpha, (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+                m = mref;
+                // This group's previous product (o_done completion n - 1) is waited
+                // for before O_g is rescaled, and on an item's last tile, so that
+                // the read-out below waits with at most one product pending.
+                // The P wait above already covers completion n - 2.
+                const bool rescale = j >= 1 && __any_sync(0xffffffffu, alpha != 1.0f);
+                if ((rescale || (j >= 1 && j == ntiles - 1)) &&
+                    !__all_sync(0xffffffffu, mbar_wait(&o_done[g], (uint32_t)(n - 1) & 1u, wc) ? 1 : 0)) {
+                    ok = false;
+                    break;
+                }
+                if (rescale) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        uint32_t o[32];
+                        tmem_ld_32x32b_x32(tmem + lane_base + col_o + c4 * 32, o);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i8 = 0; i8 < 32; ++i8) o[i8] = __float_as_uint(__uint_as_float(o[i8]) * alpha);
+                        tmem_st_x32(tmem + lane_base + col_o + c4 * 32, o);
+                    }
+                    tmem_st_wait();
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[pb]);
+            }
+            if (!ok) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(&o_done[g], (uint32_t)(n - 1) & 1u, wc) ? 1 : 0)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t o[kD];
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4)
+                tmem_ld_32x32b_x32(tmem + lane_base + col_o + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[c4 * 32]));
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&o_free[g]);
+            const float sc = __fdiv_rn(*p.g_v, l);
+            uint16_t* orow = p.out + (int64_t)(item_qrow(it, g) + r) * kD;
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+                uint32_t w[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(o[t * 8 + 2 * u]) * sc,
+                                                              __uint_as_float(o[t * 8 + 2 * u + 1]) * sc);
+                    w[u] = *reinterpret_cast<uint32_t*>(&hb);
+                }
+                *reinterpret_cast<uint4*>(orow + t * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
 // V [H*Lk, d] NVFP4 -> V^T [H*d, Lk] bf16, exact (the tensor scale g_v is
 // applied with the output).  A CTA per (64 keys, head); thread t decodes the
 // 16 code bytes of key t / 4, d = 32 (t % 4) .. + 31.  Two threads of
@@ -578,15 +995,25 @@ cudaError_t launch_attention(const uint8_t* q_codes, const uint8_t* q_sf, const 
     p.Lk = (int)Lk;
     p.H = (int)H;
     p.dev_status = dev_status;
-    e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
         (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
-    const int64_t items = (Lq / kBQ) * H;
+    // two query tiles per CTA when a head's query tiles pair up
+    // (NVFP4_ATTN_TILES=1 keeps one, for measurements)
+    const char* env = getenv("NVFP4_ATTN_TILES");
+    const bool two = (Lq / kBQ) % 2 == 0 && !(env && env[0] == '1');
+    const int64_t items = (Lq / (two ? 2 * kBQ : kBQ)) * H;
     const unsigned grid = (unsigned)(items < sms ? items : sms);     // one persistent CTA per SM
-    attn_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tvt, p);
+    if (two) {
+        e = cudaFuncSetAttribute(attn2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes2);
+        if (e != cudaSuccess) return e;
+        attn2_kernel<<<grid, kThreads2, kSmemBytes2, stream>>>(tq, tk, tvt, p);
+    } else {
+        e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attn_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tvt, p);
+    }
     count_launch(1);
     return cudaGetLastError();
 }

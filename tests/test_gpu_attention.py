@@ -53,9 +53,13 @@ def test_attention_small_all_rows(cuda_ok):
     assert np.max(np.abs(o1 - o2)) <= 4e-3 * np.abs(o1).max()
 
 
-def test_attention_sharp_rows_across_tiles(cuda_ok):
+@pytest.mark.parametrize("tiles", ["2", "1"])
+def test_attention_sharp_rows_across_tiles(cuda_ok, monkeypatch, tiles):
     """Queries aligned with one key each, the keys spread over all key tiles
-    (the running maximum jumps late and early): the online rescaling."""
+    (the running maximum jumps late and early): the online rescaling.  Two
+    query tiles per CTA (the default for an even number of tiles) and one
+    (NVFP4_ATTN_TILES=1, the kernel of odd tile counts)."""
+    monkeypatch.setenv("NVFP4_ATTN_TILES", tiles)
     H, Lq, Lk = 1, 256, 1024
     rng = np.random.default_rng(73)
     kx = rng.standard_normal((Lk, D)).astype(np.float32)
