@@ -401,11 +401,11 @@ nvfp4_status nvfp4_mx_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const ui
  *           softmax the log(s_head) term is a constant shift of every logit.
  * out       bf16 [H*Lq, d], 16-byte aligned.
  * workspace device scratch of >= nvfp4_attention_workspace_bytes(H, Lk, d)
- *           bytes, 16-byte aligned: V decoded to bf16 and transposed (once
- *           per call, then read by every query tile); not preserved.
+ *           bytes, 16-byte aligned: V decoded to bf16, [H*Lk, d] (once per
+ *           call, then read by every query tile); not preserved.
  * d == 128, Lq and Lk multiples of 128 (no masking), H <= 65535.  Two kernels:
- * the V transpose, then a persistent kernel (one CTA per SM) over the work
- * items (128 queries, head).
+ * the V decode, then a persistent kernel (one CTA per SM) over the work items
+ * (256 queries of a head when Lq / 128 is even, else 128).
  */
 size_t nvfp4_attention_workspace_bytes(int64_t H, int64_t Lk, int64_t d);   /* H * d * Lk * 2 */
 nvfp4_status nvfp4_attention(const uint8_t *q_codes, const uint8_t *q_sf, const float *q_scale,

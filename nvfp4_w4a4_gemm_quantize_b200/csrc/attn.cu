@@ -6,21 +6,21 @@
 // Q, K, V are NVFP4 tensors quantized along the head dimension d = 128
 // (blocks of 16, tensor scales g_q, g_k, g_v): Q [H*Lq, d], K and V [H*Lk, d].
 // Two kernels:
-//   v_transpose   V decoded exactly to bf16 (e2m1 * e4m3: at most 6
-//                 significant bits) and transposed to V^T [H*d, Lk] in the
-//                 caller's workspace -- once per call, instead of once per
-//                 query tile;
-//   attention     persistent, one CTA per SM; a work item is 128 queries of
-//                 one head, keys in tiles of 128:
+//   v_decode      V decoded exactly to bf16 (e2m1 * e4m3: at most 6
+//                 significant bits), [H*Lk, d] in the caller's workspace --
+//                 once per call, instead of once per query tile;
+//   attention     persistent, one CTA per SM; a work item is 128 (or 256)
+//                 queries of one head, keys in tiles of 128:
 //     S = Q K^T   block-scaled FP4 MMA (kind::mxf4nvf4, K = d), FP32 in TMEM,
 //                 two S buffers so the next tile's product overlaps softmax;
 //     softmax     one query row per thread (online: reference maximum m, sum
 //                 l), exp2 of (S * g_q g_k log2(e) / sqrt(d) + log2(s_head) - m),
 //                 P rounded to bf16 into a 128-byte-swizzled K-major tile; the
 //                 running output is rescaled in TMEM when m moves;
-//     O += P V    bf16 MMA (kind::f16) on TMA-loaded V^T tiles, FP32 in TMEM;
+//     O += P V    bf16 MMA (kind::f16) on TMA-loaded V tiles (B operand
+//                 MN-major: d contiguous), FP32 in TMEM;
 //     output      O * g_v / l, rounded to bf16.
-// Roles: warp 0 loads Q and the K ring, warp 3 the V^T ring; warp 1 owns TMEM
+// Roles: warp 0 loads Q and the K ring, warp 3 the V ring; warp 1 owns TMEM
 // and issues S = Q K^T, warp 2 issues O += P V (two issuers, so that neither
 // product waits behind the other's operands); warps 4-7 softmax and output;
 // every wait is bounded.
@@ -43,17 +43,18 @@ constexpr int kBQ = 128;                     // queries per CTA
 constexpr int kBK = 128;                     // keys per tile
 constexpr int kThreads = 256;
 constexpr int kKStages = 4;                  // K code + scale stages
-constexpr int kVStages = 3;                  // V^T stages
+constexpr int kVStages = 3;                  // V stages
 constexpr int kCodeBytes = kBK * kD / 2;     // 8 KB: 128 rows x 64 bytes
 constexpr int kSfBytes = 1024;               // two 512-byte scale atoms (128 rows x 8 blocks)
 constexpr int kKStageBytes = kCodeBytes + kSfBytes;
-constexpr int kTileBf16 = kBQ * kBK * 2;     // 32 KB: two 64-key chunks of 128 rows x 128 bytes
+constexpr int kTileBf16 = kBQ * kBK * 2;     // 32 KB: two 64-column chunks of 128 rows x 128 bytes
 constexpr int kChunk = 128 * 128;            // 16 KB
 
 // shared memory (offsets from a 1024-aligned base): two Q buffers (codes with
 // the 64-byte swizzle, scales), so that the next work item's Q lands while
-// this one runs; the K ring (codes with the 64-byte swizzle, scales); the V^T
-// ring (bf16, 128-byte swizzle); two P tiles (bf16, 128-byte swizzle)
+// this one runs; the K ring (codes with the 64-byte swizzle, scales); the V
+// ring (bf16 rows of keys, d 0-63 then d 64-127, 128-byte swizzle); two P
+// tiles (bf16, 128-byte swizzle)
 constexpr int kOffQ = 0;                     // + qb * kKStageBytes
 constexpr int kOffK = 2 * kKStageBytes;
 constexpr int kOffV = kOffK + kKStages * kKStageBytes;
@@ -126,6 +127,22 @@ __device__ __forceinline__ uint32_t e4m3_to_b2_scaled_attn(uint32_t code) {
     return b | (b << 16);
 }
 
+// The V tile as the B operand of O += P V (K = keys, N = d), MN-major: rows
+// of 128 bytes hold 64 values of d for one key, 128-byte swizzle; 8-key
+// groups are 1024 bytes apart (stride offset) and the two 64-column chunks
+// 16 KB apart (leading offset).
+__device__ __forceinline__ uint64_t sdesc_v(uint32_t saddr) { return make_sdesc(saddr, kChunk, 1024, 2); }
+
+// Start-address steps (descriptor units of 16 bytes) of the kk-th 16-key MMA
+// of a tile: in V, 16 rows of 128 bytes; in the K-major P tile, 32 bytes
+// within a 64-key chunk, chunks 16 KB apart.  Tiles lie below 256 KB, so the
+// 14-bit address field does not carry.
+__device__ __forceinline__ uint64_t v_step(int kk) { return (uint64_t)(kk * 2048 >> 4); }
+__device__ __forceinline__ uint64_t p_step(int kk) { return (uint64_t)(((kk >> 2) * kChunk + (kk & 3) * 32) >> 4); }
+
+// kind::f16 instruction descriptor with B MN-major (bit 16).
+__host__ __device__ constexpr uint32_t idesc_bf16_bmn(int M, int N) { return idesc_bf16(M, N) | (1u << 16); }
+
 // Persistent: CTA c takes work items (head, 128-query tile) c, c + grid, ...
 // Key tiles carry one running number n over all of a CTA's items, which
 // selects ring slots, S / P buffers and barrier phases, so every pipeline
@@ -133,7 +150,7 @@ __device__ __forceinline__ uint32_t e4m3_to_b2_scaled_attn(uint32_t code) {
 // while this item's last products and output finish.
 __global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-            const __grid_constant__ CUtensorMap tmap_vt, const Params p) {
+            const __grid_constant__ CUtensorMap tmap_v, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t q_full[2], q_empty[2], k_full[kKStages], k_empty[kKStages];
     __shared__ __align__(8) uint64_t v_full[kVStages], v_empty[kVStages];
@@ -178,7 +195,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
         fence_barrier_init();
         tma_prefetch_desc(&tmap_q);
         tma_prefetch_desc(&tmap_k);
-        tma_prefetch_desc(&tmap_vt);
+        tma_prefetch_desc(&tmap_v);
     }
     if (warp == 1) {
         tmem_alloc(&tmem_base_sh, 512);
@@ -231,7 +248,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
                 mbar_wait(&k_full[m % kKStages], (uint32_t)(m / kKStages) & 1u, w2);
         }
     } else if (warp == 3) {
-        // ------------------------------------------------------------ V^T producer
+        // ------------------------------------------------------------ V producer
         const uint64_t pol = policy_evict_normal();
         bool ok = true;
         int n = 0;
@@ -243,10 +260,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
                 if (!__all_sync(0xffffffffu, mbar_wait(&v_empty[s], ph ^ 1u, wc) ? 1 : 0)) { ok = false; break; }
                 uint8_t* st = smem + kOffV + s * kTileBf16;
                 if (elect_one()) {
-                    // V^T rows h*d .. h*d + 127, keys j*128 .. j*128 + 127, as two 64-key chunks
+                    // keys h*Lk + j*128 .. + 127 of V, as two 64-column chunks
                     mbar_arrive_expect_tx(&v_full[s], kTileBf16);
-                    tma_load_2d(st, &tmap_vt, &v_full[s], j * kBK, h * kD, pol);
-                    tma_load_2d(st + kChunk, &tmap_vt, &v_full[s], j * kBK + 64, h * kD, pol);
+                    tma_load_2d(st, &tmap_v, &v_full[s], 0, h * p.Lk + j * kBK, pol);
+                    tma_load_2d(st + kChunk, &tmap_v, &v_full[s], 64, h * p.Lk + j * kBK, pol);
                 }
                 __syncwarp();
             }
@@ -308,7 +325,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
         mbar_wait(&drain_s, 0, w2);
     } else {
         // ------------------------------------------------------------ O += P V issuer
-        constexpr uint32_t idesc_o = idesc_bf16(kBQ, kD);
+        constexpr uint32_t idesc_o = idesc_bf16_bmn(kBQ, kD);
         const uint32_t sm0 = smem_u32(smem);
         bool ok = true;
         int n = 0, i = 0;
@@ -327,13 +344,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
                 const uint32_t pt = sm0 + kOffP + b * kTileBf16;
                 const uint32_t vt = sm0 + kOffV + s * kTileBf16;
                 if (elect_one()) {
+                    const uint64_t ad = sdesc_kmajor_sw128(pt), bd = sdesc_v(vt);
 #pragma unroll
-                    for (int kc = 0; kc < 2; ++kc)
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            tc_mma_bf16(tmem + kColO, sdesc_kmajor_sw128(pt + kc * kChunk + ks * 32),
-                                        sdesc_kmajor_sw128(vt + kc * kChunk + ks * 32), idesc_o,
-                                        (j | kc | ks) != 0 ? 1u : 0u);
+                    for (int kk = 0; kk < 8; ++kk)             // 16 keys per MMA
+                        tc_mma_bf16(tmem + kColO, ad + p_step(kk), bd + v_step(kk), idesc_o, (j | kk) != 0 ? 1u : 0u);
                     tc_commit(&p_empty[b]);
                     tc_commit(&v_empty[s]);
                     tc_commit(&o_done);
@@ -486,7 +500,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
 
 // ---------------------------------------------------------------------------
 // Two query tiles per CTA.  A work item is 256 queries of one head (query
-// tiles A and B); the K and V^T tiles are loaded once for both.  Two softmax
+// tiles A and B); the K and V tiles are loaded once for both.  Two softmax
 // warpgroups, one per tile, take turns on the tensor core: while one computes
 // its exponentials the other's S = Q K^T runs, so the special-function units
 // (the exponentials) rather than one warp's latency set the pace.
@@ -494,9 +508,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
 // its logits are in registers), O_A, O_B, and the scale slots.  Shared
 // memory: three bf16 P tiles taken in turn by the uses A0, B0, A1, B1, ... (a
 // group writes use u once the product of use u - 3 has read that tile, so it
-// never waits for its own previous product), a 3-stage K ring, a 2-stage V^T
+// never waits for its own previous product), a 3-stage K ring, a 2-stage V
 // ring and two Q buffers per tile.
-// Roles (384 threads): warp 0 Q and K producer, warp 3 V^T producer, warp 1 S
+// Roles (384 threads): warp 0 Q and K producer, warp 3 V producer, warp 1 S
 // issuer (and TMEM owner), warp 2 P V issuer; warps 4-7 softmax of tile A,
 // warps 8-11 of tile B.  The register budget moves to the softmax warpgroups
 // (setmaxnreg: 48 for warpgroup 0, 224 for 1 and 2; 128 x 48 + 256 x 224 <=
@@ -520,14 +534,21 @@ constexpr int kRegsLow2 = 48;
 constexpr int kRegsHigh2 = 224;
 static_assert(128 * kRegsLow2 + 256 * kRegsHigh2 <= kThreads2 * 168, "register split exceeds the launch budget");
 
+// Products of group g commit o_done[2 g + (n & 1)] (n: the running tile
+// number), so a wait for tile n's product has tile n - 2's as the barrier's
+// previous phase -- which the P tile wait has already covered.  The read-out
+// after an item's last tile then needs no wait on the second-to-last.
+__device__ __forceinline__ int o_bar(int g, int n) { return 2 * g + (n & 1); }
+__device__ __forceinline__ uint32_t o_par(int n) { return (uint32_t)(n >> 1) & 1u; }
+
 __global__ void __launch_bounds__(kThreads2, 1)
 attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-             const __grid_constant__ CUtensorMap tmap_vt, const Params p) {
+             const __grid_constant__ CUtensorMap tmap_v, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t q_full[2], q_empty[2], k_full[kKStages2], k_empty[kKStages2];
     __shared__ __align__(8) uint64_t v_full[kVStages2], v_empty[kVStages2];
     __shared__ __align__(8) uint64_t s_full[2], s_empty, p_full[kPBufs2], p_empty[kPBufs2];
-    __shared__ __align__(8) uint64_t o_done[2], o_free[2];
+    __shared__ __align__(8) uint64_t o_done[4], o_free[2];
     __shared__ __align__(8) uint64_t drain_s, drain_o;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
@@ -547,7 +568,8 @@ attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
             mbar_init(&q_full[b], 1);
             mbar_init(&q_empty[b], 1);               // the item's last S product's commit
             mbar_init(&s_full[b], 1);
-            mbar_init(&o_done[b], 1);
+            mbar_init(&o_done[2 * b], 1);            // group b's products of even / odd tiles
+            mbar_init(&o_done[2 * b + 1], 1);
             mbar_init(&o_free[b], 4);                // the group's softmax warps have read O out
         }
         for (int s = 0; s < kKStages2; ++s) {
@@ -568,7 +590,7 @@ attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
         fence_barrier_init();
         tma_prefetch_desc(&tmap_q);
         tma_prefetch_desc(&tmap_k);
-        tma_prefetch_desc(&tmap_vt);
+        tma_prefetch_desc(&tmap_v);
     }
     if (warp == 1) {
         tmem_alloc(&tmem_base_sh, 512);
@@ -626,7 +648,7 @@ attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                     mbar_wait(&k_full[m % kKStages2], (uint32_t)(m / kKStages2) & 1u, w2);
             }
         } else if (warp == 3) {
-            // -------------------------------------------------------- V^T producer
+            // -------------------------------------------------------- V producer
             const uint64_t pol = policy_evict_normal();
             bool ok = true;
             int n = 0;
@@ -639,8 +661,8 @@ attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                     uint8_t* st = smem + kOffV2 + s * kTileBf16;
                     if (elect_one()) {
                         mbar_arrive_expect_tx(&v_full[s], kTileBf16);
-                        tma_load_2d(st, &tmap_vt, &v_full[s], j * kBK, h * kD, pol);
-                        tma_load_2d(st + kChunk, &tmap_vt, &v_full[s], j * kBK + 64, h * kD, pol);
+                        tma_load_2d(st, &tmap_v, &v_full[s], 0, h * p.Lk + j * kBK, pol);
+                        tma_load_2d(st + kChunk, &tmap_v, &v_full[s], 64, h * p.Lk + j * kBK, pol);
                     }
                     __syncwarp();
                 }
@@ -721,7 +743,7 @@ attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
             mbar_wait(&drain_s, 0, w2);
         } else {
             // -------------------------------------------------------- O_g += P_g V issuer
-            constexpr uint32_t idesc_o = idesc_bf16(kBQ, kD);
+            constexpr uint32_t idesc_o = idesc_bf16_bmn(kBQ, kD);
             const uint32_t sm0 = smem_u32(smem);
             bool ok = true;
             int n = 0, i = 0;
@@ -746,15 +768,13 @@ attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                         tc_fence_after();
                         const uint32_t pt = sm0 + kOffP2 + pb * kTileBf16;
                         if (elect_one()) {
+                            const uint64_t ad = sdesc_kmajor_sw128(pt), bd = sdesc_v(vt);
 #pragma unroll
-                            for (int kc = 0; kc < 2; ++kc)
-#pragma unroll
-                                for (int ks = 0; ks < 4; ++ks)
-                                    tc_mma_bf16(tmem + kColO2 + g * kD, sdesc_kmajor_sw128(pt + kc * kChunk + ks * 32),
-                                                sdesc_kmajor_sw128(vt + kc * kChunk + ks * 32), idesc_o,
-                                                (j | kc | ks) != 0 ? 1u : 0u);
+                            for (int kk = 0; kk < 8; ++kk)     // 16 keys per MMA
+                                tc_mma_bf16(tmem + kColO2 + g * kD, ad + p_step(kk), bd + v_step(kk), idesc_o,
+                                            (j | kk) != 0 ? 1u : 0u);
                             tc_commit(&p_empty[pb]);
-                            tc_commit(&o_done[g]);
+                            tc_commit(&o_done[o_bar(g, n)]);
                             if (g == 1) tc_commit(&v_empty[s]);
                         }
                         __syncwarp();
@@ -833,17 +853,12 @@ attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                 }
                 l = fmaf(l, alpha, (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
                 m = mref;
-                // This group's previous product (o_done completion n - 1) is waited
-                // for before O_g is rescaled, and on an item's last tile, so that
-                // the read-out below waits with at most one product pending.
-                // The P wait above already covers completion n - 2.
-                const bool rescale = j >= 1 && __any_sync(0xffffffffu, alpha != 1.0f);
-                if ((rescale || (j >= 1 && j == ntiles - 1)) &&
-                    !__all_sync(0xffffffffu, mbar_wait(&o_done[g], (uint32_t)(n - 1) & 1u, wc) ? 1 : 0)) {
-                    ok = false;
-                    break;
-                }
-                if (rescale) {
+                // O_g rescaled by alpha once this group's previous product is done
+                if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&o_done[o_bar(g, n - 1)], o_par(n - 1), wc) ? 1 : 0)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
@@ -862,7 +877,7 @@ attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                 if (lane == 0) mbar_arrive(&p_full[pb]);
             }
             if (!ok) break;
-            if (!__all_sync(0xffffffffu, mbar_wait(&o_done[g], (uint32_t)(n - 1) & 1u, wc) ? 1 : 0)) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&o_done[o_bar(g, n - 1)], o_par(n - 1), wc) ? 1 : 0)) {
                 ok = false;
                 break;
             }
@@ -900,64 +915,35 @@ attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     }
 }
 
-// V [H*Lk, d] NVFP4 -> V^T [H*d, Lk] bf16, exact (the tensor scale g_v is
-// applied with the output).  A CTA per (64 keys, head); thread t decodes the
-// 16 code bytes of key t / 4, d = 32 (t % 4) .. + 31.  Two threads of
-// neighbouring keys (lanes t and t ^ 4) trade halves of their bf16 pairs so
-// that each holds 32-bit words of two keys at one d -- the even-key thread
-// the even d, the odd-key thread the odd d -- and stores them into a shared
-// tile [d][32 key pairs]; its 128 rows of 128 bytes then go out in 16-byte
-// stores.  Tile row pitch 36 words and the key-pair column XORed with
-// 8 (d / 32): both the word stores and the 16-byte loads are free of bank
-// conflicts.
-constexpr int kVtKeys = 64;
-constexpr int kVtPitch = 36;                     // 32-bit words per shared row (32 key pairs + 4)
+// V [H*Lk, d] NVFP4 -> V [H*Lk, d] bf16, exact (the tensor scale g_v is
+// applied with the output).  A thread decodes one 4-byte code word (8 values,
+// half a 16-value block) into one 16-byte store, so a warp reads 128 and
+// writes 512 contiguous bytes; 4 words per thread, a block-width apart.
+constexpr int kVdThreads = 256;
+constexpr int kVdWords = 4;                      // code words per thread
 
-__global__ void __launch_bounds__(256)
-v_transpose_kernel(const uint8_t* __restrict__ v_codes, const uint8_t* __restrict__ v_sf, int Lk,
-                   uint16_t* __restrict__ vt) {
-    __shared__ __align__(16) uint32_t tile[kD * kVtPitch];
-    const int t = threadIdx.x;
-    const int h = blockIdx.y, key0 = blockIdx.x * kVtKeys;
-    const int key = t >> 2, part = t & 3;                  // 16 bytes: d = 32 part .. 32 part + 31
-    const int odd = key & 1, kp = key >> 1;
-    const int64_t row = (int64_t)h * Lk + key0 + key;      // row of V
-    const uint4 cb = *reinterpret_cast<const uint4*>(v_codes + row * (kD / 2) + part * 16);
-    const uint32_t w[4] = {cb.x, cb.y, cb.z, cb.w};
-    // scales of blocks 2 part and 2 part + 1 (16 values of d each); layout of a
-    // [rows, 128] tensor: two 512-byte atoms per 128-row group
-    const int rr = (int)(row & 127);
-    const uint8_t* sfr = v_sf + (row >> 7) * 1024 + (rr & 31) * 16 + (rr >> 5) * 4;
-    const int col = kp ^ (8 * part);
+__global__ void __launch_bounds__(kVdThreads)
+v_decode_kernel(const uint8_t* __restrict__ v_codes, const uint8_t* __restrict__ v_sf, int64_t rows,
+                uint16_t* __restrict__ v) {
+    const int64_t words = rows * (kD / 8);                 // 16 code words per row
+    const int64_t w0 = (int64_t)blockIdx.x * (kVdThreads * kVdWords) + threadIdx.x;
 #pragma unroll
-    for (int hb = 0; hb < 2; ++hb) {
-        const int blk = 2 * part + hb;
-        const uint32_t sc = e4m3_to_b2_scaled_attn(sfr[(blk >> 2) * 512 + (blk & 3)]);
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const uint32_t word = w[2 * hb + q];
-#pragma unroll
-            for (int by = 0; by < 4; ++by) {
-                // own pair (d, d + 1) of this key; the neighbour key's pair at the same d
-                const uint32_t pr = dequant_pair_attn((word >> (8 * by)) & 0xFFu, sc);
-                const uint32_t nb = __shfl_xor_sync(0xffffffffu, pr, 4);
-                const int d = 32 * part + 16 * hb + 8 * q + 2 * by + odd;
-                // word at d: (even key, odd key) values, the even key in the low half
-                const uint32_t wd = odd ? (nb >> 16) | (pr & 0xFFFF0000u) : (pr & 0xFFFFu) | (nb << 16);
-                tile[d * kVtPitch + col] = wd;
-            }
-        }
-    }
-    __syncthreads();
-    // 128 rows x 64 keys out: thread -> half a row (16 key pairs, 64 bytes)
-    const int orow = t >> 1, half = t & 1;
-    uint16_t* dst = vt + ((int64_t)h * kD + orow) * Lk + key0 + half * 32;
-    const uint32_t* src = tile + orow * kVtPitch;
-    const int sw = 8 * (orow >> 5);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const uint4 v = *reinterpret_cast<const uint4*>(src + ((16 * half + 4 * j) ^ sw));
-        *reinterpret_cast<uint4*>(dst + 8 * j) = v;
+    for (int u = 0; u < kVdWords; ++u) {
+        const int64_t w = w0 + u * kVdThreads;
+        if (w >= words) break;
+        const uint32_t cw = *reinterpret_cast<const uint32_t*>(v_codes + w * 4);
+        // scale of block (w % 16) / 2 of row w / 16; layout of a [rows, 128]
+        // tensor: two 512-byte atoms per 128-row group
+        const int64_t row = w >> 4;
+        const int blk = (int)(w & 15) >> 1, rr = (int)(row & 127);
+        const uint32_t sc = e4m3_to_b2_scaled_attn(
+            v_sf[(row >> 7) * 1024 + (blk >> 2) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + (blk & 3)]);
+        uint4 o;
+        o.x = dequant_pair_attn(cw & 0xFFu, sc);
+        o.y = dequant_pair_attn((cw >> 8) & 0xFFu, sc);
+        o.z = dequant_pair_attn((cw >> 16) & 0xFFu, sc);
+        o.w = dequant_pair_attn(cw >> 24, sc);
+        *reinterpret_cast<uint4*>(v + w * 8) = o;
     }
 }
 
@@ -970,16 +956,18 @@ cudaError_t launch_attention(const uint8_t* q_codes, const uint8_t* q_sf, const 
                              const float* g_v, const float* s_head, int64_t H, int64_t Lq, int64_t Lk, void* out,
                              void* workspace, int* dev_status, cudaStream_t stream) {
     using namespace attn;
-    uint16_t* vt = static_cast<uint16_t*>(workspace);
-    CUtensorMap tq, tk, tvt;
+    uint16_t* vd = static_cast<uint16_t*>(workspace);
+    CUtensorMap tq, tk, tv;
     if (make_tmap_2d(&tq, q_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kD / 2, (uint64_t)(H * Lq), kD / 2, kD / 2, kBQ,
                      CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
         make_tmap_2d(&tk, k_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kD / 2, (uint64_t)(H * Lk), kD / 2, kD / 2, kBK,
                      CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
-        make_tmap_2d(&tvt, vt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)Lk, (uint64_t)(H * kD),
-                     (uint64_t)Lk * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+        make_tmap_2d(&tv, vd, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, (uint64_t)(H * Lk), kD * 2, 64, kBK,
+                     CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    v_transpose_kernel<<<dim3((unsigned)(Lk / kVtKeys), (unsigned)H), 256, 0, stream>>>(v_codes, v_sf, (int)Lk, vt);
+    const int64_t vwords = H * Lk * (kD / 8);
+    v_decode_kernel<<<(unsigned)((vwords + kVdThreads * kVdWords - 1) / (kVdThreads * kVdWords)), kVdThreads, 0,
+                      stream>>>(v_codes, v_sf, H * Lk, vd);
     count_launch(1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -1008,11 +996,11 @@ cudaError_t launch_attention(const uint8_t* q_codes, const uint8_t* q_sf, const 
     if (two) {
         e = cudaFuncSetAttribute(attn2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes2);
         if (e != cudaSuccess) return e;
-        attn2_kernel<<<grid, kThreads2, kSmemBytes2, stream>>>(tq, tk, tvt, p);
+        attn2_kernel<<<grid, kThreads2, kSmemBytes2, stream>>>(tq, tk, tv, p);
     } else {
         e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (e != cudaSuccess) return e;
-        attn_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tvt, p);
+        attn_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
     }
     count_launch(1);
     return cudaGetLastError();
