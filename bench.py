@@ -442,16 +442,7 @@ def reference_points(dev, layers, w4a16_layers):
         ms = time_device(lambda: torch.matmul(x, w.t()))
         out["cublas_bf16_tflops"][L.name] = round(2 * L.M * L.N * L.K / (ms * 1e-3) / 1e12, 1)
         del x, w
-    for L in w4a16_layers:
-        x, w = synth.layer_tensors("w4a16", L.name, device=dev)
-        x = x[: L.M].contiguous()
-        W = nv.quantize(w)
-        del w
-        y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev)
-        ms = time_device(lambda: nv.gemm_w4a16(x, W, out=y))
-        out["w4a16"][L.name] = {"shape": f"{L.M}x{L.K}x{L.N}", "ms": round(ms, 4),
-                                "tflops": round(2 * L.M * L.N * L.K / (ms * 1e-3) / 1e12, 1)}
-        del x, W, y
+    out["w4a16"] = w4a16_points(dev, w4a16_layers)
     out["qat"] = qat_points(dev, layers)
     out["mlp_fc1_gelu"] = mlp_fusion_points(dev, layers)
     out["layernorm_nvfp4"] = layernorm_points(dev)
@@ -460,6 +451,31 @@ def reference_points(dev, layers, w4a16_layers):
     out["mx_and_block_size"] = mx_points(dev, layers)
     out["attention"] = attention_points(dev)
     torch.cuda.empty_cache()
+    return out
+
+
+def w4a16_points(dev, w4a16_layers):
+    """The W4A16 GEMM (bf16 activations x NVFP4 weights, dequantized in the
+    mainloop) on the weights-only workload, with cuBLAS bf16 on the same
+    shapes beside it (the dequantized product is exact in bf16, so the bf16
+    tensor rate is its bar)."""
+    import torch
+    import nvfp4_w4a4_gemm_quantize_b200 as nv
+    from nvfp4_w4a4_gemm_quantize_b200 import synth
+    out = {}
+    for L in w4a16_layers:
+        x, w = synth.layer_tensors("w4a16", L.name, device=dev)
+        x = x[: L.M].contiguous()
+        ms_ref = time_device(lambda: torch.matmul(x, w.t()))
+        W = nv.quantize(w)
+        del w
+        y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev)
+        ms = time_device(lambda: nv.gemm_w4a16(x, W, out=y))
+        flop = 2 * L.M * L.N * L.K
+        out[L.name] = {"shape": f"{L.M}x{L.K}x{L.N}", "ms": round(ms, 4),
+                       "tflops": round(flop / (ms * 1e-3) / 1e12, 1),
+                       "cublas_bf16_tflops": round(flop / (ms_ref * 1e-3) / 1e12, 1)}
+        del x, W, y
     return out
 
 
@@ -840,7 +856,8 @@ def run_ours(args):
         groups = {"qat": lambda: qat_points(dev, wl.layers), "mlp": lambda: mlp_fusion_points(dev, wl.layers),
                   "layernorm": lambda: layernorm_points(dev), "small": lambda: small_layer_points(dev),
                   "grouped": lambda: grouped_points(dev), "mx": lambda: mx_points(dev, wl.layers),
-                  "attention": lambda: attention_points(dev, args.heads or 384)}
+                  "attention": lambda: attention_points(dev, args.heads or 384),
+                  "w4a16": lambda: w4a16_points(dev, wl16.layers)}
         name = "qat" if args.qat else args.only
         if name not in groups:
             raise SystemExit(f"--only: one of {sorted(groups)}")
@@ -1052,7 +1069,7 @@ def main():
     ap.add_argument("--qat", action="store_true", help="profiling: time only the QAT kernels (fc1 / fc2 inputs)")
     ap.add_argument("--heads", type=int, default=0, help="profiling: attention heads (default 384)")
     ap.add_argument("--only", default="", help="profiling: time one group of reference points "
-                                               "(qat, mlp, layernorm, small, grouped, mx, attention)")
+                                               "(qat, mlp, layernorm, small, grouped, mx, attention, w4a16)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

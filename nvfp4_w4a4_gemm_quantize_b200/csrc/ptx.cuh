@@ -437,6 +437,27 @@ __device__ __forceinline__ void tc_mma2_mxf4(uint32_t d_tmem, uint64_t adesc, ui
         : "memory");
 }
 
+// Pair bf16 MMA (kind::f16): M = 256 (128 rows of A in each CTA), N split in
+// halves across the two CTAs' shared memory, FP32 accumulate in each CTA's TMEM.
+__device__ __forceinline__ void tc_mma2_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on an mbarrier of another CTA of the cluster with the default
+// (CTA-scope) release: it orders this thread's earlier writes to its own
+// shared memory -- made visible to the async proxy by fence.proxy.async -- for
+// this SM's tensor core, which reads them when the other CTA issues a pair MMA.
+// (A cluster-scope release costs about a microsecond per arrive here.)
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 // Arrive on the barrier at this shared-memory offset in every CTA of `mask`
 // once all prior tcgen05 operations of the pair have completed.
 __device__ __forceinline__ void tc_commit2_mc(uint64_t* bar, uint16_t mask) {

@@ -2,8 +2,10 @@
 the mainloop) vs the CPU oracle.
 
 The oracle's weight operand is its own quantization of the seeded bf16
-weights; activations are the seeded bf16 tensors.  Tolerances as for W4A4:
-bf16 output within 2e-3 of |row(x)| |row(w^)|, FP32 output within 1e-5."""
+weights; activations are the seeded bf16 tensors.  Bound: the FP32
+accumulation within 1e-5 of |row(x)| |row(w^)|; a bf16 output may add its own
+rounding, at most 2^-8 of the exact |y| (round to nearest with an 8-bit
+significand) -- which a heavy-tailed row can bring close to |x| |w^| itself."""
 import numpy as np
 import pytest
 import torch
@@ -14,8 +16,8 @@ from nvfp4_w4a4_gemm_quantize_b200 import synth
 
 pytestmark = pytest.mark.gpu
 
-TOL_BF16 = 2e-3
 TOL_F32 = 1e-5
+BF16_ROUND = 2.0 ** -8
 
 
 def upload(codes, sf, g, rows, k) -> nv.NVFP4Tensor:
@@ -26,13 +28,27 @@ def upload(codes, sf, g, rows, k) -> nv.NVFP4Tensor:
     return q
 
 
-def norm_err(y, yref, xd, wd):
+def norm_err(y, yref, xd, wd, rounding=0.0):
+    """Largest |y - yref| beyond `rounding` |yref|, over |row(x)| |row(w)|."""
     den = np.linalg.norm(xd, axis=1)[:, None] * np.linalg.norm(wd, axis=1)[None, :]
-    err = np.abs(y.astype(np.float64) - yref)
+    err = np.maximum(np.abs(y.astype(np.float64) - yref) - rounding * np.abs(yref), 0.0)
     return float(np.max(np.where(den > 0, err / np.where(den > 0, den, 1.0), err)))
 
 
-def test_one_hot_pins_dequant_layout(cuda_ok):
+# "single": one CTA per 256 x 256 tile; "pair": CTA pairs on 512 x 256 tiles;
+# "auto": the library's choice (pairs once their tiles fill half the SMs).
+KERNELS = ["auto", "single", "pair"]
+
+
+@pytest.fixture
+def kernel(request, monkeypatch):
+    if request.param != "auto":
+        monkeypatch.setenv("NVFP4_W4A16_KERNEL", request.param)
+    return request.param
+
+
+@pytest.mark.parametrize("kernel", ["single", "pair"], indirect=True)
+def test_one_hot_pins_dequant_layout(cuda_ok, kernel):
     M, N, K = 128, 256, 128
     rng = np.random.default_rng(5)
     wc = np.zeros((N, K // 2), np.uint8)
@@ -52,9 +68,11 @@ def test_one_hot_pins_dequant_layout(cuda_ok):
     assert (ref != 0).sum() > 0
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (1, 256, 128), (200, 384, 320), (300, 512, 1152), (257, 256, 4608)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (1, 256, 128), (200, 384, 320), (300, 512, 1152), (257, 256, 4608),
+                                   (1100, 776, 640), (1536, 1024, 256)])
 @pytest.mark.parametrize("out", [torch.bfloat16, torch.float32])
-def test_random_shapes_vs_oracle(cuda_ok, M, N, K, out):
+@pytest.mark.parametrize("kernel", KERNELS, indirect=True)
+def test_random_shapes_vs_oracle(cuda_ok, M, N, K, out, kernel):
     x = synth.random_bf16((M, K), seed=M + 3 * K, dist="student_t3")
     w = synth.random_bf16((N, K), seed=N + 5 * K, scale=0.015)
     wc, wsf, gw = oracle.quantize(w)
@@ -62,12 +80,14 @@ def test_random_shapes_vs_oracle(cuda_ok, M, N, K, out):
     y = nv.gemm_w4a16(x.cuda(), W, out_dtype=out)
     torch.cuda.synchronize()
     yref = oracle.gemm_w4a16(x, wc, wsf, gw)
-    e = norm_err(y.float().cpu().numpy(), yref, x.float().numpy(), oracle.dequantize(wc, wsf, gw))
-    assert e <= (TOL_BF16 if out == torch.bfloat16 else TOL_F32), e
+    e = norm_err(y.float().cpu().numpy(), yref, x.float().numpy(), oracle.dequantize(wc, wsf, gw),
+                 BF16_ROUND if out == torch.bfloat16 else 0.0)
+    assert e <= TOL_F32, e
 
 
 @pytest.mark.parametrize("layer", ["fc1", "fc2"])
-def test_w4a16_workload_full_size_sampled(cuda_ok, layer):
+@pytest.mark.parametrize("kernel", ["auto", "single"], indirect=True)
+def test_w4a16_workload_full_size_sampled(cuda_ok, layer, kernel):
     """The weights-only workload at full size (M=16384): GPU quantize of the
     weights + fused-dequant GEMM; the oracle quantizes sampled weight rows with
     the tensor scale it computes over the whole weight and forms those entries."""
@@ -88,5 +108,5 @@ def test_w4a16_workload_full_size_sampled(cuda_ok, layer):
     xs = x.cpu()[torch.from_numpy(ms)]
     yref = oracle.gemm_w4a16(xs, wc, wsf, gw)
     yg = y.float().cpu().numpy()[np.ix_(ms, ns)]
-    e = norm_err(yg, yref, xs.float().numpy(), oracle.dequantize(wc, wsf, gw))
-    assert e <= TOL_BF16, e
+    e = norm_err(yg, yref, xs.float().numpy(), oracle.dequantize(wc, wsf, gw), BF16_ROUND)
+    assert e <= TOL_F32, e
