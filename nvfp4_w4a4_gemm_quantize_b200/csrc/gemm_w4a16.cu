@@ -78,11 +78,14 @@ struct Params {
     int* dev_status;
 };
 
+// Tile t of an M-block-grouped order: groups of GM M blocks, N blocks outer
+// within a group, so the tiles in flight share few X row blocks.
+template <int GM = kGroupM>
 __device__ __forceinline__ void tile_coords(int t, int num_mb, int num_nb, int& mb, int& nb) {
-    const int per_group = kGroupM * num_nb;
+    const int per_group = GM * num_nb;
     const int group = t / per_group;
-    const int first = group * kGroupM;
-    const int gm = min(kGroupM, num_mb - first);
+    const int first = group * GM;
+    const int gm = min(GM, num_mb - first);
     const int idx = t - group * per_group;
     mb = first + idx % gm;
     nb = idx / gm;
@@ -422,6 +425,7 @@ static_assert(A2_BYTES + B2_BYTES + C2_BYTES + SF_ATOM <= STAGE2_BYTES && STAGE2
 constexpr int STAGES2 = (kSmemLimit - 1024) / STAGE2_BYTES;      // 4
 constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + 1024;
 static_assert(STAGES2 >= 3, "pipeline depth");
+constexpr int kGroupM2 = 2;                       // 512-row X blocks per tile group
 
 template <int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -481,7 +485,7 @@ gemm_w4a16_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
         bool ok = true;
         for (int t = pair; t < p.num_tiles && ok; t += npairs) {
             int mb, nb;
-            tile_coords(t, p.num_mb, p.num_nb, mb, nb);
+            tile_coords<kGroupM2>(t, p.num_mb, p.num_nb, mb, nb);
             const int xrow = mb * PM + (int)rank * 256;
             const int wrow = nb * PN + (int)rank * 128;
             const int sfrow = (nb * 2 + (int)rank) * k_atoms;
@@ -603,7 +607,7 @@ gemm_w4a16_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
         uint32_t acc_phase = 0;
         for (int t = pair; t < p.num_tiles; t += npairs) {
             int mb, nb;
-            tile_coords(t, p.num_mb, p.num_nb, mb, nb);
+            tile_coords<kGroupM2>(t, p.num_mb, p.num_nb, mb, nb);
             if (!__all_sync(0xffffffffu, mbar_wait(&accf_bar, acc_phase, wc) ? 1 : 0)) break;
             tc_fence_after();
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + h * PN;
