@@ -402,12 +402,17 @@ nvfp4_status nvfp4_mx_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const ui
  * out       bf16 [H*Lq, d], 16-byte aligned.
  * workspace device scratch of >= nvfp4_attention_workspace_bytes(H, Lk, d)
  *           bytes, 16-byte aligned: V decoded to bf16, [H*Lk, d] (once per
- *           call, then read by every query tile); not preserved.
- * d == 128, Lq and Lk multiples of 128 (no masking), H <= 65535.  Two kernels:
- * the V decode, then a persistent kernel (one CTA per SM) over the work items
- * (256 queries of a head when Lq / 128 is even, else 128).
+ *           call, then read by every query tile), then 32 four-byte words
+ *           per head that tag the head's decoded parts with a per-call
+ *           number; not preserved.  Calls that run at the same time need
+ *           workspaces of their own.
+ * d == 128, Lq and Lk multiples of 128 (no masking), H <= 65535.  When Lq / 128
+ * is even, one persistent kernel (one CTA per SM, all resident) takes 256
+ * queries of a head per work item and decodes V itself, each item a share of
+ * its head's rows; otherwise (or when the grid cannot be co-resident) a V
+ * decode kernel runs first.
  */
-size_t nvfp4_attention_workspace_bytes(int64_t H, int64_t Lk, int64_t d);   /* H * d * Lk * 2 */
+size_t nvfp4_attention_workspace_bytes(int64_t H, int64_t Lk, int64_t d);   /* H * d * Lk * 2 + H * 128 */
 nvfp4_status nvfp4_attention(const uint8_t *q_codes, const uint8_t *q_sf, const float *q_scale,
                              const uint8_t *k_codes, const uint8_t *k_sf, const float *k_scale,
                              const uint8_t *v_codes, const uint8_t *v_sf, const float *v_scale,

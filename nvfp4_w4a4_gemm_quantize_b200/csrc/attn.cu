@@ -6,18 +6,19 @@
 // Q, K, V are NVFP4 tensors quantized along the head dimension d = 128
 // (blocks of 16, tensor scales g_q, g_k, g_v): Q [H*Lq, d], K and V [H*Lk, d].
 // Two kernels:
-//   v_decode      V decoded exactly to bf16 (e2m1 * e4m3: at most 6
-//                 significant bits), [H*Lk, d] in the caller's workspace --
-//                 once per call, instead of once per query tile;
+//   v_decode      V decoded exactly to f16 (e2m1 * e4m3: at most 6
+//                 significant bits, within f16's normal range), [H*Lk, d] in
+//                 the caller's workspace -- once per call, instead of once per
+//                 query tile (the two-tile kernel decodes V itself instead);
 //   attention     persistent, one CTA per SM; a work item is 128 (or 256)
 //                 queries of one head, keys in tiles of 128:
 //     S = Q K^T   block-scaled FP4 MMA (kind::mxf4nvf4, K = d), FP32 in TMEM,
 //                 two S buffers so the next tile's product overlaps softmax;
 //     softmax     one query row per thread (online: reference maximum m, sum
 //                 l), exp2 of (S * g_q g_k log2(e) / sqrt(d) + log2(s_head) - m),
-//                 P rounded to bf16 into a 128-byte-swizzled K-major tile; the
+//                 P rounded to f16 into a 128-byte-swizzled K-major tile; the
 //                 running output is rescaled in TMEM when m moves;
-//     O += P V    bf16 MMA (kind::f16) on TMA-loaded V tiles (B operand
+//     O += P V    f16 MMA (kind::f16) on TMA-loaded V tiles (B operand
 //                 MN-major: d contiguous), FP32 in TMEM;
 //     output      O * g_v / l, rounded to bf16.
 // Roles: warp 0 loads Q and the K ring, warp 3 the V ring; warp 1 owns TMEM
@@ -28,6 +29,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -53,8 +55,8 @@ constexpr int kChunk = 128 * 128;            // 16 KB
 // shared memory (offsets from a 1024-aligned base): two Q buffers (codes with
 // the 64-byte swizzle, scales), so that the next work item's Q lands while
 // this one runs; the K ring (codes with the 64-byte swizzle, scales); the V
-// ring (bf16 rows of keys, d 0-63 then d 64-127, 128-byte swizzle); two P
-// tiles (bf16, 128-byte swizzle)
+// ring (f16 rows of keys, d 0-63 then d 64-127, 128-byte swizzle); two P
+// tiles (f16, 128-byte swizzle)
 constexpr int kOffQ = 0;                     // + qb * kKStageBytes
 constexpr int kOffK = 2 * kKStageBytes;
 constexpr int kOffV = kOffK + kKStages * kKStageBytes;
@@ -80,6 +82,13 @@ struct Params {
     uint16_t* out;                           // bf16 [H*Lq, d]
     int Lq, Lk, H;
     int* dev_status;
+    // V decoded inside the two-tile kernel (null slots: decoded by a pre-pass)
+    const uint8_t* v_codes;
+    const uint8_t* v_sf;
+    uint16_t* vd;                            // f16 V [H*Lk, d] in the workspace
+    uint32_t* slots;                         // per head 32 words: the call number once a part is decoded
+    uint32_t gen;                            // this call's number
+    int rpp;                                 // V rows per part (one part per work item of a head)
 };
 
 // K-major operand rows of 64 bytes with the 64-byte swizzle (8-row groups
@@ -104,27 +113,26 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// Two E2M1 codes (one byte, low nibble first) times their shared scale,
-// exactly, as a bf16 pair: the f16 decode shifted down three bits is the bf16
-// pattern of the value times 2^-112 (sign kept), and one bf16 multiply by the
-// scale times 2^112 gives the product (at most 6 significant bits).
-__device__ __forceinline__ uint32_t dequant_pair_attn(uint32_t byte, uint32_t scale_b2) {
+// Two E2M1 codes (one byte, low nibble first) times their block scale, as an
+// f16 pair, exactly: the product has at most 6 significant bits and lies in
+// [2^-10, 2688], inside f16's normal range.
+__device__ __forceinline__ uint32_t dequant_pair_f16(uint32_t byte, uint32_t scale_h2) {
     uint32_t h2, out;
     asm("{\n\t.reg .b8 c;\n\t"
         "cvt.u8.u32 c, %1;\n\t"
         "cvt.rn.f16x2.e2m1x2 %0, c;\n\t}"
         : "=r"(h2)
         : "r"(byte));
-    const uint32_t b2 = ((h2 >> 3) & 0x0FFF0FFFu) | (h2 & 0x80008000u);
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(out) : "r"(b2), "r"(scale_b2));
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out) : "r"(h2), "r"(scale_h2));
     return out;
 }
 
-// E4M3 byte -> bf16 of (scale * 2^112) in both halves (exact).
-__device__ __forceinline__ uint32_t e4m3_to_b2_scaled_attn(uint32_t code) {
-    const float f = e4m3_to_f32(code) * 0x1p112f;
-    const uint32_t b = __float_as_uint(f) >> 16;
-    return b | (b << 16);
+// E4M3 byte -> its value in both halves of an f16 pair (exact).
+__device__ __forceinline__ uint32_t e4m3_to_h2(uint32_t code) {
+    uint32_t h2;
+    const uint16_t in = (uint16_t)((code & 0xFFu) * 0x101u);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+    return h2;
 }
 
 // The V tile as the B operand of O += P V (K = keys, N = d), MN-major: rows
@@ -140,8 +148,117 @@ __device__ __forceinline__ uint64_t sdesc_v(uint32_t saddr) { return make_sdesc(
 __device__ __forceinline__ uint64_t v_step(int kk) { return (uint64_t)(kk * 2048 >> 4); }
 __device__ __forceinline__ uint64_t p_step(int kk) { return (uint64_t)(((kk >> 2) * kChunk + (kk & 3) * 32) >> 4); }
 
-// kind::f16 instruction descriptor with B MN-major (bit 16).
-__host__ __device__ constexpr uint32_t idesc_bf16_bmn(int M, int N) { return idesc_bf16(M, N) | (1u << 16); }
+// kind::f16 instruction descriptor: A and B f16 (formats 0 in bits [7,10) and
+// [10,13)), FP32 accumulate (bit 4), B MN-major (bit 16), N >> 3 in [17,23),
+// M >> 4 in [24,29).
+__host__ __device__ constexpr uint32_t idesc_f16_bmn(int M, int N) {
+    return (1u << 4) | (1u << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Block b of V (row b / 8, values 16 (b % 8) .. + 15): its scale byte sits in
+// the scale layout of a [rows, 128] tensor, two 512-byte atoms per 128-row
+// group; its 8 code bytes decode to 32 bytes of f16 V [H*Lk, d].
+__device__ __forceinline__ const uint8_t* v_scale_ptr(const uint8_t* v_sf, int64_t b) {
+    const int64_t row = b >> 3;
+    const int blk = (int)(b & 7), rr = (int)(row & 127);
+    return v_sf + (row >> 7) * 1024 + (blk >> 2) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + (blk & 3);
+}
+
+__device__ __forceinline__ void decode_store_v(uint2 c, uint32_t sf, int64_t b, uint16_t* __restrict__ v) {
+    const uint32_t sc = e4m3_to_h2(sf);
+    uint4 o0, o1;
+    o0.x = dequant_pair_f16(c.x & 0xFFu, sc);
+    o0.y = dequant_pair_f16((c.x >> 8) & 0xFFu, sc);
+    o0.z = dequant_pair_f16((c.x >> 16) & 0xFFu, sc);
+    o0.w = dequant_pair_f16(c.x >> 24, sc);
+    o1.x = dequant_pair_f16(c.y & 0xFFu, sc);
+    o1.y = dequant_pair_f16((c.y >> 8) & 0xFFu, sc);
+    o1.z = dequant_pair_f16((c.y >> 16) & 0xFFu, sc);
+    o1.w = dequant_pair_f16(c.y >> 24, sc);
+    uint4* dst = reinterpret_cast<uint4*>(v + b * 16);
+    dst[0] = o0;
+    dst[1] = o1;
+}
+
+// Up to four blocks b = c0 + t + stride i (i < 4, b < c1): every load is
+// issued before any value is used (V's codes and scales are read-only here),
+// so one batch costs about one memory latency.
+constexpr int kVBatch = 4;
+
+__device__ __forceinline__ void v_batch_load(const uint8_t* __restrict__ v_codes, const uint8_t* __restrict__ v_sf,
+                                             int64_t c0, int64_t c1, int t, int stride, uint2 (&c)[kVBatch],
+                                             uint32_t (&sf)[kVBatch]) {
+#pragma unroll
+    for (int i = 0; i < kVBatch; ++i) {
+        const int64_t b = c0 + t + (int64_t)stride * i;
+        if (b < c1) {
+            c[i] = __ldg(reinterpret_cast<const uint2*>(v_codes) + b);
+            sf[i] = __ldg(v_scale_ptr(v_sf, b));
+        }
+    }
+}
+
+__device__ __forceinline__ void v_batch_store(int64_t c0, int64_t c1, int t, int stride, const uint2 (&c)[kVBatch],
+                                              const uint32_t (&sf)[kVBatch], uint16_t* __restrict__ v) {
+#pragma unroll
+    for (int i = 0; i < kVBatch; ++i) {
+        const int64_t b = c0 + t + (int64_t)stride * i;
+        if (b < c1) decode_store_v(c[i], sf[i], b, v);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// V decoded inside the two-tile kernel.  Work item (head h, query pair q)
+// decodes V rows [q rpp, (q + 1) rpp) of its head into the f16 workspace --
+// rpp = ceil(Lk / qpairs), so the items of a head share its rows -- and
+// marks part q done by storing the call number in the head's slot q.
+// An item may load its head's V once every part is marked.  A CTA decodes
+// the parts of its own items two rounds ahead: items c and c + grid with all
+// its threads at the start, then, while it runs item it, the part of item
+// it + 2 grid, a slice of at most 4 blocks per lane per key tile on the V
+// producer warp (which otherwise waits for ring slots; the next slice's
+// loads are in flight during that wait).  Every wait is on parts published a round earlier
+// or at the start, never on the waiter's own progress, and the grid is
+// cooperative (every CTA resident); waits are bounded all the same.
+// Writers order their stores before the slot update with a proxy fence (the
+// readers load V by TMA) and a GPU-scope fence; readers acquire the slot and
+// fence the async proxy before their loads.
+
+// 16-value blocks of part q of head h: [first, last).
+__device__ __forceinline__ void part_blocks(const Params& p, int h, int q, int64_t& first, int64_t& last) {
+    const int r0 = q * p.rpp, r1 = min(p.Lk, (q + 1) * p.rpp);
+    first = ((int64_t)h * p.Lk + r0) * (kD / 16);
+    last = ((int64_t)h * p.Lk + (r1 > r0 ? r1 : r0)) * (kD / 16);
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Marks a part decoded for call `gen` (a store with release semantics; the
+// caller's threads have fenced the part's stores and joined).
+__device__ __forceinline__ void publish_part(uint32_t* slot, uint32_t gen) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(slot), "r"(gen) : "memory");
+}
+
+// One warp: waits (bounded) until the head's `parts` slots all carry call
+// `gen`; lane q reads slot q.
+__device__ __forceinline__ bool wait_parts(const uint32_t* slots, int parts, uint32_t gen, int lane, const WaitCtx& w) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t n = 1;; ++n) {
+        uint32_t v = gen;
+        if (lane < parts) asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(slots + lane) : "memory");
+        if (__all_sync(0xffffffffu, v == gen)) return true;
+        if ((n & 63u) == 0u) {
+            const bool give_up = *w.abort_flag || globaltimer_ns() - t0 > kWaitLimitNs;
+            if (__any_sync(0xffffffffu, give_up)) {
+                if (lane == 0 && !*w.abort_flag) report_timeout(w);
+                return false;
+            }
+        }
+        __nanosleep(64);
+    }
+}
 
 // Persistent: CTA c takes work items (head, 128-query tile) c, c + grid, ...
 // Key tiles carry one running number n over all of a CTA's items, which
@@ -325,7 +442,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
         mbar_wait(&drain_s, 0, w2);
     } else {
         // ------------------------------------------------------------ O += P V issuer
-        constexpr uint32_t idesc_o = idesc_bf16_bmn(kBQ, kD);
+        constexpr uint32_t idesc_o = idesc_f16_bmn(kBQ, kD);
         const uint32_t sm0 = smem_u32(smem);
         bool ok = true;
         int n = 0, i = 0;
@@ -414,7 +531,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
                     ok = false;
                     break;
                 }
-                // p = exp2(s c + bias - mref), rounded to bf16 into the swizzled K-major P tile
+                // p = exp2(s c + bias - mref), rounded to f16 into the swizzled K-major P tile
                 uint8_t* prow = smem + kOffP + b * kTileBf16 + r * 128;
 #pragma unroll
                 for (int c8 = 0; c8 < 16; ++c8) {              // 8 keys per 16-byte unit
@@ -424,8 +541,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
                         const float e0 = ex2(fmaf(__uint_as_float(v[c8 * 8 + 2 * t]), c, off));
                         const float e1 = ex2(fmaf(__uint_as_float(v[c8 * 8 + 2 * t + 1]), c, off));
                         sum4[t] += e0 + e1;
-                        __nv_bfloat162 hb = __floats2bfloat162_rn(e0, e1);
-                        w[t] = *reinterpret_cast<uint32_t*>(&hb);
+                        __half2 hh = __floats2half2_rn(e0, e1);
+                        w[t] = *reinterpret_cast<uint32_t*>(&hh);
                     }
                     const int kc = c8 >> 3, pos = (c8 & 7) ^ (r & 7);
                     *reinterpret_cast<uint4*>(prow + kc * kChunk + pos * 16) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -506,15 +623,15 @@ attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ 
 // (the exponentials) rather than one warp's latency set the pace.
 // TMEM: one S buffer, used in turn by A and B (a group releases it as soon as
 // its logits are in registers), O_A, O_B, and the scale slots.  Shared
-// memory: three bf16 P tiles taken in turn by the uses A0, B0, A1, B1, ... (a
+// memory: three f16 P tiles taken in turn by the uses A0, B0, A1, B1, ... (a
 // group writes use u once the product of use u - 3 has read that tile, so it
 // never waits for its own previous product), a 3-stage K ring, a 2-stage V
 // ring and two Q buffers per tile.
 // Roles (384 threads): warp 0 Q and K producer, warp 3 V producer, warp 1 S
 // issuer (and TMEM owner), warp 2 P V issuer; warps 4-7 softmax of tile A,
 // warps 8-11 of tile B.  The register budget moves to the softmax warpgroups
-// (setmaxnreg: 48 for warpgroup 0, 224 for 1 and 2; 128 x 48 + 256 x 224 <=
-// 384 x 168).
+// (setmaxnreg: 64 for warpgroup 0, whose V producer also decodes V, 208 for
+// 1 and 2; 128 x 64 + 256 x 208 <= 384 x 168).
 constexpr int kThreads2 = 384;
 constexpr int kKStages2 = 3;
 constexpr int kVStages2 = 2;
@@ -530,8 +647,8 @@ constexpr uint32_t kColS2 = 0;                               // S: [0, 128)
 constexpr uint32_t kColO2 = 128;                             // O_g: [128 + 128 g, 256 + 128 g)
 constexpr uint32_t kColSfQ2 = 384;                           // Q scales: (qb * 2 + g) * 8
 constexpr uint32_t kColSfK2 = 416;                           // K scales: (n & 1) * 8
-constexpr int kRegsLow2 = 48;
-constexpr int kRegsHigh2 = 224;
+constexpr int kRegsLow2 = 64;
+constexpr int kRegsHigh2 = 208;
 static_assert(128 * kRegsLow2 + 256 * kRegsHigh2 <= kThreads2 * 168, "register split exceeds the launch budget");
 
 // Products of group g commit o_done[2 g + (n & 1)] (n: the running tile
@@ -601,6 +718,30 @@ attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
 
+    if (p.slots != nullptr) {
+        // V decoded here: the parts of this CTA's first two items, by every thread
+        for (int k = 0; k < 2; ++k) {
+            const int it = blockIdx.x + k * gridDim.x;
+            if (it >= nitems) break;
+            int64_t b0, b1;
+            part_blocks(p, item_head(it), it % qpairs, b0, b1);
+            for (int64_t b = b0; b < b1; b += kVBatch * kThreads2) {
+                uint2 c[kVBatch];
+                uint32_t sf[kVBatch];
+                v_batch_load(p.v_codes, p.v_sf, b, b1, threadIdx.x, kThreads2, c, sf);
+                v_batch_store(b, b1, threadIdx.x, kThreads2, c, sf, p.vd);
+            }
+        }
+        fence_proxy_async_global();
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0)
+            for (int k = 0; k < 2; ++k) {
+                const int it = blockIdx.x + k * gridDim.x;
+                if (it < nitems) publish_part(p.slots + item_head(it) * 32 + it % qpairs, p.gen);
+            }
+    }
+
     if (warp < 4) {
         regs_dec<kRegsLow2>();
         if (warp == 0) {
@@ -648,12 +789,28 @@ attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                     mbar_wait(&k_full[m % kKStages2], (uint32_t)(m / kKStages2) & 1u, w2);
             }
         } else if (warp == 3) {
-            // -------------------------------------------------------- V producer
+            // -------------------------------------------------------- V producer (and decoder)
             const uint64_t pol = policy_evict_normal();
             bool ok = true;
             int n = 0;
             for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
                 const int h = item_head(it);
+                // the part of item it + 2 grid, a slice after each key tile's loads
+                const int ahead = it + 2 * (int)gridDim.x;
+                const bool decode_ahead = p.slots != nullptr && ahead < nitems;
+                int64_t a0 = 0, a1 = 0, per = 0;
+                uint2 cw[kVBatch];                            // the next slice, in flight
+                uint32_t sf[kVBatch];
+                if (p.slots != nullptr) {
+                    // every part of this item's head decoded
+                    if (!wait_parts(p.slots + h * 32, qpairs, p.gen, lane, wc)) { ok = false; break; }
+                    fence_proxy_async_global();
+                    if (decode_ahead) {
+                        part_blocks(p, item_head(ahead), ahead % qpairs, a0, a1);
+                        per = (a1 - a0 + ntiles - 1) / ntiles;      // <= 32 lanes x 4 (host check)
+                        v_batch_load(p.v_codes, p.v_sf, a0, a0 + per < a1 ? a0 + per : a1, lane, 32, cw, sf);
+                    }
+                }
                 for (int j = 0; j < ntiles; ++j, ++n) {
                     const int s = n % kVStages2;
                     const uint32_t ph = (uint32_t)(n / kVStages2) & 1u;
@@ -665,6 +822,20 @@ attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                         tma_load_2d(st + kChunk, &tmap_v, &v_full[s], 64, h * p.Lk + j * kBK, pol);
                     }
                     __syncwarp();
+                    if (decode_ahead) {
+                        const int64_t c0 = a0 + j * per, c1 = c0 + per < a1 ? c0 + per : a1;
+                        v_batch_store(c0, c1, lane, 32, cw, sf, p.vd);
+                        if (j + 1 < ntiles) {
+                            const int64_t n0 = c0 + per;
+                            v_batch_load(p.v_codes, p.v_sf, n0, n0 + per < a1 ? n0 + per : a1, lane, 32, cw, sf);
+                        }
+                        if (j == ntiles - 1) {                  // published even when the part is empty
+                            fence_proxy_async_global();
+                            __threadfence();
+                            __syncwarp();
+                            if (lane == 0) publish_part(p.slots + item_head(ahead) * 32 + ahead % qpairs, p.gen);
+                        }
+                    }
                 }
             }
             if (lane == 0) {
@@ -743,7 +914,7 @@ attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
             mbar_wait(&drain_s, 0, w2);
         } else {
             // -------------------------------------------------------- O_g += P_g V issuer
-            constexpr uint32_t idesc_o = idesc_bf16_bmn(kBQ, kD);
+            constexpr uint32_t idesc_o = idesc_f16_bmn(kBQ, kD);
             const uint32_t sm0 = smem_u32(smem);
             bool ok = true;
             int n = 0, i = 0;
@@ -845,8 +1016,8 @@ attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                         const float e0 = ex2(fmaf(__uint_as_float(v[c8 * 8 + 2 * t]), c, off));
                         const float e1 = ex2(fmaf(__uint_as_float(v[c8 * 8 + 2 * t + 1]), c, off));
                         sum4[t] += e0 + e1;
-                        __nv_bfloat162 hb = __floats2bfloat162_rn(e0, e1);
-                        w[t] = *reinterpret_cast<uint32_t*>(&hb);
+                        __half2 hh = __floats2half2_rn(e0, e1);
+                        w[t] = *reinterpret_cast<uint32_t*>(&hh);
                     }
                     const int kc = c8 >> 3, pos = (c8 & 7) ^ (r & 7);
                     *reinterpret_cast<uint4*>(pbase + kc * kChunk + pos * 16) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -915,41 +1086,30 @@ attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     }
 }
 
-// V [H*Lk, d] NVFP4 -> V [H*Lk, d] bf16, exact (the tensor scale g_v is
-// applied with the output).  A thread decodes one 4-byte code word (8 values,
-// half a 16-value block) into one 16-byte store, so a warp reads 128 and
-// writes 512 contiguous bytes; 4 words per thread, a block-width apart.
+// V [H*Lk, d] NVFP4 -> V [H*Lk, d] f16, exact (the tensor scale g_v is
+// applied with the output): kernel used when the attention kernel does not
+// decode V itself.  A thread decodes two 16-value blocks, a block-width
+// apart (8 code bytes in, 32 bytes out each).
 constexpr int kVdThreads = 256;
-constexpr int kVdWords = 4;                      // code words per thread
+constexpr int kVdBlocks = 2;                     // blocks per thread
 
 __global__ void __launch_bounds__(kVdThreads)
 v_decode_kernel(const uint8_t* __restrict__ v_codes, const uint8_t* __restrict__ v_sf, int64_t rows,
                 uint16_t* __restrict__ v) {
-    const int64_t words = rows * (kD / 8);                 // 16 code words per row
-    const int64_t w0 = (int64_t)blockIdx.x * (kVdThreads * kVdWords) + threadIdx.x;
+    const int64_t blocks = rows * (kD / 16);
+    const int64_t b0 = (int64_t)blockIdx.x * (kVdThreads * kVdBlocks) + threadIdx.x;
 #pragma unroll
-    for (int u = 0; u < kVdWords; ++u) {
-        const int64_t w = w0 + u * kVdThreads;
-        if (w >= words) break;
-        const uint32_t cw = *reinterpret_cast<const uint32_t*>(v_codes + w * 4);
-        // scale of block (w % 16) / 2 of row w / 16; layout of a [rows, 128]
-        // tensor: two 512-byte atoms per 128-row group
-        const int64_t row = w >> 4;
-        const int blk = (int)(w & 15) >> 1, rr = (int)(row & 127);
-        const uint32_t sc = e4m3_to_b2_scaled_attn(
-            v_sf[(row >> 7) * 1024 + (blk >> 2) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + (blk & 3)]);
-        uint4 o;
-        o.x = dequant_pair_attn(cw & 0xFFu, sc);
-        o.y = dequant_pair_attn((cw >> 8) & 0xFFu, sc);
-        o.z = dequant_pair_attn((cw >> 16) & 0xFFu, sc);
-        o.w = dequant_pair_attn(cw >> 24, sc);
-        *reinterpret_cast<uint4*>(v + w * 8) = o;
+    for (int u = 0; u < kVdBlocks; ++u) {
+        const int64_t b = b0 + u * kVdThreads;
+        if (b >= blocks) break;
+        decode_store_v(__ldg(reinterpret_cast<const uint2*>(v_codes) + b), __ldg(v_scale_ptr(v_sf, b)), b, v);
     }
 }
 
 }  // namespace attn
 
-size_t attention_workspace_bytes(int64_t H, int64_t Lk, int64_t d) { return (size_t)(H * d * Lk) * 2; }
+// f16 V [H*Lk, d], then 32 four-byte decode slots per head
+size_t attention_workspace_bytes(int64_t H, int64_t Lk, int64_t d) { return (size_t)(H * d * Lk) * 2 + (size_t)H * 128; }
 
 cudaError_t launch_attention(const uint8_t* q_codes, const uint8_t* q_sf, const float* g_q, const uint8_t* k_codes,
                              const uint8_t* k_sf, const float* g_k, const uint8_t* v_codes, const uint8_t* v_sf,
@@ -962,15 +1122,9 @@ cudaError_t launch_attention(const uint8_t* q_codes, const uint8_t* q_sf, const 
                      CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
         make_tmap_2d(&tk, k_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kD / 2, (uint64_t)(H * Lk), kD / 2, kD / 2, kBK,
                      CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
-        make_tmap_2d(&tv, vd, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, (uint64_t)(H * Lk), kD * 2, 64, kBK,
+        make_tmap_2d(&tv, vd, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kD, (uint64_t)(H * Lk), kD * 2, 64, kBK,
                      CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    const int64_t vwords = H * Lk * (kD / 8);
-    v_decode_kernel<<<(unsigned)((vwords + kVdThreads * kVdWords - 1) / (kVdThreads * kVdWords)), kVdThreads, 0,
-                      stream>>>(v_codes, v_sf, H * Lk, vd);
-    count_launch(1);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
     Params p;
     p.q_sf = q_sf;
     p.k_sf = k_sf;
@@ -983,7 +1137,14 @@ cudaError_t launch_attention(const uint8_t* q_codes, const uint8_t* q_sf, const 
     p.Lk = (int)Lk;
     p.H = (int)H;
     p.dev_status = dev_status;
+    p.v_codes = v_codes;
+    p.v_sf = v_sf;
+    p.vd = vd;
+    p.slots = nullptr;
+    p.gen = 0;
+    p.rpp = 0;
     int dev = 0, sms = 0;
+    cudaError_t e;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
         (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
@@ -996,6 +1157,45 @@ cudaError_t launch_attention(const uint8_t* q_codes, const uint8_t* q_sf, const 
     if (two) {
         e = cudaFuncSetAttribute(attn2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes2);
         if (e != cudaSuccess) return e;
+        // V decoded inside the kernel (a head's items share its rows; at most 32
+        // parts per head, and no more than CTAs, so that a head's items fall in
+        // at most two consecutive rounds and every part an item waits for is
+        // published before its round starts; at most one 8-word batch per lane
+        // and key tile), on a cooperative grid; NVFP4_ATTN_DECODE=prepass keeps
+        // the separate pass, for measurements
+        const char* denv = getenv("NVFP4_ATTN_DECODE");
+        const int64_t qpairs = Lq / (2 * kBQ);
+        const int64_t rpp = (Lk + qpairs - 1) / qpairs, per = (rpp * (kD / 16) + Lk / kBK - 1) / (Lk / kBK);
+        if (qpairs <= 32 && qpairs <= (int64_t)grid && per <= 32 * kVBatch && !(denv && denv[0] == 'p')) {
+            p.slots = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + (size_t)(H * kD * Lk) * 2);
+            p.gen = next_generation();
+            p.rpp = (int)rpp;
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeCooperative;      // every CTA resident: the parts' waits
+            attr[0].val.cooperative = 1;
+            cfg.gridDim = dim3(grid);
+            cfg.blockDim = dim3(kThreads2);
+            cfg.dynamicSmemBytes = kSmemBytes2;
+            cfg.stream = stream;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            e = cudaLaunchKernelEx(&cfg, attn2_kernel, tq, tk, tv, p);
+            if (e == cudaSuccess) {
+                count_launch(1);
+                return cudaGetLastError();
+            }
+            if (e != cudaErrorCooperativeLaunchTooLarge) return e;
+            (void)cudaGetLastError();                           // not co-resident: the separate pass
+            p.slots = nullptr;
+        }
+    }
+    const int64_t vblocks = H * Lk * (kD / 16);
+    v_decode_kernel<<<(unsigned)((vblocks + kVdThreads * kVdBlocks - 1) / (kVdThreads * kVdBlocks)), kVdThreads, 0,
+                      stream>>>(v_codes, v_sf, H * Lk, vd);
+    count_launch(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (two) {
         attn2_kernel<<<grid, kThreads2, kSmemBytes2, stream>>>(tq, tk, tv, p);
     } else {
         e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);

@@ -1,8 +1,9 @@
 """Attention over NVFP4 Q, K, V (Eq. 10) on the GPU vs the CPU oracle.
 
 The oracle computes softmax(q^ k^T / sqrt(d) + log s_head) v^ in double from
-the exact element values.  The kernel's deviations: P rounded to bf16 (2^-9
-relative per element), the softmax sum taken over the unrounded values, FP32
+the exact element values.  The kernel's deviations: P rounded to f16 (up to 2^-11
+relative per element for P >= 2^-14 of the running reference, an absolute 2^-25 below
+it), the softmax sum taken over the unrounded values, FP32
 accumulation, exp2 from the hardware approximation, and the bf16 output; so
 per element |O - O_ref| <= 3e-3 max|v^| + 5e-3 |O_ref| (head-wise max)."""
 import numpy as np
@@ -112,10 +113,24 @@ def _sampled_heads(xq, xk, xv, H, Lq, Lk, heads, rows, s_head=None):
             assert np.all(err <= 3e-3 * vmax + 5e-3 * np.abs(ref)), (h, r, float(err.max()))
 
 
-def test_attention_several_items_per_cta(cuda_ok):
-    """More work items (head, 128-query tile) than SMs: each persistent CTA
-    takes several, over different heads with different s_head; ring slots and
-    barrier phases run on across the item boundaries."""
+# "fused": the two-tile kernel decodes V itself, each work item a share of its
+# head's rows, two rounds ahead; "prepass": a separate V decode kernel first.
+DECODE = ["fused", "prepass"]
+
+
+@pytest.fixture
+def decode(request, monkeypatch):
+    if request.param == "prepass":
+        monkeypatch.setenv("NVFP4_ATTN_DECODE", "prepass")
+    return request.param
+
+
+@pytest.mark.parametrize("decode", DECODE, indirect=True)
+def test_attention_several_items_per_cta(cuda_ok, decode):
+    """More work items (head, 256-query pair of tiles) than SMs: each
+    persistent CTA takes several, over different heads with different s_head;
+    ring slots and barrier phases run on across the item boundaries, and a
+    head's items fall in two rounds."""
     H, Lq, Lk = 24, 2048, 512
     xq = synth.random_bf16((H * Lq, D), seed=78, dist="token_scaled")
     xk = synth.random_bf16((H * Lk, D), seed=79, dist="normal")
@@ -124,9 +139,26 @@ def test_attention_several_items_per_cta(cuda_ok):
     _sampled_heads(xq, xk, xv, H, Lq, Lk, heads=(0, 9, 10, 18, 23), rows=(0, 129, 1151, 2047), s_head=s_head)
 
 
-def test_attention_full_size_sampled(cuda_ok):
+@pytest.mark.parametrize("decode", DECODE, indirect=True)
+def test_attention_full_size_sampled(cuda_ok, decode):
     """The video DiT's spatial attention as timed: 384 heads x 2048 tokens,
-    d = 128 (6144 work items on the persistent grid), sampled heads and rows."""
+    d = 128 (3072 work items on the persistent grid), sampled heads and rows."""
     H, L = 384, 2048
     xs = [synth.random_bf16((H * L, D), seed=90 + i, dist="normal") for i in range(3)]
     _sampled_heads(*xs, H, L, L, heads=(0, 147, 148, 295, 383), rows=(0, 777, 2047))
+
+
+def test_attention_decode_parts_with_empty_shares(cuda_ok):
+    """24 work items per head over 128 keys: shares of ceil(128 / 24) = 6 rows,
+    the last two empty; 480 items, so shares are also decoded two rounds ahead
+    in the kernel's main loop -- empty ones must still be marked done."""
+    H, Lq, Lk = 20, 6144, 128
+    xq = synth.random_bf16((H * Lq, D), seed=81, dist="normal")
+    xk = synth.random_bf16((H * Lk, D), seed=82, dist="normal")
+    xv = synth.random_bf16((H * Lk, D), seed=83, dist="outlier")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Q, K, V = nv.quantize(xq.cuda()), nv.quantize(xk.cuda()), nv.quantize(xv.cuda())
+    nv.attention(Q, K, V, H, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    _sampled_heads(xq, xk, xv, H, Lq, Lk, heads=(0, 7, 19), rows=(0, 3001, 6143))
