@@ -86,7 +86,9 @@ size_t nvfp4_sf_bytes(int64_t rows, int64_t k);
  * scale from the data (no NVFP4_SCALE_GIVEN): per-CTA partial maxima, each
  * tagged with a per-call number so that the contents need no initialisation
  * (they are not preserved).  Calls that overlap on the GPU must not share a
- * workspace. */
+ * workspace.  The numbers come from a counter of this copy of the library in
+ * this process: a workspace must not be shared with another process or another
+ * loaded copy of the library, whose numbers can coincide. */
 size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t k);
 
 /*
@@ -404,7 +406,8 @@ nvfp4_status nvfp4_mx_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const ui
  *           bytes, 16-byte aligned: V decoded to bf16, [H*Lk, d] (once per
  *           call, then read by every query tile), then 32 four-byte words
  *           per head that tag the head's decoded parts with a per-call
- *           number; not preserved.  Calls that run at the same time need
+ *           number (the counter of nvfp4_quantize's workspace: the same rule
+ *           on sharing); not preserved.  Calls that run at the same time need
  *           workspaces of their own.
  * d == 128, Lq and Lk multiples of 128 (no masking), H <= 65535.  When Lq / 128
  * is even, one persistent kernel (one CTA per SM, all resident) takes 256
