@@ -40,7 +40,11 @@
 //   warps 8-15 epilogue, both CTAs: the 128 x BN FP32 accumulator slice is
 //              read into registers (two warps per TMEM lane quarter, BN/2
 //              columns each) and released to the MMA issuer at once, then
-//              converted and stored while the mainloop runs.
+//              converted and stored while the mainloop runs.  With the
+//              NVFP4 output (activation and block quantization per element:
+//              about 13 instructions per value, more than two warps per
+//              sub-partition issue within a tile's mainloop) warps 4-15: three
+//              per lane quarter, 96 (BN 256) or 64 (BN 192) columns each.
 // Producer, copier and MMA issuer run on whole warps with one elected lane
 // issuing: the descriptors, coordinates and addresses then stay warp-uniform.
 // Issued from a single lane, the same copies and MMAs took longer to issue
@@ -51,7 +55,8 @@
 // release costs about a microsecond per arrive).
 // Registers: launched at 128 per thread; warpgroups 0-1 drop to 56 and the
 // epilogue warpgroups rise to 200 (256 x 56 + 256 x 200 = 512 x 128); 80 and
-// 176 with 192-wide tiles.
+// 176 with 192-wide tiles; with the NVFP4 output warpgroup 0 drops to 56 (80)
+// and warpgroups 1-3 rise to 152 (144).
 // No load uses cluster multicast: every CTA fetches its own tiles.
 #include <cstdlib>
 #include <cuda.h>
@@ -113,7 +118,13 @@ struct Cfg {
     using L = Lay<BN, MXS>;
     static constexpr int STAGE_BYTES = L::STAGE_BYTES;
     static constexpr int EPI_BUF = OUT == OUT_F32 ? 4096 : (OUT == OUT_BF16 ? 2048 : 0);   // 32 rows x 32 cols
-    static constexpr int EPI_BYTES = kEpiWarps * 2 * EPI_BUF;
+    // epilogue warps: 8 (two per TMEM lane quarter) for bf16 / FP32 output;
+    // the NVFP4 output (activation and quantization per element, no staging
+    // buffers) takes warpgroup 1 as well: 12, three per lane quarter
+    static constexpr int EPI_WARPS = OUT == OUT_NVFP4 ? 12 : kEpiWarps;
+    static constexpr int EPI_WARP0 = kThreads / 32 - EPI_WARPS;
+    static constexpr int EPI_PARTS = EPI_WARPS / 4;               // column parts per lane quarter
+    static constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BUF;
     static constexpr int FIT = (kSmemLimit - 1024 - EPI_BYTES) / STAGE_BYTES;
     static constexpr int MAX_STAGES = BN == 192 ? 6 : 5;
     static constexpr int STAGES = FIT < MAX_STAGES ? FIT : MAX_STAGES;
@@ -128,7 +139,14 @@ struct Cfg {
     // issue order, so a copy into a slot cannot overtake the MMAs that read it
     // two stages earlier, and no barrier round trip sits between stages)
     static constexpr bool COPY_IN_MMA = SF_SLOTS < STAGES;
-    static constexpr int EPI_COLS = BN / 2;                       // accumulator columns per epilogue warp
+    static constexpr int EPI_COLS = (BN / EPI_PARTS + 31) / 32 * 32;   // accumulator columns per epilogue warp
+    // register split (setmaxnreg): warpgroup 0 (producer, MMA, copier) drops to
+    // REGS_LOW, the epilogue warpgroups rise to REGS_HIGH
+    static constexpr int REGS_LOW = Regs<BN>::LOW;
+    static constexpr int REGS_HIGH =
+        EPI_WARPS == kEpiWarps ? Regs<BN>::HIGH : (kThreads * 128 - 128 * REGS_LOW) / (32 * EPI_WARPS) / 8 * 8;
+    static_assert((kThreads - 32 * EPI_WARPS) * REGS_LOW + 32 * EPI_WARPS * REGS_HIGH <= kThreads * 128,
+                  "register split exceeds the launch budget");
     static_assert(STAGES >= 3, "pipeline depth");
     static_assert(ACC_BUFS * BN + SF_SLOTS * L::SF_COLS_STAGE <= 512, "TMEM columns");
     static_assert(EPI_COLS % 32 == 0, "epilogue chunks of 32 columns");
@@ -290,7 +308,7 @@ gemm2_kernel(const __grid_constant__ PairGroup<G> g) {
         }
         for (int b = 0; b < ACC_BUFS; ++b) {
             mbar_init(&accf_bar[b], 1);
-            mbar_init(&acce_bar[b], 2 * kEpiWarps);
+            mbar_init(&acce_bar[b], 2 * C::EPI_WARPS);
         }
         mbar_init(&drain_bar, 1);
         fence_barrier_init();
@@ -318,8 +336,8 @@ gemm2_kernel(const __grid_constant__ PairGroup<G> g) {
     // one register-budget change per warpgroup, before the roles diverge
     // (the epilogue code sits under the same branch as its increase, so that
     // ptxas allocates it against the raised budget)
-    if (warp < 8) {
-        regs_dec<Regs<BN>::LOW>();
+    if (warp < C::EPI_WARP0) {
+        if (warp < 4 || C::EPI_WARP0 == 8) regs_dec<C::REGS_LOW>();   // whole warpgroups: 0 (and 1)
         if (warp == 0) {
             // ------------------------------------------------------------ producer (both CTAs)
             const uint64_t pol_a = policy_evict_normal();
@@ -497,10 +515,10 @@ gemm2_kernel(const __grid_constant__ PairGroup<G> g) {
             }
         }
     } else {
-        regs_inc<Regs<BN>::HIGH>();
+        regs_inc<C::REGS_HIGH>();
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int q = warp & 3;                       // TMEM lane quarter
-        const int h = (warp - 8) >> 2;                // column half: [0, BN/2) or [BN/2, BN)
+        const int h = (warp - C::EPI_WARP0) >> 2;     // column part: [h EPI_COLS, (h + 1) EPI_COLS) of BN
         const int row_t = (int)rank * 128 + q * 32 + lane;    // row inside the pair tile
         // per-problem constants, refreshed when the tile sequence enters
         // another problem (MX operands have no tensor scale: a null scale
@@ -508,7 +526,7 @@ gemm2_kernel(const __grid_constant__ PairGroup<G> g) {
         int cur = -1;
         float alpha = 0.0f, g_y = 0.0f;
         ScaleConsts sc_y = scale_consts(0.0f);
-        uint8_t* ebuf = smem + STAGES * STAGE_BYTES + (warp - 8) * 2 * C::EPI_BUF;
+        uint8_t* ebuf = smem + STAGES * STAGE_BYTES + (warp - C::EPI_WARP0) * 2 * C::EPI_BUF;
         // the output is written once and not read again by this kernel: evict
         // it from L2 first, so that its write-back to DRAM happens while the
         // tensor cores run rather than in whatever kernel comes next
@@ -536,7 +554,8 @@ gemm2_kernel(const __grid_constant__ PairGroup<G> g) {
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN + h * EPI_COLS;
 #pragma unroll
             for (int c = 0; c < EPI_COLS / 32; ++c)
-                tmem_ld_32x32b_x32(tbase + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+                if (h * EPI_COLS + c * 32 < BN)           // the last part can be narrower
+                    tmem_ld_32x32b_x32(tbase + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
             tmem_ld_wait();
             // the accumulator is in registers: hand TMEM back to the MMA issuer
             tc_fence_before();
@@ -559,7 +578,7 @@ gemm2_kernel(const __grid_constant__ PairGroup<G> g) {
 #pragma unroll
                 for (int c = 0; c < EPI_COLS / 32; ++c) {
                     const int ncol = n0 + c * 32;
-                    if (ncol >= P.N) continue;
+                    if (ncol >= P.N || h * EPI_COLS + c * 32 >= BN) continue;
                     uint32_t sfh = 0u, cw[4];
 #pragma unroll
                     for (int b = 0; b < 2; ++b) {
@@ -593,7 +612,7 @@ gemm2_kernel(const __grid_constant__ PairGroup<G> g) {
             } else {
 #pragma unroll
                 for (int c = 0; c < EPI_COLS / 32; ++c) {
-                    if (n0 + c * 32 >= P.N) continue;
+                    if (n0 + c * 32 >= P.N || h * EPI_COLS + c * 32 >= BN) continue;
                     uint8_t* buf_s = ebuf + (nstore & 1) * C::EPI_BUF;
                     if (lane == 0) bulk_wait_group_read<1>();
                     __syncwarp();
