@@ -396,14 +396,15 @@ nvfp4_status nvfp4_mx_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const ui
  *   (quantized along d), head h owning rows h*Lq .. and h*Lk .. ; tensor scales
  *   q_scale, k_scale, v_scale (device floats).
  *   S = Q K^T on the block-scaled FP4 tensor cores (FP32); online softmax in
- *   FP32 with the hardware exp2; P rounded to bf16; V decoded exactly to bf16
- *   (e2m1 * e4m3); O = P V on the bf16 tensor cores (FP32), divided by the row
- *   sum and multiplied by g_v, rounded to bf16.
+ *   FP32 with the hardware exp2; P rounded to f16; V decoded exactly to f16
+ *   (e2m1 * e4m3: at most 6 significant bits within [2^-10, 2688]); O = P V on
+ *   the 16-bit tensor cores (FP32), divided by the row sum and multiplied by
+ *   g_v, rounded to bf16.
  * s_head    nullable device float [H] (1 for every head).  Within one head's
  *           softmax the log(s_head) term is a constant shift of every logit.
  * out       bf16 [H*Lq, d], 16-byte aligned.
  * workspace device scratch of >= nvfp4_attention_workspace_bytes(H, Lk, d)
- *           bytes, 16-byte aligned: V decoded to bf16, [H*Lk, d] (once per
+ *           bytes, 16-byte aligned: V decoded to f16, [H*Lk, d] (once per
  *           call, then read by every query tile), then 32 four-byte words
  *           per head that tag the head's decoded parts with a per-call
  *           number (the counter of nvfp4_quantize's workspace: the same rule
