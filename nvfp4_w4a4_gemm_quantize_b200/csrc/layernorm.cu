@@ -41,6 +41,7 @@ namespace nvfp4 {
 constexpr int kLnMaxWarps = 16;
 constexpr int kLnThreads = kLnMaxWarps * 32;
 constexpr int kLnSmemBudget = 220 * 1024;        // row buffers and affine per CTA
+constexpr int kLnStatRows = 32;                  // per warp: rows whose phase-1 statistics phase 2 reuses
 constexpr int64_t kLnMaxK = 8192;
 
 struct LnArgs {
@@ -164,8 +165,7 @@ __device__ __forceinline__ void ln_block(const uint4* row, const LnAffine& af, i
 // Largest |y| of a row in shared memory; `bad` is set when the row statistics
 // are not finite (an Inf or NaN in the row).
 __device__ __forceinline__ float ln_row_amax(const LnArgs& a, const uint4* row, const LnAffine& af, int lane,
-                                             bool& bad) {
-    float mu32, rstd32;
+                                             bool& bad, float& mu32, float& rstd32) {
     ln_stats(a, row, lane, mu32, rstd32);
     bad |= !(fabsf(mu32) <= 3.402823466e38f) || !(rstd32 <= 3.402823466e38f);
     const int kb = (int)(a.k >> 4);
@@ -182,13 +182,21 @@ __device__ __forceinline__ float ln_row_amax(const LnArgs& a, const uint4* row, 
 // Normalise and quantize row r (row null: a padding row of the scale buffer,
 // rows <= r < rows rounded up to 128, which gets zero scales).  The four
 // lanes 4i .. 4i+3 hold blocks that share one word of the scale layout; lane
-// 4i gathers and stores it.
+// 4i gathers and stores it.  `stats`, when given, holds the row's (mean,
+// 1/std) from phase 1 -- the same values ln_stats would compute again.
 __device__ __forceinline__ void ln_quantize_row(const LnArgs& a, const uint4* row, const LnAffine& af, int64_t r,
-                                                int lane, const ScaleConsts& sc) {
+                                                int lane, const ScaleConsts& sc, const float2* stats = nullptr) {
     const int kb = (int)(a.k >> 4);
     const int64_t kb4 = a.k >> 6;
     float mu32 = 0.0f, rstd32 = 0.0f;
-    if (row) ln_stats(a, row, lane, mu32, rstd32);
+    if (row) {
+        if (stats) {
+            mu32 = stats->x;
+            rstd32 = stats->y;
+        } else {
+            ln_stats(a, row, lane, mu32, rstd32);
+        }
+    }
     uint8_t* sfrow = a.sf + ((r >> 7) * kb4) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4;
     for (int c0 = 0; c0 < kb; c0 += 32) {
         const int c = c0 + lane;              // kb % 4 == 0: the four lanes of a word agree on c < kb
@@ -260,6 +268,7 @@ layernorm_quantize_kernel(const LnArgs a, int warps, int64_t per_cta) {
     __shared__ __align__(8) uint64_t bars[2 * kLnMaxWarps];
     __shared__ ScaleConsts sc_sh;
     __shared__ float red[kLnMaxWarps];
+    __shared__ float2 row_stats[kLnMaxWarps][kLnStatRows];   // phase 1's (mean, 1/std) of a warp's first rows
     __shared__ int ok_sh, abort_sh;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rowbytes = (uint32_t)(a.k * 2);
@@ -310,7 +319,11 @@ layernorm_quantize_kernel(const LnArgs a, int warps, int64_t per_cta) {
             if (i + 1 < n_real) st.issue(a, first + (i + 1) * warps, b ^ 1, lane);
             const uint4* row = st.wait(b, wc, ok);
             const int64_t r = first + i * warps;
-            if (ok) m = fmaxf(m, ln_row_amax(a, row, ln_affine(a, r, cached, aff), lane, nonfinite));
+            if (ok) {
+                float mu32, rstd32;
+                m = fmaxf(m, ln_row_amax(a, row, ln_affine(a, r, cached, aff), lane, nonfinite, mu32, rstd32));
+                if (i < kLnStatRows && lane == 0) row_stats[warp][i] = make_float2(mu32, rstd32);
+            }
             __syncwarp();
         }
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -369,8 +382,11 @@ layernorm_quantize_kernel(const LnArgs a, int warps, int64_t per_cta) {
         const int b = (int)(i & 1);
         if (i + 1 < n_real) st.issue(a, first + (n_real - 2 - i) * warps, b ^ 1, lane);
         const uint4* row = st.wait(b, wc, ok);
-        const int64_t r = first + (n_real - 1 - i) * warps;
-        if (ok) ln_quantize_row(a, row, ln_affine(a, r, cached, aff), r, lane, sc);
+        const int64_t ir = n_real - 1 - i;
+        const int64_t r = first + ir * warps;
+        if (ok)
+            ln_quantize_row(a, row, ln_affine(a, r, cached, aff), r, lane, sc,
+                            kDynamic && ir < kLnStatRows ? &row_stats[warp][ir] : nullptr);
         __syncwarp();
     }
     for (int64_t r = first + n_real * warps; r < r1; r += warps)

@@ -162,3 +162,14 @@ def test_attention_decode_parts_with_empty_shares(cuda_ok):
     torch.cuda.synchronize()
     assert st.item() == 0
     _sampled_heads(xq, xk, xv, H, Lq, Lk, heads=(0, 7, 19), rows=(0, 3001, 6143))
+
+
+def test_attention_more_items_per_head_than_slots(cuda_ok):
+    """33 work items per head (Lq = 8448): more than the 32 decode slots of a
+    head, so the library decodes V in a separate pass first; the two-tile
+    kernel then reads it as when it decodes V itself."""
+    H, Lq, Lk = 2, 8448, 256
+    xq = synth.random_bf16((H * Lq, D), seed=84, dist="normal")
+    xk = synth.random_bf16((H * Lk, D), seed=85, dist="normal")
+    xv = synth.random_bf16((H * Lk, D), seed=86, dist="student_t3")
+    _sampled_heads(xq, xk, xv, H, Lq, Lk, heads=(0, 1), rows=(0, 4321, 8447))
