@@ -847,8 +847,11 @@ attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
         } else if (warp == 1) {
             // -------------------------------------------------------- S = Q K^T issuer (and TMEM owner)
             // The S buffer's uses alternate A, B, A, B, ...; use u waits until
-            // the group of use u - 1 has read it out.
-            constexpr uint32_t idesc_s = idesc_nvf4(kBQ, kBK);
+            // the group of use u - 1 has read it out.  Each use is issued as two
+            // N = 64 products (keys 0-63, 64-127: the B operand and its scales
+            // start 64 rows -- 4 KB of codes, two TMEM columns -- on for the
+            // second), measured a little faster than one N = 128 product.
+            constexpr uint32_t idesc_s = idesc_nvf4(kBQ, 64);
             const uint32_t sm0 = smem_u32(smem);
             bool ok = true;
             int n = 0, i = 0;
@@ -893,10 +896,12 @@ attn2_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                         const uint32_t sfq = tmem + kColSfQ2 + (qb * 2 + g) * 8;
                         if (elect_one()) {
 #pragma unroll
-                            for (int ks = 0; ks < 2; ++ks)
-                                tc_mma_nvf4(tmem + kColS2, sdesc_kmajor_sw64(qs + ks * 32),
-                                            sdesc_kmajor_sw64(st + ks * 32), idesc_s, sfq + ks * 4, sfk + ks * 4,
-                                            ks != 0 ? 1u : 0u);
+                            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                                for (int ks = 0; ks < 2; ++ks)
+                                    tc_mma_nvf4(tmem + kColS2 + 64 * hh, sdesc_kmajor_sw64(qs + ks * 32),
+                                                sdesc_kmajor_sw64(st + 4096 * hh + ks * 32), idesc_s, sfq + ks * 4,
+                                                sfk + ks * 4 + 2 * hh, ks != 0 ? 1u : 0u);
                             tc_commit(&s_full[g]);
                             if (g == 1) {
                                 tc_commit(&k_empty[s]);
