@@ -257,6 +257,8 @@ def test_attention_rejects_bad_arguments(L):
     assert a(*ops, C + 2, 2, 128, 256, 128, A, C, 1 << 30, None, None) == MISALIGNED
     assert a(*ops, None, 2, 128, 256, 128, A, C, 100, None, None) == WORKSPACE
     assert a(*ops, None, 2, 128, 256, 128, A, None, 1 << 30, None, None) == WORKSPACE
+    # room for the decoded V but not for the heads' decode slots
+    assert a(*ops, None, 2, 128, 256, 128, A, C, 2 * 128 * 256 * 2, None, None) == WORKSPACE
     assert L.nvfp4_attention_workspace_bytes(2, 256, 128) == 2 * 128 * 256 * 2 + 2 * 128
 
 
