@@ -108,6 +108,18 @@ def test_quantize_shapes(cuda_ok, rows, k, ld, dist):
     _check(x, scale=float(oracle.tensor_scale(x)) * 0.75, ld=ld)
 
 
+@pytest.mark.parametrize("rows,k,ld", [(129, 192, 200), (600, 4096, 4096), (4096, 3072, 3072)])
+def test_streamed_one_kernel_form(cuda_ok, monkeypatch, rows, k, ld):
+    """The one-kernel form that streams the tiles through a ring of shared-memory
+    buffers by TMA (the default for fake quantization; for codes a switch,
+    NVFP4_QUANT_ONE_KERNEL=stream) gives the same codes, scales and tensor
+    scale.  4096 x 3072 is 384 tiles over one CTA per SM: up to three tiles a
+    CTA, so each CTA's six loads wrap its three-buffer ring."""
+    x = synth.random_bf16((rows, k), seed=rows + 7 * k, dist="student_t3")
+    monkeypatch.setenv("NVFP4_QUANT_ONE_KERNEL", "stream")
+    _check(x, ld=ld)
+
+
 def test_quantize_zero_single_and_empty(cuda_ok):
     z = torch.zeros(130, 128, dtype=torch.bfloat16)
     codes, sf, g = _gpu_quantize(z)
