@@ -12,7 +12,8 @@ Low-level (same names and argument order as the C calls):
     nvfp4_gemm_w4a4, nvfp4_gemm_w4a4_grouped, nvfp4_gemm_w4a16, nvfp4_mx_sf_bytes, nvfp4_mx_quantize,
     nvfp4_mx_dequantize, nvfp4_mx_gemm, nvfp4_attention, nvfp4_attention_workspace_bytes, nvfp4_launch_count
 Convenience (allocate outputs with torch, then call the above):
-    NVFP4Tensor, quantize, layernorm_quantize, dequantize, gemm_w4a4, gemm_w4a4_grouped, gemm_w4a16,
+    NVFP4Tensor, quantize, layernorm_quantize, dequantize, gemm_w4a4, gemm_w4a4_nvfp4_out, gemm_w4a4_grouped,
+    gemm_w4a16,
     fake_quantize, ste_backward, FakeQuantizeSTE (autograd: the two kernels),
     MXTensor, mx_quantize, mx_dequantize, mx_gemm, quantize_block, block_size_errors, select_block_size,
     attention
