@@ -31,6 +31,10 @@
  *  - Every pointer is DEVICE memory unless stated; the caller allocates and
  *    owns every buffer.  Calls are asynchronous on `stream` (a cudaStream_t;
  *    NULL = legacy default stream) and never synchronize the host.
+ *  - Kernels run on the calling thread's current CUDA device, and every buffer
+ *    must be that device's memory (the stream too must belong to it).  Where a
+ *    pointer lives is not checked: a buffer of another device is a caller
+ *    error whose outcome the library does not define.
  *  - Argument checks run on the host before any launch; a failed check
  *    returns an error and launches nothing.  Launch failures return
  *    NVFP4_ERR_CUDA.

@@ -3,7 +3,9 @@
 Python binding of the C ABI in include/nvfp4.h.  Every function below only
 marshals torch tensors into pointers and sizes and calls the library of the
 same name; all arithmetic runs in the CUDA kernels.  torch supplies device
-memory and streams.
+memory and streams.  Every tensor must live on the current CUDA device (the
+library launches there; nothing here switches devices), and the default stream
+argument is that device's current torch stream.
 
 Low-level (same names and argument order as the C calls):
     nvfp4_sf_bytes, nvfp4_quantize_workspace_bytes, nvfp4_quantize,
